@@ -1,0 +1,311 @@
+// Sparse Delta Memory (SDM) recurrent core -- CPU ORACLE.
+//
+// TEST INFRASTRUCTURE ONLY. This file is the plain, slow, obviously-correct
+// definition that the CUDA path is checked against. Only the tests, the smoke
+// check and the benchmark's CPU-baseline leg may load it. It shares no code,
+// header, table or helper with the CUDA library, and the library never calls it.
+//
+// Sources (web pages about arXiv 2607.07386, "Sparse Delta Memory: Scaling the
+// State of Linear RNNs through Sparsity"), cited below by these short names:
+//   [explainer]  papers.ananclaw.com explainer "Sparse Delta Memory：通过稀疏性扩展
+//                线性 RNN 的状态容量", section 3.1 "SDM 层的三步流程" (steps 1-3),
+//                section 3.2 (IsoFLOP), section 3.3 (equation 6).
+//   [summary]    gist.science "Technical Summary: Sparse Delta Memory (SDM)",
+//                Methodology / Core Mechanism items 1-4 and "IsoFLOP Design".
+//
+// What it computes, step by step, in the pages' order:
+//   1. Selection ([explainer] 3.1 step 1; [summary] Core Mechanism 2). The score
+//      vector x of length 2*sqrtN is split into s1 = x[0:sqrtN], s2 = x[sqrtN:].
+//      The N = sqrtN^2 slot scores are the outer SUM s1[a] + s2[b]; slot number
+//      i = a*sqrtN + b (row-major over the sqrtN x sqrtN grid). All N scores are
+//      materialised and the first K of the order (exact real sum descending,
+//      slot ascending) are kept. The exact sum is held as a double TwoSum pair
+//      (hi, lo) -- fp32 operands are exact in double, TwoSum makes hi+lo the
+//      exact real sum -- and compared lexicographically, which equals comparing
+//      the real sums because round-to-nearest is monotone.
+//   2. Sparse weights: softmax over the K selected scores, in double. The pages
+//      use the weights k^(i), q^(i) without defining them; this reading is the
+//      softmax of the selected scores with ties broken by lowest slot index.
+//   3. Write ([explainer] 3.1 step 2; [summary] Core Mechanism 3), for every
+//      selected write slot i, literally:  Mt = alpha*M[i];
+//      M[i] = Mt + beta*k_i*(v - Mt); other slots untouched. Math in double,
+//      rounded to the state dtype (fp32, or bf16 round-to-nearest-even) on store.
+//   4. Read after the write ([explainer] 3.1 step 3; [summary] Core Mechanism 4):
+//      y_t = sum over read slots of q_i * M_t[i], in double.
+//   5. Optional epilogue ([explainer] 3.1 step 3): y <- g * y / sqrt(mean(y^2)+eps).
+//
+// Parity status: selection, weights, write, read and epilogue are each pinned by
+// tests that do not re-run this file's formulas (exact-rational brute force,
+// closed forms, invariants, hand-worked fixtures, planted-mistake checks).
+//
+// ORACLE_MUTANT (default 0) plants one known mistake per value so the tests
+// can show that the pins catch it; it is never set outside those tests.
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+namespace {
+
+// One materialised slot score: exact sum hi + lo of s1[a] + s2[b].
+struct SlotScore {
+  double hi;
+  double lo;
+  int32_t slot;
+};
+
+// Knuth's TwoSum: hi = fl(x + y), lo = the exact rounding error, so hi + lo == x + y.
+inline void two_sum(double x, double y, double* hi, double* lo) {
+  const double s = x + y;
+  const double bb = s - x;
+  *hi = s;
+  *lo = (x - (s - bb)) + (y - bb);
+}
+
+// The selection order: exact sum descending, then slot ascending (ties -> lowest slot).
+inline bool precedes(const SlotScore& p, const SlotScore& q) {
+#if ORACLE_MUTANT == 3
+  if (p.hi != q.hi) return p.hi > q.hi;  // planted: the low part is ignored
+#else
+  if (p.hi != q.hi) return p.hi > q.hi;
+  if (p.lo != q.lo) return p.lo > q.lo;
+#endif
+#if ORACLE_MUTANT == 2
+  return p.slot > q.slot;  // planted: ties go to the highest slot
+#else
+  return p.slot < q.slot;
+#endif
+}
+
+// Runs fn(i) for i in [0, n) on up to n_threads threads.
+template <class Fn>
+void parallel_for(int64_t n, int n_threads, Fn fn) {
+  if (n_threads <= 1 || n <= 1) {
+    for (int64_t i = 0; i < n; ++i) fn(i);
+    return;
+  }
+  std::atomic<int64_t> next(0);
+  std::vector<std::thread> pool;
+  const int nt = static_cast<int>(std::min<int64_t>(n_threads, n));
+  for (int t = 0; t < nt; ++t) {
+    pool.emplace_back([&]() {
+      for (;;) {
+        const int64_t i = next.fetch_add(1);
+        if (i >= n) break;
+        fn(i);
+      }
+    });
+  }
+  for (auto& th : pool) th.join();
+}
+
+// Rounds a double to the nearest bf16 value (ties to even), returned as float.
+// bf16 keeps 8 significant bits and fp32's exponent range; its smallest
+// subnormal step is 2^-133.
+float round_to_bf16(double x) {
+  if (x == 0.0 || !std::isfinite(x)) return static_cast<float>(x);
+  int e = 0;
+  std::frexp(x, &e);  // x = m * 2^e with 0.5 <= |m| < 1
+  int q = e - 8;      // weight of the last kept bit
+  if (q < -133) q = -133;
+  const double r = std::nearbyint(std::ldexp(x, -q));  // default mode: nearest-even
+  return static_cast<float>(std::ldexp(r, q));
+}
+
+inline float round_state(double x, bool bf16) {
+  return bf16 ? round_to_bf16(x) : static_cast<float>(x);
+}
+
+// Selection for one score vector x[0 : 2*sqrt_n): writes K slots (selection
+// order) and their softmax weights.
+void select_one(const float* x, int32_t sqrt_n, int32_t K, std::vector<SlotScore>& grid,
+                int32_t* idx, double* w) {
+  const int64_t n = static_cast<int64_t>(sqrt_n) * sqrt_n;
+  const float* s1 = x;           // first half  -> grid row a
+  const float* s2 = x + sqrt_n;  // second half -> grid column b
+  grid.resize(static_cast<size_t>(n));
+  for (int32_t a = 0; a < sqrt_n; ++a) {
+    for (int32_t b = 0; b < sqrt_n; ++b) {
+      SlotScore& e = grid[static_cast<size_t>(a) * sqrt_n + b];
+      two_sum(static_cast<double>(s1[a]), static_cast<double>(s2[b]), &e.hi, &e.lo);
+#if ORACLE_MUTANT == 1
+      e.slot = b * sqrt_n + a;  // planted: grid numbered column-major
+#else
+      e.slot = a * sqrt_n + b;
+#endif
+    }
+  }
+  // Library sort primitive: partial_sort returns exactly the first K elements
+  // of the full sort because `precedes` is a strict total order.
+  std::partial_sort(grid.begin(), grid.begin() + K, grid.end(), precedes);
+  double mx = -INFINITY;
+  for (int32_t k = 0; k < K; ++k) mx = std::max(mx, grid[k].hi + grid[k].lo);
+  double z = 0.0;
+  for (int32_t k = 0; k < K; ++k) {
+    idx[k] = grid[k].slot;
+    w[k] = std::exp((grid[k].hi + grid[k].lo) - mx);
+    z += w[k];
+  }
+  for (int32_t k = 0; k < K; ++k) {
+#if ORACLE_MUTANT == 8
+    w[k] = 1.0 / K;  // planted: uniform weights
+#else
+    w[k] = w[k] / z;
+#endif
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_abi_version() { return 1; }
+
+float oracle_round_to_bf16(double x) { return round_to_bf16(x); }
+
+// Top-K slot selection for n_units independent score vectors.
+//   scores : [n_units, 2*sqrt_n] fp32 (bf16 inputs are widened exactly by the caller)
+//   idx_out: [n_units, K] int32, selection order;  w_out: [n_units, K] softmax weights
+// Returns 0, or -1 for invalid sizes.
+int oracle_pkm_topk(const float* scores, int64_t n_units, int32_t sqrt_n, int32_t K,
+                    int32_t* idx_out, double* w_out, int32_t n_threads) {
+  if (sqrt_n < 1 || K < 1 || static_cast<int64_t>(K) > static_cast<int64_t>(sqrt_n) * sqrt_n ||
+      n_units < 0)
+    return -1;
+  const int nt = std::max(1, n_threads);
+  const int64_t chunk = 64;
+  const int64_t n_chunks = (n_units + chunk - 1) / chunk;
+  parallel_for(n_chunks, nt, [&](int64_t c) {
+    std::vector<SlotScore> grid;
+    const int64_t u_end = std::min(n_units, (c + 1) * chunk);
+    for (int64_t u = c * chunk; u < u_end; ++u) {
+      select_one(scores + u * 2 * sqrt_n, sqrt_n, K, grid, idx_out + u * K, w_out + u * K);
+    }
+  });
+  return 0;
+}
+
+// The recurrence over a given selection.
+//   idx_w, w_w : [B,T,H,W]   idx_r, w_r : [B,T,H,R]
+//   v          : [B,T,H,d_v] alpha, beta : [B,T,H]   g: [B,T,H,d_v] or NULL
+//   M          : [B,H,N,d_v] in/out (fp32 array; with state_bf16 every stored
+//                value is rounded to bf16 and kept as an exact fp32)
+//   y          : [B,T,H,d_v] out, double
+//   op_count   : if not NULL, receives the number of scalar multiply/add
+//                operations the write and read steps performed
+// Returns 0, or -1 for invalid sizes, or -2 when an index is outside [0, N).
+int oracle_scan(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W, int32_t R,
+                const int32_t* idx_w, const double* w_w, const int32_t* idx_r, const double* w_r,
+                const float* v, const float* alpha, const float* beta, const float* g,
+                double eps, int32_t state_bf16, float* M, double* y, int32_t n_threads,
+                int64_t* op_count) {
+  if (B < 0 || T < 0 || H < 0 || N < 1 || d_v < 1 || W < 0 || R < 0) return -1;
+  for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * W; ++e)
+    if (idx_w[e] < 0 || idx_w[e] >= N) return -2;
+  for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * R; ++e)
+    if (idx_r[e] < 0 || idx_r[e] >= N) return -2;
+  const bool bf16 = state_bf16 != 0;
+  // Columns of d_v evolve independently, so the work splits over (b, h, column block).
+  const int32_t col_block = 64;
+  const int32_t n_cb = (d_v + col_block - 1) / col_block;
+  std::atomic<int64_t> ops(0);
+  parallel_for(static_cast<int64_t>(B) * H * n_cb, std::max(1, n_threads), [&](int64_t u) {
+    const int32_t cb = static_cast<int32_t>(u % n_cb);
+    const int32_t h = static_cast<int32_t>((u / n_cb) % H);
+    const int32_t b = static_cast<int32_t>(u / (static_cast<int64_t>(n_cb) * H));
+    const int32_t c0 = cb * col_block;
+    const int32_t c1 = std::min(d_v, c0 + col_block);
+    float* Mbh = M + (static_cast<int64_t>(b) * H + h) * N * d_v;
+    int64_t local_ops = 0;
+    for (int32_t t = 0; t < T; ++t) {
+      const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;  // token-head
+      const double a_t = alpha[th];
+      const double b_t = beta[th];
+      const float* v_t = v + th * d_v;
+      double* y_t = y + th * d_v;
+      auto do_reads = [&]() {
+        for (int32_t c = c0; c < c1; ++c) {
+          double acc = 0.0;
+          for (int32_t r = 0; r < R; ++r) {
+            const int64_t i = idx_r[th * R + r];
+            acc += w_r[th * R + r] * static_cast<double>(Mbh[i * d_v + c]);
+          }
+          y_t[c] = acc;
+        }
+        local_ops += static_cast<int64_t>(2) * R * (c1 - c0);
+      };
+#if ORACLE_MUTANT == 6
+      do_reads();  // planted: read before the write
+#endif
+      // Step 2: gated delta write on the selected write slots only.
+      for (int32_t j = 0; j < W; ++j) {
+        const int64_t i = idx_w[th * W + j];
+        const double k_i = w_w[th * W + j];
+        for (int32_t c = c0; c < c1; ++c) {
+          const double m_prev = Mbh[i * d_v + c];
+#if ORACLE_MUTANT == 4
+          const double m_tilde = m_prev;  // planted: forget gate dropped
+#else
+          const double m_tilde = a_t * m_prev;
+#endif
+          const double v_c = v_t[c];
+#if ORACLE_MUTANT == 5
+          const double m_new = m_tilde - b_t * k_i * (v_c - m_tilde);  // planted: sign
+#elif ORACLE_MUTANT == 7
+          const double m_new = m_tilde + b_t * (v_c - m_tilde);  // planted: k dropped
+#else
+          const double m_new = m_tilde + b_t * k_i * (v_c - m_tilde);
+#endif
+#if ORACLE_MUTANT == 10
+          Mbh[i * d_v + c] = static_cast<float>(m_new);  // planted: no state rounding
+#else
+          Mbh[i * d_v + c] = round_state(m_new, bf16);
+#endif
+        }
+        local_ops += static_cast<int64_t>(4) * (c1 - c0);
+      }
+#if ORACLE_MUTANT == 11
+      // planted: the forget gate also decays one unselected slot
+      {
+        int64_t other = (idx_w[th * W] + 1) % N;
+        bool selected = false;
+        for (int32_t j = 0; j < W; ++j) selected = selected || idx_w[th * W + j] == other;
+        if (!selected)
+          for (int32_t c = c0; c < c1; ++c)
+            Mbh[other * d_v + c] = round_state(a_t * Mbh[other * d_v + c], bf16);
+      }
+#endif
+      // Step 3: sparse read of the state after this token's write.
+#if ORACLE_MUTANT != 6
+      do_reads();
+#endif
+    }
+    ops.fetch_add(local_ops);
+  });
+  // Optional epilogue: RMS-norm over d_v per token-head, then the element-wise gate.
+  if (g != nullptr) {
+    parallel_for(static_cast<int64_t>(B) * T * H, std::max(1, n_threads), [&](int64_t th) {
+      double* y_t = y + th * d_v;
+      double ss = 0.0;
+      for (int32_t c = 0; c < d_v; ++c) ss += y_t[c] * y_t[c];
+#if ORACLE_MUTANT == 9
+      const double inv = 1.0 / std::sqrt(ss + eps);  // planted: sum instead of mean
+#else
+      const double inv = 1.0 / std::sqrt(ss / d_v + eps);
+#endif
+      for (int32_t c = 0; c < d_v; ++c) y_t[c] = static_cast<double>(g[th * d_v + c]) * y_t[c] * inv;
+    });
+  }
+  if (op_count != nullptr) *op_count = ops.load();
+  return 0;
+}
+
+}  // extern "C"
