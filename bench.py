@@ -1,0 +1,432 @@
+"""Benchmark of the SDM recurrent core on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl sdm|reference]
+
+A step is one sdm_layer_forward call over one batch of synthetic input: the
+product-key selection of k' and q', the record build, the state
+initialisation and the recurrence (epilogue off unless --epilogue). Inputs
+are resident in HBM when the timed region starts; `e2e` repeats the
+measurement with the inputs copied from pinned host memory and y copied back
+inside the timed region. With N > 1 (torchrun) each rank runs its own batch
+(weak scaling, no collective on the data path); the time is the max over
+ranks. `--impl reference` times the CPU oracle on a bounded sample instead
+(rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import sparse_memory_linear_pkm_b200 as sdm  # noqa: E402
+from sparse_memory_linear_pkm_b200 import synth  # noqa: E402
+
+METRIC = "SDM layer tokens/s (B·T) and achieved HBM/L2 GB/s vs roofline on 1 B200"
+DEFAULT_WORKLOAD = "d2048_h16_n1024_dv128"
+FALLBACK_HBM_GBS = 6650.0
+SMEM_BYTES_PER_CLK_PER_SM = 128
+NVML_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="sdm", choices=["sdm", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--epilogue", action="store_true", help="run the RMS-norm x gate epilogue")
+    ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ ranks --
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import torch.distributed as dist
+
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = True
+
+    def barrier(self, device=None):
+        if self.pg:
+            import torch.distributed as dist
+
+            if device is not None and device.type == "cuda":
+                dist.barrier(device_ids=[device.index])
+            else:
+                dist.barrier()
+
+    def max(self, x: float, device) -> float:
+        if not self.pg:
+            return x
+        import torch.distributed as dist
+
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+def aggregate_value(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """Reads SM clocks and clock-event reasons through NVML during the timed
+    region (read-only; no setting of the GPU is touched)."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.reasons = 0
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+            self._nvml = pynvml
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = repr(e)
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        names = sorted(n for bit, n in NVML_REASONS.items() if self.reasons & bit and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------- roofline --
+
+def measured_peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        try:
+            return json.loads(p.read_text())
+        except Exception:
+            pass
+    return {}
+
+
+def algorithmic_bytes_per_token_head(shape: synth.Shape, epilogue: bool) -> int:
+    """(2W + R) d_v sizeof(state) of state traffic, plus the per-token-head
+    inputs (indices + weights, v, alpha, beta, g) and the fp32 y."""
+    s_state = 2 if shape.state_dtype == synth.BF16 else 4
+    s_in = 2 if shape.in_dtype == synth.BF16 else 4
+    b = (2 * shape.W + shape.R) * shape.d_v * s_state
+    b += (shape.W + shape.R) * 8 + shape.d_v * s_in + 2 * s_in + shape.d_v * 4
+    if epilogue:
+        b += shape.d_v * s_in
+    return b
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "sparse_memory_linear_pkm_b200" / "csrc").glob("*")):
+        h.update(p.name.encode())
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, when
+    it was taken on the current kernel sources; else None."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    try:
+        entry = json.loads(p.read_text()).get(workload, {}).get(kernel)
+    except Exception:
+        return None
+    if not entry or entry.get("source_digest") != source_digest():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample_inputs(inp: dict, Bs: int, Ts: int) -> dict:
+    f = synth.to_numpy_f32
+    out = {k: f(inp[k][:Bs, :Ts]) for k in ("kp", "qp", "v", "alpha", "beta")}
+    out["M0"] = f(inp["M0"])
+    if "g" in inp:
+        out["g"] = f(inp["g"][:Bs, :Ts])
+    return out
+
+
+def time_oracle(o, shape: synth.Shape, sample: dict, threads: int) -> float:
+    t0 = time.perf_counter()
+    o.layer_forward(sample["kp"], sample["qp"], sample["v"], sample["alpha"], sample["beta"], sample["M0"],
+                    shape.W, shape.R, g=sample.get("g"), state_bf16=shape.state_dtype == synth.BF16,
+                    n_threads=threads)
+    return time.perf_counter() - t0
+
+
+def calibrate_sample(o, shape: synth.Shape, inp: dict, threads: int, target_s: float):
+    """Grows (batch rows, tokens) of the oracle sample until one run takes
+    about target_s seconds (or the whole workload is covered)."""
+    Bs, Ts = 1, 1
+    dt = time_oracle(o, shape, oracle_sample_inputs(inp, Bs, Ts), threads)
+    while dt < target_s / 2 and (Bs < shape.B or Ts < shape.T):
+        scale = max(2.0, min(16.0, target_s / max(dt, 1e-3)))
+        if Ts < shape.T:
+            Ts = min(shape.T, int(Ts * scale))
+        else:
+            Bs = min(shape.B, int(Bs * scale))
+        dt = time_oracle(o, shape, oracle_sample_inputs(inp, Bs, Ts), threads)
+    return Bs, Ts, dt
+
+
+def cpu_baseline(shape: synth.Shape, inp: dict, target_s: float, epilogue: bool) -> dict:
+    import oracle
+
+    o = oracle.get()
+    threads = oracle.default_threads()
+    Bs, Ts, dt = calibrate_sample(o, shape, inp, threads, target_s)
+    return {"value": Bs * Ts / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"batch rows 0..{Bs - 1}, first {Ts} tokens, all {shape.H} heads "
+                      f"({Bs * Ts} tokens, {dt:.1f} s){', with epilogue' if epilogue else ''}"}
+
+
+# ------------------------------------------------------------------- arms --
+
+def run_reference(args, dist: Dist):
+    """The oracle, timed on the host cores on a bounded sample per step."""
+    if dist.rank != 0:
+        return
+    import oracle
+
+    shape = synth.WORKLOADS[args.workload]
+    dev = torch.device("cuda", dist.local_rank) if torch.cuda.is_available() else torch.device("cpu")
+    inp = synth.make_inputs(shape.replace(B=1, T=min(shape.T, 4096)), seed=args.seed, device=dev,
+                            with_gate=args.epilogue)
+    o = oracle.get()
+    threads = oracle.default_threads()
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    Bs, Ts, _ = calibrate_sample(o, shape.replace(B=1, T=min(shape.T, 4096)), inp, threads, budget_s)
+    sample = oracle_sample_inputs(inp, Bs, Ts)
+    for _ in range(args.warmup):
+        time_oracle(o, shape, sample, threads)
+    t = 0.0
+    for _ in range(args.steps):
+        t += time_oracle(o, shape, sample, threads)
+    value = args.steps * Bs * Ts / t
+    desc = f"batch row 0, first {Ts} tokens, all {shape.H} heads ({Bs * Ts} tokens per step)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(shape, args, dist),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(shape: synth.Shape, args, dist: Dist) -> dict:
+    return {"workload": shape.name, "B": shape.B, "T": shape.T, "H": shape.H, "sqrt_n": shape.sqrt_n, "N": shape.N,
+            "d_v": shape.d_v, "W": shape.W, "R": shape.R, "in_dtype": shape.in_dtype,
+            "state_dtype": shape.state_dtype, "epilogue": bool(args.epilogue), "seed": args.seed,
+            "parallelism": f"dp{dist.world} (independent batch per rank)"}
+
+
+def run_sdm(args, dist: Dist):
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl sdm needs a CUDA device")
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    shape = synth.WORKLOADS[args.workload]
+    sdm.native.load()
+    inp = synth.make_inputs(shape, seed=args.seed + dist.rank, device=dev, with_gate=args.epilogue)
+    g = inp.get("g")
+    y = torch.empty((shape.B, shape.T, shape.H, shape.d_v), dtype=torch.float32, device=dev)
+    M_out = torch.empty((shape.B,) + tuple(inp["M0"].shape), dtype=inp["M0"].dtype, device=dev)
+    sh = sdm.make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
+                        shape.torch_state(), variant=args.variant)
+    ws = torch.empty(sdm.layer_forward_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+
+    def step(events=None, src=inp):
+        sdm.layer_forward(src["kp"], src["qp"], src["v"], src["alpha"], src["beta"], inp["M0"], shape.W, shape.R,
+                          g=g, variant=args.variant, y=y, M_out=M_out, workspace=ws, events=events)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step()
+    sdm.stream_check(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for row in ev:  # create the events before the timed region
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for k in range(args.steps):
+            step(events=ev[k])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    sdm.stream_check(dev)
+    ms = start.elapsed_time(end)
+    ms_max = dist.max(ms, dev)
+    stage_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps for i in range(5)]
+    tokens = shape.B * shape.T
+    value = aggregate_value(tokens * args.steps, dist.world, ms_max / 1e3)
+
+    resident = sdm.scan_variant(sh) == "resident"
+    launches_per_step = 4 + (0 if resident else 1) + (1 if args.epilogue else 0)
+    scan_ms = stage_ms[3]
+    th = shape.B * shape.T * shape.H
+    algo_bytes = algorithmic_bytes_per_token_head(shape, args.epilogue) * th
+    achieved = algo_bytes / (scan_ms / 1e3) / 1e9
+    peaks = measured_peaks()
+    clk = clocks.summary()
+    if resident:
+        mhz = clk["sm_max_mhz"] or 1965.0
+        peak = torch.cuda.get_device_properties(dev).multi_processor_count * SMEM_BYTES_PER_CLK_PER_SM * mhz / 1e3
+        roof = {"bound": "smem", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": f"derived: SMs x {SMEM_BYTES_PER_CLK_PER_SM} B/clk x {mhz:.0f} MHz "
+                               "(state tile resident in shared memory)"}
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "of fallback"}
+    kernel = "k_scan_resident" if resident else "k_scan_streaming"
+    traffic = recorded_traffic(shape.name, kernel)
+    roof.update({"traffic": traffic, "kernel": kernel, "ms_per_launch": scan_ms,
+                 "algorithmic_bytes_per_launch": algo_bytes})
+
+    e2e = None
+    if not args.no_e2e:
+        host = {k: inp[k].cpu().pin_memory() for k in ("kp", "qp", "v", "alpha", "beta")}
+        dinp = {k: torch.empty_like(inp[k]) for k in host}
+        y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = y.numel() * y.element_size()
+        k_e2e = max(3, min(args.steps, 20))
+        for _ in range(2):
+            for k in host:
+                dinp[k].copy_(host[k], non_blocking=True)
+            step(src=dinp)
+            y_host.copy_(y, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        dist.barrier(dev)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(k_e2e):
+            for k in host:
+                dinp[k].copy_(host[k], non_blocking=True)
+            step(src=dinp)
+            y_host.copy_(y, non_blocking=True)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier(dev)
+        e_ms = dist.max(s2.elapsed_time(e2), dev)
+        e2e = {"value": aggregate_value(tokens * k_e2e, dist.world, e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+               "path": "pinned host -> device copies, sdm_layer_forward, y -> pinned host, one stream"}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(shape, inp, args.cpu_seconds, args.epilogue)
+
+    if dist.rank == 0:
+        l2_mb = torch.cuda.get_device_properties(dev).L2_cache_size / 2 ** 20
+        in_mb = sum(t.numel() * t.element_size() for t in inp.values()) / 2 ** 20
+        cfg = workload_config(shape, args, dist)
+        cfg["l2"] = (f"no flush between steps: per-step inputs {in_mb:.0f} MiB and y {d2h_mib(y):.0f} MiB "
+                     f"exceed the {l2_mb:.0f} MiB L2")
+        cfg["variant"] = "resident" if resident else "streaming"
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+                "clocks": clk,
+                "stage_ms": {"select_k_and_q": stage_ms[0], "records": stage_ms[1], "state_init": stage_ms[2],
+                             "scan": stage_ms[3], "epilogue": stage_ms[4]}}
+        print(json.dumps(line), flush=True)
+    del ev
+    dist.close()
+
+
+def d2h_mib(y: torch.Tensor) -> float:
+    return y.numel() * y.element_size() / 2 ** 20
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    run_sdm(args, dist)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,189 @@
+/*
+ * sdm.h -- C ABI of the B200 (sm_100a) Sparse Delta Memory recurrent core.
+ *
+ * The Sparse Delta Memory (SDM) layer keeps, per head, an explicit memory
+ * M in R^{N x d_v} with N = sqrtN^2 slots. Per token it selects W write slots
+ * and R read slots by product-key top-k, applies a gated delta write to the
+ * write slots and reads a weighted sum of the read slots after the write.
+ *
+ * Sources (web pages about arXiv 2607.07386, "Sparse Delta Memory: Scaling the
+ * State of Linear RNNs through Sparsity"):
+ *   [explainer] papers.ananclaw.com explainer, section 3.1 "SDM 层的三步流程"
+ *               (step 1 sparse key selection, step 2 gated delta write,
+ *               step 3 sparse read), section 3.2 (isoFLOP), section 3.3 (eq. 6);
+ *   [summary]   gist.science "Technical Summary: Sparse Delta Memory (SDM)",
+ *               Methodology / Core Mechanism items 1-4.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as tensors are caller-owned DEVICE pointers to contiguous
+ *     row-major arrays, 16-byte aligned. The library allocates no memory;
+ *     scratch space is passed in by the caller ("workspace").
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Calls only enqueue work and return; results are ready when the
+ *     stream reaches them.
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     return SDM_ERR_INVALID_ARGUMENT / SDM_ERR_UNSUPPORTED; sdm_last_error()
+ *     then names the argument. A failed kernel launch returns SDM_ERR_CUDA.
+ *     Problems found on the device (an index outside [0, N), a bounded wait
+ *     that expired) set a per-device error word that sdm_stream_check()
+ *     reports as SDM_ERR_DEVICE_FAULT; such entries are skipped, never
+ *     dereferenced.
+ *   - Shapes: B batch rows, T tokens, H heads; a "token-head" is one (b,t,h).
+ *     Index order in [B,T,H,X] arrays is b slowest, X fastest.
+ *   - dtype SDM_F32 is IEEE binary32, SDM_BF16 is bfloat16 (round-to-nearest-
+ *     even on every store).
+ *   - Not thread-safe with respect to one stream; distinct streams may call
+ *     concurrently. The only library-wide state is the per-device error word
+ *     and the thread-local message behind sdm_last_error().
+ */
+#ifndef SDM_B200_SDM_H_
+#define SDM_B200_SDM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SDM_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SDM_API __attribute__((visibility("default")))
+#else
+#define SDM_API
+#endif
+
+typedef enum sdm_status {
+  SDM_OK = 0,
+  SDM_ERR_INVALID_ARGUMENT = 1, /* a null pointer, a size out of range, misalignment */
+  SDM_ERR_UNSUPPORTED = 2,      /* valid but outside what the kernels implement */
+  SDM_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
+  SDM_ERR_DEVICE_FAULT = 4      /* the device error word was set (see sdm_stream_check) */
+} sdm_status_t;
+
+typedef enum sdm_dtype { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype_t;
+
+/* Which recurrence kernel runs (sdm_shape_t.variant). */
+typedef enum sdm_variant {
+  SDM_VARIANT_AUTO = 0,      /* pick by size: resident when the state tile fits */
+  SDM_VARIANT_RESIDENT = 1,  /* the (b,h) state column tile lives in shared memory */
+  SDM_VARIANT_STREAMING = 2  /* the state stays in global memory; rows are gathered
+                                ahead of use and scattered back */
+} sdm_variant_t;
+
+/* One layer call.
+ *   B, T, H   >= 0 (T == 0 is a no-op apart from state initialisation)
+ *   sqrt_n    in [1, 1024]; N = sqrt_n * sqrt_n slots per head
+ *   W, R      write / read slots per token-head, in [1, min(N, 256)]
+ *   d_v       columns per slot, a multiple of 16, <= 8192
+ *   in_dtype    dtype of k', q', v, alpha, beta, g
+ *   state_dtype dtype of M0, M (the recurrence computes in fp32 and rounds on store)
+ *   rms_eps   epsilon of the optional RMS-norm epilogue
+ *   variant   an sdm_variant_t value */
+typedef struct sdm_shape {
+  int32_t B, T, H;
+  int32_t sqrt_n;
+  int32_t W, R;
+  int32_t d_v;
+  int32_t in_dtype;
+  int32_t state_dtype;
+  float rms_eps;
+  int32_t variant;
+} sdm_shape_t;
+
+/* ABI version of the loaded library (SDM_ABI_VERSION). */
+SDM_API int32_t sdm_abi_version(void);
+
+/* Static text for a status code. */
+SDM_API const char* sdm_status_string(sdm_status_t status);
+
+/* Text describing the last error returned on the calling host thread ("" if none). */
+SDM_API const char* sdm_last_error(void);
+
+/* Product-key top-k selection ([explainer] 3.1 step 1; [summary] Core Mechanism 2).
+ * For every token-head, x = scores[b,t,h,:] is split into s1 = x[0:sqrt_n] and
+ * s2 = x[sqrt_n:2*sqrt_n]. Slot i = a*sqrt_n + b has score s1[a] + s2[b]. The K
+ * slots first in the order (exact real sum descending, slot ascending) are
+ * found via topk(s1 (+) s2) = topk(topk(s1) (+) topk(s2)) without forming the N
+ * sums; -0 and +0 are equal. The weights are the softmax of the K selected
+ * scores, each score rounded to fp32 (the pages leave these weights undefined;
+ * this is the reading the library implements).
+ *   scores  [B,T,H,2*sqrt_n] in_dtype (NaN gives an unspecified but in-range selection)
+ *   idx_out [B,T,H,K] int32, slots in selection order
+ *   w_out   [B,T,H,K] fp32, softmax weights aligned with idx_out
+ *   K in [1, min(N, 256)]. */
+SDM_API sdm_status_t sdm_pkm_topk(const void* scores, int32_t in_dtype, int32_t B, int32_t T, int32_t H,
+                          int32_t sqrt_n, int32_t K, int32_t* idx_out, float* w_out, void* stream);
+
+/* Bytes of workspace sdm_scan needs for this shape (0 for invalid shapes). */
+SDM_API size_t sdm_scan_workspace_bytes(const sdm_shape_t* shape);
+
+/* The recurrence kernel sdm_scan / sdm_layer_forward would run for this shape
+ * on the current device: SDM_VARIANT_RESIDENT or SDM_VARIANT_STREAMING, or -1
+ * if the shape is invalid or unsupported (sdm_last_error() says why). */
+SDM_API int32_t sdm_scan_variant(const sdm_shape_t* shape);
+
+/* The sparse gated delta recurrence over a given selection, in token order
+ * ([explainer] 3.1 steps 2-3; [summary] Core Mechanism 3-4). For each token t
+ * and head: for every write slot i (distinct within a token),
+ *     M[i] <- M~ + beta_t * k_i * (v_t - M~),  M~ = alpha_t * M[i]
+ * (computed as (alpha_t*(1 - beta_t*k_i)) * M[i] + (beta_t*k_i) * v_t in fp32),
+ * other slots untouched; then y_t = sum_r q_r * M[r] over the read slots, on
+ * the updated state. With g != NULL, y_t <- g_t * y_t / sqrt(mean(y_t^2) + rms_eps).
+ *   idx_w, w_w [B,T,H,W] int32 / fp32;  idx_r, w_r [B,T,H,R] int32 / fp32
+ *   v     [B,T,H,d_v] in_dtype;  alpha, beta [B,T,H] in_dtype
+ *   g     [B,T,H,d_v] in_dtype or NULL
+ *   M     [B,H,N,d_v] state_dtype, read as M_0 and overwritten with M_T, so calls
+ *         over consecutive token ranges chain exactly
+ *   y     [B,T,H,d_v] fp32 output
+ *   workspace: device scratch of at least sdm_scan_workspace_bytes(shape), 16-byte
+ *         aligned, not read before it is written.
+ * Write indices repeated within one token-head give unspecified values. */
+SDM_API sdm_status_t sdm_scan(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w,
+                      const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
+                      const void* beta, const void* g, void* M, float* y, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* M[b] <- M0 for every batch row b (the learned initial state of the
+ * [explainer] 3.1 "learned initial state" paragraph, shared by all rows).
+ *   M0 [H,N,d_v] state_dtype;  M [B,H,N,d_v] state_dtype. */
+SDM_API sdm_status_t sdm_state_init(const sdm_shape_t* shape, const void* M0, void* M, void* stream);
+
+/* Bytes of workspace sdm_layer_forward needs for this shape (0 for invalid shapes). */
+SDM_API size_t sdm_layer_forward_workspace_bytes(const sdm_shape_t* shape);
+
+/* One SDM layer core: selection on k' (top-W) and q' (top-R), M_out <- M0 for
+ * every batch row, the recurrence, and the optional epilogue.
+ *   kp, qp [B,T,H,2*sqrt_n] in_dtype;  v, alpha, beta, g as in sdm_scan
+ *   M0     [H,N,d_v] state_dtype (not modified);  M_out [B,H,N,d_v] state_dtype (M_T)
+ *   y      [B,T,H,d_v] fp32
+ *   workspace: at least sdm_layer_forward_workspace_bytes(shape). */
+SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp,
+                               const void* v, const void* alpha, const void* beta, const void* g,
+                               const void* M0, void* M_out, float* y, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* sdm_layer_forward that also records caller-created CUDA events (cudaEvent_t
+ * passed as void*) on `stream` between its stages, for timing each kernel in
+ * place: events[0] before the selection on k', [1] after the selection on q',
+ * [2] after the record build, [3] after the state initialisation, [4] after
+ * the recurrence kernel, [5] after the epilogue (a stage that does not run
+ * leaves its event adjacent to the previous one). n_events must be 0 (no
+ * events; events may be NULL) or 6. */
+SDM_API sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const void* kp, const void* qp,
+                                      const void* v, const void* alpha, const void* beta,
+                                      const void* g, const void* M0, void* M_out, float* y,
+                                      void* workspace, size_t workspace_bytes, void* stream,
+                                      void* const* events, int32_t n_events);
+
+/* Waits for `stream`, then reads and clears the current device's error word.
+ * Returns SDM_ERR_DEVICE_FAULT if it was set (sdm_last_error() gives the bits),
+ * SDM_ERR_CUDA if the synchronisation failed, else SDM_OK. */
+SDM_API sdm_status_t sdm_stream_check(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDM_B200_SDM_H_ */

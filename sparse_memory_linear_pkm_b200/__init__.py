@@ -1,1 +1,155 @@
-"""B200-native Sparse Delta Memory recurrent core (placeholder during bring-up)."""
+"""B200-native (sm_100a) Sparse Delta Memory recurrent core.
+
+Python front end of the C ABI in include/sdm.h. Tensors are torch CUDA tensors
+(torch provides device memory and the current stream); every step of the
+computation runs in libsdm_b200.so, which must be built
+(``python -m sparse_memory_linear_pkm_b200.build``). There is no CPU path.
+
+    y, M_T = layer_forward(kp, qp, v, alpha, beta, M0, W=64, R=64)
+
+Layouts: kp, qp [B,T,H,2*sqrt_n]; v, g [B,T,H,d_v]; alpha, beta [B,T,H];
+M0 [H,N,d_v]; M [B,H,N,d_v]; y [B,T,H,d_v] fp32; idx, w [B,T,H,K].
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import native, synth
+from .native import SdmError
+
+__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "stream_check", "make_shape",
+           "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
+
+_DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
+
+
+def _code(t: torch.Tensor, what: str) -> int:
+    try:
+        return _DTYPE[t.dtype]
+    except KeyError:
+        raise TypeError(f"{what} must be float32 or bfloat16, got {t.dtype}") from None
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def make_shape(B, T, H, sqrt_n, W, R, d_v, in_dtype=torch.bfloat16, state_dtype=torch.float32,
+               rms_eps: float = 1e-6, variant: str = "auto") -> native.Shape:
+    return native.Shape(B, T, H, sqrt_n, W, R, d_v, _DTYPE[in_dtype], _DTYPE[state_dtype], rms_eps,
+                        native.VARIANTS[variant])
+
+
+def scan_variant(shape: native.Shape) -> str:
+    """'resident' or 'streaming': the recurrence kernel this shape runs on the current device."""
+    v = int(native.load().sdm_scan_variant(ctypes.byref(shape)))
+    if v < 0:
+        native.check(1)
+    return {1: "resident", 2: "streaming"}[v]
+
+
+def scan_workspace_bytes(shape: native.Shape) -> int:
+    return int(native.load().sdm_scan_workspace_bytes(ctypes.byref(shape)))
+
+
+def layer_forward_workspace_bytes(shape: native.Shape) -> int:
+    return int(native.load().sdm_layer_forward_workspace_bytes(ctypes.byref(shape)))
+
+
+def _workspace(nbytes: int, device, workspace: torch.Tensor | None) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace needs {nbytes} bytes")
+        return workspace
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def pkm_topk(scores: torch.Tensor, K: int):
+    """Product-key top-K of s1 (+) s2 per token-head; returns (idx int32, w fp32)."""
+    B, T, H, two_n = scores.shape
+    lib = native.load()
+    idx = torch.empty((B, T, H, K), dtype=torch.int32, device=scores.device)
+    w = torch.empty((B, T, H, K), dtype=torch.float32, device=scores.device)
+    native.check(lib.sdm_pkm_topk(_ptr(scores), _code(scores, "scores"), B, T, H, two_n // 2, K, _ptr(idx),
+                                  _ptr(w), _stream(scores.device)))
+    return idx, w
+
+
+def scan(idx_w, w_w, idx_r, w_r, v, alpha, beta, M, g=None, eps: float = 1e-6, variant: str = "auto",
+         y: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The write/read recurrence over a given selection. M [B,H,N,d_v] is
+    updated in place (M_0 -> M_T); returns y [B,T,H,d_v] fp32."""
+    B, T, H, W = idx_w.shape
+    R = idx_r.shape[-1]
+    d_v = v.shape[-1]
+    N = M.shape[2]
+    sqrt_n = int(round(N ** 0.5))
+    shape = native.Shape(B, T, H, sqrt_n, W, R, d_v, _code(v, "v"), _code(M, "M"), eps, native.VARIANTS[variant])
+    lib = native.load()
+    if y is None:
+        y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=v.device)
+    ws = _workspace(scan_workspace_bytes(shape), v.device, workspace)
+    native.check(lib.sdm_scan(ctypes.byref(shape), _ptr(idx_w), _ptr(w_w), _ptr(idx_r), _ptr(w_r), _ptr(v),
+                              _ptr(alpha), _ptr(beta), _ptr(g), _ptr(M), _ptr(y), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(v.device)))
+    return y
+
+
+def state_init(M0: torch.Tensor, B: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """M[b] <- M0 for b in [0, B)."""
+    H, N, d_v = M0.shape
+    sqrt_n = int(round(N ** 0.5))
+    M = out if out is not None else torch.empty((B, H, N, d_v), dtype=M0.dtype, device=M0.device)
+    shape = native.Shape(B, 1, H, sqrt_n, 1, 1, d_v, native.F32, _code(M0, "M0"), 1e-6, 0)
+    native.check(native.load().sdm_state_init(ctypes.byref(shape), _ptr(M0), _ptr(M), _stream(M0.device)))
+    return M
+
+
+def layer_forward(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float = 1e-6,
+                  variant: str = "auto", y: torch.Tensor | None = None, M_out: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, events=None):
+    """Selection (top-W of k', top-R of q'), M_out <- M0 per batch row, the
+    recurrence and the optional RMS-norm x g epilogue. Returns (y, M_out).
+
+    ``events``: optional list of 6 already-created torch.cuda.Event objects
+    recorded between the stages (see sdm_layer_forward_traced in sdm.h)."""
+    B, T, H, two_n = kp.shape
+    d_v = v.shape[-1]
+    shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M0, "M0"), eps,
+                         native.VARIANTS[variant])
+    lib = native.load()
+    if y is None:
+        y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=kp.device)
+    if M_out is None:
+        M_out = torch.empty((B,) + tuple(M0.shape), dtype=M0.dtype, device=kp.device)
+    ws = _workspace(layer_forward_workspace_bytes(shape), kp.device, workspace)
+    if events is None:
+        ev, n_ev = None, 0
+    else:
+        if len(events) != 6:
+            raise ValueError("events must hold 6 torch.cuda.Event objects")
+        ev, n_ev = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events]), 6
+    native.check(lib.sdm_layer_forward_traced(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha),
+                                              _ptr(beta), _ptr(g), _ptr(M0), _ptr(M_out), _ptr(y), _ptr(ws),
+                                              ws.numel() * ws.element_size(), _stream(kp.device), ev, n_ev))
+    return y, M_out
+
+
+def stream_check(device: torch.device | None = None) -> None:
+    """Synchronises the current stream and raises SdmError if a kernel set the
+    device error word (an index outside [0, N), an expired bounded wait)."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    native.check(native.load().sdm_stream_check(_stream(device)))

@@ -1,0 +1,564 @@
+// C ABI of the SDM recurrent core: argument validation, workspace carving and
+// kernel dispatch. See include/sdm.h for the contract of every entry point.
+//
+// This is the single translation unit of libsdm_b200.so; the kernels live in
+// the included headers.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "sdm.h"
+#include "pkm_topk.cuh"
+#include "sdm_misc.cuh"
+#include "sdm_records.cuh"
+#include "sdm_scan.cuh"
+
+namespace {
+
+using sdm::bf16;
+
+// The per-device error word (one copy per device context).
+__device__ unsigned g_device_error;
+
+thread_local std::string g_last_error;
+
+sdm_status_t fail(sdm_status_t s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+sdm_status_t ok() {
+  g_last_error.clear();
+  return SDM_OK;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem_optin = 0;
+  unsigned* err = nullptr;
+  bool ready = false;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+sdm_status_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SDM_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(SDM_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+            cudaSuccess ||
+        (e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_device_error)) != cudaSuccess)
+      return fail(SDM_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(e));
+    d.ready = true;
+  }
+  *out = &d;
+  return SDM_OK;
+}
+
+sdm_status_t launch_status(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SDM_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return SDM_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int64_t slots_of(int32_t sqrt_n) { return static_cast<int64_t>(sqrt_n) * sqrt_n; }
+
+sdm_status_t check_dtype(int32_t d, const char* name) {
+  if (d != SDM_F32 && d != SDM_BF16) return fail(SDM_ERR_INVALID_ARGUMENT, std::string(name) + " is not SDM_F32 or SDM_BF16");
+  return SDM_OK;
+}
+
+sdm_status_t check_k(int32_t K, int32_t sqrt_n, const char* name) {
+  const int64_t lim = std::min<int64_t>(slots_of(sqrt_n), 256);
+  if (K < 1 || K > lim)
+    return fail(SDM_ERR_INVALID_ARGUMENT, std::string(name) + " must be in [1, min(N, 256)], got " + std::to_string(K));
+  return SDM_OK;
+}
+
+sdm_status_t check_shape(const sdm_shape_t* s) {
+  if (s == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "shape is NULL");
+  if (s->B < 0 || s->T < 0 || s->H < 0) return fail(SDM_ERR_INVALID_ARGUMENT, "B, T and H must be >= 0");
+  if (s->sqrt_n < 1 || s->sqrt_n > 1024) return fail(SDM_ERR_INVALID_ARGUMENT, "sqrt_n must be in [1, 1024]");
+  sdm_status_t st;
+  if ((st = check_k(s->W, s->sqrt_n, "W")) != SDM_OK) return st;
+  if ((st = check_k(s->R, s->sqrt_n, "R")) != SDM_OK) return st;
+  if (s->d_v < 16 || s->d_v > 8192 || s->d_v % 16 != 0)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "d_v must be a multiple of 16 in [16, 8192]");
+  if ((st = check_dtype(s->in_dtype, "in_dtype")) != SDM_OK) return st;
+  if ((st = check_dtype(s->state_dtype, "state_dtype")) != SDM_OK) return st;
+  if (!(s->rms_eps >= 0.0f) || s->rms_eps > 1e30f) return fail(SDM_ERR_INVALID_ARGUMENT, "rms_eps must be finite and >= 0");
+  if (s->variant < SDM_VARIANT_AUTO || s->variant > SDM_VARIANT_STREAMING)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "variant must be an sdm_variant_t value");
+  if (static_cast<int64_t>(s->B) * s->H > 65535) return fail(SDM_ERR_UNSUPPORTED, "B*H above 65535");
+  return SDM_OK;
+}
+
+sdm_status_t need_ptr(const void* p, const char* name, bool nonempty) {
+  if (!nonempty) return SDM_OK;
+  if (p == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, std::string(name) + " is NULL");
+  if (!aligned16(p)) return fail(SDM_ERR_INVALID_ARGUMENT, std::string(name) + " is not 16-byte aligned");
+  return SDM_OK;
+}
+
+size_t in_size(int32_t d) { return d == SDM_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------------- selection --
+
+sdm::TopkLayout topk_layout(int n, int K) {
+  sdm::TopkLayout L{};
+  L.n = n;
+  L.K = K;
+  L.Kh = std::min(K, n);
+  int C = 0;
+  for (int ra = 0; ra < L.Kh; ++ra) C += std::min(L.Kh, K / (ra + 1));
+  L.C = C;
+  auto a16 = [](uint32_t x) { return (x + 15u) & ~15u; };
+  L.table_bytes = a16(static_cast<uint32_t>(C) * 4u);
+  uint32_t off = 0;
+  auto take = [&](uint32_t bytes) {
+    const uint32_t o = off;
+    off += a16(bytes);
+    return o;
+  };
+  L.vals = take(2u * n * 4u);
+  L.hist = take(256u * 4u);
+  L.hkey = take(static_cast<uint32_t>(L.Kh) * 8u);
+  L.hval = take(2u * L.Kh * 4u);
+  L.hidx = take(2u * L.Kh * 4u);
+  L.c_hi = take(C * 4u);
+  L.c_lo = take(C * 4u);
+  L.c_slot = take(C * 4u);
+  L.tie = take(C * 2u);
+  L.f_hi = take(K * 4u);
+  L.f_lo = take(K * 4u);
+  L.f_slot = take(K * 4u);
+  L.warp_bytes = off;
+  return L;
+}
+
+template <typename Tin>
+sdm_status_t launch_topk(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K, int32_t* idx,
+                         float* w, cudaStream_t st) {
+  if (units == 0) return SDM_OK;
+  const sdm::TopkLayout L = topk_layout(n, K);
+  int warps = 4;
+  while (warps > 1 && L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes > static_cast<size_t>(dev.max_smem_optin))
+    --warps;
+  const size_t smem = L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes;
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return fail(SDM_ERR_UNSUPPORTED, "selection scratch exceeds shared memory");
+  auto kern = sdm::k_pkm_topk<Tin>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const int64_t blocks_needed = (units + warps - 1) / warps;
+  const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, static_cast<int64_t>(dev.sms) * 16));
+  kern<<<grid, warps * 32, smem, st>>>(static_cast<const Tin*>(scores), units, L, idx, w);
+  return launch_status("pkm_topk launch");
+}
+
+sdm_status_t topk_impl(const DeviceInfo& dev, const void* scores, int32_t in_dtype, int64_t units, int n, int K,
+                       int32_t* idx, float* w, cudaStream_t st) {
+  return in_dtype == SDM_BF16 ? launch_topk<bf16>(dev, scores, units, n, K, idx, w, st)
+                              : launch_topk<float>(dev, scores, units, n, K, idx, w, st);
+}
+
+// ------------------------------------------------------------ recurrence --
+
+sdm::RecLayout rec_layout(int W, int R) {
+  sdm::RecLayout rl{};
+  rl.Wp = (W + 3) / 4 * 4;
+  rl.Rp = (R + 3) / 4 * 4;
+  rl.Fp = (W + R + 7) / 8 * 8;
+  rl.off_slot_w = 0;
+  rl.off_k_w = rl.Wp;
+  rl.off_slot_r = 2 * rl.Wp;
+  rl.off_q_r = 2 * rl.Wp + rl.Rp;
+  rl.off_fwd = 2 * rl.Wp + 2 * rl.Rp;
+  rl.off_ab = rl.off_fwd + rl.Fp / 2;
+  rl.words = rl.off_ab + 4;
+  return rl;
+}
+
+size_t records_bytes(const sdm_shape_t& s) {
+  return align256(static_cast<size_t>(s.B) * s.H * s.T * rec_layout(s.W, s.R).words * 4u);
+}
+
+struct ScanChoice {
+  bool resident = false;
+  int C = 16;
+  int P = 4;
+  int L = 16;
+  size_t smem = 0;
+};
+
+size_t resident_smem(const sdm_shape_t& s, int C, int L) {
+  const sdm::RecLayout rl = rec_layout(s.W, s.R);
+  return static_cast<size_t>(slots_of(s.sqrt_n)) * C * 4 + 2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) +
+         2ull * sdm::kScanWarps * C * 4 + 16;
+}
+size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L) {
+  const sdm::RecLayout rl = rec_layout(s.W, s.R);
+  return 2ull * P * (s.W + s.R) * C * in_size(s.state_dtype) + 2ull * L * rl.words * 4 +
+         2ull * L * C * in_size(s.in_dtype) + 2ull * sdm::kScanWarps * C * 4 + 16;
+}
+
+sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
+  const size_t lim = static_cast<size_t>(dev.max_smem_optin);
+  ScanChoice c;
+  if (s.variant != SDM_VARIANT_STREAMING) {
+    c.C = s.d_v % 32 == 0 ? 32 : 16;
+    for (int L : {16, 8, 4}) {
+      if (resident_smem(s, c.C, L) <= lim) {
+        c.resident = true;
+        c.L = L;
+        c.smem = resident_smem(s, c.C, L);
+        break;
+      }
+    }
+    if (c.resident) {
+      *out = c;
+      return SDM_OK;
+    }
+    if (s.variant == SDM_VARIANT_RESIDENT)
+      return fail(SDM_ERR_UNSUPPORTED, "the state tile does not fit in shared memory (resident variant)");
+  }
+  c.resident = false;
+  const int cst = s.state_dtype == SDM_BF16 ? 32 : 16;
+  c.C = s.d_v % cst == 0 ? cst : 16;
+  for (int P : {4, 2}) {
+    for (int L : {16, 8}) {
+      if (L > P && streaming_smem(s, c.C, P, L) <= lim) {
+        c.P = P;
+        c.L = L;
+        c.smem = streaming_smem(s, c.C, P, L);
+        *out = c;
+        return SDM_OK;
+      }
+    }
+  }
+  return fail(SDM_ERR_UNSUPPORTED, "W + R too large for the streaming stage ring");
+}
+
+template <typename Tin>
+sdm_status_t launch_records(const sdm_shape_t& s, const int32_t* idx_w, const float* w_w, const int32_t* idx_r,
+                            const float* w_r, const void* alpha, const void* beta, int P, uint32_t* rec,
+                            unsigned* err, const DeviceInfo& dev, cudaStream_t st) {
+  const sdm::RecLayout rl = rec_layout(s.W, s.R);
+  int log2_cells = 1;
+  while ((1 << log2_cells) < 2 * s.W) ++log2_cells;
+  const size_t smem =
+      P > 0 ? static_cast<size_t>(sdm::kRecTokensPerBlock + P - 1) * (size_t{1} << log2_cells) * 4 : 0;
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return fail(SDM_ERR_UNSUPPORTED, "hazard tables exceed shared memory");
+  auto kern = sdm::k_build_records<Tin>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const int tblocks = (s.T + sdm::kRecTokensPerBlock - 1) / sdm::kRecTokensPerBlock;
+  const dim3 grid(tblocks, s.B * s.H);
+  kern<<<grid, 256, smem, st>>>(idx_w, w_w, idx_r, w_r, static_cast<const Tin*>(alpha), static_cast<const Tin*>(beta),
+                                s.T, s.H, static_cast<int>(slots_of(s.sqrt_n)), s.W, s.R, P, log2_cells, rl, rec, err);
+  return launch_status("record build launch");
+}
+
+template <typename Tin, typename Tst>
+sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cudaStream_t st) {
+  const dim3 grid(a.B * a.H, a.d_v / c.C);
+  void (*kern)(sdm::ScanArgs) = nullptr;
+  if (c.resident) {
+    if (c.C == 32) {
+      if (c.L == 16) kern = sdm::k_scan_resident<Tin, Tst, 32, 16>;
+      else if (c.L == 8) kern = sdm::k_scan_resident<Tin, Tst, 32, 8>;
+      else kern = sdm::k_scan_resident<Tin, Tst, 32, 4>;
+    } else {
+      if (c.L == 16) kern = sdm::k_scan_resident<Tin, Tst, 16, 16>;
+      else if (c.L == 8) kern = sdm::k_scan_resident<Tin, Tst, 16, 8>;
+      else kern = sdm::k_scan_resident<Tin, Tst, 16, 4>;
+    }
+  } else {
+    if (c.C == 32) {
+      if (c.P == 4) kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 32, 4, 16> : sdm::k_scan_streaming<Tin, Tst, 32, 4, 8>;
+      else kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 32, 2, 16> : sdm::k_scan_streaming<Tin, Tst, 32, 2, 8>;
+    } else {
+      if (c.P == 4) kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 16, 4, 16> : sdm::k_scan_streaming<Tin, Tst, 16, 4, 8>;
+      else kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 16, 2, 16> : sdm::k_scan_streaming<Tin, Tst, 16, 2, 8>;
+    }
+  }
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
+  kern<<<grid, sdm::kScanThreads, c.smem, st>>>(a);
+  return launch_status("scan launch");
+}
+
+sdm_status_t launch_scan(const ScanChoice& c, const sdm_shape_t& s, const sdm::ScanArgs& a, cudaStream_t st) {
+  if (s.in_dtype == SDM_BF16)
+    return s.state_dtype == SDM_BF16 ? launch_scan_typed<bf16, bf16>(c, a, st) : launch_scan_typed<bf16, float>(c, a, st);
+  return s.state_dtype == SDM_BF16 ? launch_scan_typed<float, bf16>(c, a, st) : launch_scan_typed<float, float>(c, a, st);
+}
+
+sdm_status_t launch_state_init(const DeviceInfo& dev, const sdm_shape_t& s, const void* M0, void* M, cudaStream_t st) {
+  const int64_t bytes_per_row = static_cast<int64_t>(s.H) * slots_of(s.sqrt_n) * s.d_v * static_cast<int64_t>(in_size(s.state_dtype));
+  const int64_t units = bytes_per_row / 16;
+  if (units == 0 || s.B == 0) return SDM_OK;
+  const int gx = static_cast<int>(std::min<int64_t>((units + 255) / 256, std::max(1, dev.sms * 8 / std::max(1, s.B))));
+  for (int b0 = 0; b0 < s.B; b0 += 65535) {
+    const int nb = std::min(65535, s.B - b0);
+    sdm::k_state_init<<<dim3(gx, nb), 256, 0, st>>>(static_cast<const uint4*>(M0),
+                                                   static_cast<uint4*>(M) + static_cast<int64_t>(b0) * units, units);
+  }
+  return launch_status("state init launch");
+}
+
+sdm_status_t launch_epilogue(const DeviceInfo& dev, const sdm_shape_t& s, float* y, const void* g, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(s.B) * s.T * s.H;
+  if (rows == 0) return SDM_OK;
+  const int grid = static_cast<int>(std::min<int64_t>((rows + 7) / 8, static_cast<int64_t>(dev.sms) * 16));
+  if (s.in_dtype == SDM_BF16)
+    sdm::k_rmsnorm_gate<bf16><<<grid, 256, 0, st>>>(y, static_cast<const bf16*>(g), rows, s.d_v, s.rms_eps);
+  else
+    sdm::k_rmsnorm_gate<float><<<grid, 256, 0, st>>>(y, static_cast<const float*>(g), rows, s.d_v, s.rms_eps);
+  return launch_status("epilogue launch");
+}
+
+// Records + recurrence (+ epilogue). With M_in != M the resident kernel reads
+// M_in (b-stride M_in_b_stride) and writes M; the streaming kernel works in
+// place on M, which then must already hold the initial state.
+// Records a caller event (no-op without events).
+struct Trace {
+  void* const* events = nullptr;
+  void mark(int i, cudaStream_t st) const {
+    if (events != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+  }
+};
+
+sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanChoice& c, const int32_t* idx_w,
+                      const float* w_w, const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
+                      const void* beta, const void* g, const void* M_in, int64_t M_in_b_stride, void* M, float* y,
+                      uint32_t* rec, cudaStream_t st, const Trace& tr = Trace(), bool init_before_scan = false,
+                      const void* M0_for_init = nullptr) {
+  sdm_status_t r;
+  if ((r = (s.in_dtype == SDM_BF16 ? launch_records<bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, c.resident ? 0 : c.P,
+                                                          rec, dev.err, dev, st)
+                                   : launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, c.resident ? 0 : c.P,
+                                                           rec, dev.err, dev, st))) != SDM_OK)
+    return r;
+  tr.mark(2, st);
+  if (init_before_scan && (r = launch_state_init(dev, s, M0_for_init, M, st)) != SDM_OK) return r;
+  tr.mark(3, st);
+  sdm::ScanArgs a{};
+  a.B = s.B; a.T = s.T; a.H = s.H;
+  a.N = static_cast<int>(slots_of(s.sqrt_n));
+  a.d_v = s.d_v; a.W = s.W; a.R = s.R;
+  a.rl = rec_layout(s.W, s.R);
+  a.rec = rec;
+  a.v = v;
+  a.M_in = M_in;
+  a.M_in_b_stride = M_in_b_stride;
+  a.M = M;
+  a.y = y;
+  a.err = dev.err;
+  if ((r = launch_scan(c, s, a, st)) != SDM_OK) return r;
+  tr.mark(4, st);
+  if (g != nullptr && (r = launch_epilogue(dev, s, y, g, st)) != SDM_OK) return r;
+  tr.mark(5, st);
+  return SDM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sdm_abi_version(void) { return SDM_ABI_VERSION; }
+
+const char* sdm_status_string(sdm_status_t status) {
+  switch (status) {
+    case SDM_OK: return "ok";
+    case SDM_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case SDM_ERR_UNSUPPORTED: return "unsupported";
+    case SDM_ERR_CUDA: return "CUDA error";
+    case SDM_ERR_DEVICE_FAULT: return "device-side fault";
+  }
+  return "unknown status";
+}
+
+const char* sdm_last_error(void) { return g_last_error.c_str(); }
+
+sdm_status_t sdm_pkm_topk(const void* scores, int32_t in_dtype, int32_t B, int32_t T, int32_t H, int32_t sqrt_n,
+                          int32_t K, int32_t* idx_out, float* w_out, void* stream) {
+  sdm_status_t r;
+  if ((r = check_dtype(in_dtype, "in_dtype")) != SDM_OK) return r;
+  if (B < 0 || T < 0 || H < 0) return fail(SDM_ERR_INVALID_ARGUMENT, "B, T and H must be >= 0");
+  if (sqrt_n < 1 || sqrt_n > 1024) return fail(SDM_ERR_INVALID_ARGUMENT, "sqrt_n must be in [1, 1024]");
+  if ((r = check_k(K, sqrt_n, "K")) != SDM_OK) return r;
+  const int64_t units = static_cast<int64_t>(B) * T * H;
+  if ((r = need_ptr(scores, "scores", units > 0)) != SDM_OK) return r;
+  if ((r = need_ptr(idx_out, "idx_out", units > 0)) != SDM_OK) return r;
+  if ((r = need_ptr(w_out, "w_out", units > 0)) != SDM_OK) return r;
+  if (units == 0) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  if ((r = topk_impl(*dev, scores, in_dtype, units, sqrt_n, K, idx_out, w_out, static_cast<cudaStream_t>(stream))) != SDM_OK)
+    return r;
+  return ok();
+}
+
+size_t sdm_scan_workspace_bytes(const sdm_shape_t* shape) {
+  const std::string saved = g_last_error;
+  if (check_shape(shape) != SDM_OK) return 0;
+  g_last_error = saved;
+  return records_bytes(*shape);
+}
+
+int32_t sdm_scan_variant(const sdm_shape_t* shape) {
+  DeviceInfo* dev;
+  ScanChoice c;
+  if (check_shape(shape) != SDM_OK || device_info(&dev) != SDM_OK || choose_scan(*dev, *shape, &c) != SDM_OK)
+    return -1;
+  ok();
+  return c.resident ? SDM_VARIANT_RESIDENT : SDM_VARIANT_STREAMING;
+}
+
+sdm_status_t sdm_scan(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w, const int32_t* idx_r,
+                      const float* w_r, const void* v, const void* alpha, const void* beta, const void* g, void* M,
+                      float* y, void* workspace, size_t workspace_bytes, void* stream) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  const bool any = static_cast<int64_t>(s.B) * s.T * s.H > 0;
+  if ((r = need_ptr(idx_w, "idx_w", any)) || (r = need_ptr(w_w, "w_w", any)) || (r = need_ptr(idx_r, "idx_r", any)) ||
+      (r = need_ptr(w_r, "w_r", any)) || (r = need_ptr(v, "v", any)) || (r = need_ptr(alpha, "alpha", any)) ||
+      (r = need_ptr(beta, "beta", any)) || (r = need_ptr(M, "M", any)) || (r = need_ptr(y, "y", any)))
+    return r;
+  if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
+  if (!any) return ok();
+  const size_t need = records_bytes(s);
+  if (workspace_bytes < need)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "workspace_bytes below sdm_scan_workspace_bytes() = " + std::to_string(need));
+  if ((r = need_ptr(workspace, "workspace", true)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  ScanChoice c;
+  if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
+  const int64_t row_stride = static_cast<int64_t>(s.H) * slots_of(s.sqrt_n) * s.d_v;
+  if ((r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M, row_stride, M, y,
+                    static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream))) != SDM_OK)
+    return r;
+  return ok();
+}
+
+sdm_status_t sdm_state_init(const sdm_shape_t* shape, const void* M0, void* M, void* stream) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const bool any = static_cast<int64_t>(shape->B) * shape->H > 0;
+  if ((r = need_ptr(M0, "M0", any)) != SDM_OK || (r = need_ptr(M, "M", any)) != SDM_OK) return r;
+  if (!any) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  if ((r = launch_state_init(*dev, *shape, M0, M, static_cast<cudaStream_t>(stream))) != SDM_OK) return r;
+  return ok();
+}
+
+size_t sdm_layer_forward_workspace_bytes(const sdm_shape_t* shape) {
+  const std::string saved = g_last_error;
+  if (check_shape(shape) != SDM_OK) return 0;
+  g_last_error = saved;
+  const sdm_shape_t& s = *shape;
+  const size_t th = static_cast<size_t>(s.B) * s.T * s.H;
+  return 2 * align256(th * s.W * 4) + 2 * align256(th * s.R * 4) + records_bytes(s);
+}
+
+sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                      const void* alpha, const void* beta, const void* g, const void* M0,
+                                      void* M_out, float* y, void* workspace, size_t workspace_bytes, void* stream,
+                                      void* const* events, int32_t n_events) {
+  sdm_status_t r;
+  if (!(n_events == 0 || (n_events == 6 && events != nullptr)))
+    return fail(SDM_ERR_INVALID_ARGUMENT, "n_events must be 0, or 6 with a non-NULL events array");
+  Trace tr;
+  if (n_events == 6) {
+    for (int i = 0; i < 6; ++i)
+      if (events[i] == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "events[] holds a NULL event");
+    tr.events = events;
+  }
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  const int64_t th = static_cast<int64_t>(s.B) * s.T * s.H;
+  const bool any = th > 0;
+  const bool any_state = static_cast<int64_t>(s.B) * s.H > 0;
+  if ((r = need_ptr(kp, "kp", any)) || (r = need_ptr(qp, "qp", any)) || (r = need_ptr(v, "v", any)) ||
+      (r = need_ptr(alpha, "alpha", any)) || (r = need_ptr(beta, "beta", any)) || (r = need_ptr(y, "y", any)) ||
+      (r = need_ptr(M0, "M0", any_state)) || (r = need_ptr(M_out, "M_out", any_state)))
+    return r;
+  if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
+  if (!any_state) return ok();
+  const size_t need = sdm_layer_forward_workspace_bytes(shape);
+  if (any && workspace_bytes < need)
+    return fail(SDM_ERR_INVALID_ARGUMENT,
+                "workspace_bytes below sdm_layer_forward_workspace_bytes() = " + std::to_string(need));
+  if (any && (r = need_ptr(workspace, "workspace", true)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!any) return launch_state_init(*dev, s, M0, M_out, st) == SDM_OK ? ok() : SDM_ERR_CUDA;
+  ScanChoice c;
+  if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(ws);
+  ws += align256(th * s.W * 4);
+  float* w_w = reinterpret_cast<float*>(ws);
+  ws += align256(th * s.W * 4);
+  int32_t* idx_r = reinterpret_cast<int32_t*>(ws);
+  ws += align256(th * s.R * 4);
+  float* w_r = reinterpret_cast<float*>(ws);
+  ws += align256(th * s.R * 4);
+  uint32_t* rec = reinterpret_cast<uint32_t*>(ws);
+  tr.mark(0, st);
+  if ((r = topk_impl(*dev, kp, s.in_dtype, th, s.sqrt_n, s.W, idx_w, w_w, st)) != SDM_OK) return r;
+  if ((r = topk_impl(*dev, qp, s.in_dtype, th, s.sqrt_n, s.R, idx_r, w_r, st)) != SDM_OK) return r;
+  tr.mark(1, st);
+  if (c.resident) {
+    r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M0, 0, M_out, y, rec, st, tr);
+  } else {
+    r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M_out, 0, M_out, y, rec, st, tr,
+                 /*init_before_scan=*/true, M0);
+  }
+  if (r != SDM_OK) return r;
+  return ok();
+}
+
+sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                               const void* alpha, const void* beta, const void* g, const void* M0, void* M_out,
+                               float* y, void* workspace, size_t workspace_bytes, void* stream) {
+  return sdm_layer_forward_traced(shape, kp, qp, v, alpha, beta, g, M0, M_out, y, workspace, workspace_bytes,
+                                  stream, nullptr, 0);
+}
+
+sdm_status_t sdm_stream_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SDM_ERR_CUDA, std::string("cudaStreamSynchronize: ") + cudaGetErrorString(e));
+  DeviceInfo* dev;
+  sdm_status_t r;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  unsigned word = 0;
+  if ((e = cudaMemcpy(&word, dev->err, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return fail(SDM_ERR_CUDA, std::string("reading the device error word: ") + cudaGetErrorString(e));
+  if (word != 0) {
+    const unsigned zero = 0;
+    cudaMemcpy(dev->err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    std::string msg = "device error word 0x" + std::to_string(word) + ":";
+    if (word & sdm::kErrIndexOutOfRange) msg += " slot index outside [0, N) skipped;";
+    if (word & sdm::kErrWaitTimeout) msg += " bounded wait expired;";
+    return fail(SDM_ERR_DEVICE_FAULT, msg);
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,102 @@
+"""The C ABI library loads on the CPU and exports what include/sdm.h declares;
+host-side validation answers without touching a GPU."""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from sparse_memory_linear_pkm_b200 import build as build_mod
+from sparse_memory_linear_pkm_b200 import native
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "sdm.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return native.load()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    return set(re.findall(r"SDM_API\s+[\w\s\*]+?\b(sdm_\w+)\s*\(", text))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == set(native.PROTOTYPES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.sdm_abi_version() == 1
+
+
+def test_only_the_abi_is_exported(lib):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", str(native.LIBRARY)], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert exported == declared_functions()
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert lib.sdm_status_string(code)
+    assert lib.sdm_status_string(99) == b"unknown status"
+
+
+def shape(**kw):
+    d = dict(B=2, T=5, H=3, sqrt_n=8, W=4, R=4, d_v=32, in_dtype=native.BF16, state_dtype=native.F32,
+             rms_eps=1e-6, variant=0)
+    d.update(kw)
+    return native.Shape(**d)
+
+
+@pytest.mark.parametrize("bad", [dict(sqrt_n=0), dict(sqrt_n=1025), dict(W=0), dict(R=65), dict(W=257, sqrt_n=32),
+                                 dict(d_v=24), dict(d_v=8), dict(B=-1), dict(in_dtype=7), dict(variant=3),
+                                 dict(rms_eps=-1.0)])
+def test_invalid_shapes_rejected_on_host(lib, bad):
+    s = shape(**bad)
+    assert lib.sdm_scan_workspace_bytes(ctypes.byref(s)) == 0
+    assert lib.sdm_layer_forward_workspace_bytes(ctypes.byref(s)) == 0
+    st = lib.sdm_scan(ctypes.byref(s), *([None] * 10), None, 0, None)
+    assert st == 1 and lib.sdm_last_error()
+
+
+def test_workspace_sizes(lib):
+    s = shape()
+    rec_words = 4 + 4 + 4 + 4 + 8 // 2 + 4  # Wp, Wp, Rp, Rp, Fp/2, alpha/beta block
+    rec = (2 * 3 * 5 * rec_words * 4 + 255) // 256 * 256
+    assert lib.sdm_scan_workspace_bytes(ctypes.byref(s)) == rec
+    per = (2 * 5 * 3 * 4 * 4 + 255) // 256 * 256
+    assert lib.sdm_layer_forward_workspace_bytes(ctypes.byref(s)) == 4 * per + rec
+
+
+def test_argument_errors_without_gpu(lib):
+    # null pointers and K out of range are caught before any CUDA call
+    assert lib.sdm_pkm_topk(None, native.F32, 1, 1, 1, 4, 3, None, None, None) == 1
+    assert b"scores" in lib.sdm_last_error()
+    assert lib.sdm_pkm_topk(None, native.F32, 1, 1, 1, 4, 17, None, None, None) == 1
+    assert b"K" in lib.sdm_last_error()
+    # misaligned pointer
+    assert lib.sdm_pkm_topk(ctypes.c_void_p(8), native.F32, 1, 1, 1, 4, 3, ctypes.c_void_p(16),
+                            ctypes.c_void_p(32), None) == 1
+    assert b"aligned" in lib.sdm_last_error()
+    # empty problems are no-ops
+    assert lib.sdm_pkm_topk(None, native.F32, 0, 7, 3, 4, 3, None, None, None) == 0
+    s = shape(T=0)
+    assert lib.sdm_scan(ctypes.byref(s), *([None] * 10), None, 0, None) == 0
+    # too little workspace
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.sdm_scan(ctypes.byref(s), *([fake] * 7), None, fake, fake, fake, 16, None)
+    assert st == 1 and b"workspace" in lib.sdm_last_error()
+
+
+def test_build_flags_target_sm100a():
+    assert build_mod.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
