@@ -177,6 +177,31 @@ SDM_API sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const vo
                                       void* workspace, size_t workspace_bytes, void* stream,
                                       void* const* events, int32_t n_events);
 
+/* sdm_layer_forward for callers that cannot hand the library any device
+ * memory for scratch -- for example a plugin inside a host engine that owns
+ * the whole device pool and offers no workspace, or a latency-bound loop that
+ * must not call an allocator after start-up (cudaMalloc can synchronise the
+ * device and stall). The caller still passes every input and output; the
+ * scratch comes from one array of SDM_NOALLOC_SCRATCH_BYTES (16 MiB) that the
+ * library keeps in device memory on every GPU that loads it, until the
+ * process exits. Nothing is allocated or freed here.
+ *   - Shapes whose sdm_layer_forward_workspace_bytes() exceeds
+ *     SDM_NOALLOC_SCRATCH_BYTES are rejected with SDM_ERR_INVALID_ARGUMENT.
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up per device); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array and it keeps what the last
+ *     call left there (no part of it needs to start at zero). Calls whose work
+ *     overlaps on the GPU -- on different streams, or from different host
+ *     threads -- race on it; order them on one stream.
+ * The paper has no counterpart to this entry point; it is an interface for
+ * such hosts. Arguments and results are as in sdm_layer_forward. */
+#define SDM_NOALLOC_SCRATCH_BYTES (16u << 20)
+SDM_API sdm_status_t sdm_layer_forward_noalloc(const sdm_shape_t* shape, const void* kp, const void* qp,
+                                       const void* v, const void* alpha, const void* beta,
+                                       const void* g, const void* M0, void* M_out, float* y,
+                                       void* stream);
+
 /* Waits for `stream`, then reads and clears the current device's error word.
  * Returns SDM_ERR_DEVICE_FAULT if it was set (sdm_last_error() gives the bits),
  * SDM_ERR_CUDA if the synchronisation failed, else SDM_OK. */

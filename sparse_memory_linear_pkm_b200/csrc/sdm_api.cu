@@ -372,6 +372,33 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
   return SDM_OK;
 }
 
+// Scratch of sdm_layer_forward_noalloc. In host code this name only stands
+// for the device array; its device address comes from cudaGetSymbolAddress,
+// once per device (noalloc_scratch below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SDM_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up on
+// first use with that device current.
+sdm_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SDM_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(SDM_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(SDM_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SDM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -539,6 +566,21 @@ sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const v
                                float* y, void* workspace, size_t workspace_bytes, void* stream) {
   return sdm_layer_forward_traced(shape, kp, qp, v, alpha, beta, g, M0, M_out, y, workspace, workspace_bytes,
                                   stream, nullptr, 0);
+}
+
+sdm_status_t sdm_layer_forward_noalloc(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                       const void* alpha, const void* beta, const void* g, const void* M0,
+                                       void* M_out, float* y, void* stream) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const size_t need = sdm_layer_forward_workspace_bytes(shape);
+  if (need > SDM_NOALLOC_SCRATCH_BYTES)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "this shape needs " + std::to_string(need) +
+                                              " bytes of scratch; the built-in scratch holds " +
+                                              std::to_string(SDM_NOALLOC_SCRATCH_BYTES) + " bytes");
+  void* ws = nullptr;
+  if ((r = noalloc_scratch(&ws)) != SDM_OK) return r;
+  return sdm_layer_forward(shape, kp, qp, v, alpha, beta, g, M0, M_out, y, ws, SDM_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 sdm_status_t sdm_stream_check(void* stream) {

@@ -17,6 +17,7 @@ STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARGUMENT", 2: "SDM_ERR_UNSUPPOR
                 4: "SDM_ERR_DEVICE_FAULT"}
 F32, BF16 = 0, 1
 VARIANTS = {"auto": 0, "resident": 1, "streaming": 2}
+NOALLOC_SCRATCH_BYTES = 16 << 20  # SDM_NOALLOC_SCRATCH_BYTES in include/sdm.h
 
 
 class Shape(ctypes.Structure):
@@ -47,6 +48,7 @@ PROTOTYPES = {
     "sdm_layer_forward": (_i32, [_shape_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "sdm_layer_forward_traced": (_i32, [_shape_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p,
                                          ctypes.POINTER(_p), _i32]),
+    "sdm_layer_forward_noalloc": (_i32, [_shape_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p]),
     "sdm_stream_check": (_i32, [_p]),
 }
 
