@@ -139,7 +139,7 @@ __device__ __forceinline__ void warp_half_topk(const float* v, int n, int Kh, ui
 }
 
 template <typename Tin>
-__global__ void __launch_bounds__(128) k_pkm_topk(const Tin* __restrict__ scores, int64_t n_units,
+__global__ void __launch_bounds__(128) k_pkm_topk_general(const Tin* __restrict__ scores, int64_t n_units,
                                                   TopkLayout L, int32_t* __restrict__ idx_out,
                                                   float* __restrict__ w_out) {
   extern __shared__ __align__(16) unsigned char smem[];

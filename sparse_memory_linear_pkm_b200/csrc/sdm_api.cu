@@ -9,11 +9,14 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
+#include <vector>
 #include <mutex>
 #include <string>
 
 #include "sdm.h"
 #include "pkm_topk.cuh"
+#include "pkm_topk_fast.cuh"
 #include "sdm_misc.cuh"
 #include "sdm_records.cuh"
 #include "sdm_scan.cuh"
@@ -150,17 +153,79 @@ sdm::TopkLayout topk_layout(int n, int K) {
   return L;
 }
 
+template <typename Tin, int E, int EH, int EPL, int CP>
+sdm_status_t launch_topk_fast_inst(const DeviceInfo& dev, const Tin* scores, int64_t units,
+                                   const sdm::FastTopkLayout& L, int32_t* idx, float* w, cudaStream_t st) {
+  auto kern = sdm::k_pkm_topk_fast<Tin, E, EH, EPL, CP>;
+  const size_t smem = L.table_bytes + static_cast<size_t>(sdm::kFastTopkWarps) * L.warp_bytes;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  int per_sm = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sdm::kFastTopkWarps * 32, smem);
+  const int64_t blocks_needed = (units + sdm::kFastTopkWarps - 1) / sdm::kFastTopkWarps;
+  const int grid =
+      static_cast<int>(std::min<int64_t>(blocks_needed, static_cast<int64_t>(dev.sms) * std::max(1, per_sm) * 4));
+  kern<<<grid, sdm::kFastTopkWarps * 32, smem, st>>>(scores, units, L, idx, w);
+  return launch_status("pkm_topk launch");
+}
+
+// Register path for K <= 64.
+template <typename Tin>
+sdm_status_t launch_topk_fast(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K,
+                              int32_t* idx, float* w, cudaStream_t st) {
+  sdm::FastTopkLayout L{};
+  L.n = n;
+  L.K = K;
+  L.Kh = std::min(K, n);
+  int C = 0;
+  for (int ra = 0; ra < L.Kh; ++ra) C += std::min(L.Kh, K / (ra + 1));
+  L.C = C;
+  const int E = K <= 32 ? 1 : 2;                 // winners sort width / 32
+  const int EH = n <= 32 ? 1 : E;                // half sort width / 32
+  const int CP = E == 1 ? 4 : (EH == 1 ? 7 : 9);
+  if (C > 32 * CP) return fail(SDM_ERR_UNSUPPORTED, "selection candidate count above the register path");
+  auto a16 = [](uint32_t x) { return (x + 15u) & ~15u; };
+  L.table_bytes = a16(static_cast<uint32_t>(C) * 4u);
+  uint32_t off = 0;
+  auto take = [&](uint32_t bytes) {
+    const uint32_t o = off;
+    off += a16(bytes);
+    return o;
+  };
+  L.hist = take(256u * 4u);
+  L.sel = take(64u * 8u);
+  L.hv = take(2u * 64u * 4u);
+  L.hx = take(2u * 64u * 4u);
+  L.tie = take(2u * 4u * 32u * CP);
+  L.warp_bytes = off;
+  const Tin* x = static_cast<const Tin*>(scores);
+  int epl = 1;
+  if (n > 32 * EH) {
+    while (epl * 32 < n) epl *= 2;
+  }
+#define SDM_FAST_TOPK(E_, EH_, EPL_, CP_)                      \
+  if (E == E_ && EH == EH_ && epl == EPL_ && CP == CP_) \
+    return launch_topk_fast_inst<Tin, E_, EH_, EPL_, CP_>(dev, x, units, L, idx, w, st);
+  SDM_FAST_TOPK(1, 1, 1, 4) SDM_FAST_TOPK(1, 1, 2, 4) SDM_FAST_TOPK(1, 1, 4, 4) SDM_FAST_TOPK(1, 1, 8, 4)
+  SDM_FAST_TOPK(1, 1, 16, 4) SDM_FAST_TOPK(1, 1, 32, 4)
+  SDM_FAST_TOPK(2, 1, 1, 7)
+  SDM_FAST_TOPK(2, 2, 1, 9) SDM_FAST_TOPK(2, 2, 4, 9) SDM_FAST_TOPK(2, 2, 8, 9)
+  SDM_FAST_TOPK(2, 2, 16, 9) SDM_FAST_TOPK(2, 2, 32, 9)
+#undef SDM_FAST_TOPK
+  return fail(SDM_ERR_UNSUPPORTED, "no selection kernel for this sqrt_n and K");
+}
+
 template <typename Tin>
 sdm_status_t launch_topk(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K, int32_t* idx,
                          float* w, cudaStream_t st) {
   if (units == 0) return SDM_OK;
+  if (K <= sdm::kFastTopkMaxK) return launch_topk_fast<Tin>(dev, scores, units, n, K, idx, w, st);
   const sdm::TopkLayout L = topk_layout(n, K);
   int warps = 4;
   while (warps > 1 && L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes > static_cast<size_t>(dev.max_smem_optin))
     --warps;
   const size_t smem = L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes;
   if (smem > static_cast<size_t>(dev.max_smem_optin)) return fail(SDM_ERR_UNSUPPORTED, "selection scratch exceeds shared memory");
-  auto kern = sdm::k_pkm_topk<Tin>;
+  auto kern = sdm::k_pkm_topk_general<Tin>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   const int64_t blocks_needed = (units + warps - 1) / warps;
   const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, static_cast<int64_t>(dev.sms) * 16));
@@ -195,6 +260,16 @@ size_t records_bytes(const sdm_shape_t& s) {
   return align256(static_cast<size_t>(s.B) * s.H * s.T * rec_layout(s.W, s.R).words * 4u);
 }
 
+// Instantiated streaming tiles: columns per CTA, prefetch distance, staging chunk.
+struct StreamCfg {
+  int state_bytes;
+  int C, P, L;
+};
+constexpr StreamCfg kStreamCfgs[] = {
+    {4, 64, 3, 8}, {4, 64, 2, 8}, {4, 32, 6, 8}, {4, 32, 4, 8}, {4, 16, 8, 16}, {4, 16, 4, 8},
+    {2, 128, 3, 8}, {2, 64, 6, 8}, {2, 64, 4, 8}, {2, 32, 12, 16}, {2, 32, 8, 16}, {2, 16, 8, 16}, {2, 16, 4, 8},
+};
+
 struct ScanChoice {
   bool resident = false;
   int C = 16;
@@ -203,27 +278,38 @@ struct ScanChoice {
   size_t smem = 0;
 };
 
+size_t ypart_bytes(int C) { return static_cast<size_t>((2 * sdm::kScanWarps * (C + 1) + 3) & ~3) * 4; }
+
 size_t resident_smem(const sdm_shape_t& s, int C, int L) {
   const sdm::RecLayout rl = rec_layout(s.W, s.R);
   return static_cast<size_t>(slots_of(s.sqrt_n)) * C * 4 + 2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) +
-         2ull * sdm::kScanWarps * C * 4 + 16;
+         ypart_bytes(C) + 2 * 8;
 }
 size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L) {
   const sdm::RecLayout rl = rec_layout(s.W, s.R);
-  return 2ull * P * (s.W + s.R) * C * in_size(s.state_dtype) + 2ull * L * rl.words * 4 +
-         2ull * L * C * in_size(s.in_dtype) + 2ull * sdm::kScanWarps * C * 4 + 16;
+  return sdm::streaming_stage_bytes(P, s.W + s.R, s.W, C, static_cast<int>(in_size(s.state_dtype))) +
+         2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) + ypart_bytes(C) + 2 * 8;
 }
 
 sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
   const size_t lim = static_cast<size_t>(dev.max_smem_optin);
   ScanChoice c;
   if (s.variant != SDM_VARIANT_STREAMING) {
-    c.C = s.d_v % 32 == 0 ? 32 : 16;
-    for (int L : {16, 8, 4}) {
-      if (resident_smem(s, c.C, L) <= lim) {
+    // Resident tiles (C columns, staging chunk L), best first; "C,L" in
+    // SDM_RESIDENT_CFG forces one (tuning).
+    std::vector<std::pair<int, int>> order = {{32, 16}, {32, 8}, {16, 8}, {16, 16}, {32, 4}, {16, 4}};
+    if (const char* env = std::getenv("SDM_RESIDENT_CFG")) {
+      int C = 0, L = 0;
+      if (std::sscanf(env, "%d,%d", &C, &L) == 2) order.insert(order.begin(), {C, L});
+    }
+    for (const auto& cl : order) {
+      const int C = cl.first, L = cl.second;
+      if (s.d_v % C != 0 || (L != 16 && L != 8 && L != 4) || (C != 16 && C != 32)) continue;
+      if (resident_smem(s, C, L) <= lim) {
         c.resident = true;
+        c.C = C;
         c.L = L;
-        c.smem = resident_smem(s, c.C, L);
+        c.smem = resident_smem(s, C, L);
         break;
       }
     }
@@ -235,17 +321,42 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
       return fail(SDM_ERR_UNSUPPORTED, "the state tile does not fit in shared memory (resident variant)");
   }
   c.resident = false;
-  const int cst = s.state_dtype == SDM_BF16 ? 32 : 16;
-  c.C = s.d_v % cst == 0 ? cst : 16;
-  for (int P : {4, 2}) {
-    for (int L : {16, 8}) {
-      if (L > P && streaming_smem(s, c.C, P, L) <= lim) {
-        c.P = P;
-        c.L = L;
-        c.smem = streaming_smem(s, c.C, P, L);
-        *out = c;
-        return SDM_OK;
-      }
+  // Streaming tiles, best first. Random row segments of >= 256 B run HBM near
+  // its copy bandwidth, 128 B at ~75%, 64 B at ~40% (measured gathers on
+  // B200), so wide segments win while the grid still fills the SMs.
+  const int s_state = static_cast<int>(in_size(s.state_dtype));
+  const int64_t bh = static_cast<int64_t>(s.B) * s.H;
+  std::vector<StreamCfg> order;
+  for (const StreamCfg& k : kStreamCfgs) {
+    if (k.state_bytes != s_state || s.d_v % k.C != 0) continue;
+    order.push_back(k);
+  }
+  auto ctas = [&](const StreamCfg& k) { return bh * (s.d_v / k.C); };
+  std::stable_sort(order.begin(), order.end(), [&](const StreamCfg& x, const StreamCfg& y) {
+    const bool fx = ctas(x) >= dev.sms / 2, fy = ctas(y) >= dev.sms / 2;  // fills at least half the SMs
+    if (fx != fy) return fx;
+    const int rx = x.C * x.state_bytes, ry = y.C * y.state_bytes;
+    if (rx != ry) return rx > ry;  // wider row segments first
+    return x.P > y.P;
+  });
+  if (const char* env = std::getenv("SDM_STREAM_CFG")) {  // tuning override "C,P,L"
+    int C = 0, P = 0, L = 0;
+    if (std::sscanf(env, "%d,%d,%d", &C, &P, &L) == 3) {
+      std::vector<StreamCfg> forced;
+      for (const StreamCfg& k : order)
+        if (k.C == C && k.P == P && k.L == L) forced.push_back(k);
+      if (!forced.empty()) order = forced;
+    }
+  }
+  for (const StreamCfg& k : order) {
+    const size_t need = streaming_smem(s, k.C, k.P, k.L);
+    if (need <= lim) {
+      c.C = k.C;
+      c.P = k.P;
+      c.L = k.L;
+      c.smem = need;
+      *out = c;
+      return SDM_OK;
     }
   }
   return fail(SDM_ERR_UNSUPPORTED, "W + R too large for the streaming stage ring");
@@ -285,14 +396,18 @@ sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cuda
       else kern = sdm::k_scan_resident<Tin, Tst, 16, 4>;
     }
   } else {
-    if (c.C == 32) {
-      if (c.P == 4) kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 32, 4, 16> : sdm::k_scan_streaming<Tin, Tst, 32, 4, 8>;
-      else kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 32, 2, 16> : sdm::k_scan_streaming<Tin, Tst, 32, 2, 8>;
+#define SDM_STREAM(C_, P_, L_) \
+    if (c.C == C_ && c.P == P_ && c.L == L_) kern = sdm::k_scan_streaming<Tin, Tst, C_, P_, L_>;
+    if constexpr (sizeof(Tst) == 4) {
+      SDM_STREAM(64, 3, 8) SDM_STREAM(64, 2, 8) SDM_STREAM(32, 6, 8) SDM_STREAM(32, 4, 8)
+      SDM_STREAM(16, 8, 16) SDM_STREAM(16, 4, 8)
     } else {
-      if (c.P == 4) kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 16, 4, 16> : sdm::k_scan_streaming<Tin, Tst, 16, 4, 8>;
-      else kern = c.L == 16 ? sdm::k_scan_streaming<Tin, Tst, 16, 2, 16> : sdm::k_scan_streaming<Tin, Tst, 16, 2, 8>;
+      SDM_STREAM(128, 3, 8) SDM_STREAM(64, 6, 8) SDM_STREAM(64, 4, 8) SDM_STREAM(32, 12, 16)
+      SDM_STREAM(32, 8, 16) SDM_STREAM(16, 8, 16) SDM_STREAM(16, 4, 8)
     }
+#undef SDM_STREAM
   }
+  if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no streaming kernel for the chosen tile");
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
   kern<<<grid, sdm::kScanThreads, c.smem, st>>>(a);
   return launch_status("scan launch");

@@ -9,22 +9,25 @@
 // to the state dtype on every store.
 //
 // Every column of d_v evolves independently given the per-token scalars, so a
-// CTA owns one (b, h) and a tile of C columns and walks all T tokens. Within a
-// token the W writes touch distinct slots and run in parallel, one thread per
-// (entry, 16-byte unit); a barrier separates them from the R reads, whose
-// partial sums are reduced in a fixed order (bit-reproducible y). Per-token
-// records and v rows are staged a chunk of L tokens at a time with 1-D bulk
-// copies (no multicast) into a double buffer tracked by mbarriers.
+// CTA owns one (b, h) and a tile of C columns and walks all T tokens. A row
+// segment of the tile is U 16-byte units; lane q%U of a warp handles unit q
+// of one entry and a warp instruction covers 32/U entries, so each entry's
+// metadata is read once per U lanes and v_t stays in registers for the whole
+// token. The W writes of a token touch distinct slots and run in parallel; a
+// barrier separates them from the R reads, whose partial sums are reduced in a
+// fixed order (bit-reproducible y). Per-token records and v rows are staged a
+// chunk of L tokens at a time by 1-D bulk copies (no multicast) into a double
+// buffer tracked by mbarriers with bounded waits.
 //
 //   k_scan_resident  : the (b, h) column tile of the state lives in shared
 //                      memory (fp32) for the whole sequence; M_in is read once
 //                      and M_out written once. Two barriers per token.
 //   k_scan_streaming : the state stays in global memory. The rows of token t+P
-//                      are gathered (cp.async, 16 B per thread) while token t
-//                      computes, into a ring of 2P stages; the hazard plan in
-//                      the record forwards rows written by the tokens in
-//                      between from their stage. Written rows are stored back
-//                      to global memory at once.
+//                      are gathered (16-byte cp.async per lane) into a
+//                      ring of P+1 load stages while token t computes; the
+//                      hazard plan in the record forwards rows written by the
+//                      tokens in between from a ring of P written-row stages.
+//                      Written rows are stored back to global memory at once.
 #pragma once
 
 #include "sdm_device.cuh"
@@ -32,7 +35,7 @@
 
 namespace sdm {
 
-constexpr int kScanThreads = 256;
+constexpr int kScanThreads = 512;
 constexpr int kScanWarps = kScanThreads / kWarp;
 
 struct ScanArgs {
@@ -50,21 +53,19 @@ struct ScanArgs {
 // Loads VE consecutive input elements (VE * sizeof(Tin) bytes, aligned) as fp32.
 template <typename Tin, int VE>
 __device__ __forceinline__ void load_in_vec(const Tin* p, float* out) {
+  static_assert(VE % 4 == 0, "vectors of 4");
   if constexpr (sizeof(Tin) == 4) {
-    static_assert(VE % 4 == 0, "fp32 vectors of 4");
 #pragma unroll
     for (int i = 0; i < VE; i += 4) {
       const float4 f = *reinterpret_cast<const float4*>(p + i);
       out[i] = f.x; out[i + 1] = f.y; out[i + 2] = f.z; out[i + 3] = f.w;
     }
   } else {
-    static_assert(VE % 4 == 0, "bf16 vectors of 4");
 #pragma unroll
     for (int i = 0; i < VE; i += 4) {
       const uint2 u = *reinterpret_cast<const uint2*>(p + i);
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-      const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+      const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+      const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
       out[i] = fa.x; out[i + 1] = fa.y; out[i + 2] = fb.x; out[i + 3] = fb.y;
     }
   }
@@ -124,33 +125,55 @@ __device__ __forceinline__ void issue_chunk(const ScanArgs& a, int bh, int b, in
   }
 }
 
+// y of one token from the per-warp partials ypart[w][0:C) (row stride C+1):
+// warp v sums columns [v*C/NW, (v+1)*C/NW), 16 lanes per column.
+template <int C>
+__device__ __forceinline__ void reduce_y_store(const float* yp, float* yrow, int warp, int lane) {
+  constexpr int CPW = C / kScanWarps;  // columns per warp
+  static_assert(C % kScanWarps == 0 && kScanWarps == 16, "16 warps, C a multiple of 16");
+  const int part = lane & 15;
+#pragma unroll
+  for (int cc = 0; cc < (CPW + 1) / 2; ++cc) {
+    const int sub = cc * 2 + (lane >> 4);
+    const bool valid = sub < CPW;
+    const int col = warp * CPW + (valid ? sub : 0);
+    float s = valid ? yp[part * (C + 1) + col] : 0.f;
+    s += __shfl_xor_sync(0xffffffffu, s, 8);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    if (valid && part == 0) yrow[col] = s;
+  }
+}
+
 // ------------------------------------------------------------ resident ----
 
 template <typename Tin, typename Tst, int C, int L>
-__global__ void __launch_bounds__(kScanThreads) k_scan_resident(ScanArgs a) {
-  constexpr int U = C / 4;  // 16-byte units of an fp32 row segment
-  static_assert(kScanThreads % U == 0, "a thread keeps one unit column");
+__global__ void __launch_bounds__(kScanThreads, 1) k_scan_resident(ScanArgs a) {
+  constexpr int U = C / 4;         // 16-byte units of an fp32 row segment
+  constexpr int G = kWarp / U;     // entries per warp instruction
+  constexpr int GS = G * kScanWarps;
   extern __shared__ __align__(16) unsigned char smem[];
   const int N = a.N, W = a.W, R = a.R, T = a.T;
   const int words = a.rl.words;
   float* S = reinterpret_cast<float*>(smem);  // [N][C]
   uint32_t* recbuf = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(N) * C * 4);
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);
-  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][warps][C]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + 2 * kScanWarps * C);
+  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][warps][C+1]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + ((2 * kScanWarps * (C + 1) + 3) & ~3));
 
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int c0 = blockIdx.y * C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int q = tid % U;
+  const int g = lane / U, q = lane % U;
+  const int e0 = g + G * warp;  // first entry of this lane group
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     fence_mbar_init();
   }
-  // Initial state tile.
-  {
+  {  // initial state tile
     constexpr int VE = 16 / sizeof(Tst);
     const Tst* Min = static_cast<const Tst*>(a.M_in) + b * a.M_in_b_stride +
                      static_cast<int64_t>(h) * N * a.d_v + c0;
@@ -159,7 +182,8 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_resident(ScanArgs a) {
       float f[VE];
       unpack16<Tst>(*reinterpret_cast<const uint4*>(Min + static_cast<int64_t>(row) * a.d_v + u * VE), f);
 #pragma unroll
-      for (int i = 0; i < VE; ++i) S[row * C + u * VE + i] = f[i];
+      for (int i = 0; i < VE; i += 4)
+        *reinterpret_cast<float4*>(S + row * C + u * VE + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
     }
   }
   __syncthreads();
@@ -177,20 +201,20 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_resident(ScanArgs a) {
     const uint32_t* recs = recbuf + static_cast<size_t>(bi) * L * words;
     const Tin* vs = vbuf + static_cast<size_t>(bi) * L * C;
     const int nt = min(L, T - c * L);
+#pragma unroll 1
     for (int i = 0; i < nt; ++i) {
       const int t = c * L + i;
       const uint32_t* rec = recs + i * words;
       const float alpha = __uint_as_float(rec[a.rl.off_ab]);
       const float beta = __uint_as_float(rec[a.rl.off_ab + 1]);
-      // Write: W distinct slots, one (entry, unit) per thread.
-      for (int x = tid; x < W * U; x += kScanThreads) {
-        const int e = x / U;
+      float vv[4];
+      load_in_vec<Tin, 4>(vs + i * C + 4 * q, vv);
+      // Write: W distinct slots.
+      for (int e = e0; e < W; e += GS) {
         const int slot = static_cast<int>(rec[a.rl.off_slot_w + e]);
         if (slot < 0) continue;
         const float cw = beta * __uint_as_float(rec[a.rl.off_k_w + e]);
         const float aw = alpha * (1.0f - cw);
-        float vv[4];
-        load_in_vec<Tin, 4>(vs + i * C + 4 * q, vv);
         float4* p = reinterpret_cast<float4*>(S + slot * C + 4 * q);
         float4 m = *p;
         m.x = round_to<Tst>(fmaf(aw, m.x, cw * vv[0]));
@@ -202,8 +226,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_resident(ScanArgs a) {
       __syncthreads();
       // Read after the write.
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int x = tid; x < R * U; x += kScanThreads) {
-        const int r = x / U;
+      for (int r = e0; r < R; r += GS) {
         const int slot = static_cast<int>(rec[a.rl.off_slot_r + r]);
         if (slot < 0) continue;
         const float qw = __uint_as_float(rec[a.rl.off_q_r + r]);
@@ -217,15 +240,13 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_resident(ScanArgs a) {
       for (int o = U; o < kWarp; o <<= 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-      float* yp = ypart + (t & 1) * kScanWarps * C;
-      if (lane < U) *reinterpret_cast<float4*>(yp + warp * C + 4 * lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      __syncthreads();
-      if (tid < C) {
-        float s = 0.f;
+      float* yp = ypart + (t & 1) * kScanWarps * (C + 1);
+      if (lane < U) {
 #pragma unroll
-        for (int w = 0; w < kScanWarps; ++w) s += yp[w * C + tid];
-        y_bh[(static_cast<int64_t>(b) * T + t) * a.H * a.d_v + tid] = s;
+        for (int j = 0; j < 4; ++j) yp[warp * (C + 1) + 4 * q + j] = acc[j];
       }
+      __syncthreads();
+      reduce_y_store<C>(yp, y_bh + (static_cast<int64_t>(b) * T + t) * a.H * a.d_v, warp, lane);
     }
     // Every thread is past the last read of buffer bi (barrier above).
     if (tid == 0 && c + 2 < n_chunks) {
@@ -247,26 +268,37 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_resident(ScanArgs a) {
 
 // ----------------------------------------------------------- streaming ----
 
+// Shared-memory bytes of k_scan_streaming (host and device agree on this).
+__host__ __device__ constexpr size_t streaming_stage_bytes(int P, int E, int W, int C, int s_state) {
+  return (static_cast<size_t>(P + 1) * E + static_cast<size_t>(P) * W) * C * s_state;
+}
+
 template <typename Tin, typename Tst, int C, int P, int L>
-__global__ void __launch_bounds__(kScanThreads) k_scan_streaming(ScanArgs a) {
+__global__ void __launch_bounds__(kScanThreads, 1) k_scan_streaming(ScanArgs a) {
   constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
   constexpr int U = C / VE;             // units per row segment
-  constexpr int S = 2 * P;              // stage ring
-  static_assert(kScanThreads % U == 0, "a thread keeps one unit column");
+  constexpr int G = kWarp / U;          // entries per warp instruction
+  constexpr int GS = G * kScanWarps;
+  constexpr int SL = P + 1;             // load stages: current token + P in flight
+  constexpr int SW = P;                 // written-row stages: current token + P-1 before it
+  constexpr uint32_t RS = C * sizeof(Tst);
   static_assert(L > P, "a chunk must be staged before its tokens are gathered");
+  static_assert(kWarp % U == 0, "a row segment spans a divisor of the warp");
   extern __shared__ __align__(16) unsigned char smem[];
   const int W = a.W, R = a.R, T = a.T, E = W + R;
   const int words = a.rl.words;
-  Tst* stage = reinterpret_cast<Tst*>(smem);  // [S][E][C]
-  uint32_t* recbuf = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(S) * E * C * sizeof(Tst));
+  unsigned char* lstage = smem;                                    // [SL][E][RS]
+  unsigned char* wstage = smem + static_cast<size_t>(SL) * E * RS;  // [SW][W][RS]
+  uint32_t* recbuf = reinterpret_cast<uint32_t*>(smem + streaming_stage_bytes(P, E, W, C, sizeof(Tst)));
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);
-  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][warps][C]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + 2 * kScanWarps * C);
+  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][warps][C+1]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + ((2 * kScanWarps * (C + 1) + 3) & ~3));
 
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int c0 = blockIdx.y * C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int q = tid % U;
+  const int g = lane / U, q = lane % U;
+  const int e0 = g + G * warp;
   Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * a.N * a.d_v + c0;
   float* y_bh = a.y + static_cast<int64_t>(h) * a.d_v + c0;
 
@@ -276,16 +308,19 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_streaming(ScanArgs a) {
   auto fwd_of = [&](const uint32_t* rec, int e) -> int {
     return reinterpret_cast<const int16_t*>(rec + a.rl.off_fwd)[e];
   };
-  auto row_ptr = [&](int t, int e) -> Tst* { return stage + (static_cast<size_t>(t % S) * E + e) * C; };
-  // Gathers the rows of token t that the plan does not forward.
+  // Gathers the rows of token t that the plan does not forward: one 16-byte
+  // cp.async per (entry, unit), one commit group per call. (One bulk copy per
+  // row issued by a single warp measured ~3x slower: issue-bound.)
   auto gather = [&](int t) {
     const uint32_t* rec = rec_of(t);
-    for (int x = tid; x < E * U; x += kScanThreads) {
-      const int e = x / U, u = x % U;
+    const int st = t % SL;
+    for (int e = e0; e < E; e += GS) {
       const int slot = static_cast<int>(e < W ? rec[a.rl.off_slot_w + e] : rec[a.rl.off_slot_r + e - W]);
       if (slot >= 0 && fwd_of(rec, e) < 0)
-        cp_async16(row_ptr(t, e) + u * VE, Mbh + static_cast<int64_t>(slot) * a.d_v + u * VE);
+        cp_async16(lstage + (static_cast<size_t>(st) * E + e) * RS + q * 16,
+                   Mbh + static_cast<int64_t>(slot) * a.d_v + q * VE);
     }
+    cp_async_commit();
   };
 
   if (tid == 0) {
@@ -304,12 +339,12 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_streaming(ScanArgs a) {
     const bool ok = mbar_wait_bounded(&bars[0], 0, a.err);
     if (__syncthreads_or(!ok)) return;
   }
-#pragma unroll 1
   for (int t = 0; t < P; ++t) {
     if (t < T) gather(t);
-    cp_async_commit();
+    else cp_async_commit();
   }
 
+  int sl = 0, sw = 0;  // t % SL, t % SW
 #pragma unroll 1
   for (int t = 0; t < T; ++t) {
     cp_async_wait<P - 1>();
@@ -318,48 +353,60 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_streaming(ScanArgs a) {
       fence_proxy_async_smem();
       issue_chunk<Tin, C, L>(a, bh, b, h, c0, t / L + 1, recbuf, vbuf, bars);
     }
-    if (t > 0 && tid < C) {
-      const float* yp = ypart + ((t - 1) & 1) * kScanWarps * C;
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kScanWarps; ++w) s += yp[w * C + tid];
-      y_bh[(static_cast<int64_t>(b) * T + (t - 1)) * a.H * a.d_v + tid] = s;
+    if (t > 0) {
+      const float* yp = ypart + ((t - 1) & 1) * kScanWarps * (C + 1);
+      reduce_y_store<C>(yp, y_bh + (static_cast<int64_t>(b) * T + (t - 1)) * a.H * a.d_v, warp, lane);
     }
     const uint32_t* rec = rec_of(t);
     const Tin* vrow = vbuf + (static_cast<size_t>((t / L) & 1) * L + (t % L)) * C;
     const float alpha = __uint_as_float(rec[a.rl.off_ab]);
     const float beta = __uint_as_float(rec[a.rl.off_ab + 1]);
+    float vv[VE];
+    load_in_vec<Tin, VE>(vrow + q * VE, vv);
+    unsigned char* lrow = lstage + static_cast<size_t>(sl) * E * RS;
+    unsigned char* wrow = wstage + static_cast<size_t>(sw) * W * RS;
     // Write.
-    for (int x = tid; x < W * U; x += kScanThreads) {
-      const int e = x / U;
+    for (int e = e0; e < W; e += GS) {
       const int slot = static_cast<int>(rec[a.rl.off_slot_w + e]);
       if (slot < 0) continue;
       const int f = fwd_of(rec, e);
-      const Tst* src = f < 0 ? row_ptr(t, e) : row_ptr(t - (f >> 9), f & 511);
-      float m[VE], vv[VE];
-      unpack16<Tst>(*reinterpret_cast<const uint4*>(src + q * VE), m);
-      load_in_vec<Tin, VE>(vrow + q * VE, vv);
+      const unsigned char* src;
+      if (f < 0) {
+        src = lrow + e * RS;
+      } else {
+        int ws = sw - (f >> 9);
+        ws += ws < 0 ? SW : 0;
+        src = wstage + (static_cast<size_t>(ws) * W + (f & 511)) * RS;
+      }
+      float m[VE];
+      unpack16<Tst>(*reinterpret_cast<const uint4*>(src + q * 16), m);
       const float cw = beta * __uint_as_float(rec[a.rl.off_k_w + e]);
       const float aw = alpha * (1.0f - cw);
 #pragma unroll
       for (int j = 0; j < VE; ++j) m[j] = fmaf(aw, m[j], cw * vv[j]);
       const uint4 packed = pack16<Tst>(m);
-      *reinterpret_cast<uint4*>(row_ptr(t, e) + q * VE) = packed;
+      *reinterpret_cast<uint4*>(wrow + e * RS + q * 16) = packed;
       *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slot) * a.d_v + q * VE) = packed;
     }
-    __syncthreads();  // writes of t visible to the reads of t
+    __syncthreads();  // writes of t visible to the reads of t and to later gathers
     // Read after the write.
     float acc[VE];
 #pragma unroll
     for (int j = 0; j < VE; ++j) acc[j] = 0.f;
-    for (int x = tid; x < R * U; x += kScanThreads) {
-      const int r = x / U;
+    for (int r = e0; r < R; r += GS) {
       const int slot = static_cast<int>(rec[a.rl.off_slot_r + r]);
       if (slot < 0) continue;
       const int f = fwd_of(rec, W + r);
-      const Tst* src = f < 0 ? row_ptr(t, W + r) : row_ptr(t - (f >> 9), f & 511);
+      const unsigned char* src;
+      if (f < 0) {
+        src = lrow + (W + r) * RS;
+      } else {
+        int ws = sw - (f >> 9);
+        ws += ws < 0 ? SW : 0;
+        src = wstage + (static_cast<size_t>(ws) * W + (f & 511)) * RS;
+      }
       float m[VE];
-      unpack16<Tst>(*reinterpret_cast<const uint4*>(src + q * VE), m);
+      unpack16<Tst>(*reinterpret_cast<const uint4*>(src + q * 16), m);
       const float qw = __uint_as_float(rec[a.rl.off_q_r + r]);
 #pragma unroll
       for (int j = 0; j < VE; ++j) acc[j] = fmaf(qw, m[j], acc[j]);
@@ -369,32 +416,32 @@ __global__ void __launch_bounds__(kScanThreads) k_scan_streaming(ScanArgs a) {
 #pragma unroll
       for (int j = 0; j < VE; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
     if (lane < U) {
-      float* yp = ypart + (t & 1) * kScanWarps * C + warp * C + lane * VE;
+      float* yp = ypart + (t & 1) * kScanWarps * (C + 1) + warp * (C + 1) + q * VE;
 #pragma unroll
       for (int j = 0; j < VE; ++j) yp[j] = acc[j];
     }
-    // Gather token t + P (its chunk must have landed).
+    // Gather token t + P into the load stage token t - 1 used (free now).
     if (t + P < T) {
       if ((t + P) % L == 0) {
         const int c = (t + P) / L;
-        const bool ok = mbar_wait_bounded(&bars[c & 1], (c >> 1) & 1, a.err);
-        if (__syncthreads_or(!ok)) {
+        const bool okc = mbar_wait_bounded(&bars[c & 1], (c >> 1) & 1, a.err);
+        if (__syncthreads_or(!okc)) {
           cp_async_wait<0>();
           return;
         }
       }
       gather(t + P);
+    } else {
+      cp_async_commit();
     }
-    cp_async_commit();
+    sl = sl + 1 == SL ? 0 : sl + 1;
+    sw = sw + 1 == SW ? 0 : sw + 1;
   }
   cp_async_wait<0>();
   __syncthreads();
-  if (T > 0 && tid < C) {
-    const float* yp = ypart + ((T - 1) & 1) * kScanWarps * C;
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < kScanWarps; ++w) s += yp[w * C + tid];
-    y_bh[(static_cast<int64_t>(b) * T + (T - 1)) * a.H * a.d_v + tid] = s;
+  if (T > 0) {
+    const float* yp = ypart + ((T - 1) & 1) * kScanWarps * (C + 1);
+    reduce_y_store<C>(yp, y_bh + (static_cast<int64_t>(b) * T + (T - 1)) * a.H * a.d_v, warp, lane);
   }
 }
 
