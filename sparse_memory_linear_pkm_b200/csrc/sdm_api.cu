@@ -42,6 +42,7 @@ sdm_status_t ok() {
 struct DeviceInfo {
   int sms = 0;
   int max_smem_optin = 0;
+  int smem_per_sm = 0;
   unsigned* err = nullptr;
   bool ready = false;
 };
@@ -59,6 +60,8 @@ sdm_status_t device_info(DeviceInfo** out) {
   if (!d.ready) {
     if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+            cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) !=
             cudaSuccess ||
         (e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_device_error)) != cudaSuccess)
       return fail(SDM_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(e));
@@ -241,11 +244,12 @@ sdm_status_t topk_impl(const DeviceInfo& dev, const void* scores, int32_t in_dty
 
 // ------------------------------------------------------------ recurrence --
 
-sdm::RecLayout rec_layout(int W, int R) {
+// Record layout; the hazard plan is only stored for the streaming kernel.
+sdm::RecLayout rec_layout(int W, int R, bool plan = true) {
   sdm::RecLayout rl{};
   rl.Wp = (W + 3) / 4 * 4;
   rl.Rp = (R + 3) / 4 * 4;
-  rl.Fp = (W + R + 7) / 8 * 8;
+  rl.Fp = plan ? (W + R + 7) / 8 * 8 : 0;
   rl.off_slot_w = 0;
   rl.off_k_w = rl.Wp;
   rl.off_slot_r = 2 * rl.Wp;
@@ -270,20 +274,29 @@ constexpr StreamCfg kStreamCfgs[] = {
     {2, 128, 3, 8}, {2, 64, 6, 8}, {2, 64, 4, 8}, {2, 32, 12, 16}, {2, 32, 8, 16}, {2, 16, 8, 16}, {2, 16, 4, 8},
 };
 
+// Instantiated resident tiles: columns per warp, warps per CTA, staging
+// chunk, entries per lane block.
+struct ResidentCfg {
+  int CW, NWARP, L, EB;
+};
+constexpr ResidentCfg kResidentCfgs[] = {
+    {8, 1, 4, 4}, {8, 2, 4, 4}, {4, 2, 4, 2}, {16, 1, 4, 4}, {4, 4, 4, 2}, {8, 2, 8, 4}, {4, 4, 8, 2}, {8, 4, 8, 4},
+};
+
 struct ScanChoice {
   bool resident = false;
-  int C = 16;
+  int C = 16;  // columns per CTA
   int P = 4;
   int L = 16;
+  int CW = 8, NWARP = 2, EB = 4;  // resident: columns per warp, warps per CTA, entry block
   size_t smem = 0;
 };
 
 size_t ypart_bytes(int C) { return static_cast<size_t>((2 * sdm::kScanWarps * (C + 1) + 3) & ~3) * 4; }
 
-size_t resident_smem(const sdm_shape_t& s, int C, int L) {
-  const sdm::RecLayout rl = rec_layout(s.W, s.R);
-  return static_cast<size_t>(slots_of(s.sqrt_n)) * C * 4 + 2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) +
-         ypart_bytes(C) + 2 * 8;
+size_t resident_smem(const sdm_shape_t& s, const ResidentCfg& k) {
+  return sdm::resident_smem_bytes(static_cast<int>(slots_of(s.sqrt_n)), k.CW, k.NWARP, k.L,
+                                  rec_layout(s.W, s.R, false).words, static_cast<int>(in_size(s.in_dtype)));
 }
 size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L) {
   const sdm::RecLayout rl = rec_layout(s.W, s.R);
@@ -295,23 +308,31 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
   const size_t lim = static_cast<size_t>(dev.max_smem_optin);
   ScanChoice c;
   if (s.variant != SDM_VARIANT_STREAMING) {
-    // Resident tiles (C columns, staging chunk L), best first; "C,L" in
-    // SDM_RESIDENT_CFG forces one (tuning).
-    std::vector<std::pair<int, int>> order = {{32, 16}, {32, 8}, {16, 8}, {16, 16}, {32, 4}, {16, 4}};
+    // Resident tiles in order of preference (measured on B200 at N = 1024,
+    // d_v = 128: 8-column warp tiles, one warp per CTA, so up to five CTAs
+    // share an SM); the first that divides d_v and fits is taken.
+    // "CW,NWARP,L" in SDM_RESIDENT_CFG forces one (tuning).
+    std::vector<ResidentCfg> order;
+    for (const ResidentCfg& k : kResidentCfgs)
+      if (s.d_v % (k.CW * k.NWARP) == 0 && resident_smem(s, k) <= lim) order.push_back(k);
     if (const char* env = std::getenv("SDM_RESIDENT_CFG")) {
-      int C = 0, L = 0;
-      if (std::sscanf(env, "%d,%d", &C, &L) == 2) order.insert(order.begin(), {C, L});
-    }
-    for (const auto& cl : order) {
-      const int C = cl.first, L = cl.second;
-      if (s.d_v % C != 0 || (L != 16 && L != 8 && L != 4) || (C != 16 && C != 32)) continue;
-      if (resident_smem(s, C, L) <= lim) {
-        c.resident = true;
-        c.C = C;
-        c.L = L;
-        c.smem = resident_smem(s, C, L);
-        break;
+      int CW = 0, NW = 0, L = 0;
+      if (std::sscanf(env, "%d,%d,%d", &CW, &NW, &L) == 3) {
+        std::vector<ResidentCfg> forced;
+        for (const ResidentCfg& k : order)
+          if (k.CW == CW && k.NWARP == NW && k.L == L) forced.push_back(k);
+        if (!forced.empty()) order = forced;
       }
+    }
+    if (!order.empty()) {
+      const ResidentCfg& k = order.front();
+      c.resident = true;
+      c.CW = k.CW;
+      c.NWARP = k.NWARP;
+      c.EB = k.EB;
+      c.C = k.CW * k.NWARP;
+      c.L = k.L;
+      c.smem = resident_smem(s, k);
     }
     if (c.resident) {
       *out = c;
@@ -366,7 +387,7 @@ template <typename Tin>
 sdm_status_t launch_records(const sdm_shape_t& s, const int32_t* idx_w, const float* w_w, const int32_t* idx_r,
                             const float* w_r, const void* alpha, const void* beta, int P, uint32_t* rec,
                             unsigned* err, const DeviceInfo& dev, cudaStream_t st) {
-  const sdm::RecLayout rl = rec_layout(s.W, s.R);
+  const sdm::RecLayout rl = rec_layout(s.W, s.R, P > 0);
   int log2_cells = 1;
   while ((1 << log2_cells) < 2 * s.W) ++log2_cells;
   const size_t smem =
@@ -386,15 +407,11 @@ sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cuda
   const dim3 grid(a.B * a.H, a.d_v / c.C);
   void (*kern)(sdm::ScanArgs) = nullptr;
   if (c.resident) {
-    if (c.C == 32) {
-      if (c.L == 16) kern = sdm::k_scan_resident<Tin, Tst, 32, 16>;
-      else if (c.L == 8) kern = sdm::k_scan_resident<Tin, Tst, 32, 8>;
-      else kern = sdm::k_scan_resident<Tin, Tst, 32, 4>;
-    } else {
-      if (c.L == 16) kern = sdm::k_scan_resident<Tin, Tst, 16, 16>;
-      else if (c.L == 8) kern = sdm::k_scan_resident<Tin, Tst, 16, 8>;
-      else kern = sdm::k_scan_resident<Tin, Tst, 16, 4>;
-    }
+#define SDM_RES(CW_, NW_, L_, EB_) \
+    if (c.CW == CW_ && c.NWARP == NW_ && c.L == L_ && c.EB == EB_) kern = sdm::k_scan_resident<Tin, Tst, CW_, NW_, L_, EB_>;
+    SDM_RES(8, 2, 4, 4) SDM_RES(8, 1, 4, 4) SDM_RES(16, 1, 4, 4) SDM_RES(4, 4, 4, 2) SDM_RES(4, 2, 4, 2)
+    SDM_RES(8, 2, 8, 4) SDM_RES(4, 4, 8, 2) SDM_RES(8, 4, 8, 4)
+#undef SDM_RES
   } else {
 #define SDM_STREAM(C_, P_, L_) \
     if (c.C == C_ && c.P == P_ && c.L == L_) kern = sdm::k_scan_streaming<Tin, Tst, C_, P_, L_>;
@@ -409,7 +426,7 @@ sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cuda
   }
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no streaming kernel for the chosen tile");
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
-  kern<<<grid, sdm::kScanThreads, c.smem, st>>>(a);
+  kern<<<grid, c.resident ? c.NWARP * 32 : sdm::kScanThreads, c.smem, st>>>(a);
   return launch_status("scan launch");
 }
 
@@ -472,7 +489,7 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
   a.B = s.B; a.T = s.T; a.H = s.H;
   a.N = static_cast<int>(slots_of(s.sqrt_n));
   a.d_v = s.d_v; a.W = s.W; a.R = s.R;
-  a.rl = rec_layout(s.W, s.R);
+  a.rl = rec_layout(s.W, s.R, !c.resident);
   a.rec = rec;
   a.v = v;
   a.M_in = M_in;

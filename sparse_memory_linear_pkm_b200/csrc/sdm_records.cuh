@@ -5,7 +5,7 @@
 //   int32 slot_w[Wp] | f32 k_w[Wp] | int32 slot_r[Rp] | f32 q_r[Rp] |
 //   int16 fwd[Fp]    | f32 alpha, beta, 0, 0
 // (Wp, Rp rounded up to 4 entries, Fp = W+R rounded up to 8, so a record is a
-// multiple of 16 bytes). Records are laid out [B, H, T] so a run of tokens of
+// multiple of 16 bytes; Fp = 0 when the consumer needs no hazard plan). Records are laid out [B, H, T] so a run of tokens of
 // one (b, h) is one contiguous bulk copy.
 //
 // fwd[e] is the hazard plan of the streaming kernel, which gathers the state
@@ -18,7 +18,7 @@
 // write slots per token in shared memory.
 //
 // Slot indices outside [0, N) are replaced by -1 (skipped by the kernels) and
-// flagged in the device error word.
+// flagged in the device error word; the padding entries also carry slot -1.
 #pragma once
 
 #include "sdm_device.cuh"
@@ -114,7 +114,20 @@ __global__ void __launch_bounds__(256) k_build_records(
       r[rl.off_slot_r + e - W] = static_cast<uint32_t>(slot);
       r[rl.off_q_r + e - W] = __float_as_uint(wt);
     }
-    reinterpret_cast<int16_t*>(r + rl.off_fwd)[e] = static_cast<int16_t>(code);
+    if (rl.Fp > 0) reinterpret_cast<int16_t*>(r + rl.off_fwd)[e] = static_cast<int16_t>(code);
+  }
+  // Padding entries (W..Wp, R..Rp) carry slot -1.
+  const int npad = (rl.Wp - W) + (rl.Rp - R);
+  for (int x = threadIdx.x; x < (t_end - t0) * npad; x += blockDim.x) {
+    const int t = t0 + x / npad, e = x % npad;
+    uint32_t* r = rec + (static_cast<int64_t>(bh) * T + t) * rl.words;
+    if (e < rl.Wp - W) {
+      r[rl.off_slot_w + W + e] = 0xFFFFFFFFu;
+      r[rl.off_k_w + W + e] = 0u;
+    } else {
+      r[rl.off_slot_r + R + e - (rl.Wp - W)] = 0xFFFFFFFFu;
+      r[rl.off_q_r + R + e - (rl.Wp - W)] = 0u;
+    }
   }
   for (int t = t0 + static_cast<int>(threadIdx.x); t < t_end; t += blockDim.x) {
     const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;

@@ -13,15 +13,16 @@
 // segment of the tile is U 16-byte units; lane q%U of a warp handles unit q
 // of one entry and a warp instruction covers 32/U entries, so each entry's
 // metadata is read once per U lanes and v_t stays in registers for the whole
-// token. The W writes of a token touch distinct slots and run in parallel; a
-// barrier separates them from the R reads, whose partial sums are reduced in a
-// fixed order (bit-reproducible y). Per-token records and v rows are staged a
+// token. The W writes of a token touch distinct slots and run in parallel; the
+// R reads follow them, and their partial sums are reduced in a fixed order
+// (bit-reproducible y). Per-token records and v rows are staged a
 // chunk of L tokens at a time by 1-D bulk copies (no multicast) into a double
 // buffer tracked by mbarriers with bounded waits.
 //
 //   k_scan_resident  : the (b, h) column tile of the state lives in shared
 //                      memory (fp32) for the whole sequence; M_in is read once
-//                      and M_out written once. Two barriers per token.
+//                      and M_out written once. Each warp carries its own
+//                      column tile through the tokens (no barrier per token).
 //   k_scan_streaming : the state stays in global memory. The rows of token t+P
 //                      are gathered (16-byte cp.async per lane) into a
 //                      ring of P+1 load stages while token t computes; the
@@ -105,6 +106,44 @@ __device__ __forceinline__ uint4 pack16(const float* in) {
   return u;
 }
 
+// m[j] <- aw * m[j] + cw * v[j] for j < VE, two fp32 lanes per instruction.
+template <int VE>
+__device__ __forceinline__ void delta_update(float* m, const float* v, float aw, float cw) {
+  const float2 a2 = make_float2(aw, aw), c2 = make_float2(cw, cw);
+#pragma unroll
+  for (int j = 0; j < VE; j += 2) {
+    const float2 t = __fmul2_rn(c2, make_float2(v[j], v[j + 1]));
+    const float2 r = __ffma2_rn(a2, make_float2(m[j], m[j + 1]), t);
+    m[j] = r.x;
+    m[j + 1] = r.y;
+  }
+}
+// acc[j] += qw * m[j] for j < VE.
+template <int VE>
+__device__ __forceinline__ void weighted_add(float* acc, const float* m, float qw) {
+  const float2 q2 = make_float2(qw, qw);
+#pragma unroll
+  for (int j = 0; j < VE; j += 2) {
+    const float2 r = __ffma2_rn(q2, make_float2(m[j], m[j + 1]), make_float2(acc[j], acc[j + 1]));
+    acc[j] = r.x;
+    acc[j + 1] = r.y;
+  }
+}
+
+// Stores four fp32 values as four consecutive state elements (16 or 8 bytes).
+template <typename Tst>
+__device__ __forceinline__ void store_vec4(Tst* p, const float4& f) {
+  if constexpr (sizeof(Tst) == 4) {
+    *reinterpret_cast<float4*>(p) = f;
+  } else {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x, f.y), hi = __floats2bfloat162_rn(f.z, f.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+}
+
 // Issues the bulk copies of chunk c (records + v rows of up to L tokens) into
 // buffer c & 1. Called by one thread.
 template <typename Tin, int C, int L>
@@ -148,43 +187,139 @@ __device__ __forceinline__ void reduce_y_store(const float* yp, float* yrow, int
 
 // ------------------------------------------------------------ resident ----
 
-template <typename Tin, typename Tst, int C, int L>
-__global__ void __launch_bounds__(kScanThreads, 1) k_scan_resident(ScanArgs a) {
-  constexpr int U = C / 4;         // 16-byte units of an fp32 row segment
-  constexpr int G = kWarp / U;     // entries per warp instruction
-  constexpr int GS = G * kScanWarps;
+// Per-token metadata one lane group of the resident kernel needs first: its
+// first block of EB write entries and of EB read entries, alpha, beta and its
+// four columns of v.
+template <int EB>
+struct ResidentMeta {
+  int ws[EB], rs[EB];
+  float wk[EB], rq[EB];
+  float alpha, beta;
+  float v[4];
+};
+
+// EB consecutive 32-bit words (EB = 2 or 4, 8- or 16-byte aligned).
+template <int EB>
+__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* out) {
+  if constexpr (EB == 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    out[0] = u.x; out[1] = u.y; out[2] = u.z; out[3] = u.w;
+  } else {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    out[0] = u.x; out[1] = u.y;
+  }
+}
+
+// Block g of the write and of the read entries of one staged record; a lane
+// group without a block gets empty entries (slot -1, coefficient 0).
+template <typename Tin, int EB>
+__device__ __forceinline__ void load_meta(ResidentMeta<EB>& m, const RecLayout& rl, const uint32_t* rec,
+                                          const Tin* vrow, int g, int W, int R) {
+  if (g * EB < W) {
+    load_words<EB>(rec + rl.off_slot_w + g * EB, reinterpret_cast<uint32_t*>(m.ws));
+    load_words<EB>(rec + rl.off_k_w + g * EB, reinterpret_cast<uint32_t*>(m.wk));
+  } else {
+#pragma unroll
+    for (int j = 0; j < EB; ++j) { m.ws[j] = -1; m.wk[j] = 0.f; }
+  }
+  if (g * EB < R) {
+    load_words<EB>(rec + rl.off_slot_r + g * EB, reinterpret_cast<uint32_t*>(m.rs));
+    load_words<EB>(rec + rl.off_q_r + g * EB, reinterpret_cast<uint32_t*>(m.rq));
+  } else {
+#pragma unroll
+    for (int j = 0; j < EB; ++j) { m.rs[j] = -1; m.rq[j] = 0.f; }
+  }
+  const float2 ab = *reinterpret_cast<const float2*>(rec + rl.off_ab);
+  m.alpha = ab.x;
+  m.beta = ab.y;
+  load_in_vec<Tin, 4>(vrow, m.v);
+}
+
+__device__ __forceinline__ void load_row4(const float4* p, float* m) {
+  const float4 r = *p;
+  m[0] = r.x; m[1] = r.y; m[2] = r.z; m[3] = r.w;
+}
+template <typename Tst>
+__device__ __forceinline__ void store_row4(float4* p, const float* m) {
+  *p = make_float4(round_to<Tst>(m[0]), round_to<Tst>(m[1]), round_to<Tst>(m[2]), round_to<Tst>(m[3]));
+}
+
+// Sums acc[0:4) (four columns of unit q = lane % U) over the 32 / U entry
+// groups of the warp and stores the four column sums at y[0:4) of unit q.
+// Reduce-scatter over the two highest lane bits (each lane keeps half, then a
+// quarter of its values), plain butterfly over the lower group bits; the
+// order is fixed, so y does not depend on timing.
+template <int U>
+__device__ __forceinline__ void reduce_store_y(const float* acc, float* y, int lane) {
+  static_assert(U <= 8, "at least four entry groups");
+  const bool hi = lane & 16, hi2 = lane & 8;
+  float k0 = hi ? acc[2] : acc[0], k1 = hi ? acc[3] : acc[1];
+  const float s0 = hi ? acc[0] : acc[2], s1 = hi ? acc[1] : acc[3];
+  k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+  float k = hi2 ? k1 : k0;
+  k += __shfl_xor_sync(0xffffffffu, hi2 ? k0 : k1, 8);
+#pragma unroll
+  for (int o = 4; o >= U; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+  if ((lane & (7 & ~(U - 1))) == 0) y[(hi ? 2 : 0) + (hi2 ? 1 : 0)] = k;
+}
+
+// Shared-memory bytes of k_scan_resident (host and device agree on this).
+__host__ __device__ constexpr size_t resident_smem_bytes(int N, int CW, int NWARP, int L, int words, int s_in) {
+  return static_cast<size_t>(NWARP) * (N + 2) * CW * 4 + static_cast<size_t>(2) * L * words * 4 +
+         static_cast<size_t>(2) * L * CW * NWARP * s_in + 2 * 8;
+}
+
+// Each warp owns a CW-column tile of one (b, h) and carries it through all T
+// tokens on its own: lane q % U holds four fp32 columns (one 16-byte unit) of
+// the entry block g = lane / U, so one warp instruction covers G = 32 / U
+// entries. The tile never leaves the warp, so tokens need no block barrier;
+// the only block barriers are the two per staged chunk of L tokens. The read
+// sum of a token is reduced over the G entry groups with a fixed butterfly,
+// so y does not depend on timing.
+template <typename Tin, typename Tst, int CW, int NWARP, int L, int EB>
+__global__ void __launch_bounds__(NWARP * kWarp) k_scan_resident(ScanArgs a) {
+  constexpr int NT = NWARP * kWarp;
+  constexpr int C = CW * NWARP;  // columns of the CTA
+  constexpr int U = CW / 4;      // lanes per entry
+  constexpr int G = kWarp / U;   // entry blocks per warp instruction
+  static_assert(CW == 4 || CW == 8 || CW == 16 || CW == 32, "warp tile of 4..32 fp32 columns");
+  static_assert(EB == 2 || EB == 4, "entry blocks of 2 or 4");
   extern __shared__ __align__(16) unsigned char smem[];
   const int N = a.N, W = a.W, R = a.R, T = a.T;
   const int words = a.rl.words;
-  float* S = reinterpret_cast<float*>(smem);  // [N][C]
-  uint32_t* recbuf = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(N) * C * 4);
+  float* S = reinterpret_cast<float*>(smem);  // [NWARP][N + 2][CW]
+  uint32_t* recbuf = reinterpret_cast<uint32_t*>(smem + static_cast<size_t>(NWARP) * (N + 2) * CW * 4);
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);
-  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][warps][C+1]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + ((2 * kScanWarps * (C + 1) + 3) & ~3));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);
 
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int c0 = blockIdx.y * C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane / U, q = lane % U;
-  const int e0 = g + G * warp;  // first entry of this lane group
+  // Warp tile: rows 0..N-1 hold the state; row N absorbs writes of skipped
+  // entries (never read) and row N+1 stays zero for skipped reads, so the
+  // entry loops need no branches.
+  float4* Sw = reinterpret_cast<float4*>(S + static_cast<size_t>(warp) * (N + 2) * CW) + q;  // row r at Sw[r * U]
+  const int sink_w = N, zero_r = N + 1;
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     fence_mbar_init();
   }
-  {  // initial state tile
-    constexpr int VE = 16 / sizeof(Tst);
+  {  // initial state tile, four columns at a time
     const Tst* Min = static_cast<const Tst*>(a.M_in) + b * a.M_in_b_stride +
                      static_cast<int64_t>(h) * N * a.d_v + c0;
-    for (int x = tid; x < N * (C / VE); x += kScanThreads) {
-      const int row = x / (C / VE), u = x % (C / VE);
-      float f[VE];
-      unpack16<Tst>(*reinterpret_cast<const uint4*>(Min + static_cast<int64_t>(row) * a.d_v + u * VE), f);
-#pragma unroll
-      for (int i = 0; i < VE; i += 4)
-        *reinterpret_cast<float4*>(S + row * C + u * VE + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+    for (int x = tid; x < N * (C / 4); x += NT) {
+      const int row = x / (C / 4), col = (x % (C / 4)) * 4;
+      float f[4];
+      load_in_vec<Tst, 4>(Min + static_cast<int64_t>(row) * a.d_v + col, f);
+      *reinterpret_cast<float4*>(S + (static_cast<size_t>(col / CW) * (N + 2) + row) * CW + col % CW) =
+          make_float4(f[0], f[1], f[2], f[3]);
     }
+    for (int x = tid; x < NWARP * 2 * CW; x += NT)
+      S[(static_cast<size_t>(x / (2 * CW)) * (N + 2) + N) * CW + x % (2 * CW)] = 0.f;
   }
   __syncthreads();
   const int n_chunks = (T + L - 1) / L;
@@ -192,76 +327,117 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_resident(ScanArgs a) {
     issue_chunk<Tin, C, L>(a, bh, b, h, c0, 0, recbuf, vbuf, bars);
     if (n_chunks > 1) issue_chunk<Tin, C, L>(a, bh, b, h, c0, 1, recbuf, vbuf, bars);
   }
-  float* y_bh = a.y + static_cast<int64_t>(h) * a.d_v + c0;
+  if (n_chunks > 0) {
+    // Software pipeline over tokens: the metadata of token t+1 is loaded
+    // while token t computes, and the y reduction of token t-1 overlaps the
+    // row loads of token t. Two tokens per iteration, so the metadata
+    // registers alternate without copies.
+    const int vcol = warp * CW + 4 * q;  // this lane's first column within the CTA tile
+    const int64_t y_step = static_cast<int64_t>(a.H) * a.d_v;
+    float* y_t = a.y + static_cast<int64_t>(b) * T * y_step + static_cast<int64_t>(h) * a.d_v + c0 + vcol;
+    auto rec_of = [&](int t) { return recbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * words; };
+    auto vrow_of = [&](int t) { return vbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * C + vcol; };
+    auto chunk_ok = [&](int cc) {
+      const bool ok = mbar_wait_bounded(&bars[cc & 1], (cc >> 1) & 1, a.err);
+      return !__syncthreads_or(!ok);
+    };
+    if (!chunk_ok(0)) return;
+    ResidentMeta<EB> ma, mb;
+    load_meta<Tin, EB>(ma, a.rl, rec_of(0), vrow_of(0), g, W, R);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    bool failed = false;
 
-  for (int c = 0; c < n_chunks; ++c) {
-    const int bi = c & 1;
-    const bool ok = mbar_wait_bounded(&bars[bi], (c >> 1) & 1, a.err);
-    if (__syncthreads_or(!ok)) return;
-    const uint32_t* recs = recbuf + static_cast<size_t>(bi) * L * words;
-    const Tin* vs = vbuf + static_cast<size_t>(bi) * L * C;
-    const int nt = min(L, T - c * L);
+    // One token: returns false when a staging wait gave up.
+    auto step = [&](int t, const ResidentMeta<EB>& cur, ResidentMeta<EB>& nxt) -> bool {
+      // 1. row loads of the first write block
+      int wrow[EB];
+      float m[EB][4];
+#pragma unroll
+      for (int j = 0; j < EB; ++j) {
+        wrow[j] = cur.ws[j] < 0 ? sink_w : cur.ws[j];
+        load_row4(Sw + wrow[j] * U, m[j]);
+      }
+      // 2. y of token t-1 (independent of the loads in flight)
+      if (t > 0) reduce_store_y<U>(acc, y_t - y_step, lane);
+      // 3. metadata of token t+1
+      if (t + 1 < T) {
+        if ((t + 1) % L == 0 && !chunk_ok((t + 1) / L)) return false;
+        load_meta<Tin, EB>(nxt, a.rl, rec_of(t + 1), vrow_of(t + 1), g, W, R);
+      }
+      // 4. write: the W slots of a token are distinct, so a block is loaded
+      // before any of it is stored; blocks past the first (W > EB * G) are
+      // loaded here.
+#pragma unroll
+      for (int j = 0; j < EB; ++j) {
+        const float cw = cur.beta * cur.wk[j];
+        delta_update<4>(m[j], cur.v, cur.alpha * (1.0f - cw), cw);
+        store_row4<Tst>(Sw + wrow[j] * U, m[j]);
+      }
+      for (int jb = g + G; jb * EB < W; jb += G) {
+        const uint32_t* rec = rec_of(t);
+        int sl[EB];
+        float kk[EB];
+        load_words<EB>(rec + a.rl.off_slot_w + jb * EB, reinterpret_cast<uint32_t*>(sl));
+        load_words<EB>(rec + a.rl.off_k_w + jb * EB, reinterpret_cast<uint32_t*>(kk));
+#pragma unroll
+        for (int j = 0; j < EB; ++j) {
+          sl[j] = sl[j] < 0 ? sink_w : sl[j];
+          load_row4(Sw + sl[j] * U, m[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < EB; ++j) {
+          const float cw = cur.beta * kk[j];
+          delta_update<4>(m[j], cur.v, cur.alpha * (1.0f - cw), cw);
+          store_row4<Tst>(Sw + sl[j] * U, m[j]);
+        }
+      }
+      __syncwarp();  // rows written by one lane group are read by another
+      // 5. read after the write
+#pragma unroll
+      for (int j = 0; j < EB; ++j) load_row4(Sw + (cur.rs[j] < 0 ? zero_r : cur.rs[j]) * U, m[j]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] = 0.f;
+#pragma unroll
+      for (int j = 0; j < EB; ++j) weighted_add<4>(acc, m[j], cur.rq[j]);
+      for (int jb = g + G; jb * EB < R; jb += G) {
+        const uint32_t* rec = rec_of(t);
+        int sl[EB];
+        float qq[EB];
+        load_words<EB>(rec + a.rl.off_slot_r + jb * EB, reinterpret_cast<uint32_t*>(sl));
+        load_words<EB>(rec + a.rl.off_q_r + jb * EB, reinterpret_cast<uint32_t*>(qq));
+#pragma unroll
+        for (int j = 0; j < EB; ++j) load_row4(Sw + (sl[j] < 0 ? zero_r : sl[j]) * U, m[j]);
+#pragma unroll
+        for (int j = 0; j < EB; ++j) weighted_add<4>(acc, m[j], qq[j]);
+      }
+      __syncwarp();  // this token's reads precede the next token's writes
+      // 6. at the end of a chunk every warp is past its buffer: refill it
+      if (t % L == L - 1) {
+        __syncthreads();
+        if (tid == 0 && t / L + 2 < n_chunks) {
+          fence_proxy_async_smem();
+          issue_chunk<Tin, C, L>(a, bh, b, h, c0, t / L + 2, recbuf, vbuf, bars);
+        }
+      }
+      y_t += y_step;
+      return true;
+    };
+
 #pragma unroll 1
-    for (int i = 0; i < nt; ++i) {
-      const int t = c * L + i;
-      const uint32_t* rec = recs + i * words;
-      const float alpha = __uint_as_float(rec[a.rl.off_ab]);
-      const float beta = __uint_as_float(rec[a.rl.off_ab + 1]);
-      float vv[4];
-      load_in_vec<Tin, 4>(vs + i * C + 4 * q, vv);
-      // Write: W distinct slots.
-      for (int e = e0; e < W; e += GS) {
-        const int slot = static_cast<int>(rec[a.rl.off_slot_w + e]);
-        if (slot < 0) continue;
-        const float cw = beta * __uint_as_float(rec[a.rl.off_k_w + e]);
-        const float aw = alpha * (1.0f - cw);
-        float4* p = reinterpret_cast<float4*>(S + slot * C + 4 * q);
-        float4 m = *p;
-        m.x = round_to<Tst>(fmaf(aw, m.x, cw * vv[0]));
-        m.y = round_to<Tst>(fmaf(aw, m.y, cw * vv[1]));
-        m.z = round_to<Tst>(fmaf(aw, m.z, cw * vv[2]));
-        m.w = round_to<Tst>(fmaf(aw, m.w, cw * vv[3]));
-        *p = m;
-      }
-      __syncthreads();
-      // Read after the write.
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int r = e0; r < R; r += GS) {
-        const int slot = static_cast<int>(rec[a.rl.off_slot_r + r]);
-        if (slot < 0) continue;
-        const float qw = __uint_as_float(rec[a.rl.off_q_r + r]);
-        const float4 m = *reinterpret_cast<const float4*>(S + slot * C + 4 * q);
-        acc[0] = fmaf(qw, m.x, acc[0]);
-        acc[1] = fmaf(qw, m.y, acc[1]);
-        acc[2] = fmaf(qw, m.z, acc[2]);
-        acc[3] = fmaf(qw, m.w, acc[3]);
-      }
-#pragma unroll
-      for (int o = U; o < kWarp; o <<= 1)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-      float* yp = ypart + (t & 1) * kScanWarps * (C + 1);
-      if (lane < U) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) yp[warp * (C + 1) + 4 * q + j] = acc[j];
-      }
-      __syncthreads();
-      reduce_y_store<C>(yp, y_bh + (static_cast<int64_t>(b) * T + t) * a.H * a.d_v, warp, lane);
+    for (int t = 0; t < T; t += 2) {
+      if (!step(t, ma, mb)) { failed = true; break; }
+      if (t + 1 < T && !step(t + 1, mb, ma)) { failed = true; break; }
     }
-    // Every thread is past the last read of buffer bi (barrier above).
-    if (tid == 0 && c + 2 < n_chunks) {
-      fence_proxy_async_smem();
-      issue_chunk<Tin, C, L>(a, bh, b, h, c0, c + 2, recbuf, vbuf, bars);
-    }
+    if (failed) return;
+    reduce_store_y<U>(acc, y_t - y_step, lane);
   }
   __syncthreads();
   {
-    constexpr int VE = 16 / sizeof(Tst);
     Tst* Mout = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * N * a.d_v + c0;
-    for (int x = tid; x < N * (C / VE); x += kScanThreads) {
-      const int row = x / (C / VE), u = x % (C / VE);
-      *reinterpret_cast<uint4*>(Mout + static_cast<int64_t>(row) * a.d_v + u * VE) =
-          pack16<Tst>(S + row * C + u * VE);
+    for (int x = tid; x < N * (C / 4); x += NT) {
+      const int row = x / (C / 4), col = (x % (C / 4)) * 4;
+      store_vec4<Tst>(Mout + static_cast<int64_t>(row) * a.d_v + col,
+                      *reinterpret_cast<const float4*>(S + (static_cast<size_t>(col / CW) * (N + 2) + row) * CW + col % CW));
     }
   }
 }
