@@ -1,0 +1,47 @@
+"""Runs the layer (selection, recurrence, optional epilogue) on one seeded
+synthetic workload, a few times, on cuda:0 — the unit a profiler captures.
+
+    python -m sparse_memory_linear_pkm_b200.case d2048_h16_n1024_dv128 B=2 [T=... H=...] [--repeat 2]
+        [--variant auto|resident|streaming] [--epilogue]
+
+Size overrides (B, T, H) shrink a named workload while keeping its slot
+count, row width, entry counts and dtypes.
+"""
+
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import layer_forward, synth
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("workload", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("sizes", nargs="*", help="overrides such as B=2 T=1024 H=4")
+    ap.add_argument("--repeat", type=int, default=2)
+    ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming"])
+    ap.add_argument("--epilogue", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    args = ap.parse_args(argv)
+    kw = {}
+    for item in args.sizes:
+        key, val = item.split("=")
+        if key not in ("B", "T", "H"):
+            raise SystemExit(f"unknown size override {key!r} (B, T or H)")
+        kw[key] = int(val)
+    shape = synth.WORKLOADS[args.workload].replace(**kw)
+    inp = synth.make_inputs(shape, seed=args.seed, device="cuda", with_gate=args.epilogue)
+    y = torch.empty((shape.B, shape.T, shape.H, shape.d_v), dtype=torch.float32, device="cuda")
+    M = torch.empty((shape.B,) + tuple(inp["M0"].shape), dtype=inp["M0"].dtype, device="cuda")
+    for _ in range(args.repeat):
+        layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], inp["M0"], shape.W, shape.R,
+                      g=inp.get("g"), variant=args.variant, y=y, M_out=M)
+    torch.cuda.synchronize()
+    print("ok", shape, "variant", args.variant)
+
+
+if __name__ == "__main__":
+    main()
