@@ -264,14 +264,17 @@ size_t records_bytes(const sdm_shape_t& s) {
   return align256(static_cast<size_t>(s.B) * s.H * s.T * rec_layout(s.W, s.R).words * 4u);
 }
 
-// Instantiated streaming tiles: columns per CTA, prefetch distance, staging chunk.
+// Instantiated streaming tiles: state bytes, columns per CTA, prefetch
+// distance, staging chunk, warps.
 struct StreamCfg {
   int state_bytes;
-  int C, P, L;
+  int C, P, L, NW;
 };
 constexpr StreamCfg kStreamCfgs[] = {
-    {4, 64, 3, 8}, {4, 64, 2, 8}, {4, 32, 6, 8}, {4, 32, 4, 8}, {4, 16, 8, 16}, {4, 16, 4, 8},
-    {2, 128, 3, 8}, {2, 64, 6, 8}, {2, 64, 4, 8}, {2, 32, 12, 16}, {2, 32, 8, 16}, {2, 16, 8, 16}, {2, 16, 4, 8},
+    {4, 64, 3, 8, 16}, {4, 64, 2, 8, 16}, {4, 32, 4, 8, 16}, {4, 32, 4, 8, 8}, {4, 16, 8, 16, 16},
+    {4, 16, 4, 8, 8},
+    {2, 128, 3, 8, 16}, {2, 64, 4, 8, 16}, {2, 64, 6, 8, 16}, {2, 32, 8, 16, 16}, {2, 32, 8, 16, 8},
+    {2, 16, 8, 16, 16}, {2, 16, 4, 8, 8},
 };
 
 // Instantiated resident tiles: columns per warp, warps per CTA, staging
@@ -292,16 +295,14 @@ struct ScanChoice {
   size_t smem = 0;
 };
 
-size_t ypart_bytes(int C) { return static_cast<size_t>((2 * sdm::kScanWarps * (C + 1) + 3) & ~3) * 4; }
-
 size_t resident_smem(const sdm_shape_t& s, const ResidentCfg& k) {
   return sdm::resident_smem_bytes(static_cast<int>(slots_of(s.sqrt_n)), k.CW, k.NWARP, k.L,
                                   rec_layout(s.W, s.R, false).words, static_cast<int>(in_size(s.in_dtype)));
 }
-size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L) {
+size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L, int NW) {
   const sdm::RecLayout rl = rec_layout(s.W, s.R);
   return sdm::streaming_stage_bytes(P, s.W + s.R, s.W, C, static_cast<int>(in_size(s.state_dtype))) +
-         2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) + ypart_bytes(C) + 2 * 8;
+         2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) + 2ull * NW * C * 4 + 2 * 8;
 }
 
 sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
@@ -360,21 +361,23 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
     if (rx != ry) return rx > ry;  // wider row segments first
     return x.P > y.P;
   });
-  if (const char* env = std::getenv("SDM_STREAM_CFG")) {  // tuning override "C,P,L"
-    int C = 0, P = 0, L = 0;
-    if (std::sscanf(env, "%d,%d,%d", &C, &P, &L) == 3) {
+  if (const char* env = std::getenv("SDM_STREAM_CFG")) {  // tuning override "C,P,L,NW"
+    int C = 0, P = 0, L = 0, NW = 0;
+    if (std::sscanf(env, "%d,%d,%d,%d", &C, &P, &L, &NW) == 4) {
       std::vector<StreamCfg> forced;
       for (const StreamCfg& k : order)
-        if (k.C == C && k.P == P && k.L == L) forced.push_back(k);
+        if (k.C == C && k.P == P && k.L == L && k.NW == NW) forced.push_back(k);
       if (!forced.empty()) order = forced;
     }
   }
   for (const StreamCfg& k : order) {
-    const size_t need = streaming_smem(s, k.C, k.P, k.L);
+    if (k.C > 32 * k.NW) continue;
+    const size_t need = streaming_smem(s, k.C, k.P, k.L, k.NW);
     if (need <= lim) {
       c.C = k.C;
       c.P = k.P;
       c.L = k.L;
+      c.NWARP = k.NW;
       c.smem = need;
       *out = c;
       return SDM_OK;
@@ -413,20 +416,20 @@ sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cuda
     SDM_RES(8, 2, 8, 4) SDM_RES(4, 4, 8, 2) SDM_RES(8, 4, 8, 4)
 #undef SDM_RES
   } else {
-#define SDM_STREAM(C_, P_, L_) \
-    if (c.C == C_ && c.P == P_ && c.L == L_) kern = sdm::k_scan_streaming<Tin, Tst, C_, P_, L_>;
+#define SDM_STREAM(C_, P_, L_, NW_) \
+    if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWARP == NW_) kern = sdm::k_scan_streaming<Tin, Tst, C_, P_, L_, NW_>;
     if constexpr (sizeof(Tst) == 4) {
-      SDM_STREAM(64, 3, 8) SDM_STREAM(64, 2, 8) SDM_STREAM(32, 6, 8) SDM_STREAM(32, 4, 8)
-      SDM_STREAM(16, 8, 16) SDM_STREAM(16, 4, 8)
+      SDM_STREAM(64, 3, 8, 16) SDM_STREAM(64, 2, 8, 16) SDM_STREAM(32, 4, 8, 16) SDM_STREAM(32, 4, 8, 8)
+      SDM_STREAM(16, 8, 16, 16) SDM_STREAM(16, 4, 8, 8)
     } else {
-      SDM_STREAM(128, 3, 8) SDM_STREAM(64, 6, 8) SDM_STREAM(64, 4, 8) SDM_STREAM(32, 12, 16)
-      SDM_STREAM(32, 8, 16) SDM_STREAM(16, 8, 16) SDM_STREAM(16, 4, 8)
+      SDM_STREAM(128, 3, 8, 16) SDM_STREAM(64, 4, 8, 16) SDM_STREAM(64, 6, 8, 16) SDM_STREAM(32, 8, 16, 16)
+      SDM_STREAM(32, 8, 16, 8) SDM_STREAM(16, 8, 16, 16) SDM_STREAM(16, 4, 8, 8)
     }
 #undef SDM_STREAM
   }
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no streaming kernel for the chosen tile");
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
-  kern<<<grid, c.resident ? c.NWARP * 32 : sdm::kScanThreads, c.smem, st>>>(a);
+  kern<<<grid, c.NWARP * 32, c.smem, st>>>(a);
   return launch_status("scan launch");
 }
 
@@ -477,9 +480,10 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
                       uint32_t* rec, cudaStream_t st, const Trace& tr = Trace(), bool init_before_scan = false,
                       const void* M0_for_init = nullptr) {
   sdm_status_t r;
-  if ((r = (s.in_dtype == SDM_BF16 ? launch_records<bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, c.resident ? 0 : c.P,
+  const int plan_p = c.resident ? 0 : c.P + 1;  // the streaming plan looks back P tokens
+  if ((r = (s.in_dtype == SDM_BF16 ? launch_records<bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, plan_p,
                                                           rec, dev.err, dev, st)
-                                   : launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, c.resident ? 0 : c.P,
+                                   : launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, plan_p,
                                                            rec, dev.err, dev, st))) != SDM_OK)
     return r;
   tr.mark(2, st);

@@ -36,8 +36,6 @@
 
 namespace sdm {
 
-constexpr int kScanThreads = 512;
-constexpr int kScanWarps = kScanThreads / kWarp;
 
 struct ScanArgs {
   int B, T, H, N, d_v, W, R;
@@ -161,27 +159,6 @@ __device__ __forceinline__ void issue_chunk(const ScanArgs& a, int bh, int b, in
   for (int i = 0; i < nt; ++i) {
     const Tin* src = v + ((static_cast<int64_t>(b) * a.T + t0 + i) * a.H + h) * a.d_v + c0;
     bulk_g2s(vbuf + (static_cast<size_t>(bi) * L + i) * C, src, v_bytes, &bars[bi]);
-  }
-}
-
-// y of one token from the per-warp partials ypart[w][0:C) (row stride C+1):
-// warp v sums columns [v*C/NW, (v+1)*C/NW), 16 lanes per column.
-template <int C>
-__device__ __forceinline__ void reduce_y_store(const float* yp, float* yrow, int warp, int lane) {
-  constexpr int CPW = C / kScanWarps;  // columns per warp
-  static_assert(C % kScanWarps == 0 && kScanWarps == 16, "16 warps, C a multiple of 16");
-  const int part = lane & 15;
-#pragma unroll
-  for (int cc = 0; cc < (CPW + 1) / 2; ++cc) {
-    const int sub = cc * 2 + (lane >> 4);
-    const bool valid = sub < CPW;
-    const int col = warp * CPW + (valid ? sub : 0);
-    float s = valid ? yp[part * (C + 1) + col] : 0.f;
-    s += __shfl_xor_sync(0xffffffffu, s, 8);
-    s += __shfl_xor_sync(0xffffffffu, s, 4);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    if (valid && part == 0) yrow[col] = s;
   }
 }
 
@@ -444,22 +421,70 @@ __global__ void __launch_bounds__(NWARP * kWarp) k_scan_resident(ScanArgs a) {
 
 // ----------------------------------------------------------- streaming ----
 
-// Shared-memory bytes of k_scan_streaming (host and device agree on this).
-__host__ __device__ constexpr size_t streaming_stage_bytes(int P, int E, int W, int C, int s_state) {
-  return (static_cast<size_t>(P + 1) * E + static_cast<size_t>(P) * W) * C * s_state;
+// Sums a[0:VE) (the VE columns of one 16-byte unit, held by the U lanes of
+// every entry group) over the 32 / U entry groups of the warp and stores the
+// column sums at y[0:VE): reduce-scatter while a lane still holds more than
+// one value, butterfly after that; the order is fixed, so y does not depend
+// on timing.
+template <int VE, int U>
+__device__ __forceinline__ void reduce_store_unit(float (&a)[VE], float* y, int lane) {
+  int n = VE, off = 0, bmask = 0;
+#pragma unroll
+  for (int o = 16; o >= U; o >>= 1) {
+    if (n > 1) {
+      const bool hi = lane & o;
+      const int h = n / 2;
+#pragma unroll
+      for (int j = 0; j < VE / 2; ++j) {
+        if (j < h) {
+          const float keep = hi ? a[j + h] : a[j];
+          const float send = hi ? a[j] : a[j + h];
+          a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      off += hi ? h : 0;
+      n = h;
+    } else {
+      a[0] += __shfl_xor_sync(0xffffffffu, a[0], o);
+      bmask |= o;
+    }
+  }
+  if ((lane & bmask) == 0) {
+#pragma unroll
+    for (int j = 0; j < VE; ++j)
+      if (j < n) y[off + j] = a[j];
+  }
 }
 
-template <typename Tin, typename Tst, int C, int P, int L>
-__global__ void __launch_bounds__(kScanThreads, 1) k_scan_streaming(ScanArgs a) {
+// Shared-memory bytes of the stage rings of k_scan_streaming.
+__host__ __device__ constexpr size_t streaming_stage_bytes(int P, int E, int W, int C, int s_state) {
+  return (static_cast<size_t>(P + 1) * E + static_cast<size_t>(P + 1) * W) * C * s_state;
+}
+
+// The state stays in global memory. A CTA of NW warps owns one (b, h) and C
+// columns. The rows of token t+P are gathered (one 16-byte cp.async per lane
+// and unit) into a ring of P+1 load stages right after token t's barrier, so
+// the copies overlap token t's compute; the hazard plan forwards rows that
+// tokens t+P-1 .. t write from a ring of P+1 written-row stages. A read of a
+// slot written by the same token recomputes that write from its source row
+// (plan code k = 0), so the writes and reads of a token have no dependency
+// between warps: one block barrier per token orders token t's rows before
+// token t+1 and before the gathers that token t+1 issues. Written rows go
+// straight back to global memory. Warp partial sums of y are reduced in a
+// fixed order one token later.
+template <typename Tin, typename Tst, int C, int P, int L, int NW>
+__global__ void __launch_bounds__(NW * kWarp, 1) k_scan_streaming(ScanArgs a) {
+  constexpr int NT = NW * kWarp;
   constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
   constexpr int U = C / VE;             // units per row segment
   constexpr int G = kWarp / U;          // entries per warp instruction
-  constexpr int GS = G * kScanWarps;
-  constexpr int SL = P + 1;             // load stages: current token + P in flight
-  constexpr int SW = P;                 // written-row stages: current token + P-1 before it
+  constexpr int GS = G * NW;            // entries per block instruction
+  constexpr int SL = P + 1;             // load stages
+  constexpr int SW = P + 1;             // written-row stages
   constexpr uint32_t RS = C * sizeof(Tst);
   static_assert(L > P, "a chunk must be staged before its tokens are gathered");
   static_assert(kWarp % U == 0, "a row segment spans a divisor of the warp");
+  static_assert(C <= NT, "one thread per column sums y");
   extern __shared__ __align__(16) unsigned char smem[];
   const int W = a.W, R = a.R, T = a.T, E = W + R;
   const int words = a.rl.words;
@@ -467,16 +492,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_streaming(ScanArgs a) 
   unsigned char* wstage = smem + static_cast<size_t>(SL) * E * RS;  // [SW][W][RS]
   uint32_t* recbuf = reinterpret_cast<uint32_t*>(smem + streaming_stage_bytes(P, E, W, C, sizeof(Tst)));
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);
-  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][warps][C+1]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + ((2 * kScanWarps * (C + 1) + 3) & ~3));
+  float* ypart = reinterpret_cast<float*>(vbuf + 2 * L * C);  // [2][NW][C]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + 2 * NW * C);
 
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int c0 = blockIdx.y * C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane / U, q = lane % U;
   const int e0 = g + G * warp;
-  Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * a.N * a.d_v + c0;
-  float* y_bh = a.y + static_cast<int64_t>(h) * a.d_v + c0;
+  Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * a.N * a.d_v + c0 + q * VE;
+  const int64_t y_step = static_cast<int64_t>(a.H) * a.d_v;
+  float* y_bh = a.y + static_cast<int64_t>(b) * T * y_step + static_cast<int64_t>(h) * a.d_v + c0;
 
   auto rec_of = [&](int t) -> const uint32_t* {
     return recbuf + (static_cast<size_t>((t / L) & 1) * L + (t % L)) * words;
@@ -484,19 +510,27 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_streaming(ScanArgs a) 
   auto fwd_of = [&](const uint32_t* rec, int e) -> int {
     return reinterpret_cast<const int16_t*>(rec + a.rl.off_fwd)[e];
   };
+  // Row unit of entry e of token t: gathered, or forwarded from an earlier
+  // token's written row (code (k << 9) | j, k >= 1).
+  auto source = [&](int t, const uint32_t* rec, int e) -> const unsigned char* {
+    const int f = fwd_of(rec, e);
+    if (f < 0) return lstage + (static_cast<size_t>(t % SL) * E + e) * RS + q * 16;
+    return wstage + (static_cast<size_t>((t - (f >> 9)) % SW) * W + (f & 511)) * RS + q * 16;
+  };
   // Gathers the rows of token t that the plan does not forward: one 16-byte
-  // cp.async per (entry, unit), one commit group per call. (One bulk copy per
-  // row issued by a single warp measured ~3x slower: issue-bound.)
+  // cp.async per (entry, unit), one commit group per call.
   auto gather = [&](int t) {
     const uint32_t* rec = rec_of(t);
-    const int st = t % SL;
+    unsigned char* ls = lstage + static_cast<size_t>(t % SL) * E * RS + q * 16;
     for (int e = e0; e < E; e += GS) {
       const int slot = static_cast<int>(e < W ? rec[a.rl.off_slot_w + e] : rec[a.rl.off_slot_r + e - W]);
-      if (slot >= 0 && fwd_of(rec, e) < 0)
-        cp_async16(lstage + (static_cast<size_t>(st) * E + e) * RS + q * 16,
-                   Mbh + static_cast<int64_t>(slot) * a.d_v + q * VE);
+      if (slot >= 0 && fwd_of(rec, e) < 0) cp_async16(ls + e * RS, Mbh + static_cast<int64_t>(slot) * a.d_v);
     }
     cp_async_commit();
+  };
+  auto chunk_ok = [&](int cc) {
+    const bool ok = mbar_wait_bounded(&bars[cc & 1], (cc >> 1) & 1, a.err);
+    return !__syncthreads_or(!ok);
   };
 
   if (tid == 0) {
@@ -511,113 +545,87 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_scan_streaming(ScanArgs a) 
     issue_chunk<Tin, C, L>(a, bh, b, h, c0, 0, recbuf, vbuf, bars);
     if (n_chunks > 1) issue_chunk<Tin, C, L>(a, bh, b, h, c0, 1, recbuf, vbuf, bars);
   }
-  {
-    const bool ok = mbar_wait_bounded(&bars[0], 0, a.err);
-    if (__syncthreads_or(!ok)) return;
-  }
+  if (!chunk_ok(0)) return;
   for (int t = 0; t < P; ++t) {
     if (t < T) gather(t);
     else cp_async_commit();
   }
 
-  int sl = 0, sw = 0;  // t % SL, t % SW
 #pragma unroll 1
   for (int t = 0; t < T; ++t) {
     cp_async_wait<P - 1>();
-    __syncthreads();  // rows of t landed and visible; reads of t-1 done
+    __syncthreads();  // token t's rows landed; token t-1's rows written and visible
     if (t > 0 && t % L == 0 && tid == 0 && t / L + 1 < n_chunks) {
       fence_proxy_async_smem();
       issue_chunk<Tin, C, L>(a, bh, b, h, c0, t / L + 1, recbuf, vbuf, bars);
     }
-    if (t > 0) {
-      const float* yp = ypart + ((t - 1) & 1) * kScanWarps * (C + 1);
-      reduce_y_store<C>(yp, y_bh + (static_cast<int64_t>(b) * T + (t - 1)) * a.H * a.d_v, warp, lane);
+    if (t > 0 && tid < C) {  // y of token t-1: fixed-order sum of the warp partials
+      const float* yp = ypart + ((t - 1) & 1) * NW * C + tid;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) sum += yp[w * C];
+      y_bh[(t - 1) * y_step + tid] = sum;
     }
-    const uint32_t* rec = rec_of(t);
-    const Tin* vrow = vbuf + (static_cast<size_t>((t / L) & 1) * L + (t % L)) * C;
-    const float alpha = __uint_as_float(rec[a.rl.off_ab]);
-    const float beta = __uint_as_float(rec[a.rl.off_ab + 1]);
-    float vv[VE];
-    load_in_vec<Tin, VE>(vrow + q * VE, vv);
-    unsigned char* lrow = lstage + static_cast<size_t>(sl) * E * RS;
-    unsigned char* wrow = wstage + static_cast<size_t>(sw) * W * RS;
-    // Write.
-    for (int e = e0; e < W; e += GS) {
-      const int slot = static_cast<int>(rec[a.rl.off_slot_w + e]);
-      if (slot < 0) continue;
-      const int f = fwd_of(rec, e);
-      const unsigned char* src;
-      if (f < 0) {
-        src = lrow + e * RS;
-      } else {
-        int ws = sw - (f >> 9);
-        ws += ws < 0 ? SW : 0;
-        src = wstage + (static_cast<size_t>(ws) * W + (f & 511)) * RS;
-      }
-      float m[VE];
-      unpack16<Tst>(*reinterpret_cast<const uint4*>(src + q * 16), m);
-      const float cw = beta * __uint_as_float(rec[a.rl.off_k_w + e]);
-      const float aw = alpha * (1.0f - cw);
-#pragma unroll
-      for (int j = 0; j < VE; ++j) m[j] = fmaf(aw, m[j], cw * vv[j]);
-      const uint4 packed = pack16<Tst>(m);
-      *reinterpret_cast<uint4*>(wrow + e * RS + q * 16) = packed;
-      *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slot) * a.d_v + q * VE) = packed;
-    }
-    __syncthreads();  // writes of t visible to the reads of t and to later gathers
-    // Read after the write.
-    float acc[VE];
-#pragma unroll
-    for (int j = 0; j < VE; ++j) acc[j] = 0.f;
-    for (int r = e0; r < R; r += GS) {
-      const int slot = static_cast<int>(rec[a.rl.off_slot_r + r]);
-      if (slot < 0) continue;
-      const int f = fwd_of(rec, W + r);
-      const unsigned char* src;
-      if (f < 0) {
-        src = lrow + (W + r) * RS;
-      } else {
-        int ws = sw - (f >> 9);
-        ws += ws < 0 ? SW : 0;
-        src = wstage + (static_cast<size_t>(ws) * W + (f & 511)) * RS;
-      }
-      float m[VE];
-      unpack16<Tst>(*reinterpret_cast<const uint4*>(src + q * 16), m);
-      const float qw = __uint_as_float(rec[a.rl.off_q_r + r]);
-#pragma unroll
-      for (int j = 0; j < VE; ++j) acc[j] = fmaf(qw, m[j], acc[j]);
-    }
-#pragma unroll
-    for (int o = U; o < kWarp; o <<= 1)
-#pragma unroll
-      for (int j = 0; j < VE; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-    if (lane < U) {
-      float* yp = ypart + (t & 1) * kScanWarps * (C + 1) + warp * (C + 1) + q * VE;
-#pragma unroll
-      for (int j = 0; j < VE; ++j) yp[j] = acc[j];
-    }
-    // Gather token t + P into the load stage token t - 1 used (free now).
+    // Gather token t+P into the load stage token t-1 used (free after the barrier).
     if (t + P < T) {
-      if ((t + P) % L == 0) {
-        const int c = (t + P) / L;
-        const bool okc = mbar_wait_bounded(&bars[c & 1], (c >> 1) & 1, a.err);
-        if (__syncthreads_or(!okc)) {
-          cp_async_wait<0>();
-          return;
-        }
+      if ((t + P) % L == 0 && !chunk_ok((t + P) / L)) {
+        cp_async_wait<0>();
+        return;
       }
       gather(t + P);
     } else {
       cp_async_commit();
     }
-    sl = sl + 1 == SL ? 0 : sl + 1;
-    sw = sw + 1 == SW ? 0 : sw + 1;
+    const uint32_t* rec = rec_of(t);
+    const float2 ab = *reinterpret_cast<const float2*>(rec + a.rl.off_ab);
+    float vv[VE];
+    load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((t / L) & 1) * L + (t % L)) * C + q * VE, vv);
+    unsigned char* wrow = wstage + static_cast<size_t>(t % SW) * W * RS + q * 16;
+    // Entries e < W are writes, the rest reads; with reads of this token's
+    // written slots recomputed from the write's source row, the two kinds are
+    // independent, so every lane group takes the same share of either.
+    float acc[VE];
+#pragma unroll
+    for (int j = 0; j < VE; ++j) acc[j] = 0.f;
+    for (int e = e0; e < E; e += GS) {
+      if (e < W) {
+        const int slot = static_cast<int>(rec[a.rl.off_slot_w + e]);
+        if (slot < 0) continue;
+        float m[VE];
+        unpack16<Tst>(*reinterpret_cast<const uint4*>(source(t, rec, e)), m);
+        const float cw = ab.y * __uint_as_float(rec[a.rl.off_k_w + e]);
+        delta_update<VE>(m, vv, ab.x * (1.0f - cw), cw);
+        const uint4 packed = pack16<Tst>(m);
+        *reinterpret_cast<uint4*>(wrow + e * RS) = packed;
+        *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slot) * a.d_v) = packed;
+      } else {
+        const int r = e - W;
+        const int slot = static_cast<int>(rec[a.rl.off_slot_r + r]);
+        if (slot < 0) continue;
+        const int f = fwd_of(rec, e);
+        float m[VE];
+        if (f >= 0 && (f >> 9) == 0) {  // written by this token: recompute that write
+          const int j = f & 511;
+          unpack16<Tst>(*reinterpret_cast<const uint4*>(source(t, rec, j)), m);
+          const float cw = ab.y * __uint_as_float(rec[a.rl.off_k_w + j]);
+          delta_update<VE>(m, vv, ab.x * (1.0f - cw), cw);
+          unpack16<Tst>(pack16<Tst>(m), m);  // the stored (rounded) value
+        } else {
+          unpack16<Tst>(*reinterpret_cast<const uint4*>(source(t, rec, e)), m);
+        }
+        weighted_add<VE>(acc, m, __uint_as_float(rec[a.rl.off_q_r + r]));
+      }
+    }
+    reduce_store_unit<VE, U>(acc, ypart + (t & 1) * NW * C + warp * C + q * VE, lane);
   }
   cp_async_wait<0>();
   __syncthreads();
-  if (T > 0) {
-    const float* yp = ypart + ((T - 1) & 1) * kScanWarps * (C + 1);
-    reduce_y_store<C>(yp, y_bh + (static_cast<int64_t>(b) * T + (T - 1)) * a.H * a.d_v, warp, lane);
+  if (T > 0 && tid < C) {
+    const float* yp = ypart + ((T - 1) & 1) * NW * C + tid;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) sum += yp[w * C];
+    y_bh[(T - 1) * y_step + tid] = sum;
   }
 }
 
