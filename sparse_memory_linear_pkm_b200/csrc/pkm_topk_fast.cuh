@@ -39,44 +39,80 @@ __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
 }
 
 // Descending bitonic sort of 32*E 64-bit keys, each carrying a 32-bit payload;
-// position p = lane*E + s.
+// position p = lane*E + s. For E <= 2 the stage loops stay rolled (one copy
+// of the compare-exchange body instead of one per stage keeps the kernel
+// small enough for the instruction caches); wider sorts are unrolled.
 template <int E, bool PAYLOAD>
 __device__ __forceinline__ void warp_bitonic_desc(uint64_t (&k)[E], uint32_t (&pl)[E]) {
   const int lane = lane_id();
   constexpr int SZ = kWarp * E;
+  if constexpr (E <= 2) {
+#pragma unroll 1
+    for (int kk = 2; kk <= SZ; kk <<= 1) {
+#pragma unroll 1
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        if (E == 2 && j == 1) {  // partners in the same lane: positions 2*lane and 2*lane+1
+          const bool desc = ((lane * E) & kk) == 0;
+          const uint64_t a = k[0], b = k[E - 1];
+          const bool swap = desc ? (a < b) : (a > b);
+          k[0] = swap ? b : a;
+          k[E - 1] = swap ? a : b;
+          if (PAYLOAD) {
+            const uint32_t pa = pl[0], pb = pl[E - 1];
+            pl[0] = swap ? pb : pa;
+            pl[E - 1] = swap ? pa : pb;
+          }
+        } else {
 #pragma unroll
-  for (int kk = 2; kk <= SZ; kk <<= 1) {
-#pragma unroll
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      if (j < E) {
-#pragma unroll
-        for (int s = 0; s < E; ++s) {
-          const int t = s ^ j;
-          if (t > s) {
-            const bool desc = ((lane * E + s) & kk) == 0;
-            const uint64_t a = k[s], b = k[t];
-            const bool swap = desc ? (a < b) : (a > b);
-            k[s] = swap ? b : a;
-            k[t] = swap ? a : b;
+          for (int s = 0; s < E; ++s) {
+            const int p = lane * E + s;
+            const uint64_t other = shfl_xor_u64(k[s], j / E);
+            const bool keep_max = ((p & j) == 0) == ((p & kk) == 0);
+            const bool take_other = keep_max ? (other > k[s]) : (other < k[s]);
             if (PAYLOAD) {
-              const uint32_t pa = pl[s], pb = pl[t];
-              pl[s] = swap ? pb : pa;
-              pl[t] = swap ? pa : pb;
+              const uint32_t opl = __shfl_xor_sync(0xffffffffu, pl[s], j / E);
+              pl[s] = take_other ? opl : pl[s];
             }
+            k[s] = take_other ? other : k[s];
           }
         }
-      } else {
+      }
+    }
+  } else {
 #pragma unroll
-        for (int s = 0; s < E; ++s) {
-          const int p = lane * E + s;
-          const uint64_t other = shfl_xor_u64(k[s], j / E);
-          const bool keep_max = ((p & j) == 0) == ((p & kk) == 0);
-          const bool take_other = keep_max ? (other > k[s]) : (other < k[s]);
-          if (PAYLOAD) {
-            const uint32_t opl = __shfl_xor_sync(0xffffffffu, pl[s], j / E);
-            pl[s] = take_other ? opl : pl[s];
+    for (int kk = 2; kk <= SZ; kk <<= 1) {
+#pragma unroll
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        if (j < E) {
+#pragma unroll
+          for (int s = 0; s < E; ++s) {
+            const int t = s ^ j;
+            if (t > s) {
+              const bool desc = ((lane * E + s) & kk) == 0;
+              const uint64_t a = k[s], b = k[t];
+              const bool swap = desc ? (a < b) : (a > b);
+              k[s] = swap ? b : a;
+              k[t] = swap ? a : b;
+              if (PAYLOAD) {
+                const uint32_t pa = pl[s], pb = pl[t];
+                pl[s] = swap ? pb : pa;
+                pl[t] = swap ? pa : pb;
+              }
+            }
           }
-          k[s] = take_other ? other : k[s];
+        } else {
+#pragma unroll
+          for (int s = 0; s < E; ++s) {
+            const int p = lane * E + s;
+            const uint64_t other = shfl_xor_u64(k[s], j / E);
+            const bool keep_max = ((p & j) == 0) == ((p & kk) == 0);
+            const bool take_other = keep_max ? (other > k[s]) : (other < k[s]);
+            if (PAYLOAD) {
+              const uint32_t opl = __shfl_xor_sync(0xffffffffu, pl[s], j / E);
+              pl[s] = take_other ? opl : pl[s];
+            }
+            k[s] = take_other ? other : k[s];
+          }
         }
       }
     }
