@@ -442,16 +442,47 @@ __global__ void __launch_bounds__(kFastTopkWarps * kWarp) k_pkm_topk_fast(const 
       cnt += __popc(bt);
     }
     __syncwarp();
+    // Order the K winners by ord(hi):(~slot), descending: each winner's rank is
+    // the number of winner keys above it (keys are distinct: the slot is part
+    // of the key), counted against all K keys read two at a time from shared
+    // memory; then every winner moves to its rank.
     uint64_t k[E];
     uint32_t kl[E];
+    {
+      uint64_t mine[E];
+      uint32_t mlo[E];
+      int rank[E];
 #pragma unroll
-    for (int s = 0; s < E; ++s) {
-      const int p = lane * E + s;
-      k[s] = p < K ? sel[p] : 0ull;
-      kl[s] = p < K ? hist[p] : 0u;
+      for (int s = 0; s < E; ++s) {
+        const int p = lane * E + s;
+        mine[s] = p < K ? sel[p] : 0ull;
+        mlo[s] = p < K ? hist[p] : 0u;
+        rank[s] = 0;
+      }
+      const ulonglong2* sel2 = reinterpret_cast<const ulonglong2*>(sel);
+      for (int j = 0; j < K; j += 2) {
+        const ulonglong2 two = sel2[j >> 1];
+        const uint64_t second = j + 1 < K ? two.y : 0ull;  // past K: stale, never above a winner
+#pragma unroll
+        for (int s = 0; s < E; ++s) rank[s] += (two.x > mine[s]) + (second > mine[s]);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int s = 0; s < E; ++s) {
+        if (lane * E + s < K) {
+          sel[rank[s]] = mine[s];
+          hist[rank[s]] = mlo[s];
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int s = 0; s < E; ++s) {
+        const int p = lane * E + s;
+        k[s] = p < K ? sel[p] : 0ull;
+        kl[s] = p < K ? hist[p] : 0u;
+      }
+      __syncwarp();
     }
-    __syncwarp();
-    warp_bitonic_desc<E, true>(k, kl);
     // Neighbours with equal hi but different lo need the (lo desc, slot asc) order.
     bool fix = false;
     {
