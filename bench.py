@@ -16,6 +16,7 @@ ranks. `--impl reference` times the CPU oracle on a bounded sample instead
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -58,6 +59,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
+    ap.add_argument("--decode", action="store_true",
+                    help="time decode steps instead: one token per call (sdm_layer_step), state carried")
     return ap.parse_args()
 
 
@@ -419,11 +422,71 @@ def d2h_mib(y: torch.Tensor) -> float:
     return y.numel() * y.element_size() / 2 ** 20
 
 
+def run_decode(args, dist: Dist):
+    """Decode: every step is one sdm_layer_step call on one token per batch row
+    (B rows, H heads of the workload), the state carried in place; reports the
+    device time per step and the tokens per second it implies."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --decode needs a CUDA device")
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    base = synth.WORKLOADS[args.workload]
+    n_tok = args.warmup + args.steps
+    shape = base.replace(T=n_tok)
+    sdm.native.load()
+    inp = synth.make_inputs(shape, seed=args.seed + dist.rank, device=dev)
+    per_step = [{k: inp[k][:, t:t + 1].contiguous() for k in ("kp", "qp", "v", "alpha", "beta")} for t in range(n_tok)]
+    M = inp["M0"].unsqueeze(0).repeat(shape.B, 1, 1, 1).contiguous()
+    y = torch.empty((shape.B, 1, shape.H, shape.d_v), dtype=torch.float32, device=dev)
+    sh = sdm.make_shape(shape.B, 1, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
+                        shape.torch_state())
+    ws = torch.empty(max(16, int(sdm.native.load().sdm_layer_step_workspace_bytes(ctypes.byref(sh)))),
+                     dtype=torch.uint8, device=dev)
+
+    def step(t):
+        d = per_step[t]
+        sdm.layer_step(d["kp"], d["qp"], d["v"], d["alpha"], d["beta"], M, shape.W, shape.R, y=y, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    for t in range(args.warmup):
+        step(t)
+    sdm.stream_check(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for t in range(args.warmup, n_tok):
+            step(t)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    sdm.stream_check(dev)
+    ms = dist.max(start.elapsed_time(end), dev)
+    us_per_step = ms * 1e3 / args.steps
+    if dist.rank == 0:
+        cfg = workload_config(shape, args, dist)
+        cfg.update({"T": 1, "mode": "decode: one token per batch row per sdm_layer_step call, state carried",
+                    "variant": sdm.scan_variant(sh)})
+        line = {"metric": "SDM decode step latency (one token per batch row, state carried) on 1 B200",
+                "value": us_per_step, "unit": "us", "n_gpus": dist.world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": us_per_step / 1e3, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+                "tokens_per_s": aggregate_value(shape.B * args.steps, dist.world, ms / 1e3),
+                "gpu_launches": 4 * args.steps, "clocks": clocks.summary()}
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
 def main():
     args = parse_args()
     dist = Dist()
     if args.impl == "reference":
         run_reference(args, dist)
+        return
+    if args.decode:
+        run_decode(args, dist)
         return
     run_sdm(args, dist)
 

@@ -16,8 +16,9 @@
  *
  * Conventions for every entry point:
  *   - Pointers named as tensors are caller-owned DEVICE pointers to contiguous
- *     row-major arrays, 16-byte aligned. The library allocates no memory;
- *     scratch space is passed in by the caller ("workspace").
+ *     row-major arrays, 16-byte aligned (alpha and beta: aligned to their
+ *     element size). The library allocates no memory; scratch space is passed
+ *     in by the caller ("workspace").
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream). Calls only enqueue work and return; results are ready when the
  *     stream reaches them.
@@ -163,6 +164,23 @@ SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp,
                                const void* v, const void* alpha, const void* beta, const void* g,
                                const void* M0, void* M_out, float* y, void* workspace,
                                size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace sdm_layer_step needs for this shape (0 for invalid shapes). */
+SDM_API size_t sdm_layer_step_workspace_bytes(const sdm_shape_t* shape);
+
+/* One call of the layer core that carries the state across calls (the
+ * decode / streaming use: T = 1 or a few tokens per call): selection on k'
+ * (top-W) and q' (top-R), the recurrence starting from the state in M, and the
+ * optional epilogue ([explainer] 3.1 steps 1-3). M [B,H,N,d_v] state_dtype is
+ * read as the state before the first token and overwritten with the state
+ * after the last, so consecutive calls over consecutive token ranges continue
+ * one sequence (start from M[b] = M0 with sdm_state_init). Other arguments as
+ * in sdm_layer_forward; workspace: at least sdm_layer_step_workspace_bytes(shape).
+ * With the automatic variant, calls with T*(W+R) < N stream only the selected
+ * rows (a resident tile would move the whole state). */
+SDM_API sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, const void* qp,
+                            const void* v, const void* alpha, const void* beta, const void* g,
+                            void* M, float* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* sdm_layer_forward that also records caller-created CUDA events (cudaEvent_t
  * passed as void*) on `stream` between its stages, for timing each kernel in

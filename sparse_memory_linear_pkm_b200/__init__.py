@@ -20,7 +20,7 @@ import torch
 from . import native, synth
 from .native import SdmError
 
-__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "stream_check", "make_shape",
+__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "stream_check", "make_shape",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
 _DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
@@ -116,6 +116,24 @@ def state_init(M0: torch.Tensor, B: int, out: torch.Tensor | None = None) -> tor
     shape = native.Shape(B, 1, H, sqrt_n, 1, 1, d_v, native.F32, _code(M0, "M0"), 1e-6, 0)
     native.check(native.load().sdm_state_init(ctypes.byref(shape), _ptr(M0), _ptr(M), _stream(M0.device)))
     return M
+
+
+def layer_step(kp, qp, v, alpha, beta, M, W: int, R: int, g=None, eps: float = 1e-6, variant: str = "auto",
+               y: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Selection and recurrence over T tokens continuing from the state in M
+    [B,H,N,d_v], which is updated in place (decode: T = 1 per call). Returns y."""
+    B, T, H, two_n = kp.shape
+    d_v = v.shape[-1]
+    shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M, "M"), eps,
+                         native.VARIANTS[variant])
+    lib = native.load()
+    if y is None:
+        y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=kp.device)
+    ws = _workspace(int(lib.sdm_layer_step_workspace_bytes(ctypes.byref(shape))), kp.device, workspace)
+    native.check(lib.sdm_layer_step(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha), _ptr(beta),
+                                    _ptr(g), _ptr(M), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                                    _stream(kp.device)))
+    return y
 
 
 def layer_forward(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float = 1e-6,

@@ -122,6 +122,16 @@ sdm_status_t need_ptr(const void* p, const char* name, bool nonempty) {
 
 size_t in_size(int32_t d) { return d == SDM_BF16 ? 2 : 4; }
 
+// The per-token gates are read one element at a time: natural alignment
+// suffices (a one-token slice of [B, T, H] is rarely 16-byte aligned).
+sdm_status_t need_gate(const void* p, const char* name, bool nonempty, int32_t dtype) {
+  if (!nonempty) return SDM_OK;
+  if (p == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, std::string(name) + " is NULL");
+  if (reinterpret_cast<uintptr_t>(p) % in_size(dtype) != 0)
+    return fail(SDM_ERR_INVALID_ARGUMENT, std::string(name) + " is not aligned to its element size");
+  return SDM_OK;
+}
+
 // ------------------------------------------------------------- selection --
 
 sdm::TopkLayout topk_layout(int n, int K) {
@@ -308,7 +318,11 @@ size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L, int NW) {
 sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
   const size_t lim = static_cast<size_t>(dev.max_smem_optin);
   ScanChoice c;
-  if (s.variant != SDM_VARIANT_STREAMING) {
+  // A resident tile reads and writes all N rows once; below one touched row
+  // per slot (T * (W + R) < N, e.g. a decode step) streaming only the
+  // selected rows moves less.
+  const bool few_tokens = static_cast<int64_t>(s.T) * (s.W + s.R) < slots_of(s.sqrt_n);
+  if (s.variant == SDM_VARIANT_RESIDENT || (s.variant == SDM_VARIANT_AUTO && !few_tokens)) {
     // Resident tiles in order of preference (measured on B200 at N = 1024,
     // d_v = 128: 8-column warp tiles, one warp per CTA, so up to five CTAs
     // share an SM); the first that divides d_v and fits is taken.
@@ -597,8 +611,8 @@ sdm_status_t sdm_scan(const sdm_shape_t* shape, const int32_t* idx_w, const floa
   const sdm_shape_t& s = *shape;
   const bool any = static_cast<int64_t>(s.B) * s.T * s.H > 0;
   if ((r = need_ptr(idx_w, "idx_w", any)) || (r = need_ptr(w_w, "w_w", any)) || (r = need_ptr(idx_r, "idx_r", any)) ||
-      (r = need_ptr(w_r, "w_r", any)) || (r = need_ptr(v, "v", any)) || (r = need_ptr(alpha, "alpha", any)) ||
-      (r = need_ptr(beta, "beta", any)) || (r = need_ptr(M, "M", any)) || (r = need_ptr(y, "y", any)))
+      (r = need_ptr(w_r, "w_r", any)) || (r = need_ptr(v, "v", any)) || (r = need_gate(alpha, "alpha", any, s.in_dtype)) ||
+      (r = need_gate(beta, "beta", any, s.in_dtype)) || (r = need_ptr(M, "M", any)) || (r = need_ptr(y, "y", any)))
     return r;
   if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
   if (!any) return ok();
@@ -657,7 +671,7 @@ sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const void* kp, 
   const bool any = th > 0;
   const bool any_state = static_cast<int64_t>(s.B) * s.H > 0;
   if ((r = need_ptr(kp, "kp", any)) || (r = need_ptr(qp, "qp", any)) || (r = need_ptr(v, "v", any)) ||
-      (r = need_ptr(alpha, "alpha", any)) || (r = need_ptr(beta, "beta", any)) || (r = need_ptr(y, "y", any)) ||
+      (r = need_gate(alpha, "alpha", any, s.in_dtype)) || (r = need_gate(beta, "beta", any, s.in_dtype)) || (r = need_ptr(y, "y", any)) ||
       (r = need_ptr(M0, "M0", any_state)) || (r = need_ptr(M_out, "M_out", any_state)))
     return r;
   if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
@@ -702,6 +716,49 @@ sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const v
                                float* y, void* workspace, size_t workspace_bytes, void* stream) {
   return sdm_layer_forward_traced(shape, kp, qp, v, alpha, beta, g, M0, M_out, y, workspace, workspace_bytes,
                                   stream, nullptr, 0);
+}
+
+size_t sdm_layer_step_workspace_bytes(const sdm_shape_t* shape) { return sdm_layer_forward_workspace_bytes(shape); }
+
+sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                            const void* alpha, const void* beta, const void* g, void* M, float* y, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  const int64_t th = static_cast<int64_t>(s.B) * s.T * s.H;
+  const bool any = th > 0;
+  if ((r = need_ptr(kp, "kp", any)) || (r = need_ptr(qp, "qp", any)) || (r = need_ptr(v, "v", any)) ||
+      (r = need_gate(alpha, "alpha", any, s.in_dtype)) || (r = need_gate(beta, "beta", any, s.in_dtype)) || (r = need_ptr(y, "y", any)) ||
+      (r = need_ptr(M, "M", any)))
+    return r;
+  if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
+  if (!any) return ok();
+  const size_t need = sdm_layer_step_workspace_bytes(shape);
+  if (workspace_bytes < need)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "workspace_bytes below sdm_layer_step_workspace_bytes() = " + std::to_string(need));
+  if ((r = need_ptr(workspace, "workspace", true)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ScanChoice c;
+  if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(ws);
+  ws += align256(th * s.W * 4);
+  float* w_w = reinterpret_cast<float*>(ws);
+  ws += align256(th * s.W * 4);
+  int32_t* idx_r = reinterpret_cast<int32_t*>(ws);
+  ws += align256(th * s.R * 4);
+  float* w_r = reinterpret_cast<float*>(ws);
+  ws += align256(th * s.R * 4);
+  uint32_t* rec = reinterpret_cast<uint32_t*>(ws);
+  if ((r = topk_impl(*dev, kp, s.in_dtype, th, s.sqrt_n, s.W, idx_w, w_w, st)) != SDM_OK) return r;
+  if ((r = topk_impl(*dev, qp, s.in_dtype, th, s.sqrt_n, s.R, idx_r, w_r, st)) != SDM_OK) return r;
+  const int64_t row_stride = static_cast<int64_t>(s.H) * slots_of(s.sqrt_n) * s.d_v;
+  if ((r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M, row_stride, M, y, rec, st)) != SDM_OK)
+    return r;
+  return ok();
 }
 
 sdm_status_t sdm_layer_forward_noalloc(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,

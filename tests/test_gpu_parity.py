@@ -172,6 +172,38 @@ def _layer_case(sdm, oracle, dev, shape, seed, with_gate=False, variant="auto"):
         assert np.array_equal(M_T_host[b, h, untouched], M0[h, untouched])
 
 
+@pytest.mark.parametrize("name,steps", [("tiny_n1024_dv16", (1,) * 9), ("d2048_h16_n1024_dv128", (1, 1, 3, 1, 7)),
+                                        ("d2048_h4_n16384_dv512", (1,) * 6), ("long_t1m_n262144_dv2048", (1, 2, 1))])
+def test_layer_step_chain(sdm, oracle, cuda_device, name, steps):
+    """Decode-style calls carrying the state (T = 1 or a few tokens each) equal
+    the whole-sequence layer and the oracle."""
+    T = sum(steps)
+    shape = synth.WORKLOADS[name].replace(B=2, T=T, H=2)
+    if name == "long_t1m_n262144_dv2048":
+        shape = shape.replace(B=1)
+    inp = synth.make_inputs(shape, seed=23, device="cpu")
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    y_ref, M_ref = sdm.layer_forward(d["kp"], d["qp"], d["v"], d["alpha"], d["beta"], d["M0"], shape.W, shape.R)
+    M = d["M0"].unsqueeze(0).repeat(shape.B, 1, 1, 1).contiguous()
+    ys, t0 = [], 0
+    for n in steps:
+        sl = lambda x: x[:, t0:t0 + n].contiguous()
+        ys.append(sdm.layer_step(sl(d["kp"]), sl(d["qp"]), sl(d["v"]), sl(d["alpha"]), sl(d["beta"]), M,
+                                 shape.W, shape.R))
+        t0 += n
+    sdm.stream_check()
+    y = torch.cat(ys, dim=1)
+    tol = tol_for(shape.state_dtype)
+    assert_rel_close(y.cpu().numpy(), y_ref.cpu().numpy(), tol, "y (steps vs whole sequence)")
+    assert_rel_close(f32(M), f32(M_ref), tol, "M_T (steps vs whole sequence)")
+    idx_w, w_w = oracle.pkm_topk(f32(inp["kp"]), shape.W)
+    idx_r, w_r = oracle.pkm_topk(f32(inp["qp"]), shape.R)
+    M0 = f32(inp["M0"])
+    oy, _ = oracle_on_compact_state(oracle, idx_w, w_w, idx_r, w_r, f32(inp["v"]), f32(inp["alpha"]),
+                                    f32(inp["beta"]), lambda b, h, s: M0[h, s], shape.state_dtype == "bf16")
+    assert_rel_close(y.cpu().numpy(), oy, tol, "y (steps vs oracle)")
+
+
 def test_layer_forward_tiny_workload_full(sdm, oracle, cuda_device):
     _layer_case(sdm, oracle, cuda_device, synth.WORKLOADS["tiny_n1024_dv16"], seed=0)
 
