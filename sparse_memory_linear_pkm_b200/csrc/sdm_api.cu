@@ -79,6 +79,28 @@ sdm_status_t launch_status(const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Raises a kernel's dynamic shared-memory limit when a launch needs more than
+// was set before on this device (one driver call per kernel and size instead
+// of one per launch; keeps small, latency-bound calls cheap on the host).
+std::mutex g_attr_mu;
+std::vector<std::pair<std::pair<int, const void*>, size_t>> g_attr;
+void set_smem(const void* kern, size_t smem) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (auto& e : g_attr) {
+    if (e.first.first == dev && e.first.second == kern) {
+      if (smem > e.second) {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e.second = smem;
+      }
+      return;
+    }
+  }
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  g_attr.push_back({{dev, kern}, smem});
+}
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 int64_t slots_of(int32_t sqrt_n) { return static_cast<int64_t>(sqrt_n) * sqrt_n; }
@@ -171,7 +193,7 @@ sdm_status_t launch_topk_fast_inst(const DeviceInfo& dev, const Tin* scores, int
                                    const sdm::FastTopkLayout& L, int32_t* idx, float* w, cudaStream_t st) {
   auto kern = sdm::k_pkm_topk_fast<Tin, E, EH, EPL, CP>;
   const size_t smem = L.table_bytes + static_cast<size_t>(sdm::kFastTopkWarps) * L.warp_bytes;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  set_smem(reinterpret_cast<const void*>(kern), smem);
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sdm::kFastTopkWarps * 32, smem);
   const int64_t blocks_needed = (units + sdm::kFastTopkWarps - 1) / sdm::kFastTopkWarps;
@@ -239,7 +261,7 @@ sdm_status_t launch_topk(const DeviceInfo& dev, const void* scores, int64_t unit
   const size_t smem = L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes;
   if (smem > static_cast<size_t>(dev.max_smem_optin)) return fail(SDM_ERR_UNSUPPORTED, "selection scratch exceeds shared memory");
   auto kern = sdm::k_pkm_topk_general<Tin>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  set_smem(reinterpret_cast<const void*>(kern), smem);
   const int64_t blocks_needed = (units + warps - 1) / warps;
   const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, static_cast<int64_t>(dev.sms) * 16));
   kern<<<grid, warps * 32, smem, st>>>(static_cast<const Tin*>(scores), units, L, idx, w);
@@ -411,7 +433,7 @@ sdm_status_t launch_records(const sdm_shape_t& s, const int32_t* idx_w, const fl
       P > 0 ? static_cast<size_t>(sdm::kRecTokensPerBlock + P - 1) * (size_t{1} << log2_cells) * 4 : 0;
   if (smem > static_cast<size_t>(dev.max_smem_optin)) return fail(SDM_ERR_UNSUPPORTED, "hazard tables exceed shared memory");
   auto kern = sdm::k_build_records<Tin>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  set_smem(reinterpret_cast<const void*>(kern), smem);
   const int tblocks = (s.T + sdm::kRecTokensPerBlock - 1) / sdm::kRecTokensPerBlock;
   const dim3 grid(tblocks, s.B * s.H);
   kern<<<grid, 256, smem, st>>>(idx_w, w_w, idx_r, w_r, static_cast<const Tin*>(alpha), static_cast<const Tin*>(beta),
@@ -442,7 +464,7 @@ sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cuda
 #undef SDM_STREAM
   }
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no streaming kernel for the chosen tile");
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
+  set_smem(reinterpret_cast<const void*>(kern), c.smem);
   kern<<<grid, c.NWARP * 32, c.smem, st>>>(a);
   return launch_status("scan launch");
 }
