@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--decode", action="store_true",
                     help="time decode steps instead: one token per call (sdm_layer_step), state carried")
+    ap.add_argument("--slot-counts", action="store_true",
+                    help="time the slot utilisation histogram of the workload's write selection instead")
     return ap.parse_args()
 
 
@@ -506,6 +508,63 @@ def run_decode(args, dist: Dist):
     dist.close()
 
 
+def run_slot_counts(args, dist: Dist):
+    """Slot utilisation: each step counts, per (b, h), how often every slot is
+    among the W write slots of the workload's T tokens (sdm_slot_counts on the
+    indices sdm_pkm_topk chose). Reports selections counted per second and the
+    achieved HBM bandwidth: the index array read once plus one read and one
+    write of the [B, H, N] int32 counts."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --slot-counts needs a CUDA device")
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    shape = synth.WORKLOADS[args.workload]
+    sdm.native.load()
+    inp = synth.make_inputs(shape, seed=args.seed + dist.rank, device=dev)
+    idx, _ = sdm.pkm_topk(inp["kp"], shape.W)
+    del inp
+    counts = torch.zeros((shape.B, shape.H, shape.N), dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        sdm.slot_counts(idx, shape.N, counts)
+    sdm.stream_check(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        for a, b in ev:
+            flush.fill_(1)  # L2 flushed between steps
+            a.record(stream)
+            sdm.slot_counts(idx, shape.N, counts)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    sdm.stream_check(dev)
+    total = sum(counts.sum(dtype=torch.int64, dim=-1).flatten().tolist())
+    assert total == (args.warmup + args.steps) * shape.B * shape.T * shape.H * shape.W, "counts do not add up"
+    ms = dist.max(sum(a.elapsed_time(b) for a, b in ev), dev)
+    sel = shape.B * shape.T * shape.H * shape.W
+    algo = sel * 4 + 2 * shape.B * shape.H * shape.N * 4
+    if dist.rank == 0:
+        gbs = algo * args.steps / (ms / 1e3) / 1e9
+        peak = measured_peaks().get("hbm_gbs", FALLBACK_HBM_GBS)
+        cfg = workload_config(shape, args, dist)
+        cfg.update({"mode": "slot utilisation counts of the write selection", "l2": "flushed between steps"})
+        line = {"metric": "SDM slot utilisation counting throughput on 1 B200", "impl": "sdm",
+                "value": aggregate_value(sel * args.steps, dist.world, ms / 1e3), "unit": "selections/s",
+                "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "int32", "data": "synthetic", "config": cfg,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                             "frac": gbs / peak if peak else None, "algorithmic_bytes_per_launch": algo},
+                "gpu_launches": args.steps, "clocks": clocks.summary()}
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
 def main():
     args = parse_args()
     dist = Dist()
@@ -514,6 +573,9 @@ def main():
         return
     if args.decode:
         run_decode(args, dist)
+        return
+    if args.slot_counts:
+        run_slot_counts(args, dist)
         return
     run_sdm(args, dist)
 

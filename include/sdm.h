@@ -102,6 +102,16 @@ SDM_API const char* sdm_status_string(sdm_status_t status);
 /* Text describing the last error returned on the calling host thread ("" if none). */
 SDM_API const char* sdm_last_error(void);
 
+/* Slot utilisation of a selection: counts[b,h,i] += the number of (t,k) with
+ * idx[b,t,h,k] == i. The pages warn that learned sparse addressing can
+ * collapse onto few slots; this monitors it. The paper has no kernel for it.
+ *   idx    [B,T,H,K] int32 (e.g. the write slots of sdm_pkm_topk)
+ *   counts [B,H,N] int32, accumulated (zero it first; calls over consecutive
+ *          token ranges add up). Indices outside [0, N) are skipped and set the
+ *          device error word. */
+SDM_API sdm_status_t sdm_slot_counts(const int32_t* idx, int32_t B, int32_t T, int32_t H, int32_t K,
+                             int32_t N, int32_t* counts, void* stream);
+
 /* Product-key top-k selection ([explainer] 3.1 step 1; [summary] Core Mechanism 2).
  * For every token-head, x = scores[b,t,h,:] is split into s1 = x[0:sqrt_n] and
  * s2 = x[sqrt_n:2*sqrt_n]. Slot i = a*sqrt_n + b has score s1[a] + s2[b]. The K

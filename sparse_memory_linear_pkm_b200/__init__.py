@@ -20,7 +20,7 @@ import torch
 from . import native, synth
 from .native import SdmError
 
-__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "stream_check", "make_shape",
+__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "stream_check", "make_shape",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
 _DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
@@ -116,6 +116,17 @@ def state_init(M0: torch.Tensor, B: int, out: torch.Tensor | None = None) -> tor
     shape = native.Shape(B, 1, H, sqrt_n, 1, 1, d_v, native.F32, _code(M0, "M0"), 1e-6, 0)
     native.check(native.load().sdm_state_init(ctypes.byref(shape), _ptr(M0), _ptr(M), _stream(M0.device)))
     return M
+
+
+def slot_counts(idx: torch.Tensor, N: int, counts: torch.Tensor | None = None) -> torch.Tensor:
+    """Per-slot selection counts: counts[b,h,i] += #{(t,k): idx[b,t,h,k] == i};
+    idx [B,T,H,K] int32. Returns counts [B,H,N] int32 (accumulated into
+    `counts` when given)."""
+    B, T, H, K = idx.shape
+    if counts is None:
+        counts = torch.zeros((B, H, N), dtype=torch.int32, device=idx.device)
+    native.check(native.load().sdm_slot_counts(_ptr(idx), B, T, H, K, N, _ptr(counts), _stream(idx.device)))
+    return counts
 
 
 def layer_step(kp, qp, v, alpha, beta, M, W: int, R: int, g=None, eps: float = 1e-6, variant: str = "auto",

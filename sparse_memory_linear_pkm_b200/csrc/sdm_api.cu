@@ -609,6 +609,46 @@ sdm_status_t sdm_pkm_topk(const void* scores, int32_t in_dtype, int32_t B, int32
   return ok();
 }
 
+sdm_status_t sdm_slot_counts(const int32_t* idx, int32_t B, int32_t T, int32_t H, int32_t K, int32_t N,
+                             int32_t* counts, void* stream) {
+  sdm_status_t r;
+  if (B < 0 || T < 0 || H < 0) return fail(SDM_ERR_INVALID_ARGUMENT, "B, T and H must be >= 0");
+  if (K < 1 || N < 1) return fail(SDM_ERR_INVALID_ARGUMENT, "K and N must be >= 1");
+  if (static_cast<int64_t>(B) * H > 65535) return fail(SDM_ERR_UNSUPPORTED, "B*H above 65535");
+  const int64_t entries = static_cast<int64_t>(B) * T * H * K;
+  if ((r = need_ptr(idx, "idx", entries > 0)) != SDM_OK) return r;
+  if ((r = need_ptr(counts, "counts", static_cast<int64_t>(B) * H > 0)) != SDM_OK) return r;
+  if (entries == 0) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const bool local = N <= sdm::kCountSmemSlots;
+  const bool vec = K % 4 == 0 && reinterpret_cast<uintptr_t>(idx) % 16 == 0;
+  const size_t smem = local ? static_cast<size_t>(N) * 4 : 0;
+  const void* kern = local ? (vec ? reinterpret_cast<const void*>(sdm::k_slot_counts<true, true>)
+                                  : reinterpret_cast<const void*>(sdm::k_slot_counts<true, false>))
+                           : (vec ? reinterpret_cast<const void*>(sdm::k_slot_counts<false, true>)
+                                  : reinterpret_cast<const void*>(sdm::k_slot_counts<false, false>));
+  set_smem(kern, smem);
+  // About two waves of resident CTAs over all (b, h); at least 64 tokens a
+  // CTA so that the shared-memory bins are worth their zeroing and flush.
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  const int64_t want = 2LL * dev->sms * per_sm;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  const int64_t split = std::max<int64_t>(1, std::min<int64_t>((want + bh - 1) / bh, (T + 63) / 64));
+  const int tokens_per_cta = static_cast<int>((T + split - 1) / split);
+  const dim3 grid((T + tokens_per_cta - 1) / tokens_per_cta, static_cast<unsigned>(bh));
+  void* args[] = {const_cast<int32_t**>(&idx), &T, &H, &K, &N, const_cast<int*>(&tokens_per_cta), &counts,
+                  &dev->err};
+  if (cudaLaunchKernel(kern, grid, dim3(256), args, smem, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(SDM_ERR_CUDA, std::string("slot count launch: ") + cudaGetErrorString(cudaGetLastError()));
+  if ((r = launch_status("slot count launch")) != SDM_OK) return r;
+  return ok();
+}
+
 size_t sdm_scan_workspace_bytes(const sdm_shape_t* shape) {
   const std::string saved = g_last_error;
   if (check_shape(shape) != SDM_OK) return 0;

@@ -36,4 +36,90 @@ __global__ void __launch_bounds__(256) k_rmsnorm_gate(float* __restrict__ y, con
   }
 }
 
+// Slot utilisation: counts[b, h, i] += number of (t, k) with idx[b, t, h, k]
+// == i. A monitor of how the selection spreads over the N slots (uneven
+// addressing, the "addressing collapse" the SDM pages warn about). grid
+// (ceil(T / tokens_per_cta), B*H), 256 threads. With N <= kCountSmemSlots a
+// CTA counts in shared memory and adds its nonzero bins to global memory at
+// the end; otherwise it adds to global memory directly. The work is HBM-bound
+// (4 bytes of index per count), so each thread keeps kCountUnroll 16-byte
+// index loads in flight before it counts them. Indices outside [0, N) are
+// skipped and flagged.
+constexpr int kCountSmemSlots = 16384;
+constexpr int kCountUnroll = 4;
+
+template <bool kLocal>
+__device__ __forceinline__ void count_one(int slot, int N, int* bins, int32_t* out, unsigned* err) {
+  if (static_cast<unsigned>(slot) >= static_cast<unsigned>(N)) {
+    atomicOr(err, kErrIndexOutOfRange);
+    return;
+  }
+  if (kLocal) atomicAdd(&bins[slot], 1);
+  else atomicAdd(&out[slot], 1);
+}
+
+template <bool kLocal, bool kVec>
+__global__ void __launch_bounds__(256) k_slot_counts(const int32_t* __restrict__ idx, int T, int H, int K, int N,
+                                                     int tokens_per_cta, int32_t* __restrict__ counts,
+                                                     unsigned* err) {
+  extern __shared__ int bins[];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int t0 = blockIdx.x * tokens_per_cta;
+  const int t1 = min(T, t0 + tokens_per_cta);
+  int32_t* out = counts + static_cast<int64_t>(bh) * N;
+  if (kLocal) {
+    for (int i = threadIdx.x; i < N; i += blockDim.x) bins[i] = 0;
+    __syncthreads();
+  }
+  // token t's K indices start at row(t) * K, rows H apart
+  const int64_t row0 = (static_cast<int64_t>(b) * T + t0) * H + h;
+  if (kVec) {
+    const int kv = K / 4;  // int4 per token
+    const int n = (t1 - t0) * kv;
+    for (int x0 = threadIdx.x; x0 < n; x0 += blockDim.x * kCountUnroll) {
+      int4 v[kCountUnroll];
+#pragma unroll
+      for (int u = 0; u < kCountUnroll; ++u) {
+        const int x = x0 + u * blockDim.x;
+        if (x < n) {
+          const int t = x / kv, j = x - t * kv;
+          v[u] = __ldcs(reinterpret_cast<const int4*>(idx + (row0 + static_cast<int64_t>(t) * H) * K) + j);
+        } else {
+          v[u] = make_int4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCountUnroll; ++u) {
+        if (x0 + u * blockDim.x < n) {
+          count_one<kLocal>(v[u].x, N, bins, out, err);
+          count_one<kLocal>(v[u].y, N, bins, out, err);
+          count_one<kLocal>(v[u].z, N, bins, out, err);
+          count_one<kLocal>(v[u].w, N, bins, out, err);
+        }
+      }
+    }
+  } else {
+    const int n = (t1 - t0) * K;
+    for (int x0 = threadIdx.x; x0 < n; x0 += blockDim.x * kCountUnroll) {
+      int v[kCountUnroll];
+#pragma unroll
+      for (int u = 0; u < kCountUnroll; ++u) {
+        const int x = x0 + u * blockDim.x;
+        if (x < n) {
+          const int t = x / K, k = x - t * K;
+          v[u] = __ldcs(idx + (row0 + static_cast<int64_t>(t) * H) * K + k);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCountUnroll; ++u)
+        if (x0 + u * blockDim.x < n) count_one<kLocal>(v[u], N, bins, out, err);
+    }
+  }
+  if (kLocal) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x)
+      if (bins[i] != 0) atomicAdd(&out[i], bins[i]);
+  }
+}
+
 }  // namespace sdm

@@ -100,3 +100,11 @@ def test_argument_errors_without_gpu(lib):
 
 def test_build_flags_target_sm100a():
     assert build_mod.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_slot_count_arguments_without_gpu(lib):
+    assert lib.sdm_slot_counts(None, 1, 4, 1, 2, 64, None, None) == 1
+    assert b"idx" in lib.sdm_last_error()
+    assert lib.sdm_slot_counts(ctypes.c_void_p(64), 1, 4, 1, 0, 64, ctypes.c_void_p(64), None) == 1
+    assert b"K and N" in lib.sdm_last_error()
+    assert lib.sdm_slot_counts(None, 1, 0, 1, 2, 64, ctypes.c_void_p(64), None) == 0

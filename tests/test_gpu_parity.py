@@ -65,6 +65,59 @@ def test_pkm_topk_nan_stays_in_range(sdm, cuda_device):
     assert int(i.min()) >= 0 and int(i.max()) < 32 * 32
 
 
+# -------------------------------------------------------- slot utilisation --
+
+def _bincount(idx: np.ndarray, N: int) -> np.ndarray:
+    """counts[b,h,i] = #{(t,k): idx[b,t,h,k] == i}, by definition."""
+    B, _, H, _ = idx.shape
+    out = np.zeros((B, H, N), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            out[b, h] = np.bincount(idx[b, :, h, :].ravel(), minlength=N)
+    return out
+
+
+# sqrt_n, K, T: N below and above the shared-memory bin limit; T spanning
+# several 256-token blocks with a ragged tail
+SLOTS = [(32, 64, 37), (8, 40, 300), (16, 6, 301), (128, 16, 513), (256, 64, 70), (1, 1, 5)]
+
+
+@pytest.mark.parametrize("sqrt_n,K,T", SLOTS)
+def test_slot_counts_match_bincount(sdm, oracle, cuda_device, sqrt_n, K, T):
+    B, H, N = 2, 3, sqrt_n * sqrt_n
+    x = _scores("ties", B, T, H, sqrt_n, torch.float32, seed=T * 7 + K)
+    oi, _ = oracle.pkm_topk(f32(x), K)
+    counts = sdm.slot_counts(torch.from_numpy(oi).to(cuda_device), N)
+    sdm.stream_check()
+    got = counts.cpu().numpy()
+    want = _bincount(oi, N)
+    assert np.array_equal(got, want)
+    assert (got.sum(axis=-1) == T * K).all()
+
+
+def test_slot_counts_accumulate_over_token_ranges(sdm, cuda_device):
+    g = torch.Generator().manual_seed(5)
+    N = 4096
+    idx = torch.randint(0, N, (1, 600, 2, 8), generator=g, dtype=torch.int32)
+    d = idx.to(cuda_device)
+    counts = sdm.slot_counts(d[:, :257].contiguous(), N)
+    sdm.slot_counts(d[:, 257:].contiguous(), N, counts)
+    sdm.stream_check()
+    assert np.array_equal(counts.cpu().numpy(), _bincount(idx.numpy(), N))
+
+
+@pytest.mark.parametrize("K", [2, 4])  # scalar and 16-byte index loads
+def test_slot_counts_out_of_range_flagged(sdm, cuda_device, K):
+    idx = torch.zeros((1, 4, 1, K), dtype=torch.int32)
+    idx[0, 1, 0, 0] = 64
+    idx[0, 2, 0, 1] = -1
+    for N in (64, 20000):  # shared-memory and global bins
+        counts = sdm.slot_counts(idx.clone().masked_fill_(idx >= 64, N).to(cuda_device), N)
+        with pytest.raises(sdm.SdmError, match="DEVICE_FAULT"):
+            sdm.stream_check()
+        assert int(counts.sum()) == 4 * K - 2 and int(counts[0, 0, 0]) == 4 * K - 2
+
+
 # ------------------------------------------------------------ recurrence --
 
 SCAN = [
