@@ -189,17 +189,27 @@ def algorithmic_bytes_per_token_head(shape: synth.Shape, epilogue: bool) -> int:
     return b
 
 
-def source_digest() -> str:
+# The source files each timed kernel is compiled from; a recorded DRAM
+# traffic figure stays valid while these files are unchanged.
+KERNEL_SOURCES = {
+    "k_scan_resident": ("sdm_device.cuh", "sdm_records.cuh", "sdm_scan.cuh"),
+    "k_scan_streaming": ("sdm_device.cuh", "sdm_records.cuh", "sdm_scan.cuh"),
+    "k_pkm_topk_fast": ("sdm_device.cuh", "pkm_topk_fast.cuh"),
+}
+
+
+def source_digest(kernel: str) -> str:
     h = hashlib.sha256()
-    for p in sorted((ROOT / "sparse_memory_linear_pkm_b200" / "csrc").glob("*")):
-        h.update(p.name.encode())
-        h.update(p.read_bytes())
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(name.encode())
+        h.update((ROOT / "sparse_memory_linear_pkm_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, kernel: str):
+def recorded_traffic(workload: str, kernel: str, config: str):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, when
-    it was taken on the current kernel sources; else None."""
+    it was taken on the current kernel sources and the same launch
+    configuration; else None."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
@@ -207,7 +217,7 @@ def recorded_traffic(workload: str, kernel: str):
         entry = json.loads(p.read_text()).get(workload, {}).get(kernel)
     except Exception:
         return None
-    if not entry or entry.get("source_digest") != source_digest():
+    if not entry or entry.get("source_digest") != source_digest(kernel) or entry.get("config") != config:
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -363,8 +373,9 @@ def run_sdm(args, dist: Dist):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "of fallback"}
     kernel = "k_scan_resident" if resident else "k_scan_streaming"
-    traffic = recorded_traffic(shape.name, kernel)
-    roof.update({"traffic": traffic, "kernel": kernel, "ms_per_launch": scan_ms,
+    launch_cfg = sdm.scan_describe(sh)
+    traffic = recorded_traffic(shape.name, kernel, launch_cfg)
+    roof.update({"traffic": traffic, "kernel": kernel, "launch": launch_cfg, "ms_per_launch": scan_ms,
                  "algorithmic_bytes_per_launch": algo_bytes})
 
     e2e = None

@@ -103,8 +103,9 @@ SDM_API const char* sdm_status_string(sdm_status_t status);
 SDM_API const char* sdm_last_error(void);
 
 /* Slot utilisation of a selection: counts[b,h,i] += the number of (t,k) with
- * idx[b,t,h,k] == i. The pages warn that learned sparse addressing can
- * collapse onto few slots; this monitors it. The paper has no kernel for it.
+ * idx[b,t,h,k] == i ([explainer] "亮点与局限" and "工程落地关键点" item 2: the
+ * learned addressing can collapse onto few slots, so the per-slot update
+ * frequencies are worth tracking; the pages give no kernel for it).
  *   idx    [B,T,H,K] int32 (e.g. the write slots of sdm_pkm_topk)
  *   counts [B,H,N] int32, accumulated (zero it first; calls over consecutive
  *          token ranges add up). Indices outside [0, N) are skipped and set the
@@ -134,6 +135,13 @@ SDM_API size_t sdm_scan_workspace_bytes(const sdm_shape_t* shape);
  * on the current device: SDM_VARIANT_RESIDENT or SDM_VARIANT_STREAMING, or -1
  * if the shape is invalid or unsupported (sdm_last_error() says why). */
 SDM_API int32_t sdm_scan_variant(const sdm_shape_t* shape);
+
+/* The launch configuration of that kernel as text, e.g.
+ * "resident CW=8 NWARP=1 L=4 EB=4 smem=..." or
+ * "streaming C=64 P=3 L=8 NW=16 smem=...", NUL-terminated into out (caller
+ * owned, out_len bytes, truncated to fit). Returns SDM_OK, or an error for an
+ * invalid or unsupported shape (out left empty). For profiles and logs. */
+SDM_API sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_len);
 
 /* The sparse gated delta recurrence over a given selection, in token order
  * ([explainer] 3.1 steps 2-3; [summary] Core Mechanism 3-4). For each token t

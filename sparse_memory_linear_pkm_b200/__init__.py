@@ -20,7 +20,7 @@ import torch
 from . import native, synth
 from .native import SdmError
 
-__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "stream_check", "make_shape",
+__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "scan_describe", "stream_check", "make_shape",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
 _DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
@@ -59,6 +59,13 @@ def scan_variant(shape: native.Shape) -> str:
     if v < 0:
         native.check(1)
     return {1: "resident", 2: "streaming"}[v]
+
+
+def scan_describe(shape: native.Shape) -> str:
+    """The recurrence kernel's launch configuration for this shape, as text."""
+    buf = ctypes.create_string_buffer(128)
+    native.check(native.load().sdm_scan_describe(ctypes.byref(shape), buf, len(buf)))
+    return buf.value.decode()
 
 
 def scan_workspace_bytes(shape: native.Shape) -> int:

@@ -14,7 +14,7 @@ import argparse
 
 import torch
 
-from . import layer_forward, synth
+from . import layer_forward, make_shape, scan_describe, synth
 
 
 def main(argv=None) -> None:
@@ -40,7 +40,9 @@ def main(argv=None) -> None:
         layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], inp["M0"], shape.W, shape.R,
                       g=inp.get("g"), variant=args.variant, y=y, M_out=M)
     torch.cuda.synchronize()
-    print("ok", shape, "variant", args.variant)
+    sh = make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
+                    shape.torch_state(), variant=args.variant)
+    print("ok", shape, "recurrence:", scan_describe(sh))
 
 
 if __name__ == "__main__":

@@ -665,6 +665,22 @@ int32_t sdm_scan_variant(const sdm_shape_t* shape) {
   return c.resident ? SDM_VARIANT_RESIDENT : SDM_VARIANT_STREAMING;
 }
 
+sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_len) {
+  sdm_status_t r;
+  if (out == nullptr || out_len == 0) return fail(SDM_ERR_INVALID_ARGUMENT, "out is null or out_len is 0");
+  out[0] = '\0';
+  DeviceInfo* dev;
+  ScanChoice c;
+  if ((r = check_shape(shape)) != SDM_OK || (r = device_info(&dev)) != SDM_OK ||
+      (r = choose_scan(*dev, *shape, &c)) != SDM_OK)
+    return r;
+  if (c.resident)
+    snprintf(out, out_len, "resident CW=%d NWARP=%d L=%d EB=%d smem=%zu", c.CW, c.NWARP, c.L, c.EB, c.smem);
+  else
+    snprintf(out, out_len, "streaming C=%d P=%d L=%d NW=%d smem=%zu", c.C, c.P, c.L, c.NWARP, c.smem);
+  return ok();
+}
+
 sdm_status_t sdm_scan(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w, const int32_t* idx_r,
                       const float* w_r, const void* v, const void* alpha, const void* beta, const void* g, void* M,
                       float* y, void* workspace, size_t workspace_bytes, void* stream) {

@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(256) k_rmsnorm_gate(float* __restrict__ y, con
 
 // Slot utilisation: counts[b, h, i] += number of (t, k) with idx[b, t, h, k]
 // == i. A monitor of how the selection spreads over the N slots (uneven
-// addressing, the "addressing collapse" the SDM pages warn about). grid
+// addressing, the collapse onto few slots that the explainer page's
+// "亮点与局限" and "工程落地关键点" sections warn about). grid
 // (ceil(T / tokens_per_cta), B*H), 256 threads. With N <= kCountSmemSlots a
 // CTA counts in shared memory and adds its nonzero bins to global memory at
 // the end; otherwise it adds to global memory directly. The work is HBM-bound
