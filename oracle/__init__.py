@@ -87,6 +87,19 @@ class Oracle:
             _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
             ctypes.c_double, _c_i32, _c_ptr, _c_ptr, _c_i32, ctypes.POINTER(_c_i64),
         ]
+        lib.oracle_scan_f64.restype = ctypes.c_int
+        lib.oracle_scan_f64.argtypes = [
+            _c_i32, _c_i32, _c_i32, _c_i64, _c_i32, _c_i32, _c_i32,
+            _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32,
+        ]
+        lib.oracle_scan_backward.restype = ctypes.c_int
+        lib.oracle_scan_backward.argtypes = [
+            _c_i32, _c_i32, _c_i32, _c_i64, _c_i32, _c_i32, _c_i32,
+            _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr,
+            _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32,
+        ]
+        lib.oracle_pkm_topk_backward.restype = ctypes.c_int
+        lib.oracle_pkm_topk_backward.argtypes = [_c_i64, _c_i32, _c_i32, _c_ptr, _c_ptr, _c_ptr, _c_ptr]
         lib.oracle_round_to_bf16.restype = ctypes.c_float
         lib.oracle_round_to_bf16.argtypes = [ctypes.c_double]
         self.lib = lib
@@ -138,6 +151,61 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_scan failed with code {rc}")
         return y, M_T, int(ops.value)
+
+    def scan_f64(self, idx_w, w_w, idx_r, w_r, v, alpha, beta, M, n_threads: int | None = None):
+        """The recurrence with inputs and state in double, never rounded (no
+        epilogue). Returns (y float64, M_T float64)."""
+        idx_w, idx_r = _i32(idx_w), _i32(idx_r)
+        w_w, w_r = _f64(w_w), _f64(w_r)
+        v, alpha, beta = _f64(v), _f64(alpha), _f64(beta)
+        M_T = _f64(M).copy()
+        B, T, H, W = idx_w.shape
+        R = idx_r.shape[-1]
+        d_v = v.shape[-1]
+        N = M_T.shape[2]
+        y = np.zeros((B, T, H, d_v), dtype=np.float64)
+        rc = self.lib.oracle_scan_f64(B, T, H, N, d_v, W, R, _p(idx_w), _p(w_w), _p(idx_r), _p(w_r),
+                                      _p(v), _p(alpha), _p(beta), _p(M_T), _p(y), n_threads or default_threads())
+        if rc != 0:
+            raise ValueError(f"oracle_scan_f64 failed with code {rc}")
+        return y, M_T
+
+    def scan_backward(self, idx_w, w_w, idx_r, w_r, v, alpha, beta, M0, dy, dM_T=None,
+                      n_threads: int | None = None):
+        """Derivatives of L = sum <dy, y> + <dM_T, M_T> through the recurrence
+        (scan_f64's function). Returns a dict with dv, dalpha, dbeta, dw_w,
+        dw_r and dM0 (all float64)."""
+        idx_w, idx_r = _i32(idx_w), _i32(idx_r)
+        w_w, w_r = _f64(w_w), _f64(w_r)
+        v, alpha, beta, M0, dy = _f64(v), _f64(alpha), _f64(beta), _f64(M0), _f64(dy)
+        B, T, H, W = idx_w.shape
+        R = idx_r.shape[-1]
+        d_v = v.shape[-1]
+        N = M0.shape[2]
+        dM = np.zeros_like(M0) if dM_T is None else _f64(dM_T).copy()
+        out = {"dv": np.zeros_like(v), "dalpha": np.zeros_like(alpha), "dbeta": np.zeros_like(beta),
+               "dw_w": np.zeros_like(w_w), "dw_r": np.zeros_like(w_r)}
+        rc = self.lib.oracle_scan_backward(B, T, H, N, d_v, W, R, _p(idx_w), _p(w_w), _p(idx_r), _p(w_r),
+                                           _p(v), _p(alpha), _p(beta), _p(M0), _p(dy), _p(dM), _p(out["dv"]),
+                                           _p(out["dalpha"]), _p(out["dbeta"]), _p(out["dw_w"]),
+                                           _p(out["dw_r"]), n_threads or default_threads())
+        if rc != 0:
+            raise ValueError(f"oracle_scan_backward failed with code {rc}")
+        out["dM0"] = dM
+        return out
+
+    def pkm_topk_backward(self, idx, w, dw, sqrt_n: int):
+        """dL/dscores [..., 2*sqrt_n] of the selection weights for a fixed
+        selection, given dL/dw."""
+        idx, w, dw = _i32(idx), _f64(w), _f64(dw)
+        lead = idx.shape[:-1]
+        K = idx.shape[-1]
+        n_units = int(np.prod(lead)) if lead else 1
+        ds = np.zeros(lead + (2 * sqrt_n,), dtype=np.float64)
+        rc = self.lib.oracle_pkm_topk_backward(n_units, int(sqrt_n), int(K), _p(idx), _p(w), _p(dw), _p(ds))
+        if rc != 0:
+            raise ValueError(f"oracle_pkm_topk_backward failed with code {rc}")
+        return ds
 
     # -- whole layer ---------------------------------------------------------
     def layer_forward(self, kp, qp, v, alpha, beta, M0, W: int, R: int, g=None,

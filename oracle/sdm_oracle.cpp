@@ -34,9 +34,16 @@
 //      y_t = sum over read slots of q_i * M_t[i], in double.
 //   5. Optional epilogue ([explainer] 3.1 step 3): y <- g * y / sqrt(mean(y^2)+eps).
 //
+//   6. Backward (the derivatives for training): reverse-mode through steps 2-4
+//      for a fixed selection, by the chain rule on the pages' own formulas
+//      ([explainer] 3.4 "高效训练" says only that a memory-efficient backward
+//      exists and leaves its details to an appendix the pages do not show).
+//
 // Parity status: selection, weights, write, read and epilogue are each pinned by
 // tests that do not re-run this file's formulas (exact-rational brute force,
-// closed forms, invariants, hand-worked fixtures, planted-mistake checks).
+// closed forms, invariants, hand-worked fixtures, planted-mistake checks); the
+// backward is pinned by central finite differences of the double-precision
+// forward, a hand-derived one-slot closed form, and planted-mistake checks.
 //
 // ORACLE_MUTANT (default 0) plants one known mistake per value so the tests
 // can show that the pins catch it; it is never set outside those tests.
@@ -163,6 +170,128 @@ void select_one(const float* x, int32_t sqrt_n, int32_t K, std::vector<SlotScore
   }
 }
 
+// Stores a freshly computed state value: rounded to fp32 (or to bf16 and kept
+// as an exact fp32) in a float state; kept exactly in a double state.
+template <class S>
+inline S store_state(double x, bool bf16);
+template <>
+inline float store_state<float>(double x, bool bf16) {
+  return round_state(x, bf16);
+}
+template <>
+inline double store_state<double>(double x, bool) {
+  return x;
+}
+
+// The recurrence over a given selection (the body of oracle_scan and
+// oracle_scan_f64; S is the state's storage type, I the type of v, alpha, beta).
+template <class S, class I>
+int scan_impl(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W, int32_t R,
+              const int32_t* idx_w, const double* w_w, const int32_t* idx_r, const double* w_r,
+              const I* v, const I* alpha, const I* beta, const float* g,
+              double eps, int32_t state_bf16, S* M, double* y, int32_t n_threads,
+              int64_t* op_count) {
+  if (B < 0 || T < 0 || H < 0 || N < 1 || d_v < 1 || W < 0 || R < 0) return -1;
+  for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * W; ++e)
+    if (idx_w[e] < 0 || idx_w[e] >= N) return -2;
+  for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * R; ++e)
+    if (idx_r[e] < 0 || idx_r[e] >= N) return -2;
+  const bool bf16 = state_bf16 != 0;
+  // Columns of d_v evolve independently, so the work splits over (b, h, column block).
+  const int32_t col_block = 64;
+  const int32_t n_cb = (d_v + col_block - 1) / col_block;
+  std::atomic<int64_t> ops(0);
+  parallel_for(static_cast<int64_t>(B) * H * n_cb, std::max(1, n_threads), [&](int64_t u) {
+    const int32_t cb = static_cast<int32_t>(u % n_cb);
+    const int32_t h = static_cast<int32_t>((u / n_cb) % H);
+    const int32_t b = static_cast<int32_t>(u / (static_cast<int64_t>(n_cb) * H));
+    const int32_t c0 = cb * col_block;
+    const int32_t c1 = std::min(d_v, c0 + col_block);
+    S* Mbh = M + (static_cast<int64_t>(b) * H + h) * N * d_v;
+    int64_t local_ops = 0;
+    for (int32_t t = 0; t < T; ++t) {
+      const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;  // token-head
+      const double a_t = alpha[th];
+      const double b_t = beta[th];
+      const I* v_t = v + th * d_v;
+      double* y_t = y + th * d_v;
+      auto do_reads = [&]() {
+        for (int32_t c = c0; c < c1; ++c) {
+          double acc = 0.0;
+          for (int32_t r = 0; r < R; ++r) {
+            const int64_t i = idx_r[th * R + r];
+            acc += w_r[th * R + r] * static_cast<double>(Mbh[i * d_v + c]);
+          }
+          y_t[c] = acc;
+        }
+        local_ops += static_cast<int64_t>(2) * R * (c1 - c0);
+      };
+#if ORACLE_MUTANT == 6
+      do_reads();  // planted: read before the write
+#endif
+      // Step 2: gated delta write on the selected write slots only.
+      for (int32_t j = 0; j < W; ++j) {
+        const int64_t i = idx_w[th * W + j];
+        const double k_i = w_w[th * W + j];
+        for (int32_t c = c0; c < c1; ++c) {
+          const double m_prev = Mbh[i * d_v + c];
+#if ORACLE_MUTANT == 4
+          const double m_tilde = m_prev;  // planted: forget gate dropped
+#else
+          const double m_tilde = a_t * m_prev;
+#endif
+          const double v_c = v_t[c];
+#if ORACLE_MUTANT == 5
+          const double m_new = m_tilde - b_t * k_i * (v_c - m_tilde);  // planted: sign
+#elif ORACLE_MUTANT == 7
+          const double m_new = m_tilde + b_t * (v_c - m_tilde);  // planted: k dropped
+#else
+          const double m_new = m_tilde + b_t * k_i * (v_c - m_tilde);
+#endif
+#if ORACLE_MUTANT == 10
+          Mbh[i * d_v + c] = static_cast<S>(m_new);  // planted: no state rounding
+#else
+          Mbh[i * d_v + c] = store_state<S>(m_new, bf16);
+#endif
+        }
+        local_ops += static_cast<int64_t>(4) * (c1 - c0);
+      }
+#if ORACLE_MUTANT == 11
+      // planted: the forget gate also decays one unselected slot
+      {
+        int64_t other = (idx_w[th * W] + 1) % N;
+        bool selected = false;
+        for (int32_t j = 0; j < W; ++j) selected = selected || idx_w[th * W + j] == other;
+        if (!selected)
+          for (int32_t c = c0; c < c1; ++c)
+            Mbh[other * d_v + c] = store_state<S>(a_t * Mbh[other * d_v + c], bf16);
+      }
+#endif
+      // Step 3: sparse read of the state after this token's write.
+#if ORACLE_MUTANT != 6
+      do_reads();
+#endif
+    }
+    ops.fetch_add(local_ops);
+  });
+  // Optional epilogue: RMS-norm over d_v per token-head, then the element-wise gate.
+  if (g != nullptr) {
+    parallel_for(static_cast<int64_t>(B) * T * H, std::max(1, n_threads), [&](int64_t th) {
+      double* y_t = y + th * d_v;
+      double ss = 0.0;
+      for (int32_t c = 0; c < d_v; ++c) ss += y_t[c] * y_t[c];
+#if ORACLE_MUTANT == 9
+      const double inv = 1.0 / std::sqrt(ss + eps);  // planted: sum instead of mean
+#else
+      const double inv = 1.0 / std::sqrt(ss / d_v + eps);
+#endif
+      for (int32_t c = 0; c < d_v; ++c) y_t[c] = static_cast<double>(g[th * d_v + c]) * y_t[c] * inv;
+    });
+  }
+  if (op_count != nullptr) *op_count = ops.load();
+  return 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -207,104 +336,170 @@ int oracle_scan(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t
                 const float* v, const float* alpha, const float* beta, const float* g,
                 double eps, int32_t state_bf16, float* M, double* y, int32_t n_threads,
                 int64_t* op_count) {
+  return scan_impl<float, float>(B, T, H, N, d_v, W, R, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, eps, state_bf16,
+                          M, y, n_threads, op_count);
+}
+
+// The same recurrence with inputs and state in double and the state never
+// rounded: the exact function whose derivatives oracle_scan_backward computes.
+int oracle_scan_f64(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W, int32_t R,
+                    const int32_t* idx_w, const double* w_w, const int32_t* idx_r, const double* w_r,
+                    const double* v, const double* alpha, const double* beta, double* M, double* y,
+                    int32_t n_threads) {
+  return scan_impl<double, double>(B, T, H, N, d_v, W, R, idx_w, w_w, idx_r, w_r, v, alpha, beta, nullptr, 0.0, 0, M,
+                           y, n_threads, nullptr);
+}
+
+// Reverse-mode derivatives of the recurrence as oracle_scan_f64 computes it
+// (no epilogue), for the loss L = sum_t <dy_t, y_t> + <dM_T, M_T>, by the chain
+// rule through the pages' own two-step write ([explainer] 3.1 step 2):
+//   m~ = alpha * m_old;   m_new = m~ + beta * k * (v - m~)
+// and the read after the write ([explainer] 3.1 step 3): y_t = sum q_i M_t[i].
+// The forward trajectory is recomputed first, keeping every overwritten value;
+// the sweep then runs backwards over tokens (the read before the write, the
+// write entries in reverse order), restoring the state as it goes.
+//   M0   : [B,H,N,d_v] the state the forward started from (double)
+//   dy   : [B,T,H,d_v] dL/dy;  dM: [B,H,N,d_v] in: dL/dM_T, out: dL/dM_0
+//   dv   : [B,T,H,d_v] out;  dalpha, dbeta: [B,T,H] out
+//   dw_w : [B,T,H,W] out, dL/dk_i;  dw_r: [B,T,H,R] out, dL/dq_i
+// Returns 0, or -1 for invalid sizes, or -2 when an index is outside [0, N).
+int oracle_scan_backward(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W, int32_t R,
+                         const int32_t* idx_w, const double* w_w, const int32_t* idx_r, const double* w_r,
+                         const double* v, const double* alpha, const double* beta, const double* M0,
+                         const double* dy, double* dM, double* dv, double* dalpha, double* dbeta,
+                         double* dw_w, double* dw_r, int32_t n_threads) {
   if (B < 0 || T < 0 || H < 0 || N < 1 || d_v < 1 || W < 0 || R < 0) return -1;
   for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * W; ++e)
     if (idx_w[e] < 0 || idx_w[e] >= N) return -2;
   for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * R; ++e)
     if (idx_r[e] < 0 || idx_r[e] >= N) return -2;
-  const bool bf16 = state_bf16 != 0;
-  // Columns of d_v evolve independently, so the work splits over (b, h, column block).
-  const int32_t col_block = 64;
-  const int32_t n_cb = (d_v + col_block - 1) / col_block;
-  std::atomic<int64_t> ops(0);
-  parallel_for(static_cast<int64_t>(B) * H * n_cb, std::max(1, n_threads), [&](int64_t u) {
-    const int32_t cb = static_cast<int32_t>(u % n_cb);
-    const int32_t h = static_cast<int32_t>((u / n_cb) % H);
-    const int32_t b = static_cast<int32_t>(u / (static_cast<int64_t>(n_cb) * H));
-    const int32_t c0 = cb * col_block;
-    const int32_t c1 = std::min(d_v, c0 + col_block);
-    float* Mbh = M + (static_cast<int64_t>(b) * H + h) * N * d_v;
-    int64_t local_ops = 0;
+  // Every (b, h) is independent; its scalar gradients sum over all columns,
+  // so one (b, h) is one unit of work.
+  parallel_for(static_cast<int64_t>(B) * H, std::max(1, n_threads), [&](int64_t u) {
+    const int32_t h = static_cast<int32_t>(u % H);
+    const int32_t b = static_cast<int32_t>(u / H);
+    const int64_t state_off = (static_cast<int64_t>(b) * H + h) * N * d_v;
+    std::vector<double> M(M0 + state_off, M0 + state_off + N * d_v);
+    std::vector<double> old(static_cast<size_t>(T) * W * d_v);  // overwritten values, [t][j][c]
+    // Forward: the recomputed trajectory.
     for (int32_t t = 0; t < T; ++t) {
-      const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;  // token-head
-      const double a_t = alpha[th];
-      const double b_t = beta[th];
-      const float* v_t = v + th * d_v;
-      double* y_t = y + th * d_v;
-      auto do_reads = [&]() {
-        for (int32_t c = c0; c < c1; ++c) {
-          double acc = 0.0;
-          for (int32_t r = 0; r < R; ++r) {
-            const int64_t i = idx_r[th * R + r];
-            acc += w_r[th * R + r] * static_cast<double>(Mbh[i * d_v + c]);
-          }
-          y_t[c] = acc;
-        }
-        local_ops += static_cast<int64_t>(2) * R * (c1 - c0);
-      };
-#if ORACLE_MUTANT == 6
-      do_reads();  // planted: read before the write
-#endif
-      // Step 2: gated delta write on the selected write slots only.
+      const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;
       for (int32_t j = 0; j < W; ++j) {
         const int64_t i = idx_w[th * W + j];
         const double k_i = w_w[th * W + j];
-        for (int32_t c = c0; c < c1; ++c) {
-          const double m_prev = Mbh[i * d_v + c];
-#if ORACLE_MUTANT == 4
-          const double m_tilde = m_prev;  // planted: forget gate dropped
+        for (int32_t c = 0; c < d_v; ++c) {
+          const double m_old = M[i * d_v + c];
+          old[(static_cast<size_t>(t) * W + j) * d_v + c] = m_old;
+          const double m_tilde = alpha[th] * m_old;
+          M[i * d_v + c] = m_tilde + beta[th] * k_i * (v[th * d_v + c] - m_tilde);
+        }
+      }
+    }
+    // Backward: G = dL/dM_t, starting from dL/dM_T.
+    std::vector<double> G(dM + state_off, dM + state_off + N * d_v);
+    for (int32_t t = T - 1; t >= 0; --t) {
+      const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;
+      const double a_t = alpha[th];
+      const double b_t = beta[th];
+      const double* dy_t = dy + th * d_v;
+      const double* v_t = v + th * d_v;
+      double* dv_t = dv + th * d_v;
+      for (int32_t c = 0; c < d_v; ++c) dv_t[c] = 0.0;
+      // Read: y_t = sum_r q_r M_t[i_r]  ->  dq_r = <dy_t, M_t[i_r]>, G[i_r] += q_r dy_t.
+      for (int32_t r = 0; r < R; ++r) {
+        const int64_t i = idx_r[th * R + r];
+        double dq = 0.0;
+        for (int32_t c = 0; c < d_v; ++c) {
+#if ORACLE_MUTANT == 14
+          // planted: the read gradient taken from the state before the write
+          double m_c = M[i * d_v + c];
+          for (int32_t j = 0; j < W; ++j)
+            if (idx_w[th * W + j] == i) m_c = old[(static_cast<size_t>(t) * W + j) * d_v + c];
+          dq += dy_t[c] * m_c;
 #else
-          const double m_tilde = a_t * m_prev;
-#endif
-          const double v_c = v_t[c];
-#if ORACLE_MUTANT == 5
-          const double m_new = m_tilde - b_t * k_i * (v_c - m_tilde);  // planted: sign
-#elif ORACLE_MUTANT == 7
-          const double m_new = m_tilde + b_t * (v_c - m_tilde);  // planted: k dropped
-#else
-          const double m_new = m_tilde + b_t * k_i * (v_c - m_tilde);
-#endif
-#if ORACLE_MUTANT == 10
-          Mbh[i * d_v + c] = static_cast<float>(m_new);  // planted: no state rounding
-#else
-          Mbh[i * d_v + c] = round_state(m_new, bf16);
+          dq += dy_t[c] * M[i * d_v + c];
 #endif
         }
-        local_ops += static_cast<int64_t>(4) * (c1 - c0);
+        dw_r[th * R + r] = dq;
+        for (int32_t c = 0; c < d_v; ++c) G[i * d_v + c] += w_r[th * R + r] * dy_t[c];
       }
-#if ORACLE_MUTANT == 11
-      // planted: the forget gate also decays one unselected slot
-      {
-        int64_t other = (idx_w[th * W] + 1) % N;
-        bool selected = false;
-        for (int32_t j = 0; j < W; ++j) selected = selected || idx_w[th * W + j] == other;
-        if (!selected)
-          for (int32_t c = c0; c < c1; ++c)
-            Mbh[other * d_v + c] = round_state(a_t * Mbh[other * d_v + c], bf16);
-      }
+      // Write, entries in reverse order.
+      double da_t = 0.0, db_t = 0.0;
+      for (int32_t j = W - 1; j >= 0; --j) {
+        const int64_t i = idx_w[th * W + j];
+        const double k_i = w_w[th * W + j];
+        double dk = 0.0;
+        for (int32_t c = 0; c < d_v; ++c) {
+          const double m_old = old[(static_cast<size_t>(t) * W + j) * d_v + c];
+          const double m_tilde = a_t * m_old;
+          const double g = G[i * d_v + c];                   // dL/dm_new
+          const double d_tilde = g * (1.0 - b_t * k_i);      // dL/dm~
+          dv_t[c] += g * b_t * k_i;
+          db_t += g * k_i * (v_t[c] - m_tilde);
+#if ORACLE_MUTANT == 15
+          (void)d_tilde;  // planted: dk without its beta (v - m~) factor's m~ part
+          dk += g * b_t * v_t[c];
+#else
+          dk += g * b_t * (v_t[c] - m_tilde);
 #endif
-      // Step 3: sparse read of the state after this token's write.
-#if ORACLE_MUTANT != 6
-      do_reads();
+#if ORACLE_MUTANT == 12
+          da_t += g * m_old;  // planted: the (1 - beta k) factor dropped
+#else
+          da_t += d_tilde * m_old;
+#endif
+#if ORACLE_MUTANT == 13
+          G[i * d_v + c] = g;  // planted: the adjoint passes the write undecayed
+#else
+          G[i * d_v + c] = d_tilde * a_t;
+#endif
+          M[i * d_v + c] = m_old;
+        }
+        dw_w[th * W + j] = dk;
+      }
+      dalpha[th] = da_t;
+      dbeta[th] = db_t;
+    }
+    std::copy(G.begin(), G.end(), dM + state_off);
+  });
+  return 0;
+}
+
+// Derivative of the softmax selection weights with respect to the scores, for
+// a fixed selection (the selected set and its order do not move under an
+// infinitesimal change of distinct scores). With sigma_k = s1[a_k] + s2[b_k]
+// and w = softmax(sigma): dL/dsigma_k = w_k (dw_k - sum_j w_j dw_j), and each
+// sigma_k adds its derivative to s1[a_k] and to s2[b_k], slot = a*sqrt_n + b.
+//   idx, w, dw : [n_units, K];  dscores: [n_units, 2*sqrt_n] out (zero where
+//   no selected slot uses the entry). Returns 0, -1 for invalid sizes, -2 for
+//   an index outside [0, N).
+int oracle_pkm_topk_backward(int64_t n_units, int32_t sqrt_n, int32_t K, const int32_t* idx, const double* w,
+                             const double* dw, double* dscores) {
+  if (sqrt_n < 1 || K < 1 || n_units < 0) return -1;
+  const int64_t N = static_cast<int64_t>(sqrt_n) * sqrt_n;
+  for (int64_t u = 0; u < n_units; ++u) {
+    const int32_t* id = idx + u * K;
+    const double* wu = w + u * K;
+    const double* du = dw + u * K;
+    double* ds = dscores + u * 2 * sqrt_n;
+    for (int32_t x = 0; x < 2 * sqrt_n; ++x) ds[x] = 0.0;
+    double mean = 0.0;
+    for (int32_t k = 0; k < K; ++k) mean += wu[k] * du[k];
+    for (int32_t k = 0; k < K; ++k) {
+      if (id[k] < 0 || id[k] >= N) return -2;
+#if ORACLE_MUTANT == 16
+      const double dsig = wu[k] * du[k];  // planted: the weighted mean not subtracted
+#else
+      const double dsig = wu[k] * (du[k] - mean);
+#endif
+#if ORACLE_MUTANT == 17
+      ds[id[k] % sqrt_n] += dsig;  // planted: halves swapped
+      ds[sqrt_n + id[k] / sqrt_n] += dsig;
+#else
+      ds[id[k] / sqrt_n] += dsig;
+      ds[sqrt_n + id[k] % sqrt_n] += dsig;
 #endif
     }
-    ops.fetch_add(local_ops);
-  });
-  // Optional epilogue: RMS-norm over d_v per token-head, then the element-wise gate.
-  if (g != nullptr) {
-    parallel_for(static_cast<int64_t>(B) * T * H, std::max(1, n_threads), [&](int64_t th) {
-      double* y_t = y + th * d_v;
-      double ss = 0.0;
-      for (int32_t c = 0; c < d_v; ++c) ss += y_t[c] * y_t[c];
-#if ORACLE_MUTANT == 9
-      const double inv = 1.0 / std::sqrt(ss + eps);  // planted: sum instead of mean
-#else
-      const double inv = 1.0 / std::sqrt(ss / d_v + eps);
-#endif
-      for (int32_t c = 0; c < d_v; ++c) y_t[c] = static_cast<double>(g[th * d_v + c]) * y_t[c] * inv;
-    });
   }
-  if (op_count != nullptr) *op_count = ops.load();
   return 0;
 }
 

@@ -354,6 +354,121 @@ def pin_round_to_bf16(o):
         assert o.round_to_bf16(float(x)) == _bf16_rne(float(x)), x
 
 
+# ----------------------------------------------------------------- backward --
+# The backward (training derivatives) of the write/read recurrence and of the
+# selection weights. The SDM explainer's section 3.4 says only that a
+# memory-efficient backward exists; its derivatives follow from the forward
+# formulas by the chain rule, so the forward itself (pinned above) is the
+# reference: central finite differences of the double-precision forward.
+
+
+def _scan_loss(o, inp, dy, dM_T):
+    y, M_T = o.scan_f64(inp["idx_w"], inp["w_w"], inp["idx_r"], inp["w_r"], inp["v"], inp["alpha"],
+                        inp["beta"], inp["M"])
+    return float(np.sum(dy * y) + np.sum(dM_T * M_T))
+
+
+def _backward_case(seed, T=6, N=11, W=3, R=2):
+    rng = np.random.default_rng(seed)
+    inp = _scan_inputs(rng, B=1, T=T, H=2, N=N, d_v=3, W=W, R=R)
+    inp = {k: (v.astype(np.float64) if v.dtype == np.float32 else v) for k, v in inp.items()}
+    inp["M"] = rng.standard_normal(inp["M"].shape)  # O(1) state so every term matters
+    dy = rng.standard_normal(inp["v"].shape)
+    dM_T = rng.standard_normal(inp["M"].shape)
+    return rng, inp, dy, dM_T
+
+
+def pin_backward_finite_differences(o):
+    """<grad, D> equals the central difference (L(x + hD) - L(x - hD)) / 2h of
+    L = sum <dy, y> + <dM_T, M_T> for a random direction D in each input, and
+    for single coordinates of each input."""
+    for seed in (0, 1):
+        rng, inp, dy, dM_T = _backward_case(seed)
+        g = o.scan_backward(inp["idx_w"], inp["w_w"], inp["idx_r"], inp["w_r"], inp["v"], inp["alpha"],
+                            inp["beta"], inp["M"], dy, dM_T)
+        grads = {"v": g["dv"], "alpha": g["dalpha"], "beta": g["dbeta"], "w_w": g["dw_w"], "w_r": g["dw_r"],
+                 "M": g["dM0"]}
+        h = 1e-6
+        for name, grad in grads.items():
+            dirs = [rng.standard_normal(grad.shape)]
+            for _ in range(3):
+                e = np.zeros(grad.shape)
+                e[tuple(int(rng.integers(0, n)) for n in grad.shape)] = 1.0
+                dirs.append(e)
+            for D in dirs:
+                plus = dict(inp, **{name: inp[name] + h * D})
+                minus = dict(inp, **{name: inp[name] - h * D})
+                fd = (_scan_loss(o, plus, dy, dM_T) - _scan_loss(o, minus, dy, dM_T)) / (2 * h)
+                an = float(np.sum(grad * D))
+                assert abs(fd - an) <= 1e-6 * (1.0 + abs(an)), (name, seed, fd, an)
+
+
+def pin_backward_one_slot_golden(o):
+    """Hand-derived derivatives of one write and one read of one slot
+    (tests/golden/backward_one_slot.json), exact binary fractions."""
+    data = json.loads((GOLDEN / "backward_one_slot.json").read_text())
+    x = data["inputs"]
+    one = lambda val, dt=np.float64: np.full((1, 1, 1, 1), val, dtype=dt)
+    for case in data["cases"]:
+        g = o.scan_backward(one(0, np.int32), one(x["k"]), one(0, np.int32), one(x["q"]), one(x["v"]),
+                            np.full((1, 1, 1), x["alpha"]), np.full((1, 1, 1), x["beta"]), one(x["M0"]),
+                            one(case["dy"]), one(case["dM_T"]))
+        got = {"dw_r": g["dw_r"], "dM0": g["dM0"], "dv": g["dv"], "dalpha": g["dalpha"], "dbeta": g["dbeta"],
+               "dw_w": g["dw_w"]}
+        for k, arr in got.items():
+            assert float(arr.ravel()[0]) == case[k], (case["name"], k, float(arr.ravel()[0]), case[k])
+
+
+def pin_backward_unselected_pass_through(o):
+    """Slots that no token writes pass dL/dM_T to dL/dM_0 unchanged, plus the
+    read contributions sum_t q dy_t for slots that are only read."""
+    rng, inp, dy, dM_T = _backward_case(3, T=5, N=40)
+    g = o.scan_backward(inp["idx_w"], inp["w_w"], inp["idx_r"], inp["w_r"], inp["v"], inp["alpha"],
+                        inp["beta"], inp["M"], dy, dM_T)
+    written = set(inp["idx_w"].ravel().tolist())
+    for h in range(inp["M"].shape[1]):
+        for s in range(inp["M"].shape[2]):
+            if s in written:
+                continue
+            want = dM_T[0, h, s].copy()
+            for t in range(inp["idx_r"].shape[1]):
+                for r in range(inp["idx_r"].shape[3]):
+                    if inp["idx_r"][0, t, h, r] == s:
+                        want += inp["w_r"][0, t, h, r] * dy[0, t, h]
+            assert np.allclose(g["dM0"][0, h, s], want, rtol=0, atol=1e-12), (h, s)
+
+
+def _softmax_loss(o, x, dw, K):
+    idx, w = o.pkm_topk(x, K)
+    return idx, float(np.sum(dw * w))
+
+
+def pin_topk_backward(o):
+    """d/dscores of <dw, w(scores)> for a fixed selection: central differences
+    in fp32 scores with a power-of-two step (exact in fp32), and the invariant
+    that each half's derivatives sum to zero (softmax is shift invariant)."""
+    rng = np.random.default_rng(7)
+    sqrt_n, K = 6, 5
+    x = rng.standard_normal((3, 2 * sqrt_n)).astype(np.float32)
+    dw = rng.standard_normal((3, K))
+    idx, w = o.pkm_topk(x, K)
+    ds = o.pkm_topk_backward(idx, w, dw, sqrt_n)
+    assert np.allclose(ds[:, :sqrt_n].sum(-1), 0.0, atol=1e-12) and np.allclose(ds[:, sqrt_n:].sum(-1), 0.0,
+                                                                                 atol=1e-12)
+    h = np.float32(2.0 ** -12)
+    for u in range(x.shape[0]):
+        for j in range(2 * sqrt_n):
+            xp, xm = x.copy(), x.copy()
+            xp[u, j] += h
+            xm[u, j] -= h
+            ip, lp = _softmax_loss(o, xp[u:u + 1], dw[u:u + 1], K)
+            im, lm = _softmax_loss(o, xm[u:u + 1], dw[u:u + 1], K)
+            if not (np.array_equal(ip[0], idx[u]) and np.array_equal(im[0], idx[u])):
+                continue  # the step moved the selection; the derivative is not defined there
+            fd = (lp - lm) / (2 * float(h))
+            assert abs(fd - ds[u, j]) <= 1e-5 * (1.0 + abs(ds[u, j])), (u, j, fd, ds[u, j])
+
+
 ALL_PINS = {
     "selection_brute_force": pin_selection_brute_force,
     "selection_identity": pin_selection_identity,
@@ -371,6 +486,10 @@ ALL_PINS = {
     "scan_bf16_state": pin_scan_bf16_state,
     "epilogue": pin_epilogue,
     "round_to_bf16": pin_round_to_bf16,
+    "backward_finite_differences": pin_backward_finite_differences,
+    "backward_one_slot_golden": pin_backward_one_slot_golden,
+    "backward_unselected_pass_through": pin_backward_unselected_pass_through,
+    "topk_backward": pin_topk_backward,
 }
 
 

@@ -4,7 +4,9 @@ Each value of ORACLE_MUTANT compiles the oracle with one plausible error (a
 transposed slot number, a wrong tie rule, an ignored low part of the exact
 sum, a dropped forget gate, a flipped delta sign, a read before the write, a
 dropped sparse weight, uniform weights, sum instead of mean in the RMS-norm,
-a missing bf16 rounding, a decayed unselected slot). The test rebuilds the
+a missing bf16 rounding, a decayed unselected slot, and in the backward a
+dropped factor or term, an undecayed adjoint, a read gradient from the wrong
+state, a softmax derivative without its mean, swapped score halves). The test rebuilds the
 oracle on the CPU for each and requires that at least one pin fails.
 """
 
@@ -25,6 +27,12 @@ MUTANTS = {
     9: "RMS-norm over the sum, not the mean",
     10: "bf16 state not rounded",
     11: "unselected slot decayed",
+    12: "backward: (1 - beta k) dropped from dalpha",
+    13: "backward: adjoint not decayed by the write",
+    14: "backward: read gradient from the state before the write",
+    15: "backward: dk without its m~ term",
+    16: "backward: softmax mean not subtracted",
+    17: "backward: score halves swapped",
 }
 
 
