@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--decode", action="store_true",
                     help="time decode steps instead: one token per call (sdm_layer_step), state carried")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward instead: sdm_scan_backward and the two selection-weight backwards")
     ap.add_argument("--slot-counts", action="store_true",
                     help="time the slot utilisation histogram of the workload's write selection instead")
     return ap.parse_args()
@@ -519,6 +521,90 @@ def run_decode(args, dist: Dist):
     dist.close()
 
 
+def run_backward(args, dist: Dist):
+    """Backward: each step takes dy = dL/dy and computes the derivatives of
+    the recurrence (sdm_scan_backward: dv, dalpha, dbeta, dk, dq, dM_0 with the
+    forward recomputed from M_0) and of both selections' softmax weights
+    (sdm_pkm_topk_backward on k' and q'), from the forward's saved selection.
+    dL/dM_T is zero (reset every step). Reports tokens/s and, for the
+    recurrence kernel, the shared-memory state traffic of its reverse sweep
+    against the shared-memory roofline."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --backward needs a CUDA device")
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    shape = synth.WORKLOADS[args.workload]
+    sdm.native.load()
+    inp = synth.make_inputs(shape, seed=args.seed + dist.rank, device=dev)
+    idx_w, w_w = sdm.pkm_topk(inp["kp"], shape.W)
+    idx_r, w_r = sdm.pkm_topk(inp["qp"], shape.R)
+    M0 = inp["M0"].float().contiguous()
+    gen = torch.Generator(device=dev).manual_seed(args.seed + 17)
+    dy = torch.randn((shape.B, shape.T, shape.H, shape.d_v), generator=gen, device=dev)
+    dM = torch.zeros((shape.B, shape.H, shape.N, shape.d_v), dtype=torch.float32, device=dev)
+    sh = sdm.make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
+                        torch.float32)
+    ws = torch.empty(max(16, sdm.scan_backward_workspace_bytes(sh)), dtype=torch.uint8, device=dev)
+    dk = torch.empty((shape.B, shape.T, shape.H, 2 * shape.sqrt_n), dtype=torch.float32, device=dev)
+    dq = torch.empty_like(dk)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dM.zero_()
+        g = sdm.scan_backward(idx_w, w_w, idx_r, w_r, inp["v"], inp["alpha"], inp["beta"], M0, dy, dM, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        sdm.pkm_topk_backward(idx_w, w_w, g["dw_w"], shape.sqrt_n, dk)
+        sdm.pkm_topk_backward(idx_r, w_r, g["dw_r"], shape.sqrt_n, dq)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    sdm.stream_check(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for k in range(args.steps):
+            step(ev[k])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    sdm.stream_check(dev)
+    ms = dist.max(start.elapsed_time(end), dev)
+    scan_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    topk_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    if dist.rank == 0:
+        th = shape.B * shape.T * shape.H
+        algo = 3 * (shape.W + shape.R) * shape.d_v * 4 * th
+        achieved = algo / (scan_ms / 1e3) / 1e9
+        clk = clocks.summary()
+        mhz = clk["sm_max_mhz"] or 1965.0
+        peak = torch.cuda.get_device_properties(dev).multi_processor_count * SMEM_BYTES_PER_CLK_PER_SM * mhz / 1e3
+        cfg = workload_config(shape, args, dist)
+        cfg.update({"mode": "backward: recurrence (forward recomputed from M_0) and both selection-weight backwards",
+                    "l2": "inputs and outputs exceed L2"})
+        line = {"metric": "SDM backward tokens/s (B*T) on 1 B200", "impl": "sdm",
+                "value": aggregate_value(shape.B * shape.T * args.steps, dist.world, ms / 1e3), "unit": "tokens/s",
+                "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+                "stage_ms": {"scan_backward": scan_ms, "pkm_topk_backward_x2": topk_ms},
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic", "config": cfg,
+                "roofline": {"bound": "smem", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "kernel": "k_scan_backward",
+                             "algorithmic_bytes_per_launch": algo, "ms_per_launch": scan_ms,
+                             "peak_source": f"derived: SMs x {SMEM_BYTES_PER_CLK_PER_SM} B/clk x {mhz:.0f} MHz"},
+                "gpu_launches": 4 * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
 def run_slot_counts(args, dist: Dist):
     """Slot utilisation: each step counts, per (b, h), how often every slot is
     among the W write slots of the workload's T tokens (sdm_slot_counts on the
@@ -587,6 +673,9 @@ def main():
         return
     if args.slot_counts:
         run_slot_counts(args, dist)
+        return
+    if args.backward:
+        run_backward(args, dist)
         return
     run_sdm(args, dist)
 

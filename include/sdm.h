@@ -143,6 +143,56 @@ SDM_API int32_t sdm_scan_variant(const sdm_shape_t* shape);
  * invalid or unsupported shape (out left empty). For profiles and logs. */
 SDM_API sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_len);
 
+/* Bytes of workspace sdm_scan_backward needs for this shape (0 if the shape is
+ * invalid or the backward does not support it; sdm_last_error() says why). */
+SDM_API size_t sdm_scan_backward_workspace_bytes(const sdm_shape_t* shape);
+
+/* Backward of sdm_scan (no epilogue): the derivatives a training step needs
+ * ([explainer] 3.4 "高效训练" says that a memory-efficient backward exists; the
+ * derivatives follow from 3.1 steps 2-3 by the chain rule, for a fixed
+ * selection). For the loss L with dy = dL/dy and dM = dL/dM_T it computes,
+ * with a_i = alpha_t (1 - beta_t k_i), c_i = beta_t k_i, G = dL/dM_t:
+ *   dq_j     = <dy_t, M_t[j]>                        -> dw_r
+ *   dk_i     = beta_t (<G[i], v_t> - alpha_t <G[i], M_{t-1}[i]>)  -> dw_w
+ *   dv_t     = sum_i c_i G[i]
+ *   dalpha_t = sum_i (1 - beta_t k_i) <G[i], M_{t-1}[i]>
+ *   dbeta_t  = sum_i k_i (<G[i], v_t> - alpha_t <G[i], M_{t-1}[i]>)
+ *   dM       <- dL/dM_0 (in place)
+ * The state trajectory is recomputed from M_in (checkpoints every 128 tokens
+ * plus a log of overwritten rows, all in the workspace), bit-identical to the
+ * forward's. Requires an fp32 state (state_dtype SDM_F32) whose column tile
+ * and adjoint fit in shared memory (2 * N * 8 * 4 bytes <= 227 KB, or with
+ * 4-column tiles N <= about 7200); otherwise SDM_ERR_UNSUPPORTED.
+ *   idx_w, w_w, idx_r, w_r, v, alpha, beta: the forward's inputs (as sdm_scan)
+ *   M_in  fp32, the state the forward started from: [B,H,N,d_v], or [H,N,d_v]
+ *         shared by every batch row when m_in_shared != 0
+ *   dy    [B,T,H,d_v] fp32 (the derivative of the pre-epilogue y)
+ *   dM    [B,H,N,d_v] fp32, in: dL/dM_T (zeros if the final state is unused),
+ *         out: dL/dM_0 per batch row (sum over b for a shared M_0)
+ *   dv    [B,T,H,d_v] fp32; dalpha, dbeta [B,T,H] fp32; dw_w [B,T,H,W] fp32;
+ *   dw_r  [B,T,H,R] fp32 (all written, caller owned)
+ *   workspace: device scratch of sdm_scan_backward_workspace_bytes(shape).
+ * Results are deterministic. Slot indices outside [0, N) are skipped and set
+ * the device error word. */
+SDM_API sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w,
+                               const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
+                               const void* beta, const float* M_in, int32_t m_in_shared, const float* dy,
+                               float* dM, float* dv, float* dalpha, float* dbeta, float* dw_w, float* dw_r,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of the selection weights of sdm_pkm_topk for a fixed selection
+ * ([explainer] 3.1 step 1: w = softmax of the K selected sums
+ * sigma_k = s1[a_k] + s2[b_k], slot a_k * sqrt_n + b_k):
+ *   dsigma_k = w_k (dw_k - sum_j w_j dw_j);  dscores[a_k] += dsigma_k;
+ *   dscores[sqrt_n + b_k] += dsigma_k;  other entries 0.
+ *   idx, w, dw [B,T,H,K] (int32, fp32, fp32): the selection, its weights and
+ *              dL/dw;  dscores [B,T,H,2*sqrt_n] fp32 out (caller owned).
+ * Deterministic (fixed summation order). Indices outside [0, N) are skipped
+ * and set the device error word. */
+SDM_API sdm_status_t sdm_pkm_topk_backward(const int32_t* idx, const float* w, const float* dw, int32_t B,
+                                   int32_t T, int32_t H, int32_t sqrt_n, int32_t K, float* dscores,
+                                   void* stream);
+
 /* The sparse gated delta recurrence over a given selection, in token order
  * ([explainer] 3.1 steps 2-3; [summary] Core Mechanism 3-4). For each token t
  * and head: for every write slot i (distinct within a token),

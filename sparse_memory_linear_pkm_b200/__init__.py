@@ -20,7 +20,8 @@ import torch
 from . import native, synth
 from .native import SdmError
 
-__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "scan_describe", "stream_check", "make_shape",
+__all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "scan_describe",
+           "scan_backward", "pkm_topk_backward", "stream_check", "make_shape",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
 _DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
@@ -113,6 +114,58 @@ def scan(idx_w, w_w, idx_r, w_r, v, alpha, beta, M, g=None, eps: float = 1e-6, v
                               _ptr(alpha), _ptr(beta), _ptr(g), _ptr(M), _ptr(y), _ptr(ws),
                               ws.numel() * ws.element_size(), _stream(v.device)))
     return y
+
+
+def scan_backward_workspace_bytes(shape: native.Shape) -> int:
+    lib = native.load()
+    n = int(lib.sdm_scan_backward_workspace_bytes(ctypes.byref(shape)))
+    msg = lib.sdm_last_error().decode(errors="replace")
+    if n == 0 and msg:
+        raise native.SdmError(2, msg)
+    return n
+
+
+def scan_backward(idx_w, w_w, idx_r, w_r, v, alpha, beta, M_in, dy, dM: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None) -> dict:
+    """Derivatives of the recurrence (no epilogue) for dy = dL/dy and
+    dM = dL/dM_T (zeros when None). M_in is the fp32 state the forward started
+    from, [B,H,N,d_v] or [H,N,d_v] shared by the batch. Returns a dict with
+    dv, dalpha, dbeta, dw_w, dw_r (fp32) and dM0 = dL/dM_0 per batch row
+    [B,H,N,d_v] (``dM`` itself when given, updated in place)."""
+    B, T, H, W = idx_w.shape
+    R = idx_r.shape[-1]
+    d_v = v.shape[-1]
+    N = M_in.shape[-2]
+    sqrt_n = int(round(N ** 0.5))
+    shared = M_in.dim() == 3
+    dev = v.device
+    shape = native.Shape(B, T, H, sqrt_n, W, R, d_v, _code(v, "v"), _code(M_in, "M_in"), 1e-6, 0)
+    lib = native.load()
+    if dM is None:
+        dM = torch.zeros((B, H, N, d_v), dtype=torch.float32, device=dev)
+    out = {"dv": torch.empty((B, T, H, d_v), dtype=torch.float32, device=dev),
+           "dalpha": torch.empty((B, T, H), dtype=torch.float32, device=dev),
+           "dbeta": torch.empty((B, T, H), dtype=torch.float32, device=dev),
+           "dw_w": torch.empty((B, T, H, W), dtype=torch.float32, device=dev),
+           "dw_r": torch.empty((B, T, H, R), dtype=torch.float32, device=dev)}
+    ws = _workspace(scan_backward_workspace_bytes(shape), dev, workspace)
+    native.check(lib.sdm_scan_backward(ctypes.byref(shape), _ptr(idx_w), _ptr(w_w), _ptr(idx_r), _ptr(w_r), _ptr(v),
+                                       _ptr(alpha), _ptr(beta), _ptr(M_in), int(shared), _ptr(dy), _ptr(dM),
+                                       _ptr(out["dv"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]), _ptr(out["dw_w"]),
+                                       _ptr(out["dw_r"]), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev)))
+    out["dM0"] = dM
+    return out
+
+
+def pkm_topk_backward(idx: torch.Tensor, w: torch.Tensor, dw: torch.Tensor, sqrt_n: int,
+                      dscores: torch.Tensor | None = None) -> torch.Tensor:
+    """dL/dscores [B,T,H,2*sqrt_n] fp32 of the selection weights (fixed selection)."""
+    B, T, H, K = idx.shape
+    if dscores is None:
+        dscores = torch.empty((B, T, H, 2 * sqrt_n), dtype=torch.float32, device=idx.device)
+    native.check(native.load().sdm_pkm_topk_backward(_ptr(idx), _ptr(w), _ptr(dw), B, T, H, sqrt_n, K,
+                                                      _ptr(dscores), _stream(idx.device)))
+    return dscores
 
 
 def state_init(M0: torch.Tensor, B: int, out: torch.Tensor | None = None) -> torch.Tensor:

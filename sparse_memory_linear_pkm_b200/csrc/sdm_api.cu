@@ -20,6 +20,7 @@
 #include "sdm_misc.cuh"
 #include "sdm_records.cuh"
 #include "sdm_scan.cuh"
+#include "sdm_backward.cuh"
 
 namespace {
 
@@ -573,6 +574,59 @@ sdm_status_t noalloc_scratch(void** out) {
 
 }  // namespace
 
+// ------------------------------------------------------------- backward --
+
+namespace {
+
+constexpr size_t kBwdSmemLimit = 232448;  // sm_100 opt-in shared memory per block
+constexpr int kBwdChunk = 128;            // tokens per checkpoint chunk
+
+struct BwdChoice {
+  int CW = 8;
+  int C = kBwdChunk;
+  int ntile = 0;
+  size_t smem = 0;
+  size_t ckpt_bytes = 0, log_bytes = 0, part_bytes = 0;
+};
+
+sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
+  if (s.state_dtype != SDM_F32)
+    return fail(SDM_ERR_UNSUPPORTED, "sdm_scan_backward needs an fp32 state (state_dtype SDM_F32)");
+  const int64_t N = slots_of(s.sqrt_n);
+  const size_t meta = 2 * 2 * static_cast<size_t>(s.W + s.R) * 4;
+  for (int CW : {8, 4}) {
+    if (s.d_v % CW != 0) continue;
+    const size_t smem = 2 * static_cast<size_t>(N) * CW * 4 + meta;
+    if (smem > kBwdSmemLimit) continue;
+    BwdChoice c;
+    c.CW = CW;
+    c.C = std::max(1, std::min<int>(kBwdChunk, s.T));
+    c.ntile = s.d_v / CW;
+    c.smem = smem;
+    const int64_t tiles = static_cast<int64_t>(s.B) * s.H * c.ntile;
+    const int64_t nC = (static_cast<int64_t>(s.T) + c.C - 1) / c.C;
+    c.ckpt_bytes = align256(static_cast<size_t>(tiles) * std::max<int64_t>(0, nC - 1) * N * CW * 4);
+    c.log_bytes = align256(static_cast<size_t>(tiles) * c.C * s.W * CW * 4);
+    c.part_bytes = align256(static_cast<size_t>(s.B) * s.T * s.H * c.ntile * (s.W + s.R + 2) * 4);
+    *out = c;
+    return SDM_OK;
+  }
+  return fail(SDM_ERR_UNSUPPORTED,
+              "sdm_scan_backward keeps a column tile of the state and of its adjoint in shared memory; "
+              "N = " + std::to_string(N) + " rows do not fit (N <= 7200 with W, R <= 64)");
+}
+
+template <typename Tin, int CW>
+sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
+  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin, CW>);
+  set_smem(kern, c.smem);
+  const int64_t grid = static_cast<int64_t>(a.B) * a.H * c.ntile;
+  sdm::k_scan_backward<Tin, CW><<<static_cast<unsigned>(grid), 32, c.smem, st>>>(a);
+  return launch_status("backward launch");
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t sdm_abi_version(void) { return SDM_ABI_VERSION; }
@@ -663,6 +717,97 @@ int32_t sdm_scan_variant(const sdm_shape_t* shape) {
     return -1;
   ok();
   return c.resident ? SDM_VARIANT_RESIDENT : SDM_VARIANT_STREAMING;
+}
+
+
+size_t sdm_scan_backward_workspace_bytes(const sdm_shape_t* shape) {
+  const std::string saved = g_last_error;
+  BwdChoice c;
+  if (check_shape(shape) != SDM_OK || choose_bwd(*shape, &c) != SDM_OK) return 0;
+  g_last_error = saved;
+  return c.ckpt_bytes + c.log_bytes + c.part_bytes;
+}
+
+sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w,
+                               const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
+                               const void* beta, const float* M_in, int32_t m_in_shared, const float* dy, float* dM,
+                               float* dv, float* dalpha, float* dbeta, float* dw_w, float* dw_r, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  BwdChoice c;
+  if ((r = choose_bwd(s, &c)) != SDM_OK) return r;
+  const bool any = static_cast<int64_t>(s.B) * s.H > 0;
+  const bool tok = static_cast<int64_t>(s.B) * s.T * s.H > 0;
+  if ((r = need_ptr(idx_w, "idx_w", tok)) || (r = need_ptr(w_w, "w_w", tok)) || (r = need_ptr(idx_r, "idx_r", tok)) ||
+      (r = need_ptr(w_r, "w_r", tok)) || (r = need_ptr(v, "v", tok)) || (r = need_gate(alpha, "alpha", tok, s.in_dtype)) ||
+      (r = need_gate(beta, "beta", tok, s.in_dtype)) || (r = need_ptr(M_in, "M_in", any)) ||
+      (r = need_ptr(dy, "dy", tok)) || (r = need_ptr(dM, "dM", any)) || (r = need_ptr(dv, "dv", tok)) ||
+      (r = need_gate(dalpha, "dalpha", tok, SDM_F32)) || (r = need_gate(dbeta, "dbeta", tok, SDM_F32)) ||
+      (r = need_ptr(dw_w, "dw_w", tok)) || (r = need_ptr(dw_r, "dw_r", tok)))
+    return r;
+  if (!any) return ok();
+  const size_t need = c.ckpt_bytes + c.log_bytes + c.part_bytes;
+  if (workspace_bytes < need)
+    return fail(SDM_ERR_INVALID_ARGUMENT,
+                "workspace_bytes below sdm_scan_backward_workspace_bytes() = " + std::to_string(need));
+  if ((r = need_ptr(workspace, "workspace", need > 0)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  if (static_cast<size_t>(dev->max_smem_optin) < c.smem)
+    return fail(SDM_ERR_UNSUPPORTED, "the device's shared memory per block is below the backward tile's");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t N = slots_of(s.sqrt_n);
+  if (s.T == 0) return ok();  // dL/dM_0 = dL/dM_T, already in dM
+  sdm::BwdArgs a;
+  a.B = s.B; a.T = s.T; a.H = s.H; a.N = static_cast<int>(N); a.d_v = s.d_v; a.W = s.W; a.R = s.R;
+  a.C = c.C; a.ntile = c.ntile;
+  a.idx_w = idx_w; a.w_w = w_w; a.idx_r = idx_r; a.w_r = w_r;
+  a.v = v; a.alpha = alpha; a.beta = beta;
+  a.M_in = M_in;
+  a.M_in_b_stride = m_in_shared ? 0 : static_cast<int64_t>(s.H) * N * s.d_v;
+  a.dy = dy; a.dM = dM; a.dv = dv;
+  char* ws = static_cast<char*>(workspace);
+  a.part = reinterpret_cast<float*>(ws);
+  a.ckpt = reinterpret_cast<float*>(ws + c.part_bytes);
+  a.logbuf = reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes);
+  a.err = dev->err;
+  if (s.in_dtype == SDM_BF16)
+    r = c.CW == 8 ? launch_bwd_typed<sdm::bf16, 8>(c, a, st) : launch_bwd_typed<sdm::bf16, 4>(c, a, st);
+  else
+    r = c.CW == 8 ? launch_bwd_typed<float, 8>(c, a, st) : launch_bwd_typed<float, 4>(c, a, st);
+  if (r != SDM_OK) return r;
+  const int64_t n_th = static_cast<int64_t>(s.B) * s.T * s.H;
+  const int64_t total = n_th * (s.W + s.R + 2);
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8LL * dev->sms));
+  sdm::k_scan_backward_reduce<<<blocks, 256, 0, st>>>(a.part, n_th, s.W, s.R, c.ntile, dw_w, dw_r, dalpha, dbeta);
+  if ((r = launch_status("backward reduce launch")) != SDM_OK) return r;
+  return ok();
+}
+
+sdm_status_t sdm_pkm_topk_backward(const int32_t* idx, const float* w, const float* dw, int32_t B, int32_t T,
+                                   int32_t H, int32_t sqrt_n, int32_t K, float* dscores, void* stream) {
+  sdm_status_t r;
+  if (B < 0 || T < 0 || H < 0) return fail(SDM_ERR_INVALID_ARGUMENT, "B, T and H must be >= 0");
+  if (sqrt_n < 1 || sqrt_n > 1024) return fail(SDM_ERR_INVALID_ARGUMENT, "sqrt_n must be in [1, 1024]");
+  if ((r = check_k(K, sqrt_n, "K")) != SDM_OK) return r;
+  const int64_t units = static_cast<int64_t>(B) * T * H;
+  if ((r = need_ptr(idx, "idx", units > 0)) || (r = need_ptr(w, "w", units > 0)) ||
+      (r = need_ptr(dw, "dw", units > 0)) || (r = need_ptr(dscores, "dscores", units > 0)))
+    return r;
+  if (units == 0) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const int warps = 8;
+  const size_t smem = static_cast<size_t>(warps) * 3 * K * 4;
+  set_smem(reinterpret_cast<const void*>(sdm::k_pkm_topk_backward), smem);
+  const int64_t blocks = (units + warps - 1) / warps;
+  if (blocks > 0x7FFFFFFFLL) return fail(SDM_ERR_UNSUPPORTED, "too many token-heads for one launch");
+  sdm::k_pkm_topk_backward<<<static_cast<unsigned>(blocks), warps * 32, smem, static_cast<cudaStream_t>(stream)>>>(
+      idx, w, dw, units, sqrt_n, K, dscores, dev->err);
+  if ((r = launch_status("selection backward launch")) != SDM_OK) return r;
+  return ok();
 }
 
 sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_len) {

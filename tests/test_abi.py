@@ -108,3 +108,21 @@ def test_slot_count_arguments_without_gpu(lib):
     assert lib.sdm_slot_counts(ctypes.c_void_p(64), 1, 4, 1, 0, 64, ctypes.c_void_p(64), None) == 1
     assert b"K and N" in lib.sdm_last_error()
     assert lib.sdm_slot_counts(None, 1, 0, 1, 2, 64, ctypes.c_void_p(64), None) == 0
+
+
+def test_backward_workspace_and_support_without_gpu(lib):
+    # B=1, T=300, H=2, N=1024, W=R=64, d_v=128: 16 tiles of 8 columns per (b, h), 128-token chunks
+    s = shape(B=1, T=300, H=2, sqrt_n=32, W=64, R=64, d_v=128)
+    tiles = 1 * 2 * 16
+    ckpt = tiles * (3 - 1) * 1024 * 8 * 4
+    log = tiles * 128 * 64 * 8 * 4
+    part = (1 * 300 * 2 * 16 * (64 + 64 + 2) * 4 + 255) // 256 * 256
+    assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == ckpt + log + part
+    s = shape(B=1, T=300, H=2, sqrt_n=32, W=64, R=64, d_v=128, state_dtype=native.BF16)
+    assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == 0
+    assert b"fp32 state" in lib.sdm_last_error()
+    s = shape(B=1, T=4, H=1, sqrt_n=128, W=8, R=8, d_v=64)  # N = 16384 does not fit
+    assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == 0
+    assert b"shared memory" in lib.sdm_last_error()
+    assert lib.sdm_pkm_topk_backward(None, None, None, 1, 2, 1, 4, 3, None, None) == 1
+    assert lib.sdm_pkm_topk_backward(None, None, None, 0, 2, 1, 4, 3, None, None) == 0

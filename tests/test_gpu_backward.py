@@ -1,0 +1,151 @@
+"""Backward kernels against the oracle's derivatives, through the C ABI.
+
+sdm_scan_backward and sdm_pkm_topk_backward are compared element by element
+with oracle.scan_backward / oracle.pkm_topk_backward (double precision, pinned
+by finite differences) on the same seeded inputs. The GPU recomputes the
+forward in fp32, so the tolerance is the fp32-state forward's: 1e-4 * max|ref|.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from parity_helpers import TOL_F32_STATE, assert_rel_close, f32, scan_inputs
+from sparse_memory_linear_pkm_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+TOL_BWD = TOL_F32_STATE
+# softmax derivative: fp32 products and one fp32 sum of K terms per token-head
+TOL_TOPK_BWD = 1e-5
+
+BWD = [
+    # sqrt_n, d_v, W, R, in, T, B, H, M_in shared by the batch
+    (32, 128, 64, 64, "bf16", 300, 2, 2, False),  # three checkpoint chunks and a ragged tail
+    (8, 32, 5, 3, "f32", 41, 2, 1, True),
+    (64, 64, 16, 16, "bf16", 150, 1, 2, False),  # N = 4096: 4-column tiles
+    (4, 16, 16, 16, "f32", 129, 1, 1, False),  # W = N: every slot written every token
+    (16, 48, 12, 4, "f32", 1, 1, 3, True),  # one token
+    (32, 16, 8, 8, "f32", 256, 1, 2, False),  # T a multiple of the chunk
+]
+
+
+def _bwd_inputs(case, seed):
+    sqrt_n, d_v, W, R, tin, T, B, H, shared = case
+    shape = synth.Shape("t", B=B, T=T, H=H, sqrt_n=sqrt_n, d_v=d_v, W=W, R=R, in_dtype=tin, state_dtype="f32")
+    inp = scan_inputs(shape, seed=seed)
+    gen = torch.Generator().manual_seed(seed + 1)
+    M0 = inp["M"][0]
+    if shared:
+        M_in = M0.clone()
+        M_full = torch.stack([M0] * B)
+    else:
+        M_full = (inp["M"] + 0.05 * torch.randn(inp["M"].shape, generator=gen)).contiguous()
+        M_in = M_full
+    dy = torch.randn((B, T, H, d_v), generator=gen)
+    dM_T = 0.3 * torch.randn((B, H, shape.N, d_v), generator=gen)
+    return shape, inp, M_in, M_full, dy, dM_T
+
+
+def _gpu_backward(sdm, dev, inp, M_in, dy, dM_T):
+    d = {k: v.to(dev) for k, v in inp.items() if k != "M"}
+    out = sdm.scan_backward(d["idx_w"], d["w_w"], d["idx_r"], d["w_r"], d["v"], d["alpha"], d["beta"], M_in.to(dev),
+                            dy.to(dev), dM_T.to(dev).clone())
+    sdm.stream_check()
+    return out
+
+
+def _oracle_backward(oracle, inp, M_full, dy, dM_T):
+    return oracle.scan_backward(inp["idx_w"].numpy(), inp["w_w"].numpy().astype(np.float64), inp["idx_r"].numpy(),
+                                inp["w_r"].numpy().astype(np.float64), f32(inp["v"]), f32(inp["alpha"]),
+                                f32(inp["beta"]), f32(M_full), f32(dy), f32(dM_T))
+
+
+@pytest.mark.parametrize("case", BWD, ids=lambda c: "-".join(map(str, c)))
+def test_scan_backward_matches_oracle(sdm, oracle, cuda_device, case):
+    shape, inp, M_in, M_full, dy, dM_T = _bwd_inputs(case, seed=sum(case[:4]) + case[5])
+    got = _gpu_backward(sdm, cuda_device, inp, M_in, dy, dM_T)
+    want = _oracle_backward(oracle, inp, M_full, dy, dM_T)
+    for k in ("dv", "dalpha", "dbeta", "dw_w", "dw_r", "dM0"):
+        assert_rel_close(got[k].cpu().numpy(), want[k], TOL_BWD, k)
+
+
+def test_scan_backward_deterministic(sdm, cuda_device):
+    case = (32, 64, 16, 16, "bf16", 200, 2, 2, False)
+    _, inp, M_in, _, dy, dM_T = _bwd_inputs(case, seed=11)
+    a = _gpu_backward(sdm, cuda_device, inp, M_in, dy, dM_T)
+    b = _gpu_backward(sdm, cuda_device, inp, M_in, dy, dM_T)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_scan_backward_rejects_bf16_state_and_large_n(sdm, cuda_device):
+    sh = sdm.make_shape(1, 4, 1, 32, 8, 8, 64, torch.float32, torch.bfloat16)
+    with pytest.raises(sdm.SdmError, match="fp32 state"):
+        sdm.scan_backward_workspace_bytes(sh)
+    sh = sdm.make_shape(1, 4, 1, 128, 8, 8, 64, torch.float32, torch.float32)  # N = 16384
+    with pytest.raises(sdm.SdmError, match="shared memory"):
+        sdm.scan_backward_workspace_bytes(sh)
+
+
+def test_scan_backward_out_of_range_flagged(sdm, cuda_device):
+    case = (8, 32, 4, 4, "f32", 9, 1, 1, False)
+    _, inp, M_in, _, dy, dM_T = _bwd_inputs(case, seed=2)
+    inp["idx_w"][0, 3, 0, 1] = 64  # N = 64
+    inp["idx_r"][0, 5, 0, 2] = -3
+    d = {k: v.to(cuda_device) for k, v in inp.items() if k != "M"}
+    out = sdm.scan_backward(d["idx_w"], d["w_w"], d["idx_r"], d["w_r"], d["v"], d["alpha"], d["beta"],
+                            M_in.to(cuda_device), dy.to(cuda_device), dM_T.to(cuda_device).clone())
+    with pytest.raises(sdm.SdmError, match="DEVICE_FAULT"):
+        sdm.stream_check()
+    assert all(torch.isfinite(t).all() for t in out.values())
+
+
+@pytest.mark.parametrize("sqrt_n,K", [(32, 64), (8, 5), (128, 64), (4, 16), (1, 1), (16, 256)])
+def test_pkm_topk_backward_matches_oracle(sdm, oracle, cuda_device, sqrt_n, K):
+    B, T, H = 2, 37, 3
+    g = torch.Generator().manual_seed(sqrt_n + K)
+    x = torch.randn((B, T, H, 2 * sqrt_n), generator=g)
+    idx, w = oracle.pkm_topk(f32(x), K)
+    dw = torch.randn((B, T, H, K), generator=g)
+    w32 = torch.from_numpy(w.astype(np.float32))
+    got = sdm.pkm_topk_backward(torch.from_numpy(idx).to(cuda_device), w32.to(cuda_device), dw.to(cuda_device),
+                                sqrt_n)
+    sdm.stream_check()
+    want = oracle.pkm_topk_backward(idx, w32.numpy().astype(np.float64), f32(dw), sqrt_n)
+    assert_rel_close(got.cpu().numpy(), want, TOL_TOPK_BWD, "dscores")
+
+
+def test_scan_backward_full_size_sampled(sdm, oracle, cuda_device):
+    """The bench workload d2048_h16_n1024_dv128 at full size, in the launch
+    configuration the benchmark times, with a seeded synthetic selection; two
+    sampled (b, h) pairs compared with the oracle over the whole sequence."""
+    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"]
+    inp = synth.make_inputs(shape, seed=0, device=cuda_device)
+    gen = torch.Generator().manual_seed(3)
+
+    def selection(K):  # distinct slots (a + k s) mod N with s odd (N a power of two), positive weights
+        lead = (shape.B, shape.T, shape.H, 1)
+        a = torch.randint(0, shape.N, lead, generator=gen)
+        st = 2 * torch.randint(0, shape.N // 2, lead, generator=gen) + 1
+        idx = ((a + torch.arange(K) * st) % shape.N).to(torch.int32).contiguous()
+        w = torch.rand(lead[:3] + (K,), generator=gen) + 0.05
+        return idx, (w / w.sum(-1, keepdim=True)).contiguous()
+
+    idx_w, w_w = selection(shape.W)
+    idx_r, w_r = selection(shape.R)
+    dy = torch.randn((shape.B, shape.T, shape.H, shape.d_v), generator=gen)
+    dev = cuda_device
+    M0 = inp["M0"].float()
+    out = sdm.scan_backward(idx_w.to(dev), w_w.to(dev), idx_r.to(dev), w_r.to(dev), inp["v"], inp["alpha"],
+                            inp["beta"], M0, dy.to(dev))
+    sdm.stream_check()
+    for b, h in ((0, 0), (shape.B - 1, shape.H - 1)):
+        s = lambda t: t[b:b + 1, :, h:h + 1].contiguous()
+        want = oracle.scan_backward(s(idx_w).numpy(), s(w_w).numpy().astype(np.float64), s(idx_r).numpy(),
+                                    s(w_r).numpy().astype(np.float64), f32(s(inp["v"])), f32(s(inp["alpha"])),
+                                    f32(s(inp["beta"])), f32(M0[h:h + 1].unsqueeze(0)), f32(s(dy)),
+                                    np.zeros((1, 1, shape.N, shape.d_v)))
+        for k in ("dv", "dalpha", "dbeta", "dw_w", "dw_r"):
+            assert_rel_close(s(out[k]).cpu().numpy(), want[k], TOL_BWD, f"{k} (b={b}, h={h})")
+        assert_rel_close(out["dM0"][b:b + 1, h:h + 1].cpu().numpy(), want["dM0"], TOL_BWD, f"dM0 (b={b}, h={h})")
