@@ -582,46 +582,45 @@ constexpr size_t kBwdSmemLimit = 232448;  // sm_100 opt-in shared memory per blo
 constexpr int kBwdChunk = 128;            // tokens per checkpoint chunk
 
 struct BwdChoice {
-  int CW = 8;
   int C = kBwdChunk;
   int ntile = 0;
   size_t smem = 0;
-  size_t ckpt_bytes = 0, log_bytes = 0, part_bytes = 0;
+  size_t rec_bytes = 0, ckpt_bytes = 0, log_bytes = 0, part_bytes = 0;
+  size_t total() const { return rec_bytes + ckpt_bytes + log_bytes + part_bytes; }
 };
 
 sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
   if (s.state_dtype != SDM_F32)
     return fail(SDM_ERR_UNSUPPORTED, "sdm_scan_backward needs an fp32 state (state_dtype SDM_F32)");
   const int64_t N = slots_of(s.sqrt_n);
-  const size_t meta = 2 * 2 * static_cast<size_t>(s.W + s.R) * 4;
-  for (int CW : {8, 4}) {
-    if (s.d_v % CW != 0) continue;
-    const size_t smem = 2 * static_cast<size_t>(N) * CW * 4 + meta;
-    if (smem > kBwdSmemLimit) continue;
-    BwdChoice c;
-    c.CW = CW;
-    c.C = std::max(1, std::min<int>(kBwdChunk, s.T));
-    c.ntile = s.d_v / CW;
-    c.smem = smem;
-    const int64_t tiles = static_cast<int64_t>(s.B) * s.H * c.ntile;
-    const int64_t nC = (static_cast<int64_t>(s.T) + c.C - 1) / c.C;
-    c.ckpt_bytes = align256(static_cast<size_t>(tiles) * std::max<int64_t>(0, nC - 1) * N * CW * 4);
-    c.log_bytes = align256(static_cast<size_t>(tiles) * c.C * s.W * CW * 4);
-    c.part_bytes = align256(static_cast<size_t>(s.B) * s.T * s.H * c.ntile * (s.W + s.R + 2) * 4);
-    *out = c;
-    return SDM_OK;
-  }
-  return fail(SDM_ERR_UNSUPPORTED,
-              "sdm_scan_backward keeps a column tile of the state and of its adjoint in shared memory; "
-              "N = " + std::to_string(N) + " rows do not fit (N <= 7200 with W, R <= 64)");
+  const sdm::RecLayout rl = rec_layout(s.W, s.R, false);
+  constexpr int CW = sdm::kBwdCols;
+  const size_t ring = static_cast<size_t>(sdm::kBwdStages) * sdm::bwd_stage(s.W, rl.words).words * 4;
+  const size_t smem = 2 * static_cast<size_t>(N) * CW * 4 + ring;
+  if (smem > kBwdSmemLimit)
+    return fail(SDM_ERR_UNSUPPORTED,
+                "sdm_scan_backward keeps a 4-column tile of the state and of its adjoint in shared memory; "
+                "N = " + std::to_string(N) + " rows do not fit (N <= about 6900 with W, R <= 64)");
+  BwdChoice c;
+  c.C = std::max(1, std::min<int>(kBwdChunk, s.T));
+  c.ntile = s.d_v / CW;
+  c.smem = smem;
+  const int64_t tiles = static_cast<int64_t>(s.B) * s.H * c.ntile;
+  const int64_t nC = (static_cast<int64_t>(s.T) + c.C - 1) / c.C;
+  c.ckpt_bytes = align256(static_cast<size_t>(tiles) * std::max<int64_t>(0, nC - 1) * N * CW * 4);
+  c.log_bytes = align256(static_cast<size_t>(tiles) * c.C * s.W * CW * 4);
+  c.part_bytes = align256(static_cast<size_t>(s.B) * s.T * s.H * c.ntile * (s.W + s.R + 2) * 4);
+  c.rec_bytes = align256(static_cast<size_t>(s.B) * s.H * s.T * rl.words * 4);
+  *out = c;
+  return SDM_OK;
 }
 
-template <typename Tin, int CW>
+template <typename Tin>
 sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
-  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin, CW>);
+  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin>);
   set_smem(kern, c.smem);
   const int64_t grid = static_cast<int64_t>(a.B) * a.H * c.ntile;
-  sdm::k_scan_backward<Tin, CW><<<static_cast<unsigned>(grid), 32, c.smem, st>>>(a);
+  sdm::k_scan_backward<Tin><<<static_cast<unsigned>(grid), 32, c.smem, st>>>(a);
   return launch_status("backward launch");
 }
 
@@ -725,7 +724,7 @@ size_t sdm_scan_backward_workspace_bytes(const sdm_shape_t* shape) {
   BwdChoice c;
   if (check_shape(shape) != SDM_OK || choose_bwd(*shape, &c) != SDM_OK) return 0;
   g_last_error = saved;
-  return c.ckpt_bytes + c.log_bytes + c.part_bytes;
+  return c.total();
 }
 
 sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w,
@@ -748,7 +747,7 @@ sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, c
       (r = need_ptr(dw_w, "dw_w", tok)) || (r = need_ptr(dw_r, "dw_r", tok)))
     return r;
   if (!any) return ok();
-  const size_t need = c.ckpt_bytes + c.log_bytes + c.part_bytes;
+  const size_t need = c.total();
   if (workspace_bytes < need)
     return fail(SDM_ERR_INVALID_ARGUMENT,
                 "workspace_bytes below sdm_scan_backward_workspace_bytes() = " + std::to_string(need));
@@ -763,8 +762,8 @@ sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, c
   sdm::BwdArgs a;
   a.B = s.B; a.T = s.T; a.H = s.H; a.N = static_cast<int>(N); a.d_v = s.d_v; a.W = s.W; a.R = s.R;
   a.C = c.C; a.ntile = c.ntile;
-  a.idx_w = idx_w; a.w_w = w_w; a.idx_r = idx_r; a.w_r = w_r;
-  a.v = v; a.alpha = alpha; a.beta = beta;
+  a.rl = rec_layout(s.W, s.R, false);
+  a.v = v;
   a.M_in = M_in;
   a.M_in_b_stride = m_in_shared ? 0 : static_cast<int64_t>(s.H) * N * s.d_v;
   a.dy = dy; a.dM = dM; a.dv = dv;
@@ -772,11 +771,18 @@ sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, c
   a.part = reinterpret_cast<float*>(ws);
   a.ckpt = reinterpret_cast<float*>(ws + c.part_bytes);
   a.logbuf = reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes);
+  uint32_t* rec = reinterpret_cast<uint32_t*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes);
+  a.rec = rec;
   a.err = dev->err;
-  if (s.in_dtype == SDM_BF16)
-    r = c.CW == 8 ? launch_bwd_typed<sdm::bf16, 8>(c, a, st) : launch_bwd_typed<sdm::bf16, 4>(c, a, st);
-  else
-    r = c.CW == 8 ? launch_bwd_typed<float, 8>(c, a, st) : launch_bwd_typed<float, 4>(c, a, st);
+  if (s.in_dtype == SDM_BF16) {
+    if ((r = launch_records<sdm::bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
+      return r;
+    r = launch_bwd_typed<sdm::bf16>(c, a, st);
+  } else {
+    if ((r = launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
+      return r;
+    r = launch_bwd_typed<float>(c, a, st);
+  }
   if (r != SDM_OK) return r;
   const int64_t n_th = static_cast<int64_t>(s.B) * s.T * s.H;
   const int64_t total = n_th * (s.W + s.R + 2);

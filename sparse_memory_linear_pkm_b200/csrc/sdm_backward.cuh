@@ -16,7 +16,7 @@
 //
 // with G = dL/dM running backwards over the tokens from dL/dM_T, the read of a
 // token before its write. Every column of d_v is independent given the
-// per-token scalars, so one warp carries one CW-column tile of one (b, h) with
+// per-token scalars, so one warp carries one 4-column tile of one (b, h) with
 // its state M and adjoint G resident in shared memory. Memory-efficient by
 // recomputation: a first forward pass stores the tile every C tokens
 // (checkpoints); then, chunk by chunk from the end, the warp reloads the
@@ -31,251 +31,281 @@
 #pragma once
 
 #include "sdm_device.cuh"
+#include "sdm_records.cuh"
 
 namespace sdm {
 
 struct BwdArgs {
   int B, T, H, N, d_v, W, R;
   int C;      // tokens per checkpoint chunk
-  int ntile;  // d_v / CW
-  const int32_t* idx_w;
-  const float* w_w;
-  const int32_t* idx_r;
-  const float* w_r;
-  const void* v;      // [B, T, H, d_v] Tin
-  const void* alpha;  // [B, T, H] Tin
-  const void* beta;   // [B, T, H] Tin
+  int ntile;  // d_v / 4
+  RecLayout rl;
+  const uint32_t* rec;  // [B, H, T, rl.words] per-token records (slots, weights, alpha, beta; no hazard plan)
+  const void* v;        // [B, T, H, d_v] Tin
   const float* M_in;  // rows of (b, h) at M_in + b * M_in_b_stride + h * N * d_v
   int64_t M_in_b_stride;
   const float* dy;  // [B, T, H, d_v]
   float* dM;        // [B, H, N, d_v] in: dL/dM_T, out: dL/dM_0
   float* dv;        // [B, T, H, d_v]
   float* part;      // [B, T, H, ntile, W + R + 2] per-tile partial sums
-  float* ckpt;      // per tile: (ceil(T / C) - 1) * N * CW
-  float* logbuf;    // per tile: C * W * CW
+  float* ckpt;      // per tile: (ceil(T / C) - 1) * N * 4
+  float* logbuf;    // per tile: C * W * 4
   unsigned* err;
 };
 
-// 4-byte global -> shared asynchronous copy (generic proxy).
-__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+// 8-byte global -> shared asynchronous copy (generic proxy); both addresses
+// 8-byte aligned.
+__device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
                : "memory");
 }
 
-// Per-token selection metadata staged in shared memory:
-// idx_w[W] | w_w[W] | idx_r[R] | w_r[R] (32-bit words).
-__device__ __forceinline__ void stage_token_meta(const BwdArgs& a, int64_t th, int32_t* buf, int lane) {
-  for (int x = lane; x < a.W; x += kWarp) {
-    cp_async4(buf + x, a.idx_w + th * a.W + x);
-    cp_async4(buf + a.W + x, a.w_w + th * a.W + x);
-  }
-  int32_t* r = buf + 2 * a.W;
-  for (int x = lane; x < a.R; x += kWarp) {
-    cp_async4(r + x, a.idx_r + th * a.R + x);
-    cp_async4(r + a.R + x, a.w_r + th * a.R + x);
-  }
-  cp_async_commit();
+// Tile geometry: a warp owns kBwdCols = 4 columns of one (b, h); lane l
+// handles entry e0 + l of a token (32 entries per warp instruction) and its 4
+// columns as one float4, so the sums over the tile's columns stay inside the
+// lane. State and adjoint rows are 16 bytes in shared memory.
+constexpr int kBwdCols = 4;
+
+// Staging: per token, a ring stage in shared memory holds
+//   log  [W][4] f32     the values its W writes overwrote (reverse sweep only)
+//   rec  [rl.words]     its record: slots, weights, alpha, beta
+//   v    [4] Tin        this tile's columns of v_t (padded to 16 bytes)
+//   dy   [4] f32        this tile's columns of dy_t (reverse sweep only)
+// filled by cp.async kBwdStages - 1 tokens ahead of use, so the token loop
+// itself issues no global loads.
+constexpr int kBwdStages = 3;
+
+struct BwdStage {
+  int log, rec, v, dy, words;  // word offsets and the stage size (all multiples of 4)
+};
+__host__ __device__ inline BwdStage bwd_stage(int W, int rec_words) {
+  BwdStage st;
+  st.log = 0;
+  st.rec = W * kBwdCols;
+  st.v = st.rec + rec_words;
+  st.dy = st.v + 4;
+  st.words = st.dy + 4;
+  return st;
 }
 
-// Per-lane token scalars: alpha, beta and this lane's column of v and dy.
+// Per-token view of a filled stage.
 struct BwdTok {
-  float alpha, beta, v, dy;
+  const float4* log;
+  const uint32_t* rec;
+  float alpha, beta;
+  float4 v, dy;
 };
 
-template <typename Tin>
-__device__ __forceinline__ BwdTok load_token(const BwdArgs& a, int64_t th, int col, bool with_dy) {
-  BwdTok k;
-  k.alpha = to_f32<Tin>(static_cast<const Tin*>(a.alpha)[th]);
-  k.beta = to_f32<Tin>(static_cast<const Tin*>(a.beta)[th]);
-  k.v = to_f32<Tin>(static_cast<const Tin*>(a.v)[th * a.d_v + col]);
-  k.dy = with_dy ? a.dy[th * a.d_v + col] : 0.0f;
-  return k;
+__device__ __forceinline__ float dot4(const float4& a, const float4& b) {
+  return __fmaf_rn(a.w, b.w, __fmaf_rn(a.z, b.z, __fmaf_rn(a.y, b.y, a.x * b.x)));
+}
+
+// Runs body(t, token) over n tokens t = t_first + i * step of one (b, h) and
+// column tile, each with its stage filled (log rows from log_src when given,
+// dy when with_dy).
+template <typename Tin, class Body>
+__device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, int tile, int lane, int t_first,
+                                               int step, int n, float* ring, const float* log_src, int log_t0,
+                                               bool with_dy, Body body) {
+  const BwdStage L = bwd_stage(a.W, a.rl.words);
+  const int n_log = log_src != nullptr ? a.W : 0;  // 16-byte pieces: one row each
+  const int n_rec = a.rl.words / 4;
+  const int n_all = n_log + n_rec + 1 + (with_dy ? 1 : 0);
+  const int bh = b * a.H + h;
+  auto issue = [&](int i) {
+    if (i < n) {
+      const int t = t_first + i * step;
+      const int64_t th = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
+      float* st = ring + (i % kBwdStages) * L.words;
+      const float* lsrc = log_src != nullptr ? log_src + static_cast<int64_t>(t - log_t0) * a.W * kBwdCols : nullptr;
+      const uint32_t* rsrc = a.rec + (static_cast<int64_t>(bh) * a.T + t) * a.rl.words;
+      for (int x = lane; x < n_all; x += kWarp) {
+        if (x < n_log) {
+          cp_async16(st + L.log + 4 * x, lsrc + 4 * x);
+        } else if (x < n_log + n_rec) {
+          const int j = x - n_log;
+          cp_async16(st + L.rec + 4 * j, rsrc + 4 * j);
+        } else if (x == n_log + n_rec) {
+          const Tin* vsrc = static_cast<const Tin*>(a.v) + th * a.d_v + tile * kBwdCols;
+          if constexpr (sizeof(Tin) == 4) cp_async16(st + L.v, vsrc);
+          else cp_async8(st + L.v, vsrc);
+        } else {
+          cp_async16(st + L.dy, a.dy + th * a.d_v + tile * kBwdCols);
+        }
+      }
+    }
+    cp_async_commit();  // empty groups past the end keep the count uniform
+  };
+#pragma unroll
+  for (int i = 0; i < kBwdStages - 1; ++i) issue(i);
+  for (int i = 0; i < n; ++i) {
+    issue(i + kBwdStages - 1);
+    cp_async_wait<kBwdStages - 1>();
+    __syncwarp();
+    const float* st = ring + (i % kBwdStages) * L.words;
+    BwdTok k;
+    k.log = reinterpret_cast<const float4*>(st + L.log);
+    k.rec = reinterpret_cast<const uint32_t*>(st + L.rec);
+    k.alpha = __uint_as_float(k.rec[a.rl.off_ab]);
+    k.beta = __uint_as_float(k.rec[a.rl.off_ab + 1]);
+    const Tin* vv = reinterpret_cast<const Tin*>(st + L.v);
+    k.v = make_float4(to_f32<Tin>(vv[0]), to_f32<Tin>(vv[1]), to_f32<Tin>(vv[2]), to_f32<Tin>(vv[3]));
+    k.dy = with_dy ? *reinterpret_cast<const float4*>(st + L.dy) : make_float4(0.f, 0.f, 0.f, 0.f);
+    body(t_first + i * step, k);
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  __syncwarp();
 }
 
 // The forward write of one token on the tile (the forward kernels' exact fp32
-// operations). With `log`, the overwritten values are kept at log[e * CW + c].
-template <int CW>
-__device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const int32_t* meta, const BwdTok& k, float* Ms,
-                                                  float* log, int e4, int c) {
-  constexpr int EPG = kWarp / CW;
-  const float* ww = reinterpret_cast<const float*>(meta + a.W);
-  for (int e0 = 0; e0 < a.W; e0 += EPG) {
-    const int e = e0 + e4;
-    if (e < a.W) {
-      const int s = meta[e];
-      if (static_cast<unsigned>(s) < static_cast<unsigned>(a.N)) {
-        const float cw = k.beta * ww[e];
-        const float aw = k.alpha * (1.0f - cw);
-        const float m = Ms[s * CW + c];
-        if (log != nullptr) log[e * CW + c] = m;
-        Ms[s * CW + c] = __fmaf_rn(aw, m, __fmul_rn(cw, k.v));
-      }
-    }
+// operations: m <- fma(alpha (1 - beta k), m, (beta k) v)). With `log`, the
+// overwritten rows are kept at log[e].
+__device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok& k, float4* Ms, float4* log,
+                                                  int lane) {
+  const int32_t* slot = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_w);
+  const float* ww = reinterpret_cast<const float*>(k.rec + a.rl.off_k_w);
+  for (int e = lane; e < a.W; e += kWarp) {
+    const int s = slot[e];
+    if (s < 0) continue;
+    const float cw = k.beta * ww[e];
+    const float aw = k.alpha * (1.0f - cw);
+    const float4 m = Ms[s];
+    if (log != nullptr) log[e] = m;
+    Ms[s] = make_float4(__fmaf_rn(aw, m.x, __fmul_rn(cw, k.v.x)), __fmaf_rn(aw, m.y, __fmul_rn(cw, k.v.y)),
+                        __fmaf_rn(aw, m.z, __fmul_rn(cw, k.v.z)), __fmaf_rn(aw, m.w, __fmul_rn(cw, k.v.w)));
   }
 }
 
-template <typename Tin, int CW>
+template <typename Tin>
 __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
-  constexpr int EPG = kWarp / CW;
   extern __shared__ __align__(16) float bsm[];
   const int N = a.N;
-  float* Ms = bsm;                                         // [N][CW] state tile
-  float* Gs = bsm + static_cast<size_t>(N) * CW;           // [N][CW] adjoint tile
-  int32_t* meta0 = reinterpret_cast<int32_t*>(Gs + static_cast<size_t>(N) * CW);
-  const int meta_words = 2 * (a.W + a.R);
-  auto metab = [&](int i) { return meta0 + i * meta_words; };  // two staging buffers
+  float4* Ms = reinterpret_cast<float4*>(bsm);  // [N] state rows of the tile
+  float4* Gs = Ms + N;                          // [N] adjoint rows
+  float* ring = reinterpret_cast<float*>(Gs + N);
 
   const int lane = threadIdx.x;
-  const int e4 = lane / CW, c = lane % CW;
   const int tile = blockIdx.x % a.ntile;
   const int bh = blockIdx.x / a.ntile;
   const int b = bh / a.H, h = bh % a.H;
-  const int col = tile * CW + c;
+  const int col0 = tile * kBwdCols;
   const int64_t tile_id = blockIdx.x;
   const int nC = (a.T + a.C - 1) / a.C;
-  float* ckpt = a.ckpt + tile_id * static_cast<int64_t>(nC > 1 ? nC - 1 : 0) * N * CW;
-  float* logb = a.logbuf + tile_id * static_cast<int64_t>(a.C) * a.W * CW;
-  const float* Min = a.M_in + b * a.M_in_b_stride + static_cast<int64_t>(h) * N * a.d_v;
-  auto th_of = [&](int t) { return (static_cast<int64_t>(b) * a.T + t) * a.H + h; };
+  float4* ckpt = reinterpret_cast<float4*>(a.ckpt) + tile_id * static_cast<int64_t>(nC > 1 ? nC - 1 : 0) * N;
+  float4* logb = reinterpret_cast<float4*>(a.logbuf) + tile_id * static_cast<int64_t>(a.C) * a.W;
+  const float* Min = a.M_in + b * a.M_in_b_stride + static_cast<int64_t>(h) * N * a.d_v + col0;
+  auto load_min = [&]() {
+    for (int row = lane; row < N; row += kWarp)
+      Ms[row] = *reinterpret_cast<const float4*>(Min + static_cast<int64_t>(row) * a.d_v);
+  };
 
   // --------------------------------------------- pass 1: checkpoints --
-  for (int row = e4; row < N; row += EPG) Ms[row * CW + c] = Min[static_cast<int64_t>(row) * a.d_v + col];
+  load_min();
   __syncwarp();
-  if (a.T > 0) stage_token_meta(a, th_of(0), metab(0), lane);
-  BwdTok nxt = a.T > 0 ? load_token<Tin>(a, th_of(0), col, false) : BwdTok{};
-  for (int t = 0; t < a.T; ++t) {
+  bwd_token_pass<Tin>(a, b, h, tile, lane, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
     if (t > 0 && t % a.C == 0) {
-      float* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N * CW;
-      for (int row = e4; row < N; row += EPG) dst[row * CW + c] = Ms[row * CW + c];
+      float4* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N;
+      for (int row = lane; row < N; row += kWarp) dst[row] = Ms[row];
     }
-    const BwdTok cur = nxt;
-    if (t + 1 < a.T) {
-      stage_token_meta(a, th_of(t + 1), metab((t + 1) & 1), lane);
-      nxt = load_token<Tin>(a, th_of(t + 1), col, false);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncwarp();
-    const int32_t* meta = metab(t & 1);
-    if (c == 0) {  // out-of-range slots are skipped everywhere and flagged here, once
-      for (int e = e4; e < a.W; e += EPG)
-        if (static_cast<unsigned>(meta[e]) >= static_cast<unsigned>(N)) atomicOr(a.err, kErrIndexOutOfRange);
-      for (int e = e4; e < a.R; e += EPG)
-        if (static_cast<unsigned>(meta[2 * a.W + e]) >= static_cast<unsigned>(N)) atomicOr(a.err, kErrIndexOutOfRange);
-    }
-    bwd_forward_token<CW>(a, meta, cur, Ms, nullptr, e4, c);
-    __syncwarp();
-  }
+    bwd_forward_token(a, k, Ms, nullptr, lane);
+  });
 
   // ---------------------------------- pass 2: chunks from the end --
-  float* Gout = a.dM + (static_cast<int64_t>(b) * a.H + h) * N * a.d_v;
-  for (int row = e4; row < N; row += EPG) Gs[row * CW + c] = Gout[static_cast<int64_t>(row) * a.d_v + col];
+  float* Gout = a.dM + (static_cast<int64_t>(b) * a.H + h) * N * a.d_v + col0;
+  for (int row = lane; row < N; row += kWarp)
+    Gs[row] = *reinterpret_cast<const float4*>(Gout + static_cast<int64_t>(row) * a.d_v);
   const int PW = a.W + a.R + 2;
   for (int kc = nC - 1; kc >= 0; --kc) {
     const int t0 = kc * a.C, t1 = min(a.T, t0 + a.C);
     // State at the chunk start.
-    __syncwarp();
     if (kc == 0) {
-      for (int row = e4; row < N; row += EPG) Ms[row * CW + c] = Min[static_cast<int64_t>(row) * a.d_v + col];
+      load_min();
     } else {
-      const float* src = ckpt + static_cast<int64_t>(kc - 1) * N * CW;
-      for (int row = e4; row < N; row += EPG) Ms[row * CW + c] = src[row * CW + c];
+      const float4* src = ckpt + static_cast<int64_t>(kc - 1) * N;
+      for (int row = lane; row < N; row += kWarp) Ms[row] = src[row];
     }
     __syncwarp();
-    // Recompute the chunk forward, logging overwritten values.
-    stage_token_meta(a, th_of(t0), metab(0), lane);
-    nxt = load_token<Tin>(a, th_of(t0), col, false);
-    for (int t = t0; t < t1; ++t) {
-      const BwdTok cur = nxt;
-      if (t + 1 < t1) {
-        stage_token_meta(a, th_of(t + 1), metab((t + 1 - t0) & 1), lane);
-        nxt = load_token<Tin>(a, th_of(t + 1), col, false);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncwarp();
-      bwd_forward_token<CW>(a, metab((t - t0) & 1), cur, Ms, logb + static_cast<int64_t>(t - t0) * a.W * CW, e4,
-                            c);
-      __syncwarp();
-    }
+    // Recompute the chunk forward, logging overwritten rows.
+    bwd_token_pass<Tin>(a, b, h, tile, lane, t0, 1, t1 - t0, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
+      bwd_forward_token(a, k, Ms, logb + static_cast<int64_t>(t - t0) * a.W, lane);
+    });
+    // The log rows were written by other lanes; the reverse pass reads them
+    // back through cp.async.
+    __threadfence_block();
+    __syncwarp();
     // Backward sweep over the chunk.
-    stage_token_meta(a, th_of(t1 - 1), metab(0), lane);
-    nxt = load_token<Tin>(a, th_of(t1 - 1), col, true);
-    for (int t = t1 - 1; t >= t0; --t) {
-      const int64_t th = th_of(t);
-      const BwdTok k = nxt;
-      const int slot_buf = (t1 - 1 - t) & 1;
-      if (t - 1 >= t0) {
-        stage_token_meta(a, th_of(t - 1), metab(slot_buf ^ 1), lane);
-        nxt = load_token<Tin>(a, th_of(t - 1), col, true);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncwarp();
-      const int32_t* meta = metab(slot_buf);
-      const float* ww = reinterpret_cast<const float*>(meta + a.W);
-      const int32_t* ir = meta + 2 * a.W;
-      const float* wr = reinterpret_cast<const float*>(ir + a.R);
-      float* prt = a.part + (th * a.ntile + tile) * PW;
-      // Read of token t (state after its write): dq and the adjoint.
-      for (int e0 = 0; e0 < a.R; e0 += EPG) {
-        const int e = e0 + e4;
-        const int s = e < a.R ? ir[e] : -1;
-        const bool ok = static_cast<unsigned>(s) < static_cast<unsigned>(N);
-        float p = ok ? k.dy * Ms[s * CW + c] : 0.0f;
+    bwd_token_pass<Tin>(
+        a, b, h, tile, lane, t1 - 1, -1, t1 - t0, ring, reinterpret_cast<const float*>(logb), t0, true,
+        [&](int t, const BwdTok& k) {
+          const int64_t th = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
+          const int32_t* sw_ = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_w);
+          const float* ww = reinterpret_cast<const float*>(k.rec + a.rl.off_k_w);
+          const int32_t* ir = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_r);
+          const float* wr = reinterpret_cast<const float*>(k.rec + a.rl.off_q_r);
+          float* prt = a.part + (th * a.ntile + tile) * PW;
+          // Read of token t (state after its write): dq and the adjoint.
+          for (int e = lane; e < a.R; e += kWarp) {
+            const int s = ir[e];
+            float p = 0.0f;
+            if (s >= 0) {
+              const float q = wr[e];
+              const float4 m = Ms[s];
+              float4 g = Gs[s];
+              p = dot4(k.dy, m);
+              g.x = __fmaf_rn(q, k.dy.x, g.x);
+              g.y = __fmaf_rn(q, k.dy.y, g.y);
+              g.z = __fmaf_rn(q, k.dy.z, g.z);
+              g.w = __fmaf_rn(q, k.dy.w, g.w);
+              Gs[s] = g;
+            }
+            prt[a.W + e] = p;
+          }
+          __syncwarp();
+          // Write of token t, undone: derivatives, adjoint decay, state restore.
+          float4 dv = make_float4(0.f, 0.f, 0.f, 0.f);
+          float dal = 0.0f, dbe = 0.0f;
+          for (int e = lane; e < a.W; e += kWarp) {
+            const int s = sw_[e];
+            float dk = 0.0f;
+            if (s >= 0) {
+              const float kw = ww[e];
+              const float cw = k.beta * kw;
+              const float aw = k.alpha * (1.0f - cw);
+              const float4 g = Gs[s];
+              const float4 m = k.log[e];
+              const float da = dot4(g, m), dc = dot4(g, k.v);
+              const float r = dc - k.alpha * da;
+              dk = k.beta * r;
+              dal = __fmaf_rn(1.0f - cw, da, dal);
+              dbe = __fmaf_rn(kw, r, dbe);
+              dv.x = __fmaf_rn(cw, g.x, dv.x);
+              dv.y = __fmaf_rn(cw, g.y, dv.y);
+              dv.z = __fmaf_rn(cw, g.z, dv.z);
+              dv.w = __fmaf_rn(cw, g.w, dv.w);
+              Gs[s] = make_float4(aw * g.x, aw * g.y, aw * g.z, aw * g.w);
+              Ms[s] = m;
+            }
+            prt[e] = dk;
+          }
 #pragma unroll
-        for (int o = 1; o < CW; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-        if (ok) Gs[s * CW + c] = __fmaf_rn(wr[e], k.dy, Gs[s * CW + c]);
-        if (c == 0 && e < a.R) prt[a.W + e] = p;
-      }
-      __syncwarp();
-      // Write of token t, undone: derivatives, adjoint decay, state restore.
-      const float* lg = logb + static_cast<int64_t>(t - t0) * a.W * CW;
-      float dv_acc = 0.0f, dal = 0.0f, dbe = 0.0f;
-      for (int e0 = 0; e0 < a.W; e0 += EPG) {
-        const int e = e0 + e4;
-        const int s = e < a.W ? meta[e] : -1;
-        const bool ok = static_cast<unsigned>(s) < static_cast<unsigned>(N);
-        const float kw = ok ? ww[e] : 0.0f;
-        const float cw = k.beta * kw;
-        const float aw = k.alpha * (1.0f - cw);
-        const float g = ok ? Gs[s * CW + c] : 0.0f;
-        const float m = ok ? lg[e * CW + c] : 0.0f;
-        float da = g * m, dc = g * k.v;
-#pragma unroll
-        for (int o = 1; o < CW; o <<= 1) {
-          da += __shfl_xor_sync(0xffffffffu, da, o);
-          dc += __shfl_xor_sync(0xffffffffu, dc, o);
-        }
-        const float r = dc - k.alpha * da;
-        if (c == 0 && e < a.W) prt[e] = k.beta * r;
-        dal = __fmaf_rn(1.0f - cw, da, dal);
-        dbe = __fmaf_rn(kw, r, dbe);
-        dv_acc = __fmaf_rn(cw, g, dv_acc);
-        if (ok) {
-          Gs[s * CW + c] = aw * g;
-          Ms[s * CW + c] = m;
-        }
-      }
-#pragma unroll
-      for (int o = CW; o < kWarp; o <<= 1) {
-        dv_acc += __shfl_xor_sync(0xffffffffu, dv_acc, o);
-        dal += __shfl_xor_sync(0xffffffffu, dal, o);
-        dbe += __shfl_xor_sync(0xffffffffu, dbe, o);
-      }
-      if (e4 == 0) a.dv[th * a.d_v + col] = dv_acc;
-      if (lane == 0) {
-        prt[a.W + a.R] = dal;
-        prt[a.W + a.R + 1] = dbe;
-      }
-      __syncwarp();
-    }
+          for (int o = 16; o > 0; o >>= 1) {
+            dv.x += __shfl_xor_sync(0xffffffffu, dv.x, o);
+            dv.y += __shfl_xor_sync(0xffffffffu, dv.y, o);
+            dv.z += __shfl_xor_sync(0xffffffffu, dv.z, o);
+            dv.w += __shfl_xor_sync(0xffffffffu, dv.w, o);
+            dal += __shfl_xor_sync(0xffffffffu, dal, o);
+            dbe += __shfl_xor_sync(0xffffffffu, dbe, o);
+          }
+          if (lane == 0) {
+            *reinterpret_cast<float4*>(a.dv + th * a.d_v + col0) = dv;
+            prt[a.W + a.R] = dal;
+            prt[a.W + a.R + 1] = dbe;
+          }
+        });
   }
   __syncwarp();
-  for (int row = e4; row < N; row += EPG) Gout[static_cast<int64_t>(row) * a.d_v + col] = Gs[row * CW + c];
+  for (int row = lane; row < N; row += kWarp) *reinterpret_cast<float4*>(Gout + static_cast<int64_t>(row) * a.d_v) = Gs[row];
 }
 
 // Sums the per-tile partials in tile order: dw_w, dw_r [B,T,H,W|R], dalpha,

@@ -111,13 +111,14 @@ def test_slot_count_arguments_without_gpu(lib):
 
 
 def test_backward_workspace_and_support_without_gpu(lib):
-    # B=1, T=300, H=2, N=1024, W=R=64, d_v=128: 16 tiles of 8 columns per (b, h), 128-token chunks
+    # B=1, T=300, H=2, N=1024, W=R=64, d_v=128: 32 tiles of 4 columns per (b, h), 128-token chunks
     s = shape(B=1, T=300, H=2, sqrt_n=32, W=64, R=64, d_v=128)
-    tiles = 1 * 2 * 16
-    ckpt = tiles * (3 - 1) * 1024 * 8 * 4
-    log = tiles * 128 * 64 * 8 * 4
-    part = (1 * 300 * 2 * 16 * (64 + 64 + 2) * 4 + 255) // 256 * 256
-    assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == ckpt + log + part
+    tiles = 1 * 2 * 32
+    ckpt = tiles * (3 - 1) * 1024 * 4 * 4
+    log = tiles * 128 * 64 * 4 * 4
+    part = (1 * 300 * 2 * 32 * (64 + 64 + 2) * 4 + 255) // 256 * 256
+    rec = (1 * 2 * 300 * (4 * 64 + 4) * 4 + 255) // 256 * 256  # slots, weights, alpha/beta per token
+    assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == ckpt + log + part + rec
     s = shape(B=1, T=300, H=2, sqrt_n=32, W=64, R=64, d_v=128, state_dtype=native.BF16)
     assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == 0
     assert b"fp32 state" in lib.sdm_last_error()

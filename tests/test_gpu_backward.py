@@ -23,10 +23,12 @@ BWD = [
     # sqrt_n, d_v, W, R, in, T, B, H, M_in shared by the batch
     (32, 128, 64, 64, "bf16", 300, 2, 2, False),  # three checkpoint chunks and a ragged tail
     (8, 32, 5, 3, "f32", 41, 2, 1, True),
-    (64, 64, 16, 16, "bf16", 150, 1, 2, False),  # N = 4096: 4-column tiles
+    (64, 64, 16, 16, "bf16", 150, 1, 2, False),  # N = 4096
+    (8, 32, 40, 36, "f32", 33, 1, 1, False),  # W, R above one warp of entries
     (4, 16, 16, 16, "f32", 129, 1, 1, False),  # W = N: every slot written every token
     (16, 48, 12, 4, "f32", 1, 1, 3, True),  # one token
     (32, 16, 8, 8, "f32", 256, 1, 2, False),  # T a multiple of the chunk
+    (8, 32, 5, 4, "bf16", 70, 2, 1, False),  # W + R odd: padded staging
 ]
 
 
