@@ -73,7 +73,8 @@ constexpr int kBwdCols = 4;
 //   dy   [4] f32        this tile's columns of dy_t (reverse sweep only)
 // filled by cp.async kBwdStages - 1 tokens ahead of use, so the token loop
 // itself issues no global loads.
-constexpr int kBwdStages = 3;
+constexpr int kBwdStages = 4;
+constexpr int kBwdUnroll = 2;  // entries per lane handled together (W, R <= 64 in one round)
 
 struct BwdStage {
   int log, rec, v, dy, words;  // word offsets and the stage size (all multiples of 4)
@@ -96,6 +97,25 @@ struct BwdTok {
   float4 v, dy;
 };
 
+// Sums eight values over the warp with nine shuffles (reduce-scatter: each
+// exchange sends the half of the values the partner keeps). Lane l returns the
+// warp sum of value (l >> 2) & 7; lanes 4j .. 4j+3 hold value j. The order of
+// the additions is fixed, so the sums are reproducible.
+__device__ __forceinline__ float warp_sum8_transposed(float x0, float x1, float x2, float x3, float x4, float x5,
+                                                      float x6, float x7, int lane) {
+  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0, h4 = (lane & 4) != 0;
+  const float y0 = (h16 ? x4 : x0) + __shfl_xor_sync(0xffffffffu, h16 ? x0 : x4, 16);
+  const float y1 = (h16 ? x5 : x1) + __shfl_xor_sync(0xffffffffu, h16 ? x1 : x5, 16);
+  const float y2 = (h16 ? x6 : x2) + __shfl_xor_sync(0xffffffffu, h16 ? x2 : x6, 16);
+  const float y3 = (h16 ? x7 : x3) + __shfl_xor_sync(0xffffffffu, h16 ? x3 : x7, 16);
+  const float z0 = (h8 ? y2 : y0) + __shfl_xor_sync(0xffffffffu, h8 ? y0 : y2, 8);
+  const float z1 = (h8 ? y3 : y1) + __shfl_xor_sync(0xffffffffu, h8 ? y1 : y3, 8);
+  float w = (h4 ? z1 : z0) + __shfl_xor_sync(0xffffffffu, h4 ? z0 : z1, 4);
+  w += __shfl_xor_sync(0xffffffffu, w, 2);
+  w += __shfl_xor_sync(0xffffffffu, w, 1);
+  return w;
+}
+
 __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
   return __fmaf_rn(a.w, b.w, __fmaf_rn(a.z, b.z, __fmaf_rn(a.y, b.y, a.x * b.x)));
 }
@@ -110,28 +130,24 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
   const BwdStage L = bwd_stage(a.W, a.rl.words);
   const int n_log = log_src != nullptr ? a.W : 0;  // 16-byte pieces: one row each
   const int n_rec = a.rl.words / 4;
-  const int n_all = n_log + n_rec + 1 + (with_dy ? 1 : 0);
   const int bh = b * a.H + h;
   auto issue = [&](int i) {
     if (i < n) {
       const int t = t_first + i * step;
       const int64_t th = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
       float* st = ring + (i % kBwdStages) * L.words;
-      const float* lsrc = log_src != nullptr ? log_src + static_cast<int64_t>(t - log_t0) * a.W * kBwdCols : nullptr;
       const uint32_t* rsrc = a.rec + (static_cast<int64_t>(bh) * a.T + t) * a.rl.words;
-      for (int x = lane; x < n_all; x += kWarp) {
-        if (x < n_log) {
-          cp_async16(st + L.log + 4 * x, lsrc + 4 * x);
-        } else if (x < n_log + n_rec) {
-          const int j = x - n_log;
-          cp_async16(st + L.rec + 4 * j, rsrc + 4 * j);
-        } else if (x == n_log + n_rec) {
-          const Tin* vsrc = static_cast<const Tin*>(a.v) + th * a.d_v + tile * kBwdCols;
-          if constexpr (sizeof(Tin) == 4) cp_async16(st + L.v, vsrc);
-          else cp_async8(st + L.v, vsrc);
-        } else {
-          cp_async16(st + L.dy, a.dy + th * a.d_v + tile * kBwdCols);
-        }
+      for (int x = lane; x < n_rec; x += kWarp) cp_async16(st + L.rec + 4 * x, rsrc + 4 * x);
+      if (n_log > 0) {
+        const float* lsrc = log_src + static_cast<int64_t>(t - log_t0) * a.W * kBwdCols;
+        for (int x = lane; x < n_log; x += kWarp) cp_async16(st + L.log + 4 * x, lsrc + 4 * x);
+      }
+      if (lane == kWarp - 1) {
+        const Tin* vsrc = static_cast<const Tin*>(a.v) + th * a.d_v + tile * kBwdCols;
+        if constexpr (sizeof(Tin) == 4) cp_async16(st + L.v, vsrc);
+        else cp_async8(st + L.v, vsrc);
+      } else if (lane == kWarp - 2 && with_dy) {
+        cp_async16(st + L.dy, a.dy + th * a.d_v + tile * kBwdCols);
       }
     }
     cp_async_commit();  // empty groups past the end keep the count uniform
@@ -165,15 +181,29 @@ __device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok
                                                   int lane) {
   const int32_t* slot = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_w);
   const float* ww = reinterpret_cast<const float*>(k.rec + a.rl.off_k_w);
-  for (int e = lane; e < a.W; e += kWarp) {
-    const int s = slot[e];
-    if (s < 0) continue;
-    const float cw = k.beta * ww[e];
-    const float aw = k.alpha * (1.0f - cw);
-    const float4 m = Ms[s];
-    if (log != nullptr) log[e] = m;
-    Ms[s] = make_float4(__fmaf_rn(aw, m.x, __fmul_rn(cw, k.v.x)), __fmaf_rn(aw, m.y, __fmul_rn(cw, k.v.y)),
-                        __fmaf_rn(aw, m.z, __fmul_rn(cw, k.v.z)), __fmaf_rn(aw, m.w, __fmul_rn(cw, k.v.w)));
+  // kBwdUnroll entries per lane at once: their loads first, then the stores
+  // (the slots of one token are distinct, so the order is free).
+  for (int e0 = lane; e0 < a.W; e0 += kWarp * kBwdUnroll) {
+    int s[kBwdUnroll];
+    float4 m[kBwdUnroll];
+    float aw[kBwdUnroll], cw[kBwdUnroll];
+#pragma unroll
+    for (int u = 0; u < kBwdUnroll; ++u) {
+      const int e = e0 + u * kWarp;
+      s[u] = e < a.W ? slot[e] : -1;
+      cw[u] = s[u] >= 0 ? k.beta * ww[e] : 0.0f;
+      aw[u] = k.alpha * (1.0f - cw[u]);
+      m[u] = s[u] >= 0 ? Ms[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBwdUnroll; ++u) {
+      if (s[u] < 0) continue;
+      if (log != nullptr) log[e0 + u * kWarp] = m[u];
+      Ms[s[u]] = make_float4(__fmaf_rn(aw[u], m[u].x, __fmul_rn(cw[u], k.v.x)),
+                             __fmaf_rn(aw[u], m[u].y, __fmul_rn(cw[u], k.v.y)),
+                             __fmaf_rn(aw[u], m[u].z, __fmul_rn(cw[u], k.v.z)),
+                             __fmaf_rn(aw[u], m[u].w, __fmul_rn(cw[u], k.v.w)));
+    }
   }
 }
 
@@ -201,9 +231,11 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
   };
 
   // --------------------------------------------- pass 1: checkpoints --
+  // (only when the sequence has more than one chunk)
   load_min();
   __syncwarp();
-  bwd_token_pass<Tin>(a, b, h, tile, lane, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
+  if (nC > 1)
+    bwd_token_pass<Tin>(a, b, h, tile, lane, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
     if (t > 0 && t % a.C == 0) {
       float4* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N;
       for (int row = lane; row < N; row += kWarp) dst[row] = Ms[row];
@@ -245,62 +277,73 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
           const float* wr = reinterpret_cast<const float*>(k.rec + a.rl.off_q_r);
           float* prt = a.part + (th * a.ntile + tile) * PW;
           // Read of token t (state after its write): dq and the adjoint.
-          for (int e = lane; e < a.R; e += kWarp) {
-            const int s = ir[e];
-            float p = 0.0f;
-            if (s >= 0) {
-              const float q = wr[e];
-              const float4 m = Ms[s];
-              float4 g = Gs[s];
-              p = dot4(k.dy, m);
-              g.x = __fmaf_rn(q, k.dy.x, g.x);
-              g.y = __fmaf_rn(q, k.dy.y, g.y);
-              g.z = __fmaf_rn(q, k.dy.z, g.z);
-              g.w = __fmaf_rn(q, k.dy.w, g.w);
-              Gs[s] = g;
+          for (int e0 = lane; e0 < a.R; e0 += kWarp * kBwdUnroll) {
+            int s[kBwdUnroll];
+            float4 m[kBwdUnroll], g[kBwdUnroll];
+            float q[kBwdUnroll];
+#pragma unroll
+            for (int u = 0; u < kBwdUnroll; ++u) {
+              const int e = e0 + u * kWarp;
+              s[u] = e < a.R ? ir[e] : -1;
+              q[u] = s[u] >= 0 ? wr[e] : 0.0f;
+              m[u] = s[u] >= 0 ? Ms[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+              g[u] = s[u] >= 0 ? Gs[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            prt[a.W + e] = p;
+#pragma unroll
+            for (int u = 0; u < kBwdUnroll; ++u) {
+              const int e = e0 + u * kWarp;
+              if (e >= a.R) continue;
+              prt[a.W + e] = s[u] >= 0 ? dot4(k.dy, m[u]) : 0.0f;
+              if (s[u] >= 0)
+                Gs[s[u]] = make_float4(__fmaf_rn(q[u], k.dy.x, g[u].x), __fmaf_rn(q[u], k.dy.y, g[u].y),
+                                       __fmaf_rn(q[u], k.dy.z, g[u].z), __fmaf_rn(q[u], k.dy.w, g[u].w));
+            }
           }
           __syncwarp();
           // Write of token t, undone: derivatives, adjoint decay, state restore.
           float4 dv = make_float4(0.f, 0.f, 0.f, 0.f);
           float dal = 0.0f, dbe = 0.0f;
-          for (int e = lane; e < a.W; e += kWarp) {
-            const int s = sw_[e];
-            float dk = 0.0f;
-            if (s >= 0) {
-              const float kw = ww[e];
-              const float cw = k.beta * kw;
-              const float aw = k.alpha * (1.0f - cw);
-              const float4 g = Gs[s];
-              const float4 m = k.log[e];
-              const float da = dot4(g, m), dc = dot4(g, k.v);
-              const float r = dc - k.alpha * da;
-              dk = k.beta * r;
-              dal = __fmaf_rn(1.0f - cw, da, dal);
-              dbe = __fmaf_rn(kw, r, dbe);
-              dv.x = __fmaf_rn(cw, g.x, dv.x);
-              dv.y = __fmaf_rn(cw, g.y, dv.y);
-              dv.z = __fmaf_rn(cw, g.z, dv.z);
-              dv.w = __fmaf_rn(cw, g.w, dv.w);
-              Gs[s] = make_float4(aw * g.x, aw * g.y, aw * g.z, aw * g.w);
-              Ms[s] = m;
-            }
-            prt[e] = dk;
-          }
+          for (int e0 = lane; e0 < a.W; e0 += kWarp * kBwdUnroll) {
+            int s[kBwdUnroll];
+            float4 g[kBwdUnroll], m[kBwdUnroll];
+            float kw[kBwdUnroll];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            dv.x += __shfl_xor_sync(0xffffffffu, dv.x, o);
-            dv.y += __shfl_xor_sync(0xffffffffu, dv.y, o);
-            dv.z += __shfl_xor_sync(0xffffffffu, dv.z, o);
-            dv.w += __shfl_xor_sync(0xffffffffu, dv.w, o);
-            dal += __shfl_xor_sync(0xffffffffu, dal, o);
-            dbe += __shfl_xor_sync(0xffffffffu, dbe, o);
+            for (int u = 0; u < kBwdUnroll; ++u) {
+              const int e = e0 + u * kWarp;
+              s[u] = e < a.W ? sw_[e] : -1;
+              kw[u] = s[u] >= 0 ? ww[e] : 0.0f;
+              g[u] = s[u] >= 0 ? Gs[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+              m[u] = s[u] >= 0 ? k.log[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kBwdUnroll; ++u) {
+              const int e = e0 + u * kWarp;
+              if (e >= a.W) continue;
+              float dk = 0.0f;
+              if (s[u] >= 0) {
+                const float cw = k.beta * kw[u];
+                const float aw = k.alpha * (1.0f - cw);
+                const float da = dot4(g[u], m[u]), dc = dot4(g[u], k.v);
+                const float r = dc - k.alpha * da;
+                dk = k.beta * r;
+                dal = __fmaf_rn(1.0f - cw, da, dal);
+                dbe = __fmaf_rn(kw[u], r, dbe);
+                dv.x = __fmaf_rn(cw, g[u].x, dv.x);
+                dv.y = __fmaf_rn(cw, g[u].y, dv.y);
+                dv.z = __fmaf_rn(cw, g[u].z, dv.z);
+                dv.w = __fmaf_rn(cw, g[u].w, dv.w);
+                Gs[s[u]] = make_float4(aw * g[u].x, aw * g[u].y, aw * g[u].z, aw * g[u].w);
+                Ms[s[u]] = m[u];
+              }
+              prt[e] = dk;
+            }
           }
-          if (lane == 0) {
-            *reinterpret_cast<float4*>(a.dv + th * a.d_v + col0) = dv;
-            prt[a.W + a.R] = dal;
-            prt[a.W + a.R + 1] = dbe;
+          // Warp sums of dv (4 values), dalpha and dbeta: value j ends in lane 4 j.
+          const float sum = warp_sum8_transposed(dv.x, dv.y, dv.z, dv.w, dal, dbe, 0.0f, 0.0f, lane);
+          if ((lane & 3) == 0) {
+            const int j = lane >> 2;
+            if (j < 4) a.dv[th * a.d_v + col0 + j] = sum;
+            else if (j < 6) prt[a.W + a.R + (j - 4)] = sum;
           }
         });
   }
