@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -582,11 +583,13 @@ constexpr size_t kBwdSmemLimit = 232448;  // sm_100 opt-in shared memory per blo
 constexpr int kBwdChunk = 128;            // tokens per checkpoint chunk
 
 struct BwdChoice {
+  bool global = false;  // state and adjoint tiles in global memory (large N)
+  int U = 1;            // 16-byte units (4 columns) per lane and entry: tile width 4 U
   int C = kBwdChunk;
   int ntile = 0;
   size_t smem = 0;
-  size_t rec_bytes = 0, ckpt_bytes = 0, log_bytes = 0, part_bytes = 0;
-  size_t total() const { return rec_bytes + ckpt_bytes + log_bytes + part_bytes; }
+  size_t rec_bytes = 0, ckpt_bytes = 0, log_bytes = 0, part_bytes = 0, work_bytes = 0;
+  size_t total() const { return rec_bytes + ckpt_bytes + log_bytes + part_bytes + work_bytes; }
 };
 
 sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
@@ -594,34 +597,53 @@ sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
     return fail(SDM_ERR_UNSUPPORTED, "sdm_scan_backward needs an fp32 state (state_dtype SDM_F32)");
   const int64_t N = slots_of(s.sqrt_n);
   const sdm::RecLayout rl = rec_layout(s.W, s.R, false);
-  constexpr int CW = sdm::kBwdCols;
-  const size_t ring = static_cast<size_t>(sdm::kBwdStages) * sdm::bwd_stage(s.W, rl.words).words * 4;
-  const size_t smem = 2 * static_cast<size_t>(N) * CW * 4 + ring;
-  if (smem > kBwdSmemLimit)
-    return fail(SDM_ERR_UNSUPPORTED,
-                "sdm_scan_backward keeps a 4-column tile of the state and of its adjoint in shared memory; "
-                "N = " + std::to_string(N) + " rows do not fit (N <= about 6900 with W, R <= 64)");
+  const int in_bytes = static_cast<int>(in_size(s.in_dtype));
+  auto ring_bytes = [&](int U) {
+    return static_cast<size_t>(sdm::kBwdStages) * sdm::bwd_stage(s.W, rl.words, U, in_bytes).words * 4;
+  };
   BwdChoice c;
-  c.C = std::max(1, std::min<int>(kBwdChunk, s.T));
-  c.ntile = s.d_v / CW;
-  c.smem = smem;
+  const size_t on_chip = 2 * static_cast<size_t>(N) * 4 * 4 + ring_bytes(1);
+  c.global = on_chip > kBwdSmemLimit;
+  c.U = c.global ? (s.d_v % 32 == 0 ? 8 : 4) : 1;
+  c.smem = c.global ? ring_bytes(c.U) : on_chip;
+  if (c.smem > kBwdSmemLimit) return fail(SDM_ERR_UNSUPPORTED, "backward staging exceeds shared memory (W, R too large)");
+  if (c.global) {
+    // Chunk length near sqrt(T N / W): checkpoints (T / C states) and the log
+    // (C W rows) then take about the same memory.
+    const double best = std::sqrt(static_cast<double>(std::max(1, s.T)) * static_cast<double>(N) / s.W);
+    int C = kBwdChunk;
+    while (C < best && C < (1 << 20)) C *= 2;
+    c.C = std::max(1, std::min(C, s.T));
+  } else {
+    c.C = std::max(1, std::min<int>(kBwdChunk, s.T));
+  }
+  const int cols = 4 * c.U;
+  c.ntile = s.d_v / cols;
   const int64_t tiles = static_cast<int64_t>(s.B) * s.H * c.ntile;
   const int64_t nC = (static_cast<int64_t>(s.T) + c.C - 1) / c.C;
-  c.ckpt_bytes = align256(static_cast<size_t>(tiles) * std::max<int64_t>(0, nC - 1) * N * CW * 4);
-  c.log_bytes = align256(static_cast<size_t>(tiles) * c.C * s.W * CW * 4);
+  c.ckpt_bytes = align256(static_cast<size_t>(tiles) * std::max<int64_t>(0, nC - 1) * N * cols * 4);
+  c.log_bytes = align256(static_cast<size_t>(tiles) * c.C * s.W * cols * 4);
   c.part_bytes = align256(static_cast<size_t>(s.B) * s.T * s.H * c.ntile * (s.W + s.R + 2) * 4);
   c.rec_bytes = align256(static_cast<size_t>(s.B) * s.H * s.T * rl.words * 4);
+  c.work_bytes = c.global ? align256(static_cast<size_t>(s.B) * s.H * N * s.d_v * 4) : 0;
   *out = c;
   return SDM_OK;
 }
 
-template <typename Tin>
-sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
-  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin>);
+template <typename Tin, int U, bool G>
+sdm_status_t launch_bwd_inst(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
+  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin, U, G>);
   set_smem(kern, c.smem);
   const int64_t grid = static_cast<int64_t>(a.B) * a.H * c.ntile;
-  sdm::k_scan_backward<Tin><<<static_cast<unsigned>(grid), 32, c.smem, st>>>(a);
+  if (grid > 0x7FFFFFFFLL) return fail(SDM_ERR_UNSUPPORTED, "too many column tiles for one launch");
+  sdm::k_scan_backward<Tin, U, G><<<static_cast<unsigned>(grid), 32, c.smem, st>>>(a);
   return launch_status("backward launch");
+}
+
+template <typename Tin>
+sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
+  if (!c.global) return launch_bwd_inst<Tin, 1, false>(c, a, st);
+  return c.U == 8 ? launch_bwd_inst<Tin, 8, true>(c, a, st) : launch_bwd_inst<Tin, 4, true>(c, a, st);
 }
 
 }  // namespace
@@ -773,6 +795,7 @@ sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, c
   a.logbuf = reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes);
   uint32_t* rec = reinterpret_cast<uint32_t*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes);
   a.rec = rec;
+  a.Mwork = c.global ? reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes + c.rec_bytes) : nullptr;
   a.err = dev->err;
   if (s.in_dtype == SDM_BF16) {
     if ((r = launch_records<sdm::bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)

@@ -16,8 +16,9 @@
 //
 // with G = dL/dM running backwards over the tokens from dL/dM_T, the read of a
 // token before its write. Every column of d_v is independent given the
-// per-token scalars, so one warp carries one 4-column tile of one (b, h) with
-// its state M and adjoint G resident in shared memory. Memory-efficient by
+// per-token scalars, so one warp carries one column tile of one (b, h) with
+// its state M and adjoint G resident in shared memory (or, for large N, in
+// global memory). Memory-efficient by
 // recomputation: a first forward pass stores the tile every C tokens
 // (checkpoints); then, chunk by chunk from the end, the warp reloads the
 // chunk's checkpoint, recomputes the chunk forward keeping the values each
@@ -38,7 +39,7 @@ namespace sdm {
 struct BwdArgs {
   int B, T, H, N, d_v, W, R;
   int C;      // tokens per checkpoint chunk
-  int ntile;  // d_v / 4
+  int ntile;  // d_v / (4 U)
   RecLayout rl;
   const uint32_t* rec;  // [B, H, T, rl.words] per-token records (slots, weights, alpha, beta; no hazard plan)
   const void* v;        // [B, T, H, d_v] Tin
@@ -48,8 +49,9 @@ struct BwdArgs {
   float* dM;        // [B, H, N, d_v] in: dL/dM_T, out: dL/dM_0
   float* dv;        // [B, T, H, d_v]
   float* part;      // [B, T, H, ntile, W + R + 2] per-tile partial sums
-  float* ckpt;      // per tile: (ceil(T / C) - 1) * N * 4
-  float* logbuf;    // per tile: C * W * 4
+  float* ckpt;      // per tile: (ceil(T / C) - 1) * N * 4 U
+  float* logbuf;    // per tile: C * W * 4 U
+  float* Mwork;     // [B, H, N, d_v] working state when the tiles live in global memory
   unsigned* err;
 };
 
@@ -60,60 +62,71 @@ __device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) 
                : "memory");
 }
 
-// Tile geometry: a warp owns kBwdCols = 4 columns of one (b, h); lane l
-// handles entry e0 + l of a token (32 entries per warp instruction) and its 4
-// columns as one float4, so the sums over the tile's columns stay inside the
-// lane. State and adjoint rows are 16 bytes in shared memory.
-constexpr int kBwdCols = 4;
-
-// Staging: per token, a ring stage in shared memory holds
-//   log  [W][4] f32     the values its W writes overwrote (reverse sweep only)
-//   rec  [rl.words]     its record: slots, weights, alpha, beta
-//   v    [4] Tin        this tile's columns of v_t (padded to 16 bytes)
-//   dy   [4] f32        this tile's columns of dy_t (reverse sweep only)
-// filled by cp.async kBwdStages - 1 tokens ahead of use, so the token loop
-// itself issues no global loads.
+// Tile geometry: a warp owns 4 U columns of one (b, h); lane l handles entries
+// l and l + 32 of a token and walks the U 16-byte units of each entry's row
+// segment, so the sums over the tile's columns stay inside the lane. U = 1
+// keeps the state and adjoint tiles in shared memory (16 bytes per slot);
+// U = 8 (or 4) keeps them in global memory, where a lane's row segment is a
+// whole 128-byte line and wide tiles keep the per-tile partial sums few.
 constexpr int kBwdStages = 4;
-constexpr int kBwdUnroll = 2;  // entries per lane handled together (W, R <= 64 in one round)
 
 struct BwdStage {
-  int log, rec, v, dy, words;  // word offsets and the stage size (all multiples of 4)
+  int log, rec, v, vf, dy, words;  // word offsets and the stage size (all multiples of 4)
 };
-__host__ __device__ inline BwdStage bwd_stage(int W, int rec_words) {
+// log [W][4U] f32 | rec [words] | v [4U] Tin (raw) | vf [4U] f32 | dy [4U] f32
+__host__ __device__ inline BwdStage bwd_stage(int W, int rec_words, int U, int in_bytes) {
   BwdStage st;
   st.log = 0;
-  st.rec = W * kBwdCols;
+  st.rec = W * 4 * U;
   st.v = st.rec + rec_words;
-  st.dy = st.v + 4;
-  st.words = st.dy + 4;
+  st.vf = st.v + ((U * in_bytes + 3) & ~3);
+  st.dy = st.vf + 4 * U;
+  st.words = st.dy + 4 * U;
   return st;
 }
 
 // Per-token view of a filled stage.
 struct BwdTok {
-  const float4* log;
+  const float4* log;  // row e of the log at log[e * U]
   const uint32_t* rec;
+  const float4* v;    // U units of v_t (fp32)
+  const float4* dy;   // U units of dy_t
   float alpha, beta;
-  float4 v, dy;
 };
 
-// Sums eight values over the warp with nine shuffles (reduce-scatter: each
-// exchange sends the half of the values the partner keeps). Lane l returns the
-// warp sum of value (l >> 2) & 7; lanes 4j .. 4j+3 hold value j. The order of
-// the additions is fixed, so the sums are reproducible.
-__device__ __forceinline__ float warp_sum8_transposed(float x0, float x1, float x2, float x3, float x4, float x5,
-                                                      float x6, float x7, int lane) {
-  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0, h4 = (lane & 4) != 0;
-  const float y0 = (h16 ? x4 : x0) + __shfl_xor_sync(0xffffffffu, h16 ? x0 : x4, 16);
-  const float y1 = (h16 ? x5 : x1) + __shfl_xor_sync(0xffffffffu, h16 ? x1 : x5, 16);
-  const float y2 = (h16 ? x6 : x2) + __shfl_xor_sync(0xffffffffu, h16 ? x2 : x6, 16);
-  const float y3 = (h16 ? x7 : x3) + __shfl_xor_sync(0xffffffffu, h16 ? x3 : x7, 16);
-  const float z0 = (h8 ? y2 : y0) + __shfl_xor_sync(0xffffffffu, h8 ? y0 : y2, 8);
-  const float z1 = (h8 ? y3 : y1) + __shfl_xor_sync(0xffffffffu, h8 ? y1 : y3, 8);
-  float w = (h4 ? z1 : z0) + __shfl_xor_sync(0xffffffffu, h4 ? z0 : z1, 4);
-  w += __shfl_xor_sync(0xffffffffu, w, 2);
-  w += __shfl_xor_sync(0xffffffffu, w, 1);
-  return w;
+// Sums V values (V = 8 or 32) over the warp with V - 1 + log2(32 / V)
+// shuffles (reduce-scatter: each exchange sends the half of the values the
+// partner keeps). Value j ends in lanes j * (32 / V) .. j * (32 / V) + 32 / V - 1.
+// The order of the additions is fixed, so the sums are reproducible.
+// One reduce-scatter step: lanes with bit o set keep the upper half of the
+// n values and receive their partner's upper half; the others the lower.
+template <int n>
+__device__ __forceinline__ void halve_exchange(float* x, int o, int lane) {
+  const bool hi = (lane & o) != 0;
+#pragma unroll
+  for (int j = 0; j < n / 2; ++j) {
+    const float keep = hi ? x[j + n / 2] : x[j];
+    const float send = hi ? x[j] : x[j + n / 2];
+    x[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  }
+}
+template <int V>
+__device__ __forceinline__ float warp_sum_transposed(float (&x)[V], int lane) {
+  static_assert(V == 8 || V == 32, "8 or 32 values");
+  if constexpr (V == 32) {
+    halve_exchange<32>(x, 16, lane);
+    halve_exchange<16>(x, 8, lane);
+    halve_exchange<8>(x, 4, lane);
+    halve_exchange<4>(x, 2, lane);
+    halve_exchange<2>(x, 1, lane);
+  } else {
+    halve_exchange<8>(x, 16, lane);
+    halve_exchange<4>(x, 8, lane);
+    halve_exchange<2>(x, 4, lane);
+    x[0] += __shfl_xor_sync(0xffffffffu, x[0], 2);
+    x[0] += __shfl_xor_sync(0xffffffffu, x[0], 1);
+  }
+  return x[0];
 }
 
 __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
@@ -123,13 +136,14 @@ __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
 // Runs body(t, token) over n tokens t = t_first + i * step of one (b, h) and
 // column tile, each with its stage filled (log rows from log_src when given,
 // dy when with_dy).
-template <typename Tin, class Body>
+template <typename Tin, int U, class Body>
 __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, int tile, int lane, int t_first,
                                                int step, int n, float* ring, const float* log_src, int log_t0,
                                                bool with_dy, Body body) {
-  const BwdStage L = bwd_stage(a.W, a.rl.words);
-  const int n_log = log_src != nullptr ? a.W : 0;  // 16-byte pieces: one row each
+  const BwdStage L = bwd_stage(a.W, a.rl.words, U, static_cast<int>(sizeof(Tin)));
+  const int n_log = log_src != nullptr ? a.W * U : 0;  // 16-byte pieces
   const int n_rec = a.rl.words / 4;
+  constexpr int kVBytes = 4 * U * static_cast<int>(sizeof(Tin));
   const int bh = b * a.H + h;
   auto issue = [&](int i) {
     if (i < n) {
@@ -139,15 +153,19 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
       const uint32_t* rsrc = a.rec + (static_cast<int64_t>(bh) * a.T + t) * a.rl.words;
       for (int x = lane; x < n_rec; x += kWarp) cp_async16(st + L.rec + 4 * x, rsrc + 4 * x);
       if (n_log > 0) {
-        const float* lsrc = log_src + static_cast<int64_t>(t - log_t0) * a.W * kBwdCols;
+        const float* lsrc = log_src + static_cast<int64_t>(t - log_t0) * a.W * 4 * U;
         for (int x = lane; x < n_log; x += kWarp) cp_async16(st + L.log + 4 * x, lsrc + 4 * x);
       }
-      if (lane == kWarp - 1) {
-        const Tin* vsrc = static_cast<const Tin*>(a.v) + th * a.d_v + tile * kBwdCols;
-        if constexpr (sizeof(Tin) == 4) cp_async16(st + L.v, vsrc);
-        else cp_async8(st + L.v, vsrc);
-      } else if (lane == kWarp - 2 && with_dy) {
-        cp_async16(st + L.dy, a.dy + th * a.d_v + tile * kBwdCols);
+      const char* vsrc = reinterpret_cast<const char*>(static_cast<const Tin*>(a.v) + th * a.d_v + tile * 4 * U);
+      if constexpr (kVBytes >= 16) {
+        for (int x = lane; x < kVBytes / 16; x += kWarp)
+          cp_async16(reinterpret_cast<char*>(st + L.v) + 16 * x, vsrc + 16 * x);
+      } else {
+        if (lane == kWarp - 1) cp_async8(st + L.v, vsrc);
+      }
+      if (with_dy) {
+        const float* dsrc = a.dy + th * a.d_v + tile * 4 * U;
+        for (int x = lane; x < U; x += kWarp) cp_async16(st + L.dy + 4 * x, dsrc + 4 * x);
       }
     }
     cp_async_commit();  // empty groups past the end keep the count uniform
@@ -158,15 +176,16 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
     issue(i + kBwdStages - 1);
     cp_async_wait<kBwdStages - 1>();
     __syncwarp();
-    const float* st = ring + (i % kBwdStages) * L.words;
+    float* st = ring + (i % kBwdStages) * L.words;
+    if (lane < 4 * U) st[L.vf + lane] = to_f32<Tin>(reinterpret_cast<const Tin*>(st + L.v)[lane]);
+    __syncwarp();
     BwdTok k;
     k.log = reinterpret_cast<const float4*>(st + L.log);
     k.rec = reinterpret_cast<const uint32_t*>(st + L.rec);
+    k.v = reinterpret_cast<const float4*>(st + L.vf);
+    k.dy = reinterpret_cast<const float4*>(st + L.dy);
     k.alpha = __uint_as_float(k.rec[a.rl.off_ab]);
     k.beta = __uint_as_float(k.rec[a.rl.off_ab + 1]);
-    const Tin* vv = reinterpret_cast<const Tin*>(st + L.v);
-    k.v = make_float4(to_f32<Tin>(vv[0]), to_f32<Tin>(vv[1]), to_f32<Tin>(vv[2]), to_f32<Tin>(vv[3]));
-    k.dy = with_dy ? *reinterpret_cast<const float4*>(st + L.dy) : make_float4(0.f, 0.f, 0.f, 0.f);
     body(t_first + i * step, k);
     __syncwarp();
   }
@@ -174,100 +193,128 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
   __syncwarp();
 }
 
+// The rows of one tile: in shared memory (stride 4 U floats) or in a global
+// [N, d_v] array (stride d_v); row(s)[u] is unit u of slot s.
+struct BwdRows {
+  float* base;
+  int64_t stride;
+  __device__ __forceinline__ float4* row(int s) const { return reinterpret_cast<float4*>(base + s * stride); }
+};
+
 // The forward write of one token on the tile (the forward kernels' exact fp32
 // operations: m <- fma(alpha (1 - beta k), m, (beta k) v)). With `log`, the
-// overwritten rows are kept at log[e].
-__device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok& k, float4* Ms, float4* log,
+// overwritten units are kept at log[e * U + u].
+template <int U>
+__device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok& k, const BwdRows& Ms, float4* log,
                                                   int lane) {
+  constexpr int UNR = U == 1 ? 2 : 1;  // entries per lane in flight together
   const int32_t* slot = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_w);
   const float* ww = reinterpret_cast<const float*>(k.rec + a.rl.off_k_w);
-  // kBwdUnroll entries per lane at once: their loads first, then the stores
-  // (the slots of one token are distinct, so the order is free).
-  for (int e0 = lane; e0 < a.W; e0 += kWarp * kBwdUnroll) {
-    int s[kBwdUnroll];
-    float4 m[kBwdUnroll];
-    float aw[kBwdUnroll], cw[kBwdUnroll];
+  for (int e0 = lane; e0 < a.W; e0 += kWarp * UNR) {
+    int s[UNR];
+    float4 m[UNR][U];
+    float aw[UNR], cw[UNR];
 #pragma unroll
-    for (int u = 0; u < kBwdUnroll; ++u) {
-      const int e = e0 + u * kWarp;
-      s[u] = e < a.W ? slot[e] : -1;
-      cw[u] = s[u] >= 0 ? k.beta * ww[e] : 0.0f;
-      aw[u] = k.alpha * (1.0f - cw[u]);
-      m[u] = s[u] >= 0 ? Ms[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < UNR; ++q) {
+      const int e = e0 + q * kWarp;
+      s[q] = e < a.W ? slot[e] : -1;
+      cw[q] = s[q] >= 0 ? k.beta * ww[e] : 0.0f;
+      aw[q] = k.alpha * (1.0f - cw[q]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) m[q][u] = s[q] >= 0 ? Ms.row(s[q])[u] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < kBwdUnroll; ++u) {
-      if (s[u] < 0) continue;
-      if (log != nullptr) log[e0 + u * kWarp] = m[u];
-      Ms[s[u]] = make_float4(__fmaf_rn(aw[u], m[u].x, __fmul_rn(cw[u], k.v.x)),
-                             __fmaf_rn(aw[u], m[u].y, __fmul_rn(cw[u], k.v.y)),
-                             __fmaf_rn(aw[u], m[u].z, __fmul_rn(cw[u], k.v.z)),
-                             __fmaf_rn(aw[u], m[u].w, __fmul_rn(cw[u], k.v.w)));
+    for (int q = 0; q < UNR; ++q) {
+      if (s[q] < 0) continue;
+      const int e = e0 + q * kWarp;
+      float4* r = Ms.row(s[q]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float4 vv = k.v[u];
+        if (log != nullptr) log[e * U + u] = m[q][u];
+        r[u] = make_float4(__fmaf_rn(aw[q], m[q][u].x, __fmul_rn(cw[q], vv.x)),
+                           __fmaf_rn(aw[q], m[q][u].y, __fmul_rn(cw[q], vv.y)),
+                           __fmaf_rn(aw[q], m[q][u].z, __fmul_rn(cw[q], vv.z)),
+                           __fmaf_rn(aw[q], m[q][u].w, __fmul_rn(cw[q], vv.w)));
+      }
     }
   }
 }
 
-template <typename Tin>
+// kGlobal: the state and adjoint tiles live in global memory (a working copy
+// of the state in a.Mwork and dL/dM in place in a.dM) instead of shared
+// memory, for states too large to keep on chip; everything else is the same.
+template <typename Tin, int U, bool kGlobal>
 __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
   extern __shared__ __align__(16) float bsm[];
+  constexpr int UNR = U == 1 ? 2 : 1;
   const int N = a.N;
-  float4* Ms = reinterpret_cast<float4*>(bsm);  // [N] state rows of the tile
-  float4* Gs = Ms + N;                          // [N] adjoint rows
-  float* ring = reinterpret_cast<float*>(Gs + N);
-
   const int lane = threadIdx.x;
   const int tile = blockIdx.x % a.ntile;
   const int bh = blockIdx.x / a.ntile;
   const int b = bh / a.H, h = bh % a.H;
-  const int col0 = tile * kBwdCols;
+  const int col0 = tile * 4 * U;
   const int64_t tile_id = blockIdx.x;
   const int nC = (a.T + a.C - 1) / a.C;
-  float4* ckpt = reinterpret_cast<float4*>(a.ckpt) + tile_id * static_cast<int64_t>(nC > 1 ? nC - 1 : 0) * N;
-  float4* logb = reinterpret_cast<float4*>(a.logbuf) + tile_id * static_cast<int64_t>(a.C) * a.W;
+  float4* ckpt = reinterpret_cast<float4*>(a.ckpt) + tile_id * static_cast<int64_t>(nC > 1 ? nC - 1 : 0) * N * U;
+  float4* logb = reinterpret_cast<float4*>(a.logbuf) + tile_id * static_cast<int64_t>(a.C) * a.W * U;
   const float* Min = a.M_in + b * a.M_in_b_stride + static_cast<int64_t>(h) * N * a.d_v + col0;
-  auto load_min = [&]() {
-    for (int row = lane; row < N; row += kWarp)
-      Ms[row] = *reinterpret_cast<const float4*>(Min + static_cast<int64_t>(row) * a.d_v);
+  float* Gout = a.dM + (static_cast<int64_t>(b) * a.H + h) * N * a.d_v + col0;
+  BwdRows Ms, Gs;
+  float* ring;
+  if constexpr (kGlobal) {
+    Ms = BwdRows{a.Mwork + (static_cast<int64_t>(b) * a.H + h) * N * a.d_v + col0, a.d_v};
+    Gs = BwdRows{Gout, a.d_v};
+    ring = bsm;
+  } else {
+    Ms = BwdRows{bsm, 4 * U};
+    Gs = BwdRows{bsm + static_cast<size_t>(N) * 4 * U, 4 * U};
+    ring = bsm + 2 * static_cast<size_t>(N) * 4 * U;
+  }
+  // Tile-wide copies, one 16-byte unit per lane and step.
+  auto copy_in = [&](const BwdRows& dst, const float* src, int64_t src_stride) {
+    for (int x = lane; x < N * U; x += kWarp) {
+      const int row = x / U, u = x % U;
+      dst.row(row)[u] = reinterpret_cast<const float4*>(src + row * src_stride)[u];
+    }
   };
 
   // --------------------------------------------- pass 1: checkpoints --
   // (only when the sequence has more than one chunk)
-  load_min();
+  copy_in(Ms, Min, a.d_v);
   __syncwarp();
   if (nC > 1)
-    bwd_token_pass<Tin>(a, b, h, tile, lane, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
-    if (t > 0 && t % a.C == 0) {
-      float4* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N;
-      for (int row = lane; row < N; row += kWarp) dst[row] = Ms[row];
-    }
-    bwd_forward_token(a, k, Ms, nullptr, lane);
-  });
+    bwd_token_pass<Tin, U>(a, b, h, tile, lane, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
+      if (t > 0 && t % a.C == 0) {
+        float4* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N * U;
+        for (int x = lane; x < N * U; x += kWarp) dst[x] = Ms.row(x / U)[x % U];
+      }
+      bwd_forward_token<U>(a, k, Ms, nullptr, lane);
+    });
 
   // ---------------------------------- pass 2: chunks from the end --
-  float* Gout = a.dM + (static_cast<int64_t>(b) * a.H + h) * N * a.d_v + col0;
-  for (int row = lane; row < N; row += kWarp)
-    Gs[row] = *reinterpret_cast<const float4*>(Gout + static_cast<int64_t>(row) * a.d_v);
+  if constexpr (!kGlobal) copy_in(Gs, Gout, a.d_v);
   const int PW = a.W + a.R + 2;
   for (int kc = nC - 1; kc >= 0; --kc) {
     const int t0 = kc * a.C, t1 = min(a.T, t0 + a.C);
     // State at the chunk start.
     if (kc == 0) {
-      load_min();
+      copy_in(Ms, Min, a.d_v);
     } else {
-      const float4* src = ckpt + static_cast<int64_t>(kc - 1) * N;
-      for (int row = lane; row < N; row += kWarp) Ms[row] = src[row];
+      const float* src = reinterpret_cast<const float*>(ckpt + static_cast<int64_t>(kc - 1) * N * U);
+      copy_in(Ms, src, 4 * U);
     }
     __syncwarp();
-    // Recompute the chunk forward, logging overwritten rows.
-    bwd_token_pass<Tin>(a, b, h, tile, lane, t0, 1, t1 - t0, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
-      bwd_forward_token(a, k, Ms, logb + static_cast<int64_t>(t - t0) * a.W, lane);
+    // Recompute the chunk forward, logging overwritten units.
+    bwd_token_pass<Tin, U>(a, b, h, tile, lane, t0, 1, t1 - t0, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
+      bwd_forward_token<U>(a, k, Ms, logb + static_cast<int64_t>(t - t0) * a.W * U, lane);
     });
     // The log rows were written by other lanes; the reverse pass reads them
     // back through cp.async.
     __threadfence_block();
     __syncwarp();
     // Backward sweep over the chunk.
-    bwd_token_pass<Tin>(
+    bwd_token_pass<Tin, U>(
         a, b, h, tile, lane, t1 - 1, -1, t1 - t0, ring, reinterpret_cast<const float*>(logb), t0, true,
         [&](int t, const BwdTok& k) {
           const int64_t th = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
@@ -277,78 +324,136 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
           const float* wr = reinterpret_cast<const float*>(k.rec + a.rl.off_q_r);
           float* prt = a.part + (th * a.ntile + tile) * PW;
           // Read of token t (state after its write): dq and the adjoint.
-          for (int e0 = lane; e0 < a.R; e0 += kWarp * kBwdUnroll) {
-            int s[kBwdUnroll];
-            float4 m[kBwdUnroll], g[kBwdUnroll];
-            float q[kBwdUnroll];
+          for (int e0 = lane; e0 < a.R; e0 += kWarp * UNR) {
+            int s[UNR];
+            float q[UNR];
+            float4 m[UNR][U], g[UNR][U];
 #pragma unroll
-            for (int u = 0; u < kBwdUnroll; ++u) {
-              const int e = e0 + u * kWarp;
-              s[u] = e < a.R ? ir[e] : -1;
-              q[u] = s[u] >= 0 ? wr[e] : 0.0f;
-              m[u] = s[u] >= 0 ? Ms[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
-              g[u] = s[u] >= 0 ? Gs[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int qq = 0; qq < UNR; ++qq) {
+              const int e = e0 + qq * kWarp;
+              s[qq] = e < a.R ? ir[e] : -1;
+              q[qq] = s[qq] >= 0 ? wr[e] : 0.0f;
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                m[qq][u] = s[qq] >= 0 ? Ms.row(s[qq])[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+                g[qq][u] = s[qq] >= 0 ? Gs.row(s[qq])[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
             }
 #pragma unroll
-            for (int u = 0; u < kBwdUnroll; ++u) {
-              const int e = e0 + u * kWarp;
+            for (int qq = 0; qq < UNR; ++qq) {
+              const int e = e0 + qq * kWarp;
               if (e >= a.R) continue;
-              prt[a.W + e] = s[u] >= 0 ? dot4(k.dy, m[u]) : 0.0f;
-              if (s[u] >= 0)
-                Gs[s[u]] = make_float4(__fmaf_rn(q[u], k.dy.x, g[u].x), __fmaf_rn(q[u], k.dy.y, g[u].y),
-                                       __fmaf_rn(q[u], k.dy.z, g[u].z), __fmaf_rn(q[u], k.dy.w, g[u].w));
+              float p = 0.0f;
+              if (s[qq] >= 0) {
+                float4* gr = Gs.row(s[qq]);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                  const float4 d = k.dy[u];
+                  p += dot4(d, m[qq][u]);
+                  gr[u] = make_float4(__fmaf_rn(q[qq], d.x, g[qq][u].x), __fmaf_rn(q[qq], d.y, g[qq][u].y),
+                                      __fmaf_rn(q[qq], d.z, g[qq][u].z), __fmaf_rn(q[qq], d.w, g[qq][u].w));
+                }
+              }
+              prt[a.W + e] = p;
             }
           }
           __syncwarp();
           // Write of token t, undone: derivatives, adjoint decay, state restore.
-          float4 dv = make_float4(0.f, 0.f, 0.f, 0.f);
-          float dal = 0.0f, dbe = 0.0f;
-          for (int e0 = lane; e0 < a.W; e0 += kWarp * kBwdUnroll) {
-            int s[kBwdUnroll];
-            float4 g[kBwdUnroll], m[kBwdUnroll];
-            float kw[kBwdUnroll];
+          float4 dv[U];
 #pragma unroll
-            for (int u = 0; u < kBwdUnroll; ++u) {
-              const int e = e0 + u * kWarp;
-              s[u] = e < a.W ? sw_[e] : -1;
-              kw[u] = s[u] >= 0 ? ww[e] : 0.0f;
-              g[u] = s[u] >= 0 ? Gs[s[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
-              m[u] = s[u] >= 0 ? k.log[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int u = 0; u < U; ++u) dv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          float dal = 0.0f, dbe = 0.0f;
+          for (int e0 = lane; e0 < a.W; e0 += kWarp * UNR) {
+            int s[UNR];
+            float kw[UNR];
+            float4 g[UNR][U], m[UNR][U];
+#pragma unroll
+            for (int qq = 0; qq < UNR; ++qq) {
+              const int e = e0 + qq * kWarp;
+              s[qq] = e < a.W ? sw_[e] : -1;
+              kw[qq] = s[qq] >= 0 ? ww[e] : 0.0f;
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                g[qq][u] = s[qq] >= 0 ? Gs.row(s[qq])[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+                m[qq][u] = s[qq] >= 0 ? k.log[e * U + u] : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
             }
 #pragma unroll
-            for (int u = 0; u < kBwdUnroll; ++u) {
-              const int e = e0 + u * kWarp;
+            for (int qq = 0; qq < UNR; ++qq) {
+              const int e = e0 + qq * kWarp;
               if (e >= a.W) continue;
               float dk = 0.0f;
-              if (s[u] >= 0) {
-                const float cw = k.beta * kw[u];
+              if (s[qq] >= 0) {
+                const float cw = k.beta * kw[qq];
                 const float aw = k.alpha * (1.0f - cw);
-                const float da = dot4(g[u], m[u]), dc = dot4(g[u], k.v);
+                float da = 0.0f, dc = 0.0f;
+                float4* gr = Gs.row(s[qq]);
+                float4* mr = Ms.row(s[qq]);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                  const float4 gg = g[qq][u];
+                  da += dot4(gg, m[qq][u]);
+                  dc += dot4(gg, k.v[u]);
+                  dv[u].x = __fmaf_rn(cw, gg.x, dv[u].x);
+                  dv[u].y = __fmaf_rn(cw, gg.y, dv[u].y);
+                  dv[u].z = __fmaf_rn(cw, gg.z, dv[u].z);
+                  dv[u].w = __fmaf_rn(cw, gg.w, dv[u].w);
+                  gr[u] = make_float4(aw * gg.x, aw * gg.y, aw * gg.z, aw * gg.w);
+                  mr[u] = m[qq][u];
+                }
                 const float r = dc - k.alpha * da;
                 dk = k.beta * r;
                 dal = __fmaf_rn(1.0f - cw, da, dal);
-                dbe = __fmaf_rn(kw[u], r, dbe);
-                dv.x = __fmaf_rn(cw, g[u].x, dv.x);
-                dv.y = __fmaf_rn(cw, g[u].y, dv.y);
-                dv.z = __fmaf_rn(cw, g[u].z, dv.z);
-                dv.w = __fmaf_rn(cw, g[u].w, dv.w);
-                Gs[s[u]] = make_float4(aw * g[u].x, aw * g[u].y, aw * g[u].z, aw * g[u].w);
-                Ms[s[u]] = m[u];
+                dbe = __fmaf_rn(kw[qq], r, dbe);
               }
               prt[e] = dk;
             }
           }
-          // Warp sums of dv (4 values), dalpha and dbeta: value j ends in lane 4 j.
-          const float sum = warp_sum8_transposed(dv.x, dv.y, dv.z, dv.w, dal, dbe, 0.0f, 0.0f, lane);
-          if ((lane & 3) == 0) {
-            const int j = lane >> 2;
-            if (j < 4) a.dv[th * a.d_v + col0 + j] = sum;
-            else if (j < 6) prt[a.W + a.R + (j - 4)] = sum;
+          // Warp sums of dv (4 U values), dalpha and dbeta.
+          if constexpr (U == 1) {
+            float x[8] = {dv[0].x, dv[0].y, dv[0].z, dv[0].w, dal, dbe, 0.0f, 0.0f};
+            const float sum = warp_sum_transposed<8>(x, lane);  // value j in lanes 4j .. 4j+3
+            if ((lane & 3) == 0) {
+              const int j = lane >> 2;
+              if (j < 4) a.dv[th * a.d_v + col0 + j] = sum;
+              else if (j < 6) prt[a.W + a.R + (j - 4)] = sum;
+            }
+          } else {
+            float x[32];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              x[4 * u] = u < U ? dv[u < U ? u : 0].x : 0.0f;
+              x[4 * u + 1] = u < U ? dv[u < U ? u : 0].y : 0.0f;
+              x[4 * u + 2] = u < U ? dv[u < U ? u : 0].z : 0.0f;
+              x[4 * u + 3] = u < U ? dv[u < U ? u : 0].w : 0.0f;
+            }
+            if constexpr (U < 8) {  // spare slots carry dalpha and dbeta
+              x[4 * U] = dal;
+              x[4 * U + 1] = dbe;
+            }
+            const float sum = warp_sum_transposed<32>(x, lane);  // value j in lane j
+            if (lane < 4 * U) a.dv[th * a.d_v + col0 + lane] = sum;
+            if constexpr (U < 8) {
+              if (lane == 4 * U || lane == 4 * U + 1) prt[a.W + a.R + (lane - 4 * U)] = sum;
+            } else {
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) {
+                dal += __shfl_xor_sync(0xffffffffu, dal, o);
+                dbe += __shfl_xor_sync(0xffffffffu, dbe, o);
+              }
+              if (lane == 0) {
+                prt[a.W + a.R] = dal;
+                prt[a.W + a.R + 1] = dbe;
+              }
+            }
           }
         });
   }
   __syncwarp();
-  for (int row = lane; row < N; row += kWarp) *reinterpret_cast<float4*>(Gout + static_cast<int64_t>(row) * a.d_v) = Gs[row];
+  if constexpr (!kGlobal) {
+    for (int x = lane; x < N * U; x += kWarp)
+      reinterpret_cast<float4*>(Gout + static_cast<int64_t>(x / U) * a.d_v)[x % U] = Gs.row(x / U)[x % U];
+  }
 }
 
 // Sums the per-tile partials in tile order: dw_w, dw_r [B,T,H,W|R], dalpha,

@@ -29,6 +29,10 @@ BWD = [
     (16, 48, 12, 4, "f32", 1, 1, 3, True),  # one token
     (32, 16, 8, 8, "f32", 256, 1, 2, False),  # T a multiple of the chunk
     (8, 32, 5, 4, "bf16", 70, 2, 1, False),  # W + R odd: padded staging
+    # N = 16384: state and adjoint tiles in global memory
+    (128, 64, 16, 16, "bf16", 150, 1, 2, False),  # 32-column tiles, one chunk
+    (128, 48, 8, 8, "f32", 70, 2, 1, True),  # d_v not a multiple of 32: 16-column tiles
+    (128, 32, 64, 64, "bf16", 600, 1, 1, False),  # two chunks of 512
 ]
 
 
@@ -81,12 +85,9 @@ def test_scan_backward_deterministic(sdm, cuda_device):
         assert torch.equal(a[k], b[k]), k
 
 
-def test_scan_backward_rejects_bf16_state_and_large_n(sdm, cuda_device):
+def test_scan_backward_rejects_bf16_state(sdm, cuda_device):
     sh = sdm.make_shape(1, 4, 1, 32, 8, 8, 64, torch.float32, torch.bfloat16)
     with pytest.raises(sdm.SdmError, match="fp32 state"):
-        sdm.scan_backward_workspace_bytes(sh)
-    sh = sdm.make_shape(1, 4, 1, 128, 8, 8, 64, torch.float32, torch.float32)  # N = 16384
-    with pytest.raises(sdm.SdmError, match="shared memory"):
         sdm.scan_backward_workspace_bytes(sh)
 
 
@@ -118,11 +119,14 @@ def test_pkm_topk_backward_matches_oracle(sdm, oracle, cuda_device, sqrt_n, K):
     assert_rel_close(got.cpu().numpy(), want, TOL_TOPK_BWD, "dscores")
 
 
-def test_scan_backward_full_size_sampled(sdm, oracle, cuda_device):
-    """The bench workload d2048_h16_n1024_dv128 at full size, in the launch
-    configuration the benchmark times, with a seeded synthetic selection; two
-    sampled (b, h) pairs compared with the oracle over the whole sequence."""
-    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"]
+@pytest.mark.parametrize("name,pairs", [("d2048_h16_n1024_dv128", ((0, 0), (7, 15))),
+                                        ("d2048_h4_n16384_dv512", ((5, 2),))])
+def test_scan_backward_full_size_sampled(sdm, oracle, cuda_device, name, pairs):
+    """A full-size workload (the bench's, and one whose state only fits in
+    global memory), in the launch configuration the benchmark times, with a
+    seeded synthetic selection; sampled (b, h) pairs compared with the oracle
+    over the whole sequence."""
+    shape = synth.WORKLOADS[name]
     inp = synth.make_inputs(shape, seed=0, device=cuda_device)
     gen = torch.Generator().manual_seed(3)
 
@@ -142,7 +146,7 @@ def test_scan_backward_full_size_sampled(sdm, oracle, cuda_device):
     out = sdm.scan_backward(idx_w.to(dev), w_w.to(dev), idx_r.to(dev), w_r.to(dev), inp["v"], inp["alpha"],
                             inp["beta"], M0, dy.to(dev))
     sdm.stream_check()
-    for b, h in ((0, 0), (shape.B - 1, shape.H - 1)):
+    for b, h in pairs:
         s = lambda t: t[b:b + 1, :, h:h + 1].contiguous()
         want = oracle.scan_backward(s(idx_w).numpy(), s(w_w).numpy().astype(np.float64), s(idx_r).numpy(),
                                     s(w_r).numpy().astype(np.float64), f32(s(inp["v"])), f32(s(inp["alpha"])),
