@@ -158,11 +158,13 @@ SDM_API size_t sdm_scan_backward_workspace_bytes(const sdm_shape_t* shape);
  *   dalpha_t = sum_i (1 - beta_t k_i) <G[i], M_{t-1}[i]>
  *   dbeta_t  = sum_i k_i (<G[i], v_t> - alpha_t <G[i], M_{t-1}[i]>)
  *   dM       <- dL/dM_0 (in place)
- * The state trajectory is recomputed from M_in (checkpoints every 128 tokens
+ * The state trajectory is recomputed from M_in (checkpoints every C tokens
  * plus a log of overwritten rows, all in the workspace), bit-identical to the
- * forward's. Requires an fp32 state (state_dtype SDM_F32) whose column tile
- * and adjoint fit in shared memory (2 * N * 8 * 4 bytes <= 227 KB, or with
- * 4-column tiles N <= about 7200); otherwise SDM_ERR_UNSUPPORTED.
+ * forward's. Requires an fp32 state (state_dtype SDM_F32), else
+ * SDM_ERR_UNSUPPORTED. While 4-column tiles of the state and its adjoint fit
+ * in shared memory (N up to about 6900) they stay there (C = 128); larger
+ * states use 32-column tiles in global memory (a working copy of the state in
+ * the workspace, dM updated in place) with C near sqrt(T N / W).
  *   idx_w, w_w, idx_r, w_r, v, alpha, beta: the forward's inputs (as sdm_scan)
  *   M_in  fp32, the state the forward started from: [B,H,N,d_v], or [H,N,d_v]
  *         shared by every batch row when m_in_shared != 0
