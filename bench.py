@@ -516,7 +516,8 @@ def run_decode(args, dist: Dist):
                 "warmup": args.warmup, "ms_per_step": us_per_step / 1e3, "higher_is_better": False,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
                 "tokens_per_s": aggregate_value(shape.B * args.steps, dist.world, ms / 1e3),
-                "gpu_launches": 4 * args.steps, "clocks": clocks.summary()}
+                "gpu_launches": int(sdm.native.load().sdm_layer_step_launches(ctypes.byref(sh))) * args.steps,
+                "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
     dist.close()
 

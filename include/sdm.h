@@ -235,6 +235,13 @@ SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp,
                                const void* M0, void* M_out, float* y, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* Kernel launches one sdm_layer_step call makes for this shape, without the
+ * epilogue's (one more when g is given on the general path): 1 when the call
+ * takes the single-launch decode kernel (T = 1, W = R <= 64, automatic
+ * variant), else 4 (two selections, records, recurrence).
+ * -1 for an invalid shape. For profiles and logs. */
+SDM_API int32_t sdm_layer_step_launches(const sdm_shape_t* shape);
+
 /* Bytes of workspace sdm_layer_step needs for this shape (0 for invalid shapes). */
 SDM_API size_t sdm_layer_step_workspace_bytes(const sdm_shape_t* shape);
 

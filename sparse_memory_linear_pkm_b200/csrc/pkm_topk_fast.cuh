@@ -325,6 +325,220 @@ struct FastTopkLayout {
   uint32_t hist, sel, hv, hx, tie;
 };
 
+// Builds the candidate table tab[c] = (ra, rb) for the pairs (ra+1)(rb+1) <= K
+// of the per-half ranks; run by one warp.
+__device__ __forceinline__ void fast_topk_build_table(uint16_t* tab, int Kh, int K, int lane) {
+  int base = 0;
+  for (int r0 = 0; r0 < Kh; r0 += kWarp) {
+    const int ra = r0 + lane;
+    const int len = ra < Kh ? min(Kh, K / (ra + 1)) : 0;
+    int incl = len;
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int start = base + incl - len;
+    for (int rb = 0; rb < len; ++rb) {
+      tab[2 * (start + rb)] = static_cast<uint16_t>(ra);
+      tab[2 * (start + rb) + 1] = static_cast<uint16_t>(rb);
+    }
+    base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
+  }
+}
+
+// One selection by one warp: the top K slots of the score vector x[0 : 2n]
+// in selection order (io) and their softmax weights (wo); ws is the warp's
+// scratch of L.warp_bytes in shared memory.
+template <typename Tin, int E, int EH, int EPL, int CP>
+__device__ __forceinline__ void fast_topk_unit(const Tin* __restrict__ x, const FastTopkLayout& L,
+                                               const uint16_t* tab, unsigned char* ws, int32_t* io, float* wo) {
+  const int lane = lane_id();
+  const int n = L.n, K = L.K, Kh = L.Kh, C = L.C;
+  constexpr int SZ = kWarp * kFastTopkMaxK / kWarp;  // stride of the two halves in hv/hx
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+  uint64_t* sel = reinterpret_cast<uint64_t*>(ws + L.sel);
+  float* hv = reinterpret_cast<float*>(ws + L.hv);
+  int32_t* hx = reinterpret_cast<int32_t*>(ws + L.hx);
+  uint32_t* tie = reinterpret_cast<uint32_t*>(ws + L.tie);
+  const uint32_t lt = lanemask_lt();
+  warp_half_select<Tin, EH, EPL>(x, n, Kh, hist, sel, hv, hx);
+  warp_half_select<Tin, EH, EPL>(x + n, n, Kh, hist, sel, hv + SZ, hx + SZ);
+
+  // Candidates with exact scores: ck = ord(hi), cl = ~slot, clo = ord(lo).
+  uint32_t ck[CP], cl[CP], clo[CP];
+#pragma unroll
+  for (int j = 0; j < CP; ++j) {
+    const int c = j * kWarp + lane;
+    ck[j] = 0u;
+    cl[j] = 0u;
+    clo[j] = 0u;
+    if (c < C) {
+      const int ra = tab[2 * c], rb = tab[2 * c + 1];
+      float hi, lo;
+      two_sum(hv[ra], hv[SZ + rb], hi, lo);
+      ck[j] = ord_f32(canon_zero(hi));
+      clo[j] = ord_f32(canon_zero(lo));
+      cl[j] = 0xFFFFFFFFu - static_cast<uint32_t>(hx[ra] * n + hx[SZ + rb]);
+    }
+  }
+  // Winners by hi; a boundary that splits equal hi ranks that group by
+  // (lo desc, slot asc). Exact fp32 sums of bf16 inputs tie often, but such
+  // groups are small.
+  const SelectPlan sp = warp_select_plan<CP>(ck, K, hist, warp_kth_floor<CP>(ck, K));
+  const uint32_t tb = sp.thr >> sp.shift;
+  const bool split = sp.take_eq < sp.bin_count;  // only at shift 0, i.e. equal hi
+  int tie_rank[CP];
+#pragma unroll
+  for (int j = 0; j < CP; ++j) tie_rank[j] = 0;
+  if (split) {
+    int g = 0;
+#pragma unroll
+    for (int j = 0; j < CP; ++j) {
+      const bool eq = j * kWarp + lane < C && ck[j] == sp.thr;
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      if (eq) {
+        const int p = g + __popc(be & lt);
+        tie[2 * p] = clo[j];
+        tie[2 * p + 1] = cl[j];
+      }
+      g += __popc(be);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < CP; ++j) {
+      if (j * kWarp + lane < C && ck[j] == sp.thr) {
+        int r = 0;
+        for (int q = 0; q < g; ++q) {
+          const uint32_t lq = tie[2 * q], sq = tie[2 * q + 1];
+          r += (lq > clo[j]) || (lq == clo[j] && sq > cl[j]);
+        }
+        tie_rank[j] = r;
+      }
+    }
+    __syncwarp();
+  }
+  int cnt = 0;
+#pragma unroll
+  for (int j = 0; j < CP; ++j) {
+    const int c = j * kWarp + lane;
+    const uint32_t kb = ck[j] >> sp.shift;
+    const bool take = c < C && (kb > tb || (kb == tb && ck[j] >= sp.floor && (!split || tie_rank[j] < sp.take_eq)));
+    const uint32_t bt = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int p = cnt + __popc(bt & lt);
+      sel[p] = (static_cast<uint64_t>(ck[j]) << 32) | cl[j];
+      hist[p] = clo[j];
+    }
+    cnt += __popc(bt);
+  }
+  __syncwarp();
+  // Order the K winners by ord(hi):(~slot), descending: each winner's rank is
+  // the number of winner keys above it (keys are distinct: the slot is part
+  // of the key), counted against all K keys read two at a time from shared
+  // memory; then every winner moves to its rank.
+  uint64_t k[E];
+  uint32_t kl[E];
+  {
+    uint64_t mine[E];
+    uint32_t mlo[E];
+    int rank[E];
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      const int p = lane * E + s;
+      mine[s] = p < K ? sel[p] : 0ull;
+      mlo[s] = p < K ? hist[p] : 0u;
+      rank[s] = 0;
+    }
+    const ulonglong2* sel2 = reinterpret_cast<const ulonglong2*>(sel);
+    for (int j = 0; j < K; j += 2) {
+      const ulonglong2 two = sel2[j >> 1];
+      const uint64_t second = j + 1 < K ? two.y : 0ull;  // past K: stale, never above a winner
+#pragma unroll
+      for (int s = 0; s < E; ++s) rank[s] += (two.x > mine[s]) + (second > mine[s]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      if (lane * E + s < K) {
+        sel[rank[s]] = mine[s];
+        hist[rank[s]] = mlo[s];
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      const int p = lane * E + s;
+      k[s] = p < K ? sel[p] : 0ull;
+      kl[s] = p < K ? hist[p] : 0u;
+    }
+    __syncwarp();
+  }
+  // Neighbours with equal hi but different lo need the (lo desc, slot asc) order.
+  bool fix = false;
+  {
+    const uint32_t nh = __shfl_down_sync(0xffffffffu, static_cast<uint32_t>(k[0] >> 32), 1);
+    const uint32_t nl = __shfl_down_sync(0xffffffffu, kl[0], 1);
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      const int p = lane * E + s;
+      if (p + 1 < K) {
+        const uint32_t h1 = s + 1 < E ? static_cast<uint32_t>(k[(s + 1) % E] >> 32) : nh;
+        const uint32_t l1 = s + 1 < E ? kl[(s + 1) % E] : nl;
+        fix = fix || (static_cast<uint32_t>(k[s] >> 32) == h1 && kl[s] != l1);
+      }
+    }
+  }
+  const bool any_fix = __any_sync(0xffffffffu, fix);
+  // Softmax of the selected scores (order independent).
+  const float top = unord_f32(__shfl_sync(0xffffffffu, static_cast<uint32_t>(k[0] >> 32), 0));
+  float ev[E];
+  float z = 0.f;
+#pragma unroll
+  for (int s = 0; s < E; ++s) {
+    const int p = lane * E + s;
+    ev[s] = p < K ? expf(unord_f32(static_cast<uint32_t>(k[s] >> 32)) - top) : 0.f;
+    z += ev[s];
+  }
+  z = warp_sum(z);
+  const float inv_z = 1.0f / z;
+  if (!any_fix) {
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      const int p = lane * E + s;
+      if (p < K) {
+        io[p] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(k[s]));
+        wo[p] = ev[s] * inv_z;
+      }
+    }
+  } else {
+    // Rare: rank each winner by (hi desc, lo desc, slot asc).
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      const int p = lane * E + s;
+      if (p < K) {
+        sel[p] = k[s];
+        tie[p] = kl[s];
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < E; ++s) {
+      const int p = lane * E + s;
+      if (p < K) {
+        const uint32_t h = static_cast<uint32_t>(k[s] >> 32), lw = static_cast<uint32_t>(k[s]);
+        int r = 0;
+        for (int q = 0; q < K; ++q) {
+          const uint32_t hq = static_cast<uint32_t>(sel[q] >> 32), lq = static_cast<uint32_t>(sel[q]);
+          r += hq > h || (hq == h && (tie[q] > kl[s] || (tie[q] == kl[s] && lq > lw)));
+        }
+        io[r] = static_cast<int32_t>(0xFFFFFFFFu - lw);
+        wo[r] = ev[s] * inv_z;
+      }
+    }
+  }
+}
+
 // E: winners sort width / 32; EH: half sort width / 32 (1 when sqrtN <= 32);
 // EPL: half values per lane when sqrtN > 32*EH; CP: candidates per lane.
 template <typename Tin, int E, int EH, int EPL, int CP>
@@ -334,220 +548,14 @@ __global__ void __launch_bounds__(kFastTopkWarps * kWarp) k_pkm_topk_fast(const 
                                                                           float* __restrict__ w_out) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x / kWarp;
-  const int lane = lane_id();
-  const int n = L.n, K = L.K, Kh = L.Kh, C = L.C;
-  constexpr int SZ = kWarp * kFastTopkMaxK / kWarp;  // stride of the two halves in hv/hx
-
   uint16_t* tab = reinterpret_cast<uint16_t*>(smem);  // candidate c -> (ra, rb)
-  if (warp == 0) {
-    int base = 0;
-    for (int r0 = 0; r0 < Kh; r0 += kWarp) {
-      const int ra = r0 + lane;
-      const int len = ra < Kh ? min(Kh, K / (ra + 1)) : 0;
-      int incl = len;
-#pragma unroll
-      for (int o = 1; o < kWarp; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      const int start = base + incl - len;
-      for (int rb = 0; rb < len; ++rb) {
-        tab[2 * (start + rb)] = static_cast<uint16_t>(ra);
-        tab[2 * (start + rb) + 1] = static_cast<uint16_t>(rb);
-      }
-      base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
-    }
-  }
+  if (warp == 0) fast_topk_build_table(tab, L.Kh, L.K, lane_id());
   __syncthreads();
-
   unsigned char* ws = smem + L.table_bytes + static_cast<size_t>(warp) * L.warp_bytes;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + L.hist);
-  uint64_t* sel = reinterpret_cast<uint64_t*>(ws + L.sel);
-  float* hv = reinterpret_cast<float*>(ws + L.hv);
-  int32_t* hx = reinterpret_cast<int32_t*>(ws + L.hx);
-  uint32_t* tie = reinterpret_cast<uint32_t*>(ws + L.tie);
-  const uint32_t lt = lanemask_lt();
-
   for (int64_t unit = static_cast<int64_t>(blockIdx.x) * kFastTopkWarps + warp; unit < n_units;
        unit += static_cast<int64_t>(gridDim.x) * kFastTopkWarps) {
-    const Tin* x = scores + unit * 2 * n;
-    warp_half_select<Tin, EH, EPL>(x, n, Kh, hist, sel, hv, hx);
-    warp_half_select<Tin, EH, EPL>(x + n, n, Kh, hist, sel, hv + SZ, hx + SZ);
-
-    // Candidates with exact scores: ck = ord(hi), cl = ~slot, clo = ord(lo).
-    uint32_t ck[CP], cl[CP], clo[CP];
-#pragma unroll
-    for (int j = 0; j < CP; ++j) {
-      const int c = j * kWarp + lane;
-      ck[j] = 0u;
-      cl[j] = 0u;
-      clo[j] = 0u;
-      if (c < C) {
-        const int ra = tab[2 * c], rb = tab[2 * c + 1];
-        float hi, lo;
-        two_sum(hv[ra], hv[SZ + rb], hi, lo);
-        ck[j] = ord_f32(canon_zero(hi));
-        clo[j] = ord_f32(canon_zero(lo));
-        cl[j] = 0xFFFFFFFFu - static_cast<uint32_t>(hx[ra] * n + hx[SZ + rb]);
-      }
-    }
-    // Winners by hi; a boundary that splits equal hi ranks that group by
-    // (lo desc, slot asc). Exact fp32 sums of bf16 inputs tie often, but such
-    // groups are small.
-    const SelectPlan sp = warp_select_plan<CP>(ck, K, hist, warp_kth_floor<CP>(ck, K));
-    const uint32_t tb = sp.thr >> sp.shift;
-    const bool split = sp.take_eq < sp.bin_count;  // only at shift 0, i.e. equal hi
-    int tie_rank[CP];
-#pragma unroll
-    for (int j = 0; j < CP; ++j) tie_rank[j] = 0;
-    if (split) {
-      int g = 0;
-#pragma unroll
-      for (int j = 0; j < CP; ++j) {
-        const bool eq = j * kWarp + lane < C && ck[j] == sp.thr;
-        const uint32_t be = __ballot_sync(0xffffffffu, eq);
-        if (eq) {
-          const int p = g + __popc(be & lt);
-          tie[2 * p] = clo[j];
-          tie[2 * p + 1] = cl[j];
-        }
-        g += __popc(be);
-      }
-      __syncwarp();
-#pragma unroll
-      for (int j = 0; j < CP; ++j) {
-        if (j * kWarp + lane < C && ck[j] == sp.thr) {
-          int r = 0;
-          for (int q = 0; q < g; ++q) {
-            const uint32_t lq = tie[2 * q], sq = tie[2 * q + 1];
-            r += (lq > clo[j]) || (lq == clo[j] && sq > cl[j]);
-          }
-          tie_rank[j] = r;
-        }
-      }
-      __syncwarp();
-    }
-    int cnt = 0;
-#pragma unroll
-    for (int j = 0; j < CP; ++j) {
-      const int c = j * kWarp + lane;
-      const uint32_t kb = ck[j] >> sp.shift;
-      const bool take = c < C && (kb > tb || (kb == tb && ck[j] >= sp.floor && (!split || tie_rank[j] < sp.take_eq)));
-      const uint32_t bt = __ballot_sync(0xffffffffu, take);
-      if (take) {
-        const int p = cnt + __popc(bt & lt);
-        sel[p] = (static_cast<uint64_t>(ck[j]) << 32) | cl[j];
-        hist[p] = clo[j];
-      }
-      cnt += __popc(bt);
-    }
-    __syncwarp();
-    // Order the K winners by ord(hi):(~slot), descending: each winner's rank is
-    // the number of winner keys above it (keys are distinct: the slot is part
-    // of the key), counted against all K keys read two at a time from shared
-    // memory; then every winner moves to its rank.
-    uint64_t k[E];
-    uint32_t kl[E];
-    {
-      uint64_t mine[E];
-      uint32_t mlo[E];
-      int rank[E];
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        const int p = lane * E + s;
-        mine[s] = p < K ? sel[p] : 0ull;
-        mlo[s] = p < K ? hist[p] : 0u;
-        rank[s] = 0;
-      }
-      const ulonglong2* sel2 = reinterpret_cast<const ulonglong2*>(sel);
-      for (int j = 0; j < K; j += 2) {
-        const ulonglong2 two = sel2[j >> 1];
-        const uint64_t second = j + 1 < K ? two.y : 0ull;  // past K: stale, never above a winner
-#pragma unroll
-        for (int s = 0; s < E; ++s) rank[s] += (two.x > mine[s]) + (second > mine[s]);
-      }
-      __syncwarp();
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        if (lane * E + s < K) {
-          sel[rank[s]] = mine[s];
-          hist[rank[s]] = mlo[s];
-        }
-      }
-      __syncwarp();
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        const int p = lane * E + s;
-        k[s] = p < K ? sel[p] : 0ull;
-        kl[s] = p < K ? hist[p] : 0u;
-      }
-      __syncwarp();
-    }
-    // Neighbours with equal hi but different lo need the (lo desc, slot asc) order.
-    bool fix = false;
-    {
-      const uint32_t nh = __shfl_down_sync(0xffffffffu, static_cast<uint32_t>(k[0] >> 32), 1);
-      const uint32_t nl = __shfl_down_sync(0xffffffffu, kl[0], 1);
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        const int p = lane * E + s;
-        if (p + 1 < K) {
-          const uint32_t h1 = s + 1 < E ? static_cast<uint32_t>(k[(s + 1) % E] >> 32) : nh;
-          const uint32_t l1 = s + 1 < E ? kl[(s + 1) % E] : nl;
-          fix = fix || (static_cast<uint32_t>(k[s] >> 32) == h1 && kl[s] != l1);
-        }
-      }
-    }
-    const bool any_fix = __any_sync(0xffffffffu, fix);
-    // Softmax of the selected scores (order independent).
-    const float top = unord_f32(__shfl_sync(0xffffffffu, static_cast<uint32_t>(k[0] >> 32), 0));
-    float ev[E];
-    float z = 0.f;
-#pragma unroll
-    for (int s = 0; s < E; ++s) {
-      const int p = lane * E + s;
-      ev[s] = p < K ? expf(unord_f32(static_cast<uint32_t>(k[s] >> 32)) - top) : 0.f;
-      z += ev[s];
-    }
-    z = warp_sum(z);
-    const float inv_z = 1.0f / z;
-    int32_t* io = idx_out + unit * K;
-    float* wo = w_out + unit * K;
-    if (!any_fix) {
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        const int p = lane * E + s;
-        if (p < K) {
-          io[p] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(k[s]));
-          wo[p] = ev[s] * inv_z;
-        }
-      }
-    } else {
-      // Rare: rank each winner by (hi desc, lo desc, slot asc).
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        const int p = lane * E + s;
-        if (p < K) {
-          sel[p] = k[s];
-          tie[p] = kl[s];
-        }
-      }
-      __syncwarp();
-#pragma unroll
-      for (int s = 0; s < E; ++s) {
-        const int p = lane * E + s;
-        if (p < K) {
-          const uint32_t h = static_cast<uint32_t>(k[s] >> 32), lw = static_cast<uint32_t>(k[s]);
-          int r = 0;
-          for (int q = 0; q < K; ++q) {
-            const uint32_t hq = static_cast<uint32_t>(sel[q] >> 32), lq = static_cast<uint32_t>(sel[q]);
-            r += hq > h || (hq == h && (tie[q] > kl[s] || (tie[q] == kl[s] && lq > lw)));
-          }
-          io[r] = static_cast<int32_t>(0xFFFFFFFFu - lw);
-          wo[r] = ev[s] * inv_z;
-        }
-      }
-    }
+    fast_topk_unit<Tin, E, EH, EPL, CP>(scores + unit * 2 * L.n, L, tab, ws, idx_out + unit * L.K,
+                                        w_out + unit * L.K);
     __syncwarp();
   }
 }

@@ -22,6 +22,7 @@
 #include "sdm_records.cuh"
 #include "sdm_scan.cuh"
 #include "sdm_backward.cuh"
+#include "sdm_decode.cuh"
 
 namespace {
 
@@ -104,6 +105,7 @@ void set_smem(const void* kern, size_t smem) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+size_t align16(size_t x) { return (x + 15) & ~static_cast<size_t>(15); }
 
 int64_t slots_of(int32_t sqrt_n) { return static_cast<int64_t>(sqrt_n) * sqrt_n; }
 
@@ -205,21 +207,24 @@ sdm_status_t launch_topk_fast_inst(const DeviceInfo& dev, const Tin* scores, int
   return launch_status("pkm_topk launch");
 }
 
-// Register path for K <= 64.
-template <typename Tin>
-sdm_status_t launch_topk_fast(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K,
-                              int32_t* idx, float* w, cudaStream_t st) {
+// Layout and template parameters of the register-path selection (K <= 64).
+struct FastTopkPlan {
   sdm::FastTopkLayout L{};
+  int E = 1, EH = 1, epl = 1, CP = 4;
+};
+sdm_status_t fast_topk_plan(int n, int K, FastTopkPlan* out) {
+  FastTopkPlan P;
+  sdm::FastTopkLayout& L = P.L;
   L.n = n;
   L.K = K;
   L.Kh = std::min(K, n);
   int C = 0;
   for (int ra = 0; ra < L.Kh; ++ra) C += std::min(L.Kh, K / (ra + 1));
   L.C = C;
-  const int E = K <= 32 ? 1 : 2;                 // winners sort width / 32
-  const int EH = n <= 32 ? 1 : E;                // half sort width / 32
-  const int CP = E == 1 ? 4 : (EH == 1 ? 7 : 9);
-  if (C > 32 * CP) return fail(SDM_ERR_UNSUPPORTED, "selection candidate count above the register path");
+  P.E = K <= 32 ? 1 : 2;                // winners sort width / 32
+  P.EH = n <= 32 ? 1 : P.E;             // half sort width / 32
+  P.CP = P.E == 1 ? 4 : (P.EH == 1 ? 7 : 9);
+  if (C > 32 * P.CP) return fail(SDM_ERR_UNSUPPORTED, "selection candidate count above the register path");
   auto a16 = [](uint32_t x) { return (x + 15u) & ~15u; };
   L.table_bytes = a16(static_cast<uint32_t>(C) * 4u);
   uint32_t off = 0;
@@ -232,13 +237,26 @@ sdm_status_t launch_topk_fast(const DeviceInfo& dev, const void* scores, int64_t
   L.sel = take(64u * 8u);
   L.hv = take(2u * 64u * 4u);
   L.hx = take(2u * 64u * 4u);
-  L.tie = take(2u * 4u * 32u * CP);
+  L.tie = take(2u * 4u * 32u * P.CP);
   L.warp_bytes = off;
-  const Tin* x = static_cast<const Tin*>(scores);
-  int epl = 1;
-  if (n > 32 * EH) {
-    while (epl * 32 < n) epl *= 2;
+  if (n > 32 * P.EH) {
+    while (P.epl * 32 < n) P.epl *= 2;
   }
+  *out = P;
+  return SDM_OK;
+}
+
+// Register path for K <= 64.
+template <typename Tin>
+sdm_status_t launch_topk_fast(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K,
+                              int32_t* idx, float* w, cudaStream_t st) {
+  FastTopkPlan P;
+  sdm_status_t r;
+  if ((r = fast_topk_plan(n, K, &P)) != SDM_OK) return r;
+  const sdm::FastTopkLayout& L = P.L;
+  const int E = P.E, EH = P.EH, CP = P.CP;
+  const Tin* x = static_cast<const Tin*>(scores);
+  const int epl = P.epl;
 #define SDM_FAST_TOPK(E_, EH_, EPL_, CP_)                      \
   if (E == E_ && EH == EH_ && epl == EPL_ && CP == CP_) \
     return launch_topk_fast_inst<Tin, E_, EH_, EPL_, CP_>(dev, x, units, L, idx, w, st);
@@ -648,6 +666,77 @@ sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStr
 
 }  // namespace
 
+// ---------------------------------------------------------------- decode --
+
+namespace {
+
+template <typename Tin, typename Tst, int E, int EH, int EPL, int CP>
+sdm_status_t launch_decode_inst(const sdm::DecodeArgs& a, size_t smem, int grid, cudaStream_t st) {
+  auto kern = sdm::k_decode_step<Tin, Tst, E, EH, EPL, CP>;
+  set_smem(reinterpret_cast<const void*>(kern), smem);
+  kern<<<grid, sdm::kDecodeThreads, smem, st>>>(a);
+  return launch_status("decode step launch");
+}
+
+template <typename Tin, typename Tst>
+sdm_status_t launch_decode_typed(const FastTopkPlan& P, const sdm::DecodeArgs& a, size_t smem, int grid,
+                                 cudaStream_t st) {
+#define SDM_DECODE(E_, EH_, EPL_, CP_)                                 \
+  if (P.E == E_ && P.EH == EH_ && P.epl == EPL_ && P.CP == CP_) \
+    return launch_decode_inst<Tin, Tst, E_, EH_, EPL_, CP_>(a, smem, grid, st);
+  SDM_DECODE(1, 1, 1, 4) SDM_DECODE(1, 1, 2, 4) SDM_DECODE(1, 1, 4, 4) SDM_DECODE(1, 1, 8, 4)
+  SDM_DECODE(1, 1, 16, 4) SDM_DECODE(1, 1, 32, 4)
+  SDM_DECODE(2, 1, 1, 7)
+  SDM_DECODE(2, 2, 1, 9) SDM_DECODE(2, 2, 4, 9) SDM_DECODE(2, 2, 8, 9)
+  SDM_DECODE(2, 2, 16, 9) SDM_DECODE(2, 2, 32, 9)
+#undef SDM_DECODE
+  return fail(SDM_ERR_UNSUPPORTED, "no decode kernel for this sqrt_n and K");
+}
+
+// The fused single-launch decode step (T = 1, W = R <= 64, automatic
+// variant). Sets *used = false (and returns SDM_OK) when the shape is not one
+// it covers, so the caller takes the general path.
+sdm_status_t try_decode_step(const DeviceInfo& dev, const sdm_shape_t& s, const void* kp, const void* qp,
+                             const void* v, const void* alpha, const void* beta, const void* g, void* M, float* y,
+                             cudaStream_t st, bool* used) {
+  *used = false;
+  if (s.T != 1 || s.W != s.R || s.W > sdm::kFastTopkMaxK || s.variant != SDM_VARIANT_AUTO) return SDM_OK;
+  if (static_cast<int64_t>(s.B) * s.H > 0x7FFFFFFFLL) return SDM_OK;
+  FastTopkPlan P;
+  if (fast_topk_plan(s.sqrt_n, s.W, &P) != SDM_OK) {
+    g_last_error.clear();
+    return SDM_OK;
+  }
+  const int VE = 16 / static_cast<int>(in_size(s.state_dtype));
+  const int UR = s.d_v / VE;
+  const int groups = UR >= sdm::kDecodeThreads ? 1 : sdm::kDecodeThreads / UR;
+  sdm::DecodeArgs a{};
+  a.H = s.H;
+  a.N = static_cast<int>(slots_of(s.sqrt_n));
+  a.d_v = s.d_v;
+  a.K = s.W;
+  a.eps = s.rms_eps;
+  a.L = P.L;
+  a.kp = kp; a.qp = qp; a.v = v; a.alpha = alpha; a.beta = beta; a.g = g; a.M = M; a.y = y;
+  a.sel_off = static_cast<uint32_t>(align16(P.L.table_bytes + 2ull * P.L.warp_bytes));
+  a.part_off = static_cast<uint32_t>(a.sel_off + align16(16ull * s.W));
+  a.err = dev.err;
+  const size_t smem = a.part_off + static_cast<size_t>(groups) * s.d_v * 4;
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return SDM_OK;
+  const int grid = s.B * s.H;
+  sdm_status_t r;
+  if (s.in_dtype == SDM_BF16)
+    r = s.state_dtype == SDM_BF16 ? launch_decode_typed<sdm::bf16, sdm::bf16>(P, a, smem, grid, st)
+                                  : launch_decode_typed<sdm::bf16, float>(P, a, smem, grid, st);
+  else
+    r = s.state_dtype == SDM_BF16 ? launch_decode_typed<float, sdm::bf16>(P, a, smem, grid, st)
+                                  : launch_decode_typed<float, float>(P, a, smem, grid, st);
+  if (r == SDM_OK) *used = true;
+  return r;
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t sdm_abi_version(void) { return SDM_ABI_VERSION; }
@@ -972,6 +1061,17 @@ sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const v
 
 size_t sdm_layer_step_workspace_bytes(const sdm_shape_t* shape) { return sdm_layer_forward_workspace_bytes(shape); }
 
+int32_t sdm_layer_step_launches(const sdm_shape_t* shape) {
+  const std::string saved = g_last_error;
+  if (check_shape(shape) != SDM_OK) return -1;
+  const sdm_shape_t& s = *shape;
+  FastTopkPlan P;
+  const bool fused = s.T == 1 && s.W == s.R && s.W <= sdm::kFastTopkMaxK && s.variant == SDM_VARIANT_AUTO &&
+                     fast_topk_plan(s.sqrt_n, s.W, &P) == SDM_OK;
+  g_last_error = saved;
+  return fused ? 1 : 4;  // else: two selections, records, recurrence
+}
+
 sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
                             const void* alpha, const void* beta, const void* g, void* M, float* y, void* workspace,
                             size_t workspace_bytes, void* stream) {
@@ -993,6 +1093,9 @@ sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, const void
   DeviceInfo* dev;
   if ((r = device_info(&dev)) != SDM_OK) return r;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bool fused = false;
+  if ((r = try_decode_step(*dev, s, kp, qp, v, alpha, beta, g, M, y, st, &fused)) != SDM_OK) return r;
+  if (fused) return ok();
   ScanChoice c;
   if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
   unsigned char* ws = static_cast<unsigned char*>(workspace);

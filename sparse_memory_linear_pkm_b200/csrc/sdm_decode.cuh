@@ -1,0 +1,138 @@
+// One decode step of the SDM layer in one launch (sm_100a).
+//
+// For T = 1 (a new token per batch row, the state carried across calls) the
+// whole layer is small and latency-bound: selection of k' and q' (SDM
+// explainer, section 3.1 step 1), the gated delta write (step 2), the read
+// after the write (step 3) and the optional RMS-norm x gate. One CTA per
+// (b, h) does all of it: warp 0 selects the W write slots, warp 1 the R read
+// slots (the register-path selection of pkm_topk_fast.cuh, same order and
+// weights as sdm_pkm_topk), then every thread updates 16-byte units of the W
+// written rows in global memory (m <- fma(alpha (1 - beta k), m, (beta k) v),
+// rounded to the state dtype on store, as the recurrence kernels do), and
+// after a barrier the R read rows are summed into y, each column's entries
+// split into groups whose partial sums are added in group order. Slots of one
+// token are distinct, so the writes need no ordering among themselves.
+#pragma once
+
+#include "pkm_topk_fast.cuh"
+#include "sdm_scan.cuh"
+
+namespace sdm {
+
+constexpr int kDecodeThreads = 256;
+
+struct DecodeArgs {
+  int H, N, d_v, K;  // K = W = R
+  float eps;
+  FastTopkLayout L;
+  const void* kp;     // [B, 1, H, 2 sqrtN] Tin
+  const void* qp;     // [B, 1, H, 2 sqrtN] Tin
+  const void* v;      // [B, 1, H, d_v] Tin
+  const void* alpha;  // [B, 1, H] Tin
+  const void* beta;   // [B, 1, H] Tin
+  const void* g;      // [B, 1, H, d_v] Tin or null
+  void* M;            // [B, H, N, d_v] Tst, updated in place
+  float* y;           // [B, 1, H, d_v]
+  uint32_t sel_off;   // byte offsets in shared memory
+  uint32_t part_off;
+  unsigned* err;
+};
+
+// Shared memory: candidate table | 2 selection scratches | idx_w, w_w, idx_r,
+// w_r [K] each | read partial sums [groups][d_v].
+template <typename Tin, typename Tst, int E, int EH, int EPL, int CP>
+__global__ void __launch_bounds__(kDecodeThreads) k_decode_step(DecodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int tid = threadIdx.x, warp = tid / kWarp;
+  const int bh = blockIdx.x;  // = b * H + h = the token-head of this step
+  const int K = a.K, N = a.N, d_v = a.d_v;
+  uint16_t* tab = reinterpret_cast<uint16_t*>(smem);
+  int32_t* sidx = reinterpret_cast<int32_t*>(smem + a.sel_off);  // [2K]: write slots, then read slots
+  float* sw = reinterpret_cast<float*>(sidx + 2 * K);             // [2K]: their weights
+  float* part = reinterpret_cast<float*>(smem + a.part_off);
+
+  if (warp == 0) fast_topk_build_table(tab, a.L.Kh, K, lane_id());
+  __syncthreads();
+  if (warp < 2) {
+    const Tin* x = static_cast<const Tin*>(warp == 0 ? a.kp : a.qp) + static_cast<int64_t>(bh) * 2 * a.L.n;
+    unsigned char* ws = smem + a.L.table_bytes + static_cast<size_t>(warp) * a.L.warp_bytes;
+    fast_topk_unit<Tin, E, EH, EPL, CP>(x, a.L, tab, ws, sidx + warp * K, sw + warp * K);
+  }
+  __syncthreads();
+
+  constexpr int VE = 16 / static_cast<int>(sizeof(Tst));  // state columns per 16-byte unit
+  const int UR = d_v / VE;                                 // units per row
+  Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * N * d_v;
+  const Tin* vrow = static_cast<const Tin*>(a.v) + static_cast<int64_t>(bh) * d_v;
+  const float alpha = to_f32<Tin>(static_cast<const Tin*>(a.alpha)[bh]);
+  const float beta = to_f32<Tin>(static_cast<const Tin*>(a.beta)[bh]);
+
+  // Write: unit u of row idx_w[e], for every (e, u).
+  for (int x = tid; x < K * UR; x += kDecodeThreads) {
+    const int e = x / UR, u = x - e * UR;
+    const int s = sidx[e];
+    if (static_cast<unsigned>(s) >= static_cast<unsigned>(N)) {
+      atomicOr(a.err, kErrIndexOutOfRange);
+      continue;
+    }
+    const float cw = beta * sw[e];
+    const float aw = alpha * (1.0f - cw);
+    uint4* p = reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(s) * d_v + u * VE);
+    float m[VE], vv[VE];
+    unpack16<Tst>(*p, m);
+    load_in_vec<Tin, VE>(vrow + u * VE, vv);
+#pragma unroll
+    for (int j = 0; j < VE; ++j) m[j] = __fmaf_rn(aw, m[j], __fmul_rn(cw, vv[j]));
+    *p = pack16<Tst>(m);
+  }
+  __syncthreads();
+
+  // Read: groups of entries per unit, partial sums in shared memory.
+  const int groups = UR >= kDecodeThreads ? 1 : kDecodeThreads / UR;
+  for (int x = tid; x < groups * UR; x += kDecodeThreads) {
+    const int gi = x / UR, u = x - gi * UR;
+    float acc[VE];
+#pragma unroll
+    for (int j = 0; j < VE; ++j) acc[j] = 0.0f;
+    for (int e = gi; e < K; e += groups) {
+      const int s = sidx[K + e];
+      if (static_cast<unsigned>(s) >= static_cast<unsigned>(N)) {
+        atomicOr(a.err, kErrIndexOutOfRange);
+        continue;
+      }
+      const float q = sw[K + e];
+      float m[VE];
+      unpack16<Tst>(*reinterpret_cast<const uint4*>(Mbh + static_cast<int64_t>(s) * d_v + u * VE), m);
+#pragma unroll
+      for (int j = 0; j < VE; ++j) acc[j] = __fmaf_rn(q, m[j], acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < VE; ++j) part[gi * d_v + u * VE + j] = acc[j];
+  }
+  __syncthreads();
+  float* yrow = a.y + static_cast<int64_t>(bh) * d_v;
+  float ss = 0.0f;
+  for (int c = tid; c < d_v; c += kDecodeThreads) {
+    float acc = 0.0f;
+    for (int gi = 0; gi < groups; ++gi) acc += part[gi * d_v + c];
+    part[c] = acc;  // group 0's slot is read only by this thread
+    ss = __fmaf_rn(acc, acc, ss);
+  }
+  if (a.g == nullptr) {
+    for (int c = tid; c < d_v; c += kDecodeThreads) yrow[c] = part[c];
+    return;
+  }
+  // RMS-norm x gate over the row (the epilogue kernel's formula).
+  __shared__ float red[kDecodeThreads / kWarp];
+  ss = warp_sum(ss);
+  if (lane_id() == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kDecodeThreads / kWarp; ++w) tot += red[w];
+  const float inv = 1.0f / sqrtf(tot / static_cast<float>(d_v) + a.eps);
+  const Tin* grow = static_cast<const Tin*>(a.g) + static_cast<int64_t>(bh) * d_v;
+  for (int c = tid; c < d_v; c += kDecodeThreads) yrow[c] = to_f32<Tin>(grow[c]) * part[c] * inv;
+}
+
+}  // namespace sdm

@@ -131,3 +131,11 @@ def test_backward_workspace_and_support_without_gpu(lib):
     assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == log + part + rec + work
     assert lib.sdm_pkm_topk_backward(None, None, None, 1, 2, 1, 4, 3, None, None) == 1
     assert lib.sdm_pkm_topk_backward(None, None, None, 0, 2, 1, 4, 3, None, None) == 0
+
+
+def test_layer_step_launch_count(lib):
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=8))) == 1  # single-launch decode
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=2, W=8, R=8))) == 4
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=4))) == 4
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=8, variant=2))) == 4
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(sqrt_n=0))) == -1

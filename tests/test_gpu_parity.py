@@ -257,6 +257,33 @@ def test_layer_step_chain(sdm, oracle, cuda_device, name, steps):
     assert_rel_close(y.cpu().numpy(), oy, tol, "y (steps vs oracle)")
 
 
+@pytest.mark.parametrize("name,W,R,gate", [("d2048_h16_n1024_dv128", 64, 64, True), ("tiny_n1024_dv16", 8, 8, False),
+                                          ("d2048_h4_n16384_dv512", 64, 64, True),
+                                          ("long_t1m_n262144_dv2048", 64, 64, False),
+                                          ("d2048_h16_n1024_dv128", 16, 16, False)])
+def test_decode_step_single_launch_matches_general_path(sdm, cuda_device, name, W, R, gate):
+    """T = 1 calls with the automatic variant run the single-launch decode
+    kernel; they give the same state bit for bit as the general path (forced
+    streaming variant) and y up to summation order, with and without the
+    RMS-norm x gate."""
+    shape = synth.WORKLOADS[name].replace(B=2, T=5, H=3, W=W, R=R)
+    if name == "long_t1m_n262144_dv2048":
+        shape = shape.replace(B=1, H=1)
+    inp = synth.make_inputs(shape, seed=31, device="cpu", with_gate=gate)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    M_a = d["M0"].unsqueeze(0).repeat(shape.B, 1, 1, 1).contiguous()
+    M_b = M_a.clone()
+    for t in range(shape.T):
+        sl = {k: d[k][:, t:t + 1].contiguous() for k in ("kp", "qp", "v", "alpha", "beta")}
+        g = d["g"][:, t:t + 1].contiguous() if gate else None
+        ya = sdm.layer_step(sl["kp"], sl["qp"], sl["v"], sl["alpha"], sl["beta"], M_a, W, R, g=g)
+        yb = sdm.layer_step(sl["kp"], sl["qp"], sl["v"], sl["alpha"], sl["beta"], M_b, W, R, g=g,
+                            variant="streaming")
+        sdm.stream_check()
+        assert torch.equal(M_a, M_b), f"state differs after token {t}"
+        assert_rel_close(ya.cpu().numpy(), yb.cpu().numpy(), 1e-5, f"y of token {t}")
+
+
 def test_layer_forward_tiny_workload_full(sdm, oracle, cuda_device):
     _layer_case(sdm, oracle, cuda_device, synth.WORKLOADS["tiny_n1024_dv16"], seed=0)
 
