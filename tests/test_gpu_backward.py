@@ -29,6 +29,7 @@ BWD = [
     (16, 48, 12, 4, "f32", 1, 1, 3, True),  # one token
     (32, 16, 8, 8, "f32", 256, 1, 2, False),  # T a multiple of the chunk
     (8, 32, 5, 4, "bf16", 70, 2, 1, False),  # W + R odd: padded staging
+    (16, 32, 128, 96, "f32", 20, 1, 2, False),  # W, R above 64: several rounds of entries per lane
     # N = 16384: state and adjoint tiles in global memory
     (128, 64, 16, 16, "bf16", 150, 1, 2, False),  # 32-column tiles, one chunk
     (128, 48, 8, 8, "f32", 70, 2, 1, True),  # d_v not a multiple of 32: 16-column tiles
