@@ -4,14 +4,15 @@
 // whole layer is small and latency-bound: selection of k' and q' (SDM
 // explainer, section 3.1 step 1), the gated delta write (step 2), the read
 // after the write (step 3) and the optional RMS-norm x gate. One CTA per
-// (b, h) does all of it: warp 0 selects the W write slots, warp 1 the R read
-// slots (the register-path selection of pkm_topk_fast.cuh, same order and
-// weights as sdm_pkm_topk), then every thread updates 16-byte units of the W
-// written rows in global memory (m <- fma(alpha (1 - beta k), m, (beta k) v),
-// rounded to the state dtype on store, as the recurrence kernels do), and
-// after a barrier the R read rows are summed into y, each column's entries
-// split into groups whose partial sums are added in group order. Slots of one
-// token are distinct, so the writes need no ordering among themselves.
+// (b, h) does all of it: warp 0 selects the W write slots (the register-path
+// selection of pkm_topk_fast.cuh, same order and weights as sdm_pkm_topk);
+// then warps 0 and 2..7 update the 16-byte units of the W written rows in
+// global memory (m <- fma(alpha (1 - beta k), m, (beta k) v), rounded to the
+// state dtype on store, as the recurrence kernels do) while warp 1 selects the
+// R read slots; after a barrier the R read rows are summed into y, each
+// column's entries split into groups whose partial sums are added in group
+// order. Slots of one token are distinct, so the writes need no ordering
+// among themselves and their loads can all be issued before any store.
 #pragma once
 
 #include "pkm_topk_fast.cuh"
@@ -53,37 +54,60 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_step(DecodeArgs a) {
 
   if (warp == 0) fast_topk_build_table(tab, a.L.Kh, K, lane_id());
   __syncthreads();
-  if (warp < 2) {
-    const Tin* x = static_cast<const Tin*>(warp == 0 ? a.kp : a.qp) + static_cast<int64_t>(bh) * 2 * a.L.n;
-    unsigned char* ws = smem + a.L.table_bytes + static_cast<size_t>(warp) * a.L.warp_bytes;
-    fast_topk_unit<Tin, E, EH, EPL, CP>(x, a.L, tab, ws, sidx + warp * K, sw + warp * K);
-  }
-  __syncthreads();
-
   constexpr int VE = 16 / static_cast<int>(sizeof(Tst));  // state columns per 16-byte unit
   const int UR = d_v / VE;                                 // units per row
   Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * N * d_v;
-  const Tin* vrow = static_cast<const Tin*>(a.v) + static_cast<int64_t>(bh) * d_v;
-  const float alpha = to_f32<Tin>(static_cast<const Tin*>(a.alpha)[bh]);
-  const float beta = to_f32<Tin>(static_cast<const Tin*>(a.beta)[bh]);
-
-  // Write: unit u of row idx_w[e], for every (e, u).
-  for (int x = tid; x < K * UR; x += kDecodeThreads) {
-    const int e = x / UR, u = x - e * UR;
-    const int s = sidx[e];
-    if (static_cast<unsigned>(s) >= static_cast<unsigned>(N)) {
-      atomicOr(a.err, kErrIndexOutOfRange);
-      continue;
-    }
-    const float cw = beta * sw[e];
-    const float aw = alpha * (1.0f - cw);
-    uint4* p = reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(s) * d_v + u * VE);
-    float m[VE], vv[VE];
-    unpack16<Tst>(*p, m);
-    load_in_vec<Tin, VE>(vrow + u * VE, vv);
+  if (warp == 1) {
+    // The read selection runs while the other warps apply the writes.
+    unsigned char* ws = smem + a.L.table_bytes + a.L.warp_bytes;
+    fast_topk_unit<Tin, E, EH, EPL, CP>(static_cast<const Tin*>(a.qp) + static_cast<int64_t>(bh) * 2 * a.L.n, a.L,
+                                        tab, ws, sidx + K, sw + K);
+  } else {
+    if (warp == 0)
+      fast_topk_unit<Tin, E, EH, EPL, CP>(static_cast<const Tin*>(a.kp) + static_cast<int64_t>(bh) * 2 * a.L.n,
+                                          a.L, tab, smem + a.L.table_bytes, sidx, sw);
+    // Warps 0 and 2..7 meet once the write slots are known.
+    asm volatile("bar.sync 1, %0;\n" ::"r"(kDecodeThreads - kWarp) : "memory");
+    const Tin* vrow = static_cast<const Tin*>(a.v) + static_cast<int64_t>(bh) * d_v;
+    const float alpha = to_f32<Tin>(static_cast<const Tin*>(a.alpha)[bh]);
+    const float beta = to_f32<Tin>(static_cast<const Tin*>(a.beta)[bh]);
+    const int tw = warp == 0 ? tid : tid - kWarp;  // 0 .. 223
+    constexpr int kWriters = kDecodeThreads - kWarp;
+    constexpr int kBatch = 8;  // units loaded before any is stored (the rows are distinct)
+    // Write: unit u of row idx_w[e], for every (e, u).
+    for (int x0 = tw; x0 < K * UR; x0 += kWriters * kBatch) {
+      uint4 raw[kBatch];
+      int sl[kBatch];
 #pragma unroll
-    for (int j = 0; j < VE; ++j) m[j] = __fmaf_rn(aw, m[j], __fmul_rn(cw, vv[j]));
-    *p = pack16<Tst>(m);
+      for (int j = 0; j < kBatch; ++j) {
+        const int x = x0 + j * kWriters;
+        sl[j] = -1;
+        if (x < K * UR) {
+          const int e = x / UR, u = x - e * UR;
+          const int s = sidx[e];
+          if (static_cast<unsigned>(s) < static_cast<unsigned>(N)) {
+            sl[j] = s;
+            raw[j] = *reinterpret_cast<const uint4*>(Mbh + static_cast<int64_t>(s) * d_v + u * VE);
+          } else {
+            atomicOr(a.err, kErrIndexOutOfRange);
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (sl[j] < 0) continue;
+        const int x = x0 + j * kWriters;
+        const int e = x / UR, u = x - e * UR;
+        const float cw = beta * sw[e];
+        const float aw = alpha * (1.0f - cw);
+        float m[VE], vv[VE];
+        unpack16<Tst>(raw[j], m);
+        load_in_vec<Tin, VE>(vrow + u * VE, vv);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) m[i] = __fmaf_rn(aw, m[i], __fmul_rn(cw, vv[i]));
+        *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(sl[j]) * d_v + u * VE) = pack16<Tst>(m);
+      }
+    }
   }
   __syncthreads();
 
