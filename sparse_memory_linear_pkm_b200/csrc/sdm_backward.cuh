@@ -89,7 +89,8 @@ __host__ __device__ inline BwdStage bwd_stage(int W, int rec_words, int U, int i
 struct BwdTok {
   const float4* log;  // row e of the log at log[e * U]
   const uint32_t* rec;
-  const float4* v;    // U units of v_t (fp32)
+  const float4* v;    // U units of v_t (fp32; U > 1)
+  float4 v0;          // v_t itself when U = 1
   const float4* dy;   // U units of dy_t
   float alpha, beta;
 };
@@ -177,12 +178,18 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
     cp_async_wait<kBwdStages - 1>();
     __syncwarp();
     float* st = ring + (i % kBwdStages) * L.words;
-    if (lane < 4 * U) st[L.vf + lane] = to_f32<Tin>(reinterpret_cast<const Tin*>(st + L.v)[lane]);
-    __syncwarp();
+    if constexpr (U > 1) {  // v widened to fp32 once per token in shared memory
+      if (lane < 4 * U) st[L.vf + lane] = to_f32<Tin>(reinterpret_cast<const Tin*>(st + L.v)[lane]);
+      __syncwarp();
+    }
     BwdTok k;
     k.log = reinterpret_cast<const float4*>(st + L.log);
     k.rec = reinterpret_cast<const uint32_t*>(st + L.rec);
     k.v = reinterpret_cast<const float4*>(st + L.vf);
+    if constexpr (U == 1) {  // one unit: widened straight into registers
+      const Tin* vv = reinterpret_cast<const Tin*>(st + L.v);
+      k.v0 = make_float4(to_f32<Tin>(vv[0]), to_f32<Tin>(vv[1]), to_f32<Tin>(vv[2]), to_f32<Tin>(vv[3]));
+    }
     k.dy = reinterpret_cast<const float4*>(st + L.dy);
     k.alpha = __uint_as_float(k.rec[a.rl.off_ab]);
     k.beta = __uint_as_float(k.rec[a.rl.off_ab + 1]);
@@ -230,7 +237,7 @@ __device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok
       float4* r = Ms.row(s[q]);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const float4 vv = k.v[u];
+        const float4 vv = U == 1 ? k.v0 : k.v[u];
         if (log != nullptr) log[e * U + u] = m[q][u];
         r[u] = make_float4(__fmaf_rn(aw[q], m[q][u].x, __fmul_rn(cw[q], vv.x)),
                            __fmaf_rn(aw[q], m[q][u].y, __fmul_rn(cw[q], vv.y)),
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
                 for (int u = 0; u < U; ++u) {
                   const float4 gg = g[qq][u];
                   da += dot4(gg, m[qq][u]);
-                  dc += dot4(gg, k.v[u]);
+                  dc += dot4(gg, U == 1 ? k.v0 : k.v[u]);
                   dv[u].x = __fmaf_rn(cw, gg.x, dv[u].x);
                   dv[u].y = __fmaf_rn(cw, gg.y, dv[u].y);
                   dv[u].z = __fmaf_rn(cw, gg.z, dv[u].z);
