@@ -100,6 +100,11 @@ class Oracle:
         ]
         lib.oracle_pkm_topk_backward.restype = ctypes.c_int
         lib.oracle_pkm_topk_backward.argtypes = [_c_i64, _c_i32, _c_i32, _c_ptr, _c_ptr, _c_ptr, _c_ptr]
+        lib.oracle_rmsnorm_gate.restype = ctypes.c_int
+        lib.oracle_rmsnorm_gate.argtypes = [_c_i64, _c_i32, _c_ptr, _c_ptr, ctypes.c_double]
+        lib.oracle_rmsnorm_gate_backward.restype = ctypes.c_int
+        lib.oracle_rmsnorm_gate_backward.argtypes = [_c_i64, _c_i32, _c_ptr, _c_ptr, _c_ptr, ctypes.c_double,
+                                                     _c_ptr, _c_ptr]
         lib.oracle_round_to_bf16.restype = ctypes.c_float
         lib.oracle_round_to_bf16.argtypes = [ctypes.c_double]
         self.lib = lib
@@ -206,6 +211,27 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_pkm_topk_backward failed with code {rc}")
         return ds
+
+    def rmsnorm_gate(self, x, g, eps: float = 1e-6):
+        """The epilogue alone: g * x / sqrt(mean(x^2) + eps) over the last axis (double)."""
+        y = _f64(x).copy()
+        gg = _f64(g)
+        d_v = y.shape[-1]
+        rc = self.lib.oracle_rmsnorm_gate(y.size // d_v, d_v, _p(y), _p(gg), float(eps))
+        if rc != 0:
+            raise ValueError("oracle_rmsnorm_gate failed")
+        return y
+
+    def rmsnorm_gate_backward(self, x, g, dout, eps: float = 1e-6):
+        """(dL/dx, dL/dg) of the epilogue for dL/dout; x is the row before it."""
+        x, g, dout = _f64(x), _f64(g), _f64(dout)
+        d_v = x.shape[-1]
+        dx, dg = np.zeros_like(x), np.zeros_like(x)
+        rc = self.lib.oracle_rmsnorm_gate_backward(x.size // d_v, d_v, _p(x), _p(g), _p(dout), float(eps), _p(dx),
+                                                   _p(dg))
+        if rc != 0:
+            raise ValueError("oracle_rmsnorm_gate_backward failed")
+        return dx, dg
 
     # -- whole layer ---------------------------------------------------------
     def layer_forward(self, kp, qp, v, alpha, beta, M0, W: int, R: int, g=None,

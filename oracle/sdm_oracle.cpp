@@ -170,6 +170,20 @@ void select_one(const float* x, int32_t sqrt_n, int32_t K, std::vector<SlotScore
   }
 }
 
+// The epilogue on one row ([explainer] 3.1 step 3, "RMS-Norm" then the
+// element-wise gate g): y <- g * y / sqrt(mean(y^2) + eps), in double.
+template <class G>
+void rmsnorm_gate_row(double* y, const G* g, int32_t d_v, double eps) {
+  double ss = 0.0;
+  for (int32_t c = 0; c < d_v; ++c) ss += y[c] * y[c];
+#if ORACLE_MUTANT == 9
+  const double inv = 1.0 / std::sqrt(ss + eps);  // planted: sum instead of mean
+#else
+  const double inv = 1.0 / std::sqrt(ss / d_v + eps);
+#endif
+  for (int32_t c = 0; c < d_v; ++c) y[c] = static_cast<double>(g[c]) * y[c] * inv;
+}
+
 // Stores a freshly computed state value: rounded to fp32 (or to bf16 and kept
 // as an exact fp32) in a float state; kept exactly in a double state.
 template <class S>
@@ -277,15 +291,7 @@ int scan_impl(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W
   // Optional epilogue: RMS-norm over d_v per token-head, then the element-wise gate.
   if (g != nullptr) {
     parallel_for(static_cast<int64_t>(B) * T * H, std::max(1, n_threads), [&](int64_t th) {
-      double* y_t = y + th * d_v;
-      double ss = 0.0;
-      for (int32_t c = 0; c < d_v; ++c) ss += y_t[c] * y_t[c];
-#if ORACLE_MUTANT == 9
-      const double inv = 1.0 / std::sqrt(ss + eps);  // planted: sum instead of mean
-#else
-      const double inv = 1.0 / std::sqrt(ss / d_v + eps);
-#endif
-      for (int32_t c = 0; c < d_v; ++c) y_t[c] = static_cast<double>(g[th * d_v + c]) * y_t[c] * inv;
+      rmsnorm_gate_row(y + th * d_v, g + th * d_v, d_v, eps);
     });
   }
   if (op_count != nullptr) *op_count = ops.load();
@@ -498,6 +504,42 @@ int oracle_pkm_topk_backward(int64_t n_units, int32_t sqrt_n, int32_t K, const i
       ds[id[k] / sqrt_n] += dsig;
       ds[sqrt_n + id[k] % sqrt_n] += dsig;
 #endif
+    }
+  }
+  return 0;
+}
+
+// The epilogue alone on n_rows rows of d_v (double): y <- g * y / rms(y).
+int oracle_rmsnorm_gate(int64_t n_rows, int32_t d_v, double* y, const double* g, double eps) {
+  if (n_rows < 0 || d_v < 1) return -1;
+  for (int64_t r = 0; r < n_rows; ++r) rmsnorm_gate_row(y + r * d_v, g + r * d_v, d_v, eps);
+  return 0;
+}
+
+// Its derivatives for dL/dout: with x the row before the epilogue,
+// r = sqrt(mean(x^2) + eps) and out = g * x / r,
+//   dL/dx_j = g_j dout_j / r - x_j * sum_i(g_i dout_i x_i) / (d_v r^3)
+//   dL/dg_i = dout_i x_i / r.
+int oracle_rmsnorm_gate_backward(int64_t n_rows, int32_t d_v, const double* x, const double* g, const double* dout,
+                                 double eps, double* dx, double* dg) {
+  if (n_rows < 0 || d_v < 1) return -1;
+  for (int64_t r = 0; r < n_rows; ++r) {
+    const double* xr = x + r * d_v;
+    const double* gr = g + r * d_v;
+    const double* dr = dout + r * d_v;
+    double ss = 0.0, dot = 0.0;
+    for (int32_t c = 0; c < d_v; ++c) {
+      ss += xr[c] * xr[c];
+      dot += gr[c] * dr[c] * xr[c];
+    }
+    const double rms = std::sqrt(ss / d_v + eps);
+    for (int32_t c = 0; c < d_v; ++c) {
+#if ORACLE_MUTANT == 18
+      dx[r * d_v + c] = gr[c] * dr[c] / rms;  // planted: the normaliser treated as a constant
+#else
+      dx[r * d_v + c] = gr[c] * dr[c] / rms - xr[c] * dot / (d_v * rms * rms * rms);
+#endif
+      dg[r * d_v + c] = dr[c] * xr[c] / rms;
     }
   }
   return 0;

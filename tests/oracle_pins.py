@@ -469,6 +469,28 @@ def pin_topk_backward(o):
             assert abs(fd - ds[u, j]) <= 1e-5 * (1.0 + abs(ds[u, j])), (u, j, fd, ds[u, j])
 
 
+def pin_epilogue_backward(o):
+    """The epilogue's derivatives: a hand-worked row (tests/golden/epilogue_backward.json) and central
+    differences of the double-precision epilogue along random directions in x and g."""
+    data = json.loads((GOLDEN / "epilogue_backward.json").read_text())
+    dx, dg = o.rmsnorm_gate_backward(np.array([data["x"]]), np.array([data["g"]]), np.array([data["dout"]]),
+                                     eps=data["eps"])
+    assert np.array_equal(dx[0], np.array(data["dx"])) and np.array_equal(dg[0], np.array(data["dg"])), (dx, dg)
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((3, 5))
+    g = rng.standard_normal((3, 5))
+    dout = rng.standard_normal((3, 5))
+    dx, dg = o.rmsnorm_gate_backward(x, g, dout, eps=1e-3)
+    loss = lambda xx, gg: float(np.sum(dout * o.rmsnorm_gate(xx, gg, eps=1e-3)))
+    h = 1e-6
+    for _ in range(4):
+        D = rng.standard_normal(x.shape)
+        fd = (loss(x + h * D, g) - loss(x - h * D, g)) / (2 * h)
+        assert abs(fd - np.sum(dx * D)) <= 1e-6 * (1 + abs(fd)), ("dx", fd, np.sum(dx * D))
+        fd = (loss(x, g + h * D) - loss(x, g - h * D)) / (2 * h)
+        assert abs(fd - np.sum(dg * D)) <= 1e-6 * (1 + abs(fd)), ("dg", fd, np.sum(dg * D))
+
+
 ALL_PINS = {
     "selection_brute_force": pin_selection_brute_force,
     "selection_identity": pin_selection_identity,
@@ -490,6 +512,7 @@ ALL_PINS = {
     "backward_one_slot_golden": pin_backward_one_slot_golden,
     "backward_unselected_pass_through": pin_backward_unselected_pass_through,
     "topk_backward": pin_topk_backward,
+    "epilogue_backward": pin_epilogue_backward,
 }
 
 

@@ -33,6 +33,7 @@ MUTANTS = {
     15: "backward: dk without its m~ term",
     16: "backward: softmax mean not subtracted",
     17: "backward: score halves swapped",
+    18: "backward: RMS-norm normaliser treated as a constant",
 }
 
 
