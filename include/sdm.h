@@ -182,6 +182,47 @@ SDM_API sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* 
                                float* dM, float* dv, float* dalpha, float* dbeta, float* dw_w, float* dw_r,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* The RMS-norm x gate epilogue alone, in place ([explainer] 3.1 step 3):
+ * y <- g * y / sqrt(mean(y^2) + eps) over each of n_rows rows of d_v.
+ *   y [n_rows, d_v] fp32 (in/out); g [n_rows, d_v] in in_dtype (SDM_F32 or
+ *   SDM_BF16). sdm_layer_forward applies the same epilogue when given g;
+ *   training keeps the row before it (y_pre) by running the layer without g
+ *   and this afterwards. */
+SDM_API sdm_status_t sdm_rmsnorm_gate(float* y, const void* g, int32_t in_dtype, int64_t n_rows, int32_t d_v,
+                              float eps, void* stream);
+
+/* Backward of the epilogue for dout = dL/dout, with x = y_pre (the row
+ * before it), r = sqrt(mean(x^2) + eps):
+ *   dy_pre_j = g_j dout_j / r - x_j sum_i(g_i dout_i x_i) / (d_v r^3)
+ *   dg_i     = dout_i x_i / r
+ * y_pre, dout, dy_pre, dg: [n_rows, d_v] fp32; g in in_dtype. */
+SDM_API sdm_status_t sdm_rmsnorm_gate_backward(const float* y_pre, const void* g, int32_t in_dtype,
+                                       const float* dout, int64_t n_rows, int32_t d_v, float eps,
+                                       float* dy_pre, float* dg, void* stream);
+
+/* Bytes of workspace sdm_layer_backward needs (0 if unsupported; see
+ * sdm_scan_backward). */
+SDM_API size_t sdm_layer_backward_workspace_bytes(const sdm_shape_t* shape);
+
+/* Backward of the whole layer as sdm_layer_forward computes it with a shared
+ * initial state M0 [H,N,d_v] fp32: re-selects the slots of kp and qp
+ * (sdm_pkm_topk), then the epilogue's backward when g is given
+ * (sdm_rmsnorm_gate_backward on y_pre), the recurrence's
+ * (sdm_scan_backward), and both selection-weight backwards
+ * (sdm_pkm_topk_backward).
+ *   dy     [B,T,H,d_v] fp32: dL/d(layer output)
+ *   y_pre  [B,T,H,d_v] fp32: the layer output before the epilogue (only with g)
+ *   dM     [B,H,N,d_v] fp32: in dL/dM_T (zeros if unused), out dL/dM0 per
+ *          batch row (sum over b for M0's gradient)
+ *   dkp, dqp [B,T,H,2*sqrt_n]; dv [B,T,H,d_v]; dalpha, dbeta [B,T,H];
+ *   dg [B,T,H,d_v] (only with g): fp32 outputs, caller owned.
+ * Needs an fp32 state (shape.state_dtype SDM_F32). */
+SDM_API sdm_status_t sdm_layer_backward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                const void* alpha, const void* beta, const void* g, const float* M0,
+                                const float* y_pre, const float* dy, float* dM, float* dkp, float* dqp,
+                                float* dv, float* dalpha, float* dbeta, float* dg, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* Backward of the selection weights of sdm_pkm_topk for a fixed selection
  * ([explainer] 3.1 step 1: w = softmax of the K selected sums
  * sigma_k = s1[a_k] + s2[b_k], slot a_k * sqrt_n + b_k):

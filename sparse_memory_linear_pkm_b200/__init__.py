@@ -21,7 +21,7 @@ from . import native, synth
 from .native import SdmError
 
 __all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "scan_describe",
-           "scan_backward", "pkm_topk_backward", "stream_check", "make_shape",
+           "scan_backward", "pkm_topk_backward", "rmsnorm_gate", "rmsnorm_gate_backward", "layer_backward", "stream_check", "make_shape",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
 _DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
@@ -166,6 +166,57 @@ def pkm_topk_backward(idx: torch.Tensor, w: torch.Tensor, dw: torch.Tensor, sqrt
     native.check(native.load().sdm_pkm_topk_backward(_ptr(idx), _ptr(w), _ptr(dw), B, T, H, sqrt_n, K,
                                                       _ptr(dscores), _stream(idx.device)))
     return dscores
+
+
+def rmsnorm_gate(y: torch.Tensor, g: torch.Tensor, eps: float = 1e-6) -> torch.Tensor:
+    """The RMS-norm x gate epilogue in place on y [..., d_v] fp32; returns y."""
+    d_v = y.shape[-1]
+    native.check(native.load().sdm_rmsnorm_gate(_ptr(y), _ptr(g), _code(g, "g"), y.numel() // d_v, d_v,
+                                                float(eps), _stream(y.device)))
+    return y
+
+
+def rmsnorm_gate_backward(y_pre: torch.Tensor, g: torch.Tensor, dout: torch.Tensor, eps: float = 1e-6):
+    """(dL/dy_pre, dL/dg) of the epilogue for dL/dout; y_pre is the row before it."""
+    d_v = y_pre.shape[-1]
+    dy_pre = torch.empty_like(y_pre)
+    dg = torch.empty(y_pre.shape, dtype=torch.float32, device=y_pre.device)
+    native.check(native.load().sdm_rmsnorm_gate_backward(_ptr(y_pre), _ptr(g), _code(g, "g"), _ptr(dout),
+                                                         y_pre.numel() // d_v, d_v, float(eps), _ptr(dy_pre),
+                                                         _ptr(dg), _stream(y_pre.device)))
+    return dy_pre, dg
+
+
+def layer_backward(kp, qp, v, alpha, beta, M0, dy, W: int, R: int, g=None, y_pre=None, dM=None, eps: float = 1e-6,
+                   workspace: torch.Tensor | None = None) -> dict:
+    """Derivatives of the layer (selection, recurrence, optional epilogue)
+    for dy = dL/d(output) and dM = dL/dM_T (zeros when None); M0 [H,N,d_v]
+    fp32 is the shared initial state; y_pre (the output before the epilogue)
+    is needed with g. Returns dkp, dqp, dv, dalpha, dbeta, dM0 (per batch row)
+    and, with g, dg (all fp32)."""
+    B, T, H, two_n = kp.shape
+    d_v = v.shape[-1]
+    N = M0.shape[-2]
+    dev = kp.device
+    shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M0, "M0"), eps, 0)
+    lib = native.load()
+    if dM is None:
+        dM = torch.zeros((B, H, N, d_v), dtype=torch.float32, device=dev)
+    f = lambda *sh: torch.empty(sh, dtype=torch.float32, device=dev)
+    out = {"dkp": f(B, T, H, two_n), "dqp": f(B, T, H, two_n), "dv": f(B, T, H, d_v), "dalpha": f(B, T, H),
+           "dbeta": f(B, T, H)}
+    if g is not None:
+        out["dg"] = f(B, T, H, d_v)
+    need = int(lib.sdm_layer_backward_workspace_bytes(ctypes.byref(shape)))
+    if need == 0:
+        raise native.SdmError(2, lib.sdm_last_error().decode(errors="replace"))
+    ws = _workspace(need, dev, workspace)
+    native.check(lib.sdm_layer_backward(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha), _ptr(beta),
+                                        _ptr(g), _ptr(M0), _ptr(y_pre), _ptr(dy), _ptr(dM), _ptr(out["dkp"]),
+                                        _ptr(out["dqp"]), _ptr(out["dv"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]),
+                                        _ptr(out.get("dg")), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev)))
+    out["dM0"] = dM
+    return out
 
 
 def state_init(M0: torch.Tensor, B: int, out: torch.Tensor | None = None) -> torch.Tensor:

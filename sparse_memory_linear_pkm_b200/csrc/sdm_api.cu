@@ -904,6 +904,133 @@ sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, c
   return ok();
 }
 
+sdm_status_t sdm_rmsnorm_gate(float* y, const void* g, int32_t in_dtype, int64_t n_rows, int32_t d_v, float eps,
+                              void* stream) {
+  sdm_status_t r;
+  if ((r = check_dtype(in_dtype, "in_dtype")) != SDM_OK) return r;
+  if (n_rows < 0 || d_v < 1) return fail(SDM_ERR_INVALID_ARGUMENT, "n_rows must be >= 0 and d_v >= 1");
+  if (!(eps >= 0.0f)) return fail(SDM_ERR_INVALID_ARGUMENT, "eps must be >= 0");
+  if ((r = need_ptr(y, "y", n_rows > 0)) || (r = need_ptr(g, "g", n_rows > 0))) return r;
+  if (n_rows == 0) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const int grid = static_cast<int>(std::min<int64_t>((n_rows + 7) / 8, static_cast<int64_t>(dev->sms) * 16));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (in_dtype == SDM_BF16)
+    sdm::k_rmsnorm_gate<bf16><<<grid, 256, 0, st>>>(y, static_cast<const bf16*>(g), n_rows, d_v, eps);
+  else
+    sdm::k_rmsnorm_gate<float><<<grid, 256, 0, st>>>(y, static_cast<const float*>(g), n_rows, d_v, eps);
+  if ((r = launch_status("epilogue launch")) != SDM_OK) return r;
+  return ok();
+}
+
+sdm_status_t sdm_rmsnorm_gate_backward(const float* y_pre, const void* g, int32_t in_dtype, const float* dout,
+                                       int64_t n_rows, int32_t d_v, float eps, float* dy_pre, float* dg,
+                                       void* stream) {
+  sdm_status_t r;
+  if ((r = check_dtype(in_dtype, "in_dtype")) != SDM_OK) return r;
+  if (n_rows < 0 || d_v < 1) return fail(SDM_ERR_INVALID_ARGUMENT, "n_rows must be >= 0 and d_v >= 1");
+  if (!(eps >= 0.0f)) return fail(SDM_ERR_INVALID_ARGUMENT, "eps must be >= 0");
+  const bool any = n_rows > 0;
+  if ((r = need_ptr(y_pre, "y_pre", any)) || (r = need_ptr(g, "g", any)) || (r = need_ptr(dout, "dout", any)) ||
+      (r = need_ptr(dy_pre, "dy_pre", any)) || (r = need_ptr(dg, "dg", any)))
+    return r;
+  if (!any) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const int grid = static_cast<int>(std::min<int64_t>((n_rows + 7) / 8, static_cast<int64_t>(dev->sms) * 16));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (in_dtype == SDM_BF16)
+    sdm::k_rmsnorm_gate_backward<bf16><<<grid, 256, 0, st>>>(y_pre, static_cast<const bf16*>(g), dout, n_rows, d_v,
+                                                             eps, dy_pre, dg);
+  else
+    sdm::k_rmsnorm_gate_backward<float><<<grid, 256, 0, st>>>(y_pre, static_cast<const float*>(g), dout, n_rows,
+                                                              d_v, eps, dy_pre, dg);
+  if ((r = launch_status("epilogue backward launch")) != SDM_OK) return r;
+  return ok();
+}
+
+// Workspace of sdm_layer_backward: the two selections, their weight
+// derivatives, dL/dy before the epilogue, then sdm_scan_backward's.
+struct LayerBwdWs {
+  size_t idx_w, w_w, idx_r, w_r, dw_w, dw_r, dy_pre, scan, total;
+};
+LayerBwdWs layer_bwd_ws(const sdm_shape_t& s, size_t scan_bytes) {
+  const size_t th = static_cast<size_t>(s.B) * s.T * s.H;
+  LayerBwdWs L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.idx_w = take(th * s.W * 4);
+  L.w_w = take(th * s.W * 4);
+  L.idx_r = take(th * s.R * 4);
+  L.w_r = take(th * s.R * 4);
+  L.dw_w = take(th * s.W * 4);
+  L.dw_r = take(th * s.R * 4);
+  L.dy_pre = take(th * s.d_v * 4);
+  L.scan = take(scan_bytes);
+  L.total = off;
+  return L;
+}
+
+size_t sdm_layer_backward_workspace_bytes(const sdm_shape_t* shape) {
+  const std::string saved = g_last_error;
+  BwdChoice c;
+  if (check_shape(shape) != SDM_OK || choose_bwd(*shape, &c) != SDM_OK) return 0;
+  g_last_error = saved;
+  return layer_bwd_ws(*shape, c.total()).total;
+}
+
+sdm_status_t sdm_layer_backward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                const void* alpha, const void* beta, const void* g, const float* M0,
+                                const float* y_pre, const float* dy, float* dM, float* dkp, float* dqp, float* dv,
+                                float* dalpha, float* dbeta, float* dg, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  BwdChoice c;
+  if ((r = choose_bwd(s, &c)) != SDM_OK) return r;
+  const bool tok = static_cast<int64_t>(s.B) * s.T * s.H > 0;
+  if ((r = need_ptr(kp, "kp", tok)) || (r = need_ptr(qp, "qp", tok)) || (r = need_ptr(dkp, "dkp", tok)) ||
+      (r = need_ptr(dqp, "dqp", tok)))
+    return r;
+  if (g != nullptr && ((r = need_ptr(y_pre, "y_pre", tok)) || (r = need_ptr(dg, "dg", tok)))) return r;
+  const LayerBwdWs L = layer_bwd_ws(s, c.total());
+  if (workspace_bytes < L.total)
+    return fail(SDM_ERR_INVALID_ARGUMENT,
+                "workspace_bytes below sdm_layer_backward_workspace_bytes() = " + std::to_string(L.total));
+  if ((r = need_ptr(workspace, "workspace", true)) != SDM_OK) return r;
+  if (!tok) return sdm_scan_backward(shape, nullptr, nullptr, nullptr, nullptr, v, alpha, beta, M0, 1, dy, dM, dv,
+                                     dalpha, dbeta, nullptr, nullptr, nullptr, 0, stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(ws + L.idx_w);
+  float* w_w = reinterpret_cast<float*>(ws + L.w_w);
+  int32_t* idx_r = reinterpret_cast<int32_t*>(ws + L.idx_r);
+  float* w_r = reinterpret_cast<float*>(ws + L.w_r);
+  float* dw_w = reinterpret_cast<float*>(ws + L.dw_w);
+  float* dw_r = reinterpret_cast<float*>(ws + L.dw_r);
+  float* dy_pre = reinterpret_cast<float*>(ws + L.dy_pre);
+  if ((r = sdm_pkm_topk(kp, s.in_dtype, s.B, s.T, s.H, s.sqrt_n, s.W, idx_w, w_w, stream)) != SDM_OK) return r;
+  if ((r = sdm_pkm_topk(qp, s.in_dtype, s.B, s.T, s.H, s.sqrt_n, s.R, idx_r, w_r, stream)) != SDM_OK) return r;
+  const float* dy_scan = dy;
+  if (g != nullptr) {
+    if ((r = sdm_rmsnorm_gate_backward(y_pre, g, s.in_dtype, dy, static_cast<int64_t>(s.B) * s.T * s.H, s.d_v,
+                                       s.rms_eps, dy_pre, dg, stream)) != SDM_OK)
+      return r;
+    dy_scan = dy_pre;
+  }
+  if ((r = sdm_scan_backward(shape, idx_w, w_w, idx_r, w_r, v, alpha, beta, M0, 1, dy_scan, dM, dv, dalpha, dbeta,
+                             dw_w, dw_r, ws + L.scan, c.total(), stream)) != SDM_OK)
+    return r;
+  if ((r = sdm_pkm_topk_backward(idx_w, w_w, dw_w, s.B, s.T, s.H, s.sqrt_n, s.W, dkp, stream)) != SDM_OK) return r;
+  if ((r = sdm_pkm_topk_backward(idx_r, w_r, dw_r, s.B, s.T, s.H, s.sqrt_n, s.R, dqp, stream)) != SDM_OK) return r;
+  return ok();
+}
+
 sdm_status_t sdm_pkm_topk_backward(const int32_t* idx, const float* w, const float* dw, int32_t B, int32_t T,
                                    int32_t H, int32_t sqrt_n, int32_t K, float* dscores, void* stream) {
   sdm_status_t r;

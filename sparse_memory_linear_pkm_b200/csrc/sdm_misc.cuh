@@ -36,6 +36,40 @@ __global__ void __launch_bounds__(256) k_rmsnorm_gate(float* __restrict__ y, con
   }
 }
 
+// Backward of the RMS-norm x gate for dL/dout (x: the row before the
+// epilogue, r = sqrt(mean(x^2) + eps), out = g x / r):
+//   dL/dx_j = g_j dout_j / r - x_j sum_i(g_i dout_i x_i) / (d_v r^3),  dL/dg_i = dout_i x_i / r.
+// One warp per row; both row sums are reduced in a fixed order.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_rmsnorm_gate_backward(const float* __restrict__ x, const Tin* __restrict__ g,
+                                                               const float* __restrict__ dout, int64_t n_rows, int d_v,
+                                                               float eps, float* __restrict__ dx,
+                                                               float* __restrict__ dg) {
+  const int lane = lane_id();
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / kWarp);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / kWarp) + threadIdx.x / kWarp;
+       row < n_rows; row += warps) {
+    const float* xr = x + row * d_v;
+    const Tin* gr = g + row * d_v;
+    const float* dr = dout + row * d_v;
+    float ss = 0.f, dot = 0.f;
+    for (int c = lane; c < d_v; c += kWarp) {
+      ss = fmaf(xr[c], xr[c], ss);
+      dot = fmaf(to_f32<Tin>(gr[c]) * dr[c], xr[c], dot);
+    }
+    ss = warp_sum(ss);
+    dot = warp_sum(dot);
+    const float rms = sqrtf(ss / static_cast<float>(d_v) + eps);
+    const float inv = 1.0f / rms;
+    const float corr = dot * inv * inv * inv / static_cast<float>(d_v);
+    for (int c = lane; c < d_v; c += kWarp) {
+      const float gc = to_f32<Tin>(gr[c]);
+      dx[row * d_v + c] = gc * dr[c] * inv - xr[c] * corr;
+      dg[row * d_v + c] = dr[c] * xr[c] * inv;
+    }
+  }
+}
+
 // Slot utilisation: counts[b, h, i] += number of (t, k) with idx[b, t, h, k]
 // == i. A monitor of how the selection spreads over the N slots (uneven
 // addressing, the collapse onto few slots that the explainer page's

@@ -139,3 +139,19 @@ def test_layer_step_launch_count(lib):
     assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=4))) == 4
     assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=8, variant=2))) == 4
     assert lib.sdm_layer_step_launches(ctypes.byref(shape(sqrt_n=0))) == -1
+
+
+def test_layer_backward_arguments_without_gpu(lib):
+    s = shape(B=1, T=3, H=1, sqrt_n=8, W=4, R=4, d_v=32)
+    n = lib.sdm_layer_backward_workspace_bytes(ctypes.byref(s))
+    assert n > lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) > 0
+    fake = ctypes.c_void_p(1 << 20)
+    # g given without y_pre
+    st = lib.sdm_layer_backward(ctypes.byref(s), *([fake] * 6), fake, None, *([fake] * 8), fake, n, None)
+    assert st == 1 and b"y_pre" in lib.sdm_last_error()
+    # too little workspace
+    st = lib.sdm_layer_backward(ctypes.byref(s), *([fake] * 16), fake, 16, None)
+    assert st == 1 and b"workspace" in lib.sdm_last_error()
+    assert lib.sdm_rmsnorm_gate(None, None, native.F32, 2, 0, ctypes.c_float(1e-6), None) == 1
+    assert lib.sdm_rmsnorm_gate_backward(None, None, native.F32, None, 0, 8, ctypes.c_float(1e-6), None, None,
+                                         None) == 0

@@ -156,3 +156,52 @@ def test_scan_backward_full_size_sampled(sdm, oracle, cuda_device, name, pairs):
         for k in ("dv", "dalpha", "dbeta", "dw_w", "dw_r"):
             assert_rel_close(s(out[k]).cpu().numpy(), want[k], TOL_BWD, f"{k} (b={b}, h={h})")
         assert_rel_close(out["dM0"][b:b + 1, h:h + 1].cpu().numpy(), want["dM0"], TOL_BWD, f"dM0 (b={b}, h={h})")
+
+
+@pytest.mark.parametrize("gdtype", [torch.float32, torch.bfloat16])
+def test_rmsnorm_gate_and_backward_match_oracle(sdm, oracle, cuda_device, gdtype):
+    gen = torch.Generator().manual_seed(4)
+    x = torch.randn((3, 7, 2, 96), generator=gen)
+    g = torch.randn(x.shape, generator=gen).to(gdtype)
+    dout = torch.randn(x.shape, generator=gen)
+    y = sdm.rmsnorm_gate(x.to(cuda_device).clone(), g.to(cuda_device), eps=1e-6)
+    dx, dg = sdm.rmsnorm_gate_backward(x.to(cuda_device), g.to(cuda_device), dout.to(cuda_device), eps=1e-6)
+    sdm.stream_check()
+    assert_rel_close(y.cpu().numpy(), oracle.rmsnorm_gate(f32(x), f32(g), eps=1e-6), 1e-5, "epilogue")
+    wdx, wdg = oracle.rmsnorm_gate_backward(f32(x), f32(g), f32(dout), eps=1e-6)
+    assert_rel_close(dx.cpu().numpy(), wdx, 1e-5, "dL/dy_pre")
+    assert_rel_close(dg.cpu().numpy(), wdg, 1e-5, "dL/dg")
+
+
+@pytest.mark.parametrize("name,W,R,gate", [("d2048_h16_n1024_dv128", 64, 64, True), ("d2048_h16_n1024_dv128", 16, 8, False),
+                                          ("d2048_h4_n16384_dv512", 64, 64, True)])
+def test_layer_backward_matches_oracle(sdm, oracle, cuda_device, name, W, R, gate):
+    """sdm_layer_backward (selection, epilogue, recurrence and selection-weight
+    backwards in one call) against the oracle's pieces composed by hand."""
+    shape = synth.WORKLOADS[name].replace(B=2, T=37, H=2, W=W, R=R)
+    inp = synth.make_inputs(shape, seed=13, device="cpu", with_gate=gate)
+    gen = torch.Generator().manual_seed(14)
+    dy = torch.randn((shape.B, shape.T, shape.H, shape.d_v), generator=gen)
+    idx_w, w_w = oracle.pkm_topk(f32(inp["kp"]), W)
+    idx_r, w_r = oracle.pkm_topk(f32(inp["qp"]), R)
+    M0 = f32(inp["M0"])
+    M0b = np.broadcast_to(M0[None], (shape.B,) + M0.shape)
+    y_pre, _ = oracle.scan_f64(idx_w, w_w, idx_r, w_r, f32(inp["v"]), f32(inp["alpha"]), f32(inp["beta"]), M0b)
+    dy_scan = f32(dy).astype(np.float64)
+    if gate:
+        dy_scan, want_dg = oracle.rmsnorm_gate_backward(y_pre, f32(inp["g"]), f32(dy), eps=1e-6)
+    want = oracle.scan_backward(idx_w, w_w, idx_r, w_r, f32(inp["v"]), f32(inp["alpha"]), f32(inp["beta"]), M0b,
+                                dy_scan)
+    want_dkp = oracle.pkm_topk_backward(idx_w, w_w, want["dw_w"], shape.sqrt_n)
+    want_dqp = oracle.pkm_topk_backward(idx_r, w_r, want["dw_r"], shape.sqrt_n)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    got = sdm.layer_backward(d["kp"], d["qp"], d["v"], d["alpha"], d["beta"], d["M0"].float().contiguous(),
+                             dy.to(cuda_device), W, R, g=d.get("g"),
+                             y_pre=torch.from_numpy(y_pre.astype(np.float32)).to(cuda_device) if gate else None)
+    sdm.stream_check()
+    pairs = [("dkp", want_dkp), ("dqp", want_dqp), ("dv", want["dv"]), ("dalpha", want["dalpha"]),
+             ("dbeta", want["dbeta"]), ("dM0", want["dM0"])]
+    if gate:
+        pairs.append(("dg", want_dg))
+    for k, w_ in pairs:
+        assert_rel_close(got[k].cpu().numpy(), w_, TOL_BWD, k)
