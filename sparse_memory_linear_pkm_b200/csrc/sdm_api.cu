@@ -648,20 +648,25 @@ sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
   return SDM_OK;
 }
 
-template <typename Tin, int U, bool G>
+template <typename Tin, int U, bool G, int NWB>
 sdm_status_t launch_bwd_inst(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
-  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin, U, G>);
+  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin, U, G, NWB>);
   set_smem(kern, c.smem);
   const int64_t grid = static_cast<int64_t>(a.B) * a.H * c.ntile;
   if (grid > 0x7FFFFFFFLL) return fail(SDM_ERR_UNSUPPORTED, "too many column tiles for one launch");
-  sdm::k_scan_backward<Tin, U, G><<<static_cast<unsigned>(grid), 32, c.smem, st>>>(a);
+  sdm::k_scan_backward<Tin, U, G, NWB><<<static_cast<unsigned>(grid), NWB * 32, c.smem, st>>>(a);
   return launch_status("backward launch");
 }
 
 template <typename Tin>
 sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
-  if (!c.global) return launch_bwd_inst<Tin, 1, false>(c, a, st);
-  return c.U == 8 ? launch_bwd_inst<Tin, 8, true>(c, a, st) : launch_bwd_inst<Tin, 4, true>(c, a, st);
+  if (!c.global) {
+    // Two warps share each shared-memory tile (tuning override SDM_BWD_NWB=1: one).
+    const char* env = std::getenv("SDM_BWD_NWB");
+    if (env != nullptr && std::atoi(env) == 1) return launch_bwd_inst<Tin, 1, false, 1>(c, a, st);
+    return launch_bwd_inst<Tin, 1, false, 2>(c, a, st);
+  }
+  return c.U == 8 ? launch_bwd_inst<Tin, 8, true, 1>(c, a, st) : launch_bwd_inst<Tin, 4, true, 1>(c, a, st);
 }
 
 }  // namespace

@@ -134,11 +134,18 @@ __device__ __forceinline__ float dot4(const float4& a, const float4& b) {
   return __fmaf_rn(a.w, b.w, __fmaf_rn(a.z, b.z, __fmaf_rn(a.y, b.y, a.x * b.x)));
 }
 
+// The NWB warps that share one tile meet here (memory ordering included).
+template <int NWB>
+__device__ __forceinline__ void tile_sync() {
+  if constexpr (NWB == 1) __syncwarp();
+  else asm volatile("bar.sync 1, %0;\n" ::"n"(NWB * kWarp) : "memory");
+}
+
 // Runs body(t, token) over n tokens t = t_first + i * step of one (b, h) and
 // column tile, each with its stage filled (log rows from log_src when given,
 // dy when with_dy).
-template <typename Tin, int U, class Body>
-__device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, int tile, int lane, int t_first,
+template <typename Tin, int U, int NWB, class Body>
+__device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, int tile, int tid, int t_first,
                                                int step, int n, float* ring, const float* log_src, int log_t0,
                                                bool with_dy, Body body) {
   const BwdStage L = bwd_stage(a.W, a.rl.words, U, static_cast<int>(sizeof(Tin)));
@@ -152,21 +159,22 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
       const int64_t th = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
       float* st = ring + (i % kBwdStages) * L.words;
       const uint32_t* rsrc = a.rec + (static_cast<int64_t>(bh) * a.T + t) * a.rl.words;
-      for (int x = lane; x < n_rec; x += kWarp) cp_async16(st + L.rec + 4 * x, rsrc + 4 * x);
+      constexpr int NT = NWB * kWarp;
+      for (int x = tid; x < n_rec; x += NT) cp_async16(st + L.rec + 4 * x, rsrc + 4 * x);
       if (n_log > 0) {
         const float* lsrc = log_src + static_cast<int64_t>(t - log_t0) * a.W * 4 * U;
-        for (int x = lane; x < n_log; x += kWarp) cp_async16(st + L.log + 4 * x, lsrc + 4 * x);
+        for (int x = tid; x < n_log; x += NT) cp_async16(st + L.log + 4 * x, lsrc + 4 * x);
       }
       const char* vsrc = reinterpret_cast<const char*>(static_cast<const Tin*>(a.v) + th * a.d_v + tile * 4 * U);
       if constexpr (kVBytes >= 16) {
-        for (int x = lane; x < kVBytes / 16; x += kWarp)
+        for (int x = tid; x < kVBytes / 16; x += NT)
           cp_async16(reinterpret_cast<char*>(st + L.v) + 16 * x, vsrc + 16 * x);
       } else {
-        if (lane == kWarp - 1) cp_async8(st + L.v, vsrc);
+        if (tid == NT - 1) cp_async8(st + L.v, vsrc);
       }
       if (with_dy) {
         const float* dsrc = a.dy + th * a.d_v + tile * 4 * U;
-        for (int x = lane; x < U; x += kWarp) cp_async16(st + L.dy + 4 * x, dsrc + 4 * x);
+        for (int x = tid; x < U; x += NT) cp_async16(st + L.dy + 4 * x, dsrc + 4 * x);
       }
     }
     cp_async_commit();  // empty groups past the end keep the count uniform
@@ -176,11 +184,11 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
   for (int i = 0; i < n; ++i) {
     issue(i + kBwdStages - 1);
     cp_async_wait<kBwdStages - 1>();
-    __syncwarp();
+    tile_sync<NWB>();
     float* st = ring + (i % kBwdStages) * L.words;
     if constexpr (U > 1) {  // v widened to fp32 once per token in shared memory
-      if (lane < 4 * U) st[L.vf + lane] = to_f32<Tin>(reinterpret_cast<const Tin*>(st + L.v)[lane]);
-      __syncwarp();
+      if (tid < 4 * U) st[L.vf + tid] = to_f32<Tin>(reinterpret_cast<const Tin*>(st + L.v)[tid]);
+      tile_sync<NWB>();
     }
     BwdTok k;
     k.log = reinterpret_cast<const float4*>(st + L.log);
@@ -194,10 +202,10 @@ __device__ __forceinline__ void bwd_token_pass(const BwdArgs& a, int b, int h, i
     k.alpha = __uint_as_float(k.rec[a.rl.off_ab]);
     k.beta = __uint_as_float(k.rec[a.rl.off_ab + 1]);
     body(t_first + i * step, k);
-    __syncwarp();
+    tile_sync<NWB>();
   }
   cp_async_wait<0>();
-  __syncwarp();
+  tile_sync<NWB>();
 }
 
 // The rows of one tile: in shared memory (stride 4 U floats) or in a global
@@ -211,19 +219,20 @@ struct BwdRows {
 // The forward write of one token on the tile (the forward kernels' exact fp32
 // operations: m <- fma(alpha (1 - beta k), m, (beta k) v)). With `log`, the
 // overwritten units are kept at log[e * U + u].
-template <int U>
+template <int U, int NWB>
 __device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok& k, const BwdRows& Ms, float4* log,
-                                                  int lane) {
-  constexpr int UNR = U == 1 ? 2 : 1;  // entries per lane in flight together
+                                                  int tid) {
+  constexpr int UNR = U == 1 && NWB == 1 ? 2 : 1;  // entries per lane in flight together
+  constexpr int NT = NWB * kWarp;
   const int32_t* slot = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_w);
   const float* ww = reinterpret_cast<const float*>(k.rec + a.rl.off_k_w);
-  for (int e0 = lane; e0 < a.W; e0 += kWarp * UNR) {
+  for (int e0 = tid; e0 < a.W; e0 += NT * UNR) {
     int s[UNR];
     float4 m[UNR][U];
     float aw[UNR], cw[UNR];
 #pragma unroll
     for (int q = 0; q < UNR; ++q) {
-      const int e = e0 + q * kWarp;
+      const int e = e0 + q * NT;
       s[q] = e < a.W ? slot[e] : -1;
       cw[q] = s[q] >= 0 ? k.beta * ww[e] : 0.0f;
       aw[q] = k.alpha * (1.0f - cw[q]);
@@ -233,7 +242,7 @@ __device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok
 #pragma unroll
     for (int q = 0; q < UNR; ++q) {
       if (s[q] < 0) continue;
-      const int e = e0 + q * kWarp;
+      const int e = e0 + q * NT;
       float4* r = Ms.row(s[q]);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -251,12 +260,19 @@ __device__ __forceinline__ void bwd_forward_token(const BwdArgs& a, const BwdTok
 // kGlobal: the state and adjoint tiles live in global memory (a working copy
 // of the state in a.Mwork and dL/dM in place in a.dM) instead of shared
 // memory, for states too large to keep on chip; everything else is the same.
-template <typename Tin, int U, bool kGlobal>
-__global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
+// NWB warps share one tile (NWB = 2 only with shared-memory tiles): each
+// takes every NWB-th group of 32 entries of a token, and they meet at named
+// barriers between the phases of a token.
+template <typename Tin, int U, bool kGlobal, int NWB>
+__global__ void __launch_bounds__(NWB * 32) k_scan_backward(BwdArgs a) {
+  static_assert(NWB == 1 || (U == 1 && !kGlobal), "two warps per tile only for shared-memory tiles");
   extern __shared__ __align__(16) float bsm[];
-  constexpr int UNR = U == 1 ? 2 : 1;
+  __shared__ float red[8];  // the second warp's sums of dv, dalpha, dbeta
+  constexpr int UNR = U == 1 && NWB == 1 ? 2 : 1;
+  constexpr int NT = NWB * kWarp;
   const int N = a.N;
-  const int lane = threadIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid % kWarp, wid = tid / kWarp;
   const int tile = blockIdx.x % a.ntile;
   const int bh = blockIdx.x / a.ntile;
   const int b = bh / a.H, h = bh % a.H;
@@ -280,7 +296,7 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
   }
   // Tile-wide copies, one 16-byte unit per lane and step.
   auto copy_in = [&](const BwdRows& dst, const float* src, int64_t src_stride) {
-    for (int x = lane; x < N * U; x += kWarp) {
+    for (int x = tid; x < N * U; x += NT) {
       const int row = x / U, u = x % U;
       dst.row(row)[u] = reinterpret_cast<const float4*>(src + row * src_stride)[u];
     }
@@ -289,14 +305,14 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
   // --------------------------------------------- pass 1: checkpoints --
   // (only when the sequence has more than one chunk)
   copy_in(Ms, Min, a.d_v);
-  __syncwarp();
+  tile_sync<NWB>();
   if (nC > 1)
-    bwd_token_pass<Tin, U>(a, b, h, tile, lane, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
+    bwd_token_pass<Tin, U, NWB>(a, b, h, tile, tid, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
       if (t > 0 && t % a.C == 0) {
         float4* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N * U;
-        for (int x = lane; x < N * U; x += kWarp) dst[x] = Ms.row(x / U)[x % U];
+        for (int x = tid; x < N * U; x += NT) dst[x] = Ms.row(x / U)[x % U];
       }
-      bwd_forward_token<U>(a, k, Ms, nullptr, lane);
+      bwd_forward_token<U, NWB>(a, k, Ms, nullptr, tid);
     });
 
   // ---------------------------------- pass 2: chunks from the end --
@@ -311,18 +327,20 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
       const float* src = reinterpret_cast<const float*>(ckpt + static_cast<int64_t>(kc - 1) * N * U);
       copy_in(Ms, src, 4 * U);
     }
-    __syncwarp();
+    tile_sync<NWB>();
     // Recompute the chunk forward, logging overwritten units.
-    bwd_token_pass<Tin, U>(a, b, h, tile, lane, t0, 1, t1 - t0, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
-      bwd_forward_token<U>(a, k, Ms, logb + static_cast<int64_t>(t - t0) * a.W * U, lane);
-    });
-    // The log rows were written by other lanes; the reverse pass reads them
+    bwd_token_pass<Tin, U, NWB>(a, b, h, tile, tid, t0, 1, t1 - t0, ring, nullptr, 0, false,
+                                [&](int t, const BwdTok& k) {
+                                  bwd_forward_token<U, NWB>(a, k, Ms, logb + static_cast<int64_t>(t - t0) * a.W * U,
+                                                            tid);
+                                });
+    // The log rows were written by other threads; the reverse pass reads them
     // back through cp.async.
     __threadfence_block();
-    __syncwarp();
+    tile_sync<NWB>();
     // Backward sweep over the chunk.
-    bwd_token_pass<Tin, U>(
-        a, b, h, tile, lane, t1 - 1, -1, t1 - t0, ring, reinterpret_cast<const float*>(logb), t0, true,
+    bwd_token_pass<Tin, U, NWB>(
+        a, b, h, tile, tid, t1 - 1, -1, t1 - t0, ring, reinterpret_cast<const float*>(logb), t0, true,
         [&](int t, const BwdTok& k) {
           const int64_t th = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
           const int32_t* sw_ = reinterpret_cast<const int32_t*>(k.rec + a.rl.off_slot_w);
@@ -331,13 +349,13 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
           const float* wr = reinterpret_cast<const float*>(k.rec + a.rl.off_q_r);
           float* prt = a.part + (th * a.ntile + tile) * PW;
           // Read of token t (state after its write): dq and the adjoint.
-          for (int e0 = lane; e0 < a.R; e0 += kWarp * UNR) {
+          for (int e0 = tid; e0 < a.R; e0 += NT * UNR) {
             int s[UNR];
             float q[UNR];
             float4 m[UNR][U], g[UNR][U];
 #pragma unroll
             for (int qq = 0; qq < UNR; ++qq) {
-              const int e = e0 + qq * kWarp;
+              const int e = e0 + qq * NT;
               s[qq] = e < a.R ? ir[e] : -1;
               q[qq] = s[qq] >= 0 ? wr[e] : 0.0f;
 #pragma unroll
@@ -348,7 +366,7 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
             }
 #pragma unroll
             for (int qq = 0; qq < UNR; ++qq) {
-              const int e = e0 + qq * kWarp;
+              const int e = e0 + qq * NT;
               if (e >= a.R) continue;
               float p = 0.0f;
               if (s[qq] >= 0) {
@@ -364,19 +382,19 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
               prt[a.W + e] = p;
             }
           }
-          __syncwarp();
+          tile_sync<NWB>();
           // Write of token t, undone: derivatives, adjoint decay, state restore.
           float4 dv[U];
 #pragma unroll
           for (int u = 0; u < U; ++u) dv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           float dal = 0.0f, dbe = 0.0f;
-          for (int e0 = lane; e0 < a.W; e0 += kWarp * UNR) {
+          for (int e0 = tid; e0 < a.W; e0 += NT * UNR) {
             int s[UNR];
             float kw[UNR];
             float4 g[UNR][U], m[UNR][U];
 #pragma unroll
             for (int qq = 0; qq < UNR; ++qq) {
-              const int e = e0 + qq * kWarp;
+              const int e = e0 + qq * NT;
               s[qq] = e < a.W ? sw_[e] : -1;
               kw[qq] = s[qq] >= 0 ? ww[e] : 0.0f;
 #pragma unroll
@@ -387,7 +405,7 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
             }
 #pragma unroll
             for (int qq = 0; qq < UNR; ++qq) {
-              const int e = e0 + qq * kWarp;
+              const int e = e0 + qq * NT;
               if (e >= a.W) continue;
               float dk = 0.0f;
               if (s[qq] >= 0) {
@@ -419,9 +437,14 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
           // Warp sums of dv (4 U values), dalpha and dbeta.
           if constexpr (U == 1) {
             float x[8] = {dv[0].x, dv[0].y, dv[0].z, dv[0].w, dal, dbe, 0.0f, 0.0f};
-            const float sum = warp_sum_transposed<8>(x, lane);  // value j in lanes 4j .. 4j+3
-            if ((lane & 3) == 0) {
-              const int j = lane >> 2;
+            float sum = warp_sum_transposed<8>(x, lane);  // value j in lanes 4j .. 4j+3
+            const int j = lane >> 2;
+            if constexpr (NWB == 2) {  // the second warp hands its sums to the first
+              if (wid == 1 && (lane & 3) == 0 && j < 6) red[j] = sum;
+              tile_sync<NWB>();
+              if ((lane & 3) == 0 && j < 6) sum += red[j];
+            }
+            if (wid == 0 && (lane & 3) == 0) {
               if (j < 4) a.dv[th * a.d_v + col0 + j] = sum;
               else if (j < 6) prt[a.W + a.R + (j - 4)] = sum;
             }
@@ -456,9 +479,9 @@ __global__ void __launch_bounds__(32) k_scan_backward(BwdArgs a) {
           }
         });
   }
-  __syncwarp();
+  tile_sync<NWB>();
   if constexpr (!kGlobal) {
-    for (int x = lane; x < N * U; x += kWarp)
+    for (int x = tid; x < N * U; x += NT)
       reinterpret_cast<float4*>(Gout + static_cast<int64_t>(x / U) * a.d_v)[x % U] = Gs.row(x / U)[x % U];
   }
 }
