@@ -357,7 +357,7 @@ def run_sdm(args, dist: Dist):
     value = aggregate_value(tokens * args.steps, dist.world, ms_max / 1e3)
 
     resident = sdm.scan_variant(sh) == "resident"
-    launches_per_step = 4 + (0 if resident else 1) + (1 if args.epilogue else 0)
+    launches_per_step = int(sdm.native.load().sdm_layer_forward_launches(ctypes.byref(sh), int(args.epilogue)))
     scan_ms = stage_ms[3]
     th = shape.B * shape.T * shape.H
     algo_bytes = algorithmic_bytes_per_token_head(shape, args.epilogue) * th

@@ -276,6 +276,13 @@ SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp,
                                const void* M0, void* M_out, float* y, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* Kernel launches one sdm_layer_forward call makes for this shape on the
+ * current device (with_gate != 0: with the epilogue): the two selections,
+ * the record build and the recurrence, plus the state copy for the streaming
+ * recurrence, plus the epilogue. -1 for an invalid or unsupported shape. For
+ * profiles and logs. */
+SDM_API int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate);
+
 /* Kernel launches one sdm_layer_step call makes for this shape, without the
  * epilogue's (one more when g is given on the general path): 1 when the call
  * takes the single-launch decode kernel (T = 1, W = R <= 64, automatic

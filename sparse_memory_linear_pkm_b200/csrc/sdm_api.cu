@@ -1184,6 +1184,19 @@ sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const void* kp, 
   return ok();
 }
 
+int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate) {
+  const std::string saved = g_last_error;
+  DeviceInfo* dev;
+  ScanChoice c;
+  if (check_shape(shape) != SDM_OK || device_info(&dev) != SDM_OK || choose_scan(*dev, *shape, &c) != SDM_OK) {
+    g_last_error = saved;
+    return -1;
+  }
+  g_last_error = saved;
+  // two selections, records, recurrence; the streaming recurrence also copies M0 first
+  return 4 + (c.resident ? 0 : 1) + (with_gate ? 1 : 0);
+}
+
 sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
                                const void* alpha, const void* beta, const void* g, const void* M0, void* M_out,
                                float* y, void* workspace, size_t workspace_bytes, void* stream) {

@@ -155,3 +155,10 @@ def test_layer_backward_arguments_without_gpu(lib):
     assert lib.sdm_rmsnorm_gate(None, None, native.F32, 2, 0, ctypes.c_float(1e-6), None) == 1
     assert lib.sdm_rmsnorm_gate_backward(None, None, native.F32, None, 0, 8, ctypes.c_float(1e-6), None, None,
                                          None) == 0
+
+
+def test_layer_forward_launch_count_needs_device_or_fails(lib):
+    # The count depends on the recurrence variant chosen for the device; without a GPU it reports -1.
+    n = lib.sdm_layer_forward_launches(ctypes.byref(shape()), 0)
+    assert n in (-1, 4, 5)
+    assert lib.sdm_layer_forward_launches(ctypes.byref(shape(sqrt_n=0)), 0) == -1
