@@ -16,11 +16,12 @@
 //
 // with G = dL/dM running backwards over the tokens from dL/dM_T, the read of a
 // token before its write. Every column of d_v is independent given the
-// per-token scalars, so one warp carries one column tile of one (b, h) with
-// its state M and adjoint G resident in shared memory (or, for large N, in
-// global memory). Memory-efficient by
+// per-token scalars, so one CTA carries one column tile of one (b, h) with its
+// state M and adjoint G: 4 columns in shared memory, shared by two warps that
+// split each token's entries, or, for states too large for shared memory,
+// 32 columns in global memory with one warp. Memory-efficient by
 // recomputation: a first forward pass stores the tile every C tokens
-// (checkpoints); then, chunk by chunk from the end, the warp reloads the
+// (checkpoints); then, chunk by chunk from the end, the CTA reloads the
 // chunk's checkpoint, recomputes the chunk forward keeping the values each
 // write overwrites (the log), and sweeps the chunk backwards, restoring the
 // overwritten values as it goes. The recomputed trajectory is the forward
