@@ -105,6 +105,17 @@ class Oracle:
         lib.oracle_rmsnorm_gate_backward.restype = ctypes.c_int
         lib.oracle_rmsnorm_gate_backward.argtypes = [_c_i64, _c_i32, _c_ptr, _c_ptr, _c_ptr, ctypes.c_double,
                                                      _c_ptr, _c_ptr]
+        lib.oracle_round_e4m3.restype = ctypes.c_uint8
+        lib.oracle_round_e4m3.argtypes = [ctypes.c_double]
+        lib.oracle_decode_e4m3.restype = ctypes.c_double
+        lib.oracle_decode_e4m3.argtypes = [ctypes.c_uint8]
+        lib.oracle_quantize_fp8blk.restype = ctypes.c_int
+        lib.oracle_quantize_fp8blk.argtypes = [_c_ptr, _c_i64, _c_ptr, _c_ptr]
+        lib.oracle_scan_fp8blk.restype = ctypes.c_int
+        lib.oracle_scan_fp8blk.argtypes = [
+            _c_i32, _c_i32, _c_i32, _c_i64, _c_i32, _c_i32, _c_i32,
+            _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i32,
+        ]
         lib.oracle_round_to_bf16.restype = ctypes.c_float
         lib.oracle_round_to_bf16.argtypes = [ctypes.c_double]
         self.lib = lib
@@ -232,6 +243,45 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_rmsnorm_gate_backward failed")
         return dx, dg
+
+    # -- block-scaled fp8 state ---------------------------------------------------
+    def round_e4m3(self, x: float) -> int:
+        return int(self.lib.oracle_round_e4m3(float(x)))
+
+    def decode_e4m3(self, code: int) -> float:
+        return float(self.lib.oracle_decode_e4m3(int(code)))
+
+    def quantize_fp8blk(self, x):
+        """Blocks of 16 fp32 values -> (codes uint8 [..., 16k], exps int8 [..., k])."""
+        x = _f32(x)
+        nb = x.size // 16
+        codes = np.empty(x.shape, dtype=np.uint8)
+        exps = np.empty(x.shape[:-1] + (x.shape[-1] // 16,), dtype=np.int8)
+        self.lib.oracle_quantize_fp8blk(_p(x), nb, _p(codes), _p(exps))
+        return codes, exps
+
+    def dequantize_fp8blk(self, codes, exps):
+        table = np.array([self.decode_e4m3(c) for c in range(256)])
+        vals = table[np.asarray(codes)]
+        return vals * np.ldexp(1.0, np.repeat(np.asarray(exps, dtype=np.int64), 16, axis=-1))
+
+    def scan_fp8blk(self, idx_w, w_w, idx_r, w_r, v, alpha, beta, codes, exps, n_threads: int | None = None):
+        """The recurrence on the block-scaled fp8 state (codes [B,H,N,d_v],
+        exps [B,H,N,d_v/16], not modified). Returns (y float64, codes_T, exps_T)."""
+        idx_w, idx_r = _i32(idx_w), _i32(idx_r)
+        w_w, w_r, v, alpha, beta = _f32(w_w), _f32(w_r), _f32(v), _f32(alpha), _f32(beta)
+        C = np.ascontiguousarray(codes, dtype=np.uint8).copy()
+        X = np.ascontiguousarray(exps, dtype=np.int8).copy()
+        B, T, H, W = idx_w.shape
+        R = idx_r.shape[-1]
+        d_v = v.shape[-1]
+        N = C.shape[2]
+        y = np.zeros((B, T, H, d_v), dtype=np.float64)
+        rc = self.lib.oracle_scan_fp8blk(B, T, H, N, d_v, W, R, _p(idx_w), _p(w_w), _p(idx_r), _p(w_r), _p(v),
+                                         _p(alpha), _p(beta), _p(C), _p(X), _p(y), n_threads or default_threads())
+        if rc != 0:
+            raise ValueError(f"oracle_scan_fp8blk failed with code {rc}")
+        return y, C, X
 
     # -- whole layer ---------------------------------------------------------
     def layer_forward(self, kp, qp, v, alpha, beta, M0, W: int, R: int, g=None,

@@ -184,6 +184,75 @@ void rmsnorm_gate_row(double* y, const G* g, int32_t d_v, double eps) {
   for (int32_t c = 0; c < d_v; ++c) y[c] = static_cast<double>(g[c]) * y[c] * inv;
 }
 
+// ------------------------------------------------- block-scaled fp8 state --
+// A reduced-precision state ([explainer] "工程落地关键点", item 2: at N = 10^7
+// the state needs int8/fp8 quantisation; the pages fix no format). Reading:
+// OCP FP8 E4M3 values (sign, 4 exponent bits with bias 7, 3 mantissa bits;
+// subnormals down to 2^-9; no infinities; largest finite 448; S.1111.111 is
+// NaN and never produced) with one power-of-two scale 2^e per 16 consecutive
+// values of a state row (block scaling in the manner of the OCP MX formats,
+// with blocks of 16). For a block with largest magnitude m > 0 the exponent is
+// e = floor(log2 m) - 8, so that m / 2^e lies in [256, 512); every value is
+// rounded to nearest-even onto the E4M3 grid after division by 2^e and
+// clamped to +-448. An all-zero block has e = 0.
+
+// E4M3 code of a double (round to nearest, ties to even; clamped to 448).
+uint8_t round_e4m3(double x) {
+  const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  double a = std::fabs(x);
+#if ORACLE_MUTANT == 21
+  if (a >= 448.0) return static_cast<uint8_t>(sign | 0x7F);  // planted: overflow to the NaN code
+#else
+  if (a >= 448.0) return static_cast<uint8_t>(sign | 0x7E);
+#endif
+  // Grid spacing for |x| in [2^k, 2^(k+1)): 2^(k-3) for k >= -6, 2^-9 below (subnormals).
+  int k = 0;
+  if (a > 0.0) {
+    std::frexp(a, &k);
+    k -= 1;  // a in [2^k, 2^(k+1))
+  }
+  const int q = std::max(k, -6) - 3;  // weight of the last mantissa bit
+#if ORACLE_MUTANT == 20
+  const double r = std::trunc(std::ldexp(a, -q));  // planted: rounding toward zero
+#else
+  const double r = std::nearbyint(std::ldexp(a, -q));  // default mode: nearest-even
+#endif
+  double v = std::ldexp(r, q);
+  if (v > 448.0) v = 448.0;
+  // Encode v (exactly representable now).
+  if (v == 0.0) return sign;
+  int ev = 0;
+  std::frexp(v, &ev);
+  ev -= 1;  // v in [2^ev, 2^(ev+1))
+  if (ev < -6) {  // subnormal: v = m * 2^-9, m in 1..7
+    const int m = static_cast<int>(std::ldexp(v, 9));
+    return static_cast<uint8_t>(sign | m);
+  }
+  const int mant = static_cast<int>(std::ldexp(v, -ev) * 8.0) - 8;  // 0..7
+  return static_cast<uint8_t>(sign | ((ev + 7) << 3) | mant);
+}
+
+double decode_e4m3(uint8_t c) {
+  const double sign = (c & 0x80) ? -1.0 : 1.0;
+  const int e = (c >> 3) & 0x0F, m = c & 0x07;
+  if (e == 0) return sign * std::ldexp(static_cast<double>(m), -9);
+  return sign * std::ldexp(1.0 + m / 8.0, e - 7);
+}
+
+// Scale exponent of a block of n values (see above).
+int block_exponent(const float* x, int n) {
+  double mx = 0.0;
+  for (int i = 0; i < n; ++i) mx = std::max(mx, std::fabs(static_cast<double>(x[i])));
+  if (mx == 0.0) return 0;
+  int k = 0;
+  std::frexp(mx, &k);
+#if ORACLE_MUTANT == 19
+  return (k - 1) - 7;  // planted: one binade too high, the block max lands in [128, 256)
+#else
+  return (k - 1) - 8;
+#endif
+}
+
 // Stores a freshly computed state value: rounded to fp32 (or to bf16 and kept
 // as an exact fp32) in a float state; kept exactly in a double state.
 template <class S>
@@ -542,6 +611,69 @@ int oracle_rmsnorm_gate_backward(int64_t n_rows, int32_t d_v, const double* x, c
       dg[r * d_v + c] = dr[c] * xr[c] / rms;
     }
   }
+  return 0;
+}
+
+uint8_t oracle_round_e4m3(double x) { return round_e4m3(x); }
+double oracle_decode_e4m3(uint8_t c) { return decode_e4m3(c); }
+
+// Quantises n_blocks blocks of 16 fp32 values: codes [n_blocks*16] uint8,
+// exps [n_blocks] int8 (the block scale is 2^exp).
+int oracle_quantize_fp8blk(const float* x, int64_t n_blocks, uint8_t* codes, int8_t* exps) {
+  for (int64_t bI = 0; bI < n_blocks; ++bI) {
+    // (the stored exponent is an int8; blocks beyond its range use the nearest one)
+    const int e = std::max(-127, std::min(127, block_exponent(x + bI * 16, 16)));
+    exps[bI] = static_cast<int8_t>(e);
+    for (int i = 0; i < 16; ++i) codes[bI * 16 + i] = round_e4m3(std::ldexp(static_cast<double>(x[bI * 16 + i]), -e));
+  }
+  return 0;
+}
+
+// The recurrence with the block-scaled fp8 state. The state is codes
+// [B,H,N,d_v] uint8 and exps [B,H,N,d_v/16] int8 (in/out); d_v a multiple of
+// 16. A written row is computed in fp32 exactly as the recurrence kernels do
+// (cw = beta k, aw = alpha (1 - cw), m' = fma(aw, m, cw v), round-to-nearest
+// fp32 operations) from the decoded row, then every 16-value block of it is
+// quantised, so both sides take each code decision from the same fp32 value.
+// y (double) is the read of the decoded state after the write.
+// Weights w_w, w_r are the fp32 weights the kernels get.
+int oracle_scan_fp8blk(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W, int32_t R,
+                       const int32_t* idx_w, const float* w_w, const int32_t* idx_r, const float* w_r,
+                       const float* v, const float* alpha, const float* beta, uint8_t* codes, int8_t* exps,
+                       double* y, int32_t n_threads) {
+  if (B < 0 || T < 0 || H < 0 || N < 1 || d_v < 16 || d_v % 16 != 0 || W < 0 || R < 0) return -1;
+  for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * W; ++e)
+    if (idx_w[e] < 0 || idx_w[e] >= N) return -2;
+  for (int64_t e = 0; e < static_cast<int64_t>(B) * T * H * R; ++e)
+    if (idx_r[e] < 0 || idx_r[e] >= N) return -2;
+  const int32_t nb = d_v / 16;
+  parallel_for(static_cast<int64_t>(B) * H, std::max(1, n_threads), [&](int64_t u) {
+    const int32_t h = static_cast<int32_t>(u % H);
+    const int32_t b = static_cast<int32_t>(u / H);
+    uint8_t* C = codes + (static_cast<int64_t>(b) * H + h) * N * d_v;
+    int8_t* X = exps + (static_cast<int64_t>(b) * H + h) * N * nb;
+    std::vector<float> row(static_cast<size_t>(d_v));
+    auto decoded = [&](int64_t i, int32_t c) {
+      return static_cast<float>(decode_e4m3(C[i * d_v + c]) * std::ldexp(1.0, X[i * nb + c / 16]));
+    };
+    for (int32_t t = 0; t < T; ++t) {
+      const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;
+      const float a_t = alpha[th], b_t = beta[th];
+      for (int32_t j = 0; j < W; ++j) {
+        const int64_t i = idx_w[th * W + j];
+        const float cw = b_t * w_w[th * W + j];
+        const float aw = a_t * (1.0f - cw);
+        for (int32_t c = 0; c < d_v; ++c) row[c] = std::fma(aw, decoded(i, c), cw * v[th * d_v + c]);
+        oracle_quantize_fp8blk(row.data(), nb, C + i * d_v, X + i * nb);
+      }
+      for (int32_t c = 0; c < d_v; ++c) {
+        double acc = 0.0;
+        for (int32_t r = 0; r < R; ++r)
+          acc += static_cast<double>(w_r[th * R + r]) * static_cast<double>(decoded(idx_r[th * R + r], c));
+        y[th * d_v + c] = acc;
+      }
+    }
+  });
   return 0;
 }
 

@@ -491,6 +491,115 @@ def pin_epilogue_backward(o):
         assert abs(fd - np.sum(dg * D)) <= 1e-6 * (1 + abs(fd)), ("dg", fd, np.sum(dg * D))
 
 
+# --------------------------------------------------- block-scaled fp8 state --
+
+def _e4m3_grid():
+    """All non-negative finite E4M3 values, from the format's definition
+    (bias 7, 3 mantissa bits, subnormals m * 2^-9, largest 1.75 * 2^8), as
+    exact fractions with their codes."""
+    grid = []
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue  # NaN
+            val = Fraction(m, 8) * Fraction(2) ** -6 if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+            grid.append((val, (e << 3) | m))
+    return sorted(grid)
+
+
+def _rne_e4m3(x: Fraction) -> int:
+    """Exact round-to-nearest-even onto the E4M3 grid, clamped to 448."""
+    grid = _e4m3_grid()
+    sign = 0x80 if x < 0 else 0
+    a = abs(x)
+    if a >= grid[-1][0]:
+        return sign | grid[-1][1]
+    for (lo, cl), (hi, ch) in zip(grid, grid[1:]):
+        if lo <= a <= hi:
+            if a - lo < hi - a:
+                return sign | cl
+            if a - lo > hi - a:
+                return sign | ch
+            return sign | (cl if cl % 2 == 0 else ch)
+    raise AssertionError(x)
+
+
+def pin_e4m3_rounding(o):
+    """Decoding of every finite code and round-to-nearest-even (with
+    saturation) against an exact-rational reference of the format: at every
+    representable value, every midpoint, beyond 448 and at random values."""
+    grid = _e4m3_grid()
+    for val, code in grid:
+        assert o.decode_e4m3(code) == float(val) and o.decode_e4m3(0x80 | code) == -float(val), code
+    probes = [v for v, _ in grid] + [(a + b) / 2 for (a, _), (b, _) in zip(grid, grid[1:])]
+    probes += [Fraction(449), Fraction(464), Fraction(480), Fraction(10 ** 6), Fraction(1, 2 ** 11)]
+    rng = np.random.default_rng(3)
+    probes += [Fraction(float(x)) for x in np.exp(rng.uniform(-9, 6.5, 400))]
+    for p in probes:
+        for x in (p, -p):
+            got = o.round_e4m3(float(x))
+            want = _rne_e4m3(x)
+            if x == 0:
+                continue  # the sign of zero follows the input's sign bit
+            assert got == want, (float(x), got, want)
+
+
+def pin_fp8blk_blocks(o):
+    """Block scales put each block's largest magnitude in [256, 512) (an
+    all-zero block gets exponent 0), codes are the exact rounding of x / 2^e,
+    and quantising a dequantised block gives it back."""
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((40, 16)).astype(np.float32)
+    x *= np.float32(2.0) ** rng.integers(-20, 20, (40, 1)).astype(np.float32)
+    x[3] = 0.0
+    x[5, :15] = 0.0
+    codes, exps = o.quantize_fp8blk(x)
+    for i in range(x.shape[0]):
+        m = float(np.abs(x[i]).max())
+        if m == 0.0:
+            assert exps[i, 0] == 0 and not (codes[i] & 0x7F).any()
+            continue
+        e = math.frexp(m)[1] - 1 - 8
+        assert exps[i, 0] == e, (i, exps[i, 0], e)
+        for j in range(16):
+            assert codes[i, j] == _rne_e4m3(Fraction(float(x[i, j])) / Fraction(2) ** e), (i, j)
+    deq = o.dequantize_fp8blk(codes, exps).astype(np.float32)
+    c2, e2 = o.quantize_fp8blk(deq)
+    assert np.array_equal(c2, codes) and np.array_equal(e2, exps)
+
+
+def pin_fp8blk_scan(o):
+    """The recurrence on the fp8 state: alpha = 1, beta = 0 leaves every code
+    and scale unchanged; beta = 1 with one write slot of weight 1 stores
+    exactly the quantised v; a read of that slot with weight 1 returns its
+    decoded value."""
+    rng = np.random.default_rng(6)
+    B, T, H, N, d_v = 1, 5, 2, 16, 32
+    M = rng.standard_normal((B, H, N, d_v)).astype(np.float32)
+    codes, exps = o.quantize_fp8blk(M)
+    idx_w, w_w = random_selection(rng, B, T, H, N, 3)
+    idx_r, w_r = random_selection(rng, B, T, H, N, 2)
+    v = rng.standard_normal((B, T, H, d_v)).astype(np.float32)
+    ones, zeros = np.ones((B, T, H), np.float32), np.zeros((B, T, H), np.float32)
+    _, C, X = o.scan_fp8blk(idx_w, w_w, idx_r, w_r, v, ones, zeros, codes, exps)
+    assert np.array_equal(C, codes) and np.array_equal(X, exps)
+    iw = idx_w[..., :1].copy()
+    y, C, X = o.scan_fp8blk(iw, np.ones_like(iw, dtype=np.float32), iw, np.ones_like(iw, dtype=np.float32), v, ones,
+                            ones, codes, exps)
+    for t in range(T):
+        for h in range(H):
+            vc, ve = o.quantize_fp8blk(v[0, t, h])
+            deq = o.dequantize_fp8blk(vc, ve)
+            assert np.array_equal(y[0, t, h], deq), (t, h)
+    last = {}
+    for t in range(T):
+        for h in range(H):
+            last[(h, int(iw[0, t, h, 0]))] = t
+    for (h, slot), t in last.items():
+        vc, ve = o.quantize_fp8blk(v[0, t, h])
+        assert np.array_equal(C[0, h, slot], vc) and np.array_equal(X[0, h, slot], ve)
+
+
 ALL_PINS = {
     "selection_brute_force": pin_selection_brute_force,
     "selection_identity": pin_selection_identity,
@@ -513,6 +622,9 @@ ALL_PINS = {
     "backward_unselected_pass_through": pin_backward_unselected_pass_through,
     "topk_backward": pin_topk_backward,
     "epilogue_backward": pin_epilogue_backward,
+    "e4m3_rounding": pin_e4m3_rounding,
+    "fp8blk_blocks": pin_fp8blk_blocks,
+    "fp8blk_scan": pin_fp8blk_scan,
 }
 
 

@@ -34,6 +34,9 @@ MUTANTS = {
     16: "backward: softmax mean not subtracted",
     17: "backward: score halves swapped",
     18: "backward: RMS-norm normaliser treated as a constant",
+    19: "fp8 state: block scale one binade too high",
+    20: "fp8 state: rounding toward zero",
+    21: "fp8 state: overflow to the NaN code",
 }
 
 
