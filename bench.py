@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--decode", action="store_true",
                     help="time decode steps instead: one token per call (sdm_layer_step), state carried")
+    ap.add_argument("--fp8-state", action="store_true",
+                    help="with --decode: keep the state in the block-scaled fp8 format (E4M3, scale per 16 values)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward instead: sdm_scan_backward and the two selection-weight backwards")
     ap.add_argument("--slot-counts", action="store_true",
@@ -481,9 +483,11 @@ def run_decode(args, dist: Dist):
     inp = synth.make_inputs(shape, seed=args.seed + dist.rank, device=dev)
     per_step = [{k: inp[k][:, t:t + 1].contiguous() for k in ("kp", "qp", "v", "alpha", "beta")} for t in range(n_tok)]
     M = inp["M0"].unsqueeze(0).repeat(shape.B, 1, 1, 1).contiguous()
+    if args.fp8_state:
+        M = sdm.quantize_fp8blk(M.float().contiguous())
     y = torch.empty((shape.B, 1, shape.H, shape.d_v), dtype=torch.float32, device=dev)
     sh = sdm.make_shape(shape.B, 1, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
-                        shape.torch_state())
+                        torch.uint8 if args.fp8_state else shape.torch_state())
     ws = torch.empty(max(16, int(sdm.native.load().sdm_layer_step_workspace_bytes(ctypes.byref(sh)))),
                      dtype=torch.uint8, device=dev)
 
@@ -536,7 +540,11 @@ def run_decode(args, dist: Dist):
     if dist.rank == 0:
         cfg = workload_config(shape, args, dist)
         cfg.update({"T": 1, "mode": "decode: one token per batch row per sdm_layer_step call, state carried",
-                    "variant": sdm.scan_variant(sh)})
+                    "state_bytes": M.numel() * M.element_size()})
+        if args.fp8_state:
+            cfg.update({"state_dtype": "fp8 E4M3, power-of-two scale per 16 values", "variant": "single launch"})
+        else:
+            cfg["variant"] = sdm.scan_variant(sh)
         line = {"metric": "SDM decode step latency (one token per batch row, state carried) on 1 B200",
                 "value": us_per_step, "unit": "us", "eager_us_per_step": ms_eager * 1e3 / args.steps,
                 "timing": "value: one step captured in a CUDA graph and replayed; eager: one library call per step",

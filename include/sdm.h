@@ -63,7 +63,14 @@ typedef enum sdm_status {
   SDM_ERR_DEVICE_FAULT = 4      /* the device error word was set (see sdm_stream_check) */
 } sdm_status_t;
 
-typedef enum sdm_dtype { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype_t;
+/* SDM_FP8_B16 is a state dtype only: OCP FP8 E4M3 codes with one
+ * power-of-two scale per 16 consecutive values of a state row. A state of
+ * R rows of d_v values is R * d_v code bytes followed by R * d_v / 16 int8
+ * exponents (value = E4M3(code) * 2^exponent); sdm_quantize_fp8blk builds it
+ * from fp32. Only the single-launch decode step (sdm_layer_step with T = 1,
+ * W = R <= 64, automatic variant) runs on it; every other call returns
+ * SDM_ERR_UNSUPPORTED for it. */
+typedef enum sdm_dtype { SDM_F32 = 0, SDM_BF16 = 1, SDM_FP8_B16 = 2 } sdm_dtype_t;
 
 /* Which recurrence kernel runs (sdm_shape_t.variant). */
 typedef enum sdm_variant {
@@ -101,6 +108,14 @@ SDM_API const char* sdm_status_string(sdm_status_t status);
 
 /* Text describing the last error returned on the calling host thread ("" if none). */
 SDM_API const char* sdm_last_error(void);
+
+/* Quantises n_blocks blocks of 16 fp32 values into the SDM_FP8_B16 format:
+ * e = floor(log2 max|x|) - 8 per block (clamped to [-127, 127]; 0 for an
+ * all-zero block), codes = round-to-nearest-even(x / 2^e) onto the E4M3 grid,
+ * clamped to +-448. x [n_blocks * 16] fp32; codes [n_blocks * 16] uint8;
+ * exps [n_blocks] int8 (all device, caller owned; x and codes 16-byte aligned). */
+SDM_API sdm_status_t sdm_quantize_fp8blk(const float* x, int64_t n_blocks, uint8_t* codes, int8_t* exps,
+                                 void* stream);
 
 /* Slot utilisation of a selection: counts[b,h,i] += the number of (t,k) with
  * idx[b,t,h,k] == i ([explainer] "亮点与局限" and "工程落地关键点" item 2: the

@@ -21,10 +21,12 @@ from . import native, synth
 from .native import SdmError
 
 __all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "scan_describe",
-           "scan_backward", "pkm_topk_backward", "rmsnorm_gate", "rmsnorm_gate_backward", "layer_backward", "stream_check", "make_shape",
+           "scan_backward", "pkm_topk_backward", "rmsnorm_gate", "rmsnorm_gate_backward", "layer_backward",
+           "quantize_fp8blk", "fp8blk_parts", "stream_check", "make_shape",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
-_DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16}
+_DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16,
+          torch.uint8: native.FP8_B16}  # a uint8 state buffer holds the block-scaled fp8 state
 
 
 def _code(t: torch.Tensor, what: str) -> int:
@@ -217,6 +219,24 @@ def layer_backward(kp, qp, v, alpha, beta, M0, dy, W: int, R: int, g=None, y_pre
                                         _ptr(out.get("dg")), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev)))
     out["dM0"] = dM
     return out
+
+
+def quantize_fp8blk(x: torch.Tensor) -> torch.Tensor:
+    """A block-scaled fp8 state buffer (uint8: the E4M3 codes of x, then one
+    int8 exponent per 16 values) from fp32 x [..., d_v] with d_v a multiple of
+    16; pass it as the state M of layer_step (T = 1)."""
+    n = x.numel()
+    if n % 16:
+        raise ValueError("the number of values must be a multiple of 16")
+    buf = torch.empty(n + n // 16, dtype=torch.uint8, device=x.device)
+    native.check(native.load().sdm_quantize_fp8blk(_ptr(x), n // 16, _ptr(buf), ctypes.c_void_p(buf.data_ptr() + n),
+                                                   _stream(x.device)))
+    return buf
+
+
+def fp8blk_parts(buf: torch.Tensor, n_values: int):
+    """(codes uint8 [n_values], exps int8 [n_values // 16]) views of a fp8 state buffer."""
+    return buf[:n_values], buf[n_values:].view(torch.int8)
 
 
 def state_init(M0: torch.Tensor, B: int, out: torch.Tensor | None = None) -> torch.Tensor:

@@ -131,7 +131,9 @@ sdm_status_t check_shape(const sdm_shape_t* s) {
   if (s->d_v < 16 || s->d_v > 8192 || s->d_v % 16 != 0)
     return fail(SDM_ERR_INVALID_ARGUMENT, "d_v must be a multiple of 16 in [16, 8192]");
   if ((st = check_dtype(s->in_dtype, "in_dtype")) != SDM_OK) return st;
-  if ((st = check_dtype(s->state_dtype, "state_dtype")) != SDM_OK) return st;
+  if (s->state_dtype != SDM_FP8_B16 && (st = check_dtype(s->state_dtype, "state_dtype")) != SDM_OK) return st;
+  if (s->state_dtype == SDM_FP8_B16 && s->d_v % 16 != 0)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "the fp8 state needs d_v a multiple of 16");
   if (!(s->rms_eps >= 0.0f) || s->rms_eps > 1e30f) return fail(SDM_ERR_INVALID_ARGUMENT, "rms_eps must be finite and >= 0");
   if (s->variant < SDM_VARIANT_AUTO || s->variant > SDM_VARIANT_STREAMING)
     return fail(SDM_ERR_INVALID_ARGUMENT, "variant must be an sdm_variant_t value");
@@ -358,6 +360,10 @@ size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L, int NW) {
 }
 
 sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
+  if (s.state_dtype == SDM_FP8_B16)
+    return fail(SDM_ERR_UNSUPPORTED,
+                "the fp8 state (SDM_FP8_B16) runs only in the single-launch decode step: sdm_layer_step with "
+                "T = 1, W = R <= 64 and the automatic variant");
   const size_t lim = static_cast<size_t>(dev.max_smem_optin);
   ScanChoice c;
   // A resident tile reads and writes all N rows once; below one touched row
@@ -496,6 +502,8 @@ sdm_status_t launch_scan(const ScanChoice& c, const sdm_shape_t& s, const sdm::S
 }
 
 sdm_status_t launch_state_init(const DeviceInfo& dev, const sdm_shape_t& s, const void* M0, void* M, cudaStream_t st) {
+  if (s.state_dtype == SDM_FP8_B16)
+    return fail(SDM_ERR_UNSUPPORTED, "state copies of the fp8 state are not provided (build it with sdm_quantize_fp8blk)");
   const int64_t bytes_per_row = static_cast<int64_t>(s.H) * slots_of(s.sqrt_n) * s.d_v * static_cast<int64_t>(in_size(s.state_dtype));
   const int64_t units = bytes_per_row / 16;
   if (units == 0 || s.B == 0) return SDM_OK;
@@ -712,7 +720,7 @@ sdm_status_t try_decode_step(const DeviceInfo& dev, const sdm_shape_t& s, const 
     g_last_error.clear();
     return SDM_OK;
   }
-  const int VE = 16 / static_cast<int>(in_size(s.state_dtype));
+  const int VE = s.state_dtype == SDM_FP8_B16 ? 16 : 16 / static_cast<int>(in_size(s.state_dtype));
   const int UR = s.d_v / VE;
   const int groups = UR >= sdm::kDecodeThreads ? 1 : sdm::kDecodeThreads / UR;
   sdm::DecodeArgs a{};
@@ -723,6 +731,9 @@ sdm_status_t try_decode_step(const DeviceInfo& dev, const sdm_shape_t& s, const 
   a.eps = s.rms_eps;
   a.L = P.L;
   a.kp = kp; a.qp = qp; a.v = v; a.alpha = alpha; a.beta = beta; a.g = g; a.M = M; a.y = y;
+  a.exps = s.state_dtype == SDM_FP8_B16
+               ? reinterpret_cast<int8_t*>(M) + static_cast<int64_t>(s.B) * s.H * slots_of(s.sqrt_n) * s.d_v
+               : nullptr;
   a.sel_off = static_cast<uint32_t>(align16(P.L.table_bytes + 2ull * P.L.warp_bytes));
   a.part_off = static_cast<uint32_t>(a.sel_off + align16(16ull * s.W));
   a.err = dev.err;
@@ -731,11 +742,13 @@ sdm_status_t try_decode_step(const DeviceInfo& dev, const sdm_shape_t& s, const 
   const int grid = s.B * s.H;
   sdm_status_t r;
   if (s.in_dtype == SDM_BF16)
-    r = s.state_dtype == SDM_BF16 ? launch_decode_typed<sdm::bf16, sdm::bf16>(P, a, smem, grid, st)
-                                  : launch_decode_typed<sdm::bf16, float>(P, a, smem, grid, st);
+    r = s.state_dtype == SDM_FP8_B16 ? launch_decode_typed<sdm::bf16, sdm::Fp8Blk>(P, a, smem, grid, st)
+        : s.state_dtype == SDM_BF16  ? launch_decode_typed<sdm::bf16, sdm::bf16>(P, a, smem, grid, st)
+                                     : launch_decode_typed<sdm::bf16, float>(P, a, smem, grid, st);
   else
-    r = s.state_dtype == SDM_BF16 ? launch_decode_typed<float, sdm::bf16>(P, a, smem, grid, st)
-                                  : launch_decode_typed<float, float>(P, a, smem, grid, st);
+    r = s.state_dtype == SDM_FP8_B16 ? launch_decode_typed<float, sdm::Fp8Blk>(P, a, smem, grid, st)
+        : s.state_dtype == SDM_BF16  ? launch_decode_typed<float, sdm::bf16>(P, a, smem, grid, st)
+                                     : launch_decode_typed<float, float>(P, a, smem, grid, st);
   if (r == SDM_OK) *used = true;
   return r;
 }
@@ -775,6 +788,20 @@ sdm_status_t sdm_pkm_topk(const void* scores, int32_t in_dtype, int32_t B, int32
   if ((r = device_info(&dev)) != SDM_OK) return r;
   if ((r = topk_impl(*dev, scores, in_dtype, units, sqrt_n, K, idx_out, w_out, static_cast<cudaStream_t>(stream))) != SDM_OK)
     return r;
+  return ok();
+}
+
+sdm_status_t sdm_quantize_fp8blk(const float* x, int64_t n_blocks, uint8_t* codes, int8_t* exps, void* stream) {
+  sdm_status_t r;
+  if (n_blocks < 0) return fail(SDM_ERR_INVALID_ARGUMENT, "n_blocks must be >= 0");
+  if ((r = need_ptr(x, "x", n_blocks > 0)) || (r = need_ptr(codes, "codes", n_blocks > 0))) return r;
+  if (n_blocks > 0 && exps == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "exps is NULL");
+  if (n_blocks == 0) return ok();
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const int grid = static_cast<int>(std::min<int64_t>((n_blocks + 255) / 256, static_cast<int64_t>(dev->sms) * 16));
+  sdm::k_quantize_fp8blk<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, n_blocks, codes, exps);
+  if ((r = launch_status("fp8 quantize launch")) != SDM_OK) return r;
   return ok();
 }
 

@@ -15,7 +15,10 @@
 // among themselves and their loads can all be issued before any store.
 #pragma once
 
+#include <type_traits>
+
 #include "pkm_topk_fast.cuh"
+#include "sdm_fp8.cuh"
 #include "sdm_scan.cuh"
 
 namespace sdm {
@@ -32,7 +35,8 @@ struct DecodeArgs {
   const void* alpha;  // [B, 1, H] Tin
   const void* beta;   // [B, 1, H] Tin
   const void* g;      // [B, 1, H, d_v] Tin or null
-  void* M;            // [B, H, N, d_v] Tst, updated in place
+  void* M;            // [B, H, N, d_v] Tst, updated in place (fp8: the codes)
+  int8_t* exps;       // fp8 state only: [B, H, N, d_v / 16] block exponents
   float* y;           // [B, 1, H, d_v]
   uint32_t sel_off;   // byte offsets in shared memory
   uint32_t part_off;
@@ -54,7 +58,8 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_step(DecodeArgs a) {
 
   if (warp == 0) fast_topk_build_table(tab, a.L.Kh, K, lane_id());
   __syncthreads();
-  constexpr int VE = 16 / static_cast<int>(sizeof(Tst));  // state columns per 16-byte unit
+  // state columns per 16-byte unit (the fp8 tag is one byte per value)
+  constexpr int VE = std::is_same<Tst, Fp8Blk>::value ? 16 : 16 / static_cast<int>(sizeof(Tst));
   const int UR = d_v / VE;                                 // units per row
   Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * N * d_v;
   if (warp == 1) {
@@ -101,11 +106,22 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_step(DecodeArgs a) {
         const float cw = beta * sw[e];
         const float aw = alpha * (1.0f - cw);
         float m[VE], vv[VE];
-        unpack16<Tst>(raw[j], m);
         load_in_vec<Tin, VE>(vrow + u * VE, vv);
+        uint4* dst = reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(sl[j]) * d_v + u * VE);
+        if constexpr (std::is_same<Tst, Fp8Blk>::value) {
+          int8_t* ex = a.exps + (static_cast<int64_t>(bh) * N + sl[j]) * (d_v / 16) + u;
+          fp8blk_unpack16(raw[j], *ex, m);
 #pragma unroll
-        for (int i = 0; i < VE; ++i) m[i] = __fmaf_rn(aw, m[i], __fmul_rn(cw, vv[i]));
-        *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(sl[j]) * d_v + u * VE) = pack16<Tst>(m);
+          for (int i = 0; i < VE; ++i) m[i] = __fmaf_rn(aw, m[i], __fmul_rn(cw, vv[i]));
+          uint4 q;
+          *ex = static_cast<int8_t>(fp8blk_pack16(m, &q));
+          *dst = q;
+        } else {
+          unpack16<Tst>(raw[j], m);
+#pragma unroll
+          for (int i = 0; i < VE; ++i) m[i] = __fmaf_rn(aw, m[i], __fmul_rn(cw, vv[i]));
+          *dst = pack16<Tst>(m);
+        }
       }
     }
   }
@@ -126,7 +142,11 @@ __global__ void __launch_bounds__(kDecodeThreads) k_decode_step(DecodeArgs a) {
       }
       const float q = sw[K + e];
       float m[VE];
-      unpack16<Tst>(*reinterpret_cast<const uint4*>(Mbh + static_cast<int64_t>(s) * d_v + u * VE), m);
+      const uint4 raw = *reinterpret_cast<const uint4*>(Mbh + static_cast<int64_t>(s) * d_v + u * VE);
+      if constexpr (std::is_same<Tst, Fp8Blk>::value)
+        fp8blk_unpack16(raw, a.exps[(static_cast<int64_t>(bh) * N + s) * (d_v / 16) + u], m);
+      else
+        unpack16<Tst>(raw, m);
 #pragma unroll
       for (int j = 0; j < VE; ++j) acc[j] = __fmaf_rn(q, m[j], acc[j]);
     }

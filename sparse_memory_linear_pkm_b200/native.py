@@ -15,7 +15,7 @@ LIBRARY = PKG / "libsdm_b200.so"
 SDM_OK = 0
 STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARGUMENT", 2: "SDM_ERR_UNSUPPORTED", 3: "SDM_ERR_CUDA",
                 4: "SDM_ERR_DEVICE_FAULT"}
-F32, BF16 = 0, 1
+F32, BF16, FP8_B16 = 0, 1, 2  # FP8_B16: state only (E4M3 codes + a power-of-two scale per 16 values)
 VARIANTS = {"auto": 0, "resident": 1, "streaming": 2}
 NOALLOC_SCRATCH_BYTES = 16 << 20  # SDM_NOALLOC_SCRATCH_BYTES in include/sdm.h
 
@@ -58,6 +58,7 @@ PROTOTYPES = {
     "sdm_layer_backward_workspace_bytes": (_sz, [_shape_p]),
     "sdm_layer_backward": (_i32, [_shape_p] + [_p] * 17 + [_sz, _p]),
     "sdm_slot_counts": (_i32, [_p, _i32, _i32, _i32, _i32, _i32, _p, _p]),
+    "sdm_quantize_fp8blk": (_i32, [_p, ctypes.c_int64, _p, _p, _p]),
     "sdm_layer_step": (_i32, [_shape_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "sdm_layer_forward_traced": (_i32, [_shape_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p,
                                          ctypes.POINTER(_p), _i32]),
