@@ -13,6 +13,8 @@
 // R * d_v / 16 exponent bytes (int8).
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "sdm_device.cuh"
 
 namespace sdm {
@@ -24,37 +26,24 @@ __device__ __forceinline__ float pow2f(int e) {
   return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(1 << 22);
 }
 
-__device__ __forceinline__ float e4m3_decode(uint32_t c) {
-  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
-  const float mag = e == 0 ? static_cast<float>(m) * 0x1p-9f : static_cast<float>(8u + m) * pow2f(static_cast<int>(e) - 10);
-  return (c & 0x80u) ? -mag : mag;
-}
-
-// Round to nearest even onto the E4M3 grid, clamped to +-448.
-__device__ __forceinline__ uint32_t e4m3_encode(float x) {
-  const uint32_t sign = (__float_as_uint(x) >> 31) << 7;
-  const float a = fabsf(x);
-  if (a >= 448.0f) return sign | 0x7Eu;
-  const int k = a > 0.0f ? ilogbf(a) : -7;  // floor(log2 a)
-  const int q = max(k, -6) - 3;             // weight of the last mantissa bit
-  const float r = rintf(a * pow2f(-q));     // exact scaling, then nearest-even
-  if (q == -9) return sign | static_cast<uint32_t>(r);  // subnormal range (r = 8 is 2^-6, code 8)
-  // normal range: r in [8, 16]; r = 16 moves to the next binade
-  const uint32_t rr = static_cast<uint32_t>(r);
-  const int ev = rr >= 16u ? k + 1 : k;
-  const uint32_t mant = rr >= 16u ? 0u : rr - 8u;
-  return sign | (static_cast<uint32_t>(ev + 7) << 3) | mant;
-}
-
-// Decodes one 16-byte unit of codes with its block exponent.
+// Decodes one 16-byte unit of codes (value i in byte i) with its block
+// exponent. The E4M3 -> half conversion is exact (every E4M3 value is a half).
 __device__ __forceinline__ void fp8blk_unpack16(const uint4& u, int ex, float* out) {
   const float s = pow2f(ex);
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) out[i] = e4m3_decode((w[i >> 2] >> (8 * (i & 3))) & 0xFFu) * s;
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t p = static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(p, __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+    out[2 * i] = f.x * s;
+    out[2 * i + 1] = f.y * s;
+  }
 }
 
-// Quantises 16 fp32 values into one unit of codes; returns the exponent.
+// Quantises 16 fp32 values into one unit of codes; returns the exponent. The
+// division by 2^e is exact; the conversion rounds to nearest even and
+// saturates to +-448 (the format's definition).
 __device__ __forceinline__ int fp8blk_pack16(const float* x, uint4* u) {
   float mx = 0.0f;
 #pragma unroll
@@ -63,7 +52,11 @@ __device__ __forceinline__ int fp8blk_pack16(const float* x, uint4* u) {
   const float inv = pow2f(-e);
   uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) w[i >> 2] |= e4m3_encode(x[i] * inv) << (8 * (i & 3));
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t p =
+        __nv_cvt_float2_to_fp8x2(make_float2(x[2 * i] * inv, x[2 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+    w[i >> 1] |= static_cast<uint32_t>(p) << (16 * (i & 1));
+  }
   *u = make_uint4(w[0], w[1], w[2], w[3]);
   return e;
 }
