@@ -33,17 +33,21 @@
 //   4. Read after the write ([explainer] 3.1 step 3; [summary] Core Mechanism 4):
 //      y_t = sum over read slots of q_i * M_t[i], in double.
 //   5. Optional epilogue ([explainer] 3.1 step 3): y <- g * y / sqrt(mean(y^2)+eps).
-//
 //   6. Backward (the derivatives for training): reverse-mode through steps 2-4
 //      for a fixed selection, by the chain rule on the pages' own formulas
 //      ([explainer] 3.4 "高效训练" says only that a memory-efficient backward
 //      exists and leaves its details to an appendix the pages do not show).
+//   7. A block-scaled fp8 state (E4M3 values, one power-of-two scale per 16
+//      row values; see "block-scaled fp8 state" below): the recurrence with
+//      each written row computed in fp32 in the kernels' order and re-quantised.
 //
 // Parity status: selection, weights, write, read and epilogue are each pinned by
 // tests that do not re-run this file's formulas (exact-rational brute force,
 // closed forms, invariants, hand-worked fixtures, planted-mistake checks); the
 // backward is pinned by central finite differences of the double-precision
-// forward, a hand-derived one-slot closed form, and planted-mistake checks.
+// forward, a hand-derived one-slot closed form, and planted-mistake checks; the
+// fp8 state by an exact-rational model of E4M3, block invariants and scan
+// identities.
 //
 // ORACLE_MUTANT (default 0) plants one known mistake per value so the tests
 // can show that the pins catch it; it is never set outside those tests.
