@@ -64,3 +64,23 @@ def test_single_rank_needs_no_process_group():
         assert not d.pg
         assert d.max(3.25, torch.device("cpu")) == 3.25
         assert bench.aggregate_value(10.0, 1, 2.0) == 5.0
+
+
+def test_reference_arm_prints_one_contract_line():
+    """bench.py --impl reference (the oracle on the host cores) prints one JSON
+    line with the contract's keys, on the bench workload's config."""
+    import json
+    import subprocess
+
+    out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--steps", "1", "--warmup",
+                          "1", "--cpu-seconds", "0.5"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["config"]["workload"] == "d2048_h16_n1024_dv128"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
