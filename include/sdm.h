@@ -317,7 +317,11 @@ SDM_API size_t sdm_layer_step_workspace_bytes(const sdm_shape_t* shape);
  * one sequence (start from M[b] = M0 with sdm_state_init). Other arguments as
  * in sdm_layer_forward; workspace: at least sdm_layer_step_workspace_bytes(shape).
  * With the automatic variant, calls with T*(W+R) < N stream only the selected
- * rows (a resident tile would move the whole state). */
+ * rows (a resident tile would move the whole state), and calls with T = 1 and
+ * W = R <= 64 run as one fused launch (both selections, the write, the read
+ * and the epilogue). Only that fused form accepts the fp8 state
+ * (state_dtype SDM_FP8_B16: M is the code bytes followed by the block
+ * exponents, as sdm_quantize_fp8blk writes them). */
 SDM_API sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, const void* qp,
                             const void* v, const void* alpha, const void* beta, const void* g,
                             void* M, float* y, void* workspace, size_t workspace_bytes, void* stream);
