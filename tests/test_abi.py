@@ -162,3 +162,14 @@ def test_layer_forward_launch_count_needs_device_or_fails(lib):
     n = lib.sdm_layer_forward_launches(ctypes.byref(shape()), 0)
     assert n in (-1, 4, 5)
     assert lib.sdm_layer_forward_launches(ctypes.byref(shape(sqrt_n=0)), 0) == -1
+
+
+def test_fp8_state_arguments_without_gpu(lib):
+    assert lib.sdm_quantize_fp8blk(None, -1, None, None, None) == 1
+    assert lib.sdm_quantize_fp8blk(None, 2, None, None, None) == 1 and b"x" in lib.sdm_last_error()
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.sdm_quantize_fp8blk(fake, 2, fake, None, None) == 1 and b"exps" in lib.sdm_last_error()
+    assert lib.sdm_quantize_fp8blk(None, 0, None, None, None) == 0
+    # the fp8 state is a valid state dtype for shapes; as an input dtype it is not
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=8, state_dtype=native.FP8_B16))) == 1
+    assert lib.sdm_layer_step_launches(ctypes.byref(shape(in_dtype=native.FP8_B16))) == -1
