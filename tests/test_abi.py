@@ -173,3 +173,17 @@ def test_fp8_state_arguments_without_gpu(lib):
     # the fp8 state is a valid state dtype for shapes; as an input dtype it is not
     assert lib.sdm_layer_step_launches(ctypes.byref(shape(T=1, W=8, R=8, state_dtype=native.FP8_B16))) == 1
     assert lib.sdm_layer_step_launches(ctypes.byref(shape(in_dtype=native.FP8_B16))) == -1
+
+
+def test_backward_workspace_of_the_large_state_workload(lib):
+    # d2048_h4_n16384_dv512: 32-column tiles in global memory, chunks of 2048 tokens
+    # (the power of two at or above sqrt(T N / W) = 1448), a working copy of the state.
+    s = shape(B=8, T=8192, H=4, sqrt_n=128, W=64, R=64, d_v=512)
+    tiles = 8 * 4 * (512 // 32)
+    N, C = 16384, 2048
+    ckpt = tiles * (8192 // C - 1) * N * 32 * 4
+    log = tiles * C * 64 * 32 * 4
+    part = 8 * 8192 * 4 * (512 // 32) * (64 + 64 + 2) * 4
+    rec = 8 * 4 * 8192 * (4 * 64 + 4) * 4
+    work = 8 * 4 * N * 512 * 4
+    assert lib.sdm_scan_backward_workspace_bytes(ctypes.byref(s)) == ckpt + log + part + rec + work
