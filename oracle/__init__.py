@@ -269,7 +269,8 @@ class Oracle:
         """The recurrence on the block-scaled fp8 state (codes [B,H,N,d_v],
         exps [B,H,N,d_v/16], not modified). Returns (y float64, codes_T, exps_T)."""
         idx_w, idx_r = _i32(idx_w), _i32(idx_r)
-        w_w, w_r, v, alpha, beta = _f32(w_w), _f32(w_r), _f32(v), _f32(alpha), _f32(beta)
+        w_w, w_r = _f64(w_w), _f64(w_r)
+        v, alpha, beta = _f32(v), _f32(alpha), _f32(beta)
         C = np.ascontiguousarray(codes, dtype=np.uint8).copy()
         X = np.ascontiguousarray(exps, dtype=np.int8).copy()
         B, T, H, W = idx_w.shape

@@ -38,8 +38,9 @@
 //      ([explainer] 3.4 "高效训练" says only that a memory-efficient backward
 //      exists and leaves its details to an appendix the pages do not show).
 //   7. A block-scaled fp8 state (E4M3 values, one power-of-two scale per 16
-//      row values; see "block-scaled fp8 state" below): the recurrence with
-//      each written row computed in fp32 in the kernels' order and re-quantised.
+//      row values; see "block-scaled fp8 state" below): the recurrence of
+//      steps 3-4 on the decoded state, each written row computed in double by
+//      the pages' two-step write and then re-quantised.
 //
 // Parity status: selection, weights, write, read and epilogue are each pinned by
 // tests that do not re-run this file's formulas (exact-rational brute force,
@@ -195,10 +196,14 @@ void rmsnorm_gate_row(double* y, const G* g, int32_t d_v, double eps) {
 // subnormals down to 2^-9; no infinities; largest finite 448; S.1111.111 is
 // NaN and never produced) with one power-of-two scale 2^e per 16 consecutive
 // values of a state row (block scaling in the manner of the OCP MX formats,
-// with blocks of 16). For a block with largest magnitude m > 0 the exponent is
-// e = floor(log2 m) - 8, so that m / 2^e lies in [256, 512); every value is
-// rounded to nearest-even onto the E4M3 grid after division by 2^e and
-// clamped to +-448. An all-zero block has e = 0.
+// with blocks of 16). Every value is rounded to nearest-even onto the E4M3
+// grid after division by 2^e; for a block with largest magnitude m > 0, e is
+// the smallest integer for which that rounding of m / 2^e is at most 448,
+// i.e. the smallest e with m <= 464 * 2^e (464 lies halfway between 448 and
+// the next step, 480, and rounds to the even 448). So m / 2^e lies in
+// (232, 464], no value of a block is ever clamped, and re-quantising a
+// decoded block returns the same codes and exponent (its rounded maximum lies
+// in [240, 448]). An all-zero block has e = 0.
 
 // E4M3 code of a double (round to nearest, ties to even; clamped to 448).
 uint8_t round_e4m3(double x) {
@@ -243,18 +248,31 @@ double decode_e4m3(uint8_t c) {
   return sign * std::ldexp(1.0 + m / 8.0, e - 7);
 }
 
-// Scale exponent of a block of n values (see above).
-int block_exponent(const float* x, int n) {
+// Scale exponent of a block of n values (see above): the smallest e with
+// max|x| <= 464 * 2^e.
+template <class X>
+int block_exponent(const X* x, int n) {
   double mx = 0.0;
   for (int i = 0; i < n; ++i) mx = std::max(mx, std::fabs(static_cast<double>(x[i])));
   if (mx == 0.0) return 0;
   int k = 0;
-  std::frexp(mx, &k);
+  std::frexp(mx, &k);  // mx in [2^(k-1), 2^k)
+  int e = (k - 1) - 8;  // mx / 2^e in [256, 512)
 #if ORACLE_MUTANT == 19
-  return (k - 1) - 7;  // planted: one binade too high, the block max lands in [128, 256)
+  return e;  // planted: a block maximum above 464 * 2^e is clipped to 448 * 2^e
 #else
-  return (k - 1) - 8;
+  if (std::ldexp(mx, -e) > 464.0) ++e;  // (464, 512) would saturate: one binade up, (232, 256)
+  return e;
 #endif
+}
+
+// Quantises one block of 16 values: codes[16], returns the exponent (kept in
+// the int8 range; blocks beyond it use the nearest exponent).
+template <class X>
+int quantize_block(const X* x, uint8_t* codes) {
+  const int e = std::max(-127, std::min(127, block_exponent(x, 16)));
+  for (int i = 0; i < 16; ++i) codes[i] = round_e4m3(std::ldexp(static_cast<double>(x[i]), -e));
+  return e;
 }
 
 // Stores a freshly computed state value: rounded to fp32 (or to bf16 and kept
@@ -624,25 +642,20 @@ double oracle_decode_e4m3(uint8_t c) { return decode_e4m3(c); }
 // Quantises n_blocks blocks of 16 fp32 values: codes [n_blocks*16] uint8,
 // exps [n_blocks] int8 (the block scale is 2^exp).
 int oracle_quantize_fp8blk(const float* x, int64_t n_blocks, uint8_t* codes, int8_t* exps) {
-  for (int64_t bI = 0; bI < n_blocks; ++bI) {
-    // (the stored exponent is an int8; blocks beyond its range use the nearest one)
-    const int e = std::max(-127, std::min(127, block_exponent(x + bI * 16, 16)));
-    exps[bI] = static_cast<int8_t>(e);
-    for (int i = 0; i < 16; ++i) codes[bI * 16 + i] = round_e4m3(std::ldexp(static_cast<double>(x[bI * 16 + i]), -e));
-  }
+  for (int64_t bI = 0; bI < n_blocks; ++bI) exps[bI] = static_cast<int8_t>(quantize_block(x + bI * 16, codes + bI * 16));
   return 0;
 }
 
 // The recurrence with the block-scaled fp8 state. The state is codes
 // [B,H,N,d_v] uint8 and exps [B,H,N,d_v/16] int8 (in/out); d_v a multiple of
-// 16. A written row is computed in fp32 exactly as the recurrence kernels do
-// (cw = beta k, aw = alpha (1 - cw), m' = fma(aw, m, cw v), round-to-nearest
-// fp32 operations) from the decoded row, then every 16-value block of it is
-// quantised, so both sides take each code decision from the same fp32 value.
-// y (double) is the read of the decoded state after the write.
-// Weights w_w, w_r are the fp32 weights the kernels get.
+// 16. Each written row follows the pages' two-step write ([explainer] 3.1
+// step 2) in double on the decoded row: m~ = alpha * M[i];
+// M[i] = m~ + beta * k_i * (v - m~); the double row is then quantised block
+// by block (the reduced-precision store). y (double) is the read of the
+// decoded state after the write ([explainer] 3.1 step 3).
+//   w_w, w_r: the selection weights (double, e.g. from oracle_pkm_topk).
 int oracle_scan_fp8blk(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, int32_t W, int32_t R,
-                       const int32_t* idx_w, const float* w_w, const int32_t* idx_r, const float* w_r,
+                       const int32_t* idx_w, const double* w_w, const int32_t* idx_r, const double* w_r,
                        const float* v, const float* alpha, const float* beta, uint8_t* codes, int8_t* exps,
                        double* y, int32_t n_threads) {
   if (B < 0 || T < 0 || H < 0 || N < 1 || d_v < 16 || d_v % 16 != 0 || W < 0 || R < 0) return -1;
@@ -656,24 +669,23 @@ int oracle_scan_fp8blk(int32_t B, int32_t T, int32_t H, int64_t N, int32_t d_v, 
     const int32_t b = static_cast<int32_t>(u / H);
     uint8_t* C = codes + (static_cast<int64_t>(b) * H + h) * N * d_v;
     int8_t* X = exps + (static_cast<int64_t>(b) * H + h) * N * nb;
-    std::vector<float> row(static_cast<size_t>(d_v));
-    auto decoded = [&](int64_t i, int32_t c) {
-      return static_cast<float>(decode_e4m3(C[i * d_v + c]) * std::ldexp(1.0, X[i * nb + c / 16]));
-    };
+    std::vector<double> row(static_cast<size_t>(d_v));
+    auto decoded = [&](int64_t i, int32_t c) { return decode_e4m3(C[i * d_v + c]) * std::ldexp(1.0, X[i * nb + c / 16]); };
     for (int32_t t = 0; t < T; ++t) {
       const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;
-      const float a_t = alpha[th], b_t = beta[th];
+      const double a_t = alpha[th], b_t = beta[th];
       for (int32_t j = 0; j < W; ++j) {
         const int64_t i = idx_w[th * W + j];
-        const float cw = b_t * w_w[th * W + j];
-        const float aw = a_t * (1.0f - cw);
-        for (int32_t c = 0; c < d_v; ++c) row[c] = std::fma(aw, decoded(i, c), cw * v[th * d_v + c]);
-        oracle_quantize_fp8blk(row.data(), nb, C + i * d_v, X + i * nb);
+        const double k_i = w_w[th * W + j];
+        for (int32_t c = 0; c < d_v; ++c) {
+          const double m_tilde = a_t * decoded(i, c);
+          row[c] = m_tilde + b_t * k_i * (static_cast<double>(v[th * d_v + c]) - m_tilde);
+        }
+        for (int32_t q = 0; q < nb; ++q) X[i * nb + q] = static_cast<int8_t>(quantize_block(row.data() + 16 * q, C + i * d_v + 16 * q));
       }
       for (int32_t c = 0; c < d_v; ++c) {
         double acc = 0.0;
-        for (int32_t r = 0; r < R; ++r)
-          acc += static_cast<double>(w_r[th * R + r]) * static_cast<double>(decoded(idx_r[th * R + r], c));
+        for (int32_t r = 0; r < R; ++r) acc += w_r[th * R + r] * decoded(idx_r[th * R + r], c);
         y[th * d_v + c] = acc;
       }
     }

@@ -545,22 +545,29 @@ def pin_e4m3_rounding(o):
 
 
 def pin_fp8blk_blocks(o):
-    """Block scales put each block's largest magnitude in [256, 512) (an
-    all-zero block gets exponent 0), codes are the exact rounding of x / 2^e,
-    and quantising a dequantised block gives it back."""
+    """Each block's exponent is the smallest e for which the nearest-even
+    E4M3 rounding of max|x| / 2^e is at most 448, i.e. max|x| <= 464 * 2^e
+    (464 is the midpoint of 448 and the next step 480 and rounds to the even
+    448), so the largest magnitude lands in (232, 464] and nothing is clipped;
+    an all-zero block gets exponent 0. Codes are the exact rounding of
+    x / 2^e, and quantising a dequantised block gives it back."""
     rng = np.random.default_rng(4)
     x = rng.standard_normal((40, 16)).astype(np.float32)
     x *= np.float32(2.0) ** rng.integers(-20, 20, (40, 1)).astype(np.float32)
     x[3] = 0.0
     x[5, :15] = 0.0
+    x[7, 2] = np.float32(479.0 * 2.0 ** -3)  # maximum between 464 and 512 times a power of two
+    x[8, :] = np.float32(464.0 * 2.0 ** 5)   # maximum exactly on 464 * 2^e: stays in that binade
+    x[9, 4] = np.float32(450.0 * 2.0 ** -7)  # maximum between 448 and 464: rounds to 448, not clipped
     codes, exps = o.quantize_fp8blk(x)
     for i in range(x.shape[0]):
-        m = float(np.abs(x[i]).max())
-        if m == 0.0:
+        m = Fraction(float(np.abs(x[i]).max()))
+        if m == 0:
             assert exps[i, 0] == 0 and not (codes[i] & 0x7F).any()
             continue
-        e = math.frexp(m)[1] - 1 - 8
-        assert exps[i, 0] == e, (i, exps[i, 0], e)
+        e = int(exps[i, 0])
+        assert Fraction(232) < m / Fraction(2) ** e <= Fraction(464), (i, e, float(m))
+        assert _rne_e4m3(m / Fraction(2) ** e) & 0x7F == 0x7E or m / Fraction(2) ** e < 448, (i, e)
         for j in range(16):
             assert codes[i, j] == _rne_e4m3(Fraction(float(x[i, j])) / Fraction(2) ** e), (i, j)
     deq = o.dequantize_fp8blk(codes, exps).astype(np.float32)

@@ -34,7 +34,7 @@ MUTANTS = {
     16: "backward: softmax mean not subtracted",
     17: "backward: score halves swapped",
     18: "backward: RMS-norm normaliser treated as a constant",
-    19: "fp8 state: block scale one binade too high",
+    19: "fp8 state: block maximum above 448 clipped (scale one binade too low)",
     20: "fp8 state: rounding toward zero",
     21: "fp8 state: overflow to the NaN code",
 }
