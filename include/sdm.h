@@ -35,7 +35,15 @@
  *     even on every store).
  *   - Not thread-safe with respect to one stream; distinct streams may call
  *     concurrently. The only library-wide state is the per-device error word
- *     and the thread-local message behind sdm_last_error().
+ *     and the thread-local message behind sdm_last_error(). The error word is
+ *     shared by all streams of a device: sdm_stream_check() on any stream
+ *     reports (and clears) the bits set by every stream's calls since the last
+ *     check, so a multi-stream caller should check after a common sync point.
+ *   - A bounded wait that expires (kernels wait at most ~2 s on their own
+ *     copies) stops its thread block; copies it had in flight may still land
+ *     in shared memory that a later block on the same SM then uses, so after a
+ *     wait-timeout report every output of every call since the last check is
+ *     undefined and must be discarded, not only the tile that timed out.
  */
 #ifndef SDM_B200_SDM_H_
 #define SDM_B200_SDM_H_
@@ -110,9 +118,11 @@ SDM_API const char* sdm_status_string(sdm_status_t status);
 SDM_API const char* sdm_last_error(void);
 
 /* Quantises n_blocks blocks of 16 fp32 values into the SDM_FP8_B16 format:
- * e = floor(log2 max|x|) - 8 per block (clamped to [-127, 127]; 0 for an
- * all-zero block), codes = round-to-nearest-even(x / 2^e) onto the E4M3 grid,
- * clamped to +-448. x [n_blocks * 16] fp32; codes [n_blocks * 16] uint8;
+ * codes = round-to-nearest-even(x / 2^e) onto the E4M3 grid, with e per block
+ * the smallest integer for which that rounding of max|x| / 2^e is at most 448
+ * (i.e. max|x| <= 464 * 2^e; clamped to [-127, 127]; 0 for an all-zero
+ * block), so no value saturates and re-quantising a decoded block returns it
+ * unchanged. x [n_blocks * 16] fp32; codes [n_blocks * 16] uint8;
  * exps [n_blocks] int8 (all device, caller owned; x and codes 16-byte aligned). */
 SDM_API sdm_status_t sdm_quantize_fp8blk(const float* x, int64_t n_blocks, uint8_t* codes, int8_t* exps,
                                  void* stream);
@@ -364,9 +374,11 @@ SDM_API sdm_status_t sdm_layer_forward_noalloc(const sdm_shape_t* shape, const v
                                        const void* g, const void* M0, void* M_out, float* y,
                                        void* stream);
 
-/* Waits for `stream`, then reads and clears the current device's error word.
- * Returns SDM_ERR_DEVICE_FAULT if it was set (sdm_last_error() gives the bits),
- * SDM_ERR_CUDA if the synchronisation failed, else SDM_OK. */
+/* Waits for `stream`, then reads and clears the current device's error word
+ * (shared by all streams of the device; see the conventions above).
+ * Returns SDM_ERR_DEVICE_FAULT if it was set (sdm_last_error() gives the bits
+ * in hex and names them), SDM_ERR_CUDA if the synchronisation failed, else
+ * SDM_OK. */
 SDM_API sdm_status_t sdm_stream_check(void* stream);
 
 #ifdef __cplusplus

@@ -28,7 +28,9 @@ namespace {
 
 using sdm::bf16;
 
-// The per-device error word (one copy per device context).
+// The per-device error word (one copy per device context). Every stream's
+// calls on a device set bits in the same word, so a check on any stream
+// reports (and clears) them all.
 __device__ unsigned g_device_error;
 
 thread_local std::string g_last_error;
@@ -1315,9 +1317,11 @@ sdm_status_t sdm_stream_check(void* stream) {
   if (word != 0) {
     const unsigned zero = 0;
     cudaMemcpy(dev->err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
-    std::string msg = "device error word 0x" + std::to_string(word) + ":";
+    char hex[16];
+    std::snprintf(hex, sizeof(hex), "0x%x", word);
+    std::string msg = std::string("device error word ") + hex + ":";
     if (word & sdm::kErrIndexOutOfRange) msg += " slot index outside [0, N) skipped;";
-    if (word & sdm::kErrWaitTimeout) msg += " bounded wait expired;";
+    if (word & sdm::kErrWaitTimeout) msg += " bounded wait expired (the outputs of every call since the last check are undefined);";
     return fail(SDM_ERR_DEVICE_FAULT, msg);
   }
   return ok();

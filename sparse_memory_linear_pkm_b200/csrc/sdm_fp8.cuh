@@ -3,11 +3,15 @@
 // quantisation of the state at N = 10^7 (SDM explainer, "工程落地关键点", item
 // 2) without fixing a format; this one is OCP FP8 E4M3 (bias 7, subnormals
 // down to 2^-9, largest finite 448, no infinities, S.1111.111 never produced)
-// scaled in blocks of 16 as the OCP MX formats do in blocks of 32: for a block
-// whose largest magnitude is m > 0, e = floor(log2 m) - 8 (clamped to the int8
-// range), codes = round-to-nearest-even(x / 2^e) clamped to +-448; an all-zero
-// block has e = 0. Every scaling is by a power of two, exact in fp32, so the
-// code decisions depend only on the fp32 values being quantised.
+// scaled in blocks of 16 as the OCP MX formats do in blocks of 32: codes =
+// round-to-nearest-even(x / 2^e), and for a block whose largest magnitude is
+// m > 0, e is the smallest integer for which that rounding of m / 2^e stays at
+// most 448, i.e. the smallest e with m <= 464 * 2^e (464, halfway between 448
+// and the next step 480, rounds to the even 448), clamped to the int8 range;
+// an all-zero block has e = 0. So no value is ever clamped, and re-quantising
+// a decoded block gives back the same codes and exponent. Every scaling is by
+// a power of two, exact in fp32, so the code decisions depend only on the
+// fp32 values being quantised.
 //
 // Layout of a state of R rows of d_v values: R * d_v code bytes, then
 // R * d_v / 16 exponent bytes (int8).
@@ -19,7 +23,8 @@
 
 namespace sdm {
 
-struct Fp8Blk {};  // state-type tag of the block-scaled fp8 state
+struct Fp8Blk {};  // state-type tag of the block-scaled fp8 state: one code byte per value
+static_assert(sizeof(Fp8Blk) == 1, "Fp8Blk pointers step over code bytes");
 
 // 2^e as an fp32 for e in [-127, 127] (2^-127 is subnormal).
 __device__ __forceinline__ float pow2f(int e) {
@@ -48,7 +53,13 @@ __device__ __forceinline__ int fp8blk_pack16(const float* x, uint4* u) {
   float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(x[i]));
-  const int e = mx > 0.0f ? min(127, max(-127, ilogbf(mx) - 8)) : 0;
+  int e = 0;
+  if (mx > 0.0f) {
+    int k;
+    const float f = frexpf(mx, &k);            // mx = f * 2^k, f in [0.5, 1): mx / 2^(k-9) = 512 f
+    e = (k - 9) + (f > 0.90625f ? 1 : 0);      // 512 f > 464: one binade up
+    e = min(127, max(-127, e));
+  }
   const float inv = pow2f(-e);
   uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll

@@ -1,0 +1,159 @@
+"""The block-scaled fp8 state (E4M3 codes, one power-of-two scale per 16 row
+values) against the oracle, through the C ABI.
+
+Two bounds, both derived from the E4M3 grid rather than measured:
+
+* One step from the same state. The kernel forms a written row in fp32
+  (factored form), the oracle by the pages' two-step write in double; the two
+  pre-quantisation values differ by a few fp32 roundings. Rounding both to
+  nearest on the E4M3 grid then gives values at most one grid step apart (one
+  step of the coarser grid when the two sides pick different block exponents,
+  which happens only when the block maximum sits on the exponent threshold).
+  So every decoded value of a written row is within one step, taken at the
+  larger of the two magnitudes and the larger of the two exponents, and each
+  y value within sum_r |q_r| * (that step of row r) plus fp32 read rounding.
+  Each step starts from the oracle's state, so the bound does not compound.
+
+* Many steps against the unrounded double recurrence. Quantising x adds at most
+  half a step: max(2^-4 |x|, 2^-10 * 2^e) (normal and subnormal E4M3), and
+  2^e < max_block|x| / 232 because the exponent is the smallest with
+  max_block|x| <= 464 * 2^e. A write contracts an earlier error by
+  a = alpha (1 - beta k) and adds a new one, so the error bound E of every
+  state value obeys E <- a E + half_step(|x_exact| + a E); y errs by at most
+  sum_r |q_r| E[r]. Small slack terms cover the kernel's fp32 arithmetic.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from parity_helpers import f32
+from sparse_memory_linear_pkm_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+FP32_SLACK = 1e-6  # relative: fp32 products, sums and fp32 softmax weights against double
+
+
+def _dequant(oracle, codes, exps):
+    return oracle.dequantize_fp8blk(codes, exps)
+
+
+def _step_of(mag, e):
+    """Spacing of the E4M3 grid scaled by 2^e at magnitude mag (subnormal
+    spacing 2^-9 below 2^-6, 2^(j-3) in the binade [2^j, 2^(j+1)))."""
+    s = np.ldexp(mag, -e)
+    _, k = np.frexp(np.where(s > 0, s, 1.0))
+    j = np.maximum(np.where(s > 0, k - 1, -6), -6)
+    return np.ldexp(1.0, (j - 3) + e)
+
+
+def _half_step_bound(a):
+    """Upper bound of the quantisation error of values with magnitude <= a
+    [..., d_v] (blocks of 16 along the last axis)."""
+    blk = a.reshape(a.shape[:-1] + (-1, 16)).max(axis=-1)
+    floor = np.repeat(np.ldexp(blk / 232.0, -10), 16, axis=-1)
+    return np.maximum(np.ldexp(a, -4), floor)
+
+
+def _buf(codes, exps, device):
+    return torch.from_numpy(np.concatenate([codes.reshape(-1), exps.reshape(-1).view(np.uint8)])).to(device)
+
+
+def _split(buf, codes_shape, exps_shape):
+    got = buf.cpu().numpy()
+    n = int(np.prod(codes_shape))
+    return got[:n].reshape(codes_shape), got[n:].view(np.int8).reshape(exps_shape)
+
+
+def _setup(oracle, seed, **kw):
+    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"].replace(**kw)
+    inp = synth.make_inputs(shape, seed=seed, device="cpu")
+    M0 = f32(inp["M0"])
+    codes, exps = oracle.quantize_fp8blk(np.broadcast_to(M0[None], (shape.B,) + M0.shape).copy())
+    idx_w, w_w = oracle.pkm_topk(f32(inp["kp"]), shape.W)
+    idx_r, w_r = oracle.pkm_topk(f32(inp["qp"]), shape.R)
+    return shape, inp, codes, exps, (idx_w, w_w, idx_r, w_r)
+
+
+def _gpu_step(sdm, d, t, buf, shape):
+    sl = {k: d[k][:, t:t + 1].contiguous() for k in ("kp", "qp", "v", "alpha", "beta")}
+    y = sdm.layer_step(sl["kp"], sl["qp"], sl["v"], sl["alpha"], sl["beta"], buf, shape.W, shape.R)
+    sdm.stream_check()
+    return y.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("W", [64, 16])
+def test_decode_fp8_step_within_one_grid_step(sdm, oracle, cuda_device, W):
+    shape, inp, codes, exps, (idx_w, w_w, idx_r, w_r) = _setup(oracle, 41, B=2, T=6, H=2, W=W, R=W)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    v, alpha, beta = f32(inp["v"]), f32(inp["alpha"]), f32(inp["beta"])
+    for t in range(shape.T):
+        buf = _buf(codes, exps, cuda_device)
+        y = _gpu_step(sdm, d, t, buf, shape)
+        gc, ge = _split(buf, codes.shape, exps.shape)
+        sl = slice(t, t + 1)
+        oy, oc, oe = oracle.scan_fp8blk(idx_w[:, sl], w_w[:, sl], idx_r[:, sl], w_r[:, sl], v[:, sl], alpha[:, sl],
+                                        beta[:, sl], codes, exps)
+        written = np.zeros(codes.shape[:3], dtype=bool)
+        for b in range(shape.B):
+            for h in range(shape.H):
+                written[b, h, idx_w[b, t, h]] = True
+        # rows the step does not write are left bit for bit
+        assert np.array_equal(gc[~written], codes[~written]) and np.array_equal(ge[~written], exps[~written])
+        Dk, Do = _dequant(oracle, gc, ge), _dequant(oracle, oc, oe)
+        e_max = np.repeat(np.maximum(ge, oe).astype(np.int64), 16, axis=-1)
+        step = _step_of(np.maximum(np.abs(Dk), np.abs(Do)), e_max) * (1 + FP32_SLACK)
+        step[~written] = 0.0
+        diff = np.abs(Dk - Do)
+        assert np.all(diff <= step), ("state", t, float((diff - step).max()))
+        ybound = np.zeros_like(oy)
+        for b in range(shape.B):
+            for h in range(shape.H):
+                q = np.abs(w_r[b, t, h])[:, None]
+                rows = idx_r[b, t, h]
+                ybound[b, 0, h] = (q * step[b, h, rows]).sum(0) + 4 * FP32_SLACK * (q * np.abs(Do[b, h, rows])).sum(0)
+        dy = np.abs(y - oy)
+        assert np.all(dy <= ybound + 1e-30), ("y", t, float((dy - ybound).max()))
+        codes, exps = oc, oe  # the next step starts from the oracle's state
+
+
+def test_decode_fp8_state_error_against_exact_recurrence(sdm, oracle, cuda_device):
+    shape, inp, codes, exps, (idx_w, w_w, idx_r, w_r) = _setup(oracle, 43, B=2, T=8, H=2)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    v, alpha, beta = (f32(inp[k]).astype(np.float64) for k in ("v", "alpha", "beta"))
+    buf = _buf(codes, exps, cuda_device)
+    M = _dequant(oracle, codes, exps)  # the exact recurrence starts from the same decoded state
+    E = np.zeros_like(M)
+    worst = 0.0
+    for t in range(shape.T):
+        y = _gpu_step(sdm, d, t, buf, shape)
+        sl = slice(t, t + 1)
+        M_old = M
+        oy, M = oracle.scan_f64(idx_w[:, sl], w_w[:, sl], idx_r[:, sl], w_r[:, sl], v[:, sl], alpha[:, sl],
+                                beta[:, sl], M_old)
+        E_new = E.copy()
+        for b in range(shape.B):
+            for h in range(shape.H):
+                a_t, b_t = alpha[b, t, h], beta[b, t, h]
+                for j, i in enumerate(idx_w[b, t, h]):
+                    cw = b_t * w_w[b, t, h, j]
+                    aw = a_t * (1.0 - cw)
+                    carried = aw * E[b, h, i]
+                    slack = FP32_SLACK * (aw * (np.abs(M_old[b, h, i]) + E[b, h, i]) + cw * np.abs(v[b, t, h]))
+                    E_new[b, h, i] = carried + slack + _half_step_bound(np.abs(M[b, h, i]) + carried + slack)
+        E = E_new
+        gc, ge = _split(buf, codes.shape, exps.shape)
+        Dk = _dequant(oracle, gc, ge)
+        err = np.abs(Dk - M)
+        assert np.all(err <= E), ("state", t, float((err - E).max()))
+        for b in range(shape.B):
+            for h in range(shape.H):
+                q = np.abs(w_r[b, t, h])[:, None]
+                rows = idx_r[b, t, h]
+                bound = (q * E[b, h, rows]).sum(0) + 4 * FP32_SLACK * (q * (np.abs(M[b, h, rows]) + E[b, h, rows])).sum(0)
+                dy = np.abs(y[b, 0, h] - oy[b, 0, h])
+                assert np.all(dy <= bound + 1e-30), ("y", t, b, h, float((dy - bound).max()))
+        worst = max(worst, float(np.abs(y - oy).max() / max(np.abs(oy).max(), 1e-30)))
+    # the fp8 state's read error, relative to the largest read value, stays at the format's precision
+    assert worst < 0.25, worst

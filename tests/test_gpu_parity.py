@@ -375,35 +375,6 @@ def test_quantize_fp8blk_matches_oracle(sdm, oracle, cuda_device):
     assert np.array_equal(exps.cpu().numpy(), oe.reshape(-1))
 
 
-def test_decode_fp8_state_matches_oracle(sdm, oracle, cuda_device):
-    """Decode steps (T = 1) on the block-scaled fp8 state against the oracle's
-    recurrence on the same format. Both compute each written row in the same
-    fp32 order before quantising it; the selection weights differ in the last
-    bits (fp32 softmax on the GPU, double in the oracle), which can move a
-    value across a rounding boundary, so a few codes may differ by one step."""
-    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"].replace(B=2, T=6, H=2)
-    inp = synth.make_inputs(shape, seed=41, device="cpu")
-    M0 = f32(inp["M0"])
-    oc, oe = oracle.quantize_fp8blk(np.broadcast_to(M0[None], (shape.B,) + M0.shape).copy())
-    buf = torch.from_numpy(np.concatenate([oc.reshape(-1), oe.reshape(-1).view(np.uint8)])).to(cuda_device)
-    d = {k: v.to(cuda_device) for k, v in inp.items()}
-    ys = []
-    for t in range(shape.T):
-        sl = {k: d[k][:, t:t + 1].contiguous() for k in ("kp", "qp", "v", "alpha", "beta")}
-        ys.append(sdm.layer_step(sl["kp"], sl["qp"], sl["v"], sl["alpha"], sl["beta"], buf, shape.W, shape.R))
-    sdm.stream_check()
-    y = torch.cat(ys, dim=1).cpu().numpy()
-    idx_w, w_w = oracle.pkm_topk(f32(inp["kp"]), shape.W)
-    idx_r, w_r = oracle.pkm_topk(f32(inp["qp"]), shape.R)
-    oy, C, X = oracle.scan_fp8blk(idx_w, w_w.astype(np.float32), idx_r, w_r.astype(np.float32), f32(inp["v"]),
-                                  f32(inp["alpha"]), f32(inp["beta"]), oc, oe)
-    assert_rel_close(y, oy, 1e-2, "y")
-    n = C.size
-    got = buf.cpu().numpy()
-    gc, ge = got[:n].reshape(C.shape), got[n:].view(np.int8).reshape(X.shape)
-    assert (gc != C).mean() <= 1e-3 and (ge != X).mean() <= 1e-3, ((gc != C).mean(), (ge != X).mean())
-
-
 def test_fp8_state_only_in_the_decode_step(sdm, cuda_device):
     shape = synth.WORKLOADS["tiny_n1024_dv16"].replace(B=1, T=2, H=1)
     inp = synth.make_inputs(shape, seed=1, device=cuda_device)
