@@ -36,7 +36,10 @@ import sparse_memory_linear_pkm_b200 as sdm  # noqa: E402
 from sparse_memory_linear_pkm_b200 import synth  # noqa: E402
 
 METRIC = "SDM layer tokens/s (B·T) and achieved HBM/L2 GB/s vs roofline on 1 B200"
-DEFAULT_WORKLOAD = "d2048_h16_n1024_dv128"
+DEFAULT_WORKLOAD = "long_t1m_n262144_dv2048"
+# Measured after the headline at N = 1 (device time only), so one run also
+# shows the driver the smaller workloads.
+EXTRA_WORKLOADS = ("d2048_h16_n1024_dv128", "d2048_h4_n16384_dv512", "d4096_h8_n16384_dv512")
 FALLBACK_HBM_GBS = 6650.0
 SMEM_BYTES_PER_CLK_PER_SM = 128
 NVML_REASONS = {
@@ -49,8 +52,8 @@ NVML_REASONS = {
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="sdm", choices=["sdm", "reference"])
     ap.add_argument("--seed", type=int, default=0)
@@ -58,6 +61,7 @@ def parse_args():
     ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the device-time lines of the smaller workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--decode", action="store_true",
                     help="time decode steps instead: one token per call (sdm_layer_step), state carried")
@@ -285,7 +289,7 @@ def run_reference(args, dist: Dist):
                             with_gate=args.epilogue)
     o = oracle.get()
     threads = oracle.default_threads()
-    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    budget_s = min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup))
     Bs, Ts, _ = calibrate_sample(o, shape.replace(B=1, T=min(shape.T, 4096)), inp, threads, budget_s)
     sample = oracle_sample_inputs(inp, Bs, Ts)
     for _ in range(args.warmup):
@@ -309,6 +313,112 @@ def workload_config(shape: synth.Shape, args, dist: Dist) -> dict:
             "d_v": shape.d_v, "W": shape.W, "R": shape.R, "in_dtype": shape.in_dtype,
             "state_dtype": shape.state_dtype, "epilogue": bool(args.epilogue), "seed": args.seed,
             "parallelism": f"dp{dist.world} (independent batch per rank)"}
+
+
+def _cudart():
+    """The CUDA runtime torch already loaded (same context, streams and pinned
+    allocations), for the caller-side cudaMemcpyAsync calls of the e2e leg."""
+    import glob
+
+    names = glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
+                                   "libcudart.so*"))
+    names += ["libcudart.so.12", "/usr/local/cuda/lib64/libcudart.so.12"]
+    for name in names:
+        try:
+            lib = ctypes.CDLL(name)
+        except OSError:
+            continue
+        lib.cudaMemcpyAsync.restype = ctypes.c_int
+        lib.cudaMemcpyAsync.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int,
+                                        ctypes.c_void_p]
+        return lib
+    raise RuntimeError("no CUDA runtime library found for the e2e copies")
+
+
+H2D, D2H = 1, 2  # cudaMemcpyKind
+
+
+def e2e_through_c_abi(args, dist: Dist, dev, shape: synth.Shape, sh, inp: dict, g, ws, stream) -> dict:
+    """End to end through the C ABI with host buffers: every step copies its
+    inputs from pinned host memory (one cudaMemcpyAsync per tensor), calls
+    sdm_layer_forward, and copies y and M_T back to pinned host memory, all
+    inside the timed region. Copies run on two copy streams and the device
+    buffers are doubled, so step k's transfers overlap steps k-1 and k+1."""
+    rt = _cudart()
+    lib = sdm.native.load()
+    names = ("kp", "qp", "v", "alpha", "beta")
+    host = {}
+    for k in names:
+        host[k] = torch.empty(inp[k].shape, dtype=inp[k].dtype, pin_memory=True)
+        host[k].copy_(inp[k])
+    M0 = inp["M0"]
+    dinp = [{k: torch.empty_like(inp[k]) for k in names} for _ in range(2)]
+    ys = [torch.empty((shape.B, shape.T, shape.H, shape.d_v), dtype=torch.float32, device=dev) for _ in range(2)]
+    Ms = [torch.empty((shape.B,) + tuple(M0.shape), dtype=M0.dtype, device=dev) for _ in range(2)]
+    # one host copy each: the D2H copies of consecutive steps are ordered on one stream
+    y_host = torch.empty(ys[0].shape, dtype=torch.float32, pin_memory=True)
+    M_host = torch.empty(Ms[0].shape, dtype=M0.dtype, pin_memory=True)
+    nbytes = lambda t: t.numel() * t.element_size()
+    h2d = sum(nbytes(t) for t in host.values())
+    d2h = nbytes(y_host) + nbytes(M_host)
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())
+    gptr = vp(g) if g is not None else None
+
+    def copy(dst, src, n, kind, st):
+        rc = rt.cudaMemcpyAsync(vp(dst), vp(src), n, kind, ctypes.c_void_p(st.cuda_stream))
+        if rc != 0:
+            raise RuntimeError(f"cudaMemcpyAsync failed with {rc}")
+
+    def steps(n):
+        h2d_s.wait_stream(stream)
+        d2h_s.wait_stream(stream)
+        for k in range(n):
+            b = k % 2
+            if k >= 2:
+                h2d_s.wait_event(done[b])  # step k-2 has finished reading this input buffer
+            for name in names:
+                copy(dinp[b][name], host[name], nbytes(host[name]), H2D, h2d_s)
+            in_ready[b].record(h2d_s)
+            stream.wait_event(in_ready[b])
+            if k >= 2:
+                stream.wait_event(out_done[b])  # step k-2's y and M_T have left these buffers
+            d = dinp[b]
+            sdm.native.check(lib.sdm_layer_forward(ctypes.byref(sh), vp(d["kp"]), vp(d["qp"]), vp(d["v"]),
+                                                   vp(d["alpha"]), vp(d["beta"]), gptr, vp(M0), vp(Ms[b]),
+                                                   vp(ys[b]), vp(ws), nbytes(ws),
+                                                   ctypes.c_void_p(stream.cuda_stream)))
+            done[b].record(stream)
+            d2h_s.wait_event(done[b])
+            copy(y_host, ys[b], nbytes(y_host), D2H, d2h_s)
+            copy(M_host, Ms[b], nbytes(M_host), D2H, d2h_s)
+            out_done[b].record(d2h_s)
+        stream.wait_stream(h2d_s)
+        stream.wait_stream(d2h_s)
+
+    k_e2e = max(3, min(args.steps, 20 if shape.B * shape.T * shape.H <= 2 ** 22 else 5))
+    steps(2)  # warm-up
+    torch.cuda.synchronize(dev)
+    sdm.stream_check(dev)
+    dist.barrier(dev)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    steps(k_e2e)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    sdm.stream_check(dev)
+    e_ms = dist.max(s2.elapsed_time(e2), dev)
+    del dinp, ys, Ms, host, y_host, M_host
+    torch.cuda.empty_cache()
+    return {"value": aggregate_value(shape.B * shape.T * k_e2e, dist.world, e_ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+            "path": "per step through the C ABI: one cudaMemcpyAsync per input tensor from pinned host memory, "
+                    "sdm_layer_forward, cudaMemcpyAsync of y and M_T to pinned host memory; copies on two copy "
+                    "streams, device buffers doubled so transfers overlap the neighbouring steps' compute"}
 
 
 def run_sdm(args, dist: Dist):
@@ -360,85 +470,12 @@ def run_sdm(args, dist: Dist):
 
     resident = sdm.scan_variant(sh) == "resident"
     launches_per_step = int(sdm.native.load().sdm_layer_forward_launches(ctypes.byref(sh), int(args.epilogue)))
-    scan_ms = stage_ms[3]
-    th = shape.B * shape.T * shape.H
-    algo_bytes = algorithmic_bytes_per_token_head(shape, args.epilogue) * th
-    achieved = algo_bytes / (scan_ms / 1e3) / 1e9
-    peaks = measured_peaks()
     clk = clocks.summary()
-    if resident:
-        mhz = clk["sm_max_mhz"] or 1965.0
-        peak = torch.cuda.get_device_properties(dev).multi_processor_count * SMEM_BYTES_PER_CLK_PER_SM * mhz / 1e3
-        roof = {"bound": "smem", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "peak_source": f"derived: SMs x {SMEM_BYTES_PER_CLK_PER_SM} B/clk x {mhz:.0f} MHz "
-                               "(state tile resident in shared memory)"}
-    else:
-        peak = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "peak_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "of fallback"}
-    kernel = "k_scan_resident" if resident else "k_scan_streaming"
-    launch_cfg = sdm.scan_describe(sh)
-    traffic = recorded_traffic(shape.name, kernel, launch_cfg)
-    roof.update({"traffic": traffic, "kernel": kernel, "launch": launch_cfg, "ms_per_launch": scan_ms,
-                 "algorithmic_bytes_per_launch": algo_bytes})
+    roof = roofline_of(shape, sh, stage_ms[3], args.epilogue, dev, clk)
 
     e2e = None
     if not args.no_e2e:
-        # End to end through the public API: every step copies its inputs from
-        # pinned host memory and its y back to pinned host memory, inside the
-        # timed region. The copies run on two copy streams, double-buffered, so
-        # step k's transfers overlap steps k-1 and k+1's compute.
-        host = {k: inp[k].cpu().pin_memory() for k in ("kp", "qp", "v", "alpha", "beta")}
-        dinp = [{k: torch.empty_like(inp[k]) for k in host} for _ in range(2)]
-        ys = [y, torch.empty_like(y)]
-        y_host = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(2)]
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = y.numel() * y.element_size()
-        k_e2e = max(3, min(args.steps, 20))
-        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        in_ready = [torch.cuda.Event() for _ in range(2)]
-        done = [torch.cuda.Event() for _ in range(2)]
-        out_done = [torch.cuda.Event() for _ in range(2)]
-
-        def e2e_steps(n):
-            h2d_s.wait_stream(stream)
-            d2h_s.wait_stream(stream)
-            for k in range(n):
-                b = k % 2
-                with torch.cuda.stream(h2d_s):
-                    if k >= 2:
-                        h2d_s.wait_event(done[b])  # step k-2 has finished reading this input buffer
-                    for name in host:
-                        dinp[b][name].copy_(host[name], non_blocking=True)
-                    in_ready[b].record(h2d_s)
-                stream.wait_event(in_ready[b])
-                if k >= 2:
-                    stream.wait_event(out_done[b])  # step k-2's y has left this buffer
-                sdm.layer_forward(dinp[b]["kp"], dinp[b]["qp"], dinp[b]["v"], dinp[b]["alpha"], dinp[b]["beta"],
-                                  inp["M0"], shape.W, shape.R, g=g, variant=args.variant, y=ys[b], M_out=M_out,
-                                  workspace=ws)
-                done[b].record(stream)
-                with torch.cuda.stream(d2h_s):
-                    d2h_s.wait_event(done[b])
-                    y_host[b].copy_(ys[b], non_blocking=True)
-                    out_done[b].record(d2h_s)
-            stream.wait_stream(h2d_s)
-            stream.wait_stream(d2h_s)
-
-        e2e_steps(2)  # warm-up
-        torch.cuda.synchronize(dev)
-        dist.barrier(dev)
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
-        e2e_steps(k_e2e)
-        e2.record(stream)
-        torch.cuda.synchronize(dev)
-        dist.barrier(dev)
-        e_ms = dist.max(s2.elapsed_time(e2), dev)
-        e2e = {"value": aggregate_value(tokens * k_e2e, dist.world, e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
-               "path": "per step: inputs pinned host -> device, sdm_layer_forward, y -> pinned host; copies on "
-                       "two copy streams, double-buffered, overlapping the neighbouring steps' compute"}
+        e2e = e2e_through_c_abi(args, dist, dev, shape, sh, inp, g, ws, stream)
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -458,9 +495,75 @@ def run_sdm(args, dist: Dist):
                 "clocks": clk,
                 "stage_ms": {"select_k_and_q": stage_ms[0], "records": stage_ms[1], "state_init": stage_ms[2],
                              "scan": stage_ms[3], "epilogue": stage_ms[4]}}
+    del ev, inp, y, M_out, ws
+    torch.cuda.empty_cache()
+    if dist.rank == 0:
+        if dist.world == 1 and not args.no_extra and args.workload == DEFAULT_WORKLOAD:
+            line["extra_workloads"] = {name: measure_workload(name, args, dev) for name in EXTRA_WORKLOADS}
         print(json.dumps(line), flush=True)
-    del ev
     dist.close()
+
+
+def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk: dict) -> dict:
+    """Roofline of the recurrence kernel of one launch: algorithmic bytes over
+    its CUDA-event time against the measured HBM copy bandwidth (streaming),
+    or the derived shared-memory bandwidth (resident)."""
+    resident = sdm.scan_variant(sh) == "resident"
+    algo_bytes = algorithmic_bytes_per_token_head(shape, epilogue) * shape.B * shape.T * shape.H
+    achieved = algo_bytes / (scan_ms / 1e3) / 1e9
+    peaks = measured_peaks()
+    if resident:
+        mhz = clk.get("sm_max_mhz") or 1965.0
+        peak = torch.cuda.get_device_properties(dev).multi_processor_count * SMEM_BYTES_PER_CLK_PER_SM * mhz / 1e3
+        roof = {"bound": "smem", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": f"derived: SMs x {SMEM_BYTES_PER_CLK_PER_SM} B/clk x {mhz:.0f} MHz "
+                               "(state tile resident in shared memory)"}
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "of fallback"}
+    kernel = "k_scan_resident" if resident else "k_scan_streaming"
+    launch_cfg = sdm.scan_describe(sh)
+    roof.update({"traffic": recorded_traffic(shape.name, kernel, launch_cfg), "kernel": kernel, "launch": launch_cfg,
+                 "ms_per_launch": scan_ms, "algorithmic_bytes_per_launch": algo_bytes})
+    return roof
+
+
+def measure_workload(name: str, args, dev, steps: int = 5, warmup: int = 3) -> dict:
+    """Device-time throughput of one more workload (same step as the headline)."""
+    shape = synth.WORKLOADS[name]
+    inp = synth.make_inputs(shape, seed=args.seed, device=dev)
+    y = torch.empty((shape.B, shape.T, shape.H, shape.d_v), dtype=torch.float32, device=dev)
+    M_out = torch.empty((shape.B,) + tuple(inp["M0"].shape), dtype=inp["M0"].dtype, device=dev)
+    sh = sdm.make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
+                        shape.torch_state())
+    ws = torch.empty(sdm.layer_forward_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+
+    def step(events=None):
+        sdm.layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], inp["M0"], shape.W, shape.R,
+                          y=y, M_out=M_out, workspace=ws, events=events)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(steps):
+        step(ev[k])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    sdm.stream_check(dev)
+    ms = start.elapsed_time(end) / steps
+    scan_ms = sum(ev[k][3].elapsed_time(ev[k][4]) for k in range(steps)) / steps
+    roof = roofline_of(shape, sh, scan_ms, False, dev, {})
+    out = {"value": shape.B * shape.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "frac", "kernel", "launch", "ms_per_launch",
+                                              "traffic")}}
+    del inp, y, M_out, ws, ev
+    torch.cuda.empty_cache()
+    return out
 
 
 def d2h_mib(y: torch.Tensor) -> float:

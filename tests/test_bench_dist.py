@@ -73,7 +73,8 @@ def test_reference_arm_prints_one_contract_line():
     import subprocess
 
     out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--steps", "1", "--warmup",
-                          "1", "--cpu-seconds", "0.5"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+                          "1", "--cpu-seconds", "0.5", "--workload", "d2048_h16_n1024_dv128"], capture_output=True,
+                         text=True, timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
