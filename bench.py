@@ -58,7 +58,8 @@ def parse_args():
     ap.add_argument("--impl", default="sdm", choices=["sdm", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--epilogue", action="store_true", help="run the RMS-norm x gate epilogue")
-    ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming", "pipelined"])
+    ap.add_argument("--tile", type=int, default=0, help="force entry k of the kernel's tile table (0: automatic)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the device-time lines of the smaller workloads")
@@ -203,6 +204,7 @@ KERNEL_SOURCES = {
     "k_scan_resident": ("sdm_device.cuh", "sdm_records.cuh", "sdm_scan.cuh"),
     "k_scan_streaming": ("sdm_device.cuh", "sdm_records.cuh", "sdm_scan.cuh"),
     "k_pkm_topk_fast": ("sdm_device.cuh", "pkm_topk_fast.cuh"),
+    "k_scan_pipelined": ("sdm_device.cuh", "sdm_scan.cuh", "sdm_pipelined.cuh"),
 }
 
 
@@ -312,7 +314,7 @@ def workload_config(shape: synth.Shape, args, dist: Dist) -> dict:
     return {"workload": shape.name, "B": shape.B, "T": shape.T, "H": shape.H, "sqrt_n": shape.sqrt_n, "N": shape.N,
             "d_v": shape.d_v, "W": shape.W, "R": shape.R, "in_dtype": shape.in_dtype,
             "state_dtype": shape.state_dtype, "epilogue": bool(args.epilogue), "seed": args.seed,
-            "parallelism": f"dp{dist.world} (independent batch per rank)"}
+            "parallelism": f"rows partition: {dist.world} x {shape.B} batch rows over {dist.world} ranks, no collective"}
 
 
 def _cudart():
@@ -434,12 +436,12 @@ def run_sdm(args, dist: Dist):
     y = torch.empty((shape.B, shape.T, shape.H, shape.d_v), dtype=torch.float32, device=dev)
     M_out = torch.empty((shape.B,) + tuple(inp["M0"].shape), dtype=inp["M0"].dtype, device=dev)
     sh = sdm.make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
-                        shape.torch_state(), variant=args.variant)
+                        shape.torch_state(), variant=args.variant, tile=args.tile)
     ws = torch.empty(sdm.layer_forward_workspace_bytes(sh), dtype=torch.uint8, device=dev)
 
     def step(events=None, src=inp):
         sdm.layer_forward(src["kp"], src["qp"], src["v"], src["alpha"], src["beta"], inp["M0"], shape.W, shape.R,
-                          g=g, variant=args.variant, y=y, M_out=M_out, workspace=ws, events=events)
+                          g=g, variant=args.variant, y=y, M_out=M_out, workspace=ws, events=events, tile=args.tile)
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -487,7 +489,7 @@ def run_sdm(args, dist: Dist):
         cfg = workload_config(shape, args, dist)
         cfg["l2"] = (f"no flush between steps: per-step inputs {in_mb:.0f} MiB and y {d2h_mib(y):.0f} MiB "
                      f"exceed the {l2_mb:.0f} MiB L2")
-        cfg["variant"] = "resident" if resident else "streaming"
+        cfg["variant"] = sdm.scan_variant(sh)
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
@@ -522,7 +524,8 @@ def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk
         peak = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_source": "of measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "of fallback"}
-    kernel = "k_scan_resident" if resident else "k_scan_streaming"
+    kernel = {"resident": "k_scan_resident", "streaming": "k_scan_streaming",
+              "pipelined": "k_scan_pipelined"}[sdm.scan_variant(sh)]
     launch_cfg = sdm.scan_describe(sh)
     roof.update({"traffic": recorded_traffic(shape.name, kernel, launch_cfg), "kernel": kernel, "launch": launch_cfg,
                  "ms_per_launch": scan_ms, "algorithmic_bytes_per_launch": algo_bytes})

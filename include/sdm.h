@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define SDM_ABI_VERSION 1
+#define SDM_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define SDM_API __attribute__((visibility("default")))
@@ -82,10 +82,14 @@ typedef enum sdm_dtype { SDM_F32 = 0, SDM_BF16 = 1, SDM_FP8_B16 = 2 } sdm_dtype_
 
 /* Which recurrence kernel runs (sdm_shape_t.variant). */
 typedef enum sdm_variant {
-  SDM_VARIANT_AUTO = 0,      /* pick by size: resident when the state tile fits */
+  SDM_VARIANT_AUTO = 0,      /* pick by size: resident when the state tile fits, pipelined
+                                when 128-byte column tiles leave SMs idle, else streaming */
   SDM_VARIANT_RESIDENT = 1,  /* the (b,h) state column tile lives in shared memory */
-  SDM_VARIANT_STREAMING = 2  /* the state stays in global memory; rows are gathered
+  SDM_VARIANT_STREAMING = 2, /* the state stays in global memory; rows are gathered
                                 ahead of use and scattered back */
+  SDM_VARIANT_PIPELINED = 3  /* as streaming, for few (b,h) sequences: each column tile's
+                                slots are split over two CTAs (more SMs moving rows),
+                                and each CTA's warps split writes, reads and gathers */
 } sdm_variant_t;
 
 /* One layer call.
@@ -96,7 +100,12 @@ typedef enum sdm_variant {
  *   in_dtype    dtype of k', q', v, alpha, beta, g
  *   state_dtype dtype of M0, M (the recurrence computes in fp32 and rounds on store)
  *   rms_eps   epsilon of the optional RMS-norm epilogue
- *   variant   an sdm_variant_t value */
+ *   variant   an sdm_variant_t value
+ *   tile      0: the library picks the kernel's tile; k in [1, 64]: use the k-th
+ *             entry of the chosen kernel's tile table among those that fit this
+ *             shape (sdm_scan_describe names it; SDM_ERR_UNSUPPORTED if there is
+ *             no k-th). For measurements; results do not depend on it. In the
+ *             backward with shared-memory tiles, 1 selects one warp per tile. */
 typedef struct sdm_shape {
   int32_t B, T, H;
   int32_t sqrt_n;
@@ -106,6 +115,7 @@ typedef struct sdm_shape {
   int32_t state_dtype;
   float rms_eps;
   int32_t variant;
+  int32_t tile;
 } sdm_shape_t;
 
 /* ABI version of the loaded library (SDM_ABI_VERSION). */
@@ -157,13 +167,15 @@ SDM_API sdm_status_t sdm_pkm_topk(const void* scores, int32_t in_dtype, int32_t 
 SDM_API size_t sdm_scan_workspace_bytes(const sdm_shape_t* shape);
 
 /* The recurrence kernel sdm_scan / sdm_layer_forward would run for this shape
- * on the current device: SDM_VARIANT_RESIDENT or SDM_VARIANT_STREAMING, or -1
- * if the shape is invalid or unsupported (sdm_last_error() says why). */
+ * on the current device: SDM_VARIANT_RESIDENT, SDM_VARIANT_STREAMING or
+ * SDM_VARIANT_PIPELINED, or -1 if the shape is invalid or unsupported
+ * (sdm_last_error() says why). */
 SDM_API int32_t sdm_scan_variant(const sdm_shape_t* shape);
 
 /* The launch configuration of that kernel as text, e.g.
- * "resident CW=8 NWARP=1 L=4 EB=4 smem=..." or
- * "streaming C=64 P=3 L=8 NW=16 smem=...", NUL-terminated into out (caller
+ * "resident CW=8 NWARP=1 L=4 EB=4 smem=...",
+ * "streaming C=64 P=3 L=8 NW=16 smem=..." or
+ * "pipelined C=64 P=6 L=16 NWW=4 NWR=2 parts=2 smem=...", NUL-terminated into out (caller
  * owned, out_len bytes, truncated to fit). Returns SDM_OK, or an error for an
  * invalid or unsupported shape (out left empty). For profiles and logs. */
 SDM_API sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_len);
@@ -215,6 +227,22 @@ SDM_API sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* 
  *   and this afterwards. */
 SDM_API sdm_status_t sdm_rmsnorm_gate(float* y, const void* g, int32_t in_dtype, int64_t n_rows, int32_t d_v,
                               float eps, void* stream);
+
+/* Sum of squares of each of n_rows rows of d_v fp32 values, in a fixed order:
+ * ss[r] = sum_c y[r, c]^2. When the d_v columns of a layer call are split
+ * across devices (each device holding a column slice of every row), the sum of
+ * the devices' ss is the full rows' sum that the RMS-norm epilogue needs
+ * ([explainer] 3.1 step 3); one all-reduce of ss per call combines them.
+ *   y [n_rows, d_v] fp32;  ss [n_rows] fp32 out (caller owned). */
+SDM_API sdm_status_t sdm_row_sumsq(const float* y, int64_t n_rows, int32_t d_v, float* ss, void* stream);
+
+/* The RMS-norm x gate epilogue on a column slice: for n_rows rows of a layer
+ * output with d_total columns of which this slice holds d_v,
+ * y <- g * y / sqrt(ss / d_total + eps), with ss the full rows' sums of
+ * squares (e.g. sdm_row_sumsq summed over the devices).
+ *   y [n_rows, d_v] fp32 (in/out); g [n_rows, d_v] in in_dtype; ss [n_rows] fp32. */
+SDM_API sdm_status_t sdm_rmsnorm_gate_rows(float* y, const void* g, int32_t in_dtype, const float* ss, int64_t n_rows,
+                                           int32_t d_v, int32_t d_total, float eps, void* stream);
 
 /* Backward of the epilogue for dout = dL/dout, with x = y_pre (the row
  * before it), r = sqrt(mean(x^2) + eps):

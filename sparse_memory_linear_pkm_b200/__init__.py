@@ -51,17 +51,17 @@ def _stream(device: torch.device):
 
 
 def make_shape(B, T, H, sqrt_n, W, R, d_v, in_dtype=torch.bfloat16, state_dtype=torch.float32,
-               rms_eps: float = 1e-6, variant: str = "auto") -> native.Shape:
+               rms_eps: float = 1e-6, variant: str = "auto", tile: int = 0) -> native.Shape:
     return native.Shape(B, T, H, sqrt_n, W, R, d_v, _DTYPE[in_dtype], _DTYPE[state_dtype], rms_eps,
-                        native.VARIANTS[variant])
+                        native.VARIANTS[variant], tile)
 
 
 def scan_variant(shape: native.Shape) -> str:
-    """'resident' or 'streaming': the recurrence kernel this shape runs on the current device."""
+    """'resident', 'streaming' or 'pipelined': the recurrence kernel this shape runs on the current device."""
     v = int(native.load().sdm_scan_variant(ctypes.byref(shape)))
     if v < 0:
         native.check(1)
-    return {1: "resident", 2: "streaming"}[v]
+    return {1: "resident", 2: "streaming", 3: "pipelined"}[v]
 
 
 def scan_describe(shape: native.Shape) -> str:
@@ -99,7 +99,7 @@ def pkm_topk(scores: torch.Tensor, K: int):
 
 
 def scan(idx_w, w_w, idx_r, w_r, v, alpha, beta, M, g=None, eps: float = 1e-6, variant: str = "auto",
-         y: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+         y: torch.Tensor | None = None, workspace: torch.Tensor | None = None, tile: int = 0) -> torch.Tensor:
     """The write/read recurrence over a given selection. M [B,H,N,d_v] is
     updated in place (M_0 -> M_T); returns y [B,T,H,d_v] fp32."""
     B, T, H, W = idx_w.shape
@@ -107,7 +107,8 @@ def scan(idx_w, w_w, idx_r, w_r, v, alpha, beta, M, g=None, eps: float = 1e-6, v
     d_v = v.shape[-1]
     N = M.shape[2]
     sqrt_n = int(round(N ** 0.5))
-    shape = native.Shape(B, T, H, sqrt_n, W, R, d_v, _code(v, "v"), _code(M, "M"), eps, native.VARIANTS[variant])
+    shape = native.Shape(B, T, H, sqrt_n, W, R, d_v, _code(v, "v"), _code(M, "M"), eps, native.VARIANTS[variant],
+                         tile)
     lib = native.load()
     if y is None:
         y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=v.device)
@@ -175,6 +176,24 @@ def rmsnorm_gate(y: torch.Tensor, g: torch.Tensor, eps: float = 1e-6) -> torch.T
     d_v = y.shape[-1]
     native.check(native.load().sdm_rmsnorm_gate(_ptr(y), _ptr(g), _code(g, "g"), y.numel() // d_v, d_v,
                                                 float(eps), _stream(y.device)))
+    return y
+
+
+def row_sumsq(y: torch.Tensor) -> torch.Tensor:
+    """Sum of squares over the last axis of y [..., d] fp32 (fixed order); shape y.shape[:-1]."""
+    d = y.shape[-1]
+    ss = torch.empty(y.shape[:-1], dtype=torch.float32, device=y.device)
+    native.check(native.load().sdm_row_sumsq(_ptr(y), y.numel() // d, d, _ptr(ss), _stream(y.device)))
+    return ss
+
+
+def rmsnorm_gate_rows(y: torch.Tensor, g: torch.Tensor, ss: torch.Tensor, d_total: int,
+                      eps: float = 1e-6) -> torch.Tensor:
+    """The epilogue in place on a column slice y [..., d] of rows of d_total
+    values, given the full rows' sums of squares ss [...]; returns y."""
+    d = y.shape[-1]
+    native.check(native.load().sdm_rmsnorm_gate_rows(_ptr(y), _ptr(g), _code(g, "g"), _ptr(ss), y.numel() // d, d,
+                                                     int(d_total), float(eps), _stream(y.device)))
     return y
 
 
@@ -261,13 +280,13 @@ def slot_counts(idx: torch.Tensor, N: int, counts: torch.Tensor | None = None) -
 
 
 def layer_step(kp, qp, v, alpha, beta, M, W: int, R: int, g=None, eps: float = 1e-6, variant: str = "auto",
-               y: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+               y: torch.Tensor | None = None, workspace: torch.Tensor | None = None, tile: int = 0) -> torch.Tensor:
     """Selection and recurrence over T tokens continuing from the state in M
     [B,H,N,d_v], which is updated in place (decode: T = 1 per call). Returns y."""
     B, T, H, two_n = kp.shape
     d_v = v.shape[-1]
     shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M, "M"), eps,
-                         native.VARIANTS[variant])
+                         native.VARIANTS[variant], tile)
     lib = native.load()
     if y is None:
         y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=kp.device)
@@ -280,7 +299,7 @@ def layer_step(kp, qp, v, alpha, beta, M, W: int, R: int, g=None, eps: float = 1
 
 def layer_forward(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float = 1e-6,
                   variant: str = "auto", y: torch.Tensor | None = None, M_out: torch.Tensor | None = None,
-                  workspace: torch.Tensor | None = None, events=None):
+                  workspace: torch.Tensor | None = None, events=None, tile: int = 0):
     """Selection (top-W of k', top-R of q'), M_out <- M0 per batch row, the
     recurrence and the optional RMS-norm x g epilogue. Returns (y, M_out).
 
@@ -289,7 +308,7 @@ def layer_forward(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float
     B, T, H, two_n = kp.shape
     d_v = v.shape[-1]
     shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M0, "M0"), eps,
-                         native.VARIANTS[variant])
+                         native.VARIANTS[variant], tile)
     lib = native.load()
     if y is None:
         y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=kp.device)

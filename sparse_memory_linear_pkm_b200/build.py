@@ -27,7 +27,7 @@ def nvcc_path() -> str:
 
 
 def _sources():
-    return sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh")) + [INCLUDE / "sdm.h"]
+    return sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh")) + sorted(CSRC.glob("*.h")) + [INCLUDE / "sdm.h"]
 
 
 def up_to_date(out: Path = LIBRARY) -> bool:
@@ -38,15 +38,42 @@ def up_to_date(out: Path = LIBRARY) -> bool:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False, out: Path = LIBRARY) -> Path:
+    """Compiles every translation unit (csrc/*.cu) to an object in parallel,
+    then links them into the shared library."""
     if not force and up_to_date(out):
         return out
-    tmp = out.with_name(out.name + f".tmp{os.getpid()}")
-    cmd = [nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-shared",
-           "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden", "-I", str(INCLUDE), "-I", str(CSRC),
-           str(CSRC / "sdm_api.cu"), "-o", str(tmp)]
+    from concurrent.futures import ThreadPoolExecutor
+
+    nvcc = nvcc_path()
+    objdir = PKG / "_build"
+    objdir.mkdir(exist_ok=True)
+    common = [*ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
+              "-I", str(INCLUDE), "-I", str(CSRC)]
     if ptxas_verbose:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    subprocess.run(cmd, check=True)
+        common = ["-Xptxas", "-v", *common]
+    units = sorted(CSRC.glob("*.cu"))
+    objs = [objdir / (u.stem + f".{os.getpid()}.o") for u in units]
+
+    def compile_one(pair):
+        src, obj = pair
+        return subprocess.run([nvcc, *common, "-c", str(src), "-o", str(obj)], capture_output=True, text=True)
+
+    with ThreadPoolExecutor(max_workers=max(1, min(len(units), os.cpu_count() or 1))) as pool:
+        results = list(pool.map(compile_one, zip(units, objs)))
+    failed = False
+    for src, res in zip(units, results):
+        if res.stdout or res.stderr:
+            print(res.stdout + res.stderr, end="")
+        if res.returncode != 0:
+            failed = True
+            print(f"compiling {src.name} failed")
+    if failed:
+        raise subprocess.CalledProcessError(1, "nvcc")
+    tmp = out.with_name(out.name + f".tmp{os.getpid()}")
+    subprocess.run([nvcc, *ARCH_FLAGS, "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden", *map(str, objs),
+                    "-o", str(tmp)], check=True)
+    for obj in objs:
+        obj.unlink()
     os.replace(tmp, out)
     return out
 

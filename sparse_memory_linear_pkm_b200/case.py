@@ -1,11 +1,12 @@
 """Runs the layer (selection, recurrence, optional epilogue) on one seeded
 synthetic workload, a few times, on cuda:0 — the unit a profiler captures.
 
-    python -m sparse_memory_linear_pkm_b200.case d2048_h16_n1024_dv128 B=2 [T=... H=...] [--repeat 2]
-        [--variant auto|resident|streaming] [--epilogue] [--backward]
+    python -m sparse_memory_linear_pkm_b200.case d2048_h16_n1024_dv128 B=2 [T=... H=... sqrt_n=...]
+        [--repeat 2] [--variant auto|resident|streaming|pipelined] [--tile K] [--epilogue] [--backward]
 
 Size overrides (B, T, H) shrink a named workload while keeping its slot
-count, row width, entry counts and dtypes.
+count, row width, entry counts and dtypes; sqrt_n=... also changes the slot
+count (a smaller state with the same launch grid).
 """
 
 from __future__ import annotations
@@ -22,7 +23,8 @@ def main(argv=None) -> None:
     ap.add_argument("workload", choices=sorted(synth.WORKLOADS))
     ap.add_argument("sizes", nargs="*", help="overrides such as B=2 T=1024 H=4")
     ap.add_argument("--repeat", type=int, default=2)
-    ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "resident", "streaming", "pipelined"])
+    ap.add_argument("--tile", type=int, default=0)
     ap.add_argument("--epilogue", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="run the backward (sdm_scan_backward on the layer's selection, random dy) instead")
@@ -31,8 +33,8 @@ def main(argv=None) -> None:
     kw = {}
     for item in args.sizes:
         key, val = item.split("=")
-        if key not in ("B", "T", "H"):
-            raise SystemExit(f"unknown size override {key!r} (B, T or H)")
+        if key not in ("B", "T", "H", "sqrt_n"):
+            raise SystemExit(f"unknown size override {key!r} (B, T, H or sqrt_n)")
         kw[key] = int(val)
     shape = synth.WORKLOADS[args.workload].replace(**kw)
     inp = synth.make_inputs(shape, seed=args.seed, device="cuda", with_gate=args.epilogue)
@@ -51,10 +53,10 @@ def main(argv=None) -> None:
     M = torch.empty((shape.B,) + tuple(inp["M0"].shape), dtype=inp["M0"].dtype, device="cuda")
     for _ in range(args.repeat):
         layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], inp["M0"], shape.W, shape.R,
-                      g=inp.get("g"), variant=args.variant, y=y, M_out=M)
+                      g=inp.get("g"), variant=args.variant, y=y, M_out=M, tile=args.tile)
     torch.cuda.synchronize()
     sh = make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
-                    shape.torch_state(), variant=args.variant)
+                    shape.torch_state(), variant=args.variant, tile=args.tile)
     print("ok", shape, "recurrence:", scan_describe(sh))
 
 

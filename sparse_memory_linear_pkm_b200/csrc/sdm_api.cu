@@ -1,8 +1,9 @@
 // C ABI of the SDM recurrent core: argument validation, workspace carving and
 // kernel dispatch. See include/sdm.h for the contract of every entry point.
 //
-// This is the single translation unit of libsdm_b200.so; the kernels live in
-// the included headers.
+// The kernels live in the included headers; the launches of the kernels with
+// many template instances sit in translation units of their own (sdm_tu_*.cu),
+// declared in sdm_host.h, so that the library builds in parallel.
 
 #include <cuda_runtime.h>
 
@@ -16,15 +17,9 @@
 #include <string>
 
 #include "sdm.h"
-#include "pkm_topk.cuh"
-#include "pkm_topk_fast.cuh"
-#include "sdm_misc.cuh"
-#include "sdm_records.cuh"
-#include "sdm_scan.cuh"
-#include "sdm_backward.cuh"
-#include "sdm_decode.cuh"
+#include "sdm_host.h"
 
-namespace {
+namespace sdm_host {
 
 using sdm::bf16;
 
@@ -43,14 +38,6 @@ sdm_status_t ok() {
   g_last_error.clear();
   return SDM_OK;
 }
-
-struct DeviceInfo {
-  int sms = 0;
-  int max_smem_optin = 0;
-  int smem_per_sm = 0;
-  unsigned* err = nullptr;
-  bool ready = false;
-};
 
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
@@ -137,8 +124,9 @@ sdm_status_t check_shape(const sdm_shape_t* s) {
   if (s->state_dtype == SDM_FP8_B16 && s->d_v % 16 != 0)
     return fail(SDM_ERR_INVALID_ARGUMENT, "the fp8 state needs d_v a multiple of 16");
   if (!(s->rms_eps >= 0.0f) || s->rms_eps > 1e30f) return fail(SDM_ERR_INVALID_ARGUMENT, "rms_eps must be finite and >= 0");
-  if (s->variant < SDM_VARIANT_AUTO || s->variant > SDM_VARIANT_STREAMING)
+  if (s->variant < SDM_VARIANT_AUTO || s->variant > SDM_VARIANT_PIPELINED)
     return fail(SDM_ERR_INVALID_ARGUMENT, "variant must be an sdm_variant_t value");
+  if (s->tile < 0 || s->tile > 64) return fail(SDM_ERR_INVALID_ARGUMENT, "tile must be in [0, 64] (0: automatic)");
   if (static_cast<int64_t>(s->B) * s->H > 65535) return fail(SDM_ERR_UNSUPPORTED, "B*H above 65535");
   return SDM_OK;
 }
@@ -164,58 +152,6 @@ sdm_status_t need_gate(const void* p, const char* name, bool nonempty, int32_t d
 
 // ------------------------------------------------------------- selection --
 
-sdm::TopkLayout topk_layout(int n, int K) {
-  sdm::TopkLayout L{};
-  L.n = n;
-  L.K = K;
-  L.Kh = std::min(K, n);
-  int C = 0;
-  for (int ra = 0; ra < L.Kh; ++ra) C += std::min(L.Kh, K / (ra + 1));
-  L.C = C;
-  auto a16 = [](uint32_t x) { return (x + 15u) & ~15u; };
-  L.table_bytes = a16(static_cast<uint32_t>(C) * 4u);
-  uint32_t off = 0;
-  auto take = [&](uint32_t bytes) {
-    const uint32_t o = off;
-    off += a16(bytes);
-    return o;
-  };
-  L.vals = take(2u * n * 4u);
-  L.hist = take(256u * 4u);
-  L.hkey = take(static_cast<uint32_t>(L.Kh) * 8u);
-  L.hval = take(2u * L.Kh * 4u);
-  L.hidx = take(2u * L.Kh * 4u);
-  L.c_hi = take(C * 4u);
-  L.c_lo = take(C * 4u);
-  L.c_slot = take(C * 4u);
-  L.tie = take(C * 2u);
-  L.f_hi = take(K * 4u);
-  L.f_lo = take(K * 4u);
-  L.f_slot = take(K * 4u);
-  L.warp_bytes = off;
-  return L;
-}
-
-template <typename Tin, int E, int EH, int EPL, int CP>
-sdm_status_t launch_topk_fast_inst(const DeviceInfo& dev, const Tin* scores, int64_t units,
-                                   const sdm::FastTopkLayout& L, int32_t* idx, float* w, cudaStream_t st) {
-  auto kern = sdm::k_pkm_topk_fast<Tin, E, EH, EPL, CP>;
-  const size_t smem = L.table_bytes + static_cast<size_t>(sdm::kFastTopkWarps) * L.warp_bytes;
-  set_smem(reinterpret_cast<const void*>(kern), smem);
-  int per_sm = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sdm::kFastTopkWarps * 32, smem);
-  const int64_t blocks_needed = (units + sdm::kFastTopkWarps - 1) / sdm::kFastTopkWarps;
-  const int grid =
-      static_cast<int>(std::min<int64_t>(blocks_needed, static_cast<int64_t>(dev.sms) * std::max(1, per_sm) * 4));
-  kern<<<grid, sdm::kFastTopkWarps * 32, smem, st>>>(scores, units, L, idx, w);
-  return launch_status("pkm_topk launch");
-}
-
-// Layout and template parameters of the register-path selection (K <= 64).
-struct FastTopkPlan {
-  sdm::FastTopkLayout L{};
-  int E = 1, EH = 1, epl = 1, CP = 4;
-};
 sdm_status_t fast_topk_plan(int n, int K, FastTopkPlan* out) {
   FastTopkPlan P;
   sdm::FastTopkLayout& L = P.L;
@@ -250,54 +186,6 @@ sdm_status_t fast_topk_plan(int n, int K, FastTopkPlan* out) {
   return SDM_OK;
 }
 
-// Register path for K <= 64.
-template <typename Tin>
-sdm_status_t launch_topk_fast(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K,
-                              int32_t* idx, float* w, cudaStream_t st) {
-  FastTopkPlan P;
-  sdm_status_t r;
-  if ((r = fast_topk_plan(n, K, &P)) != SDM_OK) return r;
-  const sdm::FastTopkLayout& L = P.L;
-  const int E = P.E, EH = P.EH, CP = P.CP;
-  const Tin* x = static_cast<const Tin*>(scores);
-  const int epl = P.epl;
-#define SDM_FAST_TOPK(E_, EH_, EPL_, CP_)                      \
-  if (E == E_ && EH == EH_ && epl == EPL_ && CP == CP_) \
-    return launch_topk_fast_inst<Tin, E_, EH_, EPL_, CP_>(dev, x, units, L, idx, w, st);
-  SDM_FAST_TOPK(1, 1, 1, 4) SDM_FAST_TOPK(1, 1, 2, 4) SDM_FAST_TOPK(1, 1, 4, 4) SDM_FAST_TOPK(1, 1, 8, 4)
-  SDM_FAST_TOPK(1, 1, 16, 4) SDM_FAST_TOPK(1, 1, 32, 4)
-  SDM_FAST_TOPK(2, 1, 1, 7)
-  SDM_FAST_TOPK(2, 2, 1, 9) SDM_FAST_TOPK(2, 2, 4, 9) SDM_FAST_TOPK(2, 2, 8, 9)
-  SDM_FAST_TOPK(2, 2, 16, 9) SDM_FAST_TOPK(2, 2, 32, 9)
-#undef SDM_FAST_TOPK
-  return fail(SDM_ERR_UNSUPPORTED, "no selection kernel for this sqrt_n and K");
-}
-
-template <typename Tin>
-sdm_status_t launch_topk(const DeviceInfo& dev, const void* scores, int64_t units, int n, int K, int32_t* idx,
-                         float* w, cudaStream_t st) {
-  if (units == 0) return SDM_OK;
-  if (K <= sdm::kFastTopkMaxK) return launch_topk_fast<Tin>(dev, scores, units, n, K, idx, w, st);
-  const sdm::TopkLayout L = topk_layout(n, K);
-  int warps = 4;
-  while (warps > 1 && L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes > static_cast<size_t>(dev.max_smem_optin))
-    --warps;
-  const size_t smem = L.table_bytes + static_cast<size_t>(warps) * L.warp_bytes;
-  if (smem > static_cast<size_t>(dev.max_smem_optin)) return fail(SDM_ERR_UNSUPPORTED, "selection scratch exceeds shared memory");
-  auto kern = sdm::k_pkm_topk_general<Tin>;
-  set_smem(reinterpret_cast<const void*>(kern), smem);
-  const int64_t blocks_needed = (units + warps - 1) / warps;
-  const int grid = static_cast<int>(std::min<int64_t>(blocks_needed, static_cast<int64_t>(dev.sms) * 16));
-  kern<<<grid, warps * 32, smem, st>>>(static_cast<const Tin*>(scores), units, L, idx, w);
-  return launch_status("pkm_topk launch");
-}
-
-sdm_status_t topk_impl(const DeviceInfo& dev, const void* scores, int32_t in_dtype, int64_t units, int n, int K,
-                       int32_t* idx, float* w, cudaStream_t st) {
-  return in_dtype == SDM_BF16 ? launch_topk<bf16>(dev, scores, units, n, K, idx, w, st)
-                              : launch_topk<float>(dev, scores, units, n, K, idx, w, st);
-}
-
 // ------------------------------------------------------------ recurrence --
 
 // Record layout; the hazard plan is only stored for the streaming kernel.
@@ -316,10 +204,6 @@ sdm::RecLayout rec_layout(int W, int R, bool plan = true) {
   return rl;
 }
 
-size_t records_bytes(const sdm_shape_t& s) {
-  return align256(static_cast<size_t>(s.B) * s.H * s.T * rec_layout(s.W, s.R).words * 4u);
-}
-
 // Instantiated streaming tiles: state bytes, columns per CTA, prefetch
 // distance, staging chunk, warps.
 struct StreamCfg {
@@ -333,6 +217,17 @@ constexpr StreamCfg kStreamCfgs[] = {
     {2, 16, 8, 16, 16}, {2, 16, 4, 8, 8},
 };
 
+// Instantiated pipelined tiles: state bytes, columns per CTA (128-byte row
+// segments), prefetch distance, staging chunk, write warps, read warps.
+struct PipeCfg {
+  int state_bytes;
+  int C, P, L, NWW, NWR;
+};
+constexpr PipeCfg kPipeCfgs[] = {
+    {2, 64, 6, 16, 4, 4}, {2, 64, 7, 16, 4, 4}, {2, 64, 6, 16, 8, 8}, {2, 64, 5, 16, 4, 4},
+    {4, 32, 6, 16, 4, 4}, {4, 32, 4, 16, 4, 4},
+};
+
 // Instantiated resident tiles: columns per warp, warps per CTA, staging
 // chunk, entries per lane block.
 struct ResidentCfg {
@@ -340,15 +235,6 @@ struct ResidentCfg {
 };
 constexpr ResidentCfg kResidentCfgs[] = {
     {8, 1, 4, 4}, {8, 2, 4, 4}, {4, 2, 4, 2}, {16, 1, 4, 4}, {4, 4, 4, 2}, {8, 2, 8, 4}, {4, 4, 8, 2}, {8, 4, 8, 4},
-};
-
-struct ScanChoice {
-  bool resident = false;
-  int C = 16;  // columns per CTA
-  int P = 4;
-  int L = 16;
-  int CW = 8, NWARP = 2, EB = 4;  // resident: columns per warp, warps per CTA, entry block
-  size_t smem = 0;
 };
 
 size_t resident_smem(const sdm_shape_t& s, const ResidentCfg& k) {
@@ -360,13 +246,29 @@ size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L, int NW) {
   return sdm::streaming_stage_bytes(P, s.W + s.R, s.W, C, static_cast<int>(in_size(s.state_dtype))) +
          2ull * L * rl.words * 4 + 2ull * L * C * in_size(s.in_dtype) + 2ull * NW * C * 4 + 2 * 8;
 }
+size_t pipelined_smem(const sdm_shape_t& s, const PipeCfg& k) {
+  const sdm::PipeLayout pl = sdm::pipe_layout(s.W, s.R);
+  return sdm::pipe_smem_bytes(k.P, k.L, pl.Wp, pl.Rp, pl.words, k.C, static_cast<int>(in_size(s.state_dtype)),
+                              static_cast<int>(in_size(s.in_dtype)));
+}
 
+// Whether the automatic variant takes the pipelined kernel for few column
+// tiles (off while the streaming kernel measures faster there).
+constexpr bool kPipelinedAuto = false;
+
+// Picks the recurrence kernel and its tile. s.tile >= 1 forces entry s.tile
+// (1-based) of the chosen kernel's table among the entries that fit the
+// shape (for measurements); 0 takes the first that fits.
 sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
   if (s.state_dtype == SDM_FP8_B16)
     return fail(SDM_ERR_UNSUPPORTED,
                 "the fp8 state (SDM_FP8_B16) runs only in the single-launch decode step: sdm_layer_step with "
                 "T = 1, W = R <= 64 and the automatic variant");
   const size_t lim = static_cast<size_t>(dev.max_smem_optin);
+  auto pick = [&](size_t n_fit) -> int {  // index into the fitting entries, or -1
+    if (s.tile == 0) return n_fit > 0 ? 0 : -1;
+    return static_cast<size_t>(s.tile) <= n_fit ? s.tile - 1 : -1;
+  };
   ScanChoice c;
   // A resident tile reads and writes all N rows once; below one touched row
   // per slot (T * (W + R) < N, e.g. a decode step) streaming only the
@@ -376,21 +278,13 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
     // Resident tiles in order of preference (measured on B200 at N = 1024,
     // d_v = 128: 8-column warp tiles, one warp per CTA, so up to five CTAs
     // share an SM); the first that divides d_v and fits is taken.
-    // "CW,NWARP,L" in SDM_RESIDENT_CFG forces one (tuning).
     std::vector<ResidentCfg> order;
     for (const ResidentCfg& k : kResidentCfgs)
       if (s.d_v % (k.CW * k.NWARP) == 0 && resident_smem(s, k) <= lim) order.push_back(k);
-    if (const char* env = std::getenv("SDM_RESIDENT_CFG")) {
-      int CW = 0, NW = 0, L = 0;
-      if (std::sscanf(env, "%d,%d,%d", &CW, &NW, &L) == 3) {
-        std::vector<ResidentCfg> forced;
-        for (const ResidentCfg& k : order)
-          if (k.CW == CW && k.NWARP == NW && k.L == L) forced.push_back(k);
-        if (!forced.empty()) order = forced;
-      }
-    }
-    if (!order.empty()) {
-      const ResidentCfg& k = order.front();
+    const int i = pick(order.size());
+    if (i >= 0) {
+      const ResidentCfg& k = order[i];
+      c.kind = SDM_VARIANT_RESIDENT;
       c.resident = true;
       c.CW = k.CW;
       c.NWARP = k.NWARP;
@@ -398,25 +292,50 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
       c.C = k.CW * k.NWARP;
       c.L = k.L;
       c.smem = resident_smem(s, k);
-    }
-    if (c.resident) {
       *out = c;
       return SDM_OK;
     }
     if (s.variant == SDM_VARIANT_RESIDENT)
-      return fail(SDM_ERR_UNSUPPORTED, "the state tile does not fit in shared memory (resident variant)");
+      return fail(SDM_ERR_UNSUPPORTED, s.tile == 0 ? "the state tile does not fit in shared memory (resident variant)"
+                                                   : "no such resident tile for this shape");
   }
-  c.resident = false;
+  const int s_state = static_cast<int>(in_size(s.state_dtype));
+  const int64_t bh = static_cast<int64_t>(s.B) * s.H;
+  // The pipelined kernel when 128-byte column tiles alone would leave SMs
+  // idle: one SM moves about one random 128-byte row per 3 ns, so a grid
+  // smaller than the SM count cannot approach the HBM bandwidth; splitting
+  // each tile's slots over two CTAs doubles the SMs at work.
+  const int c128 = 128 / s_state;
+  const bool few_tiles = s.d_v % c128 == 0 && bh * (s.d_v / c128) < dev.sms;
+  if (s.variant == SDM_VARIANT_PIPELINED || (s.variant == SDM_VARIANT_AUTO && kPipelinedAuto && few_tiles)) {
+    std::vector<PipeCfg> order;
+    for (const PipeCfg& k : kPipeCfgs)
+      if (k.state_bytes == s_state && s.d_v % k.C == 0 && pipelined_smem(s, k) <= lim) order.push_back(k);
+    const int i = pick(order.size());
+    if (i >= 0) {
+      const PipeCfg& k = order[i];
+      c.kind = SDM_VARIANT_PIPELINED;
+      c.C = k.C;
+      c.P = k.P;
+      c.L = k.L;
+      c.NWW = k.NWW;
+      c.NWR = k.NWR;
+      c.parts = bh * (s.d_v / k.C) * 2 <= dev.sms ? 2 : 1;
+      c.smem = pipelined_smem(s, k);
+      *out = c;
+      return SDM_OK;
+    }
+    if (s.variant == SDM_VARIANT_PIPELINED)
+      return fail(SDM_ERR_UNSUPPORTED, s.tile == 0 ? "W + R too large for the pipelined stage rings"
+                                                   : "no such pipelined tile for this shape");
+  }
   // Streaming tiles, best first. Random row segments of >= 256 B run HBM near
   // its copy bandwidth, 128 B at ~75%, 64 B at ~40% (measured gathers on
   // B200), so wide segments win while the grid still fills the SMs.
-  const int s_state = static_cast<int>(in_size(s.state_dtype));
-  const int64_t bh = static_cast<int64_t>(s.B) * s.H;
   std::vector<StreamCfg> order;
-  for (const StreamCfg& k : kStreamCfgs) {
-    if (k.state_bytes != s_state || s.d_v % k.C != 0) continue;
-    order.push_back(k);
-  }
+  for (const StreamCfg& k : kStreamCfgs)
+    if (k.state_bytes == s_state && s.d_v % k.C == 0 && k.C <= 32 * k.NW && streaming_smem(s, k.C, k.P, k.L, k.NW) <= lim)
+      order.push_back(k);
   auto ctas = [&](const StreamCfg& k) { return bh * (s.d_v / k.C); };
   std::stable_sort(order.begin(), order.end(), [&](const StreamCfg& x, const StreamCfg& y) {
     const bool fx = ctas(x) >= dev.sms / 2, fy = ctas(y) >= dev.sms / 2;  // fills at least half the SMs
@@ -425,29 +344,44 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
     if (rx != ry) return rx > ry;  // wider row segments first
     return x.P > y.P;
   });
-  if (const char* env = std::getenv("SDM_STREAM_CFG")) {  // tuning override "C,P,L,NW"
-    int C = 0, P = 0, L = 0, NW = 0;
-    if (std::sscanf(env, "%d,%d,%d,%d", &C, &P, &L, &NW) == 4) {
-      std::vector<StreamCfg> forced;
-      for (const StreamCfg& k : order)
-        if (k.C == C && k.P == P && k.L == L && k.NW == NW) forced.push_back(k);
-      if (!forced.empty()) order = forced;
-    }
+  const int i = pick(order.size());
+  if (i < 0)
+    return fail(SDM_ERR_UNSUPPORTED, s.tile == 0 ? "W + R too large for the streaming stage ring"
+                                                 : "no such streaming tile for this shape");
+  const StreamCfg& k = order[i];
+  c.kind = SDM_VARIANT_STREAMING;
+  c.C = k.C;
+  c.P = k.P;
+  c.L = k.L;
+  c.NWARP = k.NW;
+  c.smem = streaming_smem(s, k.C, k.P, k.L, k.NW);
+  *out = c;
+  return SDM_OK;
+}
+
+// Workspace of the per-token records for the chosen kernel.
+size_t records_bytes(const sdm_shape_t& s, const ScanChoice& c) {
+  const int64_t n = static_cast<int64_t>(s.B) * s.H * s.T;
+  if (c.kind == SDM_VARIANT_PIPELINED)
+    return align256(static_cast<size_t>(n) * c.parts * sdm::pipe_layout(s.W, s.R).words * 4u);
+  return align256(static_cast<size_t>(n) * rec_layout(s.W, s.R).words * 4u);
+}
+// The same before a kernel is chosen (workspace queries): the chosen
+// kernel's need on the current device, or the largest of all kernels' when
+// no device can be queried.
+size_t records_bytes(const sdm_shape_t& s) {
+  const std::string saved = g_last_error;
+  DeviceInfo* dev;
+  ScanChoice c;
+  if (device_info(&dev) == SDM_OK && choose_scan(*dev, s, &c) == SDM_OK) {
+    g_last_error = saved;
+    return records_bytes(s, c);
   }
-  for (const StreamCfg& k : order) {
-    if (k.C > 32 * k.NW) continue;
-    const size_t need = streaming_smem(s, k.C, k.P, k.L, k.NW);
-    if (need <= lim) {
-      c.C = k.C;
-      c.P = k.P;
-      c.L = k.L;
-      c.NWARP = k.NW;
-      c.smem = need;
-      *out = c;
-      return SDM_OK;
-    }
-  }
-  return fail(SDM_ERR_UNSUPPORTED, "W + R too large for the streaming stage ring");
+  g_last_error = saved;
+  ScanChoice pipe;
+  pipe.kind = SDM_VARIANT_PIPELINED;
+  pipe.parts = 2;
+  return std::max(records_bytes(s, ScanChoice()), records_bytes(s, pipe));
 }
 
 template <typename Tin>
@@ -467,40 +401,6 @@ sdm_status_t launch_records(const sdm_shape_t& s, const int32_t* idx_w, const fl
   kern<<<grid, 256, smem, st>>>(idx_w, w_w, idx_r, w_r, static_cast<const Tin*>(alpha), static_cast<const Tin*>(beta),
                                 s.T, s.H, static_cast<int>(slots_of(s.sqrt_n)), s.W, s.R, P, log2_cells, rl, rec, err);
   return launch_status("record build launch");
-}
-
-template <typename Tin, typename Tst>
-sdm_status_t launch_scan_typed(const ScanChoice& c, const sdm::ScanArgs& a, cudaStream_t st) {
-  const dim3 grid(a.B * a.H, a.d_v / c.C);
-  void (*kern)(sdm::ScanArgs) = nullptr;
-  if (c.resident) {
-#define SDM_RES(CW_, NW_, L_, EB_) \
-    if (c.CW == CW_ && c.NWARP == NW_ && c.L == L_ && c.EB == EB_) kern = sdm::k_scan_resident<Tin, Tst, CW_, NW_, L_, EB_>;
-    SDM_RES(8, 2, 4, 4) SDM_RES(8, 1, 4, 4) SDM_RES(16, 1, 4, 4) SDM_RES(4, 4, 4, 2) SDM_RES(4, 2, 4, 2)
-    SDM_RES(8, 2, 8, 4) SDM_RES(4, 4, 8, 2) SDM_RES(8, 4, 8, 4)
-#undef SDM_RES
-  } else {
-#define SDM_STREAM(C_, P_, L_, NW_) \
-    if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWARP == NW_) kern = sdm::k_scan_streaming<Tin, Tst, C_, P_, L_, NW_>;
-    if constexpr (sizeof(Tst) == 4) {
-      SDM_STREAM(64, 3, 8, 16) SDM_STREAM(64, 2, 8, 16) SDM_STREAM(32, 4, 8, 16) SDM_STREAM(32, 4, 8, 8)
-      SDM_STREAM(16, 8, 16, 16) SDM_STREAM(16, 4, 8, 8)
-    } else {
-      SDM_STREAM(128, 3, 8, 16) SDM_STREAM(64, 4, 8, 16) SDM_STREAM(64, 6, 8, 16) SDM_STREAM(32, 8, 16, 16)
-      SDM_STREAM(32, 8, 16, 8) SDM_STREAM(16, 8, 16, 16) SDM_STREAM(16, 4, 8, 8)
-    }
-#undef SDM_STREAM
-  }
-  if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no streaming kernel for the chosen tile");
-  set_smem(reinterpret_cast<const void*>(kern), c.smem);
-  kern<<<grid, c.NWARP * 32, c.smem, st>>>(a);
-  return launch_status("scan launch");
-}
-
-sdm_status_t launch_scan(const ScanChoice& c, const sdm_shape_t& s, const sdm::ScanArgs& a, cudaStream_t st) {
-  if (s.in_dtype == SDM_BF16)
-    return s.state_dtype == SDM_BF16 ? launch_scan_typed<bf16, bf16>(c, a, st) : launch_scan_typed<bf16, float>(c, a, st);
-  return s.state_dtype == SDM_BF16 ? launch_scan_typed<float, bf16>(c, a, st) : launch_scan_typed<float, float>(c, a, st);
 }
 
 sdm_status_t launch_state_init(const DeviceInfo& dev, const sdm_shape_t& s, const void* M0, void* M, cudaStream_t st) {
@@ -546,6 +446,31 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
                       uint32_t* rec, cudaStream_t st, const Trace& tr = Trace(), bool init_before_scan = false,
                       const void* M0_for_init = nullptr) {
   sdm_status_t r;
+  if (c.kind == SDM_VARIANT_PIPELINED) {
+    // the parts add their read sums into y, which the record build zeroes first
+    float* y_zero = c.parts > 1 ? y : nullptr;
+    if ((r = launch_pipe_records(s, c, idx_w, w_w, idx_r, w_r, alpha, beta, rec, y_zero, dev, st)) != SDM_OK)
+      return r;
+    tr.mark(2, st);
+    if (init_before_scan && (r = launch_state_init(dev, s, M0_for_init, M, st)) != SDM_OK) return r;
+    tr.mark(3, st);
+    sdm::PipeArgs a{};
+    a.B = s.B; a.T = s.T; a.H = s.H;
+    a.N = static_cast<int>(slots_of(s.sqrt_n));
+    a.d_v = s.d_v; a.W = s.W; a.R = s.R;
+    a.parts = c.parts;
+    a.pl = sdm::pipe_layout(s.W, s.R);
+    a.rec = rec;
+    a.v = v;
+    a.M = M;
+    a.y = y;
+    a.err = dev.err;
+    if ((r = launch_pipe(c, s, a, st)) != SDM_OK) return r;
+    tr.mark(4, st);
+    if (g != nullptr && (r = launch_epilogue(dev, s, y, g, st)) != SDM_OK) return r;
+    tr.mark(5, st);
+    return SDM_OK;
+  }
   const int plan_p = c.resident ? 0 : c.P + 1;  // the streaming plan looks back P tokens
   if ((r = (s.in_dtype == SDM_BF16 ? launch_records<bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, plan_p,
                                                           rec, dev.err, dev, st)
@@ -605,20 +530,7 @@ sdm_status_t noalloc_scratch(void** out) {
 
 // ------------------------------------------------------------- backward --
 
-namespace {
-
-constexpr size_t kBwdSmemLimit = 232448;  // sm_100 opt-in shared memory per block
-constexpr int kBwdChunk = 128;            // tokens per checkpoint chunk
-
-struct BwdChoice {
-  bool global = false;  // state and adjoint tiles in global memory (large N)
-  int U = 1;            // 16-byte units (4 columns) per lane and entry: tile width 4 U
-  int C = kBwdChunk;
-  int ntile = 0;
-  size_t smem = 0;
-  size_t rec_bytes = 0, ckpt_bytes = 0, log_bytes = 0, part_bytes = 0, work_bytes = 0;
-  size_t total() const { return rec_bytes + ckpt_bytes + log_bytes + part_bytes + work_bytes; }
-};
+namespace sdm_host {
 
 sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
   if (s.state_dtype != SDM_F32)
@@ -634,6 +546,7 @@ sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
   c.global = on_chip > kBwdSmemLimit;
   c.U = c.global ? (s.d_v % 32 == 0 ? 8 : 4) : 1;
   c.smem = c.global ? ring_bytes(c.U) : on_chip;
+  c.nwb = s.tile == 1 ? 1 : 2;
   if (c.smem > kBwdSmemLimit) return fail(SDM_ERR_UNSUPPORTED, "backward staging exceeds shared memory (W, R too large)");
   if (c.global) {
     // Chunk length near sqrt(T N / W): checkpoints (T / C states) and the log
@@ -658,55 +571,11 @@ sdm_status_t choose_bwd(const sdm_shape_t& s, BwdChoice* out) {
   return SDM_OK;
 }
 
-template <typename Tin, int U, bool G, int NWB>
-sdm_status_t launch_bwd_inst(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
-  const void* kern = reinterpret_cast<const void*>(sdm::k_scan_backward<Tin, U, G, NWB>);
-  set_smem(kern, c.smem);
-  const int64_t grid = static_cast<int64_t>(a.B) * a.H * c.ntile;
-  if (grid > 0x7FFFFFFFLL) return fail(SDM_ERR_UNSUPPORTED, "too many column tiles for one launch");
-  sdm::k_scan_backward<Tin, U, G, NWB><<<static_cast<unsigned>(grid), NWB * 32, c.smem, st>>>(a);
-  return launch_status("backward launch");
-}
-
-template <typename Tin>
-sdm_status_t launch_bwd_typed(const BwdChoice& c, const sdm::BwdArgs& a, cudaStream_t st) {
-  if (!c.global) {
-    // Two warps share each shared-memory tile (tuning override SDM_BWD_NWB=1: one).
-    const char* env = std::getenv("SDM_BWD_NWB");
-    if (env != nullptr && std::atoi(env) == 1) return launch_bwd_inst<Tin, 1, false, 1>(c, a, st);
-    return launch_bwd_inst<Tin, 1, false, 2>(c, a, st);
-  }
-  return c.U == 8 ? launch_bwd_inst<Tin, 8, true, 1>(c, a, st) : launch_bwd_inst<Tin, 4, true, 1>(c, a, st);
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------- decode --
 
-namespace {
-
-template <typename Tin, typename Tst, int E, int EH, int EPL, int CP>
-sdm_status_t launch_decode_inst(const sdm::DecodeArgs& a, size_t smem, int grid, cudaStream_t st) {
-  auto kern = sdm::k_decode_step<Tin, Tst, E, EH, EPL, CP>;
-  set_smem(reinterpret_cast<const void*>(kern), smem);
-  kern<<<grid, sdm::kDecodeThreads, smem, st>>>(a);
-  return launch_status("decode step launch");
-}
-
-template <typename Tin, typename Tst>
-sdm_status_t launch_decode_typed(const FastTopkPlan& P, const sdm::DecodeArgs& a, size_t smem, int grid,
-                                 cudaStream_t st) {
-#define SDM_DECODE(E_, EH_, EPL_, CP_)                                 \
-  if (P.E == E_ && P.EH == EH_ && P.epl == EPL_ && P.CP == CP_) \
-    return launch_decode_inst<Tin, Tst, E_, EH_, EPL_, CP_>(a, smem, grid, st);
-  SDM_DECODE(1, 1, 1, 4) SDM_DECODE(1, 1, 2, 4) SDM_DECODE(1, 1, 4, 4) SDM_DECODE(1, 1, 8, 4)
-  SDM_DECODE(1, 1, 16, 4) SDM_DECODE(1, 1, 32, 4)
-  SDM_DECODE(2, 1, 1, 7)
-  SDM_DECODE(2, 2, 1, 9) SDM_DECODE(2, 2, 4, 9) SDM_DECODE(2, 2, 8, 9)
-  SDM_DECODE(2, 2, 16, 9) SDM_DECODE(2, 2, 32, 9)
-#undef SDM_DECODE
-  return fail(SDM_ERR_UNSUPPORTED, "no decode kernel for this sqrt_n and K");
-}
+namespace sdm_host {
 
 // The fused single-launch decode step (T = 1, W = R <= 64, automatic
 // variant). Sets *used = false (and returns SDM_OK) when the shape is not one
@@ -742,20 +611,14 @@ sdm_status_t try_decode_step(const DeviceInfo& dev, const sdm_shape_t& s, const 
   const size_t smem = a.part_off + static_cast<size_t>(groups) * s.d_v * 4;
   if (smem > static_cast<size_t>(dev.max_smem_optin)) return SDM_OK;
   const int grid = s.B * s.H;
-  sdm_status_t r;
-  if (s.in_dtype == SDM_BF16)
-    r = s.state_dtype == SDM_FP8_B16 ? launch_decode_typed<sdm::bf16, sdm::Fp8Blk>(P, a, smem, grid, st)
-        : s.state_dtype == SDM_BF16  ? launch_decode_typed<sdm::bf16, sdm::bf16>(P, a, smem, grid, st)
-                                     : launch_decode_typed<sdm::bf16, float>(P, a, smem, grid, st);
-  else
-    r = s.state_dtype == SDM_FP8_B16 ? launch_decode_typed<float, sdm::Fp8Blk>(P, a, smem, grid, st)
-        : s.state_dtype == SDM_BF16  ? launch_decode_typed<float, sdm::bf16>(P, a, smem, grid, st)
-                                     : launch_decode_typed<float, float>(P, a, smem, grid, st);
+  const sdm_status_t r = launch_decode(P, s.in_dtype, s.state_dtype, a, smem, grid, st);
   if (r == SDM_OK) *used = true;
   return r;
 }
 
 }  // namespace
+
+using namespace sdm_host;
 
 extern "C" {
 
@@ -860,7 +723,7 @@ int32_t sdm_scan_variant(const sdm_shape_t* shape) {
   if (check_shape(shape) != SDM_OK || device_info(&dev) != SDM_OK || choose_scan(*dev, *shape, &c) != SDM_OK)
     return -1;
   ok();
-  return c.resident ? SDM_VARIANT_RESIDENT : SDM_VARIANT_STREAMING;
+  return c.kind;
 }
 
 
@@ -923,11 +786,11 @@ sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, c
   if (s.in_dtype == SDM_BF16) {
     if ((r = launch_records<sdm::bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
       return r;
-    r = launch_bwd_typed<sdm::bf16>(c, a, st);
+    r = launch_bwd(c, SDM_BF16, a, st);
   } else {
     if ((r = launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
       return r;
-    r = launch_bwd_typed<float>(c, a, st);
+    r = launch_bwd(c, SDM_F32, a, st);
   }
   if (r != SDM_OK) return r;
   const int64_t n_th = static_cast<int64_t>(s.B) * s.T * s.H;
@@ -955,6 +818,43 @@ sdm_status_t sdm_rmsnorm_gate(float* y, const void* g, int32_t in_dtype, int64_t
   else
     sdm::k_rmsnorm_gate<float><<<grid, 256, 0, st>>>(y, static_cast<const float*>(g), n_rows, d_v, eps);
   if ((r = launch_status("epilogue launch")) != SDM_OK) return r;
+  return ok();
+}
+
+sdm_status_t sdm_row_sumsq(const float* y, int64_t n_rows, int32_t d_v, float* ss, void* stream) {
+  sdm_status_t r;
+  if (n_rows < 0 || d_v < 1) return fail(SDM_ERR_INVALID_ARGUMENT, "n_rows must be >= 0 and d_v >= 1");
+  if (n_rows == 0) return ok();
+  if ((r = need_ptr(y, "y", true)) != SDM_OK || (r = need_gate(ss, "ss", true, SDM_F32)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const int grid = static_cast<int>(std::min<int64_t>((n_rows + 7) / 8, static_cast<int64_t>(dev->sms) * 16));
+  sdm::k_row_sumsq<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(y, n_rows, d_v, ss);
+  if ((r = launch_status("row sum of squares launch")) != SDM_OK) return r;
+  return ok();
+}
+
+sdm_status_t sdm_rmsnorm_gate_rows(float* y, const void* g, int32_t in_dtype, const float* ss, int64_t n_rows,
+                                   int32_t d_v, int32_t d_total, float eps, void* stream) {
+  sdm_status_t r;
+  if (n_rows < 0 || d_v < 1 || d_total < d_v)
+    return fail(SDM_ERR_INVALID_ARGUMENT, "n_rows must be >= 0, d_v >= 1 and d_total >= d_v");
+  if (!(eps >= 0.0f)) return fail(SDM_ERR_INVALID_ARGUMENT, "eps must be >= 0");
+  if ((r = check_dtype(in_dtype, "in_dtype")) != SDM_OK) return r;
+  if (n_rows == 0) return ok();
+  if ((r = need_ptr(y, "y", true)) != SDM_OK || (r = need_gate(g, "g", true, in_dtype)) != SDM_OK ||
+      (r = need_gate(ss, "ss", true, SDM_F32)) != SDM_OK)
+    return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const int grid = static_cast<int>(std::min<int64_t>((n_rows + 7) / 8, static_cast<int64_t>(dev->sms) * 16));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (in_dtype == SDM_BF16)
+    sdm::k_rmsnorm_gate_rows<bf16><<<grid, 256, 0, st>>>(y, static_cast<const bf16*>(g), ss, n_rows, d_v, d_total, eps);
+  else
+    sdm::k_rmsnorm_gate_rows<float><<<grid, 256, 0, st>>>(y, static_cast<const float*>(g), ss, n_rows, d_v, d_total,
+                                                          eps);
+  if ((r = launch_status("column-slice epilogue launch")) != SDM_OK) return r;
   return ok();
 }
 
@@ -1098,8 +998,11 @@ sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_l
   if ((r = check_shape(shape)) != SDM_OK || (r = device_info(&dev)) != SDM_OK ||
       (r = choose_scan(*dev, *shape, &c)) != SDM_OK)
     return r;
-  if (c.resident)
+  if (c.kind == SDM_VARIANT_RESIDENT)
     snprintf(out, out_len, "resident CW=%d NWARP=%d L=%d EB=%d smem=%zu", c.CW, c.NWARP, c.L, c.EB, c.smem);
+  else if (c.kind == SDM_VARIANT_PIPELINED)
+    snprintf(out, out_len, "pipelined C=%d P=%d L=%d NWW=%d NWR=%d parts=%d smem=%zu", c.C, c.P, c.L, c.NWW, c.NWR,
+             c.parts, c.smem);
   else
     snprintf(out, out_len, "streaming C=%d P=%d L=%d NW=%d smem=%zu", c.C, c.P, c.L, c.NWARP, c.smem);
   return ok();

@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(NWB * 32) k_scan_backward(BwdArgs a) {
 
 // Sums the per-tile partials in tile order: dw_w, dw_r [B,T,H,W|R], dalpha,
 // dbeta [B,T,H]. One thread per output value.
-__global__ void __launch_bounds__(256) k_scan_backward_reduce(const float* __restrict__ part, int64_t n_th, int W,
+static __global__ void __launch_bounds__(256) k_scan_backward_reduce(const float* __restrict__ part, int64_t n_th, int W,
                                                               int R, int ntile, float* __restrict__ dw_w,
                                                               float* __restrict__ dw_r, float* __restrict__ dalpha,
                                                               float* __restrict__ dbeta) {
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(256) k_scan_backward_reduce(const float* __res
 // One warp per token-head; each lane owns score entries x = lane, lane + 32, ...
 // of the 2 sqrt_n row and sums its contributions over k in order
 // (deterministic). dscores rows are written whole (zeros where unused).
-__global__ void __launch_bounds__(256) k_pkm_topk_backward(const int32_t* __restrict__ idx,
+static __global__ void __launch_bounds__(256) k_pkm_topk_backward(const int32_t* __restrict__ idx,
                                                            const float* __restrict__ w,
                                                            const float* __restrict__ dw, int64_t n_units,
                                                            int sqrt_n, int K, float* __restrict__ dscores,

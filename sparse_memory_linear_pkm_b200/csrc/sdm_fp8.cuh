@@ -73,7 +73,7 @@ __device__ __forceinline__ int fp8blk_pack16(const float* x, uint4* u) {
 }
 
 // codes[16 b .. 16 b + 15], exps[b] <- the quantised block b of x.
-__global__ void __launch_bounds__(256) k_quantize_fp8blk(const float* __restrict__ x, int64_t n_blocks,
+static __global__ void __launch_bounds__(256) k_quantize_fp8blk(const float* __restrict__ x, int64_t n_blocks,
                                                          uint8_t* __restrict__ codes, int8_t* __restrict__ exps) {
   for (int64_t b = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; b < n_blocks;
        b += static_cast<int64_t>(gridDim.x) * blockDim.x) {

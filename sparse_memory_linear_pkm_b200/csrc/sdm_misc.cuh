@@ -8,7 +8,7 @@ namespace sdm {
 // M[b] <- M0 for every batch row: the learned initial state shared by all rows
 // (SDM explainer, section 3.1, "learned initial state"). Bandwidth-bound
 // 16-byte copies; blockIdx.y is the batch row.
-__global__ void __launch_bounds__(256) k_state_init(const uint4* __restrict__ M0, uint4* __restrict__ M,
+static __global__ void __launch_bounds__(256) k_state_init(const uint4* __restrict__ M0, uint4* __restrict__ M,
                                                     int64_t units_per_row) {
   uint4* dst = M + static_cast<int64_t>(blockIdx.y) * units_per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < units_per_row;
@@ -32,6 +32,40 @@ __global__ void __launch_bounds__(256) k_rmsnorm_gate(float* __restrict__ y, con
     for (int c = lane; c < d_v; c += kWarp) ss = fmaf(yr[c], yr[c], ss);
     ss = warp_sum(ss);
     const float inv = 1.0f / sqrtf(ss / static_cast<float>(d_v) + eps);
+    for (int c = lane; c < d_v; c += kWarp) yr[c] = to_f32<Tin>(gr[c]) * yr[c] * inv;
+  }
+}
+
+// Sum of squares of each row of y over its d_v columns (one warp per row, a
+// fixed order). When the d_v columns of a layer are split across devices,
+// adding the devices' sums gives the full row's sum for the RMS norm.
+static __global__ void __launch_bounds__(256) k_row_sumsq(const float* __restrict__ y, int64_t n_rows, int d_v,
+                                                          float* __restrict__ ss) {
+  const int lane = lane_id();
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / kWarp);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / kWarp) + threadIdx.x / kWarp;
+       row < n_rows; row += warps) {
+    const float* yr = y + row * d_v;
+    float s = 0.f;
+    for (int c = lane; c < d_v; c += kWarp) s = fmaf(yr[c], yr[c], s);
+    s = warp_sum(s);
+    if (lane == 0) ss[row] = s;
+  }
+}
+
+// The RMS-norm x gate on a column slice of rows of d_total values, given the
+// full rows' sums of squares: y <- g * y / sqrt(ss / d_total + eps).
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_rmsnorm_gate_rows(float* __restrict__ y, const Tin* __restrict__ g,
+                                                           const float* __restrict__ ss, int64_t n_rows, int d_v,
+                                                           int d_total, float eps) {
+  const int lane = lane_id();
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / kWarp);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / kWarp) + threadIdx.x / kWarp;
+       row < n_rows; row += warps) {
+    float* yr = y + row * d_v;
+    const Tin* gr = g + row * d_v;
+    const float inv = 1.0f / sqrtf(ss[row] / static_cast<float>(d_total) + eps);
     for (int c = lane; c < d_v; c += kWarp) yr[c] = to_f32<Tin>(gr[c]) * yr[c] * inv;
   }
 }

@@ -1,0 +1,506 @@
+// The sparse gated delta recurrence for states far larger than the chip,
+// when few (b, h) sequences are in flight (sm_100a).
+//
+// SDM explainer (papers.ananclaw.com), section 3.1: step 2 writes the W
+// selected slots, M~ = alpha_t M[i], M[i] = M~ + beta_t k_i (v_t - M~); step 3
+// reads y_t = sum_r q_r M_t[r] after the write. The kernel uses the factored
+// form M[i] = (alpha_t (1 - beta_t k_i)) M[i] + (beta_t k_i) v_t in fp32 and
+// rounds to the state dtype on every store, like the other recurrence
+// kernels.
+//
+// Why a third kernel. Every token touches W + R random state rows, and one
+// B200 SM moves at most about one random 128-byte row per 3 ns, however the
+// copies are issued (measured with cp.async from 4-16 warps and with TMA
+// gather4: ~40 GB/s per SM). The long-context workload has only B*H = 2
+// sequences, so a grid of one CTA per (b, h) and 128-byte column tile fills
+// 64 SMs and cannot pass ~2.5 TB/s. Here each (b, h) column tile is split
+// over `parts` CTAs by a hash bit of the slot index: a part owns a fixed
+// half of the slots, so it alone writes and reads them and the parts need no
+// synchronisation; each adds its partial read sum into y (with two parts the
+// sum 0 + a + b does not depend on their order, so y stays reproducible).
+//
+// Within a CTA, for token t:
+//   * every thread first gathers its share of the rows of token t + P - 1
+//     (16-byte cp.async, completion counted on the stage's mbarrier), so the
+//     copies run P - 1 tokens ahead of their use;
+//   * write warps apply the write to the part's write entries (each lane owns
+//     one 16-byte unit of a row), store the rows to global memory and keep
+//     them in a ring of written-row stages;
+//   * read warps sum the part's read entries; lane bits above the unit index
+//     select entries, so a warp reduces its columns with shuffles alone and
+//     adds them to y;
+//   * one block barrier ends the token.
+// A row gathered early is stale when one of the P - 1 tokens in between
+// wrote it; the hazard plan in the records names that write (token t - k,
+// write entry j of this part) and the row is taken from the written-row ring
+// instead; a read of a slot written by the same token (k = 0) recomputes that
+// write from its source.
+#pragma once
+
+#include "sdm_device.cuh"
+#include "sdm_scan.cuh"
+
+namespace sdm {
+
+// Per-token record of one part (32-bit words):
+//   uint16 src_w[Wp] | uint16 src_r[Rp] | float2 awcw[Wp] | f32 q_r[Rp] |
+//   int32 slot_w[Wp] | int32 slot_r[Rp] | int32 nw, int32 nr, 0, 0
+// The part's write and read entries are compacted to the front in selection
+// order (nw, nr of them); the rest is padding (slot -1, coefficients 0).
+// Everything a consumer lane needs is precomputed by the record build:
+//   src    the row of the kernel's stage space (shared memory, RS bytes a row)
+//          the entry's source row sits in: rows [0, P E) are the gather
+//          stages (stage s, entry e at s E + e; writes first, reads from Wp),
+//          rows P E + s Wp + j the written-row ring (token t - k's write j,
+//          s = (t - k) mod P) when a token in between wrote the slot (the
+//          hazard plan); a read of a slot written by the same token carries
+//          0x8000 | j: that write recomputed from its own source;
+//   awcw   the write's factored coefficients a = alpha (1 - beta k), c = beta k;
+//   q_r    the read weight; slot_*: the rows the part gathers and stores.
+struct PipeLayout {
+  int Wp, Rp;
+  int off_src_w, off_src_r, off_awcw, off_q_r, off_slot_w, off_slot_r, off_meta;
+  int words;
+};
+
+__host__ __device__ inline PipeLayout pipe_layout(int W, int R) {
+  PipeLayout pl{};
+  pl.Wp = (W + 7) / 8 * 8;
+  pl.Rp = (R + 7) / 8 * 8;
+  pl.off_src_w = 0;
+  pl.off_src_r = pl.Wp / 2;
+  pl.off_awcw = pl.off_src_r + pl.Rp / 2;
+  pl.off_q_r = pl.off_awcw + 2 * pl.Wp;
+  pl.off_slot_w = pl.off_q_r + pl.Rp;
+  pl.off_slot_r = pl.off_slot_w + pl.Wp;
+  pl.off_meta = pl.off_slot_r + pl.Rp;
+  pl.words = pl.off_meta + 4;
+  return pl;
+}
+
+constexpr uint32_t kSrcSameToken = 0x8000u;  // src_r flag: recompute this token's write (low bits: j)
+
+// Part of a slot: a hash bit, so that structured selections (e.g. slots that
+// share a grid column) still spread over both parts.
+__device__ __forceinline__ int slot_part(uint32_t slot, int parts) {
+  return parts == 1 ? 0 : static_cast<int>((slot * 0x9E3779B1u) >> 31);
+}
+
+constexpr int kPipeTokensPerBlock = 32;
+
+// Shared-memory bytes of k_build_pipe_records.
+__host__ __device__ constexpr size_t pipe_records_smem(int W, int R, int P, int log2_cells, int parts) {
+  return static_cast<size_t>(kPipeTokensPerBlock + P - 1) * ((size_t{1} << log2_cells) * 4 + W * 2) +
+         static_cast<size_t>(kPipeTokensPerBlock) * R * 2 + 4 + static_cast<size_t>(kPipeTokensPerBlock) * parts * 8;
+}
+
+// Records of one (b, h) and 32 tokens for every part: compaction of each
+// part's write and read entries (warp ballots, in selection order), the
+// hazard plan against the written slots of the P - 1 tokens before (one
+// open-addressing table per token, slot -> compacted write entry), and, when
+// y_zero is given, zeros for those tokens' y rows (the recurrence adds the
+// parts' sums into it). Slot indices outside [0, N) are left out and set the
+// device error word.
+template <typename Tin>
+__global__ void __launch_bounds__(256) k_build_pipe_records(
+    const int32_t* __restrict__ idx_w, const float* __restrict__ w_w, const int32_t* __restrict__ idx_r,
+    const float* __restrict__ w_r, const Tin* __restrict__ alpha, const Tin* __restrict__ beta, int T, int H, int N,
+    int W, int R, int P, int parts, int log2_cells, PipeLayout pl, uint32_t* __restrict__ rec,
+    float* __restrict__ y_zero, int d_v, unsigned* err) {
+  const int E = pl.Wp + pl.Rp;  // rows of one gather stage
+  extern __shared__ uint32_t sm[];
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int t0 = blockIdx.x * kPipeTokensPerBlock;
+  const int t_end = min(T, t0 + kPipeTokensPerBlock);
+  const int t_first = max(0, t0 - (P - 1));
+  const int n_tab = t_end - t_first, n_own = t_end - t0;
+  const int n_cells = 1 << log2_cells;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t* cells = sm;                                               // [n_tab][n_cells]
+  int16_t* jcw = reinterpret_cast<int16_t*>(cells + n_tab * n_cells);  // [n_tab][W]
+  int16_t* rcr = jcw + n_tab * W;                                     // [n_own][R]
+  const int n16 = n_tab * W + n_own * R;
+  int* cnt = reinterpret_cast<int*>(jcw + ((n16 + 1) & ~1));          // [n_own][parts][2]
+
+  for (int i = threadIdx.x; i < n_tab * n_cells; i += blockDim.x) cells[i] = kEmptyCell;
+  __syncthreads();
+
+  // 1. compaction (one warp per token) and the tables of written slots
+  for (int tt = t_first + warp; tt < t_end; tt += blockDim.x / 32) {
+    const int64_t th = (static_cast<int64_t>(b) * T + tt) * H + h;
+    uint32_t* tab = cells + (tt - t_first) * n_cells;
+    int base[2] = {0, 0};
+    for (int j0 = 0; j0 < W; j0 += 32) {
+      const int j = j0 + lane;
+      const int slot = j < W ? idx_w[th * W + j] : -1;
+      const bool valid = j < W && slot >= 0 && slot < N;
+      const int part = valid ? slot_part(static_cast<uint32_t>(slot), parts) : -1;
+      int jc = -1;
+      for (int p = 0; p < parts; ++p) {
+        const unsigned m = __ballot_sync(0xffffffffu, part == p);
+        if (part == p) jc = base[p] + __popc(m & lanemask_lt());
+        base[p] += __popc(m);
+      }
+      if (j < W) jcw[(tt - t_first) * W + j] = static_cast<int16_t>(jc);
+      if (valid) {
+        const uint32_t packed = static_cast<uint32_t>(slot) * 512u + static_cast<uint32_t>(jc);
+        uint32_t pos = slot_hash(static_cast<uint32_t>(slot), log2_cells);
+        for (int probe = 0; probe < n_cells; ++probe) {  // at most W < n_cells entries per table
+          const uint32_t prev = atomicCAS(&tab[pos], kEmptyCell, packed);
+          if (prev == kEmptyCell || (prev >> 9) == static_cast<uint32_t>(slot)) break;
+          pos = (pos + 1) & (n_cells - 1);
+        }
+      }
+    }
+    if (tt >= t0) {
+      int rbase[2] = {0, 0};
+      for (int r0 = 0; r0 < R; r0 += 32) {
+        const int r = r0 + lane;
+        const int slot = r < R ? idx_r[th * R + r] : -1;
+        const bool valid = r < R && slot >= 0 && slot < N;
+        const int part = valid ? slot_part(static_cast<uint32_t>(slot), parts) : -1;
+        int rc = -1;
+        for (int p = 0; p < parts; ++p) {
+          const unsigned m = __ballot_sync(0xffffffffu, part == p);
+          if (part == p) rc = rbase[p] + __popc(m & lanemask_lt());
+          rbase[p] += __popc(m);
+        }
+        if (r < R) rcr[(tt - t0) * R + r] = static_cast<int16_t>(rc);
+      }
+      if (lane < parts) {
+        cnt[((tt - t0) * parts + lane) * 2] = base[lane];
+        cnt[((tt - t0) * parts + lane) * 2 + 1] = rbase[lane];
+      }
+    }
+  }
+  __syncthreads();
+
+  // 2. entries: compacted position, hazard plan, source row
+  const int WR = W + R;
+  for (int x = threadIdx.x; x < n_own * WR; x += blockDim.x) {
+    const int t = t0 + x / WR, e = x % WR;
+    const int64_t th = (static_cast<int64_t>(b) * T + t) * H + h;
+    int slot, c;
+    float wt;
+    if (e < W) {
+      slot = idx_w[th * W + e];
+      wt = w_w[th * W + e];
+      c = jcw[(t - t_first) * W + e];
+    } else {
+      slot = idx_r[th * R + e - W];
+      wt = w_r[th * R + e - W];
+      c = rcr[(t - t0) * R + e - W];
+    }
+    if (c < 0) {
+      atomicOr(err, kErrIndexOutOfRange);
+      continue;
+    }
+    const int part = slot_part(static_cast<uint32_t>(slot), parts);
+    int code = -1;
+    for (int k = (e < W ? 1 : 0); k < P && code < 0; ++k) {
+      const int tt = t - k;
+      if (tt < 0) break;
+      const uint32_t* tab = cells + (tt - t_first) * n_cells;
+      uint32_t pos = slot_hash(static_cast<uint32_t>(slot), log2_cells);
+      for (int probe = 0; probe < n_cells; ++probe) {
+        const uint32_t cur = tab[pos];
+        if (cur == kEmptyCell) break;
+        if ((cur >> 9) == static_cast<uint32_t>(slot)) {
+          code = (k << 9) | static_cast<int>(cur & 511u);
+          break;
+        }
+        pos = (pos + 1) & (n_cells - 1);
+      }
+    }
+    uint32_t* r = rec + ((static_cast<int64_t>(bh) * parts + part) * T + t) * pl.words;
+    // the entry's source row in the stage space (see PipeLayout)
+    uint32_t src;
+    if (code < 0) src = static_cast<uint32_t>((t % P) * E + (e < W ? c : pl.Wp + c));
+    else if ((code >> 9) == 0) src = kSrcSameToken | static_cast<uint32_t>(code & 511);
+    else src = static_cast<uint32_t>(P * E + ((t - (code >> 9)) % P) * pl.Wp + (code & 511));
+    if (e < W) {
+      const float a_t = to_f32<Tin>(alpha[th]), b_t = to_f32<Tin>(beta[th]);
+      const float cw = b_t * wt;
+      r[pl.off_slot_w + c] = static_cast<uint32_t>(slot);
+      reinterpret_cast<float2*>(r + pl.off_awcw)[c] = make_float2(a_t * (1.0f - cw), cw);
+      reinterpret_cast<uint16_t*>(r + pl.off_src_w)[c] = static_cast<uint16_t>(src);
+    } else {
+      r[pl.off_slot_r + c] = static_cast<uint32_t>(slot);
+      r[pl.off_q_r + c] = __float_as_uint(wt);
+      reinterpret_cast<uint16_t*>(r + pl.off_src_r)[c] = static_cast<uint16_t>(src);
+    }
+  }
+
+  // 3. padding after the compacted entries, and the counts, alpha and beta
+  const int EP = pl.Wp + pl.Rp;
+  for (int x = threadIdx.x; x < n_own * parts * EP; x += blockDim.x) {
+    const int t = t0 + x / (parts * EP), rem = x % (parts * EP), part = rem / EP, pos = rem % EP;
+    const int* cn = cnt + ((t - t0) * parts + part) * 2;
+    uint32_t* r = rec + ((static_cast<int64_t>(bh) * parts + part) * T + t) * pl.words;
+    if (pos < pl.Wp) {
+      if (pos >= cn[0]) {  // padding: a gathered row of its own, coefficients that keep it
+        r[pl.off_slot_w + pos] = 0xFFFFFFFFu;
+        reinterpret_cast<float2*>(r + pl.off_awcw)[pos] = make_float2(0.f, 0.f);
+        reinterpret_cast<uint16_t*>(r + pl.off_src_w)[pos] = static_cast<uint16_t>((t % P) * E + pos);
+      }
+    } else if (pos - pl.Wp >= cn[1]) {
+      const int i = pos - pl.Wp;
+      r[pl.off_slot_r + i] = 0xFFFFFFFFu;
+      r[pl.off_q_r + i] = 0u;
+      reinterpret_cast<uint16_t*>(r + pl.off_src_r)[i] = static_cast<uint16_t>((t % P) * E + pos);
+    }
+  }
+  for (int x = threadIdx.x; x < n_own * parts; x += blockDim.x) {
+    const int t = t0 + x / parts, part = x % parts;
+    const int* cn = cnt + ((t - t0) * parts + part) * 2;
+    uint32_t* r = rec + ((static_cast<int64_t>(bh) * parts + part) * T + t) * pl.words;
+    r[pl.off_meta] = static_cast<uint32_t>(cn[0]);
+    r[pl.off_meta + 1] = static_cast<uint32_t>(cn[1]);
+    r[pl.off_meta + 2] = 0u;
+    r[pl.off_meta + 3] = 0u;
+  }
+
+  // 4. zeros for the y rows the parts add into
+  if (y_zero != nullptr) {
+    const int q4 = d_v / 4;
+    for (int x = threadIdx.x; x < n_own * q4; x += blockDim.x) {
+      const int t = t0 + x / q4;
+      float4* row = reinterpret_cast<float4*>(y_zero + ((static_cast<int64_t>(b) * T + t) * H + h) * d_v);
+      row[x % q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+}
+
+struct PipeArgs {
+  int B, T, H, N, d_v, W, R, parts;
+  PipeLayout pl;
+  const uint32_t* rec;  // [B, H, parts, T, pl.words]
+  const void* v;        // [B, T, H, d_v] in dtype
+  void* M;              // [B, H, N, d_v] state dtype, updated in place
+  float* y;             // [B, T, H, d_v]; with parts > 1 zero on entry
+  unsigned* err;
+};
+
+// Shared-memory bytes of k_scan_pipelined (host and device agree on this).
+__host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
+                                                     int s_in) {
+  return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(P) * Wp * C * s_state +
+         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in + (P + 2) * 8;
+}
+
+// Sums a[0:VE) (the VE columns of one 16-byte unit, held by the lanes that
+// share lane % UR) over the 32 / UR entry groups of the warp in a fixed
+// order, then stores the column sums to y[0:VE), or adds them there when
+// several parts contribute.
+template <int VE, int UR>
+__device__ __forceinline__ void reduce_put_unit(float (&a)[VE], float* y, int lane, bool add) {
+  int n = VE, off = 0, bmask = 0;
+#pragma unroll
+  for (int o = 16; o >= UR; o >>= 1) {
+    if (n > 1) {
+      const bool hi = lane & o;
+      const int h = n / 2;
+#pragma unroll
+      for (int j = 0; j < VE / 2; ++j) {
+        if (j < h) {
+          const float keep = hi ? a[j + h] : a[j];
+          const float send = hi ? a[j] : a[j + h];
+          a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      off += hi ? h : 0;
+      n = h;
+    } else {
+      a[0] += __shfl_xor_sync(0xffffffffu, a[0], o);
+      bmask |= o;
+    }
+  }
+  if ((lane & bmask) == 0) {
+#pragma unroll
+    for (int j = 0; j < VE; ++j) {
+      if (j < n) {
+        if (add) atomicAdd(y + off + j, a[j]);
+        else y[off + j] = a[j];
+      }
+    }
+  }
+}
+
+template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR>
+__global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeArgs a) {
+  constexpr int NT = (NWW + NWR) * kWarp;
+  constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
+  constexpr int U = C / VE;             // units per row segment
+  constexpr int RS = C * sizeof(Tst);   // bytes of a row segment
+  constexpr int UR = U / NWR;           // units per read warp
+  constexpr int GR = kWarp / UR;        // read entries per read-warp instruction
+  static_assert(U >= 1 && U <= kWarp && kWarp % U == 0, "a row segment spans a divisor of the warp");
+  static_assert(U % NWR == 0 && kWarp % UR == 0, "read warps split the units evenly");
+  static_assert(NT % U == 0, "gather lanes cover whole rows");
+  static_assert(L >= P, "a chunk of records is staged before its tokens are gathered");
+  extern __shared__ __align__(16) unsigned char smem[];
+  const PipeLayout pl = a.pl;
+  const int Wp = pl.Wp, E = pl.Wp + pl.Rp, words = pl.words, T = a.T;
+  unsigned char* lstage = smem;                                                    // [P][E][RS]
+  unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [P][Wp][RS]
+  uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(P) * Wp * RS);  // [2][L][words]
+  Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
+  uint64_t* full = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);                 // [P]
+  uint64_t* cbar = full + P;                                                       // [2]
+
+  const int part = blockIdx.x % a.parts, bh = blockIdx.x / a.parts;
+  const int b = bh / a.H, h = bh % a.H;
+  const int c0 = blockIdx.y * C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * a.N * a.d_v + c0;
+  const uint32_t* rec_g = a.rec + (static_cast<int64_t>(bh) * a.parts + part) * T * words;
+  const int64_t tok_step = static_cast<int64_t>(a.H) * a.d_v;  // [B, T, H, d_v] rows of one (b, h)
+  float* y_bh = a.y + static_cast<int64_t>(b) * T * tok_step + static_cast<int64_t>(h) * a.d_v + c0;
+  const Tin* v_bh = static_cast<const Tin*>(a.v) + static_cast<int64_t>(b) * T * tok_step + static_cast<int64_t>(h) * a.d_v + c0;
+
+  if (tid == 0) {
+    for (int s = 0; s < P; ++s) mbar_init(&full[s], NT);
+    mbar_init(&cbar[0], 1);
+    mbar_init(&cbar[1], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int n_chunks = (T + L - 1) / L;
+  if (n_chunks == 0) return;
+  int last_chunk = -1;  // thread 0: the last chunk whose copies it issued
+  auto load_chunk = [&](int c) {  // thread 0: records and v rows of tokens [cL, cL + L)
+    const int bi = c & 1, t0 = c * L, nt = min(L, T - t0);
+    const uint32_t rb = static_cast<uint32_t>(nt) * words * 4u, vb = C * sizeof(Tin);
+    mbar_arrive_expect_tx(&cbar[bi], rb + nt * vb);
+    bulk_g2s(recbuf + static_cast<size_t>(bi) * L * words, rec_g + static_cast<int64_t>(t0) * words, rb, &cbar[bi]);
+    for (int i = 0; i < nt; ++i)
+      bulk_g2s(vbuf + (static_cast<size_t>(bi) * L + i) * C, v_bh + static_cast<int64_t>(t0 + i) * tok_step, vb,
+               &cbar[bi]);
+    last_chunk = c;
+  };
+  auto rec_of = [&](int t) { return recbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * words; };
+  auto chunk_ok = [&](int c) {
+    const bool ok = mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err);
+    return !__syncthreads_or(!ok);
+  };
+  // Token u's rows of this part into stage u % P (every thread its share, one
+  // 16-byte copy per row and unit); each thread then arrives on the stage's
+  // barrier, which completes once all copies have landed.
+  auto gather = [&](int u) {
+    const uint32_t* rec = rec_of(u);
+    const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
+    unsigned char* st = lstage + static_cast<size_t>(u % P) * E * RS + (tid % U) * 16;
+    const Tst* src = Mbh + (tid % U) * VE;
+    const uint32_t* slw = rec + pl.off_slot_w;
+    const uint32_t* slr = rec + pl.off_slot_r;
+    for (int e = tid / U; e < nw; e += NT / U)
+      cp_async16(st + static_cast<size_t>(e) * RS, src + static_cast<int64_t>(slw[e]) * a.d_v);
+    for (int e = tid / U; e < nr; e += NT / U)
+      cp_async16(st + static_cast<size_t>(Wp + e) * RS, src + static_cast<int64_t>(slr[e]) * a.d_v);
+    cp_async_mbar_arrive(&full[u % P]);
+  };
+  auto finish = [&]() {  // copies in flight land before the block exits
+    cp_async_wait_all();
+    if (tid == 0)
+      for (int c = max(0, last_chunk - 1); c <= last_chunk; ++c) mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err);
+  };
+
+  if (tid == 0) {
+    load_chunk(0);
+    if (n_chunks > 1) load_chunk(1);
+  }
+  if (!chunk_ok(0)) {
+    finish();
+    return;
+  }
+  for (int u = 0; u < P - 1 && u < T; ++u) gather(u);
+
+  const bool writer = warp < NWW;
+  const int qw = lane % U;                              // write lanes: unit of every entry they take
+  const int qr = (warp - NWW) * UR + lane % UR;         // read lanes: unit, entries lane / UR + k GR
+  const int q_mine = writer ? qw : qr;
+#pragma unroll 1
+  for (int t = 0; t < T; ++t) {
+    const int u = t + P - 1;
+    if (u < T) {
+      if (u % L == 0 && !chunk_ok(u / L)) {
+        finish();
+        return;
+      }
+      gather(u);
+    }
+    const bool ok = mbar_wait_bounded(&full[t % P], (t / P) & 1, a.err);
+    if (ok) {
+      const uint32_t* rec = rec_of(t);
+      const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
+      const uint16_t* sw = reinterpret_cast<const uint16_t*>(rec + pl.off_src_w);
+      const float2* ac = reinterpret_cast<const float2*>(rec + pl.off_awcw);
+      float vv[VE];
+      load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * C + q_mine * VE, vv);
+      // the write of entry j on the 16-byte unit q of its source row (fp32 math, state rounding by the caller)
+      auto written = [&](int j, int q, float (&m)[VE]) {
+        unpack16<Tst>(*reinterpret_cast<const uint4*>(smem + static_cast<size_t>(sw[j]) * RS + q * 16), m);
+        const float2 c = ac[j];
+        delta_update<VE>(m, vv, c.x, c.y);
+      };
+      if (writer) {
+        unsigned char* ws = wstage + static_cast<size_t>(t % P) * Wp * RS + qw * 16;
+        const uint32_t* slw = rec + pl.off_slot_w;
+        const int n = nw * U;
+        // two independent units per iteration
+        for (int p0 = warp * kWarp + lane; p0 < n; p0 += 2 * NWW * kWarp) {
+          const int p1 = p0 + NWW * kWarp;
+          const bool has1 = p1 < n;
+          const int j0 = p0 / U, j1 = has1 ? p1 / U : j0;
+          float m0[VE], m1[VE];
+          written(j0, qw, m0);
+          written(j1, qw, m1);
+          const uint4 k0 = pack16<Tst>(m0), k1 = pack16<Tst>(m1);
+          *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j0) * RS) = k0;
+          *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slw[j0]) * a.d_v + qw * VE) = k0;
+          if (has1) {
+            *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j1) * RS) = k1;
+            *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slw[j1]) * a.d_v + qw * VE) = k1;
+          }
+        }
+      } else {
+        const uint16_t* sr = reinterpret_cast<const uint16_t*>(rec + pl.off_src_r);
+        const float* qw_r = reinterpret_cast<const float*>(rec + pl.off_q_r);
+        auto read_row = [&](int i, float (&m)[VE]) {
+          const uint32_t src = sr[i];
+          if (src & kSrcSameToken) {  // written by this token: that write, rounded as stored
+            written(static_cast<int>(src & 0x7FFFu), qr, m);
+            unpack16<Tst>(pack16<Tst>(m), m);
+          } else {
+            unpack16<Tst>(*reinterpret_cast<const uint4*>(smem + static_cast<size_t>(src) * RS + qr * 16), m);
+          }
+        };
+        float acc[VE];
+#pragma unroll
+        for (int j = 0; j < VE; ++j) acc[j] = 0.f;
+        for (int i0 = lane / UR; i0 < nr; i0 += 2 * GR) {
+          const int i1 = i0 + GR;
+          const bool has1 = i1 < nr;
+          float m0[VE], m1[VE];
+          read_row(i0, m0);
+          read_row(has1 ? i1 : i0, m1);
+          weighted_add<VE>(acc, m0, qw_r[i0]);
+          weighted_add<VE>(acc, m1, has1 ? qw_r[i1] : 0.0f);
+        }
+        reduce_put_unit<VE, UR>(acc, y_bh + static_cast<int64_t>(t) * tok_step + qr * VE, lane, a.parts > 1);
+      }
+    }
+    // token t done: its rows are in global memory and in the written-row ring
+    if (__syncthreads_or(!ok)) {
+      finish();
+      return;
+    }
+    if (tid == 0 && (t + 1) % L == 0 && (t + 1) / L + 1 < n_chunks) {
+      fence_proxy_async_smem();
+      load_chunk((t + 1) / L + 1);  // chunk (t+1)/L - 1 is consumed: refill its buffer
+    }
+  }
+  finish();
+}
+
+}  // namespace sdm

@@ -1,0 +1,10 @@
+// Decode-step instances for float inputs and a bf16 state.
+
+#include "sdm_decode_launch.h"
+
+namespace sdm_host {
+
+template sdm_status_t launch_decode_for<float, bf16>(const FastTopkPlan&, const sdm::DecodeArgs&, size_t, int,
+                                                        cudaStream_t);
+
+}  // namespace sdm_host

@@ -16,8 +16,9 @@ SDM_OK = 0
 STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARGUMENT", 2: "SDM_ERR_UNSUPPORTED", 3: "SDM_ERR_CUDA",
                 4: "SDM_ERR_DEVICE_FAULT"}
 F32, BF16, FP8_B16 = 0, 1, 2  # FP8_B16: state only (E4M3 codes + a power-of-two scale per 16 values)
-VARIANTS = {"auto": 0, "resident": 1, "streaming": 2}
+VARIANTS = {"auto": 0, "resident": 1, "streaming": 2, "pipelined": 3}
 NOALLOC_SCRATCH_BYTES = 16 << 20  # SDM_NOALLOC_SCRATCH_BYTES in include/sdm.h
+ABI_VERSION = 2  # SDM_ABI_VERSION in include/sdm.h
 
 
 class Shape(ctypes.Structure):
@@ -26,7 +27,7 @@ class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("sqrt_n", ctypes.c_int32), ("W", ctypes.c_int32), ("R", ctypes.c_int32),
                 ("d_v", ctypes.c_int32), ("in_dtype", ctypes.c_int32), ("state_dtype", ctypes.c_int32),
-                ("rms_eps", ctypes.c_float), ("variant", ctypes.c_int32)]
+                ("rms_eps", ctypes.c_float), ("variant", ctypes.c_int32), ("tile", ctypes.c_int32)]
 
 
 _p = ctypes.c_void_p
@@ -37,6 +38,8 @@ _shape_p = ctypes.POINTER(Shape)
 # name -> (restype, argtypes); one entry per function declared in include/sdm.h.
 PROTOTYPES = {
     "sdm_abi_version": (_i32, []),
+    "sdm_row_sumsq": (_i32, [_p, ctypes.c_int64, _i32, _p, _p]),
+    "sdm_rmsnorm_gate_rows": (_i32, [_p, _p, _i32, _p, ctypes.c_int64, _i32, _i32, ctypes.c_float, _p]),
     "sdm_status_string": (ctypes.c_char_p, [_i32]),
     "sdm_last_error": (ctypes.c_char_p, []),
     "sdm_pkm_topk": (_i32, [_p, _i32, _i32, _i32, _i32, _i32, _i32, _p, _p, _p]),
@@ -89,7 +92,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
-    if lib.sdm_abi_version() != 1:
+    if lib.sdm_abi_version() != ABI_VERSION:
         raise RuntimeError("libsdm_b200.so ABI version mismatch")
     if path is None:
         _LIB = lib

@@ -32,7 +32,7 @@ def test_header_and_binding_agree():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.sdm_abi_version() == 1
+    assert lib.sdm_abi_version() == native.ABI_VERSION == 2
 
 
 def test_only_the_abi_is_exported(lib):
@@ -58,8 +58,8 @@ def shape(**kw):
 
 
 @pytest.mark.parametrize("bad", [dict(sqrt_n=0), dict(sqrt_n=1025), dict(W=0), dict(R=65), dict(W=257, sqrt_n=32),
-                                 dict(d_v=24), dict(d_v=8), dict(B=-1), dict(in_dtype=7), dict(variant=3),
-                                 dict(rms_eps=-1.0)])
+                                 dict(d_v=24), dict(d_v=8), dict(B=-1), dict(in_dtype=7), dict(variant=4),
+                                 dict(rms_eps=-1.0), dict(tile=-1), dict(tile=65)])
 def test_invalid_shapes_rejected_on_host(lib, bad):
     s = shape(**bad)
     assert lib.sdm_scan_workspace_bytes(ctypes.byref(s)) == 0
@@ -69,9 +69,14 @@ def test_invalid_shapes_rejected_on_host(lib, bad):
 
 
 def test_workspace_sizes(lib):
+    """Without a device the records workspace is the largest any recurrence
+    kernel needs: the streaming kernel's records, or the pipelined kernel's,
+    one per slot part (two parts)."""
     s = shape()
     rec_words = 4 + 4 + 4 + 4 + 8 // 2 + 4  # Wp, Wp, Rp, Rp, Fp/2, alpha/beta block
-    rec = (2 * 3 * 5 * rec_words * 4 + 255) // 256 * 256
+    # W, R rounded to 8: uint16 source rows, (a, c) pairs, read weights, slots, counts
+    pipe_words = 8 // 2 + 8 // 2 + 2 * 8 + 8 + 8 + 8 + 4
+    rec = max((2 * 3 * 5 * rec_words * 4 + 255) // 256 * 256, (2 * 2 * 3 * 5 * pipe_words * 4 + 255) // 256 * 256)
     assert lib.sdm_scan_workspace_bytes(ctypes.byref(s)) == rec
     per = (2 * 5 * 3 * 4 * 4 + 255) // 256 * 256
     assert lib.sdm_layer_forward_workspace_bytes(ctypes.byref(s)) == 4 * per + rec

@@ -134,6 +134,16 @@ SCAN = [
     (16, 64, 7, 9, "bf16", "bf16", "resident", 33, 1, 3),
     (16, 48, 12, 4, "f32", "f32", "streaming", 19, 1, 1),
     (256, 2048, 64, 64, "bf16", "bf16", "streaming", 17, 1, 1),
+    # the pipelined kernel: slots split over two CTAs per column tile (parts = 2), except in the
+    # last case, whose 96 column tiles leave room for one CTA each (parts = 1)
+    (32, 128, 64, 64, "bf16", "f32", "pipelined", 29, 2, 2),
+    (128, 512, 64, 64, "bf16", "f32", "pipelined", 23, 1, 2),
+    (64, 64, 64, 64, "bf16", "bf16", "pipelined", 31, 1, 1),
+    (16, 64, 7, 9, "bf16", "bf16", "pipelined", 33, 1, 3),
+    (32, 128, 100, 30, "f32", "f32", "pipelined", 25, 1, 2),
+    (4, 32, 16, 16, "f32", "f32", "pipelined", 50, 1, 2),
+    (256, 2048, 64, 64, "bf16", "bf16", "pipelined", 17, 1, 1),
+    (64, 2048, 64, 64, "bf16", "bf16", "pipelined", 20, 1, 3),
 ]
 
 
@@ -160,7 +170,7 @@ def test_scan_matches_oracle(sdm, oracle, cuda_device, case):
     assert_rel_close(f32(M), oM, tol, "M_T")
 
 
-@pytest.mark.parametrize("variant", ["resident", "streaming"])
+@pytest.mark.parametrize("variant", ["resident", "streaming", "pipelined"])
 def test_scan_deterministic_and_chunkable(sdm, cuda_device, variant):
     """Two runs are bit-identical, and scanning [0, T1) then [T1, T) equals one
     scan over [0, T) bit for bit (the state is the checkpoint)."""
@@ -182,18 +192,19 @@ def test_variants_agree(sdm, cuda_device):
     shape = synth.Shape("t", B=1, T=40, H=2, sqrt_n=32, d_v=128, W=64, R=64, in_dtype="bf16", state_dtype="f32")
     inp = scan_inputs(shape, seed=9)
     ya, Ma = _run_scan(sdm, cuda_device, shape, inp, "resident")
-    yb, Mb = _run_scan(sdm, cuda_device, shape, inp, "streaming")
-    assert_rel_close(yb.cpu().numpy(), ya.cpu().numpy(), 1e-5, "y")
-    assert_rel_close(f32(Mb), f32(Ma), 1e-5, "M_T")
+    for variant in ("streaming", "pipelined"):
+        yb, Mb = _run_scan(sdm, cuda_device, shape, inp, variant)
+        assert_rel_close(yb.cpu().numpy(), ya.cpu().numpy(), 1e-5, f"y ({variant})")
+        assert_rel_close(f32(Mb), f32(Ma), 1e-5, f"M_T ({variant})")
 
 
 def test_scan_out_of_range_index_flagged(sdm, cuda_device):
-    shape = synth.Shape("t", B=1, T=8, H=1, sqrt_n=8, d_v=16, W=4, R=4, in_dtype="f32", state_dtype="f32")
+    shape = synth.Shape("t", B=1, T=8, H=1, sqrt_n=8, d_v=32, W=4, R=4, in_dtype="f32", state_dtype="f32")
     inp = scan_inputs(shape, seed=3)
     inp["idx_w"][0, 3, 0, 1] = 64  # N = 64
     inp["idx_r"][0, 5, 0, 2] = -7
     d = {k: v.to(cuda_device) for k, v in inp.items()}
-    for variant in ("resident", "streaming"):
+    for variant in ("resident", "streaming", "pipelined"):
         M = d["M"].clone()
         sdm.scan(d["idx_w"], d["w_w"], d["idx_r"], d["w_r"], d["v"], d["alpha"], d["beta"], M, variant=variant)
         with pytest.raises(sdm.SdmError, match="DEVICE_FAULT"):
@@ -295,7 +306,7 @@ def test_layer_forward_reduced_workloads(sdm, oracle, cuda_device, name):
     _layer_case(sdm, oracle, cuda_device, s.replace(B=min(s.B, 2), T=37, H=min(s.H, 3)), seed=1)
 
 
-@pytest.mark.parametrize("variant", ["resident", "streaming"])
+@pytest.mark.parametrize("variant", ["resident", "streaming", "pipelined"])
 def test_layer_forward_epilogue(sdm, oracle, cuda_device, variant):
     s = synth.WORKLOADS["d2048_h16_n1024_dv128"].replace(B=1, T=21, H=2)
     _layer_case(sdm, oracle, cuda_device, s, seed=2, with_gate=True, variant=variant)
