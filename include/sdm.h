@@ -332,8 +332,9 @@ SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp,
 /* Kernel launches one sdm_layer_forward call makes for this shape on the
  * current device (with_gate != 0: with the epilogue): the two selections,
  * the record build and the recurrence, plus the state copy for the streaming
- * recurrence, plus the epilogue. -1 for an invalid or unsupported shape. For
- * profiles and logs. */
+ * and pipelined recurrences, plus the pass that adds the second slot part's
+ * read sums into y (pipelined, two parts), plus the epilogue. -1 for an
+ * invalid or unsupported shape. For profiles and logs. */
 SDM_API int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate);
 
 /* Kernel launches one sdm_layer_step call makes for this shape, without the

@@ -359,11 +359,17 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
   return SDM_OK;
 }
 
-// Workspace of the per-token records for the chosen kernel.
+// Bytes of the second slot part's read sums (pipelined kernel with two parts).
+size_t y_other_bytes(const sdm_shape_t& s, const ScanChoice& c) {
+  if (c.kind != SDM_VARIANT_PIPELINED || c.parts < 2) return 0;
+  return align256(static_cast<size_t>(s.B) * s.T * s.H * s.d_v * 4u);
+}
+// Workspace of the chosen recurrence kernel: per-token records (and, for the
+// pipelined kernel with two parts, the second part's read sums after them).
 size_t records_bytes(const sdm_shape_t& s, const ScanChoice& c) {
   const int64_t n = static_cast<int64_t>(s.B) * s.H * s.T;
   if (c.kind == SDM_VARIANT_PIPELINED)
-    return align256(static_cast<size_t>(n) * c.parts * sdm::pipe_layout(s.W, s.R).words * 4u);
+    return align256(static_cast<size_t>(n) * c.parts * sdm::pipe_layout(s.W, s.R).words * 4u) + y_other_bytes(s, c);
   return align256(static_cast<size_t>(n) * rec_layout(s.W, s.R).words * 4u);
 }
 // The same before a kernel is chosen (workspace queries): the chosen
@@ -447,10 +453,12 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
                       const void* M0_for_init = nullptr) {
   sdm_status_t r;
   if (c.kind == SDM_VARIANT_PIPELINED) {
-    // the parts add their read sums into y, which the record build zeroes first
-    float* y_zero = c.parts > 1 ? y : nullptr;
-    if ((r = launch_pipe_records(s, c, idx_w, w_w, idx_r, w_r, alpha, beta, rec, y_zero, dev, st)) != SDM_OK)
+    if ((r = launch_pipe_records(s, c, idx_w, w_w, idx_r, w_r, alpha, beta, rec, nullptr, dev, st)) != SDM_OK)
       return r;
+    // the second part's read sums go after the records; a separate pass adds them into y
+    const size_t y_other_off = records_bytes(s, c) - y_other_bytes(s, c);
+    float* y_other = c.parts > 1 ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(rec) + y_other_off)
+                                 : nullptr;
     tr.mark(2, st);
     if (init_before_scan && (r = launch_state_init(dev, s, M0_for_init, M, st)) != SDM_OK) return r;
     tr.mark(3, st);
@@ -464,8 +472,15 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
     a.v = v;
     a.M = M;
     a.y = y;
+    a.y_other = y_other;
     a.err = dev.err;
     if ((r = launch_pipe(c, s, a, st)) != SDM_OK) return r;
+    if (y_other != nullptr) {
+      const int64_t n4 = static_cast<int64_t>(s.B) * s.T * s.H * s.d_v / 4;
+      const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, static_cast<int64_t>(dev.sms) * 8));
+      sdm::k_add_f4<<<grid, 256, 0, st>>>(reinterpret_cast<float4*>(y), reinterpret_cast<const float4*>(y_other), n4);
+      if ((r = launch_status("part sum launch")) != SDM_OK) return r;
+    }
     tr.mark(4, st);
     if (g != nullptr && (r = launch_epilogue(dev, s, y, g, st)) != SDM_OK) return r;
     tr.mark(5, st);
@@ -1125,8 +1140,10 @@ int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate) 
     return -1;
   }
   g_last_error = saved;
-  // two selections, records, recurrence; the streaming recurrence also copies M0 first
-  return 4 + (c.resident ? 0 : 1) + (with_gate ? 1 : 0);
+  // two selections, records, recurrence; the streaming and pipelined recurrences also copy M0
+  // first; the pipelined one with two slot parts adds the second part's sums into y after
+  const int parts_sum = c.kind == SDM_VARIANT_PIPELINED && c.parts > 1 ? 1 : 0;
+  return 4 + (c.resident ? 0 : 1) + parts_sum + (with_gate ? 1 : 0);
 }
 
 sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,

@@ -16,6 +16,22 @@ static __global__ void __launch_bounds__(256) k_state_init(const uint4* __restri
     dst[i] = M0[i];
 }
 
+// y[i] += other[i] for n float4s: the read sums of the second slot part of the
+// pipelined recurrence added to the first part's.
+static __global__ void __launch_bounds__(256) k_add_f4(float4* __restrict__ y, const float4* __restrict__ other,
+                                                       int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 a = y[i];
+    const float4 b = other[i];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    y[i] = a;
+  }
+}
+
 // y <- g * y / sqrt(mean(y^2) + eps) over d_v for each token-head (SDM
 // explainer, section 3.1 step 3: RMS-Norm, then element-wise gating). One warp
 // per row; the sum of squares is reduced in a fixed order.

@@ -19,19 +19,24 @@
 // synchronisation; each adds its partial read sum into y (with two parts the
 // sum 0 + a + b does not depend on their order, so y stays reproducible).
 //
-// Within a CTA, for token t:
-//   * every thread first gathers its share of the rows of token t + P - 1
-//     (16-byte cp.async, completion counted on the stage's mbarrier), so the
-//     copies run P - 1 tokens ahead of their use;
+// Within a CTA, for token t, after the block barrier that ends token t - 1:
+//   * every thread gathers its share of the rows of token t + P - 2 (16-byte
+//     cp.async, one commit group per token) into the stage token t - 2 used,
+//     then waits for its own copies of token t; the copies run P - 2 tokens
+//     ahead of their use, and a second block barrier is not needed: the one
+//     that ends token t - 1 is also the one after which the rows of token t
+//     are complete (it is taken after every thread's wait);
 //   * write warps apply the write to the part's write entries (each lane owns
 //     one 16-byte unit of a row), store the rows to global memory and keep
 //     them in a ring of written-row stages;
 //   * read warps sum the part's read entries; lane bits above the unit index
-//     select entries, so a warp reduces its columns with shuffles alone and
-//     adds them to y;
-//   * one block barrier ends the token.
-// A row gathered early is stale when one of the P - 1 tokens in between
-// wrote it; the hazard plan in the records names that write (token t - k,
+//     select entries, so a warp reduces its columns with shuffles alone; part
+//     0 stores its sums to y, part 1 to a scratch copy that a separate pass
+//     adds into y (plain stores, no atomics);
+//   * one block barrier per token.
+// A row gathered early is stale when one of the P - 1 tokens before its use
+// wrote it (the gather of token u is issued while token u - P + 1 may still
+// be writing); the hazard plan in the records names that write (token t - k,
 // write entry j of this part) and the row is taken from the written-row ring
 // instead; a read of a slot written by the same token (k = 0) recomputes that
 // write from its source.
@@ -277,7 +282,8 @@ struct PipeArgs {
   const uint32_t* rec;  // [B, H, parts, T, pl.words]
   const void* v;        // [B, T, H, d_v] in dtype
   void* M;              // [B, H, N, d_v] state dtype, updated in place
-  float* y;             // [B, T, H, d_v]; with parts > 1 zero on entry
+  float* y;             // [B, T, H, d_v]: part 0's read sums
+  float* y_other;       // [B, T, H, d_v]: part 1's read sums (parts == 2), added into y afterwards
   unsigned* err;
 };
 
@@ -285,7 +291,7 @@ struct PipeArgs {
 __host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
                                                      int s_in) {
   return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(P) * Wp * C * s_state +
-         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in + (P + 2) * 8;
+         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in + 2 * 8;
 }
 
 // Sums a[0:VE) (the VE columns of one 16-byte unit, held by the lanes that
@@ -338,6 +344,7 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
   static_assert(U % NWR == 0 && kWarp % UR == 0, "read warps split the units evenly");
   static_assert(NT % U == 0, "gather lanes cover whole rows");
   static_assert(L >= P, "a chunk of records is staged before its tokens are gathered");
+  static_assert(P >= 3, "rows are gathered P - 2 >= 1 tokens ahead");
   extern __shared__ __align__(16) unsigned char smem[];
   const PipeLayout pl = a.pl;
   const int Wp = pl.Wp, E = pl.Wp + pl.Rp, words = pl.words, T = a.T;
@@ -345,8 +352,7 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
   unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [P][Wp][RS]
   uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(P) * Wp * RS);  // [2][L][words]
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
-  uint64_t* full = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);                 // [P]
-  uint64_t* cbar = full + P;                                                       // [2]
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);                 // [2]
 
   const int part = blockIdx.x % a.parts, bh = blockIdx.x / a.parts;
   const int b = bh / a.H, h = bh % a.H;
@@ -355,11 +361,11 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
   Tst* Mbh = static_cast<Tst*>(a.M) + static_cast<int64_t>(bh) * a.N * a.d_v + c0;
   const uint32_t* rec_g = a.rec + (static_cast<int64_t>(bh) * a.parts + part) * T * words;
   const int64_t tok_step = static_cast<int64_t>(a.H) * a.d_v;  // [B, T, H, d_v] rows of one (b, h)
-  float* y_bh = a.y + static_cast<int64_t>(b) * T * tok_step + static_cast<int64_t>(h) * a.d_v + c0;
+  float* y_bh = (part == 0 ? a.y : a.y_other) + static_cast<int64_t>(b) * T * tok_step +
+                static_cast<int64_t>(h) * a.d_v + c0;
   const Tin* v_bh = static_cast<const Tin*>(a.v) + static_cast<int64_t>(b) * T * tok_step + static_cast<int64_t>(h) * a.d_v + c0;
 
   if (tid == 0) {
-    for (int s = 0; s < P; ++s) mbar_init(&full[s], NT);
     mbar_init(&cbar[0], 1);
     mbar_init(&cbar[1], 1);
     fence_mbar_init();
@@ -384,8 +390,7 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
     return !__syncthreads_or(!ok);
   };
   // Token u's rows of this part into stage u % P (every thread its share, one
-  // 16-byte copy per row and unit); each thread then arrives on the stage's
-  // barrier, which completes once all copies have landed.
+  // 16-byte copy per row and unit), one commit group per call.
   auto gather = [&](int u) {
     const uint32_t* rec = rec_of(u);
     const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
       cp_async16(st + static_cast<size_t>(e) * RS, src + static_cast<int64_t>(slw[e]) * a.d_v);
     for (int e = tid / U; e < nr; e += NT / U)
       cp_async16(st + static_cast<size_t>(Wp + e) * RS, src + static_cast<int64_t>(slr[e]) * a.d_v);
-    cp_async_mbar_arrive(&full[u % P]);
+    cp_async_commit();
   };
   auto finish = [&]() {  // copies in flight land before the block exits
     cp_async_wait_all();
@@ -413,7 +418,10 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
     finish();
     return;
   }
-  for (int u = 0; u < P - 1 && u < T; ++u) gather(u);
+  for (int u = 0; u < P - 2; ++u) {
+    if (u < T) gather(u);
+    else cp_async_commit();
+  }
 
   const bool writer = warp < NWW;
   const int qw = lane % U;                              // write lanes: unit of every entry they take
@@ -421,16 +429,24 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
   const int q_mine = writer ? qw : qr;
 #pragma unroll 1
   for (int t = 0; t < T; ++t) {
-    const int u = t + P - 1;
+    // Token t - 2 finished before the last barrier, so its stage is free.
+    const int u = t + P - 2;
     if (u < T) {
       if (u % L == 0 && !chunk_ok(u / L)) {
         finish();
         return;
       }
       gather(u);
+    } else {
+      cp_async_commit();
     }
-    const bool ok = mbar_wait_bounded(&full[t % P], (t / P) & 1, a.err);
-    if (ok) {
+    cp_async_wait<P - 2>();  // this thread's copies of token t have landed
+    __syncthreads();         // ... and everyone's; token t - 1 is complete
+    if (tid == 0 && t > 0 && t % L == 0 && t / L + 1 < n_chunks) {
+      fence_proxy_async_smem();
+      load_chunk(t / L + 1);  // every token of chunk t/L - 1 is done: refill its buffer
+    }
+    {
       const uint32_t* rec = rec_of(t);
       const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
       const uint16_t* sw = reinterpret_cast<const uint16_t*>(rec + pl.off_src_w);
@@ -487,17 +503,8 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
           weighted_add<VE>(acc, m0, qw_r[i0]);
           weighted_add<VE>(acc, m1, has1 ? qw_r[i1] : 0.0f);
         }
-        reduce_put_unit<VE, UR>(acc, y_bh + static_cast<int64_t>(t) * tok_step + qr * VE, lane, a.parts > 1);
+        reduce_put_unit<VE, UR>(acc, y_bh + static_cast<int64_t>(t) * tok_step + qr * VE, lane, false);
       }
-    }
-    // token t done: its rows are in global memory and in the written-row ring
-    if (__syncthreads_or(!ok)) {
-      finish();
-      return;
-    }
-    if (tid == 0 && (t + 1) % L == 0 && (t + 1) / L + 1 < n_chunks) {
-      fence_proxy_async_smem();
-      load_chunk((t + 1) / L + 1);  // chunk (t+1)/L - 1 is consumed: refill its buffer
     }
   }
   finish();

@@ -71,12 +71,13 @@ def test_invalid_shapes_rejected_on_host(lib, bad):
 def test_workspace_sizes(lib):
     """Without a device the records workspace is the largest any recurrence
     kernel needs: the streaming kernel's records, or the pipelined kernel's,
-    one per slot part (two parts)."""
+    one per slot part (two parts), followed by the second part's read sums."""
     s = shape()
     rec_words = 4 + 4 + 4 + 4 + 8 // 2 + 4  # Wp, Wp, Rp, Rp, Fp/2, alpha/beta block
     # W, R rounded to 8: uint16 source rows, (a, c) pairs, read weights, slots, counts
     pipe_words = 8 // 2 + 8 // 2 + 2 * 8 + 8 + 8 + 8 + 4
-    rec = max((2 * 3 * 5 * rec_words * 4 + 255) // 256 * 256, (2 * 2 * 3 * 5 * pipe_words * 4 + 255) // 256 * 256)
+    a256 = lambda x: (x + 255) // 256 * 256
+    rec = max(a256(2 * 3 * 5 * rec_words * 4), a256(2 * 2 * 3 * 5 * pipe_words * 4) + a256(2 * 5 * 3 * 32 * 4))
     assert lib.sdm_scan_workspace_bytes(ctypes.byref(s)) == rec
     per = (2 * 5 * 3 * 4 * 4 + 255) // 256 * 256
     assert lib.sdm_layer_forward_workspace_bytes(ctypes.byref(s)) == 4 * per + rec
