@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -218,14 +219,14 @@ constexpr StreamCfg kStreamCfgs[] = {
 };
 
 // Instantiated pipelined tiles: state bytes, columns per CTA (128-byte row
-// segments), prefetch distance, staging chunk, write warps, read warps.
+// segments), stages, staging chunk, write warps, read warps, producer warps.
 struct PipeCfg {
   int state_bytes;
-  int C, P, L, NWW, NWR;
+  int C, P, L, NWW, NWR, NP;
 };
 constexpr PipeCfg kPipeCfgs[] = {
-    {2, 64, 6, 16, 4, 4}, {2, 64, 7, 16, 4, 4}, {2, 64, 6, 16, 8, 8}, {2, 64, 5, 16, 4, 4},
-    {4, 32, 6, 16, 4, 4}, {4, 32, 4, 16, 4, 4},
+    {2, 64, 6, 16, 4, 4, 4}, {2, 64, 6, 16, 4, 4, 2}, {2, 64, 7, 16, 4, 4, 4}, {2, 64, 5, 16, 4, 4, 4},
+    {4, 32, 6, 16, 4, 4, 4}, {4, 32, 4, 16, 4, 4, 4},
 };
 
 // Instantiated resident tiles: columns per warp, warps per CTA, staging
@@ -307,7 +308,10 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
   // each tile's slots over two CTAs doubles the SMs at work.
   const int c128 = 128 / s_state;
   const bool few_tiles = s.d_v % c128 == 0 && bh * (s.d_v / c128) < dev.sms;
-  if (s.variant == SDM_VARIANT_PIPELINED || (s.variant == SDM_VARIANT_AUTO && kPipelinedAuto && few_tiles)) {
+  const bool rows_fit = bh * slots_of(s.sqrt_n) <= INT_MAX;  // TMA row coordinates are int32
+  if (s.variant == SDM_VARIANT_PIPELINED && !rows_fit)
+    return fail(SDM_ERR_UNSUPPORTED, "the pipelined variant needs B*H*N below 2^31 state rows");
+  if (rows_fit && (s.variant == SDM_VARIANT_PIPELINED || (s.variant == SDM_VARIANT_AUTO && kPipelinedAuto && few_tiles))) {
     std::vector<PipeCfg> order;
     for (const PipeCfg& k : kPipeCfgs)
       if (k.state_bytes == s_state && s.d_v % k.C == 0 && pipelined_smem(s, k) <= lim) order.push_back(k);
@@ -320,6 +324,7 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
       c.L = k.L;
       c.NWW = k.NWW;
       c.NWR = k.NWR;
+      c.NP = k.NP;
       c.parts = bh * (s.d_v / k.C) * 2 <= dev.sms ? 2 : 1;
       c.smem = pipelined_smem(s, k);
       *out = c;
@@ -1016,8 +1021,8 @@ sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_l
   if (c.kind == SDM_VARIANT_RESIDENT)
     snprintf(out, out_len, "resident CW=%d NWARP=%d L=%d EB=%d smem=%zu", c.CW, c.NWARP, c.L, c.EB, c.smem);
   else if (c.kind == SDM_VARIANT_PIPELINED)
-    snprintf(out, out_len, "pipelined C=%d P=%d L=%d NWW=%d NWR=%d parts=%d smem=%zu", c.C, c.P, c.L, c.NWW, c.NWR,
-             c.parts, c.smem);
+    snprintf(out, out_len, "pipelined C=%d P=%d L=%d NWW=%d NWR=%d NP=%d parts=%d smem=%zu", c.C, c.P, c.L, c.NWW,
+             c.NWR, c.NP, c.parts, c.smem);
   else
     snprintf(out, out_len, "streaming C=%d P=%d L=%d NW=%d smem=%zu", c.C, c.P, c.L, c.NWARP, c.smem);
   return ok();

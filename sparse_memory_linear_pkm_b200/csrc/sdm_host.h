@@ -49,7 +49,7 @@ struct ScanChoice {
   int P = 4;
   int L = 16;
   int CW = 8, NWARP = 2, EB = 4;  // resident: columns per warp, warps per CTA, entry block
-  int NWW = 4, NWR = 2, parts = 1;  // pipelined: write warps, read warps, slot parts per column tile
+  int NWW = 4, NWR = 4, NP = 4, parts = 1;  // pipelined: write, read and producer warps, slot parts per tile
   size_t smem = 0;
 };
 

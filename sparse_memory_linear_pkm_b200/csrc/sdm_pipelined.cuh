@@ -19,13 +19,17 @@
 // synchronisation; each adds its partial read sum into y (with two parts the
 // sum 0 + a + b does not depend on their order, so y stays reproducible).
 //
-// Within a CTA, for token t, after the block barrier that ends token t - 1:
-//   * every thread gathers its share of the rows of token t + P - 2 (16-byte
-//     cp.async, one commit group per token) into the stage token t - 2 used,
-//     then waits for its own copies of token t; the copies run P - 2 tokens
-//     ahead of their use, and a second block barrier is not needed: the one
-//     that ends token t - 1 is also the one after which the rows of token t
-//     are complete (it is taken after every thread's wait);
+// Within a CTA, for token t, after the block barrier that ends token t - 2:
+//   * producer warps request the rows of token t + P - 2 with TMA row
+//     gathers (four 128-byte rows an instruction) into the stage token t - 2
+//     used, so the copies run P - 2 tokens ahead of their use. An SM takes
+//     one random 128-byte row per ~6-7 cycles however it is asked (TMA or
+//     cp.async, or both at once), and the issuing thread waits for the
+//     acceptance; with the requests in warps of their own, the consumer
+//     warps compute while the producers wait (measured: ~650 cycles a token
+//     of request issue that the compute otherwise waited for);
+//   * one lane per warp waits for token t's rows, and one block barrier,
+//     taken after those waits, also ends token t - 1;
 //   * write warps apply the write to the part's write entries (each lane owns
 //     one 16-byte unit of a row), store the rows to global memory and keep
 //     them in a ring of written-row stages;
@@ -34,18 +38,38 @@
 //     0 stores its sums to y, part 1 to a scratch copy that a separate pass
 //     adds into y (plain stores, no atomics);
 //   * one block barrier per token.
-// A row gathered early is stale when one of the P - 1 tokens before its use
-// wrote it (the gather of token u is issued while token u - P + 1 may still
-// be writing); the hazard plan in the records names that write (token t - k,
+// Write warps fence their global stores (fence.proxy.async.global) at the
+// top of the next token, before its barrier, so the TMA gathers issued after
+// that barrier read them. A row gathered early is stale when one of the P - 1
+// tokens before its use wrote it (the gather of token u is issued while
+// token u - P + 1 may still be writing); the hazard plan in the records names that write (token t - k,
 // write entry j of this part) and the row is taken from the written-row ring
 // instead; a read of a slot written by the same token (k = 0) recomputes that
 // write from its source.
 #pragma once
 
+#include <cuda.h>
+
 #include "sdm_device.cuh"
 #include "sdm_scan.cuh"
 
 namespace sdm {
+
+// Four rows of a 2-D tensor map (row coordinates r0..r3, column x) into
+// consecutive boxes at dst, completing on bar (TMA row gather, no multicast).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int r0, int r1, int r2, int r3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+// Orders this thread's earlier generic-proxy global writes before later
+// async-proxy (TMA) reads of the same memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;\n" ::: "memory");
+}
 
 // Per-token record of one part (32-bit words):
 //   uint16 src_w[Wp] | uint16 src_r[Rp] | float2 awcw[Wp] | f32 q_r[Rp] |
@@ -277,6 +301,7 @@ __global__ void __launch_bounds__(256) k_build_pipe_records(
 }
 
 struct PipeArgs {
+  CUtensorMap state_map;  // M as rows [B*H*N, d_v] of the state dtype, box C columns x 1 row
   int B, T, H, N, d_v, W, R, parts;
   PipeLayout pl;
   const uint32_t* rec;  // [B, H, parts, T, pl.words]
@@ -291,7 +316,7 @@ struct PipeArgs {
 __host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
                                                      int s_in) {
   return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(P) * Wp * C * s_state +
-         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in + 2 * 8;
+         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in + (P + 2) * 8 + 128;
 }
 
 // Sums a[0:VE) (the VE columns of one 16-byte unit, held by the lanes that
@@ -332,9 +357,9 @@ __device__ __forceinline__ void reduce_put_unit(float (&a)[VE], float* y, int la
   }
 }
 
-template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR>
-__global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeArgs a) {
-  constexpr int NT = (NWW + NWR) * kWarp;
+template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR, int NP>
+__global__ void __launch_bounds__((NP + NWW + NWR) * kWarp, 1) k_scan_pipelined(const __grid_constant__ PipeArgs a) {
+  constexpr int NT = (NP + NWW + NWR) * kWarp;
   constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
   constexpr int U = C / VE;             // units per row segment
   constexpr int RS = C * sizeof(Tst);   // bytes of a row segment
@@ -345,14 +370,17 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
   static_assert(NT % U == 0, "gather lanes cover whole rows");
   static_assert(L >= P, "a chunk of records is staged before its tokens are gathered");
   static_assert(P >= 3, "rows are gathered P - 2 >= 1 tokens ahead");
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  // TMA boxes land at 128-byte aligned rows
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const PipeLayout pl = a.pl;
   const int Wp = pl.Wp, E = pl.Wp + pl.Rp, words = pl.words, T = a.T;
   unsigned char* lstage = smem;                                                    // [P][E][RS]
   unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [P][Wp][RS]
   uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(P) * Wp * RS);  // [2][L][words]
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
-  uint64_t* cbar = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);                 // [2]
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);                 // [2] record chunks
+  uint64_t* full = cbar + 2;                                                       // [P] gathered stages
 
   const int part = blockIdx.x % a.parts, bh = blockIdx.x / a.parts;
   const int b = bh / a.H, h = bh % a.H;
@@ -366,6 +394,7 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
   const Tin* v_bh = static_cast<const Tin*>(a.v) + static_cast<int64_t>(b) * T * tok_step + static_cast<int64_t>(h) * a.d_v + c0;
 
   if (tid == 0) {
+    for (int st = 0; st < P; ++st) mbar_init(&full[st], 1);
     mbar_init(&cbar[0], 1);
     mbar_init(&cbar[1], 1);
     fence_mbar_init();
@@ -389,25 +418,33 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
     const bool ok = mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err);
     return !__syncthreads_or(!ok);
   };
-  // Token u's rows of this part into stage u % P (every thread its share, one
-  // 16-byte copy per row and unit), one commit group per call.
+  // Token u's rows of this part into stage u % P with TMA row gathers, four
+  // rows an instruction (padding rows of a partial group read a neighbour row
+  // or the zero fill; they are never used), issued by the producer warps'
+  // lanes; thread 0 arms the stage's barrier with the token's bytes.
   auto gather = [&](int u) {
     const uint32_t* rec = rec_of(u);
     const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
-    unsigned char* st = lstage + static_cast<size_t>(u % P) * E * RS + (tid % U) * 16;
-    const Tst* src = Mbh + (tid % U) * VE;
-    const uint32_t* slw = rec + pl.off_slot_w;
-    const uint32_t* slr = rec + pl.off_slot_r;
-    for (int e = tid / U; e < nw; e += NT / U)
-      cp_async16(st + static_cast<size_t>(e) * RS, src + static_cast<int64_t>(slw[e]) * a.d_v);
-    for (int e = tid / U; e < nr; e += NT / U)
-      cp_async16(st + static_cast<size_t>(Wp + e) * RS, src + static_cast<int64_t>(slr[e]) * a.d_v);
-    cp_async_commit();
+    const int gw = (nw + 3) / 4, gr = (nr + 3) / 4;
+    uint64_t* bar = &full[u % P];
+    if (tid == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(gw + gr) * 4u * RS);
+    unsigned char* st = lstage + static_cast<size_t>(u % P) * E * RS;
+    const int row0 = bh * a.N;
+    for (int g = warp + NP * lane; g < gw + gr; g += NP * kWarp) {
+      const bool wr = g < gw;
+      const int e = wr ? 4 * g : 4 * (g - gw);
+      const uint4 sl = *reinterpret_cast<const uint4*>(rec + (wr ? pl.off_slot_w : pl.off_slot_r) + e);
+      tma_gather4(st + static_cast<size_t>(wr ? e : Wp + e) * RS, &a.state_map, c0, row0 + static_cast<int>(sl.x),
+                  row0 + static_cast<int>(sl.y), row0 + static_cast<int>(sl.z), row0 + static_cast<int>(sl.w), bar);
+    }
   };
+  int last_gathered = -1;  // the last token whose rows were requested
   auto finish = [&]() {  // copies in flight land before the block exits
-    cp_async_wait_all();
-    if (tid == 0)
+    if (tid == 0) {
       for (int c = max(0, last_chunk - 1); c <= last_chunk; ++c) mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err);
+      for (int u = max(0, last_gathered - P + 1); u <= last_gathered; ++u)
+        mbar_wait_bounded(&full[u % P], (u / P) & 1, a.err);
+    }
   };
 
   if (tid == 0) {
@@ -418,35 +455,45 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
     finish();
     return;
   }
-  for (int u = 0; u < P - 2; ++u) {
-    if (u < T) gather(u);
-    else cp_async_commit();
+  const bool producer = warp < NP;
+  const bool writer = !producer && warp < NP + NWW;
+  const int cw = warp - NP;                             // consumer warp index: writers, then readers
+  const int qw = lane % U;                              // write lanes: unit of every entry they take
+  const int qr = (cw - NWW) * UR + lane % UR;           // read lanes: unit, entries lane / UR + k GR
+  const int q_mine = writer ? qw : qr;
+  for (int u = 0; u < P - 2 && u < T; ++u) {
+    if (producer) gather(u);
+    last_gathered = u;
   }
 
-  const bool writer = warp < NWW;
-  const int qw = lane % U;                              // write lanes: unit of every entry they take
-  const int qr = (warp - NWW) * UR + lane % UR;         // read lanes: unit, entries lane / UR + k GR
-  const int q_mine = writer ? qw : qr;
 #pragma unroll 1
   for (int t = 0; t < T; ++t) {
-    // Token t - 2 finished before the last barrier, so its stage is free.
+    // The state rows this thread stored for token t - 1 become visible to
+    // the gathers (async proxy) issued after the next barrier.
+    if (writer) fence_proxy_async_global();
+    // Token t - 2 finished before the last barrier, so its stage is free, and
+    // its stores were fenced before that barrier.
     const int u = t + P - 2;
     if (u < T) {
       if (u % L == 0 && !chunk_ok(u / L)) {
         finish();
         return;
       }
-      gather(u);
-    } else {
-      cp_async_commit();
+      if (producer) gather(u);
+      last_gathered = u;
     }
-    cp_async_wait<P - 2>();  // this thread's copies of token t have landed
-    __syncthreads();         // ... and everyone's; token t - 1 is complete
+    // token t's rows have landed (one waiting lane per consumer warp)
+    bool ok = true;
+    if (!producer && lane == 0) ok = mbar_wait_bounded(&full[t % P], (t / P) & 1, a.err);
+    if (__syncthreads_or(!ok)) {  // ... token t - 1 is complete
+      finish();
+      return;
+    }
     if (tid == 0 && t > 0 && t % L == 0 && t / L + 1 < n_chunks) {
       fence_proxy_async_smem();
       load_chunk(t / L + 1);  // every token of chunk t/L - 1 is done: refill its buffer
     }
-    {
+    if (!producer) {
       const uint32_t* rec = rec_of(t);
       const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
       const uint16_t* sw = reinterpret_cast<const uint16_t*>(rec + pl.off_src_w);
@@ -464,7 +511,7 @@ __global__ void __launch_bounds__((NWW + NWR) * kWarp, 1) k_scan_pipelined(PipeA
         const uint32_t* slw = rec + pl.off_slot_w;
         const int n = nw * U;
         // two independent units per iteration
-        for (int p0 = warp * kWarp + lane; p0 < n; p0 += 2 * NWW * kWarp) {
+        for (int p0 = cw * kWarp + lane; p0 < n; p0 += 2 * NWW * kWarp) {
           const int p1 = p0 + NWW * kWarp;
           const bool has1 = p1 < n;
           const int j0 = p0 / U, j1 = has1 ? p1 / U : j0;

@@ -1,6 +1,8 @@
 // Launches of the pipelined recurrence and of its record build.
 
 #include <algorithm>
+#include <climits>
+#include <mutex>
 
 #include "sdm_host.h"
 
@@ -24,26 +26,60 @@ sdm_status_t launch_pipe_records_typed(const sdm_shape_t& s, const ScanChoice& c
   return launch_status("pipelined record build launch");
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once (no link against libcuda).
+EncodeTiledFn encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
 template <typename Tin, typename Tst>
 sdm_status_t launch_pipe_typed(const ScanChoice& c, const sdm::PipeArgs& a, cudaStream_t st) {
   const dim3 grid(a.B * a.H * a.parts, a.d_v / c.C);
   void (*kern)(sdm::PipeArgs) = nullptr;
-#define SDM_PIPE(C_, P_, L_, NWW_, NWR_)                                                       \
-  if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_)                  \
-    kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_>;
+#define SDM_PIPE(C_, P_, L_, NWW_, NWR_, NP_)                                                  \
+  if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_ && c.NP == NP_)      \
+    kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_, NP_>;
   if constexpr (sizeof(Tst) == 2) {
-    SDM_PIPE(64, 6, 16, 4, 4) SDM_PIPE(64, 7, 16, 4, 4) SDM_PIPE(64, 6, 16, 8, 8) SDM_PIPE(64, 5, 16, 4, 4)
+    SDM_PIPE(64, 6, 16, 4, 4, 4) SDM_PIPE(64, 6, 16, 4, 4, 2) SDM_PIPE(64, 7, 16, 4, 4, 4) SDM_PIPE(64, 5, 16, 4, 4, 4)
   } else {
-    SDM_PIPE(32, 6, 16, 4, 4) SDM_PIPE(32, 4, 16, 4, 4)
+    SDM_PIPE(32, 6, 16, 4, 4, 4) SDM_PIPE(32, 4, 16, 4, 4, 4)
   }
 #undef SDM_PIPE
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no pipelined kernel for the chosen tile");
   set_smem(reinterpret_cast<const void*>(kern), c.smem);
-  kern<<<grid, (c.NWW + c.NWR) * 32, c.smem, st>>>(a);
+  kern<<<grid, (c.NP + c.NWW + c.NWR) * 32, c.smem, st>>>(a);
   return launch_status("pipelined scan launch");
 }
 
-sdm_status_t launch_pipe(const ScanChoice& c, const sdm_shape_t& s, const sdm::PipeArgs& a, cudaStream_t st) {
+sdm_status_t launch_pipe(const ScanChoice& c, const sdm_shape_t& s, const sdm::PipeArgs& args, cudaStream_t st) {
+  // The state as a 2-D tensor of B*H*N rows of d_v values; one box is one
+  // C-column segment of one row (the unit the TMA row gathers fetch).
+  sdm::PipeArgs a = args;
+  const uint64_t rows = static_cast<uint64_t>(a.B) * a.H * a.N;
+  if (rows > static_cast<uint64_t>(INT_MAX)) return fail(SDM_ERR_UNSUPPORTED, "B*H*N above 2^31 - 1 state rows");
+  const EncodeTiledFn encode = encode_tiled();
+  if (encode == nullptr) return fail(SDM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.d_v), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.d_v) * in_size(s.state_dtype)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(c.C), 1u}, estride[2] = {1u, 1u};
+  const CUresult e = encode(&a.state_map, s.state_dtype == SDM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                            2, a.M, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (e != CUDA_SUCCESS) return fail(SDM_ERR_CUDA, "cuTensorMapEncodeTiled failed with " + std::to_string(e));
   if (s.in_dtype == SDM_BF16)
     return s.state_dtype == SDM_BF16 ? launch_pipe_typed<bf16, bf16>(c, a, st) : launch_pipe_typed<bf16, float>(c, a, st);
   return s.state_dtype == SDM_BF16 ? launch_pipe_typed<float, bf16>(c, a, st) : launch_pipe_typed<float, float>(c, a, st);
