@@ -543,6 +543,9 @@ def measure_workload(name: str, args, dev, steps: int = 5, warmup: int = 3) -> d
     ws = torch.empty(sdm.layer_forward_workspace_bytes(sh), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for row in ev:  # create the events before the timed region
+        for e in row:
+            e.record(stream)
 
     def step(events=None):
         sdm.layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], inp["M0"], shape.W, shape.R,

@@ -109,6 +109,34 @@ __host__ __device__ inline PipeLayout pipe_layout(int W, int R) {
 
 constexpr uint32_t kSrcSameToken = 0x8000u;  // src_r flag: recompute this token's write (low bits: j)
 
+// 16 bytes of state (8 bf16 or 4 fp32 values) as fp32, by bit operations.
+template <typename Tst>
+__device__ __forceinline__ void unpack_unit(const uint4& u, float* m) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  if constexpr (sizeof(Tst) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m[2 * i] = __uint_as_float(w[i] << 16);
+      m[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = __uint_as_float(w[i]);
+  }
+}
+// m <- a m + c v on VE values (scalar fp32 operations: the same roundings as
+// the paired ones of the other recurrence kernels).
+template <int VE>
+__device__ __forceinline__ void write_unit(float* m, const float* v, float a, float c) {
+#pragma unroll
+  for (int j = 0; j < VE; ++j) m[j] = fmaf(a, m[j], __fmul_rn(c, v[j]));
+}
+template <int VE>
+__device__ __forceinline__ void read_unit(float* acc, const float* m, float q) {
+#pragma unroll
+  for (int j = 0; j < VE; ++j) acc[j] = fmaf(q, m[j], acc[j]);
+}
+
 // Part of a slot: a hash bit, so that structured selections (e.g. slots that
 // share a grid column) still spread over both parts.
 __device__ __forceinline__ int slot_part(uint32_t slot, int parts) {
@@ -314,62 +342,50 @@ struct PipeArgs {
 
 // Shared-memory bytes of k_scan_pipelined (host and device agree on this).
 __host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
-                                                     int s_in) {
+                                                     int s_in, int NWR) {
   return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(P) * Wp * C * s_state +
-         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in + (P + 2) * 8 + 128;
+         static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in +
+         static_cast<size_t>(2) * NWR * C * 4 + (2 * P + 2) * 8 + 128;
 }
 
-// Sums a[0:VE) (the VE columns of one 16-byte unit, held by the lanes that
-// share lane % UR) over the 32 / UR entry groups of the warp in a fixed
-// order, then stores the column sums to y[0:VE), or adds them there when
-// several parts contribute.
-template <int VE, int UR>
-__device__ __forceinline__ void reduce_put_unit(float (&a)[VE], float* y, int lane, bool add) {
-  int n = VE, off = 0, bmask = 0;
+// Sums a[0:VE) (the VE columns of one 16-byte unit) over the lanes that
+// share lane % U, in a fixed butterfly order that halves the values each
+// level; returns the offset of the VE * U / 32 column sums the lane keeps in
+// a[0 : VE * U / 32).
+template <int VE, int U>
+__device__ __forceinline__ int reduce_scatter_entries(float (&a)[VE], int lane) {
+  static_assert((VE * U) % kWarp == 0, "every lane keeps at least one column");
+  int off = 0;
+  int n = VE;
 #pragma unroll
-  for (int o = 16; o >= UR; o >>= 1) {
-    if (n > 1) {
-      const bool hi = lane & o;
-      const int h = n / 2;
+  for (int o = kWarp / 2; o >= U; o >>= 1) {
+    const bool hi = lane & o;
+    const int h = n / 2;
 #pragma unroll
-      for (int j = 0; j < VE / 2; ++j) {
-        if (j < h) {
-          const float keep = hi ? a[j + h] : a[j];
-          const float send = hi ? a[j] : a[j + h];
-          a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      off += hi ? h : 0;
-      n = h;
-    } else {
-      a[0] += __shfl_xor_sync(0xffffffffu, a[0], o);
-      bmask |= o;
-    }
-  }
-  if ((lane & bmask) == 0) {
-#pragma unroll
-    for (int j = 0; j < VE; ++j) {
-      if (j < n) {
-        if (add) atomicAdd(y + off + j, a[j]);
-        else y[off + j] = a[j];
+    for (int j = 0; j < VE / 2; ++j) {
+      if (j < h) {
+        const float keep = hi ? a[j + h] : a[j];
+        const float send = hi ? a[j] : a[j + h];
+        a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
     }
+    off += hi ? h : 0;
+    n = h;
   }
+  return off;
 }
 
 template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR, int NP>
-__global__ void __launch_bounds__((NP + NWW + NWR) * kWarp, 1) k_scan_pipelined(const __grid_constant__ PipeArgs a) {
-  constexpr int NT = (NP + NWW + NWR) * kWarp;
+__global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipelined(const __grid_constant__ PipeArgs a) {
+  constexpr int NT = (NP + 1 + NWW + NWR) * kWarp;
   constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
   constexpr int U = C / VE;             // units per row segment
   constexpr int RS = C * sizeof(Tst);   // bytes of a row segment
-  constexpr int UR = U / NWR;           // units per read warp
-  constexpr int GR = kWarp / UR;        // read entries per read-warp instruction
+  constexpr int G = kWarp / U;          // entries per consumer-warp instruction
   static_assert(U >= 1 && U <= kWarp && kWarp % U == 0, "a row segment spans a divisor of the warp");
-  static_assert(U % NWR == 0 && kWarp % UR == 0, "read warps split the units evenly");
   static_assert(NT % U == 0, "gather lanes cover whole rows");
   static_assert(L >= P, "a chunk of records is staged before its tokens are gathered");
-  static_assert(P >= 3, "rows are gathered P - 2 >= 1 tokens ahead");
+  static_assert(P >= 3, "rows are gathered P - 1 >= 2 tokens ahead");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // TMA boxes land at 128-byte aligned rows
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -379,8 +395,10 @@ __global__ void __launch_bounds__((NP + NWW + NWR) * kWarp, 1) k_scan_pipelined(
   unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [P][Wp][RS]
   uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(P) * Wp * RS);  // [2][L][words]
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
-  uint64_t* cbar = reinterpret_cast<uint64_t*>(vbuf + 2 * L * C);                 // [2] record chunks
+  float* ybuf = reinterpret_cast<float*>(vbuf + 2 * L * C);                        // [2][NWR][C] read partials
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(ybuf + 2 * NWR * C);               // [2] record chunks
   uint64_t* full = cbar + 2;                                                       // [P] gathered stages
+  uint64_t* done = full + P;  // [P] the consumers are through with a token, its stores fenced
 
   const int part = blockIdx.x % a.parts, bh = blockIdx.x / a.parts;
   const int b = bh / a.H, h = bh % a.H;
@@ -394,7 +412,10 @@ __global__ void __launch_bounds__((NP + NWW + NWR) * kWarp, 1) k_scan_pipelined(
   const Tin* v_bh = static_cast<const Tin*>(a.v) + static_cast<int64_t>(b) * T * tok_step + static_cast<int64_t>(h) * a.d_v + c0;
 
   if (tid == 0) {
-    for (int st = 0; st < P; ++st) mbar_init(&full[st], 1);
+    for (int st = 0; st < P; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&done[st], 1);
+    }
     mbar_init(&cbar[0], 1);
     mbar_init(&cbar[1], 1);
     fence_mbar_init();
@@ -414,10 +435,7 @@ __global__ void __launch_bounds__((NP + NWW + NWR) * kWarp, 1) k_scan_pipelined(
     last_chunk = c;
   };
   auto rec_of = [&](int t) { return recbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * words; };
-  auto chunk_ok = [&](int c) {
-    const bool ok = mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err);
-    return !__syncthreads_or(!ok);
-  };
+  auto chunk_wait = [&](int c) { return mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err); };
   // Token u's rows of this part into stage u % P with TMA row gathers, four
   // rows an instruction (padding rows of a partial group read a neighbour row
   // or the zero fill; they are never used), issued by the producer warps'
@@ -438,123 +456,162 @@ __global__ void __launch_bounds__((NP + NWW + NWR) * kWarp, 1) k_scan_pipelined(
                   row0 + static_cast<int>(sl.y), row0 + static_cast<int>(sl.z), row0 + static_cast<int>(sl.w), bar);
     }
   };
-  int last_gathered = -1;  // the last token whose rows were requested
-  auto finish = [&]() {  // copies in flight land before the block exits
-    if (tid == 0) {
+  int last_gathered = -1;  // producer threads: the last token whose rows they requested
+  auto finish = [&]() {  // a producer's copies in flight land before it exits
+    if (tid == 0)
       for (int c = max(0, last_chunk - 1); c <= last_chunk; ++c) mbar_wait_bounded(&cbar[c & 1], (c >> 1) & 1, a.err);
-      for (int u = max(0, last_gathered - P + 1); u <= last_gathered; ++u)
-        mbar_wait_bounded(&full[u % P], (u / P) & 1, a.err);
+    for (int u = max(0, last_gathered - P + 1); u <= last_gathered; ++u)
+      mbar_wait_bounded(&full[u % P], (u / P) & 1, a.err);
+  };
+
+  // Warp roles: NP producers (row gathers, record chunks), one control warp,
+  // NWW writers, NWR readers. The control warp and the consumers (writers and
+  // readers) meet at one barrier per token; the control warp does all the
+  // waiting on copies and signalling, so that the consumers' chain from one
+  // barrier to the next holds only their own loads, arithmetic and stores.
+  // The producers run up to P - 1 tokens ahead, paced by mbarriers.
+  const bool producer = warp < NP;
+  const bool control = warp == NP;
+  const bool writer = warp > NP && warp <= NP + NWW;
+  const int cw = warp - NP - 1;  // consumer warp index: writers, then readers
+  // Consumer lanes take unit lane % U of entries lane / U + k G: one warp
+  // instruction covers every unit of G rows, all 32 banks.
+  const int qw = lane % U;
+  constexpr int stride_w = NWW * kWarp;  // write units per pass of the write warps
+  constexpr int stride_r = G * NWR;      // read entries per pass of the read warps
+  const int base_w = cw * kWarp + lane;
+  const int base_r = (cw - NWW) * G + lane / U;
+  auto row_at = [&](uint32_t src) { return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(src) * RS + qw * 16); };
+  // Token t on this consumer thread. Every row it reads is complete: the
+  // token's gathered stage and the written stages of the tokens before it.
+  auto compute = [&](int t) {
+    const uint32_t* rec = rec_of(t);
+    const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
+    const uint16_t* sw = reinterpret_cast<const uint16_t*>(rec + pl.off_src_w);
+    const float2* ac = reinterpret_cast<const float2*>(rec + pl.off_awcw);
+    float vv[VE];
+    load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * C + qw * VE, vv);
+    // the write of entry j on this thread's unit of its source row (fp32 math, state rounding by the caller)
+    auto written = [&](int j, float (&m)[VE]) {
+      unpack_unit<Tst>(row_at(sw[j]), m);
+      const float2 c = ac[j];
+      write_unit<VE>(m, vv, c.x, c.y);
+    };
+    if (writer) {
+      unsigned char* ws = wstage + static_cast<size_t>(t % P) * Wp * RS + qw * 16;
+      Tst* Mq = Mbh + qw * VE;
+      const uint32_t* slw = rec + pl.off_slot_w;
+      const int n = nw * U;
+      for (int p0 = base_w; p0 < n; p0 += 2 * stride_w) {  // two independent units per pass
+        const int p1 = p0 + stride_w;
+        const bool has1 = p1 < n;
+        const int j0 = p0 / U, j1 = has1 ? p1 / U : j0;
+        float m0[VE], m1[VE];
+        written(j0, m0);
+        written(j1, m1);
+        const uint4 k0 = pack16<Tst>(m0), k1 = pack16<Tst>(m1);
+        *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j0) * RS) = k0;
+        *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slw[j0]) * a.d_v) = k0;
+        if (has1) {
+          *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j1) * RS) = k1;
+          *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slw[j1]) * a.d_v) = k1;
+        }
+      }
+    } else {
+      const uint16_t* sr = reinterpret_cast<const uint16_t*>(rec + pl.off_src_r);
+      const float* qr = reinterpret_cast<const float*>(rec + pl.off_q_r);
+      auto read_row = [&](int i, float (&m)[VE]) {
+        const uint32_t src = sr[i];
+        if (src & kSrcSameToken) {  // written by this token: that write, rounded as stored
+          written(static_cast<int>(src & 0x7FFFu), m);
+          unpack_unit<Tst>(pack16<Tst>(m), m);
+        } else {
+          unpack_unit<Tst>(row_at(src), m);
+        }
+      };
+      float acc[VE];
+#pragma unroll
+      for (int j = 0; j < VE; ++j) acc[j] = 0.f;
+      for (int i0 = base_r; i0 < nr; i0 += 2 * stride_r) {
+        const int i1 = i0 + stride_r;
+        const bool has1 = i1 < nr;
+        float m0[VE], m1[VE];
+        read_row(i0, m0);
+        read_row(has1 ? i1 : i0, m1);
+        read_unit<VE>(acc, m0, qr[i0]);
+        read_unit<VE>(acc, m1, has1 ? qr[i1] : 0.0f);
+      }
+      const int off = reduce_scatter_entries<VE, U>(acc, lane);
+      float* yb = ybuf + (static_cast<size_t>(t & 1) * NWR + (cw - NWW)) * C + qw * VE + off;
+#pragma unroll
+      for (int j = 0; j < VE * U / kWarp; ++j) yb[j] = acc[j];
     }
   };
 
-  if (tid == 0) {
-    load_chunk(0);
-    if (n_chunks > 1) load_chunk(1);
-  }
-  if (!chunk_ok(0)) {
+  if (producer) {
+    if (tid == 0) {
+      load_chunk(0);
+      if (n_chunks > 1) load_chunk(1);
+    }
+#pragma unroll 1
+    for (int u = 0; u < T; ++u) {
+      // Stage u % P held token u - P: the consumers are through with it, and
+      // the writes of every token up to u - P were fenced (the hazard plan
+      // forwards rows written by tokens u - P + 1 .. u - 1 from shared memory).
+      bool ok = u < P || mbar_wait_backoff(&done[(u - P) % P], ((u - P) / P) & 1, a.err);
+      if (ok && u % L == 0) ok = chunk_wait(u / L);
+      if (!ok) break;
+      const int c = u / L;
+      if (tid == 0 && u % L == P - 1 && c >= 1 && c + 1 < n_chunks) {
+        fence_proxy_async_smem();
+        load_chunk(c + 1);  // the consumers are through with chunk c - 1 (token cL - 1 is done)
+      }
+      gather(u);
+      last_gathered = u;
+    }
     finish();
     return;
   }
-  const bool producer = warp < NP;
-  const bool writer = !producer && warp < NP + NWW;
-  const int cw = warp - NP;                             // consumer warp index: writers, then readers
-  const int qw = lane % U;                              // write lanes: unit of every entry they take
-  const int qr = (cw - NWW) * UR + lane % UR;           // read lanes: unit, entries lane / UR + k GR
-  const int q_mine = writer ? qw : qr;
-  for (int u = 0; u < P - 2 && u < T; ++u) {
-    if (producer) gather(u);
-    last_gathered = u;
+  constexpr int kBarThreads = (1 + NWW + NWR) * kWarp;  // the control warp and the consumers
+  if (control) {
+    // y of token s: the read warps' column sums, added in warp order
+    auto put_y = [&](int s) {
+      const float* yb = ybuf + static_cast<size_t>(s & 1) * NWR * C;
+      for (int c = lane; c < C; c += kWarp) {
+        float acc = yb[c];
+#pragma unroll
+        for (int r = 1; r < NWR; ++r) acc += yb[r * C + c];
+        y_bh[static_cast<int64_t>(s) * tok_step + c] = acc;
+      }
+    };
+    bool ok = chunk_wait(0) && mbar_wait_bounded(&full[0], 0, a.err);
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+      if (named_barrier_or(1, kBarThreads, !ok)) return;  // token t - 1 is complete, token t's rows have landed
+      if (t > 0) {
+        put_y(t - 1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&done[(t - 1) % P]);
+      }
+      if (t + 1 < T) {
+        const int s = t + 1;
+        if (s % L == 0) ok = chunk_wait(s / L);
+        if (ok) ok = mbar_wait_bounded(&full[s % P], (s / P) & 1, a.err);
+      }
+    }
+    if (!named_barrier_or(1, kBarThreads, !ok)) put_y(T - 1);
+    return;
   }
-
+  // consumers
 #pragma unroll 1
   for (int t = 0; t < T; ++t) {
-    // The state rows this thread stored for token t - 1 become visible to
-    // the gathers (async proxy) issued after the next barrier.
-    if (writer) fence_proxy_async_global();
-    // Token t - 2 finished before the last barrier, so its stage is free, and
-    // its stores were fenced before that barrier.
-    const int u = t + P - 2;
-    if (u < T) {
-      if (u % L == 0 && !chunk_ok(u / L)) {
-        finish();
-        return;
-      }
-      if (producer) gather(u);
-      last_gathered = u;
-    }
-    // token t's rows have landed (one waiting lane per consumer warp)
-    bool ok = true;
-    if (!producer && lane == 0) ok = mbar_wait_bounded(&full[t % P], (t / P) & 1, a.err);
-    if (__syncthreads_or(!ok)) {  // ... token t - 1 is complete
-      finish();
-      return;
-    }
-    if (tid == 0 && t > 0 && t % L == 0 && t / L + 1 < n_chunks) {
-      fence_proxy_async_smem();
-      load_chunk(t / L + 1);  // every token of chunk t/L - 1 is done: refill its buffer
-    }
-    if (!producer) {
-      const uint32_t* rec = rec_of(t);
-      const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
-      const uint16_t* sw = reinterpret_cast<const uint16_t*>(rec + pl.off_src_w);
-      const float2* ac = reinterpret_cast<const float2*>(rec + pl.off_awcw);
-      float vv[VE];
-      load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * C + q_mine * VE, vv);
-      // the write of entry j on the 16-byte unit q of its source row (fp32 math, state rounding by the caller)
-      auto written = [&](int j, int q, float (&m)[VE]) {
-        unpack16<Tst>(*reinterpret_cast<const uint4*>(smem + static_cast<size_t>(sw[j]) * RS + q * 16), m);
-        const float2 c = ac[j];
-        delta_update<VE>(m, vv, c.x, c.y);
-      };
-      if (writer) {
-        unsigned char* ws = wstage + static_cast<size_t>(t % P) * Wp * RS + qw * 16;
-        const uint32_t* slw = rec + pl.off_slot_w;
-        const int n = nw * U;
-        // two independent units per iteration
-        for (int p0 = cw * kWarp + lane; p0 < n; p0 += 2 * NWW * kWarp) {
-          const int p1 = p0 + NWW * kWarp;
-          const bool has1 = p1 < n;
-          const int j0 = p0 / U, j1 = has1 ? p1 / U : j0;
-          float m0[VE], m1[VE];
-          written(j0, qw, m0);
-          written(j1, qw, m1);
-          const uint4 k0 = pack16<Tst>(m0), k1 = pack16<Tst>(m1);
-          *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j0) * RS) = k0;
-          *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slw[j0]) * a.d_v + qw * VE) = k0;
-          if (has1) {
-            *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j1) * RS) = k1;
-            *reinterpret_cast<uint4*>(Mbh + static_cast<int64_t>(slw[j1]) * a.d_v + qw * VE) = k1;
-          }
-        }
-      } else {
-        const uint16_t* sr = reinterpret_cast<const uint16_t*>(rec + pl.off_src_r);
-        const float* qw_r = reinterpret_cast<const float*>(rec + pl.off_q_r);
-        auto read_row = [&](int i, float (&m)[VE]) {
-          const uint32_t src = sr[i];
-          if (src & kSrcSameToken) {  // written by this token: that write, rounded as stored
-            written(static_cast<int>(src & 0x7FFFu), qr, m);
-            unpack16<Tst>(pack16<Tst>(m), m);
-          } else {
-            unpack16<Tst>(*reinterpret_cast<const uint4*>(smem + static_cast<size_t>(src) * RS + qr * 16), m);
-          }
-        };
-        float acc[VE];
-#pragma unroll
-        for (int j = 0; j < VE; ++j) acc[j] = 0.f;
-        for (int i0 = lane / UR; i0 < nr; i0 += 2 * GR) {
-          const int i1 = i0 + GR;
-          const bool has1 = i1 < nr;
-          float m0[VE], m1[VE];
-          read_row(i0, m0);
-          read_row(has1 ? i1 : i0, m1);
-          weighted_add<VE>(acc, m0, qw_r[i0]);
-          weighted_add<VE>(acc, m1, has1 ? qw_r[i1] : 0.0f);
-        }
-        reduce_put_unit<VE, UR>(acc, y_bh + static_cast<int64_t>(t) * tok_step + qr * VE, lane, false);
-      }
-    }
+    // the state rows this thread stored for token t - 1 become visible to the
+    // gathers that the producers issue after the control warp's signal
+    if (writer && t > 0) fence_proxy_async_global();
+    if (named_barrier_or(1, kBarThreads, false)) return;
+    compute(t);
   }
-  finish();
+  named_barrier_or(1, kBarThreads, false);
 }
 
 }  // namespace sdm
