@@ -225,8 +225,8 @@ struct PipeCfg {
   int C, P, L, NWW, NWR, NP;
 };
 constexpr PipeCfg kPipeCfgs[] = {
-    {2, 64, 6, 16, 4, 4, 4}, {2, 64, 6, 16, 4, 4, 2}, {2, 64, 7, 16, 4, 4, 4}, {2, 64, 5, 16, 4, 4, 4},
-    {4, 32, 6, 16, 4, 4, 4}, {4, 32, 4, 16, 4, 4, 4},
+    {2, 64, 6, 16, 4, 3, 4}, {2, 64, 6, 16, 4, 4, 4}, {2, 64, 6, 16, 3, 4, 4}, {2, 64, 7, 16, 4, 3, 4},
+    {2, 64, 6, 16, 4, 3, 2}, {4, 32, 6, 16, 4, 3, 4}, {4, 32, 4, 16, 4, 3, 4},
 };
 
 // Instantiated resident tiles: columns per warp, warps per CTA, staging

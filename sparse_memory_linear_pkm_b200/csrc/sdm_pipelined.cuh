@@ -124,17 +124,28 @@ __device__ __forceinline__ void unpack_unit(const uint4& u, float* m) {
     for (int i = 0; i < 4; ++i) m[i] = __uint_as_float(w[i]);
   }
 }
-// m <- a m + c v on VE values (scalar fp32 operations: the same roundings as
-// the paired ones of the other recurrence kernels).
+// m <- a m + c v on VE values, two lanes of fp32 per instruction (per element
+// the same roundings as the other recurrence kernels: a product, then a fused
+// multiply-add).
 template <int VE>
 __device__ __forceinline__ void write_unit(float* m, const float* v, float a, float c) {
+  const float2 a2 = make_float2(a, a), c2 = make_float2(c, c);
 #pragma unroll
-  for (int j = 0; j < VE; ++j) m[j] = fmaf(a, m[j], __fmul_rn(c, v[j]));
+  for (int j = 0; j < VE; j += 2) {
+    const float2 r = __ffma2_rn(a2, make_float2(m[j], m[j + 1]), __fmul2_rn(c2, make_float2(v[j], v[j + 1])));
+    m[j] = r.x;
+    m[j + 1] = r.y;
+  }
 }
 template <int VE>
 __device__ __forceinline__ void read_unit(float* acc, const float* m, float q) {
+  const float2 q2 = make_float2(q, q);
 #pragma unroll
-  for (int j = 0; j < VE; ++j) acc[j] = fmaf(q, m[j], acc[j]);
+  for (int j = 0; j < VE; j += 2) {
+    const float2 r = __ffma2_rn(q2, make_float2(m[j], m[j + 1]), make_float2(acc[j], acc[j + 1]));
+    acc[j] = r.x;
+    acc[j + 1] = r.y;
+  }
 }
 
 // Part of a slot: a hash bit, so that structured selections (e.g. slots that

@@ -52,9 +52,10 @@ sdm_status_t launch_pipe_typed(const ScanChoice& c, const sdm::PipeArgs& a, cuda
   if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_ && c.NP == NP_)      \
     kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_, NP_>;
   if constexpr (sizeof(Tst) == 2) {
-    SDM_PIPE(64, 6, 16, 4, 4, 4) SDM_PIPE(64, 6, 16, 4, 4, 2) SDM_PIPE(64, 7, 16, 4, 4, 4) SDM_PIPE(64, 5, 16, 4, 4, 4)
+    SDM_PIPE(64, 6, 16, 4, 3, 4) SDM_PIPE(64, 6, 16, 4, 4, 4) SDM_PIPE(64, 6, 16, 3, 4, 4) SDM_PIPE(64, 7, 16, 4, 3, 4)
+    SDM_PIPE(64, 6, 16, 4, 3, 2)
   } else {
-    SDM_PIPE(32, 6, 16, 4, 4, 4) SDM_PIPE(32, 4, 16, 4, 4, 4)
+    SDM_PIPE(32, 6, 16, 4, 3, 4) SDM_PIPE(32, 4, 16, 4, 3, 4)
   }
 #undef SDM_PIPE
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no pipelined kernel for the chosen tile");

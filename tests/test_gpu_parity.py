@@ -147,11 +147,11 @@ SCAN = [
 ]
 
 
-def _run_scan(sdm, dev, shape, inp, variant, g=None):
+def _run_scan(sdm, dev, shape, inp, variant, g=None, tile=0):
     d = {k: v.to(dev) for k, v in inp.items()}
     M = d["M"].clone()
     y = sdm.scan(d["idx_w"], d["w_w"], d["idx_r"], d["w_r"], d["v"], d["alpha"], d["beta"], M,
-                 g=None if g is None else g.to(dev), variant=variant)
+                 g=None if g is None else g.to(dev), variant=variant, tile=tile)
     sdm.stream_check()
     return y, M
 
@@ -168,6 +168,21 @@ def test_scan_matches_oracle(sdm, oracle, cuda_device, case):
     tol = tol_for(tst)
     assert_rel_close(y.cpu().numpy(), oy, tol, "y")
     assert_rel_close(f32(M), oM, tol, "M_T")
+
+
+@pytest.mark.parametrize("tst,tile", [("bf16", k) for k in range(1, 6)] + [("f32", k) for k in range(1, 3)])
+def test_pipelined_tiles_match_oracle(sdm, oracle, cuda_device, tst, tile):
+    """Every entry of the pipelined kernel's tile table (warp counts, stage
+    depth) against the oracle, on a case with many slot collisions."""
+    shape = synth.Shape("t", B=1, T=150, H=2, sqrt_n=12, d_v=256 if tst == "bf16" else 128, W=24, R=20,
+                        in_dtype="bf16", state_dtype=tst)
+    inp = scan_inputs(shape, seed=70 + tile)
+    y, M = _run_scan(sdm, cuda_device, shape, inp, "pipelined", tile=tile)
+    oy, oM, _ = oracle.scan(inp["idx_w"].numpy(), inp["w_w"].numpy().astype(np.float64), inp["idx_r"].numpy(),
+                            inp["w_r"].numpy().astype(np.float64), f32(inp["v"]), f32(inp["alpha"]),
+                            f32(inp["beta"]), f32(inp["M"]), state_bf16=(tst == "bf16"))
+    assert_rel_close(y.cpu().numpy(), oy, tol_for(tst), "y")
+    assert_rel_close(f32(M), oM, tol_for(tst), "M_T")
 
 
 @pytest.mark.parametrize("variant", ["resident", "streaming", "pipelined"])
