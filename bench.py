@@ -6,8 +6,8 @@ A step is one sdm_layer_forward call over one batch of synthetic input: the
 product-key selection of k' and q', the record build, the state
 initialisation and the recurrence (epilogue off unless --epilogue). Inputs
 are resident in HBM when the timed region starts; `e2e` repeats the
-measurement with the inputs copied from pinned host memory and y copied back
-inside the timed region. With N > 1 (torchrun) each rank runs its own batch
+measurement through the C ABI with the inputs copied from pinned host memory
+and y and M_T copied back inside the timed region. With N > 1 (torchrun) each rank runs its own batch
 (weak scaling, no collective on the data path); the time is the max over
 ranks. `--impl reference` times the CPU oracle on a bounded sample instead
 (rank 0 only).
