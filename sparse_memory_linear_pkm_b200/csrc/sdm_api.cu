@@ -222,11 +222,11 @@ constexpr StreamCfg kStreamCfgs[] = {
 // segments), stages, staging chunk, write warps, read warps, producer warps.
 struct PipeCfg {
   int state_bytes;
-  int C, P, L, NWW, NWR, NP;
+  int C, P, L, NWW, NWR, NP, S;
 };
 constexpr PipeCfg kPipeCfgs[] = {
-    {2, 64, 6, 16, 4, 3, 4}, {2, 64, 6, 16, 4, 4, 4}, {2, 64, 6, 16, 3, 4, 4}, {2, 64, 7, 16, 4, 3, 4},
-    {2, 64, 6, 16, 4, 3, 2}, {4, 32, 6, 16, 4, 3, 4}, {4, 32, 4, 16, 4, 3, 4},
+    {2, 64, 6, 16, 4, 3, 4, 1}, {2, 64, 6, 16, 4, 3, 4, 2}, {2, 64, 7, 8, 4, 3, 4, 2}, {2, 64, 6, 16, 4, 4, 4, 1},
+    {2, 64, 6, 16, 4, 3, 2, 1}, {4, 32, 6, 16, 4, 3, 4, 1}, {4, 32, 4, 16, 4, 3, 4, 1}, {4, 32, 6, 16, 4, 3, 4, 2},
 };
 
 // Instantiated resident tiles: columns per warp, warps per CTA, staging
@@ -250,7 +250,15 @@ size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L, int NW) {
 size_t pipelined_smem(const sdm_shape_t& s, const PipeCfg& k) {
   const sdm::PipeLayout pl = sdm::pipe_layout(s.W, s.R);
   return sdm::pipe_smem_bytes(k.P, k.L, pl.Wp, pl.Rp, pl.words, k.C, static_cast<int>(in_size(s.state_dtype)),
-                              static_cast<int>(in_size(s.in_dtype)), k.NWR);
+                              static_cast<int>(in_size(s.in_dtype)), k.NWR, k.S);
+}
+
+// Whether every row of the pipelined kernel's stage space (gathered and
+// written stages) has a 13-bit source code (the bits above are flags).
+bool pipe_codes_fit(const sdm_shape_t& s, const PipeCfg& k) {
+  const sdm::PipeLayout pl = sdm::pipe_layout(s.W, s.R);
+  return static_cast<int64_t>(k.P) * (pl.Wp + pl.Rp) + static_cast<int64_t>(sdm::pipe_wstages(k.P, k.S)) * pl.Wp <=
+         static_cast<int64_t>(sdm::kRowMask);
 }
 
 // Whether the automatic variant takes the pipelined kernel for few column
@@ -315,7 +323,8 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
   if (rows_fit && (s.variant == SDM_VARIANT_PIPELINED || (s.variant == SDM_VARIANT_AUTO && kPipelinedAuto && few_tiles))) {
     std::vector<PipeCfg> order;
     for (const PipeCfg& k : kPipeCfgs)
-      if (k.state_bytes == s_state && s.d_v % k.C == 0 && pipelined_smem(s, k) <= lim) order.push_back(k);
+      if (k.state_bytes == s_state && s.d_v % k.C == 0 && pipelined_smem(s, k) <= lim && pipe_codes_fit(s, k))
+        order.push_back(k);
     const int i = pick(order.size());
     if (i >= 0) {
       const PipeCfg& k = order[i];
@@ -326,6 +335,7 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
       c.NWW = k.NWW;
       c.NWR = k.NWR;
       c.NP = k.NP;
+      c.S = k.S;
       c.parts = bh * (s.d_v / k.C) * 2 <= dev.sms ? 2 : 1;
       c.smem = pipelined_smem(s, k);
       *out = c;
@@ -1022,8 +1032,8 @@ sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_l
   if (c.kind == SDM_VARIANT_RESIDENT)
     snprintf(out, out_len, "resident CW=%d NWARP=%d L=%d EB=%d smem=%zu", c.CW, c.NWARP, c.L, c.EB, c.smem);
   else if (c.kind == SDM_VARIANT_PIPELINED)
-    snprintf(out, out_len, "pipelined C=%d P=%d L=%d NWW=%d NWR=%d NP=%d parts=%d smem=%zu", c.C, c.P, c.L, c.NWW,
-             c.NWR, c.NP, c.parts, c.smem);
+    snprintf(out, out_len, "pipelined C=%d P=%d L=%d NWW=%d NWR=%d NP=%d S=%d parts=%d smem=%zu", c.C, c.P, c.L, c.NWW,
+             c.NWR, c.NP, c.S, c.parts, c.smem);
   else
     snprintf(out, out_len, "streaming C=%d P=%d L=%d NW=%d smem=%zu", c.C, c.P, c.L, c.NWARP, c.smem);
   return ok();

@@ -50,6 +50,7 @@ struct ScanChoice {
   int L = 16;
   int CW = 8, NWARP = 2, EB = 4;  // resident: columns per warp, warps per CTA, entry block
   int NWW = 4, NWR = 4, NP = 4, parts = 1;  // pipelined: write, read and producer warps, slot parts per tile
+  int S = 1;                                  // pipelined: tokens per barrier step
   size_t smem = 0;
 };
 

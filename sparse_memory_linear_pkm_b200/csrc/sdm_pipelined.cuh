@@ -107,7 +107,15 @@ __host__ __device__ inline PipeLayout pipe_layout(int W, int R) {
   return pl;
 }
 
-constexpr uint32_t kSrcSameToken = 0x8000u;  // src_r flag: recompute this token's write (low bits: j)
+// Source codes (16 bits): a row of the stage space below 0x2000, or a flag
+// with a write entry j in the low 9 bits.
+constexpr uint32_t kSrcSameToken = 0x8000u;  // reads: recompute this token's write j
+constexpr uint32_t kSrcPrevToken = 0x4000u;  // second token of a two-token step: recompute the first token's write j
+constexpr uint32_t kSkipStore = 0x2000u;     // first token's write: the second token rewrites the slot, no HBM store
+constexpr uint32_t kRowMask = 0x1FFFu;
+constexpr uint32_t kEntryMask = 0x1FFu;
+constexpr int kTokW = 3;  // two-token step: write units of each token per pass of a write lane
+constexpr int kTokR = 3;  // two-token step: read entries of each token per pass of a read lane
 
 // 16 bytes of state (8 bf16 or 4 fp32 values) as fp32, by bit operations.
 template <typename Tst>
@@ -156,9 +164,13 @@ __device__ __forceinline__ int slot_part(uint32_t slot, int parts) {
 
 constexpr int kPipeTokensPerBlock = 32;
 
+// Written stages of the pipelined kernel: P + S - 1, so that the S tokens
+// of a step never write a stage that one of them still reads.
+__host__ __device__ constexpr int pipe_wstages(int P, int S) { return P + S - 1; }
+
 // Shared-memory bytes of k_build_pipe_records.
 __host__ __device__ constexpr size_t pipe_records_smem(int W, int R, int P, int log2_cells, int parts) {
-  return static_cast<size_t>(kPipeTokensPerBlock + P - 1) * ((size_t{1} << log2_cells) * 4 + W * 2) +
+  return static_cast<size_t>(kPipeTokensPerBlock + P) * ((size_t{1} << log2_cells) * 4 + W * 2) +
          static_cast<size_t>(kPipeTokensPerBlock) * R * 2 + 4 + static_cast<size_t>(kPipeTokensPerBlock) * parts * 8;
 }
 
@@ -167,21 +179,26 @@ __host__ __device__ constexpr size_t pipe_records_smem(int W, int R, int P, int 
 // hazard plan against the written slots of the P - 1 tokens before (one
 // open-addressing table per token, slot -> compacted write entry), and, when
 // y_zero is given, zeros for those tokens' y rows (the recurrence adds the
-// parts' sums into it). Slot indices outside [0, N) are left out and set the
-// device error word.
+// parts' sums into it). With S = 2 the recurrence takes tokens in pairs
+// (2s, 2s + 1): the second token's entries that the first one wrote become
+// kSrcPrevToken, and the first token's writes of slots the second one
+// rewrites get kSkipStore. Slot indices outside [0, N) are left out and set
+// the device error word.
 template <typename Tin>
 __global__ void __launch_bounds__(256) k_build_pipe_records(
     const int32_t* __restrict__ idx_w, const float* __restrict__ w_w, const int32_t* __restrict__ idx_r,
     const float* __restrict__ w_r, const Tin* __restrict__ alpha, const Tin* __restrict__ beta, int T, int H, int N,
-    int W, int R, int P, int parts, int log2_cells, PipeLayout pl, uint32_t* __restrict__ rec,
+    int W, int R, int P, int S, int parts, int log2_cells, PipeLayout pl, uint32_t* __restrict__ rec,
     float* __restrict__ y_zero, int d_v, unsigned* err) {
   const int E = pl.Wp + pl.Rp;  // rows of one gather stage
+  const int Q = pipe_wstages(P, S);
   extern __shared__ uint32_t sm[];
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int t0 = blockIdx.x * kPipeTokensPerBlock;
   const int t_end = min(T, t0 + kPipeTokensPerBlock);
   const int t_first = max(0, t0 - (P - 1));
-  const int n_tab = t_end - t_first, n_own = t_end - t0;
+  const int t_tab_end = min(T, t_end + (S - 1));  // the tables reach the second token of the last pair
+  const int n_tab = t_tab_end - t_first, n_own = t_end - t0;
   const int n_cells = 1 << log2_cells;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t* cells = sm;                                               // [n_tab][n_cells]
@@ -194,7 +211,7 @@ __global__ void __launch_bounds__(256) k_build_pipe_records(
   __syncthreads();
 
   // 1. compaction (one warp per token) and the tables of written slots
-  for (int tt = t_first + warp; tt < t_end; tt += blockDim.x / 32) {
+  for (int tt = t_first + warp; tt < t_tab_end; tt += blockDim.x / 32) {
     const int64_t th = (static_cast<int64_t>(b) * T + tt) * H + h;
     uint32_t* tab = cells + (tt - t_first) * n_cells;
     int base[2] = {0, 0};
@@ -220,7 +237,7 @@ __global__ void __launch_bounds__(256) k_build_pipe_records(
         }
       }
     }
-    if (tt >= t0) {
+    if (tt >= t0 && tt < t_end) {
       int rbase[2] = {0, 0};
       for (int r0 = 0; r0 < R; r0 += 32) {
         const int r = r0 + lane;
@@ -285,7 +302,21 @@ __global__ void __launch_bounds__(256) k_build_pipe_records(
     uint32_t src;
     if (code < 0) src = static_cast<uint32_t>((t % P) * E + (e < W ? c : pl.Wp + c));
     else if ((code >> 9) == 0) src = kSrcSameToken | static_cast<uint32_t>(code & 511);
-    else src = static_cast<uint32_t>(P * E + ((t - (code >> 9)) % P) * pl.Wp + (code & 511));
+    else if ((code >> 9) == 1 && S == 2 && (t & 1)) src = kSrcPrevToken | static_cast<uint32_t>(code & 511);
+    else src = static_cast<uint32_t>(P * E + ((t - (code >> 9)) % Q) * pl.Wp + (code & 511));
+    if (e < W && S == 2 && !(t & 1) && t + 1 < T) {  // does the pair's second token rewrite the slot?
+      const uint32_t* tab = cells + (t + 1 - t_first) * n_cells;
+      uint32_t pos = slot_hash(static_cast<uint32_t>(slot), log2_cells);
+      for (int probe = 0; probe < n_cells; ++probe) {
+        const uint32_t cur = tab[pos];
+        if (cur == kEmptyCell) break;
+        if ((cur >> 9) == static_cast<uint32_t>(slot)) {
+          src |= kSkipStore;
+          break;
+        }
+        pos = (pos + 1) & (n_cells - 1);
+      }
+    }
     if (e < W) {
       const float a_t = to_f32<Tin>(alpha[th]), b_t = to_f32<Tin>(beta[th]);
       const float cw = b_t * wt;
@@ -353,10 +384,10 @@ struct PipeArgs {
 
 // Shared-memory bytes of k_scan_pipelined (host and device agree on this).
 __host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
-                                                     int s_in, int NWR) {
-  return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(P) * Wp * C * s_state +
+                                                     int s_in, int NWR, int S) {
+  return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(pipe_wstages(P, S)) * Wp * C * s_state +
          static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in +
-         static_cast<size_t>(2) * NWR * C * 4 + (2 * P + 2) * 8 + 128;
+         static_cast<size_t>(2) * S * NWR * C * 4 + (2 * P + 2) * 8 + 128;
 }
 
 // Sums a[0:VE) (the VE columns of one 16-byte unit) over the lanes that
@@ -386,7 +417,7 @@ __device__ __forceinline__ int reduce_scatter_entries(float (&a)[VE], int lane) 
   return off;
 }
 
-template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR, int NP>
+template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR, int NP, int S>
 __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipelined(const __grid_constant__ PipeArgs a) {
   constexpr int NT = (NP + 1 + NWW + NWR) * kWarp;
   constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
@@ -396,6 +427,8 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   static_assert(U >= 1 && U <= kWarp && kWarp % U == 0, "a row segment spans a divisor of the warp");
   static_assert(NT % U == 0, "gather lanes cover whole rows");
   static_assert(L >= P, "a chunk of records is staged before its tokens are gathered");
+  static_assert(S == 1 || (S == 2 && L % 2 == 0 && P >= 5), "one or two tokens per step; pairs never straddle a chunk");
+  constexpr int Q = pipe_wstages(P, S);  // written stages
   static_assert(P >= 3, "rows are gathered P - 1 >= 2 tokens ahead");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // TMA boxes land at 128-byte aligned rows
@@ -403,11 +436,11 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   const PipeLayout pl = a.pl;
   const int Wp = pl.Wp, E = pl.Wp + pl.Rp, words = pl.words, T = a.T;
   unsigned char* lstage = smem;                                                    // [P][E][RS]
-  unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [P][Wp][RS]
-  uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(P) * Wp * RS);  // [2][L][words]
+  unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [Q][Wp][RS]
+  uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(Q) * Wp * RS);  // [2][L][words]
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
-  float* ybuf = reinterpret_cast<float*>(vbuf + 2 * L * C);                        // [2][NWR][C] read partials
-  uint64_t* cbar = reinterpret_cast<uint64_t*>(ybuf + 2 * NWR * C);               // [2] record chunks
+  float* ybuf = reinterpret_cast<float*>(vbuf + 2 * L * C);                        // [2][S][NWR][C] read partials
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(ybuf + 2 * S * NWR * C);           // [2] record chunks
   uint64_t* full = cbar + 2;                                                       // [P] gathered stages
   uint64_t* done = full + P;  // [P] the consumers are through with a token, its stores fenced
 
@@ -504,12 +537,12 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
     load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * C + qw * VE, vv);
     // the write of entry j on this thread's unit of its source row (fp32 math, state rounding by the caller)
     auto written = [&](int j, float (&m)[VE]) {
-      unpack_unit<Tst>(row_at(sw[j]), m);
+      unpack_unit<Tst>(row_at(sw[j] & kRowMask), m);
       const float2 c = ac[j];
       write_unit<VE>(m, vv, c.x, c.y);
     };
     if (writer) {
-      unsigned char* ws = wstage + static_cast<size_t>(t % P) * Wp * RS + qw * 16;
+      unsigned char* ws = wstage + static_cast<size_t>(t % Q) * Wp * RS + qw * 16;
       Tst* Mq = Mbh + qw * VE;
       const uint32_t* slw = rec + pl.off_slot_w;
       const int n = nw * U;
@@ -531,14 +564,10 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
     } else {
       const uint16_t* sr = reinterpret_cast<const uint16_t*>(rec + pl.off_src_r);
       const float* qr = reinterpret_cast<const float*>(rec + pl.off_q_r);
-      auto read_row = [&](int i, float (&m)[VE]) {
-        const uint32_t src = sr[i];
-        if (src & kSrcSameToken) {  // written by this token: that write, rounded as stored
-          written(static_cast<int>(src & 0x7FFFu), m);
-          unpack_unit<Tst>(pack16<Tst>(m), m);
-        } else {
-          unpack_unit<Tst>(row_at(src), m);
-        }
+      // a read of a slot this token writes: that write, rounded as stored
+      auto same_token = [&](uint32_t src, float (&m)[VE]) {
+        written(static_cast<int>(src & kEntryMask), m);
+        unpack_unit<Tst>(pack16<Tst>(m), m);
       };
       float acc[VE];
 #pragma unroll
@@ -546,9 +575,16 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
       for (int i0 = base_r; i0 < nr; i0 += 2 * stride_r) {
         const int i1 = i0 + stride_r;
         const bool has1 = i1 < nr;
+        const uint32_t src0 = sr[i0], src1 = sr[has1 ? i1 : i0];
+        // both rows first (a flagged code's low bits still name a row in
+        // shared memory), the rare recomputation after: no branch between them
         float m0[VE], m1[VE];
-        read_row(i0, m0);
-        read_row(has1 ? i1 : i0, m1);
+        unpack_unit<Tst>(row_at(src0 & kRowMask), m0);
+        unpack_unit<Tst>(row_at(src1 & kRowMask), m1);
+        if ((src0 | src1) & kSrcSameToken) {
+          if (src0 & kSrcSameToken) same_token(src0, m0);
+          if (src1 & kSrcSameToken) same_token(src1, m1);
+        }
         read_unit<VE>(acc, m0, qr[i0]);
         read_unit<VE>(acc, m1, has1 ? qr[i1] : 0.0f);
       }
@@ -556,6 +592,139 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
       float* yb = ybuf + (static_cast<size_t>(t & 1) * NWR + (cw - NWW)) * C + qw * VE + off;
 #pragma unroll
       for (int j = 0; j < VE * U / kWarp; ++j) yb[j] = acc[j];
+    }
+  };
+  // Tokens ta and ta + 1 (if hb) on this consumer thread, interleaved. Rows
+  // that the first token writes and the second one reads or rewrites are
+  // recomputed from the first token's source (as stored, rounded to the state
+  // type), so the two tokens need no barrier between them; per token, every
+  // value and every sum comes out as in the one-token step.
+  auto compute_pair = [&](int ta, bool hb) {
+    const int tb = ta + 1;
+    const uint32_t* recA = rec_of(ta);
+    const uint32_t* recB = hb ? rec_of(tb) : recA;
+    const uint16_t* swA = reinterpret_cast<const uint16_t*>(recA + pl.off_src_w);
+    const uint16_t* swB = reinterpret_cast<const uint16_t*>(recB + pl.off_src_w);
+    const float2* acA = reinterpret_cast<const float2*>(recA + pl.off_awcw);
+    const float2* acB = reinterpret_cast<const float2*>(recB + pl.off_awcw);
+    float vA[VE], vB[VE];
+    load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((ta / L) & 1) * L + ta % L) * C + qw * VE, vA);
+    load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>(((hb ? tb : ta) / L) & 1) * L + (hb ? tb : ta) % L) * C + qw * VE, vB);
+    auto writtenA = [&](int j, float (&m)[VE]) {  // the first token's write j (unrounded)
+      unpack_unit<Tst>(row_at(swA[j] & kRowMask), m);
+      const float2 c = acA[j];
+      write_unit<VE>(m, vA, c.x, c.y);
+    };
+    auto writtenB = [&](int j, float (&m)[VE]) {  // the second token's write j (unrounded)
+      const uint32_t src = swB[j];
+      if (src & kSrcPrevToken) {
+        writtenA(static_cast<int>(src & kEntryMask), m);
+        unpack_unit<Tst>(pack16<Tst>(m), m);
+      } else {
+        unpack_unit<Tst>(row_at(src & kRowMask), m);
+      }
+      const float2 c = acB[j];
+      write_unit<VE>(m, vB, c.x, c.y);
+    };
+    if (writer) {
+      unsigned char* wsA = wstage + static_cast<size_t>(ta % Q) * Wp * RS + qw * 16;
+      unsigned char* wsB = wstage + static_cast<size_t>(tb % Q) * Wp * RS + qw * 16;
+      Tst* Mq = Mbh + qw * VE;
+      const uint32_t* slwA = recA + pl.off_slot_w;
+      const uint32_t* slwB = recB + pl.off_slot_w;
+      const int nA = static_cast<int>(recA[pl.off_meta]) * U;
+      const int nB = hb ? static_cast<int>(recB[pl.off_meta]) * U : 0;
+      for (int p0 = base_w; p0 < max(nA, nB); p0 += kTokW * stride_w) {
+        // every unit computed from a record entry (past the counts: padding
+        // entries, in-bounds rows, zero coefficients); only the stores are
+        // conditional
+        int j[kTokW];
+        uint32_t srcB[kTokW];
+        float mA[kTokW][VE], mB[kTokW][VE];
+#pragma unroll
+        for (int k = 0; k < kTokW; ++k) {
+          j[k] = min((p0 + k * stride_w) / U, Wp - 1);
+          srcB[k] = swB[j[k]];
+          unpack_unit<Tst>(row_at(swA[j[k]] & kRowMask), mA[k]);
+          unpack_unit<Tst>(row_at(srcB[k] & kRowMask), mB[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kTokW; ++k) {
+          if (srcB[k] & kSrcPrevToken) {  // rare: the first token's write of the slot, as stored
+            writtenA(static_cast<int>(srcB[k] & kEntryMask), mB[k]);
+            unpack_unit<Tst>(pack16<Tst>(mB[k]), mB[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kTokW; ++k) {
+          const float2 ca = acA[j[k]], cb = acB[j[k]];
+          write_unit<VE>(mA[k], vA, ca.x, ca.y);
+          write_unit<VE>(mB[k], vB, cb.x, cb.y);
+        }
+#pragma unroll
+        for (int k = 0; k < kTokW; ++k) {
+          const int p = p0 + k * stride_w;
+          if (p < nA) {
+            const uint4 pk = pack16<Tst>(mA[k]);
+            *reinterpret_cast<uint4*>(wsA + static_cast<size_t>(j[k]) * RS) = pk;
+            if (!(swA[j[k]] & kSkipStore)) *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slwA[j[k]]) * a.d_v) = pk;
+          }
+          if (p < nB) {
+            const uint4 pk = pack16<Tst>(mB[k]);
+            *reinterpret_cast<uint4*>(wsB + static_cast<size_t>(j[k]) * RS) = pk;
+            *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slwB[j[k]]) * a.d_v) = pk;
+          }
+        }
+      }
+    } else {
+      const uint16_t* srA = reinterpret_cast<const uint16_t*>(recA + pl.off_src_r);
+      const uint16_t* srB = reinterpret_cast<const uint16_t*>(recB + pl.off_src_r);
+      const float* qrA = reinterpret_cast<const float*>(recA + pl.off_q_r);
+      const float* qrB = reinterpret_cast<const float*>(recB + pl.off_q_r);
+      const int nA = static_cast<int>(recA[pl.off_meta + 1]);
+      const int nB = hb ? static_cast<int>(recB[pl.off_meta + 1]) : 0;
+      float accA[VE], accB[VE];
+#pragma unroll
+      for (int j = 0; j < VE; ++j) accA[j] = accB[j] = 0.f;
+      for (int i0 = base_r; i0 < max(nA, nB); i0 += kTokR * stride_r) {
+        int i[kTokR];
+        uint32_t sA[kTokR], sB[kTokR];
+        float mA[kTokR][VE], mB[kTokR][VE];
+#pragma unroll
+        for (int k = 0; k < kTokR; ++k) {
+          i[k] = min(i0 + k * stride_r, pl.Rp - 1);
+          sA[k] = srA[i[k]];
+          sB[k] = srB[i[k]];
+          unpack_unit<Tst>(row_at(sA[k] & kRowMask), mA[k]);
+          unpack_unit<Tst>(row_at(sB[k] & kRowMask), mB[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < kTokR; ++k) {  // rare: reads of rows this step writes, as stored
+          if (sA[k] & kSrcSameToken) {
+            writtenA(static_cast<int>(sA[k] & kEntryMask), mA[k]);
+            unpack_unit<Tst>(pack16<Tst>(mA[k]), mA[k]);
+          }
+          if (sB[k] & (kSrcSameToken | kSrcPrevToken)) {
+            if (sB[k] & kSrcSameToken) writtenB(static_cast<int>(sB[k] & kEntryMask), mB[k]);
+            else writtenA(static_cast<int>(sB[k] & kEntryMask), mB[k]);
+            unpack_unit<Tst>(pack16<Tst>(mB[k]), mB[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kTokR; ++k) {  // rows past a token's count may hold anything: not summed
+          const int ik = i0 + k * stride_r;
+          if (ik < nA) read_unit<VE>(accA, mA[k], qrA[i[k]]);
+          if (ik < nB) read_unit<VE>(accB, mB[k], qrB[i[k]]);
+        }
+      }
+      const int off = reduce_scatter_entries<VE, U>(accA, lane);
+      reduce_scatter_entries<VE, U>(accB, lane);
+      float* yb = ybuf + (static_cast<size_t>((ta / 2) & 1) * 2 * NWR + (cw - NWW)) * C + qw * VE + off;
+#pragma unroll
+      for (int j = 0; j < VE * U / kWarp; ++j) {
+        yb[j] = accA[j];
+        yb[NWR * C + j] = accB[j];
+      }
     }
   };
 
@@ -584,43 +753,48 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
     return;
   }
   constexpr int kBarThreads = (1 + NWW + NWR) * kWarp;  // the control warp and the consumers
+  const int n_steps = (T + S - 1) / S;                  // a step: S consecutive tokens
   if (control) {
-    // y of token s: the read warps' column sums, added in warp order
-    auto put_y = [&](int s) {
-      const float* yb = ybuf + static_cast<size_t>(s & 1) * NWR * C;
+    // y of token u: the read warps' column sums, added in warp order
+    auto put_y = [&](int u) {
+      const float* yb = ybuf + (static_cast<size_t>((u / S) & 1) * S + u % S) * NWR * C;
       for (int c = lane; c < C; c += kWarp) {
         float acc = yb[c];
 #pragma unroll
         for (int r = 1; r < NWR; ++r) acc += yb[r * C + c];
-        y_bh[static_cast<int64_t>(s) * tok_step + c] = acc;
+        y_bh[static_cast<int64_t>(u) * tok_step + c] = acc;
       }
     };
-    bool ok = chunk_wait(0) && mbar_wait_bounded(&full[0], 0, a.err);
+    auto ready = [&](int u) {  // token u's records and rows are in shared memory
+      const bool ok = u % L != 0 || chunk_wait(u / L);
+      return ok && mbar_wait_bounded(&full[u % P], (u / P) & 1, a.err);
+    };
+    bool ok = true;
+    for (int u = 0; u < S && u < T; ++u) ok = ok && ready(u);
 #pragma unroll 1
-    for (int t = 0; t < T; ++t) {
-      if (named_barrier_or(1, kBarThreads, !ok)) return;  // token t - 1 is complete, token t's rows have landed
-      if (t > 0) {
-        put_y(t - 1);
+    for (int st = 0; st < n_steps; ++st) {
+      if (named_barrier_or(1, kBarThreads, !ok)) return;  // step st - 1 is complete, step st's rows have landed
+      if (st > 0) {
+        for (int u = (st - 1) * S; u < st * S; ++u) put_y(u);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&done[(t - 1) % P]);
+        if (lane == 0)
+          for (int u = (st - 1) * S; u < st * S; ++u) mbar_arrive(&done[u % P]);
       }
-      if (t + 1 < T) {
-        const int s = t + 1;
-        if (s % L == 0) ok = chunk_wait(s / L);
-        if (ok) ok = mbar_wait_bounded(&full[s % P], (s / P) & 1, a.err);
-      }
+      for (int u = (st + 1) * S; u < (st + 2) * S && u < T; ++u) ok = ok && ready(u);
     }
-    if (!named_barrier_or(1, kBarThreads, !ok)) put_y(T - 1);
+    if (!named_barrier_or(1, kBarThreads, !ok))
+      for (int u = (n_steps - 1) * S; u < T; ++u) put_y(u);
     return;
   }
   // consumers
 #pragma unroll 1
-  for (int t = 0; t < T; ++t) {
-    // the state rows this thread stored for token t - 1 become visible to the
+  for (int st = 0; st < n_steps; ++st) {
+    // the state rows this thread stored in step st - 1 become visible to the
     // gathers that the producers issue after the control warp's signal
-    if (writer && t > 0) fence_proxy_async_global();
+    if (writer && st > 0) fence_proxy_async_global();
     if (named_barrier_or(1, kBarThreads, false)) return;
-    compute(t);
+    if constexpr (S == 1) compute(st);
+    else compute_pair(2 * st, 2 * st + 1 < T);
   }
   named_barrier_or(1, kBarThreads, false);
 }

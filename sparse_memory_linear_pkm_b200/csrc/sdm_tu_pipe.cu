@@ -21,7 +21,7 @@ sdm_status_t launch_pipe_records_typed(const sdm_shape_t& s, const ScanChoice& c
   const int tblocks = (s.T + sdm::kPipeTokensPerBlock - 1) / sdm::kPipeTokensPerBlock;
   const dim3 grid(tblocks, s.B * s.H);
   kern<<<grid, 256, smem, st>>>(idx_w, w_w, idx_r, w_r, static_cast<const Tin*>(alpha), static_cast<const Tin*>(beta),
-                                s.T, s.H, static_cast<int>(slots_of(s.sqrt_n)), s.W, s.R, c.P, c.parts, log2_cells,
+                                s.T, s.H, static_cast<int>(slots_of(s.sqrt_n)), s.W, s.R, c.P, c.S, c.parts, log2_cells,
                                 sdm::pipe_layout(s.W, s.R), rec, y_zero, s.d_v, dev.err);
   return launch_status("pipelined record build launch");
 }
@@ -48,14 +48,14 @@ template <typename Tin, typename Tst>
 sdm_status_t launch_pipe_typed(const ScanChoice& c, const sdm::PipeArgs& a, cudaStream_t st) {
   const dim3 grid(a.B * a.H * a.parts, a.d_v / c.C);
   void (*kern)(sdm::PipeArgs) = nullptr;
-#define SDM_PIPE(C_, P_, L_, NWW_, NWR_, NP_)                                                  \
-  if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_ && c.NP == NP_)      \
-    kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_, NP_>;
+#define SDM_PIPE(C_, P_, L_, NWW_, NWR_, NP_, S_)                                                          \
+  if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_ && c.NP == NP_ && c.S == S_)      \
+    kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_, NP_, S_>;
   if constexpr (sizeof(Tst) == 2) {
-    SDM_PIPE(64, 6, 16, 4, 3, 4) SDM_PIPE(64, 6, 16, 4, 4, 4) SDM_PIPE(64, 6, 16, 3, 4, 4) SDM_PIPE(64, 7, 16, 4, 3, 4)
-    SDM_PIPE(64, 6, 16, 4, 3, 2)
+    SDM_PIPE(64, 6, 16, 4, 3, 4, 1) SDM_PIPE(64, 6, 16, 4, 3, 4, 2) SDM_PIPE(64, 7, 8, 4, 3, 4, 2)
+    SDM_PIPE(64, 6, 16, 4, 4, 4, 1) SDM_PIPE(64, 6, 16, 4, 3, 2, 1)
   } else {
-    SDM_PIPE(32, 6, 16, 4, 3, 4) SDM_PIPE(32, 4, 16, 4, 3, 4)
+    SDM_PIPE(32, 6, 16, 4, 3, 4, 1) SDM_PIPE(32, 4, 16, 4, 3, 4, 1) SDM_PIPE(32, 6, 16, 4, 3, 4, 2)
   }
 #undef SDM_PIPE
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no pipelined kernel for the chosen tile");

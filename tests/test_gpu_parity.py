@@ -170,7 +170,7 @@ def test_scan_matches_oracle(sdm, oracle, cuda_device, case):
     assert_rel_close(f32(M), oM, tol, "M_T")
 
 
-@pytest.mark.parametrize("tst,tile", [("bf16", k) for k in range(1, 6)] + [("f32", k) for k in range(1, 3)])
+@pytest.mark.parametrize("tst,tile", [("bf16", k) for k in range(1, 6)] + [("f32", k) for k in range(1, 4)])
 def test_pipelined_tiles_match_oracle(sdm, oracle, cuda_device, tst, tile):
     """Every entry of the pipelined kernel's tile table (warp counts, stage
     depth) against the oracle, on a case with many slot collisions."""
@@ -183,6 +183,20 @@ def test_pipelined_tiles_match_oracle(sdm, oracle, cuda_device, tst, tile):
                             f32(inp["beta"]), f32(inp["M"]), state_bf16=(tst == "bf16"))
     assert_rel_close(y.cpu().numpy(), oy, tol_for(tst), "y")
     assert_rel_close(f32(M), oM, tol_for(tst), "M_T")
+
+
+@pytest.mark.parametrize("tst,tiles", [("bf16", (1, 2, 3)), ("f32", (1, 3))])
+@pytest.mark.parametrize("T", [1, 2, 7, 64, 151])
+def test_pipelined_two_token_steps_bit_identical(sdm, cuda_device, tst, tiles, T):
+    """Tokens taken two per barrier step (the second recomputing the first's
+    writes of shared slots) give the same y and state bit for bit as one
+    token per step: every value and every sum is formed in the same order."""
+    shape = synth.Shape("t", B=2, T=T, H=1, sqrt_n=8, d_v=256 if tst == "bf16" else 128, W=16, R=12,
+                        in_dtype="bf16", state_dtype=tst)
+    inp = scan_inputs(shape, seed=90 + T)
+    outs = [_run_scan(sdm, cuda_device, shape, inp, "pipelined", tile=k) for k in tiles]
+    for y, M in outs[1:]:
+        assert torch.equal(y, outs[0][0]) and torch.equal(M, outs[0][1])
 
 
 @pytest.mark.parametrize("variant", ["resident", "streaming", "pipelined"])
