@@ -67,7 +67,8 @@ def parse_args():
     ap.add_argument("--decode", action="store_true",
                     help="time decode steps instead: one token per call (sdm_layer_step), state carried")
     ap.add_argument("--fp8-state", action="store_true",
-                    help="with --decode: keep the state in the block-scaled fp8 format (E4M3, scale per 16 values)")
+                    help="keep the state in the block-scaled fp8 format (E4M3, scale per 16 values): the layer "
+                         "(pipelined recurrence) or, with --decode, the decode step")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward instead: sdm_scan_backward and the two selection-weight backwards")
     ap.add_argument("--slot-counts", action="store_true",
@@ -186,12 +187,15 @@ def measured_peaks() -> dict:
     return {}
 
 
-def algorithmic_bytes_per_token_head(shape: synth.Shape, epilogue: bool) -> int:
+def algorithmic_bytes_per_token_head(shape: synth.Shape, epilogue: bool, fp8_state: bool = False) -> int:
     """(2W + R) d_v sizeof(state) of state traffic, plus the per-token-head
-    inputs (indices + weights, v, alpha, beta, g) and the fp32 y."""
+    inputs (indices + weights, v, alpha, beta, g) and the fp32 y. The fp8
+    state moves one code byte per value and one exponent byte per 16."""
     s_state = 2 if shape.state_dtype == synth.BF16 else 4
     s_in = 2 if shape.in_dtype == synth.BF16 else 4
     b = (2 * shape.W + shape.R) * shape.d_v * s_state
+    if fp8_state:
+        b = (2 * shape.W + shape.R) * (shape.d_v + shape.d_v // 16)
     b += (shape.W + shape.R) * 8 + shape.d_v * s_in + 2 * s_in + shape.d_v * 4
     if epilogue:
         b += shape.d_v * s_in
@@ -432,11 +436,13 @@ def run_sdm(args, dist: Dist):
     shape = synth.WORKLOADS[args.workload]
     sdm.native.load()
     inp = synth.make_inputs(shape, seed=args.seed + dist.rank, device=dev, with_gate=args.epilogue)
+    if args.fp8_state:  # M0 in the block-scaled fp8 format (the quantiser is one of the library's calls)
+        inp["M0"] = sdm.quantize_fp8blk(inp["M0"].float().contiguous())
     g = inp.get("g")
     y = torch.empty((shape.B, shape.T, shape.H, shape.d_v), dtype=torch.float32, device=dev)
     M_out = torch.empty((shape.B,) + tuple(inp["M0"].shape), dtype=inp["M0"].dtype, device=dev)
     sh = sdm.make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
-                        shape.torch_state(), variant=args.variant, tile=args.tile)
+                        torch.uint8 if args.fp8_state else shape.torch_state(), variant=args.variant, tile=args.tile)
     ws = torch.empty(sdm.layer_forward_workspace_bytes(sh), dtype=torch.uint8, device=dev)
 
     def step(events=None, src=inp):
@@ -473,14 +479,14 @@ def run_sdm(args, dist: Dist):
     resident = sdm.scan_variant(sh) == "resident"
     launches_per_step = int(sdm.native.load().sdm_layer_forward_launches(ctypes.byref(sh), int(args.epilogue)))
     clk = clocks.summary()
-    roof = roofline_of(shape, sh, stage_ms[3], args.epilogue, dev, clk)
+    roof = roofline_of(shape, sh, stage_ms[3], args.epilogue, dev, clk, fp8_state=args.fp8_state)
 
     e2e = None
     if not args.no_e2e:
         e2e = e2e_through_c_abi(args, dist, dev, shape, sh, inp, g, ws, stream)
 
     cpu = None
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline and not args.fp8_state:
         cpu = cpu_baseline(shape, inp, args.cpu_seconds, args.epilogue)
 
     if dist.rank == 0:
@@ -490,6 +496,8 @@ def run_sdm(args, dist: Dist):
         cfg["l2"] = (f"no flush between steps: per-step inputs {in_mb:.0f} MiB and y {d2h_mib(y):.0f} MiB "
                      f"exceed the {l2_mb:.0f} MiB L2")
         cfg["variant"] = sdm.scan_variant(sh)
+        if args.fp8_state:
+            cfg["state_dtype"] = "fp8 E4M3, power-of-two scale per 16 values"
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
@@ -500,18 +508,18 @@ def run_sdm(args, dist: Dist):
     del ev, inp, y, M_out, ws
     torch.cuda.empty_cache()
     if dist.rank == 0:
-        if dist.world == 1 and not args.no_extra and args.workload == DEFAULT_WORKLOAD:
+        if dist.world == 1 and not args.no_extra and args.workload == DEFAULT_WORKLOAD and not args.fp8_state:
             line["extra_workloads"] = {name: measure_workload(name, args, dev) for name in EXTRA_WORKLOADS}
         print(json.dumps(line), flush=True)
     dist.close()
 
 
-def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk: dict) -> dict:
+def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk: dict, fp8_state: bool = False) -> dict:
     """Roofline of the recurrence kernel of one launch: algorithmic bytes over
-    its CUDA-event time against the measured HBM copy bandwidth (streaming),
-    or the derived shared-memory bandwidth (resident)."""
+    its CUDA-event time against the measured HBM copy bandwidth (streaming,
+    pipelined), or the derived shared-memory bandwidth (resident)."""
     resident = sdm.scan_variant(sh) == "resident"
-    algo_bytes = algorithmic_bytes_per_token_head(shape, epilogue) * shape.B * shape.T * shape.H
+    algo_bytes = algorithmic_bytes_per_token_head(shape, epilogue, fp8_state) * shape.B * shape.T * shape.H
     achieved = algo_bytes / (scan_ms / 1e3) / 1e9
     peaks = measured_peaks()
     if resident:

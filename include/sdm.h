@@ -75,9 +75,15 @@ typedef enum sdm_status {
  * power-of-two scale per 16 consecutive values of a state row. A state of
  * R rows of d_v values is R * d_v code bytes followed by R * d_v / 16 int8
  * exponents (value = E4M3(code) * 2^exponent); sdm_quantize_fp8blk builds it
- * from fp32. Only the single-launch decode step (sdm_layer_step with T = 1,
- * W = R <= 64, automatic variant) runs on it; every other call returns
- * SDM_ERR_UNSUPPORTED for it. */
+ * from fp32 (for M0 [H,N,d_v]: H*N rows; M [B,H,N,d_v]: B*H*N rows, so M's
+ * codes of every batch row come first, then their exponents). It runs in the
+ * single-launch decode step (sdm_layer_step with T = 1, W = R <= 64,
+ * automatic variant) and in the pipelined recurrence (sdm_scan,
+ * sdm_layer_forward, sdm_layer_step with T > 1; automatic or pipelined
+ * variant; d_v a multiple of 256, so that a row's exponents fill 16-byte
+ * rows), which applies the write to each decoded 16-value block in fp32 and
+ * re-quantises it exactly as the decode step does. Other variants and the
+ * backward return SDM_ERR_UNSUPPORTED for it. */
 typedef enum sdm_dtype { SDM_F32 = 0, SDM_BF16 = 1, SDM_FP8_B16 = 2 } sdm_dtype_t;
 
 /* Which recurrence kernel runs (sdm_shape_t.variant). */
@@ -358,9 +364,9 @@ SDM_API size_t sdm_layer_step_workspace_bytes(const sdm_shape_t* shape);
  * With the automatic variant, calls with T*(W+R) < N stream only the selected
  * rows (a resident tile would move the whole state), and calls with T = 1 and
  * W = R <= 64 run as one fused launch (both selections, the write, the read
- * and the epilogue). Only that fused form accepts the fp8 state
- * (state_dtype SDM_FP8_B16: M is the code bytes followed by the block
- * exponents, as sdm_quantize_fp8blk writes them). */
+ * and the epilogue). The fp8 state (state_dtype SDM_FP8_B16: M is the code
+ * bytes followed by the block exponents, as sdm_quantize_fp8blk writes them)
+ * runs in that fused form and, for T > 1, in the pipelined recurrence. */
 SDM_API sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, const void* qp,
                             const void* v, const void* alpha, const void* beta, const void* g,
                             void* M, float* y, void* workspace, size_t workspace_bytes, void* stream);

@@ -140,6 +140,7 @@ sdm_status_t need_ptr(const void* p, const char* name, bool nonempty) {
 }
 
 size_t in_size(int32_t d) { return d == SDM_BF16 ? 2 : 4; }
+size_t state_size(int32_t d) { return d == SDM_FP8_B16 ? 1 : in_size(d); }
 
 // The per-token gates are read one element at a time: natural alignment
 // suffices (a one-token slice of [B, T, H] is rarely 16-byte aligned).
@@ -227,6 +228,7 @@ struct PipeCfg {
 constexpr PipeCfg kPipeCfgs[] = {
     {2, 64, 6, 16, 4, 3, 4, 1}, {2, 64, 6, 16, 4, 3, 4, 2}, {2, 64, 7, 8, 4, 3, 4, 2}, {2, 64, 6, 16, 4, 4, 4, 1},
     {2, 64, 6, 16, 4, 3, 2, 1}, {4, 32, 6, 16, 4, 3, 4, 1}, {4, 32, 4, 16, 4, 3, 4, 1}, {4, 32, 6, 16, 4, 3, 4, 2},
+    {1, 64, 6, 16, 4, 3, 4, 1},  // the block-scaled fp8 state: 64 codes (and 4 exponents) a row segment
 };
 
 // Instantiated resident tiles: columns per warp, warps per CTA, staging
@@ -249,8 +251,8 @@ size_t streaming_smem(const sdm_shape_t& s, int C, int P, int L, int NW) {
 }
 size_t pipelined_smem(const sdm_shape_t& s, const PipeCfg& k) {
   const sdm::PipeLayout pl = sdm::pipe_layout(s.W, s.R);
-  return sdm::pipe_smem_bytes(k.P, k.L, pl.Wp, pl.Rp, pl.words, k.C, static_cast<int>(in_size(s.state_dtype)),
-                              static_cast<int>(in_size(s.in_dtype)), k.NWR, k.S);
+  return sdm::pipe_smem_bytes(k.P, k.L, pl.Wp, pl.Rp, pl.words, k.C, static_cast<int>(state_size(s.state_dtype)),
+                              static_cast<int>(in_size(s.in_dtype)), k.NWR, k.S, s.state_dtype == SDM_FP8_B16);
 }
 
 // Whether every row of the pipelined kernel's stage space (gathered and
@@ -270,10 +272,13 @@ constexpr bool kPipelinedAuto = true;
 // (1-based) of the chosen kernel's table among the entries that fit the
 // shape (for measurements); 0 takes the first that fits.
 sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice* out) {
-  if (s.state_dtype == SDM_FP8_B16)
-    return fail(SDM_ERR_UNSUPPORTED,
-                "the fp8 state (SDM_FP8_B16) runs only in the single-launch decode step: sdm_layer_step with "
-                "T = 1, W = R <= 64 and the automatic variant");
+  // The fp8 state runs in the pipelined kernel (and in the single-launch
+  // decode step, chosen before this).
+  const bool fp8 = s.state_dtype == SDM_FP8_B16;
+  if (fp8 && s.variant != SDM_VARIANT_AUTO && s.variant != SDM_VARIANT_PIPELINED)
+    return fail(SDM_ERR_UNSUPPORTED, "the fp8 state (SDM_FP8_B16) runs in the pipelined variant only");
+  if (fp8 && s.d_v % 256 != 0)
+    return fail(SDM_ERR_UNSUPPORTED, "the fp8 state needs d_v a multiple of 256 (16-byte rows of block exponents)");
   const size_t lim = static_cast<size_t>(dev.max_smem_optin);
   auto pick = [&](size_t n_fit) -> int {  // index into the fitting entries, or -1
     if (s.tile == 0) return n_fit > 0 ? 0 : -1;
@@ -284,7 +289,7 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
   // per slot (T * (W + R) < N, e.g. a decode step) streaming only the
   // selected rows moves less.
   const bool few_tokens = static_cast<int64_t>(s.T) * (s.W + s.R) < slots_of(s.sqrt_n);
-  if (s.variant == SDM_VARIANT_RESIDENT || (s.variant == SDM_VARIANT_AUTO && !few_tokens)) {
+  if (!fp8 && (s.variant == SDM_VARIANT_RESIDENT || (s.variant == SDM_VARIANT_AUTO && !few_tokens))) {
     // Resident tiles in order of preference (measured on B200 at N = 1024,
     // d_v = 128: 8-column warp tiles, one warp per CTA, so up to five CTAs
     // share an SM); the first that divides d_v and fits is taken.
@@ -309,7 +314,7 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
       return fail(SDM_ERR_UNSUPPORTED, s.tile == 0 ? "the state tile does not fit in shared memory (resident variant)"
                                                    : "no such resident tile for this shape");
   }
-  const int s_state = static_cast<int>(in_size(s.state_dtype));
+  const int s_state = static_cast<int>(state_size(s.state_dtype));
   const int64_t bh = static_cast<int64_t>(s.B) * s.H;
   // The pipelined kernel when 128-byte column tiles alone would leave SMs
   // idle: one SM moves about one random 128-byte row per 3 ns, so a grid
@@ -318,9 +323,10 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
   const int c128 = 128 / s_state;
   const bool few_tiles = s.d_v % c128 == 0 && bh * (s.d_v / c128) < dev.sms;
   const bool rows_fit = bh * slots_of(s.sqrt_n) <= INT_MAX;  // TMA row coordinates are int32
-  if (s.variant == SDM_VARIANT_PIPELINED && !rows_fit)
+  if ((s.variant == SDM_VARIANT_PIPELINED || fp8) && !rows_fit)
     return fail(SDM_ERR_UNSUPPORTED, "the pipelined variant needs B*H*N below 2^31 state rows");
-  if (rows_fit && (s.variant == SDM_VARIANT_PIPELINED || (s.variant == SDM_VARIANT_AUTO && kPipelinedAuto && few_tiles))) {
+  if (rows_fit && (s.variant == SDM_VARIANT_PIPELINED || fp8 ||
+                   (s.variant == SDM_VARIANT_AUTO && kPipelinedAuto && few_tiles))) {
     std::vector<PipeCfg> order;
     for (const PipeCfg& k : kPipeCfgs)
       if (k.state_bytes == s_state && s.d_v % k.C == 0 && pipelined_smem(s, k) <= lim && pipe_codes_fit(s, k))
@@ -341,7 +347,7 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
       *out = c;
       return SDM_OK;
     }
-    if (s.variant == SDM_VARIANT_PIPELINED)
+    if (s.variant == SDM_VARIANT_PIPELINED || fp8)
       return fail(SDM_ERR_UNSUPPORTED, s.tile == 0 ? "W + R too large for the pipelined stage rings"
                                                    : "no such pipelined tile for this shape");
   }
@@ -425,19 +431,30 @@ sdm_status_t launch_records(const sdm_shape_t& s, const int32_t* idx_w, const fl
   return launch_status("record build launch");
 }
 
-sdm_status_t launch_state_init(const DeviceInfo& dev, const sdm_shape_t& s, const void* M0, void* M, cudaStream_t st) {
-  if (s.state_dtype == SDM_FP8_B16)
-    return fail(SDM_ERR_UNSUPPORTED, "state copies of the fp8 state are not provided (build it with sdm_quantize_fp8blk)");
-  const int64_t bytes_per_row = static_cast<int64_t>(s.H) * slots_of(s.sqrt_n) * s.d_v * static_cast<int64_t>(in_size(s.state_dtype));
-  const int64_t units = bytes_per_row / 16;
-  if (units == 0 || s.B == 0) return SDM_OK;
-  const int gx = static_cast<int>(std::min<int64_t>((units + 255) / 256, std::max(1, dev.sms * 8 / std::max(1, s.B))));
-  for (int b0 = 0; b0 < s.B; b0 += 65535) {
-    const int nb = std::min(65535, s.B - b0);
-    sdm::k_state_init<<<dim3(gx, nb), 256, 0, st>>>(static_cast<const uint4*>(M0),
-                                                   static_cast<uint4*>(M) + static_cast<int64_t>(b0) * units, units);
+// B copies of bytes_per_b bytes (a multiple of 16) of src into dst.
+sdm_status_t copy_per_batch_row(const DeviceInfo& dev, int B, int64_t bytes_per_b, const void* src, void* dst,
+                                cudaStream_t st) {
+  const int64_t units = bytes_per_b / 16;
+  if (units == 0 || B == 0) return SDM_OK;
+  const int gx = static_cast<int>(std::min<int64_t>((units + 255) / 256, std::max(1, dev.sms * 8 / std::max(1, B))));
+  for (int b0 = 0; b0 < B; b0 += 65535) {
+    const int nb = std::min(65535, B - b0);
+    sdm::k_state_init<<<dim3(gx, nb), 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                   static_cast<uint4*>(dst) + static_cast<int64_t>(b0) * units, units);
   }
   return launch_status("state init launch");
+}
+
+// M[b] <- M0 for every batch row. The fp8 state is the codes of all rows,
+// then their exponents: two copies (M0's codes and exponents into M's).
+sdm_status_t launch_state_init(const DeviceInfo& dev, const sdm_shape_t& s, const void* M0, void* M, cudaStream_t st) {
+  const int64_t values = static_cast<int64_t>(s.H) * slots_of(s.sqrt_n) * s.d_v;  // one batch row's state values
+  if (s.state_dtype != SDM_FP8_B16)
+    return copy_per_batch_row(dev, s.B, values * static_cast<int64_t>(in_size(s.state_dtype)), M0, M, st);
+  sdm_status_t r = copy_per_batch_row(dev, s.B, values, M0, M, st);
+  if (r != SDM_OK) return r;
+  return copy_per_batch_row(dev, s.B, values / 16, static_cast<const uint8_t*>(M0) + values,
+                            static_cast<uint8_t*>(M) + static_cast<int64_t>(s.B) * values, st);
 }
 
 sdm_status_t launch_epilogue(const DeviceInfo& dev, const sdm_shape_t& s, float* y, const void* g, cudaStream_t st) {
@@ -1159,7 +1176,8 @@ int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate) 
   // two selections, records, recurrence; the streaming and pipelined recurrences also copy M0
   // first; the pipelined one with two slot parts adds the second part's sums into y after
   const int parts_sum = c.kind == SDM_VARIANT_PIPELINED && c.parts > 1 ? 1 : 0;
-  return 4 + (c.resident ? 0 : 1) + parts_sum + (with_gate ? 1 : 0);
+  const int init = c.resident ? 0 : (shape->state_dtype == SDM_FP8_B16 ? 2 : 1);  // fp8: codes and exponents
+  return 4 + init + parts_sum + (with_gate ? 1 : 0);
 }
 
 sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,

@@ -39,6 +39,7 @@ sdm_status_t launch_status(const char* what);
 // Raises a kernel's dynamic shared-memory limit to at least smem on the current device.
 void set_smem(const void* kern, size_t smem);
 size_t in_size(int32_t dtype);
+size_t state_size(int32_t dtype);  // bytes of one state value (fp8 state: the code byte)
 int64_t slots_of(int32_t sqrt_n);
 
 // The recurrence kernel picked for a shape and its tile.

@@ -51,6 +51,7 @@
 #include <cuda.h>
 
 #include "sdm_device.cuh"
+#include "sdm_fp8.cuh"
 #include "sdm_scan.cuh"
 
 namespace sdm {
@@ -371,7 +372,9 @@ __global__ void __launch_bounds__(256) k_build_pipe_records(
 }
 
 struct PipeArgs {
-  CUtensorMap state_map;  // M as rows [B*H*N, d_v] of the state dtype, box C columns x 1 row
+  CUtensorMap state_map;  // M as rows [B*H*N, d_v] of the state dtype (fp8: code bytes), box C columns x 1 row
+  CUtensorMap exps_map;   // fp8 state: the block exponents as rows [B*H*N, d_v/16] of bytes, box 16 x 1 row
+  int8_t* exps;           // fp8 state: the block exponents [B, H, N, d_v/16] (after the codes)
   int B, T, H, N, d_v, W, R, parts;
   PipeLayout pl;
   const uint32_t* rec;  // [B, H, parts, T, pl.words]
@@ -383,9 +386,17 @@ struct PipeArgs {
 };
 
 // Shared-memory bytes of k_scan_pipelined (host and device agree on this).
+// fp8 state: the block exponents of the stage rows, 16 bytes a row (the TMA
+// box of 16 exponents that covers the row's C columns) in groups of four rows
+// 128 bytes apart (the landing spot of one four-row gather).
+__host__ __device__ constexpr size_t pipe_exp_bytes(int P, int Wp, int Rp, int S) {
+  return static_cast<size_t>((P * (Wp + Rp) + pipe_wstages(P, S) * Wp + 3) / 4) * 128;
+}
+
 __host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
-                                                     int s_in, int NWR, int S) {
+                                                     int s_in, int NWR, int S, bool fp8 = false) {
   return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(pipe_wstages(P, S)) * Wp * C * s_state +
+         (fp8 ? pipe_exp_bytes(P, Wp, Rp, S) : 0) +
          static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in +
          static_cast<size_t>(2) * S * NWR * C * 4 + (2 * P + 2) * 8 + 128;
 }
@@ -420,6 +431,8 @@ __device__ __forceinline__ int reduce_scatter_entries(float (&a)[VE], int lane) 
 template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR, int NP, int S>
 __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipelined(const __grid_constant__ PipeArgs a) {
   constexpr int NT = (NP + 1 + NWW + NWR) * kWarp;
+  constexpr bool kFp8 = std::is_same<Tst, Fp8Blk>::value;  // block-scaled fp8 state: 16 codes and one exponent a unit
+  static_assert(!kFp8 || S == 1, "the fp8 state takes one token per step");
   constexpr int VE = 16 / sizeof(Tst);  // state elements per 16-byte unit
   constexpr int U = C / VE;             // units per row segment
   constexpr int RS = C * sizeof(Tst);   // bytes of a row segment
@@ -437,7 +450,8 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   const int Wp = pl.Wp, E = pl.Wp + pl.Rp, words = pl.words, T = a.T;
   unsigned char* lstage = smem;                                                    // [P][E][RS]
   unsigned char* wstage = lstage + static_cast<size_t>(P) * E * RS;               // [Q][Wp][RS]
-  uint32_t* recbuf = reinterpret_cast<uint32_t*>(wstage + static_cast<size_t>(Q) * Wp * RS);  // [2][L][words]
+  unsigned char* xstage = wstage + static_cast<size_t>(Q) * Wp * RS;              // fp8: exponents of the stage rows
+  uint32_t* recbuf = reinterpret_cast<uint32_t*>(xstage + (kFp8 ? pipe_exp_bytes(P, Wp, pl.Rp, S) : 0));  // [2][L][words]
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
   float* ybuf = reinterpret_cast<float*>(vbuf + 2 * L * C);                        // [2][S][NWR][C] read partials
   uint64_t* cbar = reinterpret_cast<uint64_t*>(ybuf + 2 * S * NWR * C);           // [2] record chunks
@@ -489,15 +503,18 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
     const int nw = static_cast<int>(rec[pl.off_meta]), nr = static_cast<int>(rec[pl.off_meta + 1]);
     const int gw = (nw + 3) / 4, gr = (nr + 3) / 4;
     uint64_t* bar = &full[u % P];
-    if (tid == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(gw + gr) * 4u * RS);
-    unsigned char* st = lstage + static_cast<size_t>(u % P) * E * RS;
+    if (tid == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(gw + gr) * 4u * (RS + (kFp8 ? 16 : 0)));
     const int row0 = bh * a.N;
     for (int g = warp + NP * lane; g < gw + gr; g += NP * kWarp) {
       const bool wr = g < gw;
       const int e = wr ? 4 * g : 4 * (g - gw);
       const uint4 sl = *reinterpret_cast<const uint4*>(rec + (wr ? pl.off_slot_w : pl.off_slot_r) + e);
-      tma_gather4(st + static_cast<size_t>(wr ? e : Wp + e) * RS, &a.state_map, c0, row0 + static_cast<int>(sl.x),
-                  row0 + static_cast<int>(sl.y), row0 + static_cast<int>(sl.z), row0 + static_cast<int>(sl.w), bar);
+      const int r = (u % P) * E + (wr ? e : Wp + e);  // stage row of the group's first row (a multiple of 4)
+      const int r0 = row0 + static_cast<int>(sl.x), r1 = row0 + static_cast<int>(sl.y);
+      const int r2 = row0 + static_cast<int>(sl.z), r3 = row0 + static_cast<int>(sl.w);
+      tma_gather4(lstage + static_cast<size_t>(r) * RS, &a.state_map, c0, r0, r1, r2, r3, bar);
+      // fp8: the 16-exponent box (16-byte aligned) that holds this tile's U exponents
+      if constexpr (kFp8) tma_gather4(xstage + static_cast<size_t>(r >> 2) * 128, &a.exps_map, (c0 / 16) & ~15, r0, r1, r2, r3, bar);
     }
   };
   int last_gathered = -1;  // producer threads: the last token whose rows they requested
@@ -526,6 +543,46 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   const int base_w = cw * kWarp + lane;
   const int base_r = (cw - NWW) * G + lane / U;
   auto row_at = [&](uint32_t src) { return *reinterpret_cast<const uint4*>(smem + static_cast<size_t>(src) * RS + qw * 16); };
+  // The state as fp32 and back, per 16-byte unit: bf16 / fp32 by bits, the
+  // fp8 state with the unit's block exponent (this tile's U exponents sit at
+  // xoff .. xoff + U - 1 of a row's 16-byte exponent box).
+  const int xoff = (c0 / 16) & 15;
+  auto exp_byte = [&](uint32_t row) -> unsigned char& {
+    return xstage[static_cast<size_t>(row >> 2) * 128 + (row & 3) * 16 + xoff + qw];
+  };
+  auto load_row = [&](uint32_t src, float (&m)[VE]) {
+    if constexpr (kFp8) fp8blk_unpack16(row_at(src), static_cast<int8_t>(exp_byte(src)), m);
+    else unpack_unit<Tst>(row_at(src), m);
+  };
+  auto as_stored = [&](float (&m)[VE]) {  // m rounded as the state holds it
+    if constexpr (kFp8) {
+      uint4 q;
+      const int e = fp8blk_pack16(m, &q);
+      fp8blk_unpack16(q, e, m);
+    } else {
+      unpack_unit<Tst>(pack16<Tst>(m), m);
+    }
+  };
+  int8_t* Mx = kFp8 ? a.exps + static_cast<int64_t>(bh) * a.N * (a.d_v / 16) + c0 / 16 + qw : nullptr;
+  // m, rounded to the state type, into written-stage row wrow and, unless
+  // slot < 0, into the state in HBM
+  auto store_row = [&](const float (&m)[VE], uint32_t wrow, int64_t slot) {
+    unsigned char* dst = smem + static_cast<size_t>(wrow) * RS + qw * 16;
+    if constexpr (kFp8) {
+      uint4 q;
+      const int e = fp8blk_pack16(m, &q);
+      *reinterpret_cast<uint4*>(dst) = q;
+      exp_byte(wrow) = static_cast<unsigned char>(static_cast<int8_t>(e));
+      if (slot >= 0) {
+        *reinterpret_cast<uint4*>(Mbh + qw * VE + slot * a.d_v) = q;
+        Mx[slot * (a.d_v / 16)] = static_cast<int8_t>(e);
+      }
+    } else {
+      const uint4 pk = pack16<Tst>(m);
+      *reinterpret_cast<uint4*>(dst) = pk;
+      if (slot >= 0) *reinterpret_cast<uint4*>(Mbh + qw * VE + slot * a.d_v) = pk;
+    }
+  };
   // Token t on this consumer thread. Every row it reads is complete: the
   // token's gathered stage and the written stages of the tokens before it.
   auto compute = [&](int t) {
@@ -537,13 +594,12 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
     load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((t / L) & 1) * L + t % L) * C + qw * VE, vv);
     // the write of entry j on this thread's unit of its source row (fp32 math, state rounding by the caller)
     auto written = [&](int j, float (&m)[VE]) {
-      unpack_unit<Tst>(row_at(sw[j] & kRowMask), m);
+      load_row(sw[j] & kRowMask, m);
       const float2 c = ac[j];
       write_unit<VE>(m, vv, c.x, c.y);
     };
     if (writer) {
-      unsigned char* ws = wstage + static_cast<size_t>(t % Q) * Wp * RS + qw * 16;
-      Tst* Mq = Mbh + qw * VE;
+      const uint32_t wbase = static_cast<uint32_t>(P * E + (t % Q) * Wp);  // this token's written stage
       const uint32_t* slw = rec + pl.off_slot_w;
       const int n = nw * U;
       for (int p0 = base_w; p0 < n; p0 += 2 * stride_w) {  // two independent units per pass
@@ -553,13 +609,8 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
         float m0[VE], m1[VE];
         written(j0, m0);
         written(j1, m1);
-        const uint4 k0 = pack16<Tst>(m0), k1 = pack16<Tst>(m1);
-        *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j0) * RS) = k0;
-        *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slw[j0]) * a.d_v) = k0;
-        if (has1) {
-          *reinterpret_cast<uint4*>(ws + static_cast<size_t>(j1) * RS) = k1;
-          *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slw[j1]) * a.d_v) = k1;
-        }
+        store_row(m0, wbase + j0, slw[j0]);
+        if (has1) store_row(m1, wbase + j1, slw[j1]);
       }
     } else {
       const uint16_t* sr = reinterpret_cast<const uint16_t*>(rec + pl.off_src_r);
@@ -567,7 +618,7 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
       // a read of a slot this token writes: that write, rounded as stored
       auto same_token = [&](uint32_t src, float (&m)[VE]) {
         written(static_cast<int>(src & kEntryMask), m);
-        unpack_unit<Tst>(pack16<Tst>(m), m);
+        as_stored(m);
       };
       float acc[VE];
 #pragma unroll
@@ -579,8 +630,8 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
         // both rows first (a flagged code's low bits still name a row in
         // shared memory), the rare recomputation after: no branch between them
         float m0[VE], m1[VE];
-        unpack_unit<Tst>(row_at(src0 & kRowMask), m0);
-        unpack_unit<Tst>(row_at(src1 & kRowMask), m1);
+        load_row(src0 & kRowMask, m0);
+        load_row(src1 & kRowMask, m1);
         if ((src0 | src1) & kSrcSameToken) {
           if (src0 & kSrcSameToken) same_token(src0, m0);
           if (src1 & kSrcSameToken) same_token(src1, m1);
@@ -611,7 +662,7 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
     load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>((ta / L) & 1) * L + ta % L) * C + qw * VE, vA);
     load_in_vec<Tin, VE>(vbuf + (static_cast<size_t>(((hb ? tb : ta) / L) & 1) * L + (hb ? tb : ta) % L) * C + qw * VE, vB);
     auto writtenA = [&](int j, float (&m)[VE]) {  // the first token's write j (unrounded)
-      unpack_unit<Tst>(row_at(swA[j] & kRowMask), m);
+      load_row(swA[j] & kRowMask, m);
       const float2 c = acA[j];
       write_unit<VE>(m, vA, c.x, c.y);
     };
@@ -619,17 +670,16 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
       const uint32_t src = swB[j];
       if (src & kSrcPrevToken) {
         writtenA(static_cast<int>(src & kEntryMask), m);
-        unpack_unit<Tst>(pack16<Tst>(m), m);
+        as_stored(m);
       } else {
-        unpack_unit<Tst>(row_at(src & kRowMask), m);
+        load_row(src & kRowMask, m);
       }
       const float2 c = acB[j];
       write_unit<VE>(m, vB, c.x, c.y);
     };
     if (writer) {
-      unsigned char* wsA = wstage + static_cast<size_t>(ta % Q) * Wp * RS + qw * 16;
-      unsigned char* wsB = wstage + static_cast<size_t>(tb % Q) * Wp * RS + qw * 16;
-      Tst* Mq = Mbh + qw * VE;
+      const uint32_t wbA = static_cast<uint32_t>(P * E + (ta % Q) * Wp);  // the two tokens' written stages
+      const uint32_t wbB = static_cast<uint32_t>(P * E + (tb % Q) * Wp);
       const uint32_t* slwA = recA + pl.off_slot_w;
       const uint32_t* slwB = recB + pl.off_slot_w;
       const int nA = static_cast<int>(recA[pl.off_meta]) * U;
@@ -645,14 +695,14 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
         for (int k = 0; k < kTokW; ++k) {
           j[k] = min((p0 + k * stride_w) / U, Wp - 1);
           srcB[k] = swB[j[k]];
-          unpack_unit<Tst>(row_at(swA[j[k]] & kRowMask), mA[k]);
-          unpack_unit<Tst>(row_at(srcB[k] & kRowMask), mB[k]);
+          load_row(swA[j[k]] & kRowMask, mA[k]);
+          load_row(srcB[k] & kRowMask, mB[k]);
         }
 #pragma unroll
         for (int k = 0; k < kTokW; ++k) {
           if (srcB[k] & kSrcPrevToken) {  // rare: the first token's write of the slot, as stored
             writtenA(static_cast<int>(srcB[k] & kEntryMask), mB[k]);
-            unpack_unit<Tst>(pack16<Tst>(mB[k]), mB[k]);
+            as_stored(mB[k]);
           }
         }
 #pragma unroll
@@ -664,16 +714,9 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
 #pragma unroll
         for (int k = 0; k < kTokW; ++k) {
           const int p = p0 + k * stride_w;
-          if (p < nA) {
-            const uint4 pk = pack16<Tst>(mA[k]);
-            *reinterpret_cast<uint4*>(wsA + static_cast<size_t>(j[k]) * RS) = pk;
-            if (!(swA[j[k]] & kSkipStore)) *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slwA[j[k]]) * a.d_v) = pk;
-          }
-          if (p < nB) {
-            const uint4 pk = pack16<Tst>(mB[k]);
-            *reinterpret_cast<uint4*>(wsB + static_cast<size_t>(j[k]) * RS) = pk;
-            *reinterpret_cast<uint4*>(Mq + static_cast<int64_t>(slwB[j[k]]) * a.d_v) = pk;
-          }
+          if (p < nA)
+            store_row(mA[k], wbA + j[k], (swA[j[k]] & kSkipStore) ? int64_t{-1} : static_cast<int64_t>(slwA[j[k]]));
+          if (p < nB) store_row(mB[k], wbB + j[k], slwB[j[k]]);
         }
       }
     } else {
@@ -695,19 +738,19 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
           i[k] = min(i0 + k * stride_r, pl.Rp - 1);
           sA[k] = srA[i[k]];
           sB[k] = srB[i[k]];
-          unpack_unit<Tst>(row_at(sA[k] & kRowMask), mA[k]);
-          unpack_unit<Tst>(row_at(sB[k] & kRowMask), mB[k]);
+          load_row(sA[k] & kRowMask, mA[k]);
+          load_row(sB[k] & kRowMask, mB[k]);
         }
 #pragma unroll
         for (int k = 0; k < kTokR; ++k) {  // rare: reads of rows this step writes, as stored
           if (sA[k] & kSrcSameToken) {
             writtenA(static_cast<int>(sA[k] & kEntryMask), mA[k]);
-            unpack_unit<Tst>(pack16<Tst>(mA[k]), mA[k]);
+            as_stored(mA[k]);
           }
           if (sB[k] & (kSrcSameToken | kSrcPrevToken)) {
             if (sB[k] & kSrcSameToken) writtenB(static_cast<int>(sB[k] & kEntryMask), mB[k]);
             else writtenA(static_cast<int>(sB[k] & kEntryMask), mB[k]);
-            unpack_unit<Tst>(pack16<Tst>(mB[k]), mB[k]);
+            as_stored(mB[k]);
           }
         }
 #pragma unroll

@@ -3,6 +3,7 @@
 #include <algorithm>
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "sdm_host.h"
 
@@ -51,7 +52,9 @@ sdm_status_t launch_pipe_typed(const ScanChoice& c, const sdm::PipeArgs& a, cuda
 #define SDM_PIPE(C_, P_, L_, NWW_, NWR_, NP_, S_)                                                          \
   if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_ && c.NP == NP_ && c.S == S_)      \
     kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_, NP_, S_>;
-  if constexpr (sizeof(Tst) == 2) {
+  if constexpr (std::is_same<Tst, sdm::Fp8Blk>::value) {
+    SDM_PIPE(64, 6, 16, 4, 3, 4, 1)
+  } else if constexpr (sizeof(Tst) == 2) {
     SDM_PIPE(64, 6, 16, 4, 3, 4, 1) SDM_PIPE(64, 6, 16, 4, 3, 4, 2) SDM_PIPE(64, 7, 8, 4, 3, 4, 2)
     SDM_PIPE(64, 6, 16, 4, 4, 4, 1) SDM_PIPE(64, 6, 16, 4, 3, 2, 1)
   } else {
@@ -72,15 +75,31 @@ sdm_status_t launch_pipe(const ScanChoice& c, const sdm_shape_t& s, const sdm::P
   if (rows > static_cast<uint64_t>(INT_MAX)) return fail(SDM_ERR_UNSUPPORTED, "B*H*N above 2^31 - 1 state rows");
   const EncodeTiledFn encode = encode_tiled();
   if (encode == nullptr) return fail(SDM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const bool fp8 = s.state_dtype == SDM_FP8_B16;
   const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.d_v), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.d_v) * in_size(s.state_dtype)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.d_v) * state_size(s.state_dtype)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(c.C), 1u}, estride[2] = {1u, 1u};
-  const CUresult e = encode(&a.state_map, s.state_dtype == SDM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                            2, a.M, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                     : (s.state_dtype == SDM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+  CUresult e = encode(&a.state_map, dt, 2, a.M, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (e != CUDA_SUCCESS) return fail(SDM_ERR_CUDA, "cuTensorMapEncodeTiled failed with " + std::to_string(e));
+  if (fp8) {
+    // The block exponents after the codes: rows of d_v/16 bytes (a multiple
+    // of 16: d_v % 256 == 0, checked by the chooser); one box is the 16
+    // exponents of 256 columns, 16-byte aligned, that hold a tile's C/16.
+    a.exps = reinterpret_cast<int8_t*>(static_cast<uint8_t*>(a.M) + rows * a.d_v);
+    const cuuint64_t xdim[2] = {static_cast<cuuint64_t>(a.d_v / 16), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t xstride[1] = {static_cast<cuuint64_t>(a.d_v / 16)};
+    const cuuint32_t xbox[2] = {16u, 1u};
+    e = encode(&a.exps_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.exps, xdim, xstride, xbox, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (e != CUDA_SUCCESS) return fail(SDM_ERR_CUDA, "cuTensorMapEncodeTiled (exponents) failed with " + std::to_string(e));
+    return s.in_dtype == SDM_BF16 ? launch_pipe_typed<bf16, sdm::Fp8Blk>(c, a, st)
+                                  : launch_pipe_typed<float, sdm::Fp8Blk>(c, a, st);
+  }
   if (s.in_dtype == SDM_BF16)
     return s.state_dtype == SDM_BF16 ? launch_pipe_typed<bf16, bf16>(c, a, st) : launch_pipe_typed<bf16, float>(c, a, st);
   return s.state_dtype == SDM_BF16 ? launch_pipe_typed<float, bf16>(c, a, st) : launch_pipe_typed<float, float>(c, a, st);

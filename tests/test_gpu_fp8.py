@@ -157,3 +157,96 @@ def test_decode_fp8_state_error_against_exact_recurrence(sdm, oracle, cuda_devic
         worst = max(worst, float(np.abs(y - oy).max() / max(np.abs(oy).max(), 1e-30)))
     # the fp8 state's read error, relative to the largest read value, stays at the format's precision
     assert worst < 0.25, worst
+
+
+# ---- the fp8 state in whole-sequence calls (sdm_layer_forward, pipelined kernel)
+
+def _whole_setup(oracle, seed, T, W, sqrt_n=8):
+    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"].replace(B=2, T=T, H=2, sqrt_n=sqrt_n, d_v=256, W=W, R=W)
+    inp = synth.make_inputs(shape, seed=seed, device="cpu")
+    M0 = f32(inp["M0"])
+    c0, e0 = oracle.quantize_fp8blk(M0)  # M0 [H, N, d_v] as the fp8 state
+    return shape, inp, c0, e0
+
+
+@pytest.mark.parametrize("T,W", [(1, 16), (37, 16), (64, 64), (150, 24)])
+def test_whole_sequence_fp8_state_equals_chained_decode_steps(sdm, oracle, cuda_device, T, W):
+    """One sdm_layer_forward over T tokens on the fp8 state (pipelined kernel)
+    leaves the state bit for bit where T single-token decode steps leave it:
+    both decode a unit with its block exponent, write it in fp32 with the same
+    operations and re-quantise it with the same rule. y differs only in the
+    order of the fp32 read sums. With N = 64 slots and W = R up to 64, slots
+    collide within and across tokens all the time."""
+    shape, inp, c0, e0 = _whole_setup(oracle, 60 + T, T, W)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    M0 = _buf(c0, e0, cuda_device)
+    y_full, M_full = sdm.layer_forward(d["kp"], d["qp"], d["v"], d["alpha"], d["beta"], M0, shape.W, shape.R)
+    sdm.stream_check()
+    assert sdm.scan_variant(sdm.make_shape(shape.B, T, shape.H, shape.sqrt_n, W, W, shape.d_v, torch.bfloat16,
+                                           torch.uint8)) == "pipelined"
+    # the decode chain starts from M0 in every batch row (codes of all rows, then their exponents)
+    cb = np.broadcast_to(c0[None], (shape.B,) + c0.shape)
+    eb = np.broadcast_to(e0[None], (shape.B,) + e0.shape)
+    buf = _buf(cb, eb, cuda_device)
+    ys = [_gpu_step(sdm, d, t, buf, shape) for t in range(T)]
+    assert torch.equal(M_full.reshape(-1), buf), "state differs from the chained decode steps"
+    y_chain = np.concatenate(ys, axis=1)
+    got = y_full.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(got, y_chain, rtol=1e-5, atol=1e-6 * np.abs(y_chain).max())
+
+
+def test_whole_sequence_fp8_state_error_against_exact_recurrence(sdm, oracle, cuda_device):
+    """The whole-sequence call against the unrounded double recurrence from the
+    same decoded start, with the compounding bound of the module docstring
+    checked on every token's y and on the final state."""
+    shape, inp, c0, e0 = _whole_setup(oracle, 71, 24, 32, sqrt_n=16)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    y_full, M_full = sdm.layer_forward(d["kp"], d["qp"], d["v"], d["alpha"], d["beta"], _buf(c0, e0, cuda_device),
+                                       shape.W, shape.R)
+    sdm.stream_check()
+    y_full = y_full.cpu().numpy().astype(np.float64)
+    idx_w, w_w = oracle.pkm_topk(f32(inp["kp"]), shape.W)
+    idx_r, w_r = oracle.pkm_topk(f32(inp["qp"]), shape.R)
+    v, alpha, beta = (f32(inp[k]).astype(np.float64) for k in ("v", "alpha", "beta"))
+    D0 = _dequant(oracle, c0, e0)
+    M = np.ascontiguousarray(np.broadcast_to(D0[None], (shape.B,) + D0.shape))
+    E = np.zeros_like(M)
+    for t in range(shape.T):
+        sl = slice(t, t + 1)
+        M_old = M
+        oy, M = oracle.scan_f64(idx_w[:, sl], w_w[:, sl], idx_r[:, sl], w_r[:, sl], v[:, sl], alpha[:, sl],
+                                beta[:, sl], M_old)
+        E_new = E.copy()
+        for b in range(shape.B):
+            for h in range(shape.H):
+                a_t, b_t = alpha[b, t, h], beta[b, t, h]
+                for j, i in enumerate(idx_w[b, t, h]):
+                    cw = b_t * w_w[b, t, h, j]
+                    aw = a_t * (1.0 - cw)
+                    carried = aw * E[b, h, i]
+                    slack = FP32_SLACK * (aw * (np.abs(M_old[b, h, i]) + E[b, h, i]) + cw * np.abs(v[b, t, h]))
+                    E_new[b, h, i] = carried + slack + _half_step_bound(np.abs(M[b, h, i]) + carried + slack)
+        E = E_new
+        for b in range(shape.B):
+            for h in range(shape.H):
+                q = np.abs(w_r[b, t, h])[:, None]
+                rows = idx_r[b, t, h]
+                bound = (q * E[b, h, rows]).sum(0) + 4 * FP32_SLACK * (q * (np.abs(M[b, h, rows]) + E[b, h, rows])).sum(0)
+                dy = np.abs(y_full[b, t, h] - oy[b, 0, h])
+                assert np.all(dy <= bound + 1e-30), ("y", t, b, h, float((dy - bound).max()))
+    n = shape.B * shape.H * shape.N * shape.d_v
+    got = M_full.reshape(-1).cpu().numpy()
+    Dk = _dequant(oracle, got[:n].reshape(M.shape), got[n:].view(np.int8).reshape(M.shape[:-1] + (shape.d_v // 16,)))
+    err = np.abs(Dk - M)
+    assert np.all(err <= E), ("state", float((err - E).max()))
+
+
+def test_whole_sequence_fp8_state_rejected_where_unsupported(sdm, cuda_device):
+    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"].replace(B=1, T=4, H=1, sqrt_n=8, d_v=128, W=8, R=8)
+    inp = synth.make_inputs(shape, seed=1, device=cuda_device)
+    M0 = sdm.quantize_fp8blk(inp["M0"].float().contiguous())
+    with pytest.raises(sdm.SdmError, match="multiple of 256"):  # 16-byte exponent rows
+        sdm.layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], M0, shape.W, shape.R)
+    with pytest.raises(sdm.SdmError, match="pipelined variant only"):
+        sdm.layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], M0, shape.W, shape.R,
+                          variant="streaming")
