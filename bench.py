@@ -755,8 +755,50 @@ def run_backward(args, dist: Dist):
                              "algorithmic_bytes_per_launch": algo, "ms_per_launch": scan_ms,
                              "peak_source": f"derived: SMs x {SMEM_BYTES_PER_CLK_PER_SM} B/clk x {mhz:.0f} MHz"},
                 "gpu_launches": 4 * args.steps, "clocks": clk}
+        if dist.world == 1:
+            ck = checkpoint_comparison(shape, inp, dy, dev, stream, max(2, args.steps // 2))
+            if ck is not None:
+                line["with_forward_checkpoints"] = ck
         print(json.dumps(line), flush=True)
     dist.close()
+
+
+def _device_ms(fn, stream, reps: int) -> float:
+    """Mean CUDA-event time of fn() over reps calls (after one untimed call)."""
+    fn()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(reps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / reps
+
+
+def checkpoint_comparison(shape, inp, dy, dev, stream, reps: int):
+    """The whole layer's forward and backward (sdm_layer_forward,
+    sdm_layer_backward), with the forward storing the backward's checkpoints
+    and without: the forward's extra cost and the backward's saving. None
+    where the forward does not store checkpoints for this shape."""
+    sh = sdm.make_shape(shape.B, shape.T, shape.H, shape.sqrt_n, shape.W, shape.R, shape.d_v, shape.torch_in(),
+                        torch.float32)
+    try:
+        chunk, nbytes = sdm.layer_checkpoint_size(sh)
+    except sdm.SdmError:
+        return None
+    M0 = inp["M0"].float().contiguous()
+    args = (inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], M0, shape.W, shape.R)
+    box = {}
+    fwd_ms = _device_ms(lambda: sdm.layer_forward(*args), stream, reps)
+    fwd_ck_ms = _device_ms(lambda: box.__setitem__("ck", sdm.layer_forward_ckpt(*args)[2]), stream, reps)
+    bwd_ms = _device_ms(lambda: sdm.layer_backward(*args[:6], dy, shape.W, shape.R), stream, reps)
+    bwd_ck_ms = _device_ms(lambda: sdm.layer_backward(*args[:6], dy, shape.W, shape.R, checkpoints=box["ck"]),
+                           stream, reps)
+    sdm.stream_check(dev)
+    return {"checkpoint_tokens": chunk, "checkpoint_bytes": nbytes, "layer_forward_ms": fwd_ms,
+            "layer_forward_ckpt_ms": fwd_ck_ms, "layer_backward_ms": bwd_ms, "layer_backward_ckpt_ms": bwd_ck_ms,
+            "note": "device time per call, CUDA events; the backward given the forward's checkpoints skips its "
+                    "first pass over the tokens"}
 
 
 def run_slot_counts(args, dist: Dist):

@@ -282,6 +282,34 @@ SDM_API sdm_status_t sdm_layer_backward(const sdm_shape_t* shape, const void* kp
                                 float* dv, float* dalpha, float* dbeta, float* dg, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Checkpoints of the recurrence for a later backward of the same call, so
+ * that the backward need not recompute them ([explainer] 3.4: the memory-
+ * efficient backward recomputes the forward from stored states): the state
+ * before tokens C, 2C, ..., (n-1)C, n = ceil(T / C), as [n-1][B,H,N,d_v]
+ * fp32, where C (*chunk_tokens) is the checkpoint chunk sdm_layer_backward
+ * uses for this shape. Sets *bytes (0 when T <= C). SDM_ERR_UNSUPPORTED when
+ * the forward does not store them for this shape: only the resident
+ * recurrence with an fp32 state does (the backward then recomputes them). */
+SDM_API sdm_status_t sdm_layer_checkpoint_size(const sdm_shape_t* shape, int32_t* chunk_tokens, size_t* bytes);
+
+/* sdm_layer_forward that also writes those checkpoints into ckpt (device,
+ * 16-byte aligned, at least the bytes sdm_layer_checkpoint_size reports;
+ * caller owned). Same results as sdm_layer_forward, bit for bit. */
+SDM_API sdm_status_t sdm_layer_forward_ckpt(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                    const void* alpha, const void* beta, const void* g, const void* M0,
+                                    void* M_out, float* y, float* ckpt, size_t ckpt_bytes, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* sdm_layer_backward given the checkpoints sdm_layer_forward_ckpt stored for
+ * the same inputs (or NULL: recompute them): the recurrence backward then
+ * skips its first pass over the tokens. Same results, bit for bit (the
+ * forward's states are the states the backward recomputes). */
+SDM_API sdm_status_t sdm_layer_backward_ckpt(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                     const void* alpha, const void* beta, const void* g, const float* M0,
+                                     const float* y_pre, const float* dy, float* dM, float* dkp, float* dqp,
+                                     float* dv, float* dalpha, float* dbeta, float* dg, const float* ckpt,
+                                     size_t ckpt_bytes, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Backward of the selection weights of sdm_pkm_topk for a fixed selection
  * ([explainer] 3.1 step 1: w = softmax of the K selected sums
  * sigma_k = s1[a_k] + s2[b_k], slot a_k * sqrt_n + b_k):

@@ -22,7 +22,7 @@ from .native import SdmError
 
 __all__ = ["pkm_topk", "scan", "state_init", "layer_forward", "layer_step", "slot_counts", "scan_describe",
            "scan_backward", "pkm_topk_backward", "rmsnorm_gate", "rmsnorm_gate_backward", "layer_backward",
-           "quantize_fp8blk", "fp8blk_parts", "stream_check", "make_shape",
+           "quantize_fp8blk", "fp8blk_parts", "stream_check", "make_shape", "layer_checkpoint_size", "layer_forward_ckpt",
            "scan_workspace_bytes", "layer_forward_workspace_bytes", "scan_variant", "SdmError", "synth", "native"]
 
 _DTYPE = {torch.float32: native.F32, torch.bfloat16: native.BF16,
@@ -208,13 +208,43 @@ def rmsnorm_gate_backward(y_pre: torch.Tensor, g: torch.Tensor, dout: torch.Tens
     return dy_pre, dg
 
 
+def layer_checkpoint_size(shape: native.Shape) -> tuple[int, int]:
+    """(chunk tokens C, bytes) of the checkpoints sdm_layer_forward_ckpt stores
+    for a later backward of this shape; raises SdmError where the forward does
+    not store them."""
+    chunk, nbytes = ctypes.c_int32(0), ctypes.c_size_t(0)
+    native.check(native.load().sdm_layer_checkpoint_size(ctypes.byref(shape), ctypes.byref(chunk), ctypes.byref(nbytes)))
+    return int(chunk.value), int(nbytes.value)
+
+
+def layer_forward_ckpt(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float = 1e-6,
+                       workspace: torch.Tensor | None = None):
+    """layer_forward that also stores the backward's checkpoints (the state
+    before every chunk of C tokens after the first, [n-1,B,H,N,d_v] fp32).
+    Returns (y, M_out, checkpoints)."""
+    B, T, H, two_n = kp.shape
+    d_v = v.shape[-1]
+    shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M0, "M0"), eps, 0, 0)
+    lib = native.load()
+    chunk, nbytes = layer_checkpoint_size(shape)
+    y = torch.empty((B, T, H, d_v), dtype=torch.float32, device=kp.device)
+    M_out = torch.empty((B,) + tuple(M0.shape), dtype=M0.dtype, device=kp.device)
+    ckpt = torch.empty((max(nbytes, 16) // 4,), dtype=torch.float32, device=kp.device)
+    ws = _workspace(layer_forward_workspace_bytes(shape), kp.device, workspace)
+    native.check(lib.sdm_layer_forward_ckpt(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha), _ptr(beta),
+                                            _ptr(g), _ptr(M0), _ptr(M_out), _ptr(y), _ptr(ckpt), nbytes, _ptr(ws),
+                                            ws.numel() * ws.element_size(), _stream(kp.device)))
+    return y, M_out, ckpt[:nbytes // 4]
+
+
 def layer_backward(kp, qp, v, alpha, beta, M0, dy, W: int, R: int, g=None, y_pre=None, dM=None, eps: float = 1e-6,
-                   workspace: torch.Tensor | None = None) -> dict:
+                   workspace: torch.Tensor | None = None, checkpoints: torch.Tensor | None = None) -> dict:
     """Derivatives of the layer (selection, recurrence, optional epilogue)
     for dy = dL/d(output) and dM = dL/dM_T (zeros when None); M0 [H,N,d_v]
     fp32 is the shared initial state; y_pre (the output before the epilogue)
     is needed with g. Returns dkp, dqp, dv, dalpha, dbeta, dM0 (per batch row)
-    and, with g, dg (all fp32)."""
+    and, with g, dg (all fp32). ``checkpoints``: the ones layer_forward_ckpt
+    stored for the same inputs (the backward then skips recomputing them)."""
     B, T, H, two_n = kp.shape
     d_v = v.shape[-1]
     N = M0.shape[-2]
@@ -232,10 +262,12 @@ def layer_backward(kp, qp, v, alpha, beta, M0, dy, W: int, R: int, g=None, y_pre
     if need == 0:
         raise native.SdmError(2, lib.sdm_last_error().decode(errors="replace"))
     ws = _workspace(need, dev, workspace)
-    native.check(lib.sdm_layer_backward(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha), _ptr(beta),
-                                        _ptr(g), _ptr(M0), _ptr(y_pre), _ptr(dy), _ptr(dM), _ptr(out["dkp"]),
-                                        _ptr(out["dqp"]), _ptr(out["dv"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]),
-                                        _ptr(out.get("dg")), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev)))
+    ck_bytes = 0 if checkpoints is None else checkpoints.numel() * checkpoints.element_size()
+    native.check(lib.sdm_layer_backward_ckpt(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha),
+                                             _ptr(beta), _ptr(g), _ptr(M0), _ptr(y_pre), _ptr(dy), _ptr(dM),
+                                             _ptr(out["dkp"]), _ptr(out["dqp"]), _ptr(out["dv"]), _ptr(out["dalpha"]),
+                                             _ptr(out["dbeta"]), _ptr(out.get("dg")), _ptr(checkpoints), ck_bytes,
+                                             _ptr(ws), ws.numel() * ws.element_size(), _stream(dev)))
     out["dM0"] = dM
     return out
 

@@ -483,7 +483,7 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
                       const float* w_w, const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
                       const void* beta, const void* g, const void* M_in, int64_t M_in_b_stride, void* M, float* y,
                       uint32_t* rec, cudaStream_t st, const Trace& tr = Trace(), bool init_before_scan = false,
-                      const void* M0_for_init = nullptr) {
+                      const void* M0_for_init = nullptr, float* ckpt = nullptr, int ckpt_C = 0) {
   sdm_status_t r;
   if (c.kind == SDM_VARIANT_PIPELINED) {
     if ((r = launch_pipe_records(s, c, idx_w, w_w, idx_r, w_r, alpha, beta, rec, nullptr, dev, st)) != SDM_OK)
@@ -539,6 +539,8 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
   a.M_in_b_stride = M_in_b_stride;
   a.M = M;
   a.y = y;
+  a.ckpt = ckpt;
+  a.ckpt_C = ckpt_C;
   a.err = dev.err;
   if ((r = launch_scan(c, s, a, st)) != SDM_OK) return r;
   tr.mark(4, st);
@@ -666,6 +668,165 @@ sdm_status_t try_decode_step(const DeviceInfo& dev, const sdm_shape_t& s, const 
 
 }  // namespace
 
+namespace sdm_host {
+// sdm_scan_backward, optionally with the forward's checkpoints (ckpt_ext:
+// [ceil(T / C) - 1][B,H,N,d_v] fp32 for this shape's backward chunk C), which
+// replace the backward's own first pass.
+sdm_status_t scan_backward_impl(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w,
+                                const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
+                                const void* beta, const float* M_in, int32_t m_in_shared, const float* dy, float* dM,
+                                float* dv, float* dalpha, float* dbeta, float* dw_w, float* dw_r, void* workspace,
+                                size_t workspace_bytes, void* stream, const float* ckpt_ext) {
+  sdm_status_t r;
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  BwdChoice c;
+  if ((r = choose_bwd(s, &c)) != SDM_OK) return r;
+  const bool any = static_cast<int64_t>(s.B) * s.H > 0;
+  const bool tok = static_cast<int64_t>(s.B) * s.T * s.H > 0;
+  if ((r = need_ptr(idx_w, "idx_w", tok)) || (r = need_ptr(w_w, "w_w", tok)) || (r = need_ptr(idx_r, "idx_r", tok)) ||
+      (r = need_ptr(w_r, "w_r", tok)) || (r = need_ptr(v, "v", tok)) || (r = need_gate(alpha, "alpha", tok, s.in_dtype)) ||
+      (r = need_gate(beta, "beta", tok, s.in_dtype)) || (r = need_ptr(M_in, "M_in", any)) ||
+      (r = need_ptr(dy, "dy", tok)) || (r = need_ptr(dM, "dM", any)) || (r = need_ptr(dv, "dv", tok)) ||
+      (r = need_gate(dalpha, "dalpha", tok, SDM_F32)) || (r = need_gate(dbeta, "dbeta", tok, SDM_F32)) ||
+      (r = need_ptr(dw_w, "dw_w", tok)) || (r = need_ptr(dw_r, "dw_r", tok)))
+    return r;
+  if (!any) return ok();
+  const size_t need = c.total();
+  if (workspace_bytes < need)
+    return fail(SDM_ERR_INVALID_ARGUMENT,
+                "workspace_bytes below sdm_scan_backward_workspace_bytes() = " + std::to_string(need));
+  if ((r = need_ptr(workspace, "workspace", need > 0)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  if (static_cast<size_t>(dev->max_smem_optin) < c.smem)
+    return fail(SDM_ERR_UNSUPPORTED, "the device's shared memory per block is below the backward tile's");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t N = slots_of(s.sqrt_n);
+  if (s.T == 0) return ok();  // dL/dM_0 = dL/dM_T, already in dM
+  sdm::BwdArgs a;
+  a.B = s.B; a.T = s.T; a.H = s.H; a.N = static_cast<int>(N); a.d_v = s.d_v; a.W = s.W; a.R = s.R;
+  a.C = c.C; a.ntile = c.ntile;
+  a.rl = rec_layout(s.W, s.R, false);
+  a.v = v;
+  a.M_in = M_in;
+  a.M_in_b_stride = m_in_shared ? 0 : static_cast<int64_t>(s.H) * N * s.d_v;
+  a.dy = dy; a.dM = dM; a.dv = dv;
+  char* ws = static_cast<char*>(workspace);
+  a.part = reinterpret_cast<float*>(ws);
+  a.ckpt = reinterpret_cast<float*>(ws + c.part_bytes);
+  a.logbuf = reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes);
+  uint32_t* rec = reinterpret_cast<uint32_t*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes);
+  a.rec = rec;
+  a.Mwork = c.global ? reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes + c.rec_bytes) : nullptr;
+  a.ckpt_ext = ckpt_ext;
+  a.err = dev->err;
+  if (s.in_dtype == SDM_BF16) {
+    if ((r = launch_records<sdm::bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
+      return r;
+    r = launch_bwd(c, SDM_BF16, a, st);
+  } else {
+    if ((r = launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
+      return r;
+    r = launch_bwd(c, SDM_F32, a, st);
+  }
+  if (r != SDM_OK) return r;
+  const int64_t n_th = static_cast<int64_t>(s.B) * s.T * s.H;
+  const int64_t total = n_th * (s.W + s.R + 2);
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8LL * dev->sms));
+  sdm::k_scan_backward_reduce<<<blocks, 256, 0, st>>>(a.part, n_th, s.W, s.R, c.ntile, dw_w, dw_r, dalpha, dbeta);
+  if ((r = launch_status("backward reduce launch")) != SDM_OK) return r;
+  return ok();
+}
+
+// The chunk and bytes of the checkpoints the forward stores for the
+// backward of this shape: the resident recurrence with an fp32 state only.
+sdm_status_t checkpoint_size(const DeviceInfo& dev, const sdm_shape_t& s, int32_t* chunk, size_t* bytes) {
+  ScanChoice c;
+  sdm_status_t r;
+  if ((r = choose_scan(dev, s, &c)) != SDM_OK) return r;
+  if (!c.resident || s.state_dtype != SDM_F32)
+    return fail(SDM_ERR_UNSUPPORTED,
+                "the forward stores backward checkpoints only with the resident recurrence and an fp32 state");
+  BwdChoice b;
+  if ((r = choose_bwd(s, &b)) != SDM_OK) return r;
+  const int64_t n = (static_cast<int64_t>(s.T) + b.C - 1) / b.C;
+  *chunk = b.C;
+  *bytes = static_cast<size_t>(std::max<int64_t>(n - 1, 0)) * s.B * s.H * slots_of(s.sqrt_n) * s.d_v * 4;
+  return SDM_OK;
+}
+}  // namespace sdm_host
+
+namespace sdm_host {
+sdm_status_t layer_forward_impl(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                const void* alpha, const void* beta, const void* g, const void* M0, void* M_out,
+                                float* y, void* workspace, size_t workspace_bytes, void* stream, void* const* events,
+                                int32_t n_events, float* ckpt, size_t ckpt_bytes) {
+  sdm_status_t r;
+  if (!(n_events == 0 || (n_events == 6 && events != nullptr)))
+    return fail(SDM_ERR_INVALID_ARGUMENT, "n_events must be 0, or 6 with a non-NULL events array");
+  Trace tr;
+  if (n_events == 6) {
+    for (int i = 0; i < 6; ++i)
+      if (events[i] == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "events[] holds a NULL event");
+    tr.events = events;
+  }
+  if ((r = check_shape(shape)) != SDM_OK) return r;
+  const sdm_shape_t& s = *shape;
+  const int64_t th = static_cast<int64_t>(s.B) * s.T * s.H;
+  const bool any = th > 0;
+  const bool any_state = static_cast<int64_t>(s.B) * s.H > 0;
+  if ((r = need_ptr(kp, "kp", any)) || (r = need_ptr(qp, "qp", any)) || (r = need_ptr(v, "v", any)) ||
+      (r = need_gate(alpha, "alpha", any, s.in_dtype)) || (r = need_gate(beta, "beta", any, s.in_dtype)) || (r = need_ptr(y, "y", any)) ||
+      (r = need_ptr(M0, "M0", any_state)) || (r = need_ptr(M_out, "M_out", any_state)))
+    return r;
+  if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
+  if (!any_state) return ok();
+  const size_t need = sdm_layer_forward_workspace_bytes(shape);
+  if (any && workspace_bytes < need)
+    return fail(SDM_ERR_INVALID_ARGUMENT,
+                "workspace_bytes below sdm_layer_forward_workspace_bytes() = " + std::to_string(need));
+  if (any && (r = need_ptr(workspace, "workspace", true)) != SDM_OK) return r;
+  DeviceInfo* dev;
+  if ((r = device_info(&dev)) != SDM_OK) return r;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!any) return launch_state_init(*dev, s, M0, M_out, st) == SDM_OK ? ok() : SDM_ERR_CUDA;
+  ScanChoice c;
+  if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
+  int32_t ckpt_C = 0;
+  if (ckpt != nullptr) {
+    size_t need_ckpt = 0;
+    if ((r = checkpoint_size(*dev, s, &ckpt_C, &need_ckpt)) != SDM_OK) return r;
+    if (ckpt_bytes < need_ckpt)
+      return fail(SDM_ERR_INVALID_ARGUMENT, "ckpt_bytes below sdm_layer_checkpoint_size() = " + std::to_string(need_ckpt));
+    if (reinterpret_cast<uintptr_t>(ckpt) % 16 != 0) return fail(SDM_ERR_INVALID_ARGUMENT, "ckpt is not 16-byte aligned");
+  }
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(ws);
+  ws += align256(th * s.W * 4);
+  float* w_w = reinterpret_cast<float*>(ws);
+  ws += align256(th * s.W * 4);
+  int32_t* idx_r = reinterpret_cast<int32_t*>(ws);
+  ws += align256(th * s.R * 4);
+  float* w_r = reinterpret_cast<float*>(ws);
+  ws += align256(th * s.R * 4);
+  uint32_t* rec = reinterpret_cast<uint32_t*>(ws);
+  tr.mark(0, st);
+  if ((r = topk_impl(*dev, kp, s.in_dtype, th, s.sqrt_n, s.W, idx_w, w_w, st)) != SDM_OK) return r;
+  if ((r = topk_impl(*dev, qp, s.in_dtype, th, s.sqrt_n, s.R, idx_r, w_r, st)) != SDM_OK) return r;
+  tr.mark(1, st);
+  if (c.resident) {
+    r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M0, 0, M_out, y, rec, st, tr, false, nullptr,
+                 ckpt, ckpt_C);
+  } else {
+    r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M_out, 0, M_out, y, rec, st, tr,
+                 /*init_before_scan=*/true, M0);
+  }
+  if (r != SDM_OK) return r;
+  return ok();
+}
+}  // namespace sdm_host
+
 using namespace sdm_host;
 
 extern "C" {
@@ -783,69 +944,23 @@ size_t sdm_scan_backward_workspace_bytes(const sdm_shape_t* shape) {
   return c.total();
 }
 
+
 sdm_status_t sdm_scan_backward(const sdm_shape_t* shape, const int32_t* idx_w, const float* w_w,
                                const int32_t* idx_r, const float* w_r, const void* v, const void* alpha,
                                const void* beta, const float* M_in, int32_t m_in_shared, const float* dy, float* dM,
                                float* dv, float* dalpha, float* dbeta, float* dw_w, float* dw_r, void* workspace,
                                size_t workspace_bytes, void* stream) {
+  return scan_backward_impl(shape, idx_w, w_w, idx_r, w_r, v, alpha, beta, M_in, m_in_shared, dy, dM, dv, dalpha,
+                            dbeta, dw_w, dw_r, workspace, workspace_bytes, stream, nullptr);
+}
+
+sdm_status_t sdm_layer_checkpoint_size(const sdm_shape_t* shape, int32_t* chunk_tokens, size_t* bytes) {
   sdm_status_t r;
+  if (chunk_tokens == nullptr || bytes == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "chunk_tokens or bytes is NULL");
   if ((r = check_shape(shape)) != SDM_OK) return r;
-  const sdm_shape_t& s = *shape;
-  BwdChoice c;
-  if ((r = choose_bwd(s, &c)) != SDM_OK) return r;
-  const bool any = static_cast<int64_t>(s.B) * s.H > 0;
-  const bool tok = static_cast<int64_t>(s.B) * s.T * s.H > 0;
-  if ((r = need_ptr(idx_w, "idx_w", tok)) || (r = need_ptr(w_w, "w_w", tok)) || (r = need_ptr(idx_r, "idx_r", tok)) ||
-      (r = need_ptr(w_r, "w_r", tok)) || (r = need_ptr(v, "v", tok)) || (r = need_gate(alpha, "alpha", tok, s.in_dtype)) ||
-      (r = need_gate(beta, "beta", tok, s.in_dtype)) || (r = need_ptr(M_in, "M_in", any)) ||
-      (r = need_ptr(dy, "dy", tok)) || (r = need_ptr(dM, "dM", any)) || (r = need_ptr(dv, "dv", tok)) ||
-      (r = need_gate(dalpha, "dalpha", tok, SDM_F32)) || (r = need_gate(dbeta, "dbeta", tok, SDM_F32)) ||
-      (r = need_ptr(dw_w, "dw_w", tok)) || (r = need_ptr(dw_r, "dw_r", tok)))
-    return r;
-  if (!any) return ok();
-  const size_t need = c.total();
-  if (workspace_bytes < need)
-    return fail(SDM_ERR_INVALID_ARGUMENT,
-                "workspace_bytes below sdm_scan_backward_workspace_bytes() = " + std::to_string(need));
-  if ((r = need_ptr(workspace, "workspace", need > 0)) != SDM_OK) return r;
   DeviceInfo* dev;
   if ((r = device_info(&dev)) != SDM_OK) return r;
-  if (static_cast<size_t>(dev->max_smem_optin) < c.smem)
-    return fail(SDM_ERR_UNSUPPORTED, "the device's shared memory per block is below the backward tile's");
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t N = slots_of(s.sqrt_n);
-  if (s.T == 0) return ok();  // dL/dM_0 = dL/dM_T, already in dM
-  sdm::BwdArgs a;
-  a.B = s.B; a.T = s.T; a.H = s.H; a.N = static_cast<int>(N); a.d_v = s.d_v; a.W = s.W; a.R = s.R;
-  a.C = c.C; a.ntile = c.ntile;
-  a.rl = rec_layout(s.W, s.R, false);
-  a.v = v;
-  a.M_in = M_in;
-  a.M_in_b_stride = m_in_shared ? 0 : static_cast<int64_t>(s.H) * N * s.d_v;
-  a.dy = dy; a.dM = dM; a.dv = dv;
-  char* ws = static_cast<char*>(workspace);
-  a.part = reinterpret_cast<float*>(ws);
-  a.ckpt = reinterpret_cast<float*>(ws + c.part_bytes);
-  a.logbuf = reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes);
-  uint32_t* rec = reinterpret_cast<uint32_t*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes);
-  a.rec = rec;
-  a.Mwork = c.global ? reinterpret_cast<float*>(ws + c.part_bytes + c.ckpt_bytes + c.log_bytes + c.rec_bytes) : nullptr;
-  a.err = dev->err;
-  if (s.in_dtype == SDM_BF16) {
-    if ((r = launch_records<sdm::bf16>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
-      return r;
-    r = launch_bwd(c, SDM_BF16, a, st);
-  } else {
-    if ((r = launch_records<float>(s, idx_w, w_w, idx_r, w_r, alpha, beta, 0, rec, dev->err, *dev, st)) != SDM_OK)
-      return r;
-    r = launch_bwd(c, SDM_F32, a, st);
-  }
-  if (r != SDM_OK) return r;
-  const int64_t n_th = static_cast<int64_t>(s.B) * s.T * s.H;
-  const int64_t total = n_th * (s.W + s.R + 2);
-  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8LL * dev->sms));
-  sdm::k_scan_backward_reduce<<<blocks, 256, 0, st>>>(a.part, n_th, s.W, s.R, c.ntile, dw_w, dw_r, dalpha, dbeta);
-  if ((r = launch_status("backward reduce launch")) != SDM_OK) return r;
+  if ((r = checkpoint_size(*dev, *shape, chunk_tokens, bytes)) != SDM_OK) return r;
   return ok();
 }
 
@@ -971,11 +1086,30 @@ sdm_status_t sdm_layer_backward(const sdm_shape_t* shape, const void* kp, const 
                                 const float* y_pre, const float* dy, float* dM, float* dkp, float* dqp, float* dv,
                                 float* dalpha, float* dbeta, float* dg, void* workspace, size_t workspace_bytes,
                                 void* stream) {
+  return sdm_layer_backward_ckpt(shape, kp, qp, v, alpha, beta, g, M0, y_pre, dy, dM, dkp, dqp, dv, dalpha, dbeta, dg,
+                                 nullptr, 0, workspace, workspace_bytes, stream);
+}
+
+sdm_status_t sdm_layer_backward_ckpt(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                     const void* alpha, const void* beta, const void* g, const float* M0,
+                                     const float* y_pre, const float* dy, float* dM, float* dkp, float* dqp, float* dv,
+                                     float* dalpha, float* dbeta, float* dg, const float* ckpt, size_t ckpt_bytes,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
   sdm_status_t r;
   if ((r = check_shape(shape)) != SDM_OK) return r;
   const sdm_shape_t& s = *shape;
   BwdChoice c;
   if ((r = choose_bwd(s, &c)) != SDM_OK) return r;
+  if (ckpt != nullptr) {
+    DeviceInfo* dev;
+    if ((r = device_info(&dev)) != SDM_OK) return r;
+    int32_t chunk = 0;
+    size_t need_ckpt = 0;
+    if ((r = checkpoint_size(*dev, s, &chunk, &need_ckpt)) != SDM_OK) return r;
+    if (ckpt_bytes < need_ckpt)
+      return fail(SDM_ERR_INVALID_ARGUMENT, "ckpt_bytes below sdm_layer_checkpoint_size() = " + std::to_string(need_ckpt));
+    if (reinterpret_cast<uintptr_t>(ckpt) % 16 != 0) return fail(SDM_ERR_INVALID_ARGUMENT, "ckpt is not 16-byte aligned");
+  }
   const bool tok = static_cast<int64_t>(s.B) * s.T * s.H > 0;
   if ((r = need_ptr(kp, "kp", tok)) || (r = need_ptr(qp, "qp", tok)) || (r = need_ptr(dkp, "dkp", tok)) ||
       (r = need_ptr(dqp, "dqp", tok)))
@@ -1005,8 +1139,8 @@ sdm_status_t sdm_layer_backward(const sdm_shape_t* shape, const void* kp, const 
       return r;
     dy_scan = dy_pre;
   }
-  if ((r = sdm_scan_backward(shape, idx_w, w_w, idx_r, w_r, v, alpha, beta, M0, 1, dy_scan, dM, dv, dalpha, dbeta,
-                             dw_w, dw_r, ws + L.scan, c.total(), stream)) != SDM_OK)
+  if ((r = scan_backward_impl(shape, idx_w, w_w, idx_r, w_r, v, alpha, beta, M0, 1, dy_scan, dM, dv, dalpha, dbeta,
+                              dw_w, dw_r, ws + L.scan, c.total(), stream, ckpt)) != SDM_OK)
     return r;
   if ((r = sdm_pkm_topk_backward(idx_w, w_w, dw_w, s.B, s.T, s.H, s.sqrt_n, s.W, dkp, stream)) != SDM_OK) return r;
   if ((r = sdm_pkm_topk_backward(idx_r, w_r, dw_r, s.B, s.T, s.H, s.sqrt_n, s.R, dqp, stream)) != SDM_OK) return r;
@@ -1105,63 +1239,23 @@ size_t sdm_layer_forward_workspace_bytes(const sdm_shape_t* shape) {
   return 2 * align256(th * s.W * 4) + 2 * align256(th * s.R * 4) + records_bytes(s);
 }
 
+
 sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
                                       const void* alpha, const void* beta, const void* g, const void* M0,
                                       void* M_out, float* y, void* workspace, size_t workspace_bytes, void* stream,
                                       void* const* events, int32_t n_events) {
+  return layer_forward_impl(shape, kp, qp, v, alpha, beta, g, M0, M_out, y, workspace, workspace_bytes, stream, events,
+                            n_events, nullptr, 0);
+}
+
+sdm_status_t sdm_layer_forward_ckpt(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
+                                    const void* alpha, const void* beta, const void* g, const void* M0, void* M_out,
+                                    float* y, float* ckpt, size_t ckpt_bytes, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
   sdm_status_t r;
-  if (!(n_events == 0 || (n_events == 6 && events != nullptr)))
-    return fail(SDM_ERR_INVALID_ARGUMENT, "n_events must be 0, or 6 with a non-NULL events array");
-  Trace tr;
-  if (n_events == 6) {
-    for (int i = 0; i < 6; ++i)
-      if (events[i] == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "events[] holds a NULL event");
-    tr.events = events;
-  }
-  if ((r = check_shape(shape)) != SDM_OK) return r;
-  const sdm_shape_t& s = *shape;
-  const int64_t th = static_cast<int64_t>(s.B) * s.T * s.H;
-  const bool any = th > 0;
-  const bool any_state = static_cast<int64_t>(s.B) * s.H > 0;
-  if ((r = need_ptr(kp, "kp", any)) || (r = need_ptr(qp, "qp", any)) || (r = need_ptr(v, "v", any)) ||
-      (r = need_gate(alpha, "alpha", any, s.in_dtype)) || (r = need_gate(beta, "beta", any, s.in_dtype)) || (r = need_ptr(y, "y", any)) ||
-      (r = need_ptr(M0, "M0", any_state)) || (r = need_ptr(M_out, "M_out", any_state)))
-    return r;
-  if (g != nullptr && (r = need_ptr(g, "g", any)) != SDM_OK) return r;
-  if (!any_state) return ok();
-  const size_t need = sdm_layer_forward_workspace_bytes(shape);
-  if (any && workspace_bytes < need)
-    return fail(SDM_ERR_INVALID_ARGUMENT,
-                "workspace_bytes below sdm_layer_forward_workspace_bytes() = " + std::to_string(need));
-  if (any && (r = need_ptr(workspace, "workspace", true)) != SDM_OK) return r;
-  DeviceInfo* dev;
-  if ((r = device_info(&dev)) != SDM_OK) return r;
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!any) return launch_state_init(*dev, s, M0, M_out, st) == SDM_OK ? ok() : SDM_ERR_CUDA;
-  ScanChoice c;
-  if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  int32_t* idx_w = reinterpret_cast<int32_t*>(ws);
-  ws += align256(th * s.W * 4);
-  float* w_w = reinterpret_cast<float*>(ws);
-  ws += align256(th * s.W * 4);
-  int32_t* idx_r = reinterpret_cast<int32_t*>(ws);
-  ws += align256(th * s.R * 4);
-  float* w_r = reinterpret_cast<float*>(ws);
-  ws += align256(th * s.R * 4);
-  uint32_t* rec = reinterpret_cast<uint32_t*>(ws);
-  tr.mark(0, st);
-  if ((r = topk_impl(*dev, kp, s.in_dtype, th, s.sqrt_n, s.W, idx_w, w_w, st)) != SDM_OK) return r;
-  if ((r = topk_impl(*dev, qp, s.in_dtype, th, s.sqrt_n, s.R, idx_r, w_r, st)) != SDM_OK) return r;
-  tr.mark(1, st);
-  if (c.resident) {
-    r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M0, 0, M_out, y, rec, st, tr);
-  } else {
-    r = run_scan(*dev, s, c, idx_w, w_w, idx_r, w_r, v, alpha, beta, g, M_out, 0, M_out, y, rec, st, tr,
-                 /*init_before_scan=*/true, M0);
-  }
-  if (r != SDM_OK) return r;
-  return ok();
+  if ((r = need_ptr(ckpt, "ckpt", true)) != SDM_OK) return r;
+  return layer_forward_impl(shape, kp, qp, v, alpha, beta, g, M0, M_out, y, workspace, workspace_bytes, stream,
+                            nullptr, 0, ckpt, ckpt_bytes);
 }
 
 int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate) {

@@ -51,6 +51,7 @@ struct BwdArgs {
   float* dv;        // [B, T, H, d_v]
   float* part;      // [B, T, H, ntile, W + R + 2] per-tile partial sums
   float* ckpt;      // per tile: (ceil(T / C) - 1) * N * 4 U
+  const float* ckpt_ext;  // or the forward's checkpoints: [ceil(T / C) - 1][B, H, N, d_v] (then no pass 1)
   float* logbuf;    // per tile: C * W * 4 U
   float* Mwork;     // [B, H, N, d_v] working state when the tiles live in global memory
   unsigned* err;
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(NWB * 32) k_scan_backward(BwdArgs a) {
   // (only when the sequence has more than one chunk)
   copy_in(Ms, Min, a.d_v);
   tile_sync<NWB>();
-  if (nC > 1)
+  if (nC > 1 && a.ckpt_ext == nullptr)
     bwd_token_pass<Tin, U, NWB>(a, b, h, tile, tid, 0, 1, a.T, ring, nullptr, 0, false, [&](int t, const BwdTok& k) {
       if (t > 0 && t % a.C == 0) {
         float4* dst = ckpt + static_cast<int64_t>(t / a.C - 1) * N * U;
@@ -324,6 +325,8 @@ __global__ void __launch_bounds__(NWB * 32) k_scan_backward(BwdArgs a) {
     // State at the chunk start.
     if (kc == 0) {
       copy_in(Ms, Min, a.d_v);
+    } else if (a.ckpt_ext != nullptr) {
+      copy_in(Ms, a.ckpt_ext + (static_cast<int64_t>(kc - 1) * a.B * a.H + bh) * N * a.d_v + col0, a.d_v);
     } else {
       const float* src = reinterpret_cast<const float*>(ckpt + static_cast<int64_t>(kc - 1) * N * U);
       copy_in(Ms, src, 4 * U);

@@ -46,6 +46,8 @@ struct ScanArgs {
   int64_t M_in_b_stride;
   void* M;              // [B, H, N, d_v] final state (resident) / state in place (streaming)
   float* y;             // [B, T, H, d_v]
+  float* ckpt;          // resident, fp32 state: the state before tokens C, 2C, ... ([n-1][B,H,N,d_v]) or NULL
+  int ckpt_C;           // C: tokens per checkpoint chunk
   unsigned* err;
 };
 
@@ -324,8 +326,20 @@ __global__ void __launch_bounds__(NWARP * kWarp) k_scan_resident(ScanArgs a) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     bool failed = false;
 
+    // The warp's tile as the state before token t, into checkpoint t / C - 1
+    // (the backward reads it instead of recomputing the chunk start).
+    auto store_checkpoint = [&](int t) {
+      float* dst = a.ckpt + (static_cast<int64_t>(t / a.ckpt_C - 1) * a.B * a.H + bh) * N * a.d_v + c0 + warp * CW;
+      const float* src = S + static_cast<size_t>(warp) * (N + 2) * CW;
+      for (int x = lane; x < N * (CW / 4); x += kWarp) {
+        const int row = x / (CW / 4), col = (x % (CW / 4)) * 4;
+        *reinterpret_cast<float4*>(dst + static_cast<int64_t>(row) * a.d_v + col) =
+            *reinterpret_cast<const float4*>(src + static_cast<size_t>(row) * CW + col);
+      }
+    };
     // One token: returns false when a staging wait gave up.
     auto step = [&](int t, const ResidentMeta<EB>& cur, ResidentMeta<EB>& nxt) -> bool {
+      if (a.ckpt != nullptr && t > 0 && t % a.ckpt_C == 0) store_checkpoint(t);  // the warp's tile is past token t - 1
       // 1. row loads of the first write block
       int wrow[EB];
       float m[EB][4];

@@ -60,6 +60,9 @@ PROTOTYPES = {
     "sdm_rmsnorm_gate_backward": (_i32, [_p, _p, _i32, _p, ctypes.c_int64, _i32, ctypes.c_float, _p, _p, _p]),
     "sdm_layer_backward_workspace_bytes": (_sz, [_shape_p]),
     "sdm_layer_backward": (_i32, [_shape_p] + [_p] * 17 + [_sz, _p]),
+    "sdm_layer_checkpoint_size": (_i32, [_shape_p, _p, _p]),
+    "sdm_layer_forward_ckpt": (_i32, [_shape_p] + [_p] * 10 + [_sz, _p, _sz, _p]),
+    "sdm_layer_backward_ckpt": (_i32, [_shape_p] + [_p] * 17 + [_sz, _p, _sz, _p]),
     "sdm_slot_counts": (_i32, [_p, _i32, _i32, _i32, _i32, _i32, _p, _p]),
     "sdm_quantize_fp8blk": (_i32, [_p, ctypes.c_int64, _p, _p, _p]),
     "sdm_layer_step": (_i32, [_shape_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),

@@ -205,3 +205,43 @@ def test_layer_backward_matches_oracle(sdm, oracle, cuda_device, name, W, R, gat
         pairs.append(("dg", want_dg))
     for k, w_ in pairs:
         assert_rel_close(got[k].cpu().numpy(), w_, TOL_BWD, k)
+
+
+@pytest.mark.parametrize("T,sqrt_n,d_v,W,R", [(300, 32, 128, 64, 64), (257, 16, 64, 16, 8), (128, 32, 128, 64, 64)])
+def test_forward_checkpoints_replace_the_backward_recompute(sdm, cuda_device, T, sqrt_n, d_v, W, R):
+    """sdm_layer_forward_ckpt gives the forward's results bit for bit, each
+    stored checkpoint is the state after the tokens before it (a forward over
+    that prefix), and the backward given them returns every derivative bit for
+    bit as the backward that recomputes them."""
+    shape = synth.WORKLOADS["d2048_h16_n1024_dv128"].replace(B=2, T=T, H=2, sqrt_n=sqrt_n, d_v=d_v, W=W, R=R)
+    inp = synth.make_inputs(shape, seed=T, device=cuda_device, with_gate=True)
+    args = (inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], inp["M0"], W, R)
+    y0, M0_out = sdm.layer_forward(*args)
+    y1, M1_out, ck = sdm.layer_forward_ckpt(*args)
+    sdm.stream_check()
+    assert torch.equal(y0, y1) and torch.equal(M0_out, M1_out)
+    sh = sdm.make_shape(shape.B, T, shape.H, sqrt_n, W, R, d_v, torch.bfloat16, torch.float32)
+    C, nbytes = sdm.layer_checkpoint_size(sh)
+    n = (T + C - 1) // C
+    assert nbytes == (n - 1) * shape.B * shape.H * shape.N * d_v * 4 and ck.numel() * 4 == nbytes
+    ck = ck.view(max(n - 1, 0), shape.B, shape.H, shape.N, d_v)
+    for k in range(1, n):
+        pre = [t[:, :k * C].contiguous() for t in args[:5]]
+        _, Mk = sdm.layer_forward(*pre, inp["M0"], W, R)
+        assert torch.equal(ck[k - 1], Mk), f"checkpoint {k}"
+    # the backward with the gate, from the pre-epilogue output, with and without the checkpoints
+    gen = torch.Generator(device="cpu").manual_seed(T + 1)
+    dy = torch.randn((shape.B, T, shape.H, d_v), generator=gen).to(cuda_device)
+    y_pre = y0
+    ref = sdm.layer_backward(*args[:6], dy, W, R, g=inp["g"], y_pre=y_pre)
+    got = sdm.layer_backward(*args[:6], dy, W, R, g=inp["g"], y_pre=y_pre, checkpoints=ck.reshape(-1))
+    sdm.stream_check()
+    for k in ref:
+        assert torch.equal(ref[k], got[k]), k
+
+
+def test_forward_checkpoints_only_where_the_forward_stores_them(sdm, cuda_device):
+    long = synth.WORKLOADS["long_t1m_n262144_dv2048"]
+    sh = sdm.make_shape(1, 64, long.H, long.sqrt_n, long.W, long.R, long.d_v, torch.bfloat16, torch.bfloat16)
+    with pytest.raises(sdm.SdmError, match="resident recurrence"):
+        sdm.layer_checkpoint_size(sh)
