@@ -539,10 +539,8 @@ sdm_status_t run_scan(const DeviceInfo& dev, const sdm_shape_t& s, const ScanCho
   a.M_in_b_stride = M_in_b_stride;
   a.M = M;
   a.y = y;
-  a.ckpt = ckpt;
-  a.ckpt_C = ckpt_C;
   a.err = dev.err;
-  if ((r = launch_scan(c, s, a, st)) != SDM_OK) return r;
+  if ((r = launch_scan(c, s, a, st, ckpt, ckpt_C)) != SDM_OK) return r;
   tr.mark(4, st);
   if (g != nullptr && (r = launch_epilogue(dev, s, y, g, st)) != SDM_OK) return r;
   tr.mark(5, st);

@@ -80,7 +80,10 @@ sdm_status_t fast_topk_plan(int n, int K, FastTopkPlan* out);
 sdm_status_t topk_impl(const DeviceInfo& dev, const void* scores, int32_t in_dtype, int64_t units, int n, int K,
                        int32_t* idx, float* w, cudaStream_t st);
 // sdm_tu_scan.cu: the resident and streaming recurrence kernels.
-sdm_status_t launch_scan(const ScanChoice& c, const sdm_shape_t& s, const sdm::ScanArgs& a, cudaStream_t st);
+// ckpt (resident kernel, fp32 state): also store the backward's checkpoints
+// every ckpt_C tokens ([n-1][B,H,N,d_v] fp32).
+sdm_status_t launch_scan(const ScanChoice& c, const sdm_shape_t& s, const sdm::ScanArgs& a, cudaStream_t st,
+                         float* ckpt = nullptr, int ckpt_C = 0);
 // sdm_tu_pipe.cu: the pipelined recurrence and its records (y_zero: rows the parts add into, or null).
 sdm_status_t launch_pipe_records(const sdm_shape_t& s, const ScanChoice& c, const int32_t* idx_w, const float* w_w,
                                  const int32_t* idx_r, const float* w_r, const void* alpha, const void* beta,

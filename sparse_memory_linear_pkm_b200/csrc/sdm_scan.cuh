@@ -46,8 +46,6 @@ struct ScanArgs {
   int64_t M_in_b_stride;
   void* M;              // [B, H, N, d_v] final state (resident) / state in place (streaming)
   float* y;             // [B, T, H, d_v]
-  float* ckpt;          // resident, fp32 state: the state before tokens C, 2C, ... ([n-1][B,H,N,d_v]) or NULL
-  int ckpt_C;           // C: tokens per checkpoint chunk
   unsigned* err;
 };
 
@@ -243,6 +241,20 @@ __device__ __forceinline__ void reduce_store_y(const float* acc, float* y, int l
   if ((lane & (7 & ~(U - 1))) == 0) y[(hi ? 2 : 0) + (hi2 ? 1 : 0)] = k;
 }
 
+// A resident warp tile (N rows of CW fp32 columns) into checkpoint k of
+// the state ([k][B,H,N,d_v]) at columns col..col+CW of (b, h) = bh. Kept out
+// of line: it runs once per checkpoint chunk, outside the per-token chain.
+template <int CW>
+__device__ __noinline__ void resident_store_checkpoint(float* ckpt, int64_t bhs, int N, int d_v, const float* tile,
+                                                       int k, int bh, int col, int lane) {
+  float* dst = ckpt + (static_cast<int64_t>(k) * bhs + bh) * N * d_v + col;
+  for (int x = lane; x < N * (CW / 4); x += kWarp) {
+    const int row = x / (CW / 4), c = (x % (CW / 4)) * 4;
+    *reinterpret_cast<float4*>(dst + static_cast<int64_t>(row) * d_v + c) =
+        *reinterpret_cast<const float4*>(tile + static_cast<size_t>(row) * CW + c);
+  }
+}
+
 // Shared-memory bytes of k_scan_resident (host and device agree on this).
 __host__ __device__ constexpr size_t resident_smem_bytes(int N, int CW, int NWARP, int L, int words, int s_in) {
   return static_cast<size_t>(NWARP) * (N + 2) * CW * 4 + static_cast<size_t>(2) * L * words * 4 +
@@ -256,8 +268,11 @@ __host__ __device__ constexpr size_t resident_smem_bytes(int N, int CW, int NWAR
 // the only block barriers are the two per staged chunk of L tokens. The read
 // sum of a token is reduced over the G entry groups with a fixed butterfly,
 // so y does not depend on timing.
-template <typename Tin, typename Tst, int CW, int NWARP, int L, int EB>
-__global__ void __launch_bounds__(NWARP * kWarp) k_scan_resident(ScanArgs a) {
+// kCkpt builds also store the backward's checkpoints: the state before tokens
+// ckpt_C, 2 ckpt_C, ... into ckpt ([n-1][B,H,N,d_v] fp32). (Kernel
+// parameters of their own: growing ScanArgs changed this kernel's code.)
+template <typename Tin, typename Tst, int CW, int NWARP, int L, int EB, bool kCkpt = false>
+__global__ void __launch_bounds__(NWARP * kWarp) k_scan_resident(ScanArgs a, float* ckpt, int ckpt_C) {
   constexpr int NT = NWARP * kWarp;
   constexpr int C = CW * NWARP;  // columns of the CTA
   constexpr int U = CW / 4;      // lanes per entry
@@ -326,20 +341,19 @@ __global__ void __launch_bounds__(NWARP * kWarp) k_scan_resident(ScanArgs a) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     bool failed = false;
 
-    // The warp's tile as the state before token t, into checkpoint t / C - 1
-    // (the backward reads it instead of recomputing the chunk start).
-    auto store_checkpoint = [&](int t) {
-      float* dst = a.ckpt + (static_cast<int64_t>(t / a.ckpt_C - 1) * a.B * a.H + bh) * N * a.d_v + c0 + warp * CW;
-      const float* src = S + static_cast<size_t>(warp) * (N + 2) * CW;
-      for (int x = lane; x < N * (CW / 4); x += kWarp) {
-        const int row = x / (CW / 4), col = (x % (CW / 4)) * 4;
-        *reinterpret_cast<float4*>(dst + static_cast<int64_t>(row) * a.d_v + col) =
-            *reinterpret_cast<const float4*>(src + static_cast<size_t>(row) * CW + col);
-      }
-    };
+    // Checkpoints (kCkpt builds only): the token before which the next one
+    // is taken.
+    int next_ckpt = ckpt_C;
     // One token: returns false when a staging wait gave up.
     auto step = [&](int t, const ResidentMeta<EB>& cur, ResidentMeta<EB>& nxt) -> bool {
-      if (a.ckpt != nullptr && t > 0 && t % a.ckpt_C == 0) store_checkpoint(t);  // the warp's tile is past token t - 1
+      if constexpr (kCkpt) {
+        if (t == next_ckpt) {  // the warp's tile is past token t - 1
+          resident_store_checkpoint<CW>(ckpt, static_cast<int64_t>(a.B) * a.H, N, a.d_v,
+                                        S + static_cast<size_t>(warp) * (N + 2) * CW, t / ckpt_C - 1, bh,
+                                        c0 + warp * CW, lane);
+          next_ckpt += ckpt_C;
+        }
+      }
       // 1. row loads of the first write block
       int wrow[EB];
       float m[EB][4];
