@@ -63,7 +63,7 @@ sdm_status_t launch_pipe_typed(const ScanChoice& c, const sdm::PipeArgs& a, cuda
 #undef SDM_PIPE
   if (kern == nullptr) return fail(SDM_ERR_UNSUPPORTED, "no pipelined kernel for the chosen tile");
   set_smem(reinterpret_cast<const void*>(kern), c.smem);
-  kern<<<grid, (c.NP + 1 + c.NWW + c.NWR) * 32, c.smem, st>>>(a);  // producers, the y warp, writers, readers
+  kern<<<grid, (c.NP + 1 + c.NWW + c.NWR) * 32, c.smem, st>>>(a);  // producers, the control warp, writers, readers
   return launch_status("pipelined scan launch");
 }
 
