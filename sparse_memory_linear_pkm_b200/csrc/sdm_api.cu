@@ -294,8 +294,12 @@ sdm_status_t choose_scan(const DeviceInfo& dev, const sdm_shape_t& s, ScanChoice
     // d_v = 128: 8-column warp tiles, one warp per CTA, so up to five CTAs
     // share an SM); the first that divides d_v and fits is taken.
     std::vector<ResidentCfg> order;
+    // (a CTA stages each token's v row of CW * NWARP columns with a 1-D bulk
+    // copy: whole 16-byte units only)
     for (const ResidentCfg& k : kResidentCfgs)
-      if (s.d_v % (k.CW * k.NWARP) == 0 && resident_smem(s, k) <= lim) order.push_back(k);
+      if (s.d_v % (k.CW * k.NWARP) == 0 && resident_smem(s, k) <= lim &&
+          (k.CW * k.NWARP * in_size(s.in_dtype)) % 16 == 0)
+        order.push_back(k);
     const int i = pick(order.size());
     if (i >= 0) {
       const ResidentCfg& k = order[i];
