@@ -258,8 +258,8 @@ __device__ __forceinline__ SelectPlan warp_select_plan(const uint32_t (&key)[P],
 // Per-half top-Kh by (value desc, index asc), sorted, into hv/hx[0:Kh).
 // x: the half's n input values in global memory (-0 is taken as +0).
 template <typename Tin, int E, int EPL>
-__device__ __forceinline__ void warp_half_select(const Tin* __restrict__ x, int n, int Kh, uint32_t* hist,
-                                                 uint64_t* sel, float* hv, int32_t* hx) {
+__device__ __forceinline__ void warp_half_select_body(const Tin* __restrict__ x, int n, int Kh, uint32_t* hist,
+                                                      uint64_t* sel, float* hv, int32_t* hx) {
   constexpr int SZ = kWarp * E;  // this half's sort width
   const int lane = lane_id();
   uint64_t k[E];
@@ -315,6 +315,24 @@ __device__ __forceinline__ void warp_half_select(const Tin* __restrict__ x, int 
     }
   }
   __syncwarp();
+}
+
+// The wide paths (4 or more values per lane, sqrtN >= 128) share one
+// out-of-line copy between a selection's two halves: fully unrolled over the
+// lane's values, two inlined copies do not fit the instruction caches (at
+// sqrtN = 512 the kernel stalled mostly on instruction fetch; one shared copy
+// takes its time from 83 to 65 ms per layer step, and 3.90 to 3.77 ms at 128).
+constexpr int kHalfSelectOutOfLine = 4;
+template <typename Tin, int E, int EPL>
+__device__ __noinline__ void warp_half_select_call(const Tin* __restrict__ x, int n, int Kh, uint32_t* hist,
+                                                   uint64_t* sel, float* hv, int32_t* hx) {
+  warp_half_select_body<Tin, E, EPL>(x, n, Kh, hist, sel, hv, hx);
+}
+template <typename Tin, int E, int EPL>
+__device__ __forceinline__ void warp_half_select(const Tin* __restrict__ x, int n, int Kh, uint32_t* hist,
+                                                 uint64_t* sel, float* hv, int32_t* hx) {
+  if constexpr (EPL >= kHalfSelectOutOfLine) warp_half_select_call<Tin, E, EPL>(x, n, Kh, hist, sel, hv, hx);
+  else warp_half_select_body<Tin, E, EPL>(x, n, Kh, hist, sel, hv, hx);
 }
 
 // Per-warp shared scratch (byte offsets): hist 256 words | sel 64 keys |
