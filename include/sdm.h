@@ -89,7 +89,8 @@ typedef enum sdm_dtype { SDM_F32 = 0, SDM_BF16 = 1, SDM_FP8_B16 = 2 } sdm_dtype_
 /* Which recurrence kernel runs (sdm_shape_t.variant). */
 typedef enum sdm_variant {
   SDM_VARIANT_AUTO = 0,      /* pick by size: resident when the state tile fits, pipelined
-                                when 128-byte column tiles leave SMs idle, else streaming */
+                                when 128-byte column tiles leave SMs idle (and for the fp8
+                                state), else streaming */
   SDM_VARIANT_RESIDENT = 1,  /* the (b,h) state column tile lives in shared memory */
   SDM_VARIANT_STREAMING = 2, /* the state stays in global memory; rows are gathered
                                 ahead of use and scattered back */
@@ -110,8 +111,9 @@ typedef enum sdm_variant {
  *   tile      0: the library picks the kernel's tile; k in [1, 64]: use the k-th
  *             entry of the chosen kernel's tile table among those that fit this
  *             shape (sdm_scan_describe names it; SDM_ERR_UNSUPPORTED if there is
- *             no k-th). For measurements; results do not depend on it. In the
- *             backward with shared-memory tiles, 1 selects one warp per tile. */
+ *             no k-th). For measurements: the state comes out the same, y the
+ *             same up to the order of its fp32 sums. In the backward with
+ *             shared-memory tiles, 1 selects one warp per tile. */
 typedef struct sdm_shape {
   int32_t B, T, H;
   int32_t sqrt_n;
