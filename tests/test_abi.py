@@ -164,9 +164,10 @@ def test_layer_backward_arguments_without_gpu(lib):
 
 
 def test_layer_forward_launch_count_needs_device_or_fails(lib):
-    # The count depends on the recurrence variant chosen for the device; without a GPU it reports -1.
+    # The count depends on the recurrence variant chosen for the device (resident 4, streaming 5,
+    # pipelined 5 or 6 with the slot parts' sum); without a GPU it reports -1.
     n = lib.sdm_layer_forward_launches(ctypes.byref(shape()), 0)
-    assert n in (-1, 4, 5)
+    assert n in (-1, 4, 5, 6)
     assert lib.sdm_layer_forward_launches(ctypes.byref(shape(sqrt_n=0)), 0) == -1
 
 
