@@ -226,9 +226,10 @@ struct PipeCfg {
   int C, P, L, NWW, NWR, NP, S;
 };
 constexpr PipeCfg kPipeCfgs[] = {
-    {2, 64, 6, 16, 4, 3, 4, 1}, {2, 64, 6, 16, 4, 3, 4, 2}, {2, 64, 7, 8, 4, 3, 4, 2}, {2, 64, 6, 16, 4, 4, 4, 1},
-    {2, 64, 6, 16, 4, 3, 2, 1}, {4, 32, 6, 16, 4, 3, 4, 1}, {4, 32, 4, 16, 4, 3, 4, 1}, {4, 32, 6, 16, 4, 3, 4, 2},
-    {1, 64, 6, 16, 4, 3, 4, 1},  // the block-scaled fp8 state: 64 codes (and 4 exponents) a row segment
+    {2, 64, 6, 16, 4, 3, 8, 1}, {2, 64, 6, 16, 4, 3, 4, 2}, {2, 64, 7, 8, 4, 3, 4, 2}, {2, 64, 6, 16, 4, 4, 8, 1},
+    {2, 64, 6, 16, 4, 3, 4, 1}, {4, 32, 6, 16, 4, 3, 4, 1}, {4, 32, 4, 16, 4, 3, 4, 1}, {4, 32, 6, 16, 4, 3, 4, 2},
+    // the block-scaled fp8 state: 64 codes (and 4 exponents) a row segment
+    {1, 64, 6, 16, 4, 3, 8, 1}, {1, 64, 6, 16, 4, 3, 4, 1},
 };
 
 // Instantiated resident tiles: columns per warp, warps per CTA, staging

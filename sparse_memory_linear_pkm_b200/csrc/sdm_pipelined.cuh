@@ -393,39 +393,16 @@ __host__ __device__ constexpr size_t pipe_exp_bytes(int P, int Wp, int Rp, int S
   return static_cast<size_t>((P * (Wp + Rp) + pipe_wstages(P, S) * Wp + 3) / 4) * 128;
 }
 
+// Entries one consumer-warp instruction covers: 32 lanes over the 16-byte
+// units of a C-column row segment.
+__host__ __device__ constexpr int pipe_entry_groups(int C, int s_state) { return 32 * 16 / (C * s_state); }
+
 __host__ __device__ constexpr size_t pipe_smem_bytes(int P, int L, int Wp, int Rp, int words, int C, int s_state,
                                                      int s_in, int NWR, int S, bool fp8 = false) {
   return static_cast<size_t>(P) * (Wp + Rp) * C * s_state + static_cast<size_t>(pipe_wstages(P, S)) * Wp * C * s_state +
          (fp8 ? pipe_exp_bytes(P, Wp, Rp, S) : 0) +
          static_cast<size_t>(2) * L * words * 4 + static_cast<size_t>(2) * L * C * s_in +
-         static_cast<size_t>(2) * S * NWR * C * 4 + (2 * P + 2) * 8 + 128;
-}
-
-// Sums a[0:VE) (the VE columns of one 16-byte unit) over the lanes that
-// share lane % U, in a fixed butterfly order that halves the values each
-// level; returns the offset of the VE * U / 32 column sums the lane keeps in
-// a[0 : VE * U / 32).
-template <int VE, int U>
-__device__ __forceinline__ int reduce_scatter_entries(float (&a)[VE], int lane) {
-  static_assert((VE * U) % kWarp == 0, "every lane keeps at least one column");
-  int off = 0;
-  int n = VE;
-#pragma unroll
-  for (int o = kWarp / 2; o >= U; o >>= 1) {
-    const bool hi = lane & o;
-    const int h = n / 2;
-#pragma unroll
-    for (int j = 0; j < VE / 2; ++j) {
-      if (j < h) {
-        const float keep = hi ? a[j + h] : a[j];
-        const float send = hi ? a[j] : a[j + h];
-        a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-    off += hi ? h : 0;
-    n = h;
-  }
-  return off;
+         static_cast<size_t>(2) * S * NWR * pipe_entry_groups(C, s_state) * C * 4 + (2 * P + 2) * 8 + 128;
 }
 
 template <typename Tin, typename Tst, int C, int P, int L, int NWW, int NWR, int NP, int S>
@@ -437,6 +414,7 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   constexpr int U = C / VE;             // units per row segment
   constexpr int RS = C * sizeof(Tst);   // bytes of a row segment
   constexpr int G = kWarp / U;          // entries per consumer-warp instruction
+  static_assert(G == pipe_entry_groups(C, sizeof(Tst)), "the host sizes the read partials by the same count");
   static_assert(U >= 1 && U <= kWarp && kWarp % U == 0, "a row segment spans a divisor of the warp");
   static_assert(NT % U == 0, "gather lanes cover whole rows");
   static_assert(L >= P, "a chunk of records is staged before its tokens are gathered");
@@ -453,8 +431,8 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   unsigned char* xstage = wstage + static_cast<size_t>(Q) * Wp * RS;              // fp8: exponents of the stage rows
   uint32_t* recbuf = reinterpret_cast<uint32_t*>(xstage + (kFp8 ? pipe_exp_bytes(P, Wp, pl.Rp, S) : 0));  // [2][L][words]
   Tin* vbuf = reinterpret_cast<Tin*>(recbuf + 2 * L * words);                      // [2][L][C]
-  float* ybuf = reinterpret_cast<float*>(vbuf + 2 * L * C);                        // [2][S][NWR][C] read partials
-  uint64_t* cbar = reinterpret_cast<uint64_t*>(ybuf + 2 * S * NWR * C);           // [2] record chunks
+  float* ybuf = reinterpret_cast<float*>(vbuf + 2 * L * C);                        // [2][S][NWR][G][C] read partials
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(ybuf + 2 * S * NWR * G * C);       // [2] record chunks
   uint64_t* full = cbar + 2;                                                       // [P] gathered stages
   uint64_t* done = full + P;  // [P] the consumers are through with a token, its stores fenced
 
@@ -639,10 +617,11 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
         read_unit<VE>(acc, m0, qr[i0]);
         read_unit<VE>(acc, m1, has1 ? qr[i1] : 0.0f);
       }
-      const int off = reduce_scatter_entries<VE, U>(acc, lane);
-      float* yb = ybuf + (static_cast<size_t>(t & 1) * NWR + (cw - NWW)) * C + qw * VE + off;
+      // this lane's sums of its unit over its entry group; the control warp adds
+      // the NWR * G groups of a column in a fixed order
+      float* yb = ybuf + ((static_cast<size_t>(t & 1) * NWR + (cw - NWW)) * G + lane / U) * C + qw * VE;
 #pragma unroll
-      for (int j = 0; j < VE * U / kWarp; ++j) yb[j] = acc[j];
+      for (int j = 0; j < VE; j += 4) *reinterpret_cast<float4*>(yb + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
     }
   };
   // Tokens ta and ta + 1 (if hb) on this consumer thread, interleaved. Rows
@@ -760,13 +739,11 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
           if (ik < nB) read_unit<VE>(accB, mB[k], qrB[i[k]]);
         }
       }
-      const int off = reduce_scatter_entries<VE, U>(accA, lane);
-      reduce_scatter_entries<VE, U>(accB, lane);
-      float* yb = ybuf + (static_cast<size_t>((ta / 2) & 1) * 2 * NWR + (cw - NWW)) * C + qw * VE + off;
+      float* yb = ybuf + ((static_cast<size_t>((ta / 2) & 1) * 2 * NWR + (cw - NWW)) * G + lane / U) * C + qw * VE;
 #pragma unroll
-      for (int j = 0; j < VE * U / kWarp; ++j) {
-        yb[j] = accA[j];
-        yb[NWR * C + j] = accB[j];
+      for (int j = 0; j < VE; j += 4) {
+        *reinterpret_cast<float4*>(yb + j) = make_float4(accA[j], accA[j + 1], accA[j + 2], accA[j + 3]);
+        *reinterpret_cast<float4*>(yb + NWR * G * C + j) = make_float4(accB[j], accB[j + 1], accB[j + 2], accB[j + 3]);
       }
     }
   };
@@ -781,7 +758,10 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
       // Stage u % P held token u - P: the consumers are through with it, and
       // the writes of every token up to u - P were fenced (the hazard plan
       // forwards rows written by tokens u - P + 1 .. u - 1 from shared memory).
-      bool ok = u < P || mbar_wait_backoff(&done[(u - P) % P], ((u - P) / P) & 1, a.err);
+      // Tokens finish in order, so one wait serves two: an even token waits for
+      // token u - P + 1, which also frees the stage of the odd token after it.
+      const int need = u < P ? -1 : (u % 2 == 0 ? u - P + 1 : (u - 1 < P ? u - P : -1));
+      bool ok = need < 0 || mbar_wait_backoff(&done[need % P], (need / P) & 1, a.err);
       if (ok && u % L == 0) ok = chunk_wait(u / L);
       if (!ok) break;
       const int c = u / L;
@@ -798,14 +778,20 @@ __global__ void __launch_bounds__((NP + 1 + NWW + NWR) * kWarp, 1) k_scan_pipeli
   constexpr int kBarThreads = (1 + NWW + NWR) * kWarp;  // the control warp and the consumers
   const int n_steps = (T + S - 1) / S;                  // a step: S consecutive tokens
   if (control) {
-    // y of token u: the read warps' column sums, added in warp order
+    // y of token u: the read lanes' partial sums, added in (read warp, entry
+    // group) order, two adjacent columns a lane
     auto put_y = [&](int u) {
-      const float* yb = ybuf + (static_cast<size_t>((u / S) & 1) * S + u % S) * NWR * C;
-      for (int c = lane; c < C; c += kWarp) {
-        float acc = yb[c];
+      static_assert(C % 2 == 0 && C <= 2 * kWarp, "one column pair a lane");
+      if (2 * lane < C) {
+        const float* yb = ybuf + (static_cast<size_t>((u / S) & 1) * S + u % S) * NWR * G * C + 2 * lane;
+        float2 acc = *reinterpret_cast<const float2*>(yb);
 #pragma unroll
-        for (int r = 1; r < NWR; ++r) acc += yb[r * C + c];
-        y_bh[static_cast<int64_t>(u) * tok_step + c] = acc;
+        for (int k = 1; k < NWR * G; ++k) {
+          const float2 p = *reinterpret_cast<const float2*>(yb + k * C);
+          acc.x += p.x;
+          acc.y += p.y;
+        }
+        *reinterpret_cast<float2*>(y_bh + static_cast<int64_t>(u) * tok_step + 2 * lane) = acc;
       }
     };
     auto ready = [&](int u) {  // token u's records and rows are in shared memory

@@ -53,10 +53,10 @@ sdm_status_t launch_pipe_typed(const ScanChoice& c, const sdm::PipeArgs& a, cuda
   if (c.C == C_ && c.P == P_ && c.L == L_ && c.NWW == NWW_ && c.NWR == NWR_ && c.NP == NP_ && c.S == S_)      \
     kern = sdm::k_scan_pipelined<Tin, Tst, C_, P_, L_, NWW_, NWR_, NP_, S_>;
   if constexpr (std::is_same<Tst, sdm::Fp8Blk>::value) {
-    SDM_PIPE(64, 6, 16, 4, 3, 4, 1)
+    SDM_PIPE(64, 6, 16, 4, 3, 8, 1) SDM_PIPE(64, 6, 16, 4, 3, 4, 1)
   } else if constexpr (sizeof(Tst) == 2) {
-    SDM_PIPE(64, 6, 16, 4, 3, 4, 1) SDM_PIPE(64, 6, 16, 4, 3, 4, 2) SDM_PIPE(64, 7, 8, 4, 3, 4, 2)
-    SDM_PIPE(64, 6, 16, 4, 4, 4, 1) SDM_PIPE(64, 6, 16, 4, 3, 2, 1)
+    SDM_PIPE(64, 6, 16, 4, 3, 8, 1) SDM_PIPE(64, 6, 16, 4, 3, 4, 2) SDM_PIPE(64, 7, 8, 4, 3, 4, 2)
+    SDM_PIPE(64, 6, 16, 4, 4, 8, 1) SDM_PIPE(64, 6, 16, 4, 3, 4, 1)
   } else {
     SDM_PIPE(32, 6, 16, 4, 3, 4, 1) SDM_PIPE(32, 4, 16, 4, 3, 4, 1) SDM_PIPE(32, 6, 16, 4, 3, 4, 2)
   }
