@@ -183,7 +183,7 @@ SDM_API int32_t sdm_scan_variant(const sdm_shape_t* shape);
 /* The launch configuration of that kernel as text, e.g.
  * "resident CW=8 NWARP=1 L=4 EB=4 smem=...",
  * "streaming C=64 P=3 L=8 NW=16 smem=..." or
- * "pipelined C=64 P=6 L=16 NWW=4 NWR=2 parts=2 smem=...", NUL-terminated into out (caller
+ * "pipelined C=64 P=6 L=16 NWW=4 NWR=3 NP=8 S=1 parts=2 smem=...", NUL-terminated into out (caller
  * owned, out_len bytes, truncated to fit). Returns SDM_OK, or an error for an
  * invalid or unsupported shape (out left empty). For profiles and logs. */
 SDM_API sdm_status_t sdm_scan_describe(const sdm_shape_t* shape, char* out, size_t out_len);
