@@ -453,7 +453,10 @@ def run_sdm(args, dist: Dist):
     for _ in range(args.warmup):
         step()
     sdm.stream_check(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # an overlapped call (token chunks) also brackets each chunk's recurrence launch
+    chunks = sdm.layer_forward_chunks(sh)
+    n_ev = 6 + (2 * chunks if chunks > 1 else 0)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     for row in ev:  # create the events before the timed region
         for e in row:
             e.record(stream)
@@ -473,13 +476,16 @@ def run_sdm(args, dist: Dist):
     ms = start.elapsed_time(end)
     ms_max = dist.max(ms, dev)
     stage_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps for i in range(5)]
+    # the recurrence kernel's own time a step: its launch (one pass) or the sum of its chunk launches
+    kernel_ms = stage_ms[3] if chunks == 1 else sum(
+        ev[k][6 + 2 * c].elapsed_time(ev[k][7 + 2 * c]) for k in range(args.steps) for c in range(chunks)) / args.steps
     tokens = shape.B * shape.T
     value = aggregate_value(tokens * args.steps, dist.world, ms_max / 1e3)
 
     resident = sdm.scan_variant(sh) == "resident"
     launches_per_step = int(sdm.native.load().sdm_layer_forward_launches(ctypes.byref(sh), int(args.epilogue)))
     clk = clocks.summary()
-    roof = roofline_of(shape, sh, stage_ms[3], args.epilogue, dev, clk, fp8_state=args.fp8_state)
+    roof = roofline_of(shape, sh, kernel_ms, args.epilogue, dev, clk, fp8_state=args.fp8_state, launches=chunks)
 
     e2e = None
     if not args.no_e2e:
@@ -504,7 +510,12 @@ def run_sdm(args, dist: Dist):
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
                 "clocks": clk,
                 "stage_ms": {"select_k_and_q": stage_ms[0], "records": stage_ms[1], "state_init": stage_ms[2],
-                             "scan": stage_ms[3], "epilogue": stage_ms[4]}}
+                             "scan": stage_ms[3], "epilogue": stage_ms[4], "recurrence_kernel": kernel_ms}}
+        if chunks > 1:
+            line["config"]["overlap"] = (f"{chunks} token chunks: each next chunk's selection on the SMs the "
+                                         "recurrence leaves free; stage_ms select/records cover the first chunk, "
+                                         "scan the first chunk's recurrence to the last one's end with the "
+                                         "records in between; recurrence_kernel the sum of its launches")
     del ev, inp, y, M_out, ws
     torch.cuda.empty_cache()
     if dist.rank == 0:
@@ -514,9 +525,11 @@ def run_sdm(args, dist: Dist):
     dist.close()
 
 
-def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk: dict, fp8_state: bool = False) -> dict:
-    """Roofline of the recurrence kernel of one launch: algorithmic bytes over
-    its CUDA-event time against the measured HBM copy bandwidth (streaming,
+def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk: dict, fp8_state: bool = False,
+                launches: int = 1) -> dict:
+    """Roofline of the recurrence kernel: algorithmic bytes over its CUDA-event
+    time (scan_ms a layer call, over `launches` launches: the token chunks of
+    an overlapped call) against the measured HBM copy bandwidth (streaming,
     pipelined), or the derived shared-memory bandwidth (resident)."""
     resident = sdm.scan_variant(sh) == "resident"
     algo_bytes = algorithmic_bytes_per_token_head(shape, epilogue, fp8_state) * shape.B * shape.T * shape.H
@@ -535,8 +548,10 @@ def roofline_of(shape: synth.Shape, sh, scan_ms: float, epilogue: bool, dev, clk
     kernel = {"resident": "k_scan_resident", "streaming": "k_scan_streaming",
               "pipelined": "k_scan_pipelined"}[sdm.scan_variant(sh)]
     launch_cfg = sdm.scan_describe(sh)
-    roof.update({"traffic": recorded_traffic(shape.name, kernel, launch_cfg), "kernel": kernel, "launch": launch_cfg,
-                 "ms_per_launch": scan_ms, "algorithmic_bytes_per_launch": algo_bytes})
+    traffic = recorded_traffic(shape.name, kernel, launch_cfg)
+    roof.update({"traffic": None if traffic is None else traffic / launches, "kernel": kernel, "launch": launch_cfg,
+                 "ms_per_launch": scan_ms / launches, "algorithmic_bytes_per_launch": algo_bytes / launches,
+                 "launches_per_step": launches})
     return roof
 
 

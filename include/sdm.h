@@ -359,7 +359,17 @@ SDM_API size_t sdm_layer_forward_workspace_bytes(const sdm_shape_t* shape);
  *   kp, qp [B,T,H,2*sqrt_n] in_dtype;  v, alpha, beta, g as in sdm_scan
  *   M0     [H,N,d_v] state_dtype (not modified);  M_out [B,H,N,d_v] state_dtype (M_T)
  *   y      [B,T,H,d_v] fp32
- *   workspace: at least sdm_layer_forward_workspace_bytes(shape). */
+ *   workspace: at least sdm_layer_forward_workspace_bytes(shape).
+ * Overlapped call: with one batch row (B = 1), the pipelined recurrence and
+ * T >= 131072, the call runs as chunks of 65536 tokens (sdm_layer_forward_chunks):
+ * the selection of the next chunk runs on the SMs the recurrence leaves free
+ * while the recurrence of the current chunk runs, on two streams the library
+ * creates per device (one at the greatest, one at the least priority). They
+ * start after the work enqueued on `stream` before the call, and `stream`
+ * waits for all of their work, so to the caller the call is ordered on
+ * `stream` as any other. The outputs are those of the one-pass call bit for bit
+ * (the recurrence over consecutive chunks continues from the state in M_out;
+ * selection and records are per token). */
 SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp,
                                const void* v, const void* alpha, const void* beta, const void* g,
                                const void* M0, void* M_out, float* y, void* workspace,
@@ -372,6 +382,12 @@ SDM_API sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp,
  * read sums into y (pipelined, two parts), plus the epilogue. -1 for an
  * invalid or unsupported shape. For profiles and logs. */
 SDM_API int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate);
+
+/* Token chunks one sdm_layer_forward call runs this shape as on the current
+ * device: 1 for a one-pass call, more for an overlapped call (see
+ * sdm_layer_forward); each chunk makes two selections, a record build and a
+ * recurrence launch. -1 for an invalid or unsupported shape. */
+SDM_API int32_t sdm_layer_forward_chunks(const sdm_shape_t* shape);
 
 /* Kernel launches one sdm_layer_step call makes for this shape, without the
  * epilogue's (one more when g is given on the general path): 1 when the call
@@ -407,7 +423,13 @@ SDM_API sdm_status_t sdm_layer_step(const sdm_shape_t* shape, const void* kp, co
  * [2] after the record build, [3] after the state initialisation, [4] after
  * the recurrence kernel, [5] after the epilogue (a stage that does not run
  * leaves its event adjacent to the previous one). n_events must be 0 (no
- * events; events may be NULL) or 6. */
+ * events; events may be NULL) or 6. In an overlapped call the events go on
+ * the library's streams: [1] and [2] after the first chunk's selection and
+ * records, [3] before the first chunk's recurrence, [4] after the last
+ * chunk's recurrence and the part sum, [5] after the epilogue; there
+ * n_events may also be 6 + 2 * sdm_layer_forward_chunks(shape), and
+ * events[6 + 2k] and events[7 + 2k] are recorded right before and after the
+ * recurrence launch of chunk k (the recurrence kernel's own time). */
 SDM_API sdm_status_t sdm_layer_forward_traced(const sdm_shape_t* shape, const void* kp, const void* qp,
                                       const void* v, const void* alpha, const void* beta,
                                       const void* g, const void* M0, void* M_out, float* y,

@@ -79,6 +79,14 @@ def layer_forward_workspace_bytes(shape: native.Shape) -> int:
     return int(native.load().sdm_layer_forward_workspace_bytes(ctypes.byref(shape)))
 
 
+def layer_forward_chunks(shape: native.Shape) -> int:
+    """Token chunks a layer_forward call of this shape runs as (1: one pass; more: overlapped)."""
+    n = int(native.load().sdm_layer_forward_chunks(ctypes.byref(shape)))
+    if n < 0:
+        native.check(1)
+    return n
+
+
 def _workspace(nbytes: int, device, workspace: torch.Tensor | None) -> torch.Tensor:
     if workspace is not None:
         if workspace.numel() * workspace.element_size() < nbytes:
@@ -336,7 +344,8 @@ def layer_forward(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float
     recurrence and the optional RMS-norm x g epilogue. Returns (y, M_out).
 
     ``events``: optional list of 6 already-created torch.cuda.Event objects
-    recorded between the stages (see sdm_layer_forward_traced in sdm.h)."""
+    recorded between the stages, or 6 + 2 per chunk of an overlapped call
+    (see sdm_layer_forward_traced in sdm.h)."""
     B, T, H, two_n = kp.shape
     d_v = v.shape[-1]
     shape = native.Shape(B, T, H, two_n // 2, W, R, d_v, _code(kp, "kp"), _code(M0, "M0"), eps,
@@ -350,9 +359,9 @@ def layer_forward(kp, qp, v, alpha, beta, M0, W: int, R: int, g=None, eps: float
     if events is None:
         ev, n_ev = None, 0
     else:
-        if len(events) != 6:
-            raise ValueError("events must hold 6 torch.cuda.Event objects")
-        ev, n_ev = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events]), 6
+        if len(events) < 6 or len(events) % 2:
+            raise ValueError("events must hold 6 (+ 2 a chunk) torch.cuda.Event objects")
+        ev, n_ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events]), len(events)
     native.check(lib.sdm_layer_forward_traced(ctypes.byref(shape), _ptr(kp), _ptr(qp), _ptr(v), _ptr(alpha),
                                               _ptr(beta), _ptr(g), _ptr(M0), _ptr(M_out), _ptr(y), _ptr(ws),
                                               ws.numel() * ws.element_size(), _stream(kp.device), ev, n_ev))

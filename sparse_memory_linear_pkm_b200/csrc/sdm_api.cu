@@ -479,8 +479,12 @@ sdm_status_t launch_epilogue(const DeviceInfo& dev, const sdm_shape_t& s, float*
 // Records a caller event (no-op without events).
 struct Trace {
   void* const* events = nullptr;
+  void* const* chunk_events = nullptr;  // an overlapped call: two a chunk around its recurrence launch
   void mark(int i, cudaStream_t st) const {
     if (events != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+  }
+  void mark_chunk(int64_t i, cudaStream_t st) const {
+    if (chunk_events != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(chunk_events[i]), st);
   }
 };
 
@@ -761,18 +765,199 @@ sdm_status_t checkpoint_size(const DeviceInfo& dev, const sdm_shape_t& s, int32_
 }  // namespace sdm_host
 
 namespace sdm_host {
+// ------------------------------------------------- overlapped layer call --
+//
+// The pipelined recurrence runs few CTAs (one per SM, 2 x 2 x 32 = 128 on the
+// long-context workload), so SMs are left over while it runs. A layer call
+// with one batch row and at least two chunks of kOverlapChunk tokens runs as
+// chunks: the selection of chunk k + 1 runs on a low-priority stream (on the
+// spare SMs: its shared memory does not fit beside a recurrence CTA) while
+// the recurrence of chunk k runs on a high-priority stream, continuing from
+// the state in M_out; each chunk's records are built on the high-priority
+// stream just before its recurrence (the spare SMs alone are too few for
+// both selection and records in a chunk's recurrence time). The recurrence over chunks
+// equals one recurrence bit for bit (the state is the checkpoint; the hazard
+// plan only changes where a row is read from), and selection and records are
+// per token, so the outputs are those of the one-pass call. Every dependency
+// is a stream event on work enqueued earlier (no kernel waits on another).
+constexpr int32_t kOverlapChunk = 65536;
+
+bool overlapped(const sdm_shape_t& s, const ScanChoice& c) {
+  return c.kind == SDM_VARIANT_PIPELINED && s.B == 1 && s.T >= 2 * kOverlapChunk;
+}
+int64_t overlap_chunks(const sdm_shape_t& s) { return (static_cast<int64_t>(s.T) + kOverlapChunk - 1) / kOverlapChunk; }
+
+// Workspace of an overlapped call: two chunk buffers of selections, one of
+// records, and the second slot part's read sums of the whole call.
+size_t overlap_workspace(const sdm_shape_t& s, const ScanChoice& c) {
+  const size_t tch = static_cast<size_t>(kOverlapChunk) * s.H;
+  const size_t sel = 2 * align256(tch * s.W * 4) + 2 * align256(tch * s.R * 4);
+  return 2 * sel + align256(tch * c.parts * sdm::pipe_layout(s.W, s.R).words * 4u) + y_other_bytes(s, c);
+}
+
+// The library's two streams on the current device, created on first use:
+// the first at the greatest priority (the recurrence), the second at the
+// least (selection and records), so that pending recurrence CTAs are placed
+// first when SMs free up.
+std::mutex g_lane_mu;
+cudaStream_t g_lane[64][2] = {};
+sdm_status_t lane_streams(cudaStream_t* hi, cudaStream_t* lo) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SDM_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(SDM_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_lane_mu);
+  if (g_lane[dev][0] == nullptr) {
+    int least = 0, greatest = 0;
+    cudaStream_t a = nullptr, b = nullptr;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess ||
+        (e = cudaStreamCreateWithPriority(&a, cudaStreamNonBlocking, greatest)) != cudaSuccess ||
+        (e = cudaStreamCreateWithPriority(&b, cudaStreamNonBlocking, least)) != cudaSuccess) {
+      if (a != nullptr) cudaStreamDestroy(a);
+      return fail(SDM_ERR_CUDA, std::string("stream creation: ") + cudaGetErrorString(e));
+    }
+    g_lane[dev][0] = a;
+    g_lane[dev][1] = b;
+  }
+  *hi = g_lane[dev][0];
+  *lo = g_lane[dev][1];
+  return SDM_OK;
+}
+
+// Events of one overlapped call, released once the call is enqueued (the
+// driver keeps an event until the work recorded in it completes).
+struct CallEvents {
+  cudaEvent_t e[7] = {};
+  ~CallEvents() {
+    for (cudaEvent_t x : e)
+      if (x != nullptr) cudaEventDestroy(x);
+  }
+  sdm_status_t create() {
+    for (cudaEvent_t& x : e) {
+      const cudaError_t err = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+      if (err != cudaSuccess) return fail(SDM_ERR_CUDA, std::string("cudaEventCreate: ") + cudaGetErrorString(err));
+    }
+    return SDM_OK;
+  }
+};
+
+sdm_status_t layer_forward_overlapped(const DeviceInfo& dev, const sdm_shape_t& s, const ScanChoice& c,
+                                      const void* kp, const void* qp, const void* v, const void* alpha,
+                                      const void* beta, const void* g, const void* M0, void* M_out, float* y,
+                                      unsigned char* ws, cudaStream_t caller, const Trace& tr) {
+  sdm_status_t r;
+  cudaStream_t hi = nullptr, lo = nullptr;
+  if ((r = lane_streams(&hi, &lo)) != SDM_OK) return r;
+  CallEvents ev;  // 0 fork; 1, 2 selection into buffer 0, 1; 3, 4 records from buffer 0, 1; 5, 6 join
+  if ((r = ev.create()) != SDM_OK) return r;
+  const int64_t tch = static_cast<int64_t>(kOverlapChunk) * s.H;
+  const size_t rec_b = align256(static_cast<size_t>(tch) * c.parts * sdm::pipe_layout(s.W, s.R).words * 4u);
+  int32_t* idx_w[2];
+  float* w_w[2];
+  int32_t* idx_r[2];
+  float* w_r[2];
+  for (int b = 0; b < 2; ++b) {
+    idx_w[b] = reinterpret_cast<int32_t*>(ws);
+    ws += align256(tch * s.W * 4);
+    w_w[b] = reinterpret_cast<float*>(ws);
+    ws += align256(tch * s.W * 4);
+    idx_r[b] = reinterpret_cast<int32_t*>(ws);
+    ws += align256(tch * s.R * 4);
+    w_r[b] = reinterpret_cast<float*>(ws);
+    ws += align256(tch * s.R * 4);
+  }
+  uint32_t* rec = reinterpret_cast<uint32_t*>(ws);
+  ws += rec_b;
+  float* y_other = c.parts > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+  // Both lanes start after the caller's earlier work; the caller's stream
+  // continues after both lanes' work, also when an enqueue fails part way.
+  tr.mark(0, caller);
+  cudaEventRecord(ev.e[0], caller);
+  cudaStreamWaitEvent(hi, ev.e[0], 0);
+  cudaStreamWaitEvent(lo, ev.e[0], 0);
+  auto finish = [&](sdm_status_t status) {
+    cudaEventRecord(ev.e[5], lo);
+    cudaEventRecord(ev.e[6], hi);
+    cudaStreamWaitEvent(caller, ev.e[5], 0);
+    cudaStreamWaitEvent(caller, ev.e[6], 0);
+    return status;
+  };
+  if ((r = launch_state_init(dev, s, M0, M_out, hi)) != SDM_OK) return finish(r);
+  const size_t in_b = in_size(s.in_dtype);
+  const auto* kpb = static_cast<const unsigned char*>(kp);
+  const auto* qpb = static_cast<const unsigned char*>(qp);
+  const auto* vb = static_cast<const unsigned char*>(v);
+  const auto* ab = static_cast<const unsigned char*>(alpha);
+  const auto* bb = static_cast<const unsigned char*>(beta);
+  const int64_t key_row = 2LL * s.sqrt_n, n_chunks = overlap_chunks(s);
+  for (int64_t k = 0; k < n_chunks; ++k) {
+    const int b = static_cast<int>(k & 1);
+    const int64_t t0 = k * kOverlapChunk;
+    sdm_shape_t sk = s;
+    sk.T = static_cast<int32_t>(std::min<int64_t>(kOverlapChunk, s.T - t0));
+    const int64_t th = static_cast<int64_t>(sk.T) * s.H, h0 = t0 * s.H;  // the chunk's token-heads, its first one
+    // chunk k's selection on the low-priority lane, once chunk k - 2's
+    // records are through with buffer b
+    if (k >= 2) cudaStreamWaitEvent(lo, ev.e[3 + b], 0);
+    if ((r = topk_impl(dev, kpb + h0 * key_row * in_b, s.in_dtype, th, s.sqrt_n, s.W, idx_w[b], w_w[b], lo)) != SDM_OK ||
+        (r = topk_impl(dev, qpb + h0 * key_row * in_b, s.in_dtype, th, s.sqrt_n, s.R, idx_r[b], w_r[b], lo)) != SDM_OK)
+      return finish(r);
+    if (k == 0) tr.mark(1, lo);
+    cudaEventRecord(ev.e[1 + b], lo);
+    // chunk k's records and recurrence on the high-priority lane
+    cudaStreamWaitEvent(hi, ev.e[1 + b], 0);
+    if ((r = launch_pipe_records(sk, c, idx_w[b], w_w[b], idx_r[b], w_r[b], ab + h0 * in_b, bb + h0 * in_b, rec,
+                                 nullptr, dev, hi)) != SDM_OK)
+      return finish(r);
+    cudaEventRecord(ev.e[3 + b], hi);
+    if (k == 0) {
+      tr.mark(2, hi);
+      tr.mark(3, hi);
+    }
+    sdm::PipeArgs a{};
+    a.B = 1; a.T = sk.T; a.H = s.H;
+    a.N = static_cast<int>(slots_of(s.sqrt_n));
+    a.d_v = s.d_v; a.W = s.W; a.R = s.R;
+    a.parts = c.parts;
+    a.pl = sdm::pipe_layout(s.W, s.R);
+    a.rec = rec;
+    a.v = vb + h0 * s.d_v * in_b;
+    a.M = M_out;
+    a.y = y + h0 * s.d_v;
+    a.y_other = y_other != nullptr ? y_other + h0 * s.d_v : nullptr;
+    a.err = dev.err;
+    tr.mark_chunk(2 * k, hi);
+    if ((r = launch_pipe(c, sk, a, hi)) != SDM_OK) return finish(r);
+    tr.mark_chunk(2 * k + 1, hi);
+  }
+  if (y_other != nullptr) {
+    const int64_t n4 = static_cast<int64_t>(s.T) * s.H * s.d_v / 4;
+    const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, static_cast<int64_t>(dev.sms) * 8));
+    sdm::k_add_f4<<<grid, 256, 0, hi>>>(reinterpret_cast<float4*>(y), reinterpret_cast<const float4*>(y_other), n4);
+    if ((r = launch_status("part sum launch")) != SDM_OK) return finish(r);
+  }
+  tr.mark(4, hi);
+  if (g != nullptr && (r = launch_epilogue(dev, s, y, g, hi)) != SDM_OK) return finish(r);
+  tr.mark(5, hi);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return finish(fail(SDM_ERR_CUDA, std::string("overlapped layer call: ") + cudaGetErrorString(e)));
+  return finish(SDM_OK);
+}
+
 sdm_status_t layer_forward_impl(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,
                                 const void* alpha, const void* beta, const void* g, const void* M0, void* M_out,
                                 float* y, void* workspace, size_t workspace_bytes, void* stream, void* const* events,
                                 int32_t n_events, float* ckpt, size_t ckpt_bytes) {
   sdm_status_t r;
-  if (!(n_events == 0 || (n_events == 6 && events != nullptr)))
-    return fail(SDM_ERR_INVALID_ARGUMENT, "n_events must be 0, or 6 with a non-NULL events array");
+  if (!(n_events == 0 || (n_events >= 6 && n_events % 2 == 0 && events != nullptr)))
+    return fail(SDM_ERR_INVALID_ARGUMENT,
+                "n_events must be 0, or 6 (+ 2 a chunk of an overlapped call) with a non-NULL events array");
   Trace tr;
-  if (n_events == 6) {
-    for (int i = 0; i < 6; ++i)
+  if (n_events > 0) {
+    for (int i = 0; i < n_events; ++i)
       if (events[i] == nullptr) return fail(SDM_ERR_INVALID_ARGUMENT, "events[] holds a NULL event");
     tr.events = events;
+    if (n_events > 6) tr.chunk_events = events + 6;
   }
   if ((r = check_shape(shape)) != SDM_OK) return r;
   const sdm_shape_t& s = *shape;
@@ -796,6 +981,11 @@ sdm_status_t layer_forward_impl(const sdm_shape_t* shape, const void* kp, const 
   if (!any) return launch_state_init(*dev, s, M0, M_out, st) == SDM_OK ? ok() : SDM_ERR_CUDA;
   ScanChoice c;
   if ((r = choose_scan(*dev, s, &c)) != SDM_OK) return r;
+  const bool overlap = ckpt == nullptr && overlapped(s, c) && overlap_workspace(s, c) <= workspace_bytes;
+  if (n_events > 6 && !(overlap && n_events == 6 + 2 * overlap_chunks(s)))
+    return fail(SDM_ERR_INVALID_ARGUMENT, "n_events must be 6 + 2 * sdm_layer_forward_chunks() = " +
+                                              std::to_string(6 + 2 * (overlap ? overlap_chunks(s) : 0)) +
+                                              " for per-chunk events, or 6");
   int32_t ckpt_C = 0;
   if (ckpt != nullptr) {
     size_t need_ckpt = 0;
@@ -805,6 +995,10 @@ sdm_status_t layer_forward_impl(const sdm_shape_t* shape, const void* kp, const 
     if (reinterpret_cast<uintptr_t>(ckpt) % 16 != 0) return fail(SDM_ERR_INVALID_ARGUMENT, "ckpt is not 16-byte aligned");
   }
   unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (overlap) {
+    r = layer_forward_overlapped(*dev, s, c, kp, qp, v, alpha, beta, g, M0, M_out, y, ws, st, tr);
+    return r == SDM_OK ? ok() : r;
+  }
   int32_t* idx_w = reinterpret_cast<int32_t*>(ws);
   ws += align256(th * s.W * 4);
   float* w_w = reinterpret_cast<float*>(ws);
@@ -1261,6 +1455,16 @@ sdm_status_t sdm_layer_forward_ckpt(const sdm_shape_t* shape, const void* kp, co
                             nullptr, 0, ckpt, ckpt_bytes);
 }
 
+int32_t sdm_layer_forward_chunks(const sdm_shape_t* shape) {
+  const std::string saved = g_last_error;
+  DeviceInfo* dev;
+  ScanChoice c;
+  if (check_shape(shape) != SDM_OK || device_info(&dev) != SDM_OK || choose_scan(*dev, *shape, &c) != SDM_OK)
+    return -1;
+  g_last_error = saved;
+  return overlapped(*shape, c) ? static_cast<int32_t>(overlap_chunks(*shape)) : 1;
+}
+
 int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate) {
   const std::string saved = g_last_error;
   DeviceInfo* dev;
@@ -1274,7 +1478,9 @@ int32_t sdm_layer_forward_launches(const sdm_shape_t* shape, int32_t with_gate) 
   // first; the pipelined one with two slot parts adds the second part's sums into y after
   const int parts_sum = c.kind == SDM_VARIANT_PIPELINED && c.parts > 1 ? 1 : 0;
   const int init = c.resident ? 0 : (shape->state_dtype == SDM_FP8_B16 ? 2 : 1);  // fp8: codes and exponents
-  return 4 + init + parts_sum + (with_gate ? 1 : 0);
+  // an overlapped call: two selections, records and the recurrence per chunk
+  const int64_t per_call = overlapped(*shape, c) ? 4 * overlap_chunks(*shape) : 4;
+  return static_cast<int32_t>(per_call) + init + parts_sum + (with_gate ? 1 : 0);
 }
 
 sdm_status_t sdm_layer_forward(const sdm_shape_t* shape, const void* kp, const void* qp, const void* v,

@@ -52,6 +52,7 @@ PROTOTYPES = {
     "sdm_layer_step_workspace_bytes": (_sz, [_shape_p]),
     "sdm_layer_step_launches": (_i32, [_shape_p]),
     "sdm_layer_forward_launches": (_i32, [_shape_p, _i32]),
+    "sdm_layer_forward_chunks": (_i32, [_shape_p]),
     "sdm_scan_describe": (_i32, [_shape_p, ctypes.c_char_p, _sz]),
     "sdm_scan_backward_workspace_bytes": (_sz, [_shape_p]),
     "sdm_scan_backward": (_i32, [_shape_p] + [_p] * 8 + [_i32] + [_p] * 8 + [_sz, _p]),
