@@ -66,3 +66,24 @@ def test_overlapped_layer_call_with_epilogue_and_repeat(sdm, cuda_device):
     sdm.stream_check()
     for y, M_T in outs:
         assert torch.equal(M_T, M) and torch.equal(y, y1)
+
+
+def test_overlapped_layer_call_fp8_state(sdm, cuda_device):
+    """The block-scaled fp8 state through the overlapped call equals one
+    sdm_layer_step over the whole sequence (one pass from the same state)."""
+    T = 2 * CHUNK + 301
+    shape = synth.Shape("overlap_fp8", B=1, T=T, H=2, sqrt_n=32, d_v=256, W=16, R=16, in_dtype="bf16",
+                        state_dtype="bf16")
+    inp = synth.make_inputs(shape, seed=23, device=cuda_device)
+    M0 = sdm.quantize_fp8blk(inp["M0"].float().contiguous())
+    sh = sdm.make_shape(1, T, 2, 32, 16, 16, 256, torch.bfloat16, torch.uint8, variant="pipelined")
+    assert sdm.layer_forward_chunks(sh) == 3
+    y, M_T = sdm.layer_forward(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], M0, shape.W, shape.R,
+                               variant="pipelined")
+    sdm.stream_check()
+    M = M0.clone()
+    y1 = sdm.layer_step(inp["kp"], inp["qp"], inp["v"], inp["alpha"], inp["beta"], M, shape.W, shape.R,
+                        variant="pipelined")
+    sdm.stream_check()
+    assert torch.equal(M_T.reshape(-1), M), "fp8 state differs from the one-pass call"
+    assert torch.equal(y, y1), "y differs from the one-pass call"
