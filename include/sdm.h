@@ -34,8 +34,12 @@
  *   - dtype SDM_F32 is IEEE binary32, SDM_BF16 is bfloat16 (round-to-nearest-
  *     even on every store).
  *   - Not thread-safe with respect to one stream; distinct streams may call
- *     concurrently. The only library-wide state is the per-device error word
- *     and the thread-local message behind sdm_last_error(). The error word is
+ *     concurrently. Library-wide state: the per-device error word, the
+ *     thread-local message behind sdm_last_error(), and per-device caches
+ *     made on first use (device attributes, the scratch address of
+ *     sdm_layer_forward_noalloc, the two streams of an overlapped
+ *     sdm_layer_forward call). The caches do not survive cudaDeviceReset():
+ *     reload the library after a reset. The error word is
  *     shared by all streams of a device: sdm_stream_check() on any stream
  *     reports (and clears) the bits set by every stream's calls since the last
  *     check, so a multi-stream caller should check after a common sync point.
