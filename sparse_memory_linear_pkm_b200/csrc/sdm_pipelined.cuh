@@ -19,31 +19,31 @@
 // synchronisation; each adds its partial read sum into y (with two parts the
 // sum 0 + a + b does not depend on their order, so y stays reproducible).
 //
-// Within a CTA, for token t, after the block barrier that ends token t - 2:
-//   * producer warps request the rows of token t + P - 2 with TMA row
-//     gathers (four 128-byte rows an instruction) into the stage token t - 2
-//     used, so the copies run P - 2 tokens ahead of their use. An SM takes
-//     one random 128-byte row per ~6-7 cycles however it is asked (TMA or
-//     cp.async, or both at once), and the issuing thread waits for the
-//     acceptance; with the requests in warps of their own, the consumer
-//     warps compute while the producers wait (measured: ~650 cycles a token
-//     of request issue that the compute otherwise waited for);
-//   * one lane per warp waits for token t's rows, and one block barrier,
-//     taken after those waits, also ends token t - 1;
+// Within a CTA (warp roles; one token a step, or two with S = 2):
+//   * producer warps request each token's rows with TMA row gathers (four
+//     128-byte rows an instruction, two instructions a warp at W = R = 64)
+//     into a ring of P stages, up to P - 1 tokens ahead, and reload the
+//     record and v chunks; before reusing a stage they wait on a per-token
+//     `done` mbarrier, once per token pair (tokens finish in order). An SM
+//     takes one random 128-byte row per ~6-7 cycles however it is asked, and
+//     the issuing thread waits for the acceptance, so the requests live in
+//     warps of their own;
+//   * the control warp waits for the next token's rows and records, sums the
+//     read lanes' partial sums of the previous token in a fixed order and
+//     stores them to y (part 0) or to a scratch copy that a separate pass adds
+//     into y (part 1; plain stores, no atomics), and arrives on `done`;
 //   * write warps apply the write to the part's write entries (each lane owns
 //     one 16-byte unit of a row), store the rows to global memory and keep
 //     them in a ring of written-row stages;
-//   * read warps sum the part's read entries; lane bits above the unit index
-//     select entries, so a warp reduces its columns with shuffles alone; part
-//     0 stores its sums to y, part 1 to a scratch copy that a separate pass
-//     adds into y (plain stores, no atomics);
-//   * one block barrier per token.
-// Write warps fence their global stores (fence.proxy.async.global) at the
-// top of the next token, before its barrier, so the TMA gathers issued after
-// that barrier read them. A row gathered early is stale when one of the P - 1
-// tokens before its use wrote it (the gather of token u is issued while
-// token u - P + 1 may still be writing); the hazard plan in the records names that write (token t - k,
-// write entry j of this part) and the row is taken from the written-row ring
+//   * read warps sum the part's read entries, each lane its unit over its
+//     entry group, and store those partial sums for the control warp;
+//   * the control warp and the consumers meet at one named barrier a step
+//     (barrier.cta.red.or: a failed wait in the control warp ends them all).
+// Write warps fence their global stores (fence.proxy.async.global) before
+// the next barrier, so the TMA gathers issued after `done` read them. A row
+// gathered early is stale when one of the P - 1 tokens before its use wrote
+// it; the hazard plan in the records names that write (token t - k, write
+// entry j of this part) and the row is taken from the written-row ring
 // instead; a read of a slot written by the same token (k = 0) recomputes that
 // write from its source.
 #pragma once
